@@ -1,0 +1,148 @@
+"""KDA oracle: a plain, slow, float64 CPU implementation of Kimi Delta Attention.
+
+TEST INFRASTRUCTURE ONLY.  The tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline / reference legs are the only callers.  The CUDA path
+(``gated_delta_rule_74_b200``) never imports this package and shares no code
+with it; the only module both sides use is ``kda_inputs`` (seeded random
+inputs, none of the method's arithmetic).
+
+Contents
+  * ``prefill`` / ``decode``: ctypes front end of ``kda_oracle.cpp``, the
+    token-by-token float64 recurrence
+        S_t = (I - beta_t k_t k_t^T) Diag(exp(g_t)) S_{t-1} + beta_t k_t v_t^T,
+        o_t = S_t^T q_t
+    (miniKimiK3 model card, Architecture, "Kimi Delta Attention" bullet), with
+    the state reset to each document's own initial state at every cu_seqlens
+    boundary (Mini-K3-1H-mamba2 model card, packed-document paragraph).
+  * ``reference.recurrence_literal``: the same recurrence in numpy with the
+    dk x dk factor (I - beta k k^T) materialised, for tiny inputs.
+  * ``reference.chunked``: the chunked (WY / UT transform) form of the same
+    recurrence in float64 numpy, for checking the chunked algebra the GPU
+    kernels implement ("trains through a chunked parallel form", same bullet).
+
+Pins: tests/test_oracle.py checks these routines against closed forms,
+invariants, a hand-worked example (tests/golden/) and brute force.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+from . import reference  # noqa: F401  (numpy routines)
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kda_oracle.cpp")
+_SO = os.path.join(_HERE, "libkda_oracle.so")
+_lib = None
+_lock = threading.Lock()
+
+__all__ = ["build", "prefill", "decode", "max_threads", "reference"]
+
+
+def build(force: bool = False) -> str:
+    """Compile kda_oracle.cpp into libkda_oracle.so next to it (no fast-math)."""
+    if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(_SRC):
+        cmd = ["g++", "-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
+               "-shared", "-fPIC", "-std=c++17", _SRC, "-o", _SO + ".tmp"]
+        subprocess.run(cmd, check=True)
+        os.replace(_SO + ".tmp", _SO)
+    return _SO
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_SO)
+            dp = ctypes.POINTER(ctypes.c_double)
+            lib.kda_oracle_prefill.argtypes = [dp, dp, dp, dp, dp, dp,
+                                               ctypes.POINTER(ctypes.c_int32), dp, dp,
+                                               ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                               ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                               ctypes.c_int, ctypes.c_int]
+            lib.kda_oracle_prefill.restype = ctypes.c_int
+            lib.kda_oracle_decode.argtypes = [dp, dp, dp, dp, dp, dp, dp,
+                                              ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                              ctypes.c_int, ctypes.c_longlong,
+                                              ctypes.c_longlong, ctypes.c_int]
+            lib.kda_oracle_decode.restype = ctypes.c_int
+            lib.kda_oracle_max_threads.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def max_threads() -> int:
+    return int(_load().kda_oracle_max_threads())
+
+
+def _f64(x) -> np.ndarray:
+    """Exact upcast of a torch tensor (bf16/f32) or array to contiguous float64."""
+    if x is None:
+        return None
+    if hasattr(x, "detach"):
+        x = x.detach().to("cpu").double().numpy()
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def prefill(q, k, v, g, beta, h0=None, cu_seqlens=None, heads=None, nthreads: int = 0):
+    """Float64 KDA prefill by recurrence.
+
+    q, k [B,T,H,dk]; v [B,T,H,dv]; g [B,T,H,dk]; beta [B,T,H]; h0 [Nseq,H,dk,dv]
+    or None; cu_seqlens int [Nseq+1] or None (then tensors are [1,T,H,*]).
+    ``heads``: optional (lo, hi) range; only those heads are computed and returned.
+    Returns (out [B,T,H',dv], hT [Nseq,H',dk,dv]) as float64 numpy arrays.
+    """
+    if heads is not None:
+        lo, hi = heads
+        q, k, v, g, beta = (x[:, :, lo:hi] for x in (q, k, v, g, beta))
+        if h0 is not None:
+            h0 = h0[:, lo:hi]
+    q, k, v, g, beta, h0 = (_f64(x) for x in (q, k, v, g, beta, h0))
+    Bt, T, H, dk = q.shape
+    dv = v.shape[-1]
+    cu = None
+    if cu_seqlens is not None:
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens.cpu() if hasattr(cu_seqlens, "cpu")
+                                             else cu_seqlens), dtype=np.int32)
+        nseq = cu.shape[0] - 1
+        if Bt != 1:
+            raise ValueError("packed (cu_seqlens) inputs must have B == 1 in the tensors")
+    else:
+        nseq = Bt
+    out = np.zeros((Bt, T, H, dv), dtype=np.float64)
+    hT = np.zeros((nseq, H, dk, dv), dtype=np.float64)
+    rc = _load().kda_oracle_prefill(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
+        None if cu is None else cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+        _ptr(out), _ptr(hT), nseq, T, H, dk, dv, 0, H, int(nthreads))
+    if rc != 0:
+        raise ValueError(f"kda_oracle_prefill rejected its arguments (rc={rc})")
+    return out, hT
+
+
+def decode(q, k, v, g, beta, S, nthreads: int = 0):
+    """One float64 KDA decode step.  q,k [N,H,dk]; v [N,H,dv]; g [N,H,dk];
+    beta [N,H]; S [N,H,dk,dv].  Returns (out [N,H,dv], S_new) as float64 arrays
+    (S is copied, not modified)."""
+    q, k, v, g, beta = (_f64(x) for x in (q, k, v, g, beta))
+    S = _f64(S).copy()
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    out = np.zeros((N, H, dv), dtype=np.float64)
+    rc = _load().kda_oracle_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                   _ptr(S), _ptr(out), N, H, dk, dv, 0, N * H,
+                                   int(nthreads))
+    if rc != 0:
+        raise ValueError(f"kda_oracle_decode rejected its arguments (rc={rc})")
+    return out, S
