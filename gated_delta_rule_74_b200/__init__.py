@@ -1,0 +1,176 @@
+"""gated_delta_rule_74_b200: B200 (sm_100a) Kimi Delta Attention (KDA).
+
+Thin ctypes binding over libkda.so, whose C ABI is declared in include/kda.h.
+The functions here only marshal torch CUDA tensors into pointers and sizes and
+call the library on the current torch stream; every step of the computation runs
+in the library's CUDA kernels.  There is no fallback: if libkda.so is missing or a
+call fails, an exception is raised.
+
+    out, hT = kda_chunk_fwd(q, k, v, g, beta, h0=None, cu_seqlens=None)
+    out     = kda_decode_step(q, k, v, g, beta, S)        # S updated in place
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional
+
+import torch
+
+__all__ = ["kda_chunk_fwd", "kda_decode_step", "kda_status_string", "kda_version",
+           "lib", "library_path", "header_symbols", "KdaError",
+           "KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED", "KDA_ERR_CUDA",
+           "KDA_ERR_TIMEOUT", "KDA_BF16", "KDA_F32"]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_ROOT = os.path.dirname(_PKG)
+_SO = os.path.join(_PKG, "libkda.so")
+_HEADER = os.path.join(_ROOT, "include", "kda.h")
+
+KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = 0, -1, -2, -3, -4
+KDA_BF16, KDA_F32 = 0, 1
+
+_DTYPES = {torch.bfloat16: KDA_BF16, torch.float32: KDA_F32}
+_lib = None
+
+
+class KdaError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {kda_status_string(status)} ({status})")
+
+
+def library_path() -> str:
+    return _SO
+
+
+def lib() -> ctypes.CDLL:
+    """Load libkda.so (built in-tree by gated_delta_rule_74_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_SO):
+            raise RuntimeError(f"libkda.so is not built ({_SO}); run "
+                               "`python -m gated_delta_rule_74_b200.build`")
+        L = ctypes.CDLL(_SO)
+        vp, fp, ip = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int
+        L.kda_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, fp, vp, vp, fp,
+                                    ip, ip, ip, ip, ip, ip, vp]
+        L.kda_chunk_fwd.restype = ctypes.c_int
+        L.kda_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, vp, ip, ip, ip, ip, ip, vp]
+        L.kda_decode_step.restype = ctypes.c_int
+        L.kda_status_string.argtypes = [ctypes.c_int]
+        L.kda_status_string.restype = ctypes.c_char_p
+        L.kda_version.argtypes = []
+        L.kda_version.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def header_symbols() -> list[str]:
+    """Names of the functions include/kda.h declares."""
+    with open(_HEADER) as f:
+        text = f.read()
+    return re.findall(r"^KDA_API\s+[\w\s\*]*?\b(kda_\w+)\s*\(", text, flags=re.M)
+
+
+def kda_status_string(status: int) -> str:
+    return lib().kda_status_string(int(status)).decode()
+
+
+def kda_version() -> int:
+    return int(lib().kda_version())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(name: str, t: torch.Tensor, dtype=None, shape=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def kda_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+                  beta: torch.Tensor, h0: Optional[torch.Tensor] = None,
+                  cu_seqlens: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                  hT: Optional[torch.Tensor] = None, output_final_state: bool = True,
+                  stream=None):
+    """KDA prefill (chunked form).  q, k [B,T,H,dk]; v [B,T,H,dv]; g [B,T,H,dk] f32;
+    beta [B,T,H] f32; h0 [Nseq,H,dk,dv] f32 or None; cu_seqlens int32 [Nseq+1] on
+    the device, or None.  Returns (out, hT) (hT None if output_final_state is
+    False and no hT buffer was given)."""
+    if q.dim() != 4:
+        raise ValueError("q must be [B, T, H, dk]")
+    Bt, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = _DTYPES.get(q.dtype)
+    if dt is None:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    _check("q", q)
+    _check("k", k, q.dtype, (Bt, T, H, dk))
+    _check("v", v, q.dtype, (Bt, T, H, dv))
+    _check("g", g, torch.float32, (Bt, T, H, dk))
+    _check("beta", beta, torch.float32, (Bt, T, H))
+    if cu_seqlens is not None:
+        _check("cu_seqlens", cu_seqlens, torch.int32)
+        if Bt != 1:
+            raise ValueError("packed inputs (cu_seqlens) must have B == 1")
+        nseq = cu_seqlens.numel() - 1
+    else:
+        nseq = Bt
+    if h0 is not None:
+        _check("h0", h0, torch.float32, (nseq, H, dk, dv))
+    if out is None:
+        out = torch.empty((Bt, T, H, dv), dtype=q.dtype, device=q.device)
+    _check("out", out, q.dtype, (Bt, T, H, dv))
+    if hT is None and output_final_state:
+        hT = torch.empty((nseq, H, dk, dv), dtype=torch.float32, device=q.device)
+    if hT is not None:
+        _check("hT", hT, torch.float32, (nseq, H, dk, dv))
+    rc = lib().kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
+                             _ptr(cu_seqlens), _ptr(out), _ptr(hT),
+                             nseq, T, H, dk, dv, dt, _stream(stream))
+    if rc != KDA_OK:
+        raise KdaError("kda_chunk_fwd", rc)
+    return out, hT
+
+
+def kda_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+                    beta: torch.Tensor, S: torch.Tensor, out: Optional[torch.Tensor] = None,
+                    stream=None) -> torch.Tensor:
+    """One KDA decode step.  q, k [N,H,dk]; v [N,H,dv]; g [N,H,dk] f32; beta [N,H] f32;
+    S [N,H,dk,dv] f32, updated in place.  Returns out [N,H,dv]."""
+    if q.dim() != 3:
+        raise ValueError("q must be [N, H, dk]")
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = _DTYPES.get(q.dtype)
+    if dt is None:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    _check("q", q)
+    _check("k", k, q.dtype, (N, H, dk))
+    _check("v", v, q.dtype, (N, H, dv))
+    _check("g", g, torch.float32, (N, H, dk))
+    _check("beta", beta, torch.float32, (N, H))
+    _check("S", S, torch.float32, (N, H, dk, dv))
+    if out is None:
+        out = torch.empty((N, H, dv), dtype=q.dtype, device=q.device)
+    _check("out", out, q.dtype, (N, H, dv))
+    rc = lib().kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S),
+                               _ptr(out), N, H, dk, dv, dt, _stream(stream))
+    if rc != KDA_OK:
+        raise KdaError("kda_decode_step", rc)
+    return out

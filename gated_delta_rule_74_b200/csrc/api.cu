@@ -1,0 +1,84 @@
+// C ABI of libkda: host-side argument validation and kernel dispatch.
+// The entry points and their contracts are declared and documented in kda.h.
+#include <stdint.h>
+
+#include <initializer_list>
+
+#include "kda_common.cuh"
+
+namespace {
+
+constexpr int kVersionMajor = 0;
+constexpr int kVersionMinor = 1;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool head_ok(int d) { return d == 64 || d == 128; }
+
+int status_from(cudaError_t e) {
+  if (e == cudaSuccess) return KDA_OK;
+  (void)cudaGetLastError();   // clear a sticky launch-config error for the caller
+  return KDA_ERR_CUDA;
+}
+
+// All required pointers non-null and every given pointer 16-byte aligned.
+bool pointers_ok(std::initializer_list<const void*> required,
+                 std::initializer_list<const void*> optional) {
+  for (const void* p : required)
+    if (p == nullptr || !aligned16(p)) return false;
+  for (const void* p : optional)
+    if (p != nullptr && !aligned16(p)) return false;
+  return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+int kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
+                  const float* beta, const float* h0, const int32_t* cu_seqlens, void* out,
+                  float* hT, int B, int T, int H, int dk, int dv, int in_dtype,
+                  void* stream) {
+  if (B < 1 || T < 0 || H < 1) return KDA_ERR_INVALID_ARG;
+  if (in_dtype != KDA_BF16 && in_dtype != KDA_F32) return KDA_ERR_INVALID_ARG;
+  const long long rows = cu_seqlens ? (long long)T : (long long)B * T;
+  if (rows > 0) {
+    if (!pointers_ok({q, k, v, g, beta, out}, {h0, hT, cu_seqlens})) return KDA_ERR_INVALID_ARG;
+  } else {
+    // no tokens: the token tensors may be empty (null); only the states are used
+    if (!pointers_ok({}, {q, k, v, g, beta, out, h0, hT, cu_seqlens})) return KDA_ERR_INVALID_ARG;
+  }
+  if (!head_ok(dk) || !head_ok(dv)) return KDA_ERR_UNSUPPORTED;
+  // element counts must fit the kernels' 64-bit indexing and the grid limits
+  if (rows * H * (long long)(dk > dv ? dk : dv) > (1LL << 40)) return KDA_ERR_INVALID_ARG;
+  if ((long long)B > 65535LL || H > 65535) return KDA_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return status_from(kda::launch_chunk_simt(q, k, v, g, beta, h0, cu_seqlens, out, hT, B, T,
+                                            H, dk, dv, in_dtype, st));
+}
+
+int kda_decode_step(const void* q, const void* k, const void* v, const float* g,
+                    const float* beta, float* S, void* out, int N, int H, int dk, int dv,
+                    int in_dtype, void* stream) {
+  if (N < 1 || H < 1) return KDA_ERR_INVALID_ARG;
+  if (in_dtype != KDA_BF16 && in_dtype != KDA_F32) return KDA_ERR_INVALID_ARG;
+  if (!pointers_ok({q, k, v, g, beta, S, out}, {})) return KDA_ERR_INVALID_ARG;
+  if (!head_ok(dk) || !head_ok(dv)) return KDA_ERR_UNSUPPORTED;
+  if ((long long)N * H > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return status_from(kda::launch_decode(q, k, v, g, beta, S, out, N, H, dk, dv, in_dtype, st));
+}
+
+const char* kda_status_string(int status) {
+  switch (status) {
+    case KDA_OK: return "KDA_OK";
+    case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG";
+    case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED";
+    case KDA_ERR_CUDA: return "KDA_ERR_CUDA";
+    case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT";
+    default: return "KDA_ERR_UNKNOWN";
+  }
+}
+
+int kda_version(void) { return (kVersionMajor << 16) | kVersionMinor; }
+
+}  // extern "C"

@@ -1,0 +1,32 @@
+// Internal helpers shared by the KDA CUDA kernels (not part of the C ABI).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kda.h"
+
+namespace kda {
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Launchers implemented in the kernel translation units.  Each returns a
+// cudaError_t from the launch (cudaSuccess when the launch was accepted).
+cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* g,
+                          const float* beta, float* S, void* out, int N, int H, int dk,
+                          int dv, int in_dtype, cudaStream_t stream);
+
+cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const float* g,
+                              const float* beta, const float* h0, const int32_t* cu_seqlens,
+                              void* out, float* hT, int B, int T, int H, int dk, int dv,
+                              int in_dtype, cudaStream_t stream);
+
+}  // namespace kda

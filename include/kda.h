@@ -1,0 +1,126 @@
+/*
+ * kda.h -- C ABI of the B200 (sm_100a) Kimi Delta Attention library, libkda.so.
+ *
+ * Kimi Delta Attention (KDA) is a gated delta-rule linear attention with a fixed
+ * fp32 dk x dv state S per head.  Per token t (miniKimiK3 model card, Architecture,
+ * "Kimi Delta Attention" bullet: one gradient-descent step on ||S^T k - v||^2, an
+ * error-correcting write, per-channel gated decay, a chunked parallel form for
+ * training/prefill and a recurrence for decoding):
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(exp(g_t)) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = S_t^T q_t
+ *
+ * g_t (one log-decay per key channel, <= 0 in normal use) decays the rows of S.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     never frees them.  Every pointer must be 16-byte aligned.
+ *   - Layouts are dense row-major, last index fastest:
+ *       q, k [.., dk]   v, out [.., dv]   g [.., dk] (fp32)   beta [..] (fp32)
+ *       states [.., dk, dv] fp32 (row c = key channel, dv contiguous).
+ *   - in_dtype (kda_dtype_t) is the storage type of q, k, v and out.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream)
+ *     and is asynchronous: a KDA_OK return means the work was launched, not done.
+ *   - Supported head sizes: dk, dv in {64, 128}.  Others: KDA_ERR_UNSUPPORTED.
+ *   - Arguments are validated on the host before anything is launched; on an
+ *     error nothing is enqueued and no output is touched.  The library does not
+ *     normalise q/k, scale q, or clamp g/beta: those are the caller's inputs.
+ *   - Thread safety: calls are independent; concurrent calls on different
+ *     streams are safe as long as their output buffers do not overlap.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KDA_API __attribute__((visibility("default")))
+#else
+#define KDA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KDA_OK = 0,
+  KDA_ERR_INVALID_ARG = -1,   /* null required pointer, bad size, misalignment */
+  KDA_ERR_UNSUPPORTED = -2,   /* valid request this build does not implement   */
+  KDA_ERR_CUDA = -3,          /* a CUDA runtime call or kernel launch failed    */
+  KDA_ERR_TIMEOUT = -4        /* reserved: a bounded device-side wait expired   */
+} kda_status_t;
+
+typedef enum {
+  KDA_BF16 = 0,               /* bfloat16 q, k, v, out */
+  KDA_F32 = 1                 /* float32  q, k, v, out */
+} kda_dtype_t;
+
+/*
+ * kda_chunk_fwd -- KDA prefill through the chunked (C = 64) parallel form.
+ *
+ * Passage: miniKimiK3 model card, "Kimi Delta Attention" bullet ("trains through a
+ * chunked parallel form"); packed-document isolation as in the Mini-K3-1H-mamba2
+ * card's packed-document paragraph (state flow reset at every document boundary).
+ * The result equals the token-by-token recurrence above up to rounding.
+ *
+ * Fixed-length mode (cu_seqlens == NULL): B sequences of T tokens each.
+ *     q, k, g [B, T, H, dk]   v, out [B, T, H, dv]   beta [B, T, H]
+ *     h0, hT  [B, H, dk, dv]
+ * Packed mode (cu_seqlens != NULL): B documents packed into one row of T tokens.
+ *     q, k, g [1, T, H, dk]   v, out [1, T, H, dv]   beta [1, T, H]
+ *     h0, hT  [B, H, dk, dv]  (one state slot per document)
+ *     cu_seqlens: DEVICE int32 [B + 1], cu_seqlens[0] = 0, non-decreasing,
+ *     cu_seqlens[B] = T.  Documents may be empty.  Document d is tokens
+ *     [cu_seqlens[d], cu_seqlens[d+1]) and starts from h0[d] (or zero); no state
+ *     crosses a boundary, and chunks restart at every document start, so a
+ *     document's result does not depend on its neighbours.  The contents of
+ *     cu_seqlens are device memory and are NOT checked on the host; malformed
+ *     offsets give undefined results for the affected documents, but every
+ *     access stays inside [0, T) (offsets are clamped on the device).
+ *
+ * h0: initial state, or NULL for zeros.   hT: final state out, or NULL to skip.
+ * out must not alias any input.  hT may alias h0 (in-place state update).
+ * B >= 1, T >= 0, H >= 1.  T == 0 writes hT = h0 (or zeros) and nothing else.
+ *
+ * Precision: g, beta and the state are fp32.  With KDA_BF16 inputs the chunk
+ * contractions run on the tensor cores with bf16 operands and fp32
+ * accumulation; with KDA_F32 inputs every step runs in fp32 on the CUDA cores.
+ *
+ * Returns KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED or KDA_ERR_CUDA.
+ */
+KDA_API int kda_chunk_fwd(const void* q, const void* k, const void* v,
+                  const float* g, const float* beta, const float* h0,
+                  const int32_t* cu_seqlens, void* out, float* hT,
+                  int B, int T, int H, int dk, int dv,
+                  int in_dtype, void* stream);
+
+/*
+ * kda_decode_step -- one recurrent KDA step for N independent sequences.
+ *
+ * Passage: miniKimiK3 model card, "Kimi Delta Attention" bullet ("decodes as a
+ * recurrence with a fixed state per head, so cost per token is constant");
+ * the Kimi-K3-Tiny-L13 card's serving paragraph (decode concurrency is bound by
+ * the KDA state pool).  Applies the update above once per (n, h), in place:
+ *     q, k, g [N, H, dk]   v, out [N, H, dv]   beta [N, H]   S [N, H, dk, dv]
+ * S is read once and written once.  out must not alias S or any input.
+ * N >= 1, H >= 1.
+ *
+ * Returns KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED or KDA_ERR_CUDA.
+ */
+KDA_API int kda_decode_step(const void* q, const void* k, const void* v,
+                    const float* g, const float* beta, float* S, void* out,
+                    int N, int H, int dk, int dv, int in_dtype, void* stream);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+KDA_API const char* kda_status_string(int status);
+
+/* Library ABI version: (major << 16) | minor. */
+KDA_API int kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

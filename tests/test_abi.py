@@ -1,0 +1,74 @@
+"""The C-ABI library loads, exports every declared symbol and validates its
+arguments on the host.  No test here launches GPU work: each call carries at
+least one invalid argument, so the library returns before touching CUDA."""
+import ctypes
+
+import pytest
+
+import gated_delta_rule_74_b200 as kda
+
+
+@pytest.fixture(scope="module")
+def L():
+    from gated_delta_rule_74_b200 import build
+    build.build()
+    return kda.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = kda.header_symbols()
+    assert set(names) >= {"kda_chunk_fwd", "kda_decode_step", "kda_status_string", "kda_version"}
+    for n in names:
+        assert hasattr(L, n), f"libkda.so does not export {n}"
+
+
+def test_status_strings_and_version(L):
+    assert kda.kda_status_string(0) == "KDA_OK"
+    assert kda.kda_status_string(-1) == "KDA_ERR_INVALID_ARG"
+    assert kda.kda_status_string(-2) == "KDA_ERR_UNSUPPORTED"
+    assert kda.kda_status_string(-3) == "KDA_ERR_CUDA"
+    assert kda.kda_status_string(-4) == "KDA_ERR_TIMEOUT"
+    assert kda.kda_status_string(12345) == "KDA_ERR_UNKNOWN"
+    assert kda.kda_version() >= 1
+
+
+P = 0x10000   # a 16-byte aligned fake address; never dereferenced by these calls
+
+
+def _chunk(L, q=P, k=P, v=P, g=P, beta=P, h0=None, cu=None, out=P, hT=None,
+           B=1, T=64, H=2, dk=64, dv=64, dt=0):
+    return L.kda_chunk_fwd(q, k, v, g, beta, h0, cu, out, hT, B, T, H, dk, dv, dt, None)
+
+
+def _decode(L, q=P, k=P, v=P, g=P, beta=P, S=P, out=P, N=1, H=1, dk=64, dv=64, dt=0):
+    return L.kda_decode_step(q, k, v, g, beta, S, out, N, H, dk, dv, dt, None)
+
+
+@pytest.mark.parametrize("bad", [dict(q=None), dict(k=None), dict(v=None), dict(g=None),
+                                 dict(beta=None), dict(out=None), dict(q=P + 4),
+                                 dict(h0=P + 8), dict(hT=P + 2), dict(cu=P + 4),
+                                 dict(B=0), dict(T=-1), dict(H=0), dict(dt=7)])
+def test_chunk_fwd_rejects_invalid(L, bad):
+    assert _chunk(L, **bad) == kda.KDA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("dims", [dict(dk=32), dict(dv=96), dict(dk=256, dv=256)])
+def test_chunk_fwd_rejects_unsupported_heads(L, dims):
+    assert _chunk(L, **dims) == kda.KDA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("bad", [dict(q=None), dict(S=None), dict(out=None), dict(S=P + 4),
+                                 dict(N=0), dict(H=0), dict(dt=-1)])
+def test_decode_rejects_invalid(L, bad):
+    assert _decode(L, **bad) == kda.KDA_ERR_INVALID_ARG
+
+
+def test_decode_rejects_unsupported_heads(L):
+    assert _decode(L, dk=48) == kda.KDA_ERR_UNSUPPORTED
+
+
+def test_binding_rejects_cpu_tensors(L):
+    import torch
+    x = torch.zeros(1, 4, 1, 64)
+    with pytest.raises(ValueError):
+        kda.kda_chunk_fwd(x, x, x, x, torch.zeros(1, 4, 1))

@@ -1,0 +1,182 @@
+"""GPU parity of kda_chunk_fwd against the float64 oracle, on the workload
+shapes, on small ragged shapes and on the edge cases of the chunked form."""
+import numpy as np
+import pytest
+import torch
+
+import kda_inputs as ki
+import oracle
+from _helpers import TOL, gpu_prefill, oracle_prefill, rel_err, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _check(x, heads=None, with_h0=True):
+    out, hT = gpu_prefill(x, with_h0=with_h0)
+    o_ref, s_ref = oracle_prefill(x, heads=heads, with_h0=with_h0)
+    if heads is not None:
+        out = out[:, :, heads[0]:heads[1]]
+        hT = hT[:, heads[0]:heads[1]]
+    tol = TOL[x["dtype"]]
+    eo, es = rel_err(out, o_ref), rel_err(hT, s_ref)
+    assert eo <= tol and es <= tol, (x["name"], eo, es)
+    return eo, es
+
+
+# ---- the five workloads and the headline shape -------------------------------
+def test_cfg0_fp32():
+    _check(ki.make_prefill("cfg0"))
+
+
+def test_cfg1_bf16():
+    _check(ki.make_prefill("cfg1"))
+
+
+def test_cfg2_varlen():
+    _check(ki.make_prefill("cfg2"))
+
+
+def test_metric_shape():
+    _check(ki.make_prefill("metric"))
+
+
+def test_cfg3_sampled_heads():
+    """B=1, T=32768, H=96, d=128 with h0 ~ N(0, 0.02) on the GPU; the oracle
+    checks heads 0, 1 and 95 over the whole sequence."""
+    x = ki.make_prefill("cfg3")
+    out, hT = gpu_prefill(x)
+    for lo, hi in ((0, 2), (95, 96)):
+        o_ref, s_ref = oracle_prefill(x, heads=(lo, hi))
+        assert rel_err(out[:, :, lo:hi], o_ref) <= TOL["bf16"]
+        assert rel_err(hT[:, lo:hi], s_ref) <= TOL["bf16"]
+
+
+# ---- small shapes: several chunks and a ragged tail --------------------------
+def _spec(dtype, dk, dv, decay="alog", h0=False, B=2, T=130, H=3, seed=11):
+    return ki.PrefillSpec("small", B=B, T=T, H=H, dk=dk, dv=dv, dtype=dtype, decay=decay,
+                          seed=seed, h0=h0)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 128), (64, 128), (128, 64)])
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 130])
+def test_small_ragged(dtype, dk, dv, T):
+    _check(ki.make_prefill(_spec(dtype, dk, dv, T=T, h0=True)))
+
+
+@pytest.mark.parametrize("decay", ["logsigmoid", "alog"])
+def test_without_h0_and_without_hT(decay):
+    x = ki.make_prefill(_spec("bf16", 128, 128, decay=decay, T=200))
+    d = to_dev(x)
+    import gated_delta_rule_74_b200 as kda
+    out, hT = kda.kda_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"],
+                                output_final_state=False)
+    assert hT is None
+    o_ref, _ = oracle_prefill(x)
+    assert rel_err(out, o_ref) <= TOL["bf16"]
+
+
+def test_T_zero_copies_h0():
+    x = ki.make_prefill(_spec("bf16", 128, 128, T=0, h0=True))
+    out, hT = gpu_prefill(x)
+    assert out.numel() == 0
+    assert torch.equal(hT.cpu(), x["h0"])
+
+
+def test_hT_aliases_h0():
+    x = ki.make_prefill(_spec("bf16", 128, 128, T=150, h0=True))
+    d = to_dev(x)
+    import gated_delta_rule_74_b200 as kda
+    state = d["h0"].clone()
+    kda.kda_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], h0=state, hT=state)
+    torch.cuda.synchronize()
+    _, s_ref = oracle_prefill(x)
+    assert rel_err(state, s_ref) <= TOL["bf16"]
+
+
+# ---- packed documents ----------------------------------------------------------
+@pytest.mark.parametrize("lens", [[1, 64, 0, 65, 200, 3], [300, 0, 0, 17], [64, 64, 64]])
+def test_varlen_edge_documents(lens):
+    spec = ki.PrefillSpec("varlen", B=0, T=0, H=2, dk=128, dv=128, dtype="bf16",
+                          decay="alog", seed=5, h0=True, varlen=True)
+    _check(ki.make_prefill(spec, doc_lens=lens))
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_packed_equals_separate_bitwise(seed):
+    """A document gives bit-identical results packed or alone: chunks restart at
+    each document start, so nothing is shared across a boundary (Mini-K3-1H-
+    mamba2 card, packed-document paragraph)."""
+    spec = ki.PrefillSpec("varlen", B=0, T=0, H=4, dk=128, dv=128, dtype="bf16",
+                          decay="alog", seed=seed, h0=True, varlen=True)
+    lens = [70, 129, 5, 256]
+    x = ki.make_prefill(spec, doc_lens=lens)
+    out, hT = gpu_prefill(x)
+    cu = x["cu_seqlens"].tolist()
+    for dno, (s, e) in enumerate(zip(cu[:-1], cu[1:])):
+        xs = dict(x)
+        for key in ("q", "k", "v", "g", "beta"):
+            xs[key] = x[key][:, s:e].contiguous()
+        xs["h0"] = x["h0"][dno:dno + 1].contiguous()
+        xs["cu_seqlens"] = None
+        o1, s1 = gpu_prefill(xs)
+        assert torch.equal(out[:, s:e], o1)
+        assert torch.equal(hT[dno:dno + 1], s1)
+
+
+def test_perturbing_earlier_document_changes_nothing_later():
+    spec = ki.PrefillSpec("varlen", B=0, T=0, H=2, dk=128, dv=128, dtype="bf16",
+                          decay="alog", seed=3, h0=True, varlen=True)
+    x = ki.make_prefill(spec, doc_lens=[100, 150, 90])
+    out, hT = gpu_prefill(x)
+    y = {k: (v.clone() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    s, e = 100, 250
+    for key in ("q", "k", "v"):
+        y[key][:, s:e] = torch.randn_like(y[key][:, s:e].float()).to(y[key].dtype)
+    y["g"][:, s:e] *= 0.3
+    y["h0"][1] += 1.0
+    out2, hT2 = gpu_prefill(y)
+    assert torch.equal(out2[:, :s], out[:, :s]) and torch.equal(out2[:, e:], out[:, e:])
+    assert torch.equal(hT2[0], hT[0]) and torch.equal(hT2[2], hT[2])
+    assert not torch.equal(out2[:, s:e], out[:, s:e])
+
+
+# ---- the state is the only carry ---------------------------------------------
+def test_split_sequence_consistency():
+    x = ki.make_prefill(_spec("bf16", 128, 128, T=300, h0=True, B=1))
+    out, hT = gpu_prefill(x)
+    t = 137
+    a, b = dict(x), dict(x)
+    for key in ("q", "k", "v", "g", "beta"):
+        a[key] = x[key][:, :t].contiguous()
+        b[key] = x[key][:, t:].contiguous()
+    a["T"], b["T"] = t, 300 - t
+    o1, s1 = gpu_prefill(a)
+    b["h0"] = s1.cpu()
+    o2, s2 = gpu_prefill(b)
+    o_ref, s_ref = oracle_prefill(x)
+    assert rel_err(torch.cat([o1, o2], dim=1), o_ref) <= TOL["bf16"]
+    assert rel_err(s2, s_ref) <= TOL["bf16"]
+
+
+def test_decode_matches_prefill():
+    """16 kda_decode_step calls agree with kda_chunk_fwd over the same 16 tokens
+    with h0 = the decode state (same recurrence in both modes)."""
+    import gated_delta_rule_74_b200 as kda
+    d = ki.make_decode(ki.DecodeSpec("t", N=8, H=4, dk=128, dv=128, steps=16, dtype="bf16",
+                                     decay="alog", seed=9))
+    S = d["S0"].cuda()
+    outs = []
+    for t in range(16):
+        outs.append(kda.kda_decode_step(d["q"][t].cuda(), d["k"][t].cuda(), d["v"][t].cuda(),
+                                        d["g"][t].cuda(), d["beta"][t].cuda(), S))
+    dec = torch.stack(outs, dim=1)                       # [N, 16, H, dv]
+    perm = lambda t: t.transpose(0, 1).contiguous().cuda()
+    out, hT = kda.kda_chunk_fwd(perm(d["q"]), perm(d["k"]), perm(d["v"]), perm(d["g"]),
+                                perm(d["beta"]), h0=d["S0"].cuda())
+    torch.cuda.synchronize()
+    o_ref, s_ref = oracle.prefill(d["q"].transpose(0, 1), d["k"].transpose(0, 1),
+                                  d["v"].transpose(0, 1), d["g"].transpose(0, 1),
+                                  d["beta"].transpose(0, 1), d["S0"])
+    assert rel_err(dec, o_ref) <= TOL["bf16"] and rel_err(out, o_ref) <= TOL["bf16"]
+    assert rel_err(S, s_ref) <= TOL["bf16"] and rel_err(hT, s_ref) <= TOL["bf16"]
