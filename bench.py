@@ -1,0 +1,420 @@
+"""Benchmark of the KDA hot path on B200: chunked prefill and recurrent decode.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload metric|cfg1|cfg2|cfg3]
+
+One JSON line on rank 0.  `value` is prefill tokens/s over all ranks for the
+headline prefill shape (B=1, T=8192, H=12, dk=dv=128, bf16; "metric" workload),
+measured over K timed calls of kda_chunk_fwd with the inputs already in HBM.
+Each rank runs its own shard (independent sequences, no collective: weak
+scaling).  The `decode` object is the second half of the metric: K timed
+kda_decode_step calls on the config-4 shape (N=256 sequences x H=96 heads,
+d=128, 1.61 GB of fp32 state), reported as GB/s of algorithmic traffic and as a
+fraction of the measured HBM peak.
+
+L2: every prefill step reads a different one of three resident input sets
+(3 x 152 MB > 126 MB L2), so no step finds its inputs in L2; the decode state
+(1.61 GB) is far larger than L2.
+
+`--impl reference` times the float64 CPU oracle on a bounded sample of the same
+workload (rank 0 only) and prints the same metric and unit with "impl":
+"reference".
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KDA prefill tokens/s (H=12,d=128,T=8192); decode state GB/s vs HBM peak"
+UNIT = "tokens/s"
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work per call (bytes the method must move at minimum; flops of
+# the chunked form counted as dense tensor-core work)
+# ---------------------------------------------------------------------------
+def prefill_bytes(T_rows: int, H: int, dk: int, dv: int, s_in: int, nseq: int,
+                  h0: bool, hT: bool) -> int:
+    per_tok = (2 * dk + dv) * s_in + 4 * dk + 4 + dv * s_in
+    return T_rows * H * per_tok + nseq * H * 4 * dk * dv * (int(h0) + int(hT))
+
+
+def prefill_flops(T_rows: int, H: int, dk: int, dv: int, C: int = 64) -> int:
+    return T_rows * H * (2 * C * (3 * dk + 2 * dv) + 6 * dk * dv)
+
+
+def decode_bytes(N: int, H: int, dk: int, dv: int, s_in: int) -> int:
+    return N * H * (8 * dk * dv + (2 * dk + dv) * s_in + 4 * dk + 4 + dv * s_in)
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines: list[str] = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def mark(self) -> int:
+        return len(self.lines)
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            if self.t is not None:
+                self.t.join(timeout=2)
+
+    def summary(self, lo: int, hi: int) -> dict:
+        rows = []
+        for line in self.lines[lo:hi] or self.lines[-3:]:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == len(self.FIELDS):
+                rows.append(parts)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "", 1).isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[3 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(rows[0][1]) if rows[0][1].replace(".", "", 1).isdigit() else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+def _dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def run_reference(args, world, rank):
+    """The float64 oracle on the host cores, bounded sample of the workload."""
+    if rank != 0:
+        return 0
+    import kda_inputs as ki
+    import oracle
+    oracle.build()
+    spec = ki.PREFILL_SPECS[args.workload]
+    x = ki.make_prefill(spec)
+    Tb = min(x["T"], args.ref_tokens)
+    q, k, v, g, b = (x[n][:, :Tb] for n in ("q", "k", "v", "g", "beta"))
+    pairs = q.shape[0] * x["H"]
+    threads = min(oracle.max_threads(), pairs)
+    times = []
+    for _ in range(max(1, args.ref_steps)):
+        t0 = time.perf_counter()
+        oracle.prefill(q, k, v, g, b, None, None, nthreads=threads)
+        times.append(time.perf_counter() - t0)
+    tok = Tb * q.shape[0]
+    val = tok / statistics.median(times)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": len(times), "warmup": 0, "ms_per_step": 1e3 * statistics.median(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": _config(args, x, world),
+        "cpu_baseline": {"value": val, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"first {Tb} tokens x {x['H']} heads of the {args.workload} "
+                                   f"workload, float64 recurrence"},
+        "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _config(args, x, world):
+    return {"workload": f"{args.workload}: B={x['B']} T={x['T']} H={x['H']} dk={x['dk']} "
+                        f"dv={x['dv']} {x['dtype']} (seeded synthetic)",
+            "global_batch": x["B"] * world, "seq_len": x["T"], "heads": x["H"],
+            "head_dim": x["dk"], "parallelism": f"dp{world} (independent sequences per rank)",
+            "l2": "prefill rotates 3 resident input sets (3 x inputs > 126 MB L2); decode "
+                  "state 1.61 GB > L2",
+            "decode_workload": "cfg4: N=256 H=96 d=128 bf16, fp32 state 1.61 GB"}
+
+
+def cpu_baseline(args):
+    """Oracle timed on the host cores for a bounded sample (about 10-30 s)."""
+    import kda_inputs as ki
+    import oracle
+    oracle.build()
+    x = ki.make_prefill(args.workload)
+    Tb = min(x["T"], args.ref_tokens)
+    q, k, v, g, b = (x[n][:, :Tb] for n in ("q", "k", "v", "g", "beta"))
+    pairs = q.shape[0] * x["H"]
+    threads = min(oracle.max_threads(), pairs)
+    t0 = time.perf_counter()
+    oracle.prefill(q, k, v, g, b, None, None, nthreads=threads)
+    dt = time.perf_counter() - t0
+    return {"value": Tb * q.shape[0] / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"first {Tb} tokens x {x['H']} heads of the {args.workload} workload "
+                      f"(float64 recurrence, {dt:.1f} s)"}
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    import torch.distributed as dist
+
+    import gated_delta_rule_74_b200 as kda
+    import kda_inputs as ki
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    hbm, tf_burst, tf_sust, peak_kind = _peaks()
+    spec = ki.PREFILL_SPECS[args.workload]
+
+    # ---- prefill inputs: 3 resident sets (different seeds per set and rank)
+    sets = []
+    for i in range(3):
+        x = ki.make_prefill(spec, seed=spec.seed + 1000 * rank + i)
+        d = {n: (t.to(dev) if isinstance(t, torch.Tensor) else t) for n, t in x.items()}
+        d["out"] = torch.empty_like(d["v"])
+        d["hT"] = torch.empty(x["B"], x["H"], x["dk"], x["dv"], device=dev)
+        sets.append(d)
+    x0 = sets[0]
+    rows = x0["T"] if x0["cu_seqlens"] is not None else x0["B"] * x0["T"]
+    s_in = 2 if x0["dtype"] == "bf16" else 4
+    bytes_call = prefill_bytes(rows, x0["H"], x0["dk"], x0["dv"], s_in, x0["B"],
+                               x0["h0"] is not None, True)
+    flops_call = prefill_flops(rows, x0["H"], x0["dk"], x0["dv"])
+    stream = torch.cuda.current_stream()
+
+    def prefill(i):
+        d = sets[i % 3]
+        kda.kda_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], h0=d["h0"],
+                          cu_seqlens=d["cu_seqlens"], out=d["out"], hT=d["hT"], stream=stream)
+
+    clocks = ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                          int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local]))
+    clocks.start()
+    time.sleep(0.3)
+
+    for i in range(args.warmup):
+        prefill(i)
+    torch.cuda.synchronize()
+
+    # ---- timed prefill region
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    mark0 = clocks.mark()
+    n0 = kda.kda_launch_count()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        prefill(i)
+        ev[i][1].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    launches = kda.kda_launch_count() - n0
+    mark1 = clocks.mark()
+    ms_local = t_start.elapsed_time(t_end)
+    per_call = [a.elapsed_time(b) for a, b in ev]
+    ms_max = ms_local
+    if world > 1:
+        t = torch.tensor([ms_local], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+    tokens_total = rows * world * args.steps
+    value = tokens_total / (ms_max / 1e3)
+    call_ms = sum(per_call) / len(per_call)
+    achieved_gbs = bytes_call / (call_ms / 1e3) / 1e9
+    achieved_tf = flops_call / (call_ms / 1e3) / 1e12
+
+    # ---- e2e: host buffers through the C ABI, copies inside the timed region
+    hx = {n: sets[0][n].cpu().pin_memory() for n in ("q", "k", "v", "g", "beta")}
+    h_out = torch.empty(sets[0]["out"].shape, dtype=sets[0]["out"].dtype).pin_memory()
+    h_hT = torch.empty(sets[0]["hT"].shape, dtype=torch.float32).pin_memory()
+    dx = {n: torch.empty_like(sets[0][n]) for n in hx}
+    h2d = sum(t.numel() * t.element_size() for t in hx.values())
+    d2h = h_out.numel() * h_out.element_size() + h_hT.numel() * 4
+    e2e_steps = max(3, args.steps // 4)
+
+    def e2e_step():
+        for n in hx:
+            dx[n].copy_(hx[n], non_blocking=True)
+        kda.kda_chunk_fwd(dx["q"], dx["k"], dx["v"], dx["g"], dx["beta"], h0=sets[0]["h0"],
+                          cu_seqlens=sets[0]["cu_seqlens"], out=sets[0]["out"],
+                          hT=sets[0]["hT"], stream=stream)
+        h_out.copy_(sets[0]["out"], non_blocking=True)
+        h_hT.copy_(sets[0]["hT"], non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_val = rows * world * e2e_steps / (e2e_ms / 1e3)
+    del dx, hx
+
+    # ---- decode leg (config-4 shape)
+    dec = None
+    if not args.no_decode:
+        dspec = ki.DECODE_SPECS["cfg4"]
+        dd = ki.make_decode(dspec, steps=1, seed=dspec.seed + 1000 * rank)
+        S = dd["S0"].to(dev)
+        dq, dk_, dv_, dg, db = (dd[n][0].to(dev) for n in ("q", "k", "v", "g", "beta"))
+        dout = torch.empty(dd["N"], dd["H"], dd["dv"], dtype=dq.dtype, device=dev)
+        dsteps = args.decode_steps
+        for _ in range(args.warmup):
+            kda.kda_decode_step(dq, dk_, dv_, dg, db, S, out=dout, stream=stream)
+        torch.cuda.synchronize()
+        barrier()
+        dmark0 = clocks.mark()
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d0.record(stream)
+        for _ in range(dsteps):
+            kda.kda_decode_step(dq, dk_, dv_, dg, db, S, out=dout, stream=stream)
+        d1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        dmark1 = clocks.mark()
+        dms = d0.elapsed_time(d1)
+        if world > 1:
+            t = torch.tensor([dms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            dms = float(t.item())
+        dbytes = decode_bytes(dd["N"], dd["H"], dd["dk"], dd["dv"], 2)
+        step_ms = dms / dsteps
+        gbs = dbytes / (step_ms / 1e3) / 1e9
+        dec = {"metric": "decode state GB/s vs HBM peak", "gbs": gbs, "frac_of_hbm_peak": gbs / hbm,
+               "peak_gbs": hbm, "peak_kind": peak_kind, "steps_per_s": 1e3 / step_ms,
+               "tokens_per_s": dd["N"] * world * 1e3 / step_ms, "ms_per_step": step_ms,
+               "steps": dsteps, "bytes_per_step": dbytes,
+               "clocks": clocks.summary(dmark0, dmark1)}
+        del S
+    clocks.stop()
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args)
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        try:
+            with open(tpath) as f:
+                traffic = json.load(f).get(args.workload)
+        except Exception:
+            traffic = None
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if s_in == 2 else "f32",
+        "data": "synthetic (seeded random inputs shaped like the pages' models)",
+        "config": _config(args, x0, world),
+        "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved_gbs / hbm, "traffic": traffic,
+                     "kernel": "kda_chunk_fwd (prefill)", "peak_kind": peak_kind,
+                     "algorithmic_bytes_per_launch": bytes_call,
+                     "avg_launch_ms": call_ms,
+                     "tensor": {"achieved_tflops": achieved_tf, "peak_sustained": tf_sust,
+                                "frac_sustained": achieved_tf / tf_sust,
+                                "flops_per_launch": flops_call}},
+        "decode": dec,
+        "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": launches,
+        "clocks": clocks.summary(mark0, mark1),
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="metric", choices=["metric", "cfg1", "cfg2", "cfg3"])
+    ap.add_argument("--decode-steps", type=int, default=100)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-tokens", type=int, default=2048,
+                    help="tokens of the workload the oracle processes per timed sample")
+    ap.add_argument("--ref-steps", type=int, default=1)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)     # at least 3 untimed warm-up steps
+    world, rank, local = _dist()
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+    return run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -19,6 +19,7 @@ from typing import Optional
 import torch
 
 __all__ = ["kda_chunk_fwd", "kda_decode_step", "kda_status_string", "kda_version",
+           "kda_launch_count",
            "lib", "library_path", "header_symbols", "KdaError",
            "KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED", "KDA_ERR_CUDA",
            "KDA_ERR_TIMEOUT", "KDA_BF16", "KDA_F32"]
@@ -63,6 +64,8 @@ def lib() -> ctypes.CDLL:
         L.kda_status_string.restype = ctypes.c_char_p
         L.kda_version.argtypes = []
         L.kda_version.restype = ctypes.c_int
+        L.kda_launch_count.argtypes = []
+        L.kda_launch_count.restype = ctypes.c_ulonglong
         _lib = L
     return _lib
 
@@ -80,6 +83,11 @@ def kda_status_string(status: int) -> str:
 
 def kda_version() -> int:
     return int(lib().kda_version())
+
+
+def kda_launch_count() -> int:
+    """Kernels launched by libkda in this process so far."""
+    return int(lib().kda_launch_count())
 
 
 def _ptr(t: Optional[torch.Tensor]):

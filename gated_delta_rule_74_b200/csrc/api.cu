@@ -2,9 +2,15 @@
 // The entry points and their contracts are declared and documented in kda.h.
 #include <stdint.h>
 
+#include <atomic>
 #include <initializer_list>
 
 #include "kda_common.cuh"
+
+namespace kda {
+static std::atomic<unsigned long long> g_launches{0};
+void note_launches(unsigned long long n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+}  // namespace kda
 
 namespace {
 
@@ -80,5 +86,9 @@ const char* kda_status_string(int status) {
 }
 
 int kda_version(void) { return (kVersionMajor << 16) | kVersionMinor; }
+
+unsigned long long kda_launch_count(void) {
+  return kda::g_launches.load(std::memory_order_relaxed);
+}
 
 }  // extern "C"

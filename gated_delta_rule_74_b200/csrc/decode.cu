@@ -125,6 +125,7 @@ cudaError_t launch_t(const void* q, const void* k, const void* v, const float* g
   kda_decode_kernel<Tin, DK, DV><<<(unsigned)pairs, kThreads, 0, stream>>>(
       static_cast<const Tin*>(q), static_cast<const Tin*>(k), static_cast<const Tin*>(v),
       g, beta, S, static_cast<Tin*>(out));
+  note_launches(1);
   return cudaGetLastError();
 }
 

@@ -18,6 +18,9 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
   return __float2bfloat16_rn(x);
 }
 
+// Count of kernel launches made by the library (see kda_launch_count()).
+void note_launches(unsigned long long n);
+
 // Launchers implemented in the kernel translation units.  Each returns a
 // cudaError_t from the launch (cudaSuccess when the launch was accepted).
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* g,

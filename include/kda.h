@@ -119,6 +119,10 @@ KDA_API const char* kda_status_string(int status);
 /* Library ABI version: (major << 16) | minor. */
 KDA_API int kda_version(void);
 
+/* Number of CUDA kernels this library has launched in the calling process
+ * since it was loaded (all threads, all devices).  Diagnostic only. */
+KDA_API unsigned long long kda_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif
