@@ -138,29 +138,15 @@ def run_reference(args, world, rank):
     if rank != 0:
         return 0
     import kda_inputs as ki
-    import oracle
-    oracle.build()
-    spec = ki.PREFILL_SPECS[args.workload]
-    x = ki.make_prefill(spec)
-    Tb = min(x["T"], args.ref_tokens)
-    q, k, v, g, b = (x[n][:, :Tb] for n in ("q", "k", "v", "g", "beta"))
-    pairs = q.shape[0] * x["H"]
-    threads = min(oracle.max_threads(), pairs)
-    times = []
-    for _ in range(max(1, args.ref_steps)):
-        t0 = time.perf_counter()
-        oracle.prefill(q, k, v, g, b, None, None, nthreads=threads)
-        times.append(time.perf_counter() - t0)
-    tok = Tb * q.shape[0]
-    val = tok / statistics.median(times)
+    val, threads, desc, times = _oracle_timing(args)
+    x = ki.make_prefill(args.workload)
     line = {
         "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus,
         "steps": len(times), "warmup": 0, "ms_per_step": 1e3 * statistics.median(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": _config(args, x, world),
         "cpu_baseline": {"value": val, "unit": UNIT, "cores": threads, "kind": "oracle",
-                         "sample": f"first {Tb} tokens x {x['H']} heads of the {args.workload} "
-                                   f"workload, float64 recurrence"},
+                         "sample": desc},
         "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -177,47 +163,63 @@ def _config(args, x, world):
             "decode_workload": "cfg4: N=256 H=96 d=128 bf16, fp32 state 1.61 GB"}
 
 
-def cpu_baseline(args):
-    """Oracle timed on the host cores for a bounded sample (about 10-30 s)."""
+def _oracle_timing(args):
+    """Float64 oracle over the whole workload (or its first --ref-tokens tokens),
+    repeated until about --ref-seconds of CPU time have passed.  Returns
+    (tokens/s of the median pass, threads used, sample description, pass times)."""
     import kda_inputs as ki
     import oracle
     oracle.build()
     x = ki.make_prefill(args.workload)
-    Tb = min(x["T"], args.ref_tokens)
+    Tb = min(x["T"], args.ref_tokens) if args.ref_tokens > 0 else x["T"]
     q, k, v, g, b = (x[n][:, :Tb] for n in ("q", "k", "v", "g", "beta"))
-    pairs = q.shape[0] * x["H"]
-    threads = min(oracle.max_threads(), pairs)
-    t0 = time.perf_counter()
-    oracle.prefill(q, k, v, g, b, None, None, nthreads=threads)
-    dt = time.perf_counter() - t0
-    return {"value": Tb * q.shape[0] / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": f"first {Tb} tokens x {x['H']} heads of the {args.workload} workload "
-                      f"(float64 recurrence, {dt:.1f} s)"}
+    cu = None
+    if x["cu_seqlens"] is not None:
+        import torch
+        cu = torch.clamp(x["cu_seqlens"], max=Tb)
+    pairs = (q.shape[0] if cu is None else cu.numel() - 1) * x["H"]
+    threads = max(1, min(oracle.max_threads(), pairs))
+    times = []
+    t_all = time.perf_counter()
+    while True:
+        t0 = time.perf_counter()
+        oracle.prefill(q, k, v, g, b, None, cu, nthreads=threads)
+        times.append(time.perf_counter() - t0)
+        if time.perf_counter() - t_all >= args.ref_seconds or len(times) >= 50:
+            break
+    tok = Tb * q.shape[0]
+    med = statistics.median(times)
+    desc = (f"{'all' if Tb == x['T'] else 'first'} {Tb} tokens x {x['H']} heads of the "
+            f"{args.workload} workload, float64 recurrence, {len(times)} passes "
+            f"({sum(times):.1f} s)")
+    return tok / med, threads, desc, times
 
 
-def run_ours(args, world, rank, local):
+def cpu_baseline(args):
+    """Oracle timed on the host cores on a bounded sample (about 10-30 s)."""
+    val, threads, desc, _ = _oracle_timing(args)
+    return {"value": val, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
+
+
+def _max_over_ranks(val, world, dev):
+    if world == 1:
+        return val
     import torch
     import torch.distributed as dist
+    t = torch.tensor([val], device=dev, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def prefill_leg(args, world, rank, dev, stream, barrier, clocks):
+    """K timed kda_chunk_fwd calls on resident inputs, then the e2e leg."""
+    import torch
 
     import gated_delta_rule_74_b200 as kda
     import kda_inputs as ki
 
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    hbm, tf_burst, tf_sust, peak_kind = _peaks()
     spec = ki.PREFILL_SPECS[args.workload]
-
-    # ---- prefill inputs: 3 resident sets (different seeds per set and rank)
-    sets = []
+    sets = []                       # 3 resident input sets (L2 rotation)
     for i in range(3):
         x = ki.make_prefill(spec, seed=spec.seed + 1000 * rank + i)
         d = {n: (t.to(dev) if isinstance(t, torch.Tensor) else t) for n, t in x.items()}
@@ -230,31 +232,23 @@ def run_ours(args, world, rank, local):
     bytes_call = prefill_bytes(rows, x0["H"], x0["dk"], x0["dv"], s_in, x0["B"],
                                x0["h0"] is not None, True)
     flops_call = prefill_flops(rows, x0["H"], x0["dk"], x0["dv"])
-    stream = torch.cuda.current_stream()
 
     def prefill(i):
         d = sets[i % 3]
         kda.kda_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], h0=d["h0"],
                           cu_seqlens=d["cu_seqlens"], out=d["out"], hT=d["hT"], stream=stream)
 
-    clocks = ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ else
-                          int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local]))
-    clocks.start()
-    time.sleep(0.3)
-
     for i in range(args.warmup):
         prefill(i)
     torch.cuda.synchronize()
-
-    # ---- timed prefill region
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     mark0 = clocks.mark()
     n0 = kda.kda_launch_count()
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
     for i in range(args.steps):
         ev[i][0].record(stream)
@@ -265,24 +259,14 @@ def run_ours(args, world, rank, local):
     barrier()
     launches = kda.kda_launch_count() - n0
     mark1 = clocks.mark()
-    ms_local = t_start.elapsed_time(t_end)
-    per_call = [a.elapsed_time(b) for a, b in ev]
-    ms_max = ms_local
-    if world > 1:
-        t = torch.tensor([ms_local], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
-    tokens_total = rows * world * args.steps
-    value = tokens_total / (ms_max / 1e3)
-    call_ms = sum(per_call) / len(per_call)
-    achieved_gbs = bytes_call / (call_ms / 1e3) / 1e9
-    achieved_tf = flops_call / (call_ms / 1e3) / 1e12
+    ms_max = _max_over_ranks(t_start.elapsed_time(t_end), world, dev)
+    call_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
 
-    # ---- e2e: host buffers through the C ABI, copies inside the timed region
-    hx = {n: sets[0][n].cpu().pin_memory() for n in ("q", "k", "v", "g", "beta")}
-    h_out = torch.empty(sets[0]["out"].shape, dtype=sets[0]["out"].dtype).pin_memory()
-    h_hT = torch.empty(sets[0]["hT"].shape, dtype=torch.float32).pin_memory()
-    dx = {n: torch.empty_like(sets[0][n]) for n in hx}
+    # e2e: pinned host buffers -> device -> kda_chunk_fwd -> host, all timed
+    hx = {n: x0[n].cpu().pin_memory() for n in ("q", "k", "v", "g", "beta")}
+    h_out = torch.empty(x0["out"].shape, dtype=x0["out"].dtype).pin_memory()
+    h_hT = torch.empty(x0["hT"].shape, dtype=torch.float32).pin_memory()
+    dx = {n: torch.empty_like(x0[n]) for n in hx}
     h2d = sum(t.numel() * t.element_size() for t in hx.values())
     d2h = h_out.numel() * h_out.element_size() + h_hT.numel() * 4
     e2e_steps = max(3, args.steps // 4)
@@ -290,11 +274,11 @@ def run_ours(args, world, rank, local):
     def e2e_step():
         for n in hx:
             dx[n].copy_(hx[n], non_blocking=True)
-        kda.kda_chunk_fwd(dx["q"], dx["k"], dx["v"], dx["g"], dx["beta"], h0=sets[0]["h0"],
-                          cu_seqlens=sets[0]["cu_seqlens"], out=sets[0]["out"],
-                          hT=sets[0]["hT"], stream=stream)
-        h_out.copy_(sets[0]["out"], non_blocking=True)
-        h_hT.copy_(sets[0]["hT"], non_blocking=True)
+        kda.kda_chunk_fwd(dx["q"], dx["k"], dx["v"], dx["g"], dx["beta"], h0=x0["h0"],
+                          cu_seqlens=x0["cu_seqlens"], out=x0["out"], hT=x0["hT"],
+                          stream=stream)
+        h_out.copy_(x0["out"], non_blocking=True)
+        h_hT.copy_(x0["hT"], non_blocking=True)
 
     for _ in range(2):
         e2e_step()
@@ -306,53 +290,89 @@ def run_ours(args, world, rank, local):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_val = rows * world * e2e_steps / (e2e_ms / 1e3)
-    del dx, hx
+    barrier()
+    e2e_ms = _max_over_ranks(e0.elapsed_time(e1), world, dev)
+    return dict(x0=x0, rows=rows, s_in=s_in, bytes_call=bytes_call, flops_call=flops_call,
+                value=rows * world * args.steps / (ms_max / 1e3), ms_max=ms_max,
+                call_ms=call_ms, launches=launches, clocks=clocks.summary(mark0, mark1),
+                e2e={"value": rows * world * e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
+                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                     "steps": e2e_steps})
 
-    # ---- decode leg (config-4 shape)
+
+def decode_leg(args, world, rank, dev, stream, barrier, clocks, hbm, peak_kind):
+    """K timed kda_decode_step calls on the config-4 shape (state in HBM)."""
+    import torch
+
+    import gated_delta_rule_74_b200 as kda
+    import kda_inputs as ki
+
+    dspec = ki.DECODE_SPECS["cfg4"]
+    dd = ki.make_decode(dspec, steps=1, seed=dspec.seed + 1000 * rank, N=args.decode_n or None)
+    S = dd["S0"].to(dev)
+    q, k, v, g, b = (dd[n][0].to(dev) for n in ("q", "k", "v", "g", "beta"))
+    out = torch.empty(dd["N"], dd["H"], dd["dv"], dtype=q.dtype, device=dev)
+    for _ in range(args.warmup):
+        kda.kda_decode_step(q, k, v, g, b, S, out=out, stream=stream)
+    torch.cuda.synchronize()
+    barrier()
+    mark0 = clocks.mark()
+    n0 = kda.kda_launch_count()
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    d0.record(stream)
+    for _ in range(args.decode_steps):
+        kda.kda_decode_step(q, k, v, g, b, S, out=out, stream=stream)
+    d1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    launches = kda.kda_launch_count() - n0
+    dms = _max_over_ranks(d0.elapsed_time(d1), world, dev)
+    dbytes = decode_bytes(dd["N"], dd["H"], dd["dk"], dd["dv"], 2)
+    step_ms = dms / args.decode_steps
+    gbs = dbytes / (step_ms / 1e3) / 1e9
+    return {"metric": "decode state GB/s vs HBM peak", "workload":
+            f"cfg4 shape: N={dd['N']} H={dd['H']} dk=dv=128 bf16 q/k/v, fp32 state "
+            f"{dd['N'] * dd['H'] * 65536 / 1e9:.2f} GB", "gbs": gbs,
+            "frac_of_hbm_peak": gbs / hbm, "peak_gbs": hbm, "peak_kind": peak_kind,
+            "steps_per_s": 1e3 / step_ms, "tokens_per_s": dd["N"] * world * 1e3 / step_ms,
+            "ms_per_step": step_ms, "steps": args.decode_steps, "bytes_per_step": dbytes,
+            "gpu_launches": launches, "clocks": clocks.summary(mark0, clocks.mark())}
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    import torch.distributed as dist
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    hbm, tf_burst, tf_sust, peak_kind = _peaks()
+    stream = torch.cuda.current_stream()
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    clocks = ClockSampler(int(vis.split(",")[local]) if vis else local)
+    clocks.start()
+    time.sleep(0.3)
+    pf = None
+    if not args.decode_only:
+        pf = prefill_leg(args, world, rank, dev, stream, barrier, clocks)
     dec = None
     if not args.no_decode:
-        dspec = ki.DECODE_SPECS["cfg4"]
-        dd = ki.make_decode(dspec, steps=1, seed=dspec.seed + 1000 * rank)
-        S = dd["S0"].to(dev)
-        dq, dk_, dv_, dg, db = (dd[n][0].to(dev) for n in ("q", "k", "v", "g", "beta"))
-        dout = torch.empty(dd["N"], dd["H"], dd["dv"], dtype=dq.dtype, device=dev)
-        dsteps = args.decode_steps
-        for _ in range(args.warmup):
-            kda.kda_decode_step(dq, dk_, dv_, dg, db, S, out=dout, stream=stream)
-        torch.cuda.synchronize()
-        barrier()
-        dmark0 = clocks.mark()
-        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        d0.record(stream)
-        for _ in range(dsteps):
-            kda.kda_decode_step(dq, dk_, dv_, dg, db, S, out=dout, stream=stream)
-        d1.record(stream)
-        torch.cuda.synchronize()
-        barrier()
-        dmark1 = clocks.mark()
-        dms = d0.elapsed_time(d1)
-        if world > 1:
-            t = torch.tensor([dms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            dms = float(t.item())
-        dbytes = decode_bytes(dd["N"], dd["H"], dd["dk"], dd["dv"], 2)
-        step_ms = dms / dsteps
-        gbs = dbytes / (step_ms / 1e3) / 1e9
-        dec = {"metric": "decode state GB/s vs HBM peak", "gbs": gbs, "frac_of_hbm_peak": gbs / hbm,
-               "peak_gbs": hbm, "peak_kind": peak_kind, "steps_per_s": 1e3 / step_ms,
-               "tokens_per_s": dd["N"] * world * 1e3 / step_ms, "ms_per_step": step_ms,
-               "steps": dsteps, "bytes_per_step": dbytes,
-               "clocks": clocks.summary(dmark0, dmark1)}
-        del S
+        dec = decode_leg(args, world, rank, dev, stream, barrier, clocks, hbm, peak_kind)
     clocks.stop()
 
     if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
+    if pf is None:
+        print(json.dumps({"metric": METRIC, "decode_only": True, "decode": dec}), flush=True)
         if world > 1:
             dist.destroy_process_group()
         return 0
@@ -368,26 +388,25 @@ def run_ours(args, world, rank, local):
                 traffic = json.load(f).get(args.workload)
         except Exception:
             traffic = None
+    achieved_gbs = pf["bytes_call"] / (pf["call_ms"] / 1e3) / 1e9
+    achieved_tf = pf["flops_call"] / (pf["call_ms"] / 1e3) / 1e12
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if s_in == 2 else "f32",
+        "metric": METRIC, "value": pf["value"], "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": pf["ms_max"] / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if pf["s_in"] == 2 else "f32",
         "data": "synthetic (seeded random inputs shaped like the pages' models)",
-        "config": _config(args, x0, world),
+        "config": _config(args, pf["x0"], world),
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm, "unit": "GB/s",
                      "frac": achieved_gbs / hbm, "traffic": traffic,
                      "kernel": "kda_chunk_fwd (prefill)", "peak_kind": peak_kind,
-                     "algorithmic_bytes_per_launch": bytes_call,
-                     "avg_launch_ms": call_ms,
+                     "algorithmic_bytes_per_launch": pf["bytes_call"],
+                     "avg_launch_ms": pf["call_ms"],
                      "tensor": {"achieved_tflops": achieved_tf, "peak_sustained": tf_sust,
                                 "frac_sustained": achieved_tf / tf_sust,
-                                "flops_per_launch": flops_call}},
-        "decode": dec,
-        "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
-        "gpu_launches": launches,
-        "clocks": clocks.summary(mark0, mark1),
-        "cpu_baseline": cpu,
+                                "flops_per_launch": pf["flops_call"]}},
+        "decode": dec, "e2e": pf["e2e"], "gpu_launches": pf["launches"],
+        "clocks": pf["clocks"], "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)
     if world > 1:
@@ -404,10 +423,15 @@ def main():
     ap.add_argument("--workload", default="metric", choices=["metric", "cfg1", "cfg2", "cfg3"])
     ap.add_argument("--decode-steps", type=int, default=100)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="skip the prefill legs (for profiling the decode kernel)")
+    ap.add_argument("--decode-n", type=int, default=0,
+                    help="sequences in the decode leg (0 = the config-4 value, 256)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ref-tokens", type=int, default=2048,
-                    help="tokens of the workload the oracle processes per timed sample")
-    ap.add_argument("--ref-steps", type=int, default=1)
+    ap.add_argument("--ref-tokens", type=int, default=0,
+                    help="tokens of the workload the oracle processes per pass (0 = all)")
+    ap.add_argument("--ref-seconds", type=float, default=10.0,
+                    help="repeat oracle passes until this much time has passed")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)     # at least 3 untimed warm-up steps
     world, rank, local = _dist()
