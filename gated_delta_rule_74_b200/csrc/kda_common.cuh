@@ -32,4 +32,10 @@ cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const
                               void* out, float* hT, int B, int T, int H, int dk, int dv,
                               int in_dtype, cudaStream_t stream);
 
+// Tensor-core chunked prefill (bf16, dk = dv = 128).
+bool chunk_tc_supported(int dk, int dv, int in_dtype);
+cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const float* g,
+                            const float* beta, const float* h0, const int32_t* cu_seqlens,
+                            void* out, float* hT, int B, int T, int H, cudaStream_t stream);
+
 }  // namespace kda
