@@ -13,18 +13,20 @@
 //     Delta    = U - W S
 //     O        = Qbar S + Aqk Delta,                     Qbar_r = exp(G_r) q_r
 //     S_next   = Diag(exp(G_63)) S + Kend^T Delta,       Kend_i = exp(G_63 - G_i) k_i
-// Rows past the end of a sequence are zero (k = q = v = beta = g = 0) and so
+// Rows past the end of a sequence are zero (k = q = beta = g = 0) and so
 // contribute nothing.
 //
 // Decay factoring.  exp(G_r - G_i) is split through reference points so that no
 // factor overflows: rows are grouped in 16-token blocks a; P_a = G at row 16a.
-//   diagonal block (i, r in block a):  (k_r e^{G_r - P_a}) . (k_i e^{P_a - G_i})
-//     first factor <= 1, second <= e^{decay over <= 15 tokens} (clamped at e^80)
-//   i in an earlier block b < a:        (k_r e^{G_r - P_a}) . (k_i e^{P_a - G_i})
-//     with e^{P_a - G_i} = e^{P_{b+1} - G_i} e^{P_a - P_{b+1}}, both <= 1.
-// So the Gram of row block a is one MMA against R^(a) = [k_i e^{P_a - G_i}]_{i<16(a+1)}.
-// The only range limit: within one 16-token block the cumulative log-decay must
-// stay above -80 per channel (|g| below about 5 per token on average).
+//   i, r in block a:   (k_r e^{G_r - P_a}) (k_i e^{P_a - G_i})
+//       first factor <= 1; second <= e^{decay over <= 15 tokens}, clamped at e^80
+//   i in block b < a:  (k_r e^{G_r - P_a}) (k_i e^{P_b - G_i} e^{P_a - P_b})
+//       with e^{P_a - G_i} <= 1.
+// So the Gram of row block a is one MMA against R^(a) = [k_i e^{P_a - G_i}]_{i<16(a+1)},
+// and every other operand is one of these factors times a per-(block, channel)
+// constant: two exponentials per element in all.  The only range limit: within
+// one 16-token block the cumulative log-decay must stay above -80 per channel
+// (|g| below about 5 per token on average).
 //
 // Everything is computed transposed so that every MMA has M = 128 (the channel
 // or value index on the TMEM lanes):
@@ -36,16 +38,16 @@
 //   S^T   += Delta^T Kend   (after S^T <- S^T Diag(exp(G_63)))
 // The state S^T [dv x dk] stays in TMEM in fp32 for the whole sequence; a bf16
 // copy is the MMA operand.  The 64 x 64 triangular inverse runs on the CUDA
-// cores in fp32 (16 x 16 diagonal blocks by forward substitution, then the
-// off-diagonal blocks block-row by block-row).
+// cores in fp32: 16 x 16 diagonal blocks by forward substitution, then
+// T_ab = -sum_{m=b}^{a-1} (T_aa B_am) T_mb block-row by block-row.
 //
 // Mapping: one CTA (256 threads) per (sequence, head) walks the chunks in order.
-// Threads 0-127 ("channel threads", thread c <-> key channel c = TMEM lane c)
-// build the decayed operands; threads 128-255 ("value threads", j <-> value
-// column j = TMEM lane j) own the state and the outputs.  Thread 0 issues the
-// MMAs.  Packed documents restart the state from their own h0 slot and restart
-// chunking at the document start (Mini-K3-1H-mamba2 card, packed-document
-// paragraph: state flow resets at every boundary).
+// The next chunk's inputs are fetched with cp.async while the current chunk
+// computes.  Threads 0-127 map to key channels / TMEM lanes for the operands
+// with M = dk; threads 128-255 own the state rows S^T[j] and the outputs.
+// Thread 0 issues the MMAs.  Packed documents restart the state from their own
+// h0 slot and restart chunking at the document start (Mini-K3-1H-mamba2 card,
+// packed-document paragraph: state flow resets at every boundary).
 #include "kda_common.cuh"
 #include "sm100.cuh"
 
@@ -62,24 +64,27 @@ constexpr int C = 64;
 constexpr int D = 128;
 constexpr int NT = 256;
 
-// shared memory map (bytes from a 1024-aligned base)
-// region A [0, 64K): staging during operand build, then the small operands
+// ---- shared memory map (bytes from a 1024-aligned base)
+// region A [0, 64K): cp.async staging of q, k (bf16 row-major) and g (fp32)
 constexpr uint32_t OFF_SQ = 0, OFF_SK = 16384, OFF_SG = 32768;
-constexpr uint32_t OFF_AQK = 0, OFF_TB = 8192, OFF_WT = 16384;
-// region B [64K, 136K): Gram operands, then the triangular-solve scratch
-constexpr uint32_t OFF_L = 65536;
-// R^(a) buffers: N = 16(a+1) tokens x 128 channels, MN-major SW32 (4, 8, 12, 16 KB)
-__host__ __device__ constexpr uint32_t off_r(int a) {
+// region B [64K, 136K): Gram operands during the build ...
+constexpr uint32_t OFF_L = 65536;                       // [Lk; Lq], 32 KB
+__host__ __device__ constexpr uint32_t off_r(int a) {   // R^(a): 4, 8, 12, 16 KB
   return a == 0 ? 98304u : a == 1 ? 102400u : a == 2 ? 110592u : 122880u;
 }
-constexpr uint32_t OFF_A32 = 65536, OFF_T32 = 65536 + 17408, OFF_Y = 65536 + 34816;
-constexpr int LDA = 65;   // padded fp32 row stride of the solve scratch
+// ... then, once the Gram has been read: solve scratch and small operands
+constexpr int LDA = 68;                                 // fp32 row stride (16-byte rows)
+constexpr uint32_t OFF_B32 = 65536;                     // diag(beta) A, fp32
+constexpr uint32_t OFF_T32 = 65536 + 17408;             // T, fp32
+constexpr uint32_t OFF_M32 = 65536 + 34816;             // T_aa B_am, 6 x 16 x 16 fp32
+constexpr uint32_t OFF_AQK = 106496, OFF_TB = 114688, OFF_WT = 122880;
+constexpr uint32_t OFF_OUT = 65536;                     // output tile (after the solve)
 // region C [136K, 184K)
 constexpr uint32_t OFF_V = 139264, OFF_QB = 155648, OFF_KE = 172032;
 constexpr uint32_t SMEM_USED = 188416;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
 
-// TMEM columns (512 allocated)
+// ---- TMEM columns (512 allocated)
 constexpr uint32_t TM_S = 0;        // S^T fp32        [128 lanes x 128]
 constexpr uint32_t TM_SB = 128;     // S^T bf16 (A)    [128 x 64]
 constexpr uint32_t TM_KB = 192;     // Kbar^T bf16 (A) [128 x 32], later Delta^T bf16 (A)
@@ -91,9 +96,101 @@ constexpr uint32_t TM_U = 448;      // U^T [128 x 64]
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kWaitLimit = 1u << 22;
 
-__device__ __forceinline__ void st_shared_v4(uint8_t* base, uint32_t off, uint32_t a, uint32_t b,
-                                             uint32_t c, uint32_t d) {
+__device__ __forceinline__ void st_v4(uint8_t* base, uint32_t off, uint32_t a, uint32_t b,
+                                      uint32_t c, uint32_t d) {
   *reinterpret_cast<uint4*>(base + off) = make_uint4(a, b, c, d);
+}
+__device__ __forceinline__ void st_v4f(uint8_t* base, uint32_t off, const float (&x)[8], float s) {
+  st_v4(base, off, pack_bf16(x[0] * s, x[1] * s), pack_bf16(x[2] * s, x[3] * s),
+        pack_bf16(x[4] * s, x[5] * s), pack_bf16(x[6] * s, x[7] * s));
+}
+
+// Issue the cp.async loads of one chunk's q, k, g into the staging region
+// (rows >= L zero-filled; their source address is clamped in bounds).
+__device__ __forceinline__ void prefetch_qkg(uint8_t* sm, const bf16* q, const bf16* k,
+                                             const float* g, long long rowbase, int L, int H,
+                                             int h, int tid) {
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int idx = tid + it * NT;
+    const int r = idx >> 4, ch = idx & 15;
+    const long long e = ((rowbase + min(r, L - 1)) * H + h) * D + ch * 8;
+    const uint32_t n = r < L ? 16u : 0u;
+    cp_async16(sm + OFF_SQ + r * 256 + ch * 16, q + e, n);
+    cp_async16(sm + OFF_SK + r * 256 + ch * 16, k + e, n);
+  }
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int idx = tid + it * NT;
+    const int r = idx >> 5, ch = idx & 31;
+    const long long e = ((rowbase + min(r, L - 1)) * H + h) * D + ch * 4;
+    cp_async16(sm + OFF_SG + r * 512 + ch * 16, g + e, r < L ? 16u : 0u);
+  }
+}
+// v rows go straight into the MN-major SW128 operand layout (M = value j, K = token).
+__device__ __forceinline__ void prefetch_v(uint8_t* sm, const bf16* v, long long rowbase, int L,
+                                           int H, int h, int tid) {
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int idx = tid + it * NT;
+    const int r = idx >> 4, ch = idx & 15;
+    const long long e = ((rowbase + min(r, L - 1)) * H + h) * D + ch * 8;
+    cp_async16(sm + OFF_V + chunk_mnmajor_sw128(ch, r, C), v + e, r < L ? 16u : 0u);
+  }
+}
+
+// Operand build for rows [32*HF, 32*HF + 32) of the chunk, key channel c;
+// gv holds the cumulative log-decay of those rows.
+template <int HF>
+__device__ __forceinline__ void build_half(uint8_t* sm, const float (&gv)[32], const bf16* kc,
+                                           const bf16* qc, int c, float P0, float P1, float P2,
+                                           float P3, float G63, uint32_t tm_kb) {
+  const float P[4] = {P0, P1, P2, P3};
+  uint32_t kbw[16];
+#pragma unroll
+  for (int lb = 0; lb < 2; ++lb) {
+    const int a = 2 * HF + lb;
+    const float Pa = P[a];
+    const float eP = __expf(Pa);                 // Kbar, Qbar: e^{G_r} = e^{G_r - P_a} e^{P_a}
+    const float eE = __expf(G63 - Pa);           // Kend: e^{G63 - G_i} = e^{P_a - G_i} e^{G63 - P_a}
+    const float f1 = a + 1 <= 3 ? __expf(P[a + 1 <= 3 ? a + 1 : 3] - Pa) : 0.f;
+    const float f2 = a + 2 <= 3 ? __expf(P[a + 2 <= 3 ? a + 2 : 3] - Pa) : 0.f;
+    const float f3 = a + 3 <= 3 ? __expf(P[3] - Pa) : 0.f;
+#pragma unroll
+    for (int gg = 0; gg < 2; ++gg) {
+      const int g8 = 2 * a + gg;                 // global group of 8 rows
+      float lk[8], lq[8], kr[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int r = g8 * 8 + e;
+        const float x = gv[r - 32 * HF] - Pa;
+        const float ell = __expf(x);
+        const float rho = __expf(fminf(-x, 80.f));
+        const float kv = __bfloat162float(kc[r * D]);
+        const float qv = __bfloat162float(qc[r * D]);
+        lk[e] = kv * ell;
+        lq[e] = qv * ell;
+        kr[e] = kv * rho;                        // k_i e^{P_a - G_i}
+      }
+      // L = [Lk ; Lq]: A operand of the Gram, MN-major SW128 (M = 128, K = channels)
+      st_v4f(sm, OFF_L + chunk_mnmajor_sw128(g8, c, D), lk, 1.f);
+      st_v4f(sm, OFF_L + chunk_mnmajor_sw128(8 + g8, c, D), lq, 1.f);
+      // Qbar^T: B operand of O^T, MN-major SW128 (N = tokens, K = channels)
+      st_v4f(sm, OFF_QB + chunk_mnmajor_sw128(g8, c, D), lq, eP);
+      // Kend^T: B operand of the state update, K-major SW128 (N = channels, K = tokens)
+      st_v4f(sm, OFF_KE + chunk_kmajor_sw128(c, g8, D), kr, eE);
+      // R^(a'), a' >= a: B operands of the Gram, MN-major SW32 (N = 16(a'+1), K = channels)
+      st_v4f(sm, off_r(a) + chunk_mnmajor_sw32(g8, c, D), kr, 1.f);
+      if (a + 1 <= 3) st_v4f(sm, off_r(a + 1 <= 3 ? a + 1 : 3) + chunk_mnmajor_sw32(g8, c, D), kr, f1);
+      if (a + 2 <= 3) st_v4f(sm, off_r(a + 2 <= 3 ? a + 2 : 3) + chunk_mnmajor_sw32(g8, c, D), kr, f2);
+      if (a + 3 <= 3) st_v4f(sm, off_r(3) + chunk_mnmajor_sw32(g8, c, D), kr, f3);
+      // Kbar^T: A operand in TMEM, lane c, two tokens per 32-bit column
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        kbw[(lb * 2 + gg) * 4 + e] = pack_bf16(lk[2 * e] * eP, lk[2 * e + 1] * eP);
+    }
+  }
+  tmem_st16(tm_kb + 16 * HF, kbw);
 }
 
 __global__ void __launch_bounds__(NT, 1)
@@ -109,10 +206,11 @@ kda_chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   __shared__ uint32_t tmem_base_sh;
   __shared__ float s_beta[C];
   __shared__ float s_gamma[D];
+  __shared__ float s_pref[5][D];       // P0, P1, P2, P3, G63 per channel
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = blockIdx.x, s = blockIdx.y;
-  const bool is_val = tid >= 128;
+  const bool upper = tid >= 128;       // second warpgroup
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
 
   long long row0, t_beg, t_end;
@@ -134,24 +232,31 @@ kda_chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     mbar_init(&bar, 1);
     fence_mbar_init();
   }
+  // first chunk's inputs
+  float beta_next = 0.f;
+  if (t_beg < t_end) {
+    const int L0 = (int)min((long long)C, t_end - t_beg);
+    prefetch_qkg(sm, q, k, g, row0 + t_beg, L0, H, h, tid);
+    prefetch_v(sm, v, row0 + t_beg, L0, H, h, tid);
+    cp_async_commit();
+    if (tid < C && tid < L0) beta_next = beta[(row0 + t_beg + tid) * H + h];
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = tmem_base_sh;
   uint32_t phase = 0;
 
-  // ---- initial state: value thread j holds row j of S^T (= column j of S)
-  if (is_val) {
+  // ---- initial state: upper thread j holds row j of S^T (= column j of S)
+  if (upper) {
     const int j = tid - 128;
 #pragma unroll 1
     for (int c0 = 0; c0 < D; c0 += 32) {
       uint32_t f[16], f2[16], pk[16];
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
-        const float x0 = h0 ? h0[sbase + (long long)(c0 + e) * D + j] : 0.f;
-        const float x1 = h0 ? h0[sbase + (long long)(c0 + 16 + e) * D + j] : 0.f;
-        f[e] = __float_as_uint(x0);
-        f2[e] = __float_as_uint(x1);
+        f[e] = __float_as_uint(h0 ? h0[sbase + (long long)(c0 + e) * D + j] : 0.f);
+        f2[e] = __float_as_uint(h0 ? h0[sbase + (long long)(c0 + 16 + e) * D + j] : 0.f);
       }
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
@@ -168,7 +273,7 @@ kda_chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   __syncthreads();
 
   auto mma_wait = [&]() -> bool {
-    bool good = mbar_wait(&bar, phase, kWaitLimit);
+    const bool good = mbar_wait(&bar, phase, kWaitLimit);
     phase ^= 1u;
     tc_fence_after();
     return __syncthreads_or(!good) == 0;
@@ -176,130 +281,60 @@ kda_chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
 
   bool alive = true;
 #pragma unroll 1
-  for (long long t0 = t_beg; t0 < t_end && alive; t0 += C) {
+  for (long long t0 = t_beg; t0 < t_end; t0 += C) {
     const int L = (int)min((long long)C, t_end - t0);
+    const bool has_next = t0 + C < t_end;
+    const int Ln = has_next ? (int)min((long long)C, t_end - t0 - C) : 0;
 
-    // ================= P0: load the chunk (zero rows >= L) ==================
-    {
-#pragma unroll
-      for (int it = 0; it < 4; ++it) {                      // q, k: 1024 chunks each
-        const int idx = tid + it * NT;
-        const int r = idx >> 4, ch = idx & 15;
-        uint4 qa = make_uint4(0, 0, 0, 0), ka = make_uint4(0, 0, 0, 0);
-        if (r < L) {
-          const long long e = ((row0 + t0 + r) * H + h) * D + ch * 8;
-          qa = __ldg(reinterpret_cast<const uint4*>(q + e));
-          ka = __ldg(reinterpret_cast<const uint4*>(k + e));
-        }
-        *reinterpret_cast<uint4*>(sm + OFF_SQ + r * 256 + ch * 16) = qa;
-        *reinterpret_cast<uint4*>(sm + OFF_SK + r * 256 + ch * 16) = ka;
-      }
-#pragma unroll
-      for (int it = 0; it < 8; ++it) {                      // g: 2048 chunks
-        const int idx = tid + it * NT;
-        const int r = idx >> 5, ch = idx & 31;
-        float4 ga = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (r < L) ga = __ldg(reinterpret_cast<const float4*>(g + ((row0 + t0 + r) * H + h) * D + ch * 4));
-        *reinterpret_cast<float4*>(sm + OFF_SG + r * 512 + ch * 16) = ga;
-      }
-#pragma unroll
-      for (int it = 0; it < 4; ++it) {                      // v -> MN-major SW128 (M = j, K = r)
-        const int idx = tid + it * NT;
-        const int r = idx >> 4, ch = idx & 15;
-        uint4 va = make_uint4(0, 0, 0, 0);
-        if (r < L) va = __ldg(reinterpret_cast<const uint4*>(v + ((row0 + t0 + r) * H + h) * D + ch * 8));
-        *reinterpret_cast<uint4*>(sm + OFF_V + chunk_mnmajor_sw128(ch, r, C)) = va;
-      }
-      if (tid < C) s_beta[tid] = tid < L ? beta[(row0 + t0 + tid) * H + h] : 0.f;
-    }
+    // ================= P0: this chunk's inputs have landed ====================
+    cp_async_wait_all();
+    if (tid < C) s_beta[tid] = beta_next;
+    fence_async_smem();
     __syncthreads();
 
-    // ================= P1: decay scan and operand build (channel threads) ====
-    if (!is_val) {
-      const int c = tid;
-      float* Gc = reinterpret_cast<float*>(sm + OFF_SG) + c;   // column c, row stride 128
-      float acc = 0.f;
-#pragma unroll 8
-      for (int r = 0; r < C; ++r) { acc += Gc[r * D]; Gc[r * D] = acc; }
-      const float P0 = Gc[0], P1 = Gc[16 * D], P2 = Gc[32 * D], P3 = Gc[48 * D], G63 = acc;
-      const float P[4] = {P0, P1, P2, P3};
-      s_gamma[c] = __expf(G63);
-      float eP[4], eE1[3];
+    // ================= P1: decay scan and operand build (all threads) ========
+    {
+      const int c = tid & 127, hf = tid >> 7;
+      const float* Gc = reinterpret_cast<const float*>(sm + OFF_SG) + c;   // column c
+      float gv[32];
 #pragma unroll
-      for (int a = 0; a < 4; ++a) eP[a] = __expf(P[a]);
-      eE1[0] = __expf(G63 - P1); eE1[1] = __expf(G63 - P2); eE1[2] = __expf(G63 - P3);
-      // f1[a'][b] = e^{P_a' - P_{b+1}} for a' > b  (a' = b + 1 gives 1)
-      const float f1_20 = __expf(P2 - P1), f1_30 = __expf(P3 - P1), f1_31 = __expf(P3 - P2);
-
+      for (int r = 0; r < 32; ++r) gv[r] = Gc[(32 * hf + r) * D];
+#pragma unroll
+      for (int r = 1; r < 32; ++r) gv[r] += gv[r - 1];
+      if (hf == 0) {
+        s_pref[0][c] = gv[0];
+        s_pref[1][c] = gv[16];
+        s_pref[4][c] = gv[31];                                  // G_31 for the upper half
+      }
+      __syncthreads();
+      if (hf == 1) {
+        const float off = s_pref[4][c];
+#pragma unroll
+        for (int r = 0; r < 32; ++r) gv[r] += off;
+        s_pref[2][c] = gv[0];
+        s_pref[3][c] = gv[16];
+        s_pref[4][c] = gv[31];                                  // G_63
+        s_gamma[c] = __expf(gv[31]);
+      }
+      __syncthreads();
+      const float P0 = s_pref[0][c], P1 = s_pref[1][c], P2 = s_pref[2][c], P3 = s_pref[3][c];
+      const float G63 = s_pref[4][c];
       const bf16* kc = reinterpret_cast<const bf16*>(sm + OFF_SK) + c;
       const bf16* qc = reinterpret_cast<const bf16*>(sm + OFF_SQ) + c;
-      uint32_t kb_words[32];
-#pragma unroll
-      for (int g8 = 0; g8 < 8; ++g8) {
-        const int a = g8 >> 1;
-        float lk[8], lq[8], ke[8], rd[8], ro1[8], ro2[8], ro3[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int r = g8 * 8 + e;
-          const float Gr = Gc[r * D];
-          const float x = Gr - P[a];
-          const float ell = __expf(x);
-          const float rho = __expf(fminf(-x, 80.f));
-          const float sig = a < 3 ? __expf(P[a < 3 ? a + 1 : 3] - Gr) : __expf(G63 - Gr);
-          const float kv = __bfloat162float(kc[r * D]);
-          const float qv = __bfloat162float(qc[r * D]);
-          lk[e] = kv * ell;
-          lq[e] = qv * ell;
-          ke[e] = a < 3 ? kv * sig * eE1[a < 3 ? a : 0] : kv * sig;
-          rd[e] = kv * rho;
-          const float ks = kv * sig;
-          ro1[e] = ks;                                  // R^(a+1): factor 1
-          ro2[e] = ks * (a == 0 ? f1_20 : f1_31);       // R^(a+2)
-          ro3[e] = ks * f1_30;                          // R^(a+3) (a == 0 only)
-        }
-        // L = [Lk ; Lq]: A operand, MN-major SW128, M = 128, K = 128 rows (channels)
-        st_shared_v4(sm, OFF_L + chunk_mnmajor_sw128(g8, c, D), pack_bf16(lk[0], lk[1]),
-                     pack_bf16(lk[2], lk[3]), pack_bf16(lk[4], lk[5]), pack_bf16(lk[6], lk[7]));
-        st_shared_v4(sm, OFF_L + chunk_mnmajor_sw128(8 + g8, c, D), pack_bf16(lq[0], lq[1]),
-                     pack_bf16(lq[2], lq[3]), pack_bf16(lq[4], lq[5]), pack_bf16(lq[6], lq[7]));
-        // Qbar^T: B operand, MN-major SW128, N = 64 (tokens), K = 128 (channels)
-        const float ea = eP[a];
-        st_shared_v4(sm, OFF_QB + chunk_mnmajor_sw128(g8, c, D), pack_bf16(lq[0] * ea, lq[1] * ea),
-                     pack_bf16(lq[2] * ea, lq[3] * ea), pack_bf16(lq[4] * ea, lq[5] * ea),
-                     pack_bf16(lq[6] * ea, lq[7] * ea));
-        // Kbar^T: A operand in TMEM (lane c, 2 tokens per column)
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          kb_words[g8 * 4 + e] = pack_bf16(lk[2 * e] * ea, lk[2 * e + 1] * ea);
-        // Kend^T: B operand, K-major SW128, N = 128 (channels), K = 64 (tokens)
-        st_shared_v4(sm, OFF_KE + chunk_kmajor_sw128(c, g8, D), pack_bf16(ke[0], ke[1]),
-                     pack_bf16(ke[2], ke[3]), pack_bf16(ke[4], ke[5]), pack_bf16(ke[6], ke[7]));
-        // R^(a') for a' >= a: B operands, MN-major SW32, N = 16(a'+1), K = 128
-        st_shared_v4(sm, off_r(a) + chunk_mnmajor_sw32(g8, c, D), pack_bf16(rd[0], rd[1]),
-                     pack_bf16(rd[2], rd[3]), pack_bf16(rd[4], rd[5]), pack_bf16(rd[6], rd[7]));
-        if (a + 1 <= 3)
-          st_shared_v4(sm, off_r(a + 1) + chunk_mnmajor_sw32(g8, c, D),
-                       pack_bf16(ro1[0], ro1[1]), pack_bf16(ro1[2], ro1[3]),
-                       pack_bf16(ro1[4], ro1[5]), pack_bf16(ro1[6], ro1[7]));
-        if (a + 2 <= 3)
-          st_shared_v4(sm, off_r(a + 2) + chunk_mnmajor_sw32(g8, c, D),
-                       pack_bf16(ro2[0], ro2[1]), pack_bf16(ro2[2], ro2[3]),
-                       pack_bf16(ro2[4], ro2[5]), pack_bf16(ro2[6], ro2[7]));
-        if (a + 3 <= 3)
-          st_shared_v4(sm, off_r(3) + chunk_mnmajor_sw32(g8, c, D), pack_bf16(ro3[0], ro3[1]),
-                       pack_bf16(ro3[2], ro3[3]), pack_bf16(ro3[4], ro3[5]),
-                       pack_bf16(ro3[6], ro3[7]));
-      }
-      uint32_t w0[16], w1[16];
-#pragma unroll
-      for (int e = 0; e < 16; ++e) { w0[e] = kb_words[e]; w1[e] = kb_words[16 + e]; }
-      tmem_st16(tb + lane_base + TM_KB, w0);
-      tmem_st16(tb + lane_base + TM_KB + 16, w1);
+      if (hf == 0) build_half<0>(sm, gv, kc, qc, c, P0, P1, P2, P3, G63, tb + lane_base + TM_KB);
+      else build_half<1>(sm, gv, kc, qc, c, P0, P1, P2, P3, G63, tb + lane_base + TM_KB);
       tmem_wait_st();
       fence_async_smem();
     }
     tc_fence_before();
     __syncthreads();
+
+    // staging is free: fetch the next chunk's q, k, g (and beta) behind the MMAs
+    if (has_next) {
+      prefetch_qkg(sm, q, k, g, row0 + t0 + C, Ln, H, h, tid);
+      cp_async_commit();
+      if (tid < C) beta_next = tid < Ln ? beta[(row0 + t0 + C + tid) * H + h] : 0.f;
+    }
 
     // ================= P2: Gram MMAs ==========================================
     if (tid == 0) {
@@ -321,67 +356,64 @@ kda_chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     __syncwarp();
     if (!mma_wait()) { alive = false; break; }
 
-    // ================= P3: read A / Aqk, triangular inverse ===================
-    float* A32 = reinterpret_cast<float*>(sm + OFF_A32);
+    // ================= P3: read A / Aqk ======================================
+    float* B32 = reinterpret_cast<float*>(sm + OFF_B32);
     float* T32 = reinterpret_cast<float*>(sm + OFF_T32);
-    float* Y32 = reinterpret_cast<float*>(sm + OFF_Y);
-    if (!is_val) {
-      // warp w reads TMEM lanes 32w..32w+31: w=0,1 -> A rows, w=2,3 -> Aqk rows
-      const int r = (warp & 1) * 32 + lane;
-      const bool isA = warp < 2;
-      const int a_lo = (warp & 1) * 2;            // blocks a_lo, a_lo + 1 in this warp
-      const int colA = a_lo == 0 ? 0 : 48;        // D^(a_lo) column offset in the Gram
-      const int colB = a_lo == 0 ? 16 : 96;       // D^(a_lo+1)
-      const int nA = 16 * (a_lo + 1), nB = 16 * (a_lo + 2);
-      const int a_me = r >> 4;
+    float* M32 = reinterpret_cast<float*>(sm + OFF_M32);
+    {
+      // warp w (mod 4) reads TMEM lanes 32w..32w+31: w%4 = 0,1 -> A rows, 2,3 -> Aqk rows.
+      // Rows of a warp lie in blocks a0, a0+1; the lower warpgroup handles block a0
+      // and the upper warpgroup block a0+1.
+      const int w4 = warp & 3;
+      const int r = (w4 & 1) * 32 + lane;
+      const bool isA = w4 < 2;
+      const int a0 = (w4 & 1) * 2;
+      const int ab = a0 + (upper ? 1 : 0);            // block handled by this thread
+      const int colb = ab == 0 ? 0 : ab == 1 ? 16 : ab == 2 ? 48 : 96;
+      const int nb = 16 * (ab + 1);
+      const bool mine = (r >> 4) == ab;
       float vals[64];
 #pragma unroll
       for (int i = 0; i < 64; ++i) vals[i] = 0.f;
-      // first block of the pair
-#pragma unroll
-      for (int i0 = 0; i0 < 48; i0 += 16) {
-        if (i0 < nA) {
-          uint32_t t[16];
-          tmem_ld16(tb + lane_base + TM_G + colA + i0, t);
-          tmem_wait_ld();
-          if (a_me == a_lo) {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) vals[i0 + e] = __uint_as_float(t[e]);
-          }
-        }
-      }
 #pragma unroll
       for (int i0 = 0; i0 < 64; i0 += 16) {
-        if (i0 < nB) {
+        if (i0 < nb) {
           uint32_t t[16];
-          tmem_ld16(tb + lane_base + TM_G + colB + i0, t);
+          tmem_ld16(tb + lane_base + TM_G + colb + i0, t);
           tmem_wait_ld();
-          if (a_me == a_lo + 1) {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) vals[i0 + e] = __uint_as_float(t[e]);
-          }
+          for (int e = 0; e < 16; ++e) vals[i0 + e] = __uint_as_float(t[e]);
         }
       }
-      if (isA) {
+      if (mine) {
+        if (isA) {
+          const float br = s_beta[r];
 #pragma unroll
-        for (int i = 0; i < 64; ++i) A32[r * LDA + i] = (i < r) ? vals[i] : 0.f;
-      } else {
-        // Aqk: B operand of O^T += Delta^T Aqk^T, K-major SW128, N = 64 (r), K = 64 (i)
+          for (int i4 = 0; i4 < 16; ++i4) {
+            float4 w;
+            w.x = (4 * i4 + 0 < r) ? br * vals[4 * i4 + 0] : 0.f;
+            w.y = (4 * i4 + 1 < r) ? br * vals[4 * i4 + 1] : 0.f;
+            w.z = (4 * i4 + 2 < r) ? br * vals[4 * i4 + 2] : 0.f;
+            w.w = (4 * i4 + 3 < r) ? br * vals[4 * i4 + 3] : 0.f;
+            *reinterpret_cast<float4*>(B32 + r * LDA + 4 * i4) = w;
+          }
+        } else {
+          // Aqk: B operand of O^T += Delta^T Aqk^T, K-major SW128, N = 64 (r), K = 64 (i)
 #pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
-          float w[8];
+          for (int c8 = 0; c8 < 8; ++c8) {
+            float w[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) w[e] = (c8 * 8 + e <= r) ? vals[c8 * 8 + e] : 0.f;
-          st_shared_v4(sm, OFF_AQK + chunk_kmajor_sw128(r, c8, C), pack_bf16(w[0], w[1]),
-                       pack_bf16(w[2], w[3]), pack_bf16(w[4], w[5]), pack_bf16(w[6], w[7]));
+            for (int e = 0; e < 8; ++e) w[e] = (c8 * 8 + e <= r) ? vals[c8 * 8 + e] : 0.f;
+            st_v4f(sm, OFF_AQK + chunk_kmajor_sw128(r, c8, C), w, 1.f);
+          }
         }
       }
     }
     tc_fence_before();
     __syncthreads();
 
-    // diagonal 16 x 16 blocks of T = (I + diag(beta) A)^-1 by forward substitution
-    if (tid < 64) {
+    // ================= triangular inverse T = (I + B)^-1, B = diag(beta) A ====
+    if (tid < 64) {                         // diagonal blocks: forward substitution
       const int a = tid >> 4, jj = tid & 15, o = 16 * a;
       float x[16];
 #pragma unroll
@@ -390,39 +422,66 @@ kda_chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       for (int i = 1; i < 16; ++i) {
         float acc = 0.f;
 #pragma unroll
-        for (int m = 0; m < i; ++m) acc = fmaf(A32[(o + i) * LDA + o + m], x[m], acc);
-        if (i > jj) x[i] = -s_beta[o + i] * acc;
+        for (int m = 0; m < i; ++m) acc = fmaf(B32[(o + i) * LDA + o + m], x[m], acc);
+        if (i > jj) x[i] = -acc;
       }
 #pragma unroll
       for (int i = 0; i < 16; ++i) T32[(o + i) * LDA + o + jj] = x[i];
     }
     __syncthreads();
-    // off-diagonal blocks, by distance d from the diagonal
-#pragma unroll 1
-    for (int d = 1; d < 4; ++d) {
-      const int nblk = 4 - d;
-      for (int idx = tid; idx < nblk * 256; idx += NT) {
-        const int bi = idx >> 8, i = (idx >> 4) & 15, jj = idx & 15;
-        const int a = bi + d, b = bi;
-        const int row = 16 * a + i;
-        float acc = 0.f;
-        for (int m = 16 * b; m < 16 * a; ++m) acc = fmaf(A32[row * LDA + m], T32[m * LDA + 16 * b + jj], acc);
-        Y32[idx] = s_beta[row] * acc;
-      }
-      __syncthreads();
-      for (int idx = tid; idx < nblk * 256; idx += NT) {
-        const int bi = idx >> 8, i = (idx >> 4) & 15, jj = idx & 15;
-        const int a = bi + d, b = bi;
-        float acc = 0.f;
+    if (tid < 192) {                        // M_am = T_aa B_am for the 6 pairs a > m
+      const int a = 1 + (tid >> 6), i = (tid >> 2) & 15, jq = tid & 3;
+      float trow[16];
 #pragma unroll
-        for (int mm = 0; mm < 16; ++mm)
-          acc = fmaf(T32[(16 * a + i) * LDA + 16 * a + mm], Y32[(bi << 8) + (mm << 4) + jj], acc);
-        T32[(16 * a + i) * LDA + 16 * b + jj] = -acc;
+      for (int l4 = 0; l4 < 4; ++l4) {
+        const float4 t4 = *reinterpret_cast<const float4*>(T32 + (16 * a + i) * LDA + 16 * a + 4 * l4);
+        trow[4 * l4] = t4.x; trow[4 * l4 + 1] = t4.y; trow[4 * l4 + 2] = t4.z; trow[4 * l4 + 3] = t4.w;
+      }
+#pragma unroll
+      for (int m = 0; m < 3; ++m) {
+        if (m < a) {
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int l = 0; l < 16; ++l) {
+            const float4 b4 = *reinterpret_cast<const float4*>(B32 + (16 * a + l) * LDA + 16 * m + 4 * jq);
+            acc.x = fmaf(trow[l], b4.x, acc.x); acc.y = fmaf(trow[l], b4.y, acc.y);
+            acc.z = fmaf(trow[l], b4.z, acc.z); acc.w = fmaf(trow[l], b4.w, acc.w);
+          }
+          *reinterpret_cast<float4*>(M32 + (a * (a - 1) / 2 + m) * 256 + i * 16 + 4 * jq) = acc;
+        }
+      }
+    }
+    __syncthreads();
+    // block rows a = 1, 2, 3: T_ab = -sum_{m=b}^{a-1} M_am T_mb
+#pragma unroll 1
+    for (int a = 1; a < 4; ++a) {
+      if (tid < 64 * a) {
+        const int i = tid / (4 * a), q4 = tid % (4 * a);
+        const int b = q4 >> 2, jq = q4 & 3;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int m = b; m < a; ++m) {
+          const float* Mrow = M32 + (a * (a - 1) / 2 + m) * 256 + i * 16;
+#pragma unroll
+          for (int l4 = 0; l4 < 4; ++l4) {
+            const float4 m4 = *reinterpret_cast<const float4*>(Mrow + 4 * l4);
+            const float mv[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float4 t4 = *reinterpret_cast<const float4*>(T32 + (16 * m + 4 * l4 + e) * LDA + 16 * b + 4 * jq);
+              acc.x = fmaf(mv[e], t4.x, acc.x); acc.y = fmaf(mv[e], t4.y, acc.y);
+              acc.z = fmaf(mv[e], t4.z, acc.z); acc.w = fmaf(mv[e], t4.w, acc.w);
+            }
+          }
+        }
+        *reinterpret_cast<float4*>(T32 + (16 * a + i) * LDA + 16 * b + 4 * jq) =
+            make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
       }
       __syncthreads();
     }
     // T diag(beta) as bf16: B operand of W^T / U^T, K-major SW128, N = 64 (r'), K = 64 (r)
-    for (int idx = tid; idx < C * 8; idx += NT) {
+#pragma unroll
+    for (int it = 0; it < 2; ++it) {
+      const int idx = tid + it * NT;
       const int rp = idx >> 3, c8 = idx & 7;
       float w[8];
 #pragma unroll
@@ -430,8 +489,7 @@ kda_chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
         const int r = c8 * 8 + e;
         w[e] = (r <= rp) ? T32[rp * LDA + r] * s_beta[r] : 0.f;
       }
-      st_shared_v4(sm, OFF_TB + chunk_kmajor_sw128(rp, c8, C), pack_bf16(w[0], w[1]),
-                   pack_bf16(w[2], w[3]), pack_bf16(w[4], w[5]), pack_bf16(w[6], w[7]));
+      st_v4f(sm, OFF_TB + chunk_kmajor_sw128(rp, c8, C), w, 1.f);
     }
     fence_async_smem();
     tc_fence_before();
@@ -459,9 +517,14 @@ kda_chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     }
     __syncwarp();
     if (!mma_wait()) { alive = false; break; }
+    // V has been consumed: fetch the next chunk's v
+    if (has_next) {
+      prefetch_v(sm, v, row0 + t0 + C, Ln, H, h, tid);
+      cp_async_commit();
+    }
 
     // ================= P5: W^T -> bf16 smem; S^T <- S^T Diag(gamma) ===========
-    if (!is_val) {
+    if (!upper) {
       const int c = tid;
 #pragma unroll
       for (int r0 = 0; r0 < C; r0 += 16) {
@@ -471,14 +534,13 @@ kda_chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
 #pragma unroll
         for (int h8 = 0; h8 < 2; ++h8) {
           const float* f = reinterpret_cast<const float*>(t) + 8 * h8;
-          st_shared_v4(sm, OFF_WT + chunk_mnmajor_sw128((r0 >> 3) + h8, c, D),
-                       pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
-                       pack_bf16(f[6], f[7]));
+          st_v4(sm, OFF_WT + chunk_mnmajor_sw128((r0 >> 3) + h8, c, D), pack_bf16(f[0], f[1]),
+                pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]), pack_bf16(f[6], f[7]));
         }
       }
       fence_async_smem();
     } else {
-#pragma unroll 1
+#pragma unroll 2
       for (int c0 = 0; c0 < D; c0 += 16) {
         uint32_t t[16];
         tmem_ld16(tb + lane_base + TM_S + c0, t);
@@ -505,8 +567,8 @@ kda_chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     __syncwarp();
     if (!mma_wait()) { alive = false; break; }
 
-    // ================= P7: Delta^T = U^T - P -> bf16 TMEM (value threads) =====
-    if (is_val) {
+    // ================= P7: Delta^T = U^T - P -> bf16 TMEM (upper threads) =====
+    if (upper) {
       uint32_t dw[32];
 #pragma unroll
       for (int r0 = 0; r0 < C; r0 += 16) {
@@ -547,18 +609,16 @@ kda_chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     if (!mma_wait()) { alive = false; break; }
 
     // ================= P9: outputs; bf16 copy of the new state =================
-    if (is_val) {
+    if (upper) {
       const int j = tid - 128;
+      bf16* otile = reinterpret_cast<bf16*>(sm + OFF_OUT);      // [64 tokens][128] row-major
 #pragma unroll
       for (int r0 = 0; r0 < C; r0 += 16) {
         uint32_t t[16];
         tmem_ld16(tb + lane_base + TM_O + r0, t);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int r = r0 + e;
-          if (r < L) out[((row0 + t0 + r) * H + h) * D + j] = __float2bfloat16_rn(__uint_as_float(t[e]));
-        }
+        for (int e = 0; e < 16; ++e) otile[(r0 + e) * D + j] = __float2bfloat16_rn(__uint_as_float(t[e]));
       }
 #pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 32) {
@@ -574,13 +634,24 @@ kda_chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
         tmem_st16(tb + lane_base + TM_SB + c0 / 2, pk);
       }
       tmem_wait_st();
+      named_bar(1, 128);
+      // coalesced 16-byte stores of the output tile (16 threads per 256-byte row)
+#pragma unroll
+      for (int it = 0; it < 8; ++it) {
+        const int idx = j + it * 128;
+        const int r = idx >> 4, ch = idx & 15;
+        if (r < L) {
+          const uint4 val = *reinterpret_cast<const uint4*>(sm + OFF_OUT + r * 256 + ch * 16);
+          *reinterpret_cast<uint4*>(out + ((row0 + t0 + r) * H + h) * D + ch * 8) = val;
+        }
+      }
     }
     tc_fence_before();
     __syncthreads();
   }
 
   // ---- final state
-  if (alive && is_val && hT) {
+  if (alive && upper && hT) {
     const int j = tid - 128;
 #pragma unroll 1
     for (int c0 = 0; c0 < D; c0 += 16) {
@@ -591,6 +662,7 @@ kda_chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       for (int e = 0; e < 16; ++e) hT[sbase + (long long)(c0 + e) * D + j] = __uint_as_float(t[e]);
     }
   }
+  cp_async_wait_all();
   if (!alive && tid == 0) {
     atomicExch(&g_chunk_tc_timeout, 1);
     // let any MMA still in flight finish before the TMEM is released
