@@ -74,8 +74,11 @@ typedef enum {
  *     cu_seqlens: DEVICE int32 [B + 1], cu_seqlens[0] = 0, non-decreasing,
  *     cu_seqlens[B] = T.  Documents may be empty.  Document d is tokens
  *     [cu_seqlens[d], cu_seqlens[d+1]) and starts from h0[d] (or zero); no state
- *     crosses a boundary, and chunks restart at every document start, so a
- *     document's result does not depend on its neighbours.  The contents of
+ *     crosses a boundary and chunks restart at every document start.  A
+ *     document run in one piece gives bit-identical results packed or alone;
+ *     when few (document, head) pairs leave SMs idle, long documents are split
+ *     into segments whose states are chained afterwards, and then packed and
+ *     separate results may differ in rounding order only.  The contents of
  *     cu_seqlens are device memory and are NOT checked on the host; malformed
  *     offsets give undefined results for the affected documents, but every
  *     access stays inside [0, T) (offsets are clamped on the device).
@@ -83,6 +86,12 @@ typedef enum {
  * h0: initial state, or NULL for zeros.   hT: final state out, or NULL to skip.
  * out must not alias any input.  hT may alias h0 (in-place state update).
  * B >= 1, T >= 0, H >= 1.  T == 0 writes hT = h0 (or zeros) and nothing else.
+ *
+ * Scratch: when a call splits sequences into segments (dk = dv = 128, bf16,
+ * few (sequence, head) pairs) it takes 2 * 64 KB per segment and head from a
+ * library-owned, stream-ordered memory pool of the current device; the pool
+ * keeps its memory for later calls.  If that allocation fails the call runs
+ * unsplit instead.
  *
  * Precision: g, beta and the state are fp32.  With KDA_BF16 inputs the chunk
  * contractions run on the tensor cores with bf16 operands and fp32

@@ -42,6 +42,7 @@ CASES = [
     (1, 0, 64, 64),                                                       # U^T = V^T (T beta)^T
     (2, 1, 64, 128),                                                      # P = S^T W^T, O^T = S^T Qbar^T
     (2, 0, 128, 64),                                                      # S^T += Delta^T Kend
+    (0, 1, 128, 128),                                                     # segment combine: X S
     (0, 0, 128, 128), (0, 1, 64, 128), (2, 2, 32, 64),                    # other combinations
 ]
 
