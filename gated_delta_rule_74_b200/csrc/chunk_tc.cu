@@ -1073,4 +1073,53 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const f
   return e;
 }
 
+// Same plan as launch_chunk_tc, run on caller-provided scratch: no pool, no
+// allocation of any kind.  Returns a kda_status_t: KDA_ERR_INVALID_ARG when the
+// split this call would use needs more than `capacity` bytes of scratch.
+int run_chunk_tc_static(const void* q, const void* k, const void* v, const float* g,
+                        const float* beta, const float* h0, const int32_t* cu_seqlens, void* out,
+                        float* hT, int B, int T, int H, cudaStream_t stream, float* scratch,
+                        size_t capacity) {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaFuncSetAttribute(kda_chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           SMEM_BYTES) != cudaSuccess ||
+      cudaFuncSetAttribute(kda_seg_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kCombineSmem) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return KDA_ERR_CUDA;
+  }
+  const bf16* qb = static_cast<const bf16*>(q);
+  const bf16* kb = static_cast<const bf16*>(k);
+  const bf16* vb = static_cast<const bf16*>(v);
+  bf16* ob = static_cast<bf16*>(out);
+  SegArgs sa{0, 1, 0, 0, nullptr, nullptr};
+  const int G = plan_segments(B, T, H, cu_seqlens != nullptr, sms);
+  const long long nch = ((long long)T + C - 1) / C;
+  if (G > 0 && (nch + G - 1) / G >= 2) {
+    const int P = (int)((nch + G - 1) / G);
+    const long long slots = cu_seqlens ? (long long)P + B : (long long)B * P;
+    const size_t bytes = (size_t)2 * slots * H * D * D * sizeof(float);
+    if (bytes > capacity || scratch == nullptr) return KDA_ERR_INVALID_ARG;
+    sa = SegArgs{G, P, 1, (int)slots, scratch, scratch + (size_t)slots * H * D * D};
+  }
+  if (sa.pass == 0) {
+    kda_chunk_tc_kernel<<<dim3(H, B, 1), NT, SMEM_BYTES, stream>>>(qb, kb, vb, g, beta, h0,
+                                                                  cu_seqlens, ob, hT, T, H, sa);
+    note_launches(1);
+  } else {
+    kda_chunk_tc_kernel<<<dim3(H, B, 2 * sa.P), NT, SMEM_BYTES, stream>>>(
+        qb, kb, vb, g, beta, h0, cu_seqlens, ob, hT, T, H, sa);
+    kda_seg_combine_kernel<<<dim3(H, B), kCombineThreads, kCombineSmem, stream>>>(cu_seqlens,
+                                                                                  T, H, sa);
+    sa.pass = 2;
+    kda_chunk_tc_kernel<<<dim3(H, B, sa.P - 1), NT, SMEM_BYTES, stream>>>(
+        qb, kb, vb, g, beta, h0, cu_seqlens, ob, hT, T, H, sa);
+    note_launches(3);
+  }
+  if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
+  return KDA_OK;
+}
+
 }  // namespace kda

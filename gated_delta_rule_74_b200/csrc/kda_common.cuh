@@ -38,4 +38,10 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const f
                             const float* beta, const float* h0, const int32_t* cu_seqlens,
                             void* out, float* hT, int B, int T, int H, cudaStream_t stream);
 
+// The tensor-core prefill on caller-provided scratch (allocates nothing).
+int run_chunk_tc_static(const void* q, const void* k, const void* v, const float* g,
+                        const float* beta, const float* h0, const int32_t* cu_seqlens, void* out,
+                        float* hT, int B, int T, int H, cudaStream_t stream, float* scratch,
+                        size_t capacity);
+
 }  // namespace kda

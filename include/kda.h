@@ -122,6 +122,38 @@ KDA_API int kda_decode_step(const void* q, const void* k, const void* v,
                     const float* g, const float* beta, float* S, void* out,
                     int N, int H, int dk, int dv, int in_dtype, void* stream);
 
+/*
+ * kda_chunk_fwd_noalloc -- kda_chunk_fwd for callers that cannot allocate.
+ *
+ * The pages have no counterpart: this is a deployment variant.  Some callers
+ * cannot call cudaMalloc or any allocator: code that runs inside a CUDA graph
+ * being captured or replayed under a fixed memory budget, embedders that hand
+ * the library only pre-sized buffers, or processes whose allocator is owned by
+ * another runtime.  kda_chunk_fwd may take segment scratch from a library pool
+ * (see its Scratch note); this entry point instead uses a fixed array of
+ * KDA_NOALLOC_SCRATCH_BYTES that lives in the library's device image, so it
+ * never allocates, frees or calls an allocating routine.
+ *
+ * Arguments, layouts, results and error codes are those of kda_chunk_fwd, plus:
+ *   - KDA_ERR_INVALID_ARG (nothing launched) when the segment split this call
+ *     would use needs more than KDA_NOALLOC_SCRATCH_BYTES of scratch:
+ *     2 * 64 KB * H * (number of segment slots); a B=1, T=8192, H=12, d=128
+ *     bf16 call needs 19.5 MiB.
+ *   - Every GPU that loads the library holds the array (KDA_NOALLOC_SCRATCH_BYTES)
+ *     until the process exits.
+ *   - The first call on a device looks up the array's device address (one
+ *     cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the one array: calls that overlap on the GPU
+ *     (different streams without ordering) race on it.  Serialize them.
+ */
+#define KDA_NOALLOC_SCRATCH_BYTES (32u << 20)
+KDA_API int kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
+                                  const float* g, const float* beta, const float* h0,
+                                  const int32_t* cu_seqlens, void* out, float* hT,
+                                  int B, int T, int H, int dk, int dv,
+                                  int in_dtype, void* stream);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 KDA_API const char* kda_status_string(int status);
 
