@@ -30,12 +30,15 @@
 //
 // Everything is computed transposed so that every MMA has M = 128 (the channel
 // or value index on the TMEM lanes):
-//   Gram   D^(a) [128 x 16(a+1)] = [Lk ; Lq] R^(a)^T       rows 0-63: A, 64-127: Aqk
+//   Gram   [D^(0) .. D^(3)] [128 x 160] = [Lk ; Lq] [R^(0); ..; R^(3)]^T
+//          (rows 0-63: A, rows 64-127: Aqk; row block a is read from D^(a))
 //   W^T    [dk x 64] = Kbar^T (T beta)^T                    A operand in TMEM
 //   U^T    [dv x 64] = V^T (T beta)^T
-//   O^T    [dv x 64] = S^T Qbar^T + Delta^T Aqk^T           S^T, Delta^T in TMEM
-//   P      [dv x 64] = S^T W^T          Delta^T = U^T - P
-//   S^T   += Delta^T Kend   (after S^T <- S^T Diag(exp(G_63)))
+//   [O^T | P]   [dv x 128] = S^T [Qbar^T | W^T]^T            S^T (bf16 copy) in TMEM
+//   Delta^T = U^T - P
+//   [S^T | O^T] [dv x 192] += Delta^T [Kend^T ; Aqk]^T      (after S^T <- S^T Diag(exp(G_63)))
+// Products that share an operand are merged into one wide MMA: each tcgen05.mma
+// costs about the same whatever its N, so fewer, wider instructions are faster.
 // The state S^T [dv x dk] stays in TMEM in fp32 for the whole sequence; a bf16
 // copy is the MMA operand.  The 64 x 64 triangular inverse runs on the CUDA
 // cores in fp32: 16 x 16 diagonal blocks by forward substitution, then
@@ -80,22 +83,28 @@ constexpr int LDA = 68;                                 // fp32 row stride (16-b
 constexpr uint32_t OFF_B32 = 65536;                     // diag(beta) A, fp32
 constexpr uint32_t OFF_T32 = 65536 + 17408;             // T, fp32
 constexpr uint32_t OFF_M32 = 65536 + 34816;             // T_aa B_am, 6 x 16 x 16 fp32
-constexpr uint32_t OFF_AQK = 106496, OFF_TB = 114688, OFF_WT = 122880;
+constexpr uint32_t OFF_TB = 114688;                      // T diag(beta), bf16 K-major
 constexpr uint32_t OFF_OUT = 65536;                     // output tile (after the solve)
 // region C [136K, 184K)
-constexpr uint32_t OFF_V = 139264, OFF_QB = 155648, OFF_KE = 172032;
-constexpr uint32_t SMEM_USED = 188416;
+// region C [136K, 208K): V; then [Qbar^T | W^T] as one MN-major B operand of
+// N = 128 (two 64-wide blocks, 16 KB apart); then [Kend^T ; Aqk] as one K-major B
+// operand of 192 rows (Kend^T rows 0-127, Aqk rows 128-191)
+constexpr uint32_t OFF_V = 139264, OFF_QB = 155648, OFF_WT = OFF_QB + 16384;
+constexpr uint32_t OFF_KE = 188416, OFF_AQK = OFF_KE + 16384;
+constexpr uint32_t SMEM_USED = 212992;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
 
 // ---- TMEM columns (512 allocated)
+// [S^T | O^T] and [O^T | P] are each the accumulator of one MMA, so O^T sits
+// between S^T and P.
 constexpr uint32_t TM_S = 0;        // S^T fp32        [128 lanes x 128]
-constexpr uint32_t TM_SB = 128;     // S^T bf16 (A)    [128 x 64]
-constexpr uint32_t TM_KB = 192;     // Kbar^T bf16 (A) [128 x 32], later Delta^T bf16 (A)
-constexpr uint32_t TM_G = 224;      // Gram D^(0..3) at +0, +16, +48, +96 (160 columns)
-constexpr uint32_t TM_P = 224;      // P  [128 x 64] (after the Gram is read)
-constexpr uint32_t TM_O = 288;      // O^T [128 x 64]
-constexpr uint32_t TM_W = 384;      // W^T [128 x 64]
-constexpr uint32_t TM_U = 448;      // U^T [128 x 64]
+constexpr uint32_t TM_O = 128;      // O^T             [128 x 64]
+constexpr uint32_t TM_P = 192;      // P               [128 x 64]
+constexpr uint32_t TM_SB = 256;     // S^T bf16 (A)    [128 x 64]
+constexpr uint32_t TM_KB = 320;     // Kbar^T bf16 (A) [128 x 32], later Delta^T bf16 (A)
+constexpr uint32_t TM_G = 352;      // Gram D^(0..3) at +0, +16, +48, +96 (160 columns)
+constexpr uint32_t TM_W = 352;      // W^T [128 x 64]  (after the Gram is read)
+constexpr uint32_t TM_U = 416;      // U^T [128 x 64]
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kWaitLimit = 1u << 22;
 
@@ -431,33 +440,35 @@ kda_chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
 
     // ================= P2: Gram MMAs ==========================================
     if (tid == 0) {
+      // the four R^(a) buffers are consecutive 16-token blocks of one MN-major B
+      // operand of N = 160, so the four Gram products are one MMA per K step
       tc_fence_after();
       const uint32_t l_base = smem_u32(sm + OFF_L);
-      uint32_t col = TM_G;
+      const uint32_t r_base = smem_u32(sm + off_r(0));
+      const uint32_t idesc = idesc_bf16(128, 160, true, true);
 #pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        const uint32_t idesc = idesc_bf16(128, 16 * (a + 1), true, true);
-        const uint32_t r_base = smem_u32(sm + off_r(a));
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tb + col, desc_mnmajor_sw128(l_base, D, kk), desc_mnmajor_sw32(r_base, D, kk),
-                 idesc, kk > 0);
-        col += 16 * (a + 1);
-      }
+      for (int kk = 0; kk < D / 16; ++kk)
+        mma_ss(tb + TM_G, desc_mnmajor_sw128(l_base, D, kk), desc_mnmajor_sw32(r_base, D, kk),
+               idesc, kk > 0);
       mma_commit(&bar);
     }
     __syncwarp();
     // while the Gram runs: S^T <- S^T Diag(exp(G_63)) (upper threads, own TMEM rows;
     // the MMAs read only the bf16 copy of the state until the update in P8)
     if (upper) {
-#pragma unroll 2
-      for (int c0 = 0; c0 < D; c0 += 16) {
-        uint32_t t[16];
-        tmem_ld16(tb + lane_base + TM_S + c0, t);
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 64) {
+        uint32_t t[4][16];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) tmem_ld16(tb + lane_base + TM_S + c0 + 16 * q4, t[q4]);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 16; ++e) t[e] = __float_as_uint(__uint_as_float(t[e]) * s_gamma[c0 + e]);
-        tmem_st16(tb + lane_base + TM_S + c0, t);
+        for (int q4 = 0; q4 < 4; ++q4) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            t[q4][e] = __float_as_uint(__uint_as_float(t[q4][e]) * s_gamma[c0 + 16 * q4 + e]);
+          tmem_st16(tb + lane_base + TM_S + c0 + 16 * q4, t[q4]);
+        }
       }
       tmem_wait_st();
       tc_fence_before();
@@ -480,19 +491,19 @@ kda_chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       const int colb = ab == 0 ? 0 : ab == 1 ? 16 : ab == 2 ? 48 : 96;
       const int nb = 16 * (ab + 1);
       const bool mine = (r >> 4) == ab;
-      float vals[64];
+      uint32_t tv[4][16];
 #pragma unroll
-      for (int i = 0; i < 64; ++i) vals[i] = 0.f;
+      for (int q4 = 0; q4 < 4; ++q4) {
+        if (16 * q4 < nb) tmem_ld16(tb + lane_base + TM_G + colb + 16 * q4, tv[q4]);
+        else {
 #pragma unroll
-      for (int i0 = 0; i0 < 64; i0 += 16) {
-        if (i0 < nb) {
-          uint32_t t[16];
-          tmem_ld16(tb + lane_base + TM_G + colb + i0, t);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 16; ++e) vals[i0 + e] = __uint_as_float(t[e]);
+          for (int e = 0; e < 16; ++e) tv[q4][e] = 0u;
         }
       }
+      tmem_wait_ld();
+      float vals[64];
+#pragma unroll
+      for (int i = 0; i < 64; ++i) vals[i] = __uint_as_float(tv[i >> 4][i & 15]);
       if (mine) {
         if (isA) {
           const float br = s_beta[r];
@@ -537,55 +548,84 @@ kda_chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       for (int i = 0; i < 16; ++i) T32[(o + i) * LDA + o + jj] = x[i];
     }
     __syncthreads();
-    if (tid < 192) {                        // M_am = T_aa B_am for the 6 pairs a > m
-      const int a = 1 + (tid >> 6), i = (tid >> 2) & 15, jq = tid & 3;
-      float trow[16];
+    // M_am = T_aa B_am for the 6 pairs a > m (p = a(a-1)/2 + m); 384 items of
+    // 4 outputs, two accumulator chains each
+#pragma unroll 1
+    for (int w = tid; w < 384; w += NT) {
+      const int p = w >> 6, i = (w >> 2) & 15, jq = w & 3;
+      const int a = p == 0 ? 1 : (p < 3 ? 2 : 3);
+      const int m = p - a * (a - 1) / 2;
+      const float* Ti = T32 + (16 * a + i) * LDA + 16 * a;
+      const float* Bc = B32 + 16 * a * LDA + 16 * m + 4 * jq;
+      float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;
 #pragma unroll
-      for (int l4 = 0; l4 < 4; ++l4) {
-        const float4 t4 = *reinterpret_cast<const float4*>(T32 + (16 * a + i) * LDA + 16 * a + 4 * l4);
-        trow[4 * l4] = t4.x; trow[4 * l4 + 1] = t4.y; trow[4 * l4 + 2] = t4.z; trow[4 * l4 + 3] = t4.w;
+      for (int l = 0; l < 16; l += 2) {
+        const float4 b0 = *reinterpret_cast<const float4*>(Bc + l * LDA);
+        const float4 b1 = *reinterpret_cast<const float4*>(Bc + (l + 1) * LDA);
+        const float t0v = Ti[l], t1v = Ti[l + 1];
+        s0.x = fmaf(t0v, b0.x, s0.x); s0.y = fmaf(t0v, b0.y, s0.y);
+        s0.z = fmaf(t0v, b0.z, s0.z); s0.w = fmaf(t0v, b0.w, s0.w);
+        s1.x = fmaf(t1v, b1.x, s1.x); s1.y = fmaf(t1v, b1.y, s1.y);
+        s1.z = fmaf(t1v, b1.z, s1.z); s1.w = fmaf(t1v, b1.w, s1.w);
       }
-#pragma unroll
-      for (int m = 0; m < 3; ++m) {
-        if (m < a) {
-          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-          for (int l = 0; l < 16; ++l) {
-            const float4 b4 = *reinterpret_cast<const float4*>(B32 + (16 * a + l) * LDA + 16 * m + 4 * jq);
-            acc.x = fmaf(trow[l], b4.x, acc.x); acc.y = fmaf(trow[l], b4.y, acc.y);
-            acc.z = fmaf(trow[l], b4.z, acc.z); acc.w = fmaf(trow[l], b4.w, acc.w);
-          }
-          *reinterpret_cast<float4*>(M32 + (a * (a - 1) / 2 + m) * 256 + i * 16 + 4 * jq) = acc;
-        }
-      }
+      *reinterpret_cast<float4*>(M32 + p * 256 + i * 16 + 4 * jq) =
+          make_float4(s0.x + s1.x, s0.y + s1.y, s0.z + s1.z, s0.w + s1.w);
     }
     __syncthreads();
-    // block rows a = 1, 2, 3: T_ab = -sum_{m=b}^{a-1} M_am T_mb
-#pragma unroll 1
-    for (int a = 1; a < 4; ++a) {
-      if (tid < 64 * a) {
-        const int i = tid / (4 * a), q4 = tid % (4 * a);
-        const int b = q4 >> 2, jq = q4 & 3;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int m = b; m < a; ++m) {
-          const float* Mrow = M32 + (a * (a - 1) / 2 + m) * 256 + i * 16;
+    // block rows a = 1, 2, 3: T_ab = -sum_{m=b}^{a-1} M_am T_mb; thread (q, i, jq)
+    // computes 4 columns of row i of block (a, q)
+    auto mt = [&](int p, int m, int i, int col) -> float4 {   // (M_p T)[i][col..col+3] over block m
+      const float* Mr = M32 + p * 256 + i * 16;
+      const float* Tc = T32 + 16 * m * LDA + col;
+      float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;
 #pragma unroll
-          for (int l4 = 0; l4 < 4; ++l4) {
-            const float4 m4 = *reinterpret_cast<const float4*>(Mrow + 4 * l4);
-            const float mv[4] = {m4.x, m4.y, m4.z, m4.w};
+      for (int l4 = 0; l4 < 4; ++l4) {
+        const float4 m4 = *reinterpret_cast<const float4*>(Mr + 4 * l4);
+        const float mv[4] = {m4.x, m4.y, m4.z, m4.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float4 t4 = *reinterpret_cast<const float4*>(T32 + (16 * m + 4 * l4 + e) * LDA + 16 * b + 4 * jq);
-              acc.x = fmaf(mv[e], t4.x, acc.x); acc.y = fmaf(mv[e], t4.y, acc.y);
-              acc.z = fmaf(mv[e], t4.z, acc.z); acc.w = fmaf(mv[e], t4.w, acc.w);
-            }
-          }
+        for (int e = 0; e < 4; ++e) {
+          const float4 t4 = *reinterpret_cast<const float4*>(Tc + (4 * l4 + e) * LDA);
+          float4& sacc = (e & 1) ? s1 : s0;
+          sacc.x = fmaf(mv[e], t4.x, sacc.x); sacc.y = fmaf(mv[e], t4.y, sacc.y);
+          sacc.z = fmaf(mv[e], t4.z, sacc.z); sacc.w = fmaf(mv[e], t4.w, sacc.w);
         }
-        *reinterpret_cast<float4*>(T32 + (16 * a + i) * LDA + 16 * b + 4 * jq) =
-            make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
       }
-      __syncthreads();
+      return make_float4(s0.x + s1.x, s0.y + s1.y, s0.z + s1.z, s0.w + s1.w);
+    };
+    auto put = [&](int row, int col, float4 x) {
+      *reinterpret_cast<float4*>(T32 + row * LDA + col) = make_float4(-x.x, -x.y, -x.z, -x.w);
+    };
+    if (tid < 64) {                                            // T_10
+      const int i = tid >> 2, jq = tid & 3;
+      put(16 + i, 4 * jq, mt(0, 0, i, 4 * jq));
     }
+    __syncthreads();
+    if (tid < 128) {                                           // T_20, T_21
+      const int q = tid >> 6, i = (tid >> 2) & 15, jq = tid & 3;
+      const int col = 16 * q + 4 * jq;
+      float4 x = mt(2, 1, i, col);                             // M_21 T_1q
+      if (q == 0) {
+        const float4 y = mt(1, 0, i, col);                     // M_20 T_00
+        x.x += y.x; x.y += y.y; x.z += y.z; x.w += y.w;
+      }
+      put(32 + i, col, x);
+    }
+    __syncthreads();
+    if (tid < 192) {                                           // T_30, T_31, T_32
+      const int q = tid >> 6, i = (tid >> 2) & 15, jq = tid & 3;
+      const int col = 16 * q + 4 * jq;
+      float4 x = mt(5, 2, i, col);                             // M_32 T_2q
+      if (q <= 1) {
+        const float4 y = mt(4, 1, i, col);                     // M_31 T_1q
+        x.x += y.x; x.y += y.y; x.z += y.z; x.w += y.w;
+      }
+      if (q == 0) {
+        const float4 y = mt(3, 0, i, col);                     // M_30 T_00
+        x.x += y.x; x.y += y.y; x.z += y.z; x.w += y.w;
+      }
+      put(48 + i, col, x);
+    }
+    __syncthreads();
     // T diag(beta) as bf16: B operand of W^T / U^T, K-major SW128, N = 64 (r'), K = 64 (r)
 #pragma unroll
     for (int it = 0; it < 2; ++it) {
@@ -603,25 +643,18 @@ kda_chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     tc_fence_before();
     __syncthreads();
 
-    // ================= P4: W^T, U^T, O^T = S^T Qbar^T ==========================
+    // ================= P4: W^T, U^T =============================================
     if (tid == 0) {
       tc_fence_after();
       const uint32_t tb_base = smem_u32(sm + OFF_TB);
       const uint32_t v_base = smem_u32(sm + OFF_V);
-      const uint32_t qb_base = smem_u32(sm + OFF_QB);
       const uint32_t id_w = idesc_bf16(128, 64, false, false);
       const uint32_t id_u = idesc_bf16(128, 64, true, false);
-      const uint32_t id_o = idesc_bf16(128, 64, false, true);
 #pragma unroll
       for (int kk = 0; kk < C / 16; ++kk) {
         const uint64_t bt = desc_kmajor_sw128(tb_base, C, kk);
         mma_ts(tb + TM_W, tb + TM_KB + kk * 8, bt, id_w, kk > 0);
         mma_ss(tb + TM_U, desc_mnmajor_sw128(v_base, C, kk), bt, id_u, kk > 0);
-      }
-      if (outputs) {
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ts(tb + TM_O, tb + TM_SB + kk * 8, desc_mnmajor_sw128(qb_base, D, kk), id_o, kk > 0);
       }
       mma_commit(&bar);
     }
@@ -636,15 +669,16 @@ kda_chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     // ================= P5: W^T -> bf16 smem ====================================
     if (!upper) {
       const int c = tid;
+      uint32_t t[4][16];
 #pragma unroll
-      for (int r0 = 0; r0 < C; r0 += 16) {
-        uint32_t t[16];
-        tmem_ld16(tb + lane_base + TM_W + r0, t);
-        tmem_wait_ld();
+      for (int q4 = 0; q4 < 4; ++q4) tmem_ld16(tb + lane_base + TM_W + 16 * q4, t[q4]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
 #pragma unroll
         for (int h8 = 0; h8 < 2; ++h8) {
-          const float* f = reinterpret_cast<const float*>(t) + 8 * h8;
-          st_v4(sm, OFF_WT + chunk_mnmajor_sw128((r0 >> 3) + h8, c, D), pack_bf16(f[0], f[1]),
+          const float* f = reinterpret_cast<const float*>(t[q4]) + 8 * h8;
+          st_v4(sm, OFF_WT + chunk_mnmajor_sw128(2 * q4 + h8, c, D), pack_bf16(f[0], f[1]),
                 pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]), pack_bf16(f[6], f[7]));
         }
       }
@@ -653,14 +687,22 @@ kda_chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     tc_fence_before();
     __syncthreads();
 
-    // ================= P6: P = S^T W^T ==========================================
+    // ================= P6: [O^T | P] = S^T [Qbar^T | W^T]^T =====================
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t wt_base = smem_u32(sm + OFF_WT);
-      const uint32_t id_p = idesc_bf16(128, 64, false, true);
+      if (outputs) {
+        const uint32_t qb_base = smem_u32(sm + OFF_QB);        // W^T follows 16 KB later
+        const uint32_t id_op = idesc_bf16(128, 128, false, true);
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk)
-        mma_ts(tb + TM_P, tb + TM_SB + kk * 8, desc_mnmajor_sw128(wt_base, D, kk), id_p, kk > 0);
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ts(tb + TM_O, tb + TM_SB + kk * 8, desc_mnmajor_sw128(qb_base, D, kk), id_op, kk > 0);
+      } else {
+        const uint32_t wt_base = smem_u32(sm + OFF_WT);
+        const uint32_t id_p = idesc_bf16(128, 64, false, true);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ts(tb + TM_P, tb + TM_SB + kk * 8, desc_mnmajor_sw128(wt_base, D, kk), id_p, kk > 0);
+      }
       mma_commit(&bar);
     }
     __syncwarp();
@@ -670,19 +712,26 @@ kda_chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     if (upper) {
       uint32_t dw[32];
 #pragma unroll
-      for (int r0 = 0; r0 < C; r0 += 16) {
-        uint32_t tu[16], tp[16];
-        tmem_ld16(tb + lane_base + TM_U + r0, tu);
-        tmem_ld16(tb + lane_base + TM_P + r0, tp);
-        tmem_wait_ld();
-        if (homog) {
+      for (int r0 = 0; r0 < C; r0 += 32) {
+        uint32_t tu[2][16], tp[2][16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) tu[e] = 0u;
+        for (int q2 = 0; q2 < 2; ++q2) {
+          tmem_ld16(tb + lane_base + TM_U + r0 + 16 * q2, tu[q2]);
+          tmem_ld16(tb + lane_base + TM_P + r0 + 16 * q2, tp[q2]);
         }
+        tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-          dw[r0 / 2 + e] = pack_bf16(__uint_as_float(tu[2 * e]) - __uint_as_float(tp[2 * e]),
-                                     __uint_as_float(tu[2 * e + 1]) - __uint_as_float(tp[2 * e + 1]));
+        for (int q2 = 0; q2 < 2; ++q2) {
+          if (homog) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) tu[q2][e] = 0u;
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            dw[(r0 + 16 * q2) / 2 + e] =
+                pack_bf16(__uint_as_float(tu[q2][2 * e]) - __uint_as_float(tp[q2][2 * e]),
+                          __uint_as_float(tu[q2][2 * e + 1]) - __uint_as_float(tp[q2][2 * e + 1]));
+        }
       }
       uint32_t w0[16], w1[16];
 #pragma unroll
@@ -694,19 +743,16 @@ kda_chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     tc_fence_before();
     __syncthreads();
 
-    // ================= P8: S^T += Delta^T Kend; O^T += Delta^T Aqk^T ============
+    // ================= P8: [S^T | O^T] += Delta^T [Kend^T ; Aqk]^T =============
     if (tid == 0) {
       tc_fence_after();
+      // Kend^T (128 rows) and Aqk (64 rows) form one K-major B operand of 192 rows
       const uint32_t ke_base = smem_u32(sm + OFF_KE);
-      const uint32_t aq_base = smem_u32(sm + OFF_AQK);
-      const uint32_t id_s = idesc_bf16(128, 128, false, false);
-      const uint32_t id_o = idesc_bf16(128, 64, false, false);
+      const int n = outputs ? D + C : D;
+      const uint32_t id_s = idesc_bf16(128, n, false, false);
 #pragma unroll
-      for (int kk = 0; kk < C / 16; ++kk) {
-        mma_ts(tb + TM_S, tb + TM_KB + kk * 8, desc_kmajor_sw128(ke_base, D, kk), id_s, 1);
-        if (outputs)
-          mma_ts(tb + TM_O, tb + TM_KB + kk * 8, desc_kmajor_sw128(aq_base, C, kk), id_o, 1);
-      }
+      for (int kk = 0; kk < C / 16; ++kk)
+        mma_ts(tb + TM_S, tb + TM_KB + kk * 8, desc_kmajor_sw128(ke_base, n, kk), id_s, 1);
       mma_commit(&bar);
     }
     __syncwarp();
@@ -716,26 +762,33 @@ kda_chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     if (upper) {
       const int j = tid - 128;
       bf16* otile = reinterpret_cast<bf16*>(sm + OFF_OUT);      // [64 tokens][128] row-major
+      if (outputs) {
+        uint32_t t[4][16];
 #pragma unroll
-      for (int r0 = 0; r0 < (outputs ? C : 0); r0 += 16) {
-        uint32_t t[16];
-        tmem_ld16(tb + lane_base + TM_O + r0, t);
+        for (int q4 = 0; q4 < 4; ++q4) tmem_ld16(tb + lane_base + TM_O + 16 * q4, t[q4]);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 16; ++e) otile[(r0 + e) * D + j] = __float2bfloat16_rn(__uint_as_float(t[e]));
+        for (int q4 = 0; q4 < 4; ++q4)
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            otile[(16 * q4 + e) * D + j] = __float2bfloat16_rn(__uint_as_float(t[q4][e]));
       }
 #pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t t0w[16], t1w[16], pk[16];
-        tmem_ld16(tb + lane_base + TM_S + c0, t0w);
-        tmem_ld16(tb + lane_base + TM_S + c0 + 16, t1w);
+      for (int c0 = 0; c0 < D; c0 += 64) {
+        uint32_t t[4][16], pk[2][16];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) tmem_ld16(tb + lane_base + TM_S + c0 + 16 * q4, t[q4]);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          pk[e] = pack_bf16(__uint_as_float(t0w[2 * e]), __uint_as_float(t0w[2 * e + 1]));
-          pk[8 + e] = pack_bf16(__uint_as_float(t1w[2 * e]), __uint_as_float(t1w[2 * e + 1]));
+        for (int q2 = 0; q2 < 2; ++q2) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            pk[q2][e] = pack_bf16(__uint_as_float(t[2 * q2][2 * e]), __uint_as_float(t[2 * q2][2 * e + 1]));
+            pk[q2][8 + e] =
+                pack_bf16(__uint_as_float(t[2 * q2 + 1][2 * e]), __uint_as_float(t[2 * q2 + 1][2 * e + 1]));
+          }
+          tmem_st16(tb + lane_base + TM_SB + c0 / 2 + 16 * q2, pk[q2]);
         }
-        tmem_st16(tb + lane_base + TM_SB + c0 / 2, pk);
       }
       tmem_wait_st();
       named_bar(1, 128);
