@@ -58,6 +58,9 @@ int kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
   if (rows * H * (long long)(dk > dv ? dk : dv) > (1LL << 40)) return KDA_ERR_INVALID_ARG;
   if ((long long)B > 65535LL || H > 65535) return KDA_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (kda::chunk_split_supported(dk, dv, in_dtype))
+    return status_from(kda::launch_chunk_split(q, k, v, g, beta, h0, cu_seqlens, out, hT, B, T,
+                                               H, st));
   if (kda::chunk_tc_supported(dk, dv, in_dtype))
     return status_from(kda::launch_chunk_tc(q, k, v, g, beta, h0, cu_seqlens, out, hT, B, T, H,
                                             st));

@@ -1,0 +1,938 @@
+// KDA prefill in two kernels on the sm_100a tensor cores, dk = dv = 128, bf16
+// q/k/v, fp32 g/beta/state.
+//
+// Chunked form (miniKimiK3 model card, "Kimi Delta Attention" bullet: training
+// and prefill run through a chunked parallel form; "Inside Kimi" outline,
+// DeltaNet lesson: chunkwise prefill trades arithmetic for parallel hardware
+// use).  For one chunk of L <= 64 tokens with initial state S (dk x dv) and
+// G_r = g_0 + ... + g_r (per key channel, restarting at the chunk):
+//     A[r,i]   = sum_c k_rc k_ic exp(G_rc - G_ic)        i <  r
+//     Aqk[r,i] = sum_c q_rc k_ic exp(G_rc - G_ic)        i <= r
+//     T        = (I + diag(beta) A)^-1
+//     W = T diag(beta) Kbar,  U = T diag(beta) V,        Kbar_r = exp(G_r) k_r
+//     Delta    = U - W S
+//     O        = Qbar S + Aqk Delta,                     Qbar_r = exp(G_r) q_r
+//     S_next   = Diag(exp(G_last)) S + Kend^T Delta,     Kend_i = exp(G_last - G_i) k_i
+// Rows past the end of a sequence are zero (k = q = beta = g = 0) and so
+// contribute nothing; G_last = G_63 then equals G at the last real row.
+//
+// Split.  Everything above except the last three lines depends on the chunk
+// alone, so it is computed for all (chunk, head) pairs at once by the prep
+// kernel (one CTA per pair, two CTAs per SM) and written out as a chunk record:
+// the operands of the state update, stored as the exact shared-memory images
+// the tensor cores read.  The state pass then walks each sequence's chunks in
+// order doing only the state-dependent work,
+//     [O^T | P]   [dv x 128] = S^T [Qbar^T | W^T]^T      (S^T bf16 copy in TMEM)
+//     Delta^T = U^T - P
+//     [S^T | O^T] [dv x 192] += Delta^T [Kend^T ; Aqk]^T  (after S^T <- S^T Diag(exp(G_last)))
+// with one bulk copy per record, two records ahead.  S^T stays in TMEM in fp32
+// for the whole chain.  Packed documents restart the state from their own h0
+// slot and restart chunking at the document start (Mini-K3-1H-mamba2 card,
+// packed-document paragraph: state flow resets at every boundary).
+//
+// Decay factoring in the prep kernel (exp(G_r - G_i) split through reference
+// points so no factor overflows): rows are grouped in 16-token blocks a with
+// P_a = G at row 16a.
+//   i, r in block a:   (k_r e^{G_r - P_a}) (k_i e^{P_a - G_i})
+//       first factor <= 1; second <= e^{decay over <= 15 tokens}, clamped at e^80
+//   i in block b < a:  (k_r e^{G_r - P_a}) (k_i e^{P_b - G_i} e^{P_a - P_b})
+// so the Gram of row block a is one product against R^(a) = [k_i e^{P_a - G_i}]
+// over i < 16(a+1): two exponentials per element.  Range limit: within one
+// 16-token block the cumulative log-decay must stay above -80 per channel.
+// All four products (A and Aqk rows for all blocks) are one MMA of N = 160:
+//   [D^(0) .. D^(3)] [128 x 160] = [Lk ; Lq] [R^(0); ..; R^(3)]^T
+#include <type_traits>
+
+#include "kda_common.cuh"
+#include "segments.cuh"
+#include "sm100.cuh"
+
+namespace kda {
+
+// Set when a bounded wait of the split prefill gives up (diagnostic).
+__device__ int g_chunk_split_timeout = 0;
+
+namespace {
+using namespace sm100;
+using bf16 = __nv_bfloat16;
+
+constexpr int C = kChunk;
+constexpr int D = kHead;
+constexpr int NT = 256;
+constexpr uint32_t kWaitLimit = 1u << 22;
+
+// ---- chunk record (one per (head, chunk)), byte offsets
+constexpr uint32_t REC_QW = 0;          // [Qbar^T | W^T]: MN-major SW128, N = 128 (2 x 64 tokens,
+                                        // 16 KB apart), K = dk
+constexpr uint32_t REC_KA = 32768;      // [Kend^T ; Aqk]: K-major SW128, 192 rows x 64 tokens
+constexpr uint32_t REC_AQK = REC_KA + 16384;
+constexpr uint32_t REC_U = 57344;       // U^T [dv][64 tokens] bf16: 128-byte rows, 16-byte
+                                        // chunks XOR-swizzled with (row % 8)
+constexpr uint32_t REC_DECAY = 73728;   // exp(G_last) per key channel, fp32 [dk]
+constexpr uint32_t REC_BYTES = 74240;
+
+// ---- prep kernel: shared memory (from a 1024-aligned base) and TMEM
+constexpr uint32_t Q_V = 0;             // V: MN-major SW128 A operand of U^T (M = value, K = token)
+constexpr uint32_t Q_KB = 16384;        // Kbar^T: K-major SW128 A operand of W^T
+constexpr uint32_t Q_L = 32768;         // [Lk ; Lq]: MN-major SW128 A operand of the Gram
+constexpr uint32_t Q_R = 65536;         // R^(0..3): MN-major SW32 B operand of the Gram, 40 KB
+__host__ __device__ constexpr uint32_t q_r(int a) {
+  return Q_R + (a == 0 ? 0u : a == 1 ? 4096u : a == 2 ? 12288u : 24576u);
+}
+// after the Gram has been read, the L / R region holds the solve
+constexpr int LDA = 68;                 // fp32 row stride (16-byte rows)
+constexpr uint32_t Q_B32 = 32768;       // diag(beta) A, fp32
+constexpr uint32_t Q_T32 = Q_B32 + 17408;   // T, fp32
+constexpr uint32_t Q_M32 = Q_T32 + 17408;   // T_aa B_am, 6 x 16 x 16 fp32
+constexpr uint32_t Q_TB = 73728;        // T diag(beta): K-major SW128 B operand of W^T / U^T
+constexpr uint32_t PREP_SMEM = 106496 + 1024;
+constexpr uint32_t PT_G = 0;            // Gram D^(0..3) at +0, +16, +48, +96 (160 columns)
+constexpr uint32_t PT_W = 0;            // W^T [128 x 64] (after the Gram is read)
+constexpr uint32_t PT_U = 64;           // U^T [128 x 64]
+constexpr uint32_t kPrepTmemCols = 256;
+
+// ---- state pass: shared memory and TMEM
+constexpr uint32_t S_BUF = 74752;       // record buffer stride (two buffers)
+constexpr uint32_t S_OUT = 2 * S_BUF;   // output tile [64 tokens][128] bf16
+constexpr uint32_t STATE_SMEM = S_OUT + 16384 + 1024;
+// [S^T | O^T] and [O^T | P] are each the accumulator of one MMA, so O^T sits
+// between S^T and P.
+constexpr uint32_t ST_S = 0;            // S^T fp32        [128 lanes x 128]
+constexpr uint32_t ST_O = 128;          // O^T             [128 x 64]
+constexpr uint32_t ST_P = 192;          // P               [128 x 64]
+constexpr uint32_t ST_SB = 256;         // S^T bf16 (A)    [128 x 64]
+constexpr uint32_t ST_D = 320;          // Delta^T bf16 (A) [128 x 32]
+constexpr uint32_t kStateTmemCols = 512;
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+__device__ __forceinline__ uint4 pack8(const float (&x)[8], float s) {
+  return make_uint4(pack_bf16(x[0] * s, x[1] * s), pack_bf16(x[2] * s, x[3] * s),
+                    pack_bf16(x[4] * s, x[5] * s), pack_bf16(x[6] * s, x[7] * s));
+}
+__device__ __forceinline__ void sts16(uint8_t* base, uint32_t off, uint4 v) {
+  *reinterpret_cast<uint4*>(base + off) = v;
+}
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// ============================================================================
+// Prep kernel: one CTA per (chunk slot, head).
+// ============================================================================
+__global__ void __launch_bounds__(NT, 2)
+kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
+                      const bf16* __restrict__ v, const float* __restrict__ g,
+                      const float* __restrict__ beta, const int32_t* __restrict__ cu_seqlens,
+                      uint8_t* __restrict__ rec, int B, int T, int H, long long nslots) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = align1024(smem_raw);
+  __shared__ uint64_t bar;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ float s_beta[C];
+  __shared__ float2 s_sum[4][64];       // per 16-row block: its total log-decay (channel pair)
+  __shared__ float2 s_first[4][64];     // per 16-row block: g at its first row
+
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const long long slot = blockIdx.x;
+  const int h = blockIdx.y;
+
+  // which chunk of which sequence this slot is (uniform over the CTA)
+  long long row0 = 0, t_beg = 0, t_end = 0, n = 0;
+  if (!cu_seqlens) {
+    const long long per = chunk_count(T);
+    if (per == 0 || slot >= per * B) return;
+    const int s = (int)(slot / per);
+    n = slot - (long long)s * per;
+    seq_range(nullptr, s, T, row0, t_beg, t_end);
+  } else {
+    long long base = 0;
+    bool found = false;
+    for (int d = 0; d < B && !found; ++d) {
+      seq_range(cu_seqlens, d, T, row0, t_beg, t_end);
+      const long long nc = chunk_count(t_end - t_beg);
+      if (slot < base + nc) { n = slot - base; found = true; }
+      base += nc;
+    }
+    if (!found) return;
+  }
+  const long long t0 = t_beg + n * C;
+  const int L = (int)min((long long)C, t_end - t0);
+  const long long rbase = row0 + t0;                   // first token row of the chunk
+  uint8_t* rc = rec + ((size_t)h * (size_t)nslots + (size_t)slot) * REC_BYTES;
+
+  // v goes straight into the MN-major operand of U^T (rows >= L zero-filled)
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int idx = tid + it * NT;
+    const int r = idx >> 4, ch = idx & 15;
+    const long long e = ((rbase + min(r, L - 1)) * H + h) * D + ch * 8;
+    cp_async16(sm + Q_V + chunk_mnmajor_sw128(ch, r, C), v + e, r < L ? 16u : 0u);
+  }
+  cp_async_commit();
+  if (tid < C) s_beta[tid] = tid < L ? beta[(rbase + tid) * H + h] : 0.f;
+  if (warp == 0) {
+    tmem_alloc(&tmem_base_sh, kPrepTmemCols);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+
+  // ---- P1: per thread a channel pair (2cp, 2cp+1) and a 16-row block a
+  const int cp = tid & 63, a = tid >> 6, c0 = 2 * cp;
+  float2 gq[16];
+  uint32_t kw[16], qw[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const int r = 16 * a + e;
+    if (r < L) {
+      const long long idx = ((rbase + r) * H + h) * D + c0;
+      gq[e] = __ldg(reinterpret_cast<const float2*>(g + idx));
+      kw[e] = __ldg(reinterpret_cast<const unsigned int*>(k + idx));
+      qw[e] = __ldg(reinterpret_cast<const unsigned int*>(q + idx));
+    } else {
+      gq[e] = make_float2(0.f, 0.f);
+      kw[e] = 0u;
+      qw[e] = 0u;
+    }
+  }
+#pragma unroll
+  for (int e = 1; e < 16; ++e) {
+    gq[e].x += gq[e - 1].x;
+    gq[e].y += gq[e - 1].y;
+  }
+  s_sum[a][cp] = gq[15];
+  s_first[a][cp] = gq[0];
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = tmem_base_sh;
+  const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+
+  float2 Pr[4], Pown = make_float2(0.f, 0.f), off = make_float2(0.f, 0.f),
+               run = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int a2 = 0; a2 < 4; ++a2) {
+    const float2 f = s_first[a2][cp], sm2 = s_sum[a2][cp];
+    Pr[a2] = make_float2(run.x + f.x, run.y + f.y);
+    if (a2 == a) { off = run; Pown = Pr[a2]; }
+    run.x += sm2.x;
+    run.y += sm2.y;
+  }
+  const float2 Glast = run;
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    gq[e].x += off.x;
+    gq[e].y += off.y;
+  }
+
+#pragma unroll
+  for (int ch = 0; ch < 2; ++ch) {
+    const int c = c0 + ch;
+    const float Pa = ch ? Pown.y : Pown.x;
+    const float Gl = ch ? Glast.y : Glast.x;
+    const float eP = __expf(Pa);               // Kbar, Qbar: e^{G_r} = e^{G_r - P_a} e^{P_a}
+    const float eE = __expf(Gl - Pa);          // Kend: e^{G_last - G_i} = e^{P_a - G_i} e^{G_last - P_a}
+    float f[4];
+#pragma unroll
+    for (int a2 = 0; a2 < 4; ++a2)
+      f[a2] = a2 > a ? __expf((ch ? Pr[a2].y : Pr[a2].x) - Pa) : 1.f;
+#pragma unroll
+    for (int gg = 0; gg < 2; ++gg) {
+      const int g8 = 2 * a + gg;               // group of 8 rows
+      float lk[8], lq[8], kr[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int idx = 8 * gg + e;
+        const float x = (ch ? gq[idx].y : gq[idx].x) - Pa;
+        const float ell = __expf(x);
+        const float rho = __expf(fminf(-x, 80.f));
+        const float kv = ch ? bf_hi(kw[idx]) : bf_lo(kw[idx]);
+        const float qv = ch ? bf_hi(qw[idx]) : bf_lo(qw[idx]);
+        lk[e] = kv * ell;
+        lq[e] = qv * ell;
+        kr[e] = kv * rho;                      // k_i e^{P_a - G_i}
+      }
+      sts16(sm, Q_L + chunk_mnmajor_sw128(g8, c, D), pack8(lk, 1.f));
+      sts16(sm, Q_L + chunk_mnmajor_sw128(8 + g8, c, D), pack8(lq, 1.f));
+      sts16(sm, Q_KB + chunk_kmajor_sw128(c, g8, D), pack8(lk, eP));
+#pragma unroll
+      for (int a2 = 0; a2 < 4; ++a2)
+        if (a2 >= a) sts16(sm, q_r(a2) + chunk_mnmajor_sw32(g8, c, D), pack8(kr, f[a2]));
+      // record: Qbar^T (MN-major, N = tokens, K = channels) and Kend^T (K-major)
+      *reinterpret_cast<uint4*>(rc + REC_QW + chunk_mnmajor_sw128(g8, c, D)) = pack8(lq, eP);
+      *reinterpret_cast<uint4*>(rc + REC_KA + chunk_kmajor_sw128(c, g8, D)) = pack8(kr, eE);
+    }
+  }
+  if (a == 3)
+    *reinterpret_cast<float2*>(rc + REC_DECAY + 4 * c0) =
+        make_float2(__expf(Glast.x), __expf(Glast.y));
+  cp_async_wait_all();
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+
+  uint32_t phase = 0;
+  auto mma_wait = [&]() -> bool {
+    const bool good = mbar_wait(&bar, phase, kWaitLimit);
+    phase ^= 1u;
+    tc_fence_after();
+    return __syncthreads_or(!good) == 0;
+  };
+  bool alive = true;
+
+  // ---- P2: Gram (one MMA per K step, N = 160)
+  if (tid == 0) {
+    tc_fence_after();
+    const uint32_t l_base = smem_u32(sm + Q_L), r_base = smem_u32(sm + q_r(0));
+    const uint32_t idesc = idesc_bf16(128, 160, true, true);
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk)
+      mma_ss(tb + PT_G, desc_mnmajor_sw128(l_base, D, kk), desc_mnmajor_sw32(r_base, D, kk), idesc,
+             kk > 0);
+    mma_commit(&bar);
+  }
+  __syncwarp();
+  if (!mma_wait()) alive = false;
+
+  float* B32 = reinterpret_cast<float*>(sm + Q_B32);
+  float* T32 = reinterpret_cast<float*>(sm + Q_T32);
+  float* M32 = reinterpret_cast<float*>(sm + Q_M32);
+  if (alive) {
+    // ---- P3: read A (beta-scaled, strictly lower, into B32) and Aqk (record)
+    // warp w (mod 4) reads TMEM lanes 32w..32w+31: w%4 = 0,1 -> A rows, 2,3 -> Aqk rows.
+    // Rows of a warp lie in blocks a0, a0+1; the lower warpgroup handles block a0
+    // and the upper warpgroup block a0+1.
+    const bool upper = tid >= 128;
+    const int w4 = warp & 3;
+    const int lane = tid & 31;
+    const int r = (w4 & 1) * 32 + lane;
+    const bool isA = w4 < 2;
+    const int a0 = (w4 & 1) * 2;
+    const int ab = a0 + (upper ? 1 : 0);
+    const int colb = ab == 0 ? 0 : ab == 1 ? 16 : ab == 2 ? 48 : 96;
+    const int nb = 16 * (ab + 1);
+    const bool mine = (r >> 4) == ab;
+    uint32_t tv[4][16];
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+      if (16 * q4 < nb) tmem_ld16(tb + lane_base + PT_G + colb + 16 * q4, tv[q4]);
+      else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) tv[q4][e] = 0u;
+      }
+    }
+    tmem_wait_ld();
+    if (mine) {
+      if (isA) {
+        const float br = s_beta[r];
+#pragma unroll
+        for (int i4 = 0; i4 < 16; ++i4) {
+          float4 w;
+          w.x = (4 * i4 + 0 < r) ? br * __uint_as_float(tv[i4 >> 2][(4 * i4 + 0) & 15]) : 0.f;
+          w.y = (4 * i4 + 1 < r) ? br * __uint_as_float(tv[i4 >> 2][(4 * i4 + 1) & 15]) : 0.f;
+          w.z = (4 * i4 + 2 < r) ? br * __uint_as_float(tv[i4 >> 2][(4 * i4 + 2) & 15]) : 0.f;
+          w.w = (4 * i4 + 3 < r) ? br * __uint_as_float(tv[i4 >> 2][(4 * i4 + 3) & 15]) : 0.f;
+          *reinterpret_cast<float4*>(B32 + r * LDA + 4 * i4) = w;
+        }
+      } else {
+        // Aqk row r: rows 128.. of the K-major [Kend^T ; Aqk] record operand
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) {
+          float w[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            w[e] = (c8 * 8 + e <= r) ? __uint_as_float(tv[c8 >> 1][(c8 & 1) * 8 + e]) : 0.f;
+          *reinterpret_cast<uint4*>(rc + REC_AQK + chunk_kmajor_sw128(r, c8, C)) = pack8(w, 1.f);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+
+  if (alive) {
+    // ---- triangular inverse T = (I + B)^-1, B = diag(beta) A
+    if (tid < 64) {                         // diagonal blocks: forward substitution
+      const int ab = tid >> 4, jj = tid & 15, o = 16 * ab;
+      float x[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) x[i] = (i == jj) ? 1.f : 0.f;
+#pragma unroll
+      for (int i = 1; i < 16; ++i) {
+        float acc = 0.f;
+#pragma unroll
+        for (int m = 0; m < i; ++m) acc = fmaf(B32[(o + i) * LDA + o + m], x[m], acc);
+        if (i > jj) x[i] = -acc;
+      }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) T32[(o + i) * LDA + o + jj] = x[i];
+    }
+    __syncthreads();
+    // M_am = T_aa B_am for the 6 pairs a > m (p = a(a-1)/2 + m); 384 items of
+    // 4 outputs, two accumulator chains each
+#pragma unroll 1
+    for (int w = tid; w < 384; w += NT) {
+      const int p = w >> 6, i = (w >> 2) & 15, jq = w & 3;
+      const int ar = p == 0 ? 1 : (p < 3 ? 2 : 3);
+      const int m = p - ar * (ar - 1) / 2;
+      const float* Ti = T32 + (16 * ar + i) * LDA + 16 * ar;
+      const float* Bc = B32 + 16 * ar * LDA + 16 * m + 4 * jq;
+      float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;
+#pragma unroll
+      for (int l = 0; l < 16; l += 2) {
+        const float4 b0 = *reinterpret_cast<const float4*>(Bc + l * LDA);
+        const float4 b1 = *reinterpret_cast<const float4*>(Bc + (l + 1) * LDA);
+        const float t0v = Ti[l], t1v = Ti[l + 1];
+        s0.x = fmaf(t0v, b0.x, s0.x); s0.y = fmaf(t0v, b0.y, s0.y);
+        s0.z = fmaf(t0v, b0.z, s0.z); s0.w = fmaf(t0v, b0.w, s0.w);
+        s1.x = fmaf(t1v, b1.x, s1.x); s1.y = fmaf(t1v, b1.y, s1.y);
+        s1.z = fmaf(t1v, b1.z, s1.z); s1.w = fmaf(t1v, b1.w, s1.w);
+      }
+      *reinterpret_cast<float4*>(M32 + p * 256 + i * 16 + 4 * jq) =
+          make_float4(s0.x + s1.x, s0.y + s1.y, s0.z + s1.z, s0.w + s1.w);
+    }
+    __syncthreads();
+    // block rows a = 1, 2, 3: T_ab = -sum_{m=b}^{a-1} M_am T_mb; thread (q, i, jq)
+    // computes 4 columns of row i of block (a, q)
+    auto mt = [&](int p, int m, int i, int col) -> float4 {   // (M_p T)[i][col..col+3] over block m
+      const float* Mr = M32 + p * 256 + i * 16;
+      const float* Tc = T32 + 16 * m * LDA + col;
+      float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;
+#pragma unroll
+      for (int l4 = 0; l4 < 4; ++l4) {
+        const float4 m4 = *reinterpret_cast<const float4*>(Mr + 4 * l4);
+        const float mv[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float4 t4 = *reinterpret_cast<const float4*>(Tc + (4 * l4 + e) * LDA);
+          float4& sacc = (e & 1) ? s1 : s0;
+          sacc.x = fmaf(mv[e], t4.x, sacc.x); sacc.y = fmaf(mv[e], t4.y, sacc.y);
+          sacc.z = fmaf(mv[e], t4.z, sacc.z); sacc.w = fmaf(mv[e], t4.w, sacc.w);
+        }
+      }
+      return make_float4(s0.x + s1.x, s0.y + s1.y, s0.z + s1.z, s0.w + s1.w);
+    };
+    auto put = [&](int row, int col, float4 x) {
+      *reinterpret_cast<float4*>(T32 + row * LDA + col) = make_float4(-x.x, -x.y, -x.z, -x.w);
+    };
+    if (tid < 64) {                                            // T_10
+      const int i = tid >> 2, jq = tid & 3;
+      put(16 + i, 4 * jq, mt(0, 0, i, 4 * jq));
+    }
+    __syncthreads();
+    if (tid < 128) {                                           // T_20, T_21
+      const int qb = tid >> 6, i = (tid >> 2) & 15, jq = tid & 3;
+      const int col = 16 * qb + 4 * jq;
+      float4 x = mt(2, 1, i, col);                             // M_21 T_1q
+      if (qb == 0) {
+        const float4 y = mt(1, 0, i, col);                     // M_20 T_00
+        x.x += y.x; x.y += y.y; x.z += y.z; x.w += y.w;
+      }
+      put(32 + i, col, x);
+    }
+    __syncthreads();
+    if (tid < 192) {                                           // T_30, T_31, T_32
+      const int qb = tid >> 6, i = (tid >> 2) & 15, jq = tid & 3;
+      const int col = 16 * qb + 4 * jq;
+      float4 x = mt(5, 2, i, col);                             // M_32 T_2q
+      if (qb <= 1) {
+        const float4 y = mt(4, 1, i, col);                     // M_31 T_1q
+        x.x += y.x; x.y += y.y; x.z += y.z; x.w += y.w;
+      }
+      if (qb == 0) {
+        const float4 y = mt(3, 0, i, col);                     // M_30 T_00
+        x.x += y.x; x.y += y.y; x.z += y.z; x.w += y.w;
+      }
+      put(48 + i, col, x);
+    }
+    __syncthreads();
+    // T diag(beta) as bf16: B operand of W^T / U^T, K-major SW128, N = 64 (r'), K = 64 (r)
+#pragma unroll
+    for (int it = 0; it < 2; ++it) {
+      const int idx = tid + it * NT;
+      const int rp = idx >> 3, c8 = idx & 7;
+      float w[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int rr = c8 * 8 + e;
+        w[e] = (rr <= rp) ? T32[rp * LDA + rr] * s_beta[rr] : 0.f;
+      }
+      sts16(sm, Q_TB + chunk_kmajor_sw128(rp, c8, C), pack8(w, 1.f));
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+
+    // ---- P4: W^T = Kbar^T (T beta)^T, U^T = V^T (T beta)^T
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t tb_base = smem_u32(sm + Q_TB);
+      const uint32_t kb_base = smem_u32(sm + Q_KB);
+      const uint32_t v_base = smem_u32(sm + Q_V);
+      const uint32_t id_w = idesc_bf16(128, 64, false, false);
+      const uint32_t id_u = idesc_bf16(128, 64, true, false);
+#pragma unroll
+      for (int kk = 0; kk < C / 16; ++kk) {
+        const uint64_t bt = desc_kmajor_sw128(tb_base, C, kk);
+        mma_ss(tb + PT_W, desc_kmajor_sw128(kb_base, D, kk), bt, id_w, kk > 0);
+        mma_ss(tb + PT_U, desc_mnmajor_sw128(v_base, C, kk), bt, id_u, kk > 0);
+      }
+      mma_commit(&bar);
+    }
+    __syncwarp();
+    if (!mma_wait()) alive = false;
+  }
+
+  if (alive) {
+    // ---- P5: W^T (lower warpgroup) and U^T (upper) -> bf16 record images
+    const int j = tid & 127;
+    uint32_t t[4][16];
+    const uint32_t col = tid < 128 ? PT_W : PT_U;
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) tmem_ld16(tb + lane_base + col + 16 * q4, t[q4]);
+    tmem_wait_ld();
+#pragma unroll
+    for (int g8 = 0; g8 < 8; ++g8) {
+      const uint32_t* f = t[g8 >> 1] + 8 * (g8 & 1);
+      const uint4 val = make_uint4(pack_bf16(__uint_as_float(f[0]), __uint_as_float(f[1])),
+                                   pack_bf16(__uint_as_float(f[2]), __uint_as_float(f[3])),
+                                   pack_bf16(__uint_as_float(f[4]), __uint_as_float(f[5])),
+                                   pack_bf16(__uint_as_float(f[6]), __uint_as_float(f[7])));
+      const uint32_t o = tid < 128 ? REC_QW + 16384 + chunk_mnmajor_sw128(g8, j, D)
+                                   : REC_U + j * 128 + (((uint32_t)g8 ^ (j & 7u)) << 4);
+      *reinterpret_cast<uint4*>(rc + o) = val;
+    }
+  }
+
+  if (!alive && tid == 0) {
+    atomicExch(&g_chunk_split_timeout, 1);
+    mbar_wait(&bar, phase, kWaitLimit);   // let an MMA still in flight finish
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tb, kPrepTmemCols);
+  }
+}
+
+// ============================================================================
+// State pass: one CTA per chain (sequence, head[, segment]).
+// ============================================================================
+__global__ void __launch_bounds__(NT, 1)
+kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
+                      const int32_t* __restrict__ cu_seqlens, bf16* __restrict__ out, float* hT,
+                      int T, int H, long long nslots, SegArgs sa) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = align1024(smem_raw);
+  __shared__ uint64_t full[2];
+  __shared__ uint64_t mbar;
+  __shared__ uint32_t tmem_base_sh;
+
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int h = blockIdx.x, s = blockIdx.y;
+  const int wg = tid >> 7, j = tid & 127;
+  const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+
+  long long row0, t_beg, t_end;
+  seq_range(cu_seqlens, s, T, row0, t_beg, t_end);
+  const long long seq_t0 = t_beg;
+  // what this chain computes: a token range, where its state starts, where it ends
+  const long long hoff = ((long long)s * H + h) * D * D;
+  const float* init = h0 ? h0 + hoff : nullptr;   // nullptr: zero state
+  bool init_identity = false;
+  float* fin = hT ? hT + hoff : nullptr;          // nullptr: final state not kept
+  bool outputs = true, homog = false;
+  if (sa.pass != 0) {
+    const int Ps = seg_count(t_end - t_beg, sa.G);
+    const int z = blockIdx.z;
+    const long long seg_tok = (long long)sa.G * C;
+    auto slot_off = [&](int p) -> long long {
+      const int sl = seg_slot_base(cu_seqlens, s, T, sa.G) + p;
+      return sl < sa.slots ? ((long long)sl * H + h) * D * D : -1;
+    };
+    if (sa.pass == 1) {
+      const bool xtype = z >= sa.P;
+      const int p = xtype ? z - sa.P : z;
+      if (Ps <= 1) {
+        if (z != 0) return;                       // whole sequence in this one chain
+      } else if (!xtype) {
+        if (p > Ps - 2) return;
+        const long long o = slot_off(p);
+        if (o < 0) return;
+        if (p > 0) { init = nullptr; outputs = false; }
+        fin = sa.sbuf + o;
+        t_beg += p * seg_tok;
+        t_end = min(t_end, t_beg + seg_tok);
+      } else {
+        if (p < 1 || p > Ps - 2) return;
+        const long long o = slot_off(p);
+        if (o < 0) return;
+        init = nullptr; init_identity = true; outputs = false; homog = true;
+        fin = sa.xbuf + o;
+        t_beg += p * seg_tok;
+        t_end = min(t_end, t_beg + seg_tok);
+      }
+    } else {
+      const int p = z + 1;
+      if (Ps <= 1 || p > Ps - 1) return;
+      const long long o = slot_off(p - 1);
+      if (o < 0) return;
+      init = sa.sbuf + o;
+      if (p != Ps - 1) fin = nullptr;
+      t_beg += p * seg_tok;
+      t_end = min(t_end, t_beg + seg_tok);
+    }
+  }
+  const int nch = (int)chunk_count(t_end - t_beg);
+  const long long cg0 = seq_chunk_base(cu_seqlens, s, T) + (t_beg - seq_t0) / C;
+  const uint8_t* rec_h = rec + (size_t)h * (size_t)nslots * REC_BYTES;
+  auto rec_ptr = [&](int i) { return rec_h + (size_t)(cg0 + i) * REC_BYTES; };
+
+  if (warp == 0) {
+    tmem_alloc(&tmem_base_sh, kStateTmemCols);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(&full[0], 1);
+    mbar_init(&full[1], 1);
+    mbar_init(&mbar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    for (int i = 0; i < 2 && i < nch; ++i) {
+      mbar_arrive_expect_tx(&full[i], REC_BYTES);
+      bulk_g2s(sm + i * S_BUF, rec_ptr(i), REC_BYTES, &full[i]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = tmem_base_sh;
+
+  // ---- initial state: thread (wg, j) holds row j of S^T, columns [64 wg, 64 wg + 64)
+#pragma unroll 1
+  for (int cc = 0; cc < 64; cc += 32) {
+    const int c = 64 * wg + cc;
+    uint32_t f0[16], f1[16], pk[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      float x0 = init ? init[(long long)(c + e) * D + j] : 0.f;
+      float x1 = init ? init[(long long)(c + 16 + e) * D + j] : 0.f;
+      if (init_identity) { x0 = (c + e == j) ? 1.f : 0.f; x1 = (c + 16 + e == j) ? 1.f : 0.f; }
+      f0[e] = __float_as_uint(x0);
+      f1[e] = __float_as_uint(x1);
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      pk[e] = pack_bf16(__uint_as_float(f0[2 * e]), __uint_as_float(f0[2 * e + 1]));
+      pk[8 + e] = pack_bf16(__uint_as_float(f1[2 * e]), __uint_as_float(f1[2 * e + 1]));
+    }
+    tmem_st16(tb + lane_base + ST_S + c, f0);
+    tmem_st16(tb + lane_base + ST_S + c + 16, f1);
+    tmem_st16(tb + lane_base + ST_SB + c / 2, pk);
+  }
+  tmem_wait_st();
+  bool good = nch == 0 || mbar_wait(&full[0], 0, kWaitLimit);
+  tc_fence_before();
+  bool alive = __syncthreads_or(!good) == 0;
+  tc_fence_after();
+
+  uint32_t mphase = 0;
+  int waited = alive && nch > 0 ? 1 : 0;             // records whose arrival has been seen
+  int issued = nch < 2 ? nch : 2;                    // records requested
+#pragma unroll 1
+  for (int i = 0; i < nch && alive; ++i) {
+    const int buf = i & 1;
+    uint8_t* rb = sm + buf * S_BUF;
+    const long long t0 = t_beg + (long long)i * C;
+    const int L = (int)min((long long)C, t_end - t0);
+
+    // ---- [O^T | P] = S^T [Qbar^T | W^T]^T   (P only when no outputs are kept)
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t qw = smem_u32(rb + REC_QW);
+      if (outputs) {
+        const uint32_t id = idesc_bf16(128, 128, false, true);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ts(tb + ST_O, tb + ST_SB + kk * 8, desc_mnmajor_sw128(qw, D, kk), id, kk > 0);
+      } else {
+        const uint32_t id = idesc_bf16(128, 64, false, true);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ts(tb + ST_P, tb + ST_SB + kk * 8, desc_mnmajor_sw128(qw + 16384, D, kk), id,
+                 kk > 0);
+      }
+      mma_commit(&mbar);
+    }
+    __syncwarp();
+    // meanwhile S^T <- S^T Diag(exp(G_last)) (the MMA reads only the bf16 copy)
+    {
+      const float* dec = reinterpret_cast<const float*>(rb + REC_DECAY) + 64 * wg;
+      uint32_t t[4][16];
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) tmem_ld16(tb + lane_base + ST_S + 64 * wg + 16 * q4, t[q4]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          t[q4][e] = __float_as_uint(__uint_as_float(t[q4][e]) * dec[16 * q4 + e]);
+        tmem_st16(tb + lane_base + ST_S + 64 * wg + 16 * q4, t[q4]);
+      }
+      tmem_wait_st();
+    }
+    tc_fence_before();
+    good = mbar_wait(&mbar, mphase, kWaitLimit);
+    mphase ^= 1u;
+    tc_fence_after();
+    if (__syncthreads_or(!good)) { alive = false; break; }
+
+    // ---- Delta^T = U^T - P for tokens [32 wg, 32 wg + 32) -> bf16 TMEM
+    {
+      uint32_t tp[2][16];
+      tmem_ld16(tb + lane_base + ST_P + 32 * wg, tp[0]);
+      tmem_ld16(tb + lane_base + ST_P + 32 * wg + 16, tp[1]);
+      uint4 u[4];
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4)
+        u[c4] = homog ? make_uint4(0u, 0u, 0u, 0u)
+                      : *reinterpret_cast<const uint4*>(
+                            rb + REC_U + j * 128 + ((((uint32_t)(4 * wg + c4)) ^ (j & 7u)) << 4));
+      tmem_wait_ld();
+      uint32_t dw[16];
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {
+        const uint32_t uw[4] = {u[c4].x, u[c4].y, u[c4].z, u[c4].w};
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2) {
+          const float p0 = __uint_as_float(tp[c4 >> 1][(c4 & 1) * 8 + 2 * e2]);
+          const float p1 = __uint_as_float(tp[c4 >> 1][(c4 & 1) * 8 + 2 * e2 + 1]);
+          dw[4 * c4 + e2] = pack_bf16(bf_lo(uw[e2]) - p0, bf_hi(uw[e2]) - p1);
+        }
+      }
+      tmem_st16(tb + lane_base + ST_D + 16 * wg, dw);
+      tmem_wait_st();
+    }
+    tc_fence_before();
+    __syncthreads();
+
+    // ---- [S^T | O^T] += Delta^T [Kend^T ; Aqk]^T
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t ka = smem_u32(rb + REC_KA);
+      const int n = outputs ? D + C : D;
+      const uint32_t id = idesc_bf16(128, n, false, false);
+#pragma unroll
+      for (int kk = 0; kk < C / 16; ++kk)
+        mma_ts(tb + ST_S, tb + ST_D + kk * 8, desc_kmajor_sw128(ka, n, kk), id, 1);
+      mma_commit(&mbar);
+    }
+    __syncwarp();
+    good = mbar_wait(&mbar, mphase, kWaitLimit);
+    mphase ^= 1u;
+    tc_fence_after();
+    if (__syncthreads_or(!good)) { alive = false; break; }
+
+    // the record in this buffer is consumed: fetch record i + 2 into it
+    if (tid == 0 && i + 2 < nch) {
+      fence_async_smem();
+      mbar_arrive_expect_tx(&full[buf], REC_BYTES);
+      bulk_g2s(rb, rec_ptr(i + 2), REC_BYTES, &full[buf]);
+    }
+    if (i + 2 < nch) ++issued;
+
+    // ---- lower warpgroup: bf16 copy of the new state; upper: outputs to the tile
+    bf16* otile = reinterpret_cast<bf16*>(sm + S_OUT);
+    if (wg == 0) {
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 64) {
+        uint32_t t[4][16], pk[2][16];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) tmem_ld16(tb + lane_base + ST_S + c0 + 16 * q4, t[q4]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int q2 = 0; q2 < 2; ++q2) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            pk[q2][e] = pack_bf16(__uint_as_float(t[2 * q2][2 * e]),
+                                  __uint_as_float(t[2 * q2][2 * e + 1]));
+            pk[q2][8 + e] = pack_bf16(__uint_as_float(t[2 * q2 + 1][2 * e]),
+                                      __uint_as_float(t[2 * q2 + 1][2 * e + 1]));
+          }
+          tmem_st16(tb + lane_base + ST_SB + c0 / 2 + 16 * q2, pk[q2]);
+        }
+      }
+      tmem_wait_st();
+    } else if (outputs) {
+      uint32_t t[4][16];
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) tmem_ld16(tb + lane_base + ST_O + 16 * q4, t[q4]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4)
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          otile[(16 * q4 + e) * D + j] = __float2bfloat16_rn(__uint_as_float(t[q4][e]));
+    }
+    tc_fence_before();
+    good = true;
+    if (i + 1 < nch) {
+      good = mbar_wait(&full[(i + 1) & 1], ((i + 1) >> 1) & 1, kWaitLimit);
+      if (good) waited = i + 2;
+    }
+    if (__syncthreads_or(!good)) { alive = false; break; }
+    tc_fence_after();
+    // upper warpgroup: coalesced 16-byte stores of the tile (overlap the next MMA)
+    if (wg == 1 && outputs) {
+#pragma unroll
+      for (int it = 0; it < 8; ++it) {
+        const int idx = j + it * 128;
+        const int r = idx >> 4, ch = idx & 15;
+        if (r < L) {
+          const uint4 val = *reinterpret_cast<const uint4*>(sm + S_OUT + r * 256 + ch * 16);
+          *reinterpret_cast<uint4*>(out + ((row0 + t0 + r) * H + h) * D + ch * 8) = val;
+        }
+      }
+    }
+  }
+
+  // ---- final state
+  if (alive && fin) {
+#pragma unroll 1
+    for (int c0 = 64 * wg; c0 < 64 * wg + 64; c0 += 16) {
+      uint32_t t[16];
+      tmem_ld16(tb + lane_base + ST_S + c0, t);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 16; ++e) fin[(long long)(c0 + e) * D + j] = __uint_as_float(t[e]);
+    }
+  }
+  if (!alive && tid == 0) {
+    atomicExch(&g_chunk_split_timeout, 1);
+    // let the MMA and the copies still in flight finish before the CTA exits
+    mbar_wait(&mbar, mphase, kWaitLimit);
+    for (int r = waited; r < issued; ++r) mbar_wait(&full[r & 1], (r >> 1) & 1, kWaitLimit);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tb, kStateTmemCols);
+  }
+}
+
+// Dynamic shared memory of the kernels, set once per device.
+bool set_attrs() {
+  static bool done[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (!done[dev]) {
+    if (cudaFuncSetAttribute(kda_chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             PREP_SMEM) != cudaSuccess ||
+        cudaFuncSetAttribute(kda_state_pass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             STATE_SMEM) != cudaSuccess)
+      return false;
+    done[dev] = true;
+  }
+  return true;
+}
+
+// Chunks per segment (0: no split).  Cost model in units of one state-pass
+// chunk step: pass A runs NH*(2P-3) chains, pass C NH*(P-1), each G chunks
+// long, in waves of one chain per SM; the combine costs kCombine steps per
+// segment.
+constexpr double kCombine = 12.0;
+int plan_split(int B, int T, int H, bool varlen, int sms) {
+  const long long NH = (long long)B * H;
+  const long long nch = ((long long)T + C - 1) / C;
+  if (NH >= sms || nch < 8) return 0;
+  if (varlen) return nch >= 2 * 16 ? 16 : 0;
+  const long long w1 = (NH + sms - 1) / sms;
+  double best = (double)(nch * w1);
+  int bestG = 0;
+  for (int P = 2; P <= 64 && P <= nch; ++P) {
+    const long long G = (nch + P - 1) / P;
+    const long long Pe = (nch + G - 1) / G;
+    if (Pe < 2) continue;
+    const long long wA = (NH * (2 * Pe - 3) + sms - 1) / sms;
+    const long long wC = (NH * (Pe - 1) + sms - 1) / sms;
+    const double cost = (double)G * (double)(wA + wC) + kCombine * (double)(Pe - 2) + 2.0;
+    if (cost < best) { best = cost; bestG = (int)G; }
+  }
+  return bestG;
+}
+
+}  // namespace
+
+bool chunk_split_supported(int dk, int dv, int in_dtype) {
+  return in_dtype == KDA_BF16 && dk == D && dv == D;
+}
+
+cudaError_t launch_chunk_split(const void* q, const void* k, const void* v, const float* g,
+                               const float* beta, const float* h0, const int32_t* cu_seqlens,
+                               void* out, float* hT, int B, int T, int H, cudaStream_t stream) {
+  int sms = 148;
+  cudaMemPool_t pool = nullptr;
+  if (!device_ctx(&sms, &pool) || !set_attrs()) return cudaErrorInvalidDevice;
+  if (!pool) return cudaErrorMemoryAllocation;
+  const bf16* qb = static_cast<const bf16*>(q);
+  const bf16* kb = static_cast<const bf16*>(k);
+  const bf16* vb = static_cast<const bf16*>(v);
+  bf16* ob = static_cast<bf16*>(out);
+  const bool varlen = cu_seqlens != nullptr;
+
+  const long long nslots = chunk_slots(B, T, varlen);
+  const size_t rec_bytes = (size_t)nslots * H * REC_BYTES;
+  const int G = plan_split(B, T, H, varlen, sms);
+  const long long nch_all = ((long long)T + C - 1) / C;
+  int P = 0;
+  long long slots = 0;
+  size_t seg_bytes = 0;
+  if (G > 0 && (nch_all + G - 1) / G >= 2) {
+    P = (int)((nch_all + G - 1) / G);
+    slots = varlen ? (long long)P + B : (long long)B * P;
+    seg_bytes = (size_t)2 * slots * H * D * D * sizeof(float);
+  }
+  void* scratch = nullptr;
+  if (rec_bytes + seg_bytes > 0) {
+    const cudaError_t e = cudaMallocFromPoolAsync(&scratch, rec_bytes + seg_bytes, pool, stream);
+    if (e != cudaSuccess) return e;
+  }
+  uint8_t* rec = static_cast<uint8_t*>(scratch);
+  float* segbuf = reinterpret_cast<float*>(rec + rec_bytes);
+
+  cudaError_t e = cudaSuccess;
+  if (nslots > 0) {
+    kda_chunk_prep_kernel<<<dim3((unsigned)nslots, H), NT, PREP_SMEM, stream>>>(
+        qb, kb, vb, g, beta, cu_seqlens, rec, B, T, H, nslots);
+    note_launches(1);
+  }
+  if (P == 0) {
+    SegArgs sa{0, 1, 0, 0, nullptr, nullptr};
+    kda_state_pass_kernel<<<dim3(H, B, 1), NT, STATE_SMEM, stream>>>(rec, h0, cu_seqlens, ob, hT,
+                                                                     T, H, nslots, sa);
+    note_launches(1);
+  } else {
+    SegArgs sa{G, P, 1, (int)slots, segbuf, segbuf + (size_t)slots * H * D * D};
+    kda_state_pass_kernel<<<dim3(H, B, 2 * P), NT, STATE_SMEM, stream>>>(rec, h0, cu_seqlens, ob,
+                                                                         hT, T, H, nslots, sa);
+    const cudaError_t ec = launch_seg_combine(cu_seqlens, B, T, H, sa, stream);
+    sa.pass = 2;
+    kda_state_pass_kernel<<<dim3(H, B, P - 1), NT, STATE_SMEM, stream>>>(rec, h0, cu_seqlens, ob,
+                                                                         hT, T, H, nslots, sa);
+    note_launches(2);
+    if (ec != cudaSuccess) e = ec;
+  }
+  const cudaError_t el = cudaGetLastError();
+  if (e == cudaSuccess) e = el;
+  if (scratch) cudaFreeAsync(scratch, stream);
+  return e;
+}
+
+}  // namespace kda

@@ -55,6 +55,7 @@
 #include <type_traits>
 
 #include "kda_common.cuh"
+#include "segments.cuh"
 #include "sm100.cuh"
 
 namespace kda {
@@ -66,8 +67,8 @@ namespace {
 using namespace sm100;
 using bf16 = __nv_bfloat16;
 
-constexpr int C = 64;
-constexpr int D = 128;
+constexpr int C = kChunk;
+constexpr int D = kHead;
 constexpr int NT = 256;
 
 // ---- shared memory map (bytes from a 1024-aligned base)
@@ -203,54 +204,6 @@ __device__ __forceinline__ void build_half(uint8_t* sm, const float (&gv)[32], c
     }
   }
   tmem_st16(tm_kb + 16 * HF, kbw);
-}
-
-// Sequence splitting.  When there are too few (sequence, head) pairs to fill
-// the GPU, each sequence is cut into segments of G chunks and the scan runs in
-// three launches:
-//   pass A  segment 0 runs from h0 and writes its outputs; segments p >= 1 run
-//           from a zero state (no outputs) and keep their local end state
-//           Sloc_p; further CTAs run segments 1 <= p <= Ps-2 from the identity
-//           with the write term dropped (U = 0), which yields the segment's
-//           transition X_p (S_end = X_p S_start + Sloc_p, both dk x dk / dk x dv);
-//   combine S_start,1 = S_end,0 and S_start,p+1 = X_p S_start,p + Sloc_p (fp32);
-//   pass C  segments p >= 1 run again from S_start,p and write their outputs;
-//           the last one writes hT.
-// This is the chunked recurrence's own affine structure over chunks, grouped.
-struct SegArgs {
-  int G;          // chunks per segment; 0 = one CTA walks the whole sequence
-  int P;          // segment slots per sequence in the grid (z extent of pass C)
-  int pass;       // 0 = single pass, 1 = pass A, 2 = pass C
-  int slots;      // number of (segment) slots the scratch holds per head
-  float* sbuf;    // [slots][H][D][D] fp32: Sloc_p, then S_start,p+1
-  float* xbuf;    // [slots][H][D][D] fp32: X_p
-};
-
-__device__ __forceinline__ void seq_range(const int32_t* cu, int s, int T, long long& row0,
-                                          long long& t_beg, long long& t_end) {
-  if (cu) {
-    int a = cu[s], b = cu[s + 1];
-    a = min(max(a, 0), T);
-    b = min(max(b, a), T);
-    row0 = 0; t_beg = a; t_end = b;
-  } else {
-    row0 = (long long)s * T; t_beg = 0; t_end = T;
-  }
-}
-__device__ __forceinline__ int seg_count(long long len, int G) {
-  const long long nch = (len + C - 1) / C;
-  return (int)((nch + G - 1) / G);
-}
-// first scratch slot of sequence s: segments of all earlier sequences
-__device__ __forceinline__ int seg_slot_base(const int32_t* cu, int s, int T, int G) {
-  if (!cu) return s * seg_count(T, G);
-  int base = 0;
-  for (int d = 0; d < s; ++d) {
-    long long r0, a, b;
-    seq_range(cu, d, T, r0, a, b);
-    base += seg_count(b - a, G);
-  }
-  return base;
 }
 
 __global__ void __launch_bounds__(NT, 1)
@@ -833,180 +786,6 @@ kda_chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   }
 }
 
-// Combine of the segment maps:
-//   S_start,1 = S_end,0;  S_start,p+1 = X_p S_start,p + Sloc_p  (p = 1 .. Ps-2),
-// S_start,p+1 overwriting Sloc_p's slot.  One CTA per (sequence, head) runs the
-// chain on the tensor cores with fp32-level accuracy: each fp32 operand is split
-// into bf16 hi + lo parts and X S = Xh Sh + Xh Sl + Xl Sh (the dropped Xl Sl is
-// ~2^-16 relative), accumulated in fp32 in TMEM.  Global traffic is coalesced
-// (warp w, lane l handles rows w + 4i, columns 4l..4l+3); thread c reads row c
-// of the product from TMEM lane c.
-constexpr int kCombineThreads = 128;
-constexpr uint32_t CB_AH = 0, CB_AL = 32768, CB_BH = 65536, CB_BL = 98304;
-constexpr uint32_t CB_LOC = 131072;                          // fp32 rows [D][LOC_LD]
-constexpr int LOC_LD = 132;                                   // padded: float4 rows conflict-free
-constexpr size_t kCombineSmem = 131072 + D * LOC_LD * 4 + 1024;
-
-__device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
-  hi = pack_bf16(a, b);
-  lo = pack_bf16(a - __uint_as_float(hi << 16), b - __uint_as_float(hi & 0xffff0000u));
-}
-
-__global__ void __launch_bounds__(kCombineThreads, 1)
-kda_seg_combine_kernel(const int32_t* __restrict__ cu_seqlens, int T, int H, SegArgs sa) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                           ~uintptr_t(1023));
-  __shared__ uint64_t bar;
-  __shared__ uint32_t tmem_base_sh;
-  const int h = blockIdx.x, s = blockIdx.y;
-  long long r0, a, b;
-  seq_range(cu_seqlens, s, T, r0, a, b);
-  const int Ps = seg_count(b - a, sa.G);
-  if (Ps <= 2) return;
-  const int base = seg_slot_base(cu_seqlens, s, T, sa.G);
-  if (base + Ps - 1 > sa.slots) return;                    // offsets beyond the planned scratch
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, c = tid;
-  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-  float* loc = reinterpret_cast<float*>(sm + CB_LOC);
-  auto slot = [&](int p) { return ((long long)(base + p) * H + h) * D * D; };
-
-  // coalesced row copy global -> padded smem rows (cp.async)
-  auto load_loc = [&](const float* src) {
-#pragma unroll 8
-    for (int i = 0; i < D / 4; ++i) {
-      const int r = warp + 4 * i;
-      cp_async16(loc + r * LOC_LD + 4 * lane, src + (long long)r * D + 4 * lane, 16u);
-    }
-    cp_async_commit();
-  };
-  // X rows into registers, coalesced: xr[i] = X[warp + 4i][4 lane .. 4 lane + 3]
-  float4 xr[D / 4];
-  auto load_x = [&](const float* src) {
-#pragma unroll
-    for (int i = 0; i < D / 4; ++i)
-      xr[i] = *reinterpret_cast<const float4*>(src + (long long)(warp + 4 * i) * D + 4 * lane);
-  };
-  // A (K-major): element (row r, k) -> 8-byte piece of chunk (r, k / 8)
-  auto store_a = [&]() {
-#pragma unroll
-    for (int i = 0; i < D / 4; ++i) {
-      const int r = warp + 4 * i, k = 4 * lane;
-      uint32_t h0, l0, h1, l1;
-      split2(xr[i].x, xr[i].y, h0, l0);
-      split2(xr[i].z, xr[i].w, h1, l1);
-      const uint32_t o = chunk_kmajor_sw128(r, k >> 3, D) + (k & 7) * 2;
-      *reinterpret_cast<uint2*>(sm + CB_AH + o) = make_uint2(h0, h1);
-      *reinterpret_cast<uint2*>(sm + CB_AL + o) = make_uint2(l0, l1);
-    }
-  };
-  // B (MN-major) K-row c from loc row c
-  auto store_b = [&]() {
-    const float* lr = loc + c * LOC_LD;
-#pragma unroll
-    for (int c8 = 0; c8 < D / 8; ++c8) {
-      const float4 u = *reinterpret_cast<const float4*>(lr + c8 * 8);
-      const float4 w = *reinterpret_cast<const float4*>(lr + c8 * 8 + 4);
-      uint32_t hw[4], lw[4];
-      split2(u.x, u.y, hw[0], lw[0]); split2(u.z, u.w, hw[1], lw[1]);
-      split2(w.x, w.y, hw[2], lw[2]); split2(w.z, w.w, hw[3], lw[3]);
-      const uint32_t o = chunk_mnmajor_sw128(c8, c, D);
-      *reinterpret_cast<uint4*>(sm + CB_BH + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-      *reinterpret_cast<uint4*>(sm + CB_BL + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-    }
-  };
-
-  if (warp == 0) {
-    tmem_alloc(&tmem_base_sh, 128);
-    tmem_relinquish();
-  }
-  if (tid == 0) {
-    mbar_init(&bar, 1);
-    fence_mbar_init();
-  }
-  load_loc(sa.sbuf + slot(0));                             // S_start,1
-  load_x(sa.xbuf + slot(1));
-  cp_async_wait_all();
-  __syncthreads();
-  store_b();
-  store_a();
-  fence_async_smem();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tb = tmem_base_sh;
-  uint32_t phase = 0;
-  bool ok = true;
-  const uint32_t idesc = idesc_bf16(128, 128, false, true);
-  for (int p = 1; p <= Ps - 2 && ok; ++p) {
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t ah = smem_u32(sm + CB_AH), al = smem_u32(sm + CB_AL);
-      const uint32_t bh = smem_u32(sm + CB_BH), bl = smem_u32(sm + CB_BL);
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        mma_ss(tb, desc_kmajor_sw128(ah, D, kk), desc_mnmajor_sw128(bh, D, kk), idesc, kk > 0);
-        mma_ss(tb, desc_kmajor_sw128(ah, D, kk), desc_mnmajor_sw128(bl, D, kk), idesc, 1);
-        mma_ss(tb, desc_kmajor_sw128(al, D, kk), desc_mnmajor_sw128(bh, D, kk), idesc, 1);
-      }
-      mma_commit(&bar);
-    }
-    __syncwarp();
-    // while the tensor cores work: Sloc_p -> loc (the B operand is already in
-    // smem), X_{p+1} -> registers
-    float* Sp = sa.sbuf + slot(p);
-    load_loc(Sp);
-    const bool more = p + 1 <= Ps - 2;
-    if (more) load_x(sa.xbuf + slot(p + 1));
-    const bool good = mbar_wait(&bar, phase, 1u << 22);
-    phase ^= 1u;
-    tc_fence_after();
-    cp_async_wait_all();
-    if (__syncthreads_or(!good)) { ok = false; break; }
-    // S_start,p+1 = X_p S_start,p + Sloc_p: row c from TMEM lane c
-    {
-      float* lr = loc + c * LOC_LD;
-#pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 16) {
-        uint32_t t[16];
-        tmem_ld16(tb + lane_base + c0, t);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e4 = 0; e4 < 4; ++e4) {
-          float4 l4 = *reinterpret_cast<float4*>(lr + c0 + 4 * e4);
-          l4.x += __uint_as_float(t[4 * e4]);
-          l4.y += __uint_as_float(t[4 * e4 + 1]);
-          l4.z += __uint_as_float(t[4 * e4 + 2]);
-          l4.w += __uint_as_float(t[4 * e4 + 3]);
-          *reinterpret_cast<float4*>(lr + c0 + 4 * e4) = l4;
-        }
-      }
-    }
-    tc_fence_before();
-    __syncthreads();
-    // coalesced store of S_start,p+1 into Sloc_p's slot; next operands
-#pragma unroll 8
-    for (int i = 0; i < D / 4; ++i) {
-      const int r = warp + 4 * i;
-      *reinterpret_cast<float4*>(Sp + (long long)r * D + 4 * lane) =
-          *reinterpret_cast<const float4*>(loc + r * LOC_LD + 4 * lane);
-    }
-    if (more) {
-      store_b();
-      store_a();
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-  }
-  if (!ok && tid == 0) mbar_wait(&bar, phase, 1u << 22);
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) {
-    tc_fence_after();
-    tmem_dealloc(tb, 128);
-  }
-}
 
 }  // namespace
 
@@ -1016,44 +795,18 @@ bool chunk_tc_supported(int dk, int dv, int in_dtype) {
 
 namespace {
 
-struct DeviceInfo {
-  bool init = false;
-  int sms = 148;
-  cudaMemPool_t pool = nullptr;
-};
-std::mutex g_dev_mu;
-DeviceInfo g_dev[64];
-
-// Per-device state: SM count, the kernel attributes and a private stream-ordered
-// memory pool for the segment scratch (it keeps its memory between calls, so a
-// steady stream of calls does not go back to the driver).
-DeviceInfo* device_info() {
+// Dynamic shared memory of the kernel, set once per device.
+bool set_attrs() {
+  static bool done[64] = {};
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lk(g_dev_mu);
-  DeviceInfo& d = g_dev[dev];
-  if (!d.init) {
-    cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (!done[dev]) {
     if (cudaFuncSetAttribute(kda_chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(kda_seg_combine_kernel,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kCombineSmem) != cudaSuccess)
-      return nullptr;
-    cudaMemPoolProps props = {};
-    props.allocType = cudaMemAllocationTypePinned;
-    props.location.type = cudaMemLocationTypeDevice;
-    props.location.id = dev;
-    if (cudaMemPoolCreate(&d.pool, &props) == cudaSuccess) {
-      uint64_t keep = UINT64_MAX;
-      cudaMemPoolSetAttribute(d.pool, cudaMemPoolAttrReleaseThreshold, &keep);
-    } else {
-      d.pool = nullptr;
-      (void)cudaGetLastError();
-    }
-    d.init = true;
+                             SMEM_BYTES) != cudaSuccess)
+      return false;
+    done[dev] = true;
   }
-  return &d;
+  return true;
 }
 
 // Chunks per segment (0: no split).  Cost model in units of one chunk step:
@@ -1083,23 +836,24 @@ int plan_segments(int B, int T, int H, bool varlen, int sms) {
 cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const float* g,
                             const float* beta, const float* h0, const int32_t* cu_seqlens,
                             void* out, float* hT, int B, int T, int H, cudaStream_t stream) {
-  DeviceInfo* di = device_info();
-  if (!di) return cudaErrorInvalidDevice;
+  int sms = 148;
+  cudaMemPool_t pool = nullptr;
+  if (!device_ctx(&sms, &pool) || !set_attrs()) return cudaErrorInvalidDevice;
   const bf16* qb = static_cast<const bf16*>(q);
   const bf16* kb = static_cast<const bf16*>(k);
   const bf16* vb = static_cast<const bf16*>(v);
   bf16* ob = static_cast<bf16*>(out);
 
   SegArgs sa{0, 1, 0, 0, nullptr, nullptr};
-  const int G = plan_segments(B, T, H, cu_seqlens != nullptr, di->sms);
+  const int G = plan_segments(B, T, H, cu_seqlens != nullptr, sms);
   void* scratch = nullptr;
   const long long nch_all = ((long long)T + C - 1) / C;
-  if (G > 0 && di->pool && (nch_all + G - 1) / G >= 2) {
+  if (G > 0 && pool && (nch_all + G - 1) / G >= 2) {
     const long long nch = nch_all;
     const int P = (int)((nch + G - 1) / G);
     const long long slots = cu_seqlens ? (long long)P + B : (long long)B * P;
     const size_t bytes = (size_t)2 * slots * H * D * D * sizeof(float);
-    if (cudaMallocFromPoolAsync(&scratch, bytes, di->pool, stream) == cudaSuccess) {
+    if (cudaMallocFromPoolAsync(&scratch, bytes, pool, stream) == cudaSuccess) {
       sa = SegArgs{G, P, 1, (int)slots, static_cast<float*>(scratch),
                    static_cast<float*>(scratch) + (size_t)slots * H * D * D};
     } else {
@@ -1115,13 +869,13 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const f
   }
   kda_chunk_tc_kernel<<<dim3(H, B, 2 * sa.P), NT, SMEM_BYTES, stream>>>(
       qb, kb, vb, g, beta, h0, cu_seqlens, ob, hT, T, H, sa);
-  kda_seg_combine_kernel<<<dim3(H, B), kCombineThreads, kCombineSmem, stream>>>(cu_seqlens, T,
-                                                                                H, sa);
+  cudaError_t ec = launch_seg_combine(cu_seqlens, B, T, H, sa, stream);
   sa.pass = 2;
   kda_chunk_tc_kernel<<<dim3(H, B, sa.P - 1), NT, SMEM_BYTES, stream>>>(
       qb, kb, vb, g, beta, h0, cu_seqlens, ob, hT, T, H, sa);
-  note_launches(3);
-  const cudaError_t e = cudaGetLastError();
+  note_launches(2);
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = ec;
   cudaFreeAsync(scratch, stream);
   return e;
 }
@@ -1136,10 +890,7 @@ int run_chunk_tc_static(const void* q, const void* k, const void* v, const float
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-      cudaFuncSetAttribute(kda_chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           SMEM_BYTES) != cudaSuccess ||
-      cudaFuncSetAttribute(kda_seg_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)kCombineSmem) != cudaSuccess) {
+      !set_attrs()) {
     (void)cudaGetLastError();
     return KDA_ERR_CUDA;
   }
@@ -1164,12 +915,11 @@ int run_chunk_tc_static(const void* q, const void* k, const void* v, const float
   } else {
     kda_chunk_tc_kernel<<<dim3(H, B, 2 * sa.P), NT, SMEM_BYTES, stream>>>(
         qb, kb, vb, g, beta, h0, cu_seqlens, ob, hT, T, H, sa);
-    kda_seg_combine_kernel<<<dim3(H, B), kCombineThreads, kCombineSmem, stream>>>(cu_seqlens,
-                                                                                  T, H, sa);
+    if (launch_seg_combine(cu_seqlens, B, T, H, sa, stream) != cudaSuccess) return KDA_ERR_CUDA;
     sa.pass = 2;
     kda_chunk_tc_kernel<<<dim3(H, B, sa.P - 1), NT, SMEM_BYTES, stream>>>(
         qb, kb, vb, g, beta, h0, cu_seqlens, ob, hT, T, H, sa);
-    note_launches(3);
+    note_launches(2);
   }
   if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
   return KDA_OK;
