@@ -275,11 +275,15 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   __syncthreads();
 
   uint32_t phase = 0;
+  // one warp polls the MMA barrier; the others sleep in the CTA barrier and
+  // leave the issue slots to the SM's other CTA
   auto mma_wait = [&]() -> bool {
-    const bool good = mbar_wait(&bar, phase, kWaitLimit);
+    bool good = true;
+    if (warp == 0) good = mbar_wait(&bar, phase, kWaitLimit);
     phase ^= 1u;
+    const bool ok = __syncthreads_or(!good) == 0;
     tc_fence_after();
-    return __syncthreads_or(!good) == 0;
+    return ok;
   };
   bool alive = true;
 
@@ -509,7 +513,7 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
 
   if (!alive && tid == 0) {
     atomicExch(&g_chunk_split_timeout, 1);
-    mbar_wait(&bar, phase, kWaitLimit);   // let an MMA still in flight finish
+    mbar_wait(&bar, phase ^ 1u, kWaitLimit);   // let an MMA still in flight finish
   }
   tc_fence_before();
   __syncthreads();
@@ -520,9 +524,14 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
 }
 
 // ============================================================================
-// State pass: one CTA per chain (sequence, head[, segment]).
+// State pass: one CTA per chain (sequence, head[, segment]), 512 threads.
+// Thread (wq, j) with j = 32 (warp % 4) + lane owns TMEM lane j, i.e. row j of
+// S^T, and the quarter wq = warp / 4 of every phase's columns.  Thread 0 issues
+// the MMAs and the record copies (two records ahead).
 // ============================================================================
-__global__ void __launch_bounds__(NT, 1)
+constexpr int NT_S = 512;
+
+__global__ void __launch_bounds__(NT_S, 1)
 kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
                       const int32_t* __restrict__ cu_seqlens, bf16* __restrict__ out, float* hT,
                       int T, int H, long long nslots, SegArgs sa) {
@@ -532,9 +541,9 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
   __shared__ uint64_t mbar;
   __shared__ uint32_t tmem_base_sh;
 
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = blockIdx.x, s = blockIdx.y;
-  const int wg = tid >> 7, j = tid & 127;
+  const int wq = warp >> 2, j = 32 * (warp & 3) + lane;
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
 
   long long row0, t_beg, t_end;
@@ -603,8 +612,9 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
     fence_mbar_init();
   }
   __syncthreads();
+  int issued = nch < 2 ? nch : 2;                    // thread 0: records requested
   if (tid == 0) {
-    for (int i = 0; i < 2 && i < nch; ++i) {
+    for (int i = 0; i < issued; ++i) {
       mbar_arrive_expect_tx(&full[i], REC_BYTES);
       bulk_g2s(sm + i * S_BUF, rec_ptr(i), REC_BYTES, &full[i]);
     }
@@ -613,11 +623,11 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = tmem_base_sh;
+  const uint32_t tl = tb + lane_base;
 
-  // ---- initial state: thread (wg, j) holds row j of S^T, columns [64 wg, 64 wg + 64)
-#pragma unroll 1
-  for (int cc = 0; cc < 64; cc += 32) {
-    const int c = 64 * wg + cc;
+  // ---- initial state: columns [32 wq, 32 wq + 32) of row j of S^T, and its bf16 copy
+  {
+    const int c = 32 * wq;
     uint32_t f0[16], f1[16], pk[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
@@ -632,11 +642,11 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
       pk[e] = pack_bf16(__uint_as_float(f0[2 * e]), __uint_as_float(f0[2 * e + 1]));
       pk[8 + e] = pack_bf16(__uint_as_float(f1[2 * e]), __uint_as_float(f1[2 * e + 1]));
     }
-    tmem_st16(tb + lane_base + ST_S + c, f0);
-    tmem_st16(tb + lane_base + ST_S + c + 16, f1);
-    tmem_st16(tb + lane_base + ST_SB + c / 2, pk);
+    tmem_st16(tl + ST_S + c, f0);
+    tmem_st16(tl + ST_S + c + 16, f1);
+    tmem_st16(tl + ST_SB + c / 2, pk);
+    tmem_wait_st();
   }
-  tmem_wait_st();
   bool good = nch == 0 || mbar_wait(&full[0], 0, kWaitLimit);
   tc_fence_before();
   bool alive = __syncthreads_or(!good) == 0;
@@ -644,7 +654,6 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
 
   uint32_t mphase = 0;
   int waited = alive && nch > 0 ? 1 : 0;             // records whose arrival has been seen
-  int issued = nch < 2 ? nch : 2;                    // records requested
 #pragma unroll 1
   for (int i = 0; i < nch && alive; ++i) {
     const int buf = i & 1;
@@ -671,19 +680,19 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
       mma_commit(&mbar);
     }
     __syncwarp();
-    // meanwhile S^T <- S^T Diag(exp(G_last)) (the MMA reads only the bf16 copy)
+    // meanwhile S^T <- S^T Diag(exp(G_last)), columns [32 wq, 32 wq + 32)
     {
-      const float* dec = reinterpret_cast<const float*>(rb + REC_DECAY) + 64 * wg;
-      uint32_t t[4][16];
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) tmem_ld16(tb + lane_base + ST_S + 64 * wg + 16 * q4, t[q4]);
+      const float* dec = reinterpret_cast<const float*>(rb + REC_DECAY) + 32 * wq;
+      uint32_t t[2][16];
+      tmem_ld16(tl + ST_S + 32 * wq, t[0]);
+      tmem_ld16(tl + ST_S + 32 * wq + 16, t[1]);
       tmem_wait_ld();
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
+      for (int q2 = 0; q2 < 2; ++q2) {
 #pragma unroll
         for (int e = 0; e < 16; ++e)
-          t[q4][e] = __float_as_uint(__uint_as_float(t[q4][e]) * dec[16 * q4 + e]);
-        tmem_st16(tb + lane_base + ST_S + 64 * wg + 16 * q4, t[q4]);
+          t[q2][e] = __float_as_uint(__uint_as_float(t[q2][e]) * dec[16 * q2 + e]);
+        tmem_st16(tl + ST_S + 32 * wq + 16 * q2, t[q2]);
       }
       tmem_wait_st();
     }
@@ -693,30 +702,27 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
     tc_fence_after();
     if (__syncthreads_or(!good)) { alive = false; break; }
 
-    // ---- Delta^T = U^T - P for tokens [32 wg, 32 wg + 32) -> bf16 TMEM
+    // ---- Delta^T = U^T - P for tokens [16 wq, 16 wq + 16) -> bf16 TMEM
     {
-      uint32_t tp[2][16];
-      tmem_ld16(tb + lane_base + ST_P + 32 * wg, tp[0]);
-      tmem_ld16(tb + lane_base + ST_P + 32 * wg + 16, tp[1]);
-      uint4 u[4];
+      uint32_t tp[16];
+      tmem_ld16(tl + ST_P + 16 * wq, tp);
+      uint4 u[2];
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4)
-        u[c4] = homog ? make_uint4(0u, 0u, 0u, 0u)
+      for (int c2 = 0; c2 < 2; ++c2)
+        u[c2] = homog ? make_uint4(0u, 0u, 0u, 0u)
                       : *reinterpret_cast<const uint4*>(
-                            rb + REC_U + j * 128 + ((((uint32_t)(4 * wg + c4)) ^ (j & 7u)) << 4));
+                            rb + REC_U + j * 128 + ((((uint32_t)(2 * wq + c2)) ^ (j & 7u)) << 4));
       tmem_wait_ld();
-      uint32_t dw[16];
+      uint32_t dw[8];
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        const uint32_t uw[4] = {u[c4].x, u[c4].y, u[c4].z, u[c4].w};
+      for (int c2 = 0; c2 < 2; ++c2) {
+        const uint32_t uw[4] = {u[c2].x, u[c2].y, u[c2].z, u[c2].w};
 #pragma unroll
-        for (int e2 = 0; e2 < 4; ++e2) {
-          const float p0 = __uint_as_float(tp[c4 >> 1][(c4 & 1) * 8 + 2 * e2]);
-          const float p1 = __uint_as_float(tp[c4 >> 1][(c4 & 1) * 8 + 2 * e2 + 1]);
-          dw[4 * c4 + e2] = pack_bf16(bf_lo(uw[e2]) - p0, bf_hi(uw[e2]) - p1);
-        }
+        for (int e2 = 0; e2 < 4; ++e2)
+          dw[4 * c2 + e2] = pack_bf16(bf_lo(uw[e2]) - __uint_as_float(tp[8 * c2 + 2 * e2]),
+                                      bf_hi(uw[e2]) - __uint_as_float(tp[8 * c2 + 2 * e2 + 1]));
       }
-      tmem_st16(tb + lane_base + ST_D + 16 * wg, dw);
+      tmem_st8(tl + ST_D + 8 * wq, dw);
       tmem_wait_st();
     }
     tc_fence_before();
@@ -740,45 +746,36 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
     if (__syncthreads_or(!good)) { alive = false; break; }
 
     // the record in this buffer is consumed: fetch record i + 2 into it
-    if (tid == 0 && i + 2 < nch) {
-      fence_async_smem();
-      mbar_arrive_expect_tx(&full[buf], REC_BYTES);
-      bulk_g2s(rb, rec_ptr(i + 2), REC_BYTES, &full[buf]);
-    }
-    if (i + 2 < nch) ++issued;
-
-    // ---- lower warpgroup: bf16 copy of the new state; upper: outputs to the tile
-    bf16* otile = reinterpret_cast<bf16*>(sm + S_OUT);
-    if (wg == 0) {
-#pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 64) {
-        uint32_t t[4][16], pk[2][16];
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) tmem_ld16(tb + lane_base + ST_S + c0 + 16 * q4, t[q4]);
-        tmem_wait_ld();
-#pragma unroll
-        for (int q2 = 0; q2 < 2; ++q2) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            pk[q2][e] = pack_bf16(__uint_as_float(t[2 * q2][2 * e]),
-                                  __uint_as_float(t[2 * q2][2 * e + 1]));
-            pk[q2][8 + e] = pack_bf16(__uint_as_float(t[2 * q2 + 1][2 * e]),
-                                      __uint_as_float(t[2 * q2 + 1][2 * e + 1]));
-          }
-          tmem_st16(tb + lane_base + ST_SB + c0 / 2 + 16 * q2, pk[q2]);
-        }
+    if (i + 2 < nch) {
+      if (tid == 0) {
+        fence_async_smem();
+        mbar_arrive_expect_tx(&full[buf], REC_BYTES);
+        bulk_g2s(rb, rec_ptr(i + 2), REC_BYTES, &full[buf]);
       }
-      tmem_wait_st();
-    } else if (outputs) {
-      uint32_t t[4][16];
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) tmem_ld16(tb + lane_base + ST_O + 16 * q4, t[q4]);
+      ++issued;
+    }
+
+    // ---- bf16 copy of the new state (columns [32 wq, +32)); O^T (tokens [16 wq, +16))
+    {
+      bf16* otile = reinterpret_cast<bf16*>(sm + S_OUT);
+      uint32_t t[2][16], to[16];
+      tmem_ld16(tl + ST_S + 32 * wq, t[0]);
+      tmem_ld16(tl + ST_S + 32 * wq + 16, t[1]);
+      if (outputs) tmem_ld16(tl + ST_O + 16 * wq, to);
       tmem_wait_ld();
+      uint32_t pk[16];
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4)
+      for (int e = 0; e < 8; ++e) {
+        pk[e] = pack_bf16(__uint_as_float(t[0][2 * e]), __uint_as_float(t[0][2 * e + 1]));
+        pk[8 + e] = pack_bf16(__uint_as_float(t[1][2 * e]), __uint_as_float(t[1][2 * e + 1]));
+      }
+      tmem_st16(tl + ST_SB + 16 * wq, pk);
+      if (outputs) {
 #pragma unroll
         for (int e = 0; e < 16; ++e)
-          otile[(16 * q4 + e) * D + j] = __float2bfloat16_rn(__uint_as_float(t[q4][e]));
+          otile[(16 * wq + e) * D + j] = __float2bfloat16_rn(__uint_as_float(to[e]));
+      }
+      tmem_wait_st();
     }
     tc_fence_before();
     good = true;
@@ -788,11 +785,11 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
     }
     if (__syncthreads_or(!good)) { alive = false; break; }
     tc_fence_after();
-    // upper warpgroup: coalesced 16-byte stores of the tile (overlap the next MMA)
-    if (wg == 1 && outputs) {
+    // coalesced 16-byte stores of the tile (overlap the next MMA)
+    if (outputs) {
 #pragma unroll
-      for (int it = 0; it < 8; ++it) {
-        const int idx = j + it * 128;
+      for (int it = 0; it < 2; ++it) {
+        const int idx = tid + it * NT_S;
         const int r = idx >> 4, ch = idx & 15;
         if (r < L) {
           const uint4 val = *reinterpret_cast<const uint4*>(sm + S_OUT + r * 256 + ch * 16);
@@ -804,19 +801,18 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
 
   // ---- final state
   if (alive && fin) {
-#pragma unroll 1
-    for (int c0 = 64 * wg; c0 < 64 * wg + 64; c0 += 16) {
-      uint32_t t[16];
-      tmem_ld16(tb + lane_base + ST_S + c0, t);
-      tmem_wait_ld();
+    uint32_t t[2][16];
+    tmem_ld16(tl + ST_S + 32 * wq, t[0]);
+    tmem_ld16(tl + ST_S + 32 * wq + 16, t[1]);
+    tmem_wait_ld();
 #pragma unroll
-      for (int e = 0; e < 16; ++e) fin[(long long)(c0 + e) * D + j] = __uint_as_float(t[e]);
-    }
+    for (int e = 0; e < 32; ++e)
+      fin[(long long)(32 * wq + e) * D + j] = __uint_as_float(t[e >> 4][e & 15]);
   }
   if (!alive && tid == 0) {
     atomicExch(&g_chunk_split_timeout, 1);
     // let the MMA and the copies still in flight finish before the CTA exits
-    mbar_wait(&mbar, mphase, kWaitLimit);
+    mbar_wait(&mbar, mphase ^ 1u, kWaitLimit);
     for (int r = waited; r < issued; ++r) mbar_wait(&full[r & 1], (r >> 1) & 1, kWaitLimit);
   }
   tc_fence_before();
@@ -915,16 +911,16 @@ cudaError_t launch_chunk_split(const void* q, const void* k, const void* v, cons
   }
   if (P == 0) {
     SegArgs sa{0, 1, 0, 0, nullptr, nullptr};
-    kda_state_pass_kernel<<<dim3(H, B, 1), NT, STATE_SMEM, stream>>>(rec, h0, cu_seqlens, ob, hT,
+    kda_state_pass_kernel<<<dim3(H, B, 1), NT_S, STATE_SMEM, stream>>>(rec, h0, cu_seqlens, ob, hT,
                                                                      T, H, nslots, sa);
     note_launches(1);
   } else {
     SegArgs sa{G, P, 1, (int)slots, segbuf, segbuf + (size_t)slots * H * D * D};
-    kda_state_pass_kernel<<<dim3(H, B, 2 * P), NT, STATE_SMEM, stream>>>(rec, h0, cu_seqlens, ob,
+    kda_state_pass_kernel<<<dim3(H, B, 2 * P), NT_S, STATE_SMEM, stream>>>(rec, h0, cu_seqlens, ob,
                                                                          hT, T, H, nslots, sa);
     const cudaError_t ec = launch_seg_combine(cu_seqlens, B, T, H, sa, stream);
     sa.pass = 2;
-    kda_state_pass_kernel<<<dim3(H, B, P - 1), NT, STATE_SMEM, stream>>>(rec, h0, cu_seqlens, ob,
+    kda_state_pass_kernel<<<dim3(H, B, P - 1), NT_S, STATE_SMEM, stream>>>(rec, h0, cu_seqlens, ob,
                                                                          hT, T, H, nslots, sa);
     note_launches(2);
     if (ec != cudaSuccess) e = ec;
