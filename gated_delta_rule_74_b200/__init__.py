@@ -42,6 +42,11 @@ class KdaError(RuntimeError):
         super().__init__(f"{fn} failed: {kda_status_string(status)} ({status})")
 
 
+def _check_status(rc: int, fn: str = "kda_timing") -> None:
+    if rc != 0:
+        raise KdaError(fn, rc)
+
+
 def library_path() -> str:
     return _SO
 
@@ -66,6 +71,13 @@ def lib() -> ctypes.CDLL:
         L.kda_version.restype = ctypes.c_int
         L.kda_launch_count.argtypes = []
         L.kda_launch_count.restype = ctypes.c_ulonglong
+        L.kda_timing_start.argtypes = []
+        L.kda_timing_start.restype = ctypes.c_int
+        L.kda_timing_stop.argtypes = []
+        L.kda_timing_stop.restype = ctypes.c_int
+        L.kda_timing_read.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_ulonglong),
+                                      ctypes.POINTER(ctypes.c_double)]
+        L.kda_timing_read.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -88,6 +100,29 @@ def kda_version() -> int:
 def kda_launch_count() -> int:
     """Kernels launched by libkda in this process so far."""
     return int(lib().kda_launch_count())
+
+
+KERNEL_KINDS = {"prep": 0, "state": 1, "combine": 2, "fused": 3, "simt": 4, "decode": 5}
+
+
+def kda_timing_start() -> None:
+    """Start bracketing every library kernel launch with CUDA events."""
+    _check_status(lib().kda_timing_start())
+
+
+def kda_timing_stop() -> None:
+    _check_status(lib().kda_timing_stop())
+
+
+def kda_timing_read() -> dict:
+    """{kind: (launches, total_ms)} since kda_timing_start(); waits for the events."""
+    res = {}
+    for name, kind in KERNEL_KINDS.items():
+        n = ctypes.c_ulonglong(0)
+        ms = ctypes.c_double(0.0)
+        _check_status(lib().kda_timing_read(kind, ctypes.byref(n), ctypes.byref(ms)))
+        res[name] = (int(n.value), float(ms.value))
+    return res
 
 
 def _ptr(t: Optional[torch.Tensor]):

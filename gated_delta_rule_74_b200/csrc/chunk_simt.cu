@@ -201,9 +201,10 @@ cudaError_t launch_t(const void* q, const void* k, const void* v, const float* g
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(dv / DVT, H, B);
-  kda_chunk_simt_kernel<Tin, DK><<<grid, NT, smem, stream>>>(
-      static_cast<const Tin*>(q), static_cast<const Tin*>(k), static_cast<const Tin*>(v), g,
-      beta, h0, cu, static_cast<Tin*>(out), hT, T, H, dv);
+  KDA_TIMED(KDA_KERNEL_SIMT, stream,
+            kda_chunk_simt_kernel<Tin, DK><<<grid, NT, smem, stream>>>(
+                static_cast<const Tin*>(q), static_cast<const Tin*>(k), static_cast<const Tin*>(v), g,
+                beta, h0, cu, static_cast<Tin*>(out), hT, T, H, dv));
   note_launches(1);
   return cudaGetLastError();
 }

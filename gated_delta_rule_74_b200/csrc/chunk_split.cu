@@ -905,23 +905,27 @@ cudaError_t launch_chunk_split(const void* q, const void* k, const void* v, cons
 
   cudaError_t e = cudaSuccess;
   if (nslots > 0) {
-    kda_chunk_prep_kernel<<<dim3((unsigned)nslots, H), NT, PREP_SMEM, stream>>>(
-        qb, kb, vb, g, beta, cu_seqlens, rec, B, T, H, nslots);
+    KDA_TIMED(KDA_KERNEL_PREP, stream,
+              kda_chunk_prep_kernel<<<dim3((unsigned)nslots, H), NT, PREP_SMEM, stream>>>(
+                  qb, kb, vb, g, beta, cu_seqlens, rec, B, T, H, nslots));
     note_launches(1);
   }
   if (P == 0) {
     SegArgs sa{0, 1, 0, 0, nullptr, nullptr};
-    kda_state_pass_kernel<<<dim3(H, B, 1), NT_S, STATE_SMEM, stream>>>(rec, h0, cu_seqlens, ob, hT,
-                                                                     T, H, nslots, sa);
+    KDA_TIMED(KDA_KERNEL_STATE, stream,
+              kda_state_pass_kernel<<<dim3(H, B, 1), NT_S, STATE_SMEM, stream>>>(rec, h0, cu_seqlens, ob, hT,
+                                                                               T, H, nslots, sa));
     note_launches(1);
   } else {
     SegArgs sa{G, P, 1, (int)slots, segbuf, segbuf + (size_t)slots * H * D * D};
-    kda_state_pass_kernel<<<dim3(H, B, 2 * P), NT_S, STATE_SMEM, stream>>>(rec, h0, cu_seqlens, ob,
-                                                                         hT, T, H, nslots, sa);
+    KDA_TIMED(KDA_KERNEL_STATE, stream,
+              kda_state_pass_kernel<<<dim3(H, B, 2 * P), NT_S, STATE_SMEM, stream>>>(rec, h0, cu_seqlens, ob,
+                                                                                   hT, T, H, nslots, sa));
     const cudaError_t ec = launch_seg_combine(cu_seqlens, B, T, H, sa, stream);
     sa.pass = 2;
-    kda_state_pass_kernel<<<dim3(H, B, P - 1), NT_S, STATE_SMEM, stream>>>(rec, h0, cu_seqlens, ob,
-                                                                         hT, T, H, nslots, sa);
+    KDA_TIMED(KDA_KERNEL_STATE, stream,
+              kda_state_pass_kernel<<<dim3(H, B, P - 1), NT_S, STATE_SMEM, stream>>>(rec, h0, cu_seqlens, ob,
+                                                                                   hT, T, H, nslots, sa));
     note_launches(2);
     if (ec != cudaSuccess) e = ec;
   }

@@ -862,17 +862,20 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const f
     }
   }
   if (sa.pass == 0) {
-    kda_chunk_tc_kernel<<<dim3(H, B, 1), NT, SMEM_BYTES, stream>>>(qb, kb, vb, g, beta, h0,
-                                                                  cu_seqlens, ob, hT, T, H, sa);
+    KDA_TIMED(KDA_KERNEL_FUSED, stream,
+              kda_chunk_tc_kernel<<<dim3(H, B, 1), NT, SMEM_BYTES, stream>>>(qb, kb, vb, g, beta, h0,
+                                                                            cu_seqlens, ob, hT, T, H, sa));
     note_launches(1);
     return cudaGetLastError();
   }
-  kda_chunk_tc_kernel<<<dim3(H, B, 2 * sa.P), NT, SMEM_BYTES, stream>>>(
-      qb, kb, vb, g, beta, h0, cu_seqlens, ob, hT, T, H, sa);
+  KDA_TIMED(KDA_KERNEL_FUSED, stream,
+            kda_chunk_tc_kernel<<<dim3(H, B, 2 * sa.P), NT, SMEM_BYTES, stream>>>(
+                qb, kb, vb, g, beta, h0, cu_seqlens, ob, hT, T, H, sa));
   cudaError_t ec = launch_seg_combine(cu_seqlens, B, T, H, sa, stream);
   sa.pass = 2;
-  kda_chunk_tc_kernel<<<dim3(H, B, sa.P - 1), NT, SMEM_BYTES, stream>>>(
-      qb, kb, vb, g, beta, h0, cu_seqlens, ob, hT, T, H, sa);
+  KDA_TIMED(KDA_KERNEL_FUSED, stream,
+            kda_chunk_tc_kernel<<<dim3(H, B, sa.P - 1), NT, SMEM_BYTES, stream>>>(
+                qb, kb, vb, g, beta, h0, cu_seqlens, ob, hT, T, H, sa));
   note_launches(2);
   cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess) e = ec;
@@ -909,16 +912,19 @@ int run_chunk_tc_static(const void* q, const void* k, const void* v, const float
     sa = SegArgs{G, P, 1, (int)slots, scratch, scratch + (size_t)slots * H * D * D};
   }
   if (sa.pass == 0) {
-    kda_chunk_tc_kernel<<<dim3(H, B, 1), NT, SMEM_BYTES, stream>>>(qb, kb, vb, g, beta, h0,
-                                                                  cu_seqlens, ob, hT, T, H, sa);
+    KDA_TIMED(KDA_KERNEL_FUSED, stream,
+              kda_chunk_tc_kernel<<<dim3(H, B, 1), NT, SMEM_BYTES, stream>>>(qb, kb, vb, g, beta, h0,
+                                                                            cu_seqlens, ob, hT, T, H, sa));
     note_launches(1);
   } else {
-    kda_chunk_tc_kernel<<<dim3(H, B, 2 * sa.P), NT, SMEM_BYTES, stream>>>(
-        qb, kb, vb, g, beta, h0, cu_seqlens, ob, hT, T, H, sa);
+    KDA_TIMED(KDA_KERNEL_FUSED, stream,
+              kda_chunk_tc_kernel<<<dim3(H, B, 2 * sa.P), NT, SMEM_BYTES, stream>>>(
+                  qb, kb, vb, g, beta, h0, cu_seqlens, ob, hT, T, H, sa));
     if (launch_seg_combine(cu_seqlens, B, T, H, sa, stream) != cudaSuccess) return KDA_ERR_CUDA;
     sa.pass = 2;
-    kda_chunk_tc_kernel<<<dim3(H, B, sa.P - 1), NT, SMEM_BYTES, stream>>>(
-        qb, kb, vb, g, beta, h0, cu_seqlens, ob, hT, T, H, sa);
+    KDA_TIMED(KDA_KERNEL_FUSED, stream,
+              kda_chunk_tc_kernel<<<dim3(H, B, sa.P - 1), NT, SMEM_BYTES, stream>>>(
+                  qb, kb, vb, g, beta, h0, cu_seqlens, ob, hT, T, H, sa));
     note_launches(2);
   }
   if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;

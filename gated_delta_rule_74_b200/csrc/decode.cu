@@ -122,9 +122,10 @@ cudaError_t launch_t(const void* q, const void* k, const void* v, const float* g
                      const float* beta, float* S, void* out, long long pairs,
                      cudaStream_t stream) {
   // pairs <= INT32_MAX by construction (N, H are ints and N*H is checked).
-  kda_decode_kernel<Tin, DK, DV><<<(unsigned)pairs, kThreads, 0, stream>>>(
-      static_cast<const Tin*>(q), static_cast<const Tin*>(k), static_cast<const Tin*>(v),
-      g, beta, S, static_cast<Tin*>(out));
+  KDA_TIMED(KDA_KERNEL_DECODE, stream,
+            kda_decode_kernel<Tin, DK, DV><<<(unsigned)pairs, kThreads, 0, stream>>>(
+                static_cast<const Tin*>(q), static_cast<const Tin*>(k), static_cast<const Tin*>(v),
+                g, beta, S, static_cast<Tin*>(out)));
   note_launches(1);
   return cudaGetLastError();
 }

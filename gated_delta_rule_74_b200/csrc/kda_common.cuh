@@ -21,6 +21,17 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 // Count of kernel launches made by the library (see kda_launch_count()).
 void note_launches(unsigned long long n);
 
+// Per-kernel timing (kda_timing_*): bracket one launch of kernel kind `kind`
+// on `stream`; timing_begin returns a handle (-1 when timing is off).
+int timing_begin(int kind, cudaStream_t stream);
+void timing_end(int handle, cudaStream_t stream);
+#define KDA_TIMED(kind, stream, ...)                  \
+  do {                                                \
+    const int kda_th_ = timing_begin(kind, stream);   \
+    __VA_ARGS__;                                      \
+    timing_end(kda_th_, stream);                      \
+  } while (0)
+
 // Launchers implemented in the kernel translation units.  Each returns a
 // cudaError_t from the launch (cudaSuccess when the launch was accepted).
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* g,

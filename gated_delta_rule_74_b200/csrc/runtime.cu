@@ -3,6 +3,7 @@
 // memory between calls (release threshold = everything), so a steady stream of
 // calls does not go back to the driver.
 #include <mutex>
+#include <vector>
 
 #include "kda_common.cuh"
 #include "segments.cuh"
@@ -47,3 +48,105 @@ bool device_ctx(int* sms, cudaMemPool_t* pool) {
 }
 
 }  // namespace kda
+
+// ---------------------------------------------------------------------------
+// Per-kernel timing (kda_timing_*): events around each launch while enabled.
+namespace kda {
+namespace {
+
+constexpr size_t kMaxTimed = 65536;
+struct TimedLaunch {
+  int kind;
+  cudaEvent_t a, b;
+};
+struct Timing {
+  std::mutex mu;
+  bool on = false;
+  std::vector<TimedLaunch> recs;
+  std::vector<cudaEvent_t> pool;      // events released by kda_timing_start / stop
+};
+Timing g_timing;
+
+cudaEvent_t take_event() {
+  cudaEvent_t e = nullptr;
+  if (!g_timing.pool.empty()) {
+    e = g_timing.pool.back();
+    g_timing.pool.pop_back();
+    return e;
+  }
+  if (cudaEventCreate(&e) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  return e;
+}
+void release_all() {
+  for (auto& r : g_timing.recs) {
+    g_timing.pool.push_back(r.a);
+    g_timing.pool.push_back(r.b);
+  }
+  g_timing.recs.clear();
+}
+
+}  // namespace
+
+int timing_begin(int kind, cudaStream_t stream) {
+  if (!g_timing.on) return -1;
+  std::lock_guard<std::mutex> lk(g_timing.mu);
+  if (!g_timing.on || g_timing.recs.size() >= kMaxTimed) return -1;
+  TimedLaunch t{kind, take_event(), take_event()};
+  if (!t.a || !t.b || cudaEventRecord(t.a, stream) != cudaSuccess) {
+    (void)cudaGetLastError();
+    if (t.a) g_timing.pool.push_back(t.a);
+    if (t.b) g_timing.pool.push_back(t.b);
+    return -1;
+  }
+  g_timing.recs.push_back(t);
+  return (int)g_timing.recs.size() - 1;
+}
+
+void timing_end(int handle, cudaStream_t stream) {
+  if (handle < 0) return;
+  std::lock_guard<std::mutex> lk(g_timing.mu);
+  if ((size_t)handle < g_timing.recs.size())
+    if (cudaEventRecord(g_timing.recs[handle].b, stream) != cudaSuccess) (void)cudaGetLastError();
+}
+
+}  // namespace kda
+
+extern "C" {
+
+int kda_timing_start(void) {
+  std::lock_guard<std::mutex> lk(kda::g_timing.mu);
+  kda::release_all();
+  kda::g_timing.on = true;
+  return KDA_OK;
+}
+
+int kda_timing_stop(void) {
+  std::lock_guard<std::mutex> lk(kda::g_timing.mu);
+  kda::g_timing.on = false;
+  return KDA_OK;
+}
+
+int kda_timing_read(int kind, unsigned long long* launches, double* total_ms) {
+  if (kind < 0 || kind >= KDA_KERNEL_KINDS || !launches || !total_ms) return KDA_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(kda::g_timing.mu);
+  unsigned long long n = 0;
+  double ms = 0.0;
+  for (auto& r : kda::g_timing.recs) {
+    if (r.kind != kind) continue;
+    float t = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return KDA_ERR_CUDA;
+    }
+    ++n;
+    ms += t;
+  }
+  *launches = n;
+  *total_ms = ms;
+  return KDA_OK;
+}
+
+}  // extern "C"

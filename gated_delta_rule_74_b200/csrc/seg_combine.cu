@@ -196,8 +196,9 @@ cudaError_t launch_seg_combine(const int32_t* cu_seqlens, int B, int T, int H, c
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  kda_seg_combine_kernel<<<dim3(H, B), kCombineThreads, kCombineSmem, stream>>>(cu_seqlens, T, H,
-                                                                                sa);
+  KDA_TIMED(KDA_KERNEL_COMBINE, stream,
+            kda_seg_combine_kernel<<<dim3(H, B), kCombineThreads, kCombineSmem, stream>>>(cu_seqlens, T, H,
+                                                                                          sa));
   note_launches(1);
   return cudaGetLastError();
 }

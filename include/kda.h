@@ -164,6 +164,31 @@ KDA_API int kda_version(void);
  * since it was loaded (all threads, all devices).  Diagnostic only. */
 KDA_API unsigned long long kda_launch_count(void);
 
+/* Per-kernel timing (diagnostic; this library's own facility, with no
+ * counterpart on the pages).  Between kda_timing_start() and
+ * kda_timing_stop(), every kernel the library launches is bracketed by two CUDA
+ * events recorded on the stream it is launched on (the events cost a few
+ * hundred nanoseconds of stream time each; nothing else changes).
+ * kda_timing_read(kind, ...) waits for the recorded events and returns the
+ * number of launches of that kernel kind and their summed duration in
+ * milliseconds since the last kda_timing_start().  At most 65536 launches are
+ * recorded; later ones are counted in kda_launch_count() only.  Process-wide,
+ * not thread-safe against concurrent start/stop.  Returns KDA_OK,
+ * KDA_ERR_INVALID_ARG for an unknown kind or null outputs, KDA_ERR_CUDA if an
+ * event could not be created or read. */
+typedef enum {
+  KDA_KERNEL_PREP = 0,          /* per-chunk prep of the split prefill            */
+  KDA_KERNEL_STATE = 1,         /* state pass of the split prefill                */
+  KDA_KERNEL_COMBINE = 2,       /* segment combine                                */
+  KDA_KERNEL_FUSED = 3,         /* single-kernel tensor-core prefill              */
+  KDA_KERNEL_SIMT = 4,          /* CUDA-core prefill (fp32, d = 64)               */
+  KDA_KERNEL_DECODE = 5,        /* decode step                                    */
+  KDA_KERNEL_KINDS = 6
+} kda_kernel_kind_t;
+KDA_API int kda_timing_start(void);
+KDA_API int kda_timing_stop(void);
+KDA_API int kda_timing_read(int kind, unsigned long long* launches, double* total_ms);
+
 #ifdef __cplusplus
 }
 #endif
