@@ -369,7 +369,44 @@ def _traffic(workload: str) -> dict:
         return {}
     if t.get("source_hash") != _source_hash():
         return {}
-    return t.get("workloads", {}).get(workload, {})
+    w = dict(t.get("workloads", {}).get(workload, {}))
+    w.pop("launches_captured", None)
+    return w
+
+
+def ingest_ncu(csv_path: str, workload: str) -> int:
+    """Write profiles/traffic.json from an ncu --csv launch list that holds
+    dram__bytes_read.sum and dram__bytes_write.sum per launch: the average DRAM
+    bytes per launch of each kernel kind, tagged with the hash of the kernel
+    sources it was taken on."""
+    import csv
+    rows = list(csv.reader(open(csv_path)))
+    hdr = next(i for i, r in enumerate(rows) if r and r[0] == "ID")
+    H = rows[hdr]
+    ki, mi, vi, ii = H.index("Kernel Name"), H.index("Metric Name"), H.index("Metric Value"), 0
+    per = {}
+    for r in rows[hdr + 1:]:
+        if len(r) <= vi or not r[mi].startswith("dram__bytes_"):
+            continue
+        kind = next((k for k, n in KERNEL_NAMES.items() if n in r[ki]), None)
+        if kind is None:
+            continue
+        per.setdefault(kind, {}).setdefault(r[ii], 0)
+        per[kind][r[ii]] += int(float(r[vi].replace(",", "")))
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(tpath) as f:
+            t = json.load(f)
+    except Exception:
+        t = {}
+    if t.get("source_hash") != _source_hash():
+        t = {"source_hash": _source_hash(), "workloads": {}}
+    t["workloads"][workload] = {k: sum(v.values()) / len(v) for k, v in per.items()}
+    t["workloads"][workload]["launches_captured"] = {k: len(v) for k, v in per.items()}
+    with open(tpath, "w") as f:
+        json.dump(t, f, indent=1)
+    print(json.dumps(t["workloads"][workload]))
+    return 0
 
 
 def _roofline(args, pf, hbm, tf_sust, peak_kind) -> dict:
@@ -482,7 +519,7 @@ def run_ours(args, world, rank, local):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="metric", choices=["metric", "cfg1", "cfg2", "cfg3"])
@@ -497,7 +534,11 @@ def main():
                     help="tokens of the workload the oracle processes per pass (0 = all)")
     ap.add_argument("--ref-seconds", type=float, default=10.0,
                     help="repeat oracle passes until this much time has passed")
+    ap.add_argument("--ingest-ncu", default="",
+                    help="write profiles/traffic.json from this ncu --csv launch list (no GPU run)")
     args = ap.parse_args()
+    if args.ingest_ncu:
+        return ingest_ncu(args.ingest_ncu, args.workload)
     args.warmup = max(args.warmup, 3)     # at least 3 untimed warm-up steps
     world, rank, local = _dist()
     if args.impl == "reference":
