@@ -334,7 +334,40 @@ def decode_leg(args, world, rank, dev, stream, barrier, clocks, hbm, peak_kind):
     dbytes = decode_bytes(dd["N"], dd["H"], dd["dk"], dd["dv"], 2)
     step_ms = dms / args.decode_steps
     gbs = dbytes / (step_ms / 1e3) / 1e9
-    return {"metric": "decode state GB/s vs HBM peak", "workload":
+    # fused multi-token decode: all 16 tokens of the config-4 workload in one launch
+    fused = None
+    if not args.no_fused_decode:
+        L = dspec.steps
+        dt = ki.make_decode(dspec, steps=L, seed=dspec.seed + 1000 * rank, N=args.decode_n or None)
+        tq = {n: dt[n].transpose(0, 1).contiguous().to(dev) for n in ("q", "k", "v", "g", "beta")}
+        del dt
+        tout = torch.empty(dd["N"], L, dd["H"], dd["dv"], dtype=q.dtype, device=dev)
+        for _ in range(3):
+            kda.kda_decode_tokens(tq["q"], tq["k"], tq["v"], tq["g"], tq["beta"], S, out=tout,
+                                  stream=stream)
+        torch.cuda.synchronize()
+        barrier()
+        nf = max(3, args.decode_steps // 8)
+        n1 = kda.kda_launch_count()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(nf):
+            kda.kda_decode_tokens(tq["q"], tq["k"], tq["v"], tq["g"], tq["beta"], S, out=tout,
+                                  stream=stream)
+        f1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        fl = kda.kda_launch_count() - n1
+        fms = _max_over_ranks(f0.elapsed_time(f1), world, dev) / nf
+        fbytes = dd["N"] * dd["H"] * (8 * dd["dk"] * dd["dv"] + L * ((2 * dd["dk"] + dd["dv"]) * 2
+                                                                   + 4 * dd["dk"] + 4 + dd["dv"] * 2))
+        fgbs = fbytes / (fms / 1e3) / 1e9
+        fused = {"call": "kda_decode_tokens", "tokens_per_launch_per_sequence": L,
+                 "ms_per_launch": fms, "tokens_per_s": dd["N"] * L * world * 1e3 / fms,
+                 "bytes_per_launch": fbytes, "gbs": fgbs, "frac_of_hbm_peak": fgbs / hbm,
+                 "speedup_vs_single_steps": (step_ms * L) / fms, "launches": fl}
+        del tq, tout
+    return {"metric": "decode state GB/s vs HBM peak", "fused_tokens": fused, "workload":
             f"cfg4 shape: N={dd['N']} H={dd['H']} dk=dv=128 bf16 q/k/v, fp32 state "
             f"{dd['N'] * dd['H'] * 65536 / 1e9:.2f} GB", "gbs": gbs,
             "frac_of_hbm_peak": gbs / hbm, "peak_gbs": hbm, "peak_kind": peak_kind,
@@ -525,6 +558,8 @@ def main():
     ap.add_argument("--workload", default="metric", choices=["metric", "cfg1", "cfg2", "cfg3"])
     ap.add_argument("--decode-steps", type=int, default=100)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-fused-decode", action="store_true",
+                    help="skip the multi-token decode (kda_decode_tokens) leg")
     ap.add_argument("--decode-only", action="store_true",
                     help="skip the prefill legs (for profiling the decode kernel)")
     ap.add_argument("--decode-n", type=int, default=0,

@@ -65,6 +65,8 @@ def lib() -> ctypes.CDLL:
         L.kda_chunk_fwd.restype = ctypes.c_int
         L.kda_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, vp, ip, ip, ip, ip, ip, vp]
         L.kda_decode_step.restype = ctypes.c_int
+        L.kda_decode_tokens.argtypes = [vp, vp, vp, fp, fp, fp, vp, ip, ip, ip, ip, ip, ip, vp]
+        L.kda_decode_tokens.restype = ctypes.c_int
         L.kda_status_string.argtypes = [ctypes.c_int]
         L.kda_status_string.restype = ctypes.c_char_p
         L.kda_version.argtypes = []
@@ -216,4 +218,34 @@ def kda_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.
                                _ptr(out), N, H, dk, dv, dt, _stream(stream))
     if rc != KDA_OK:
         raise KdaError("kda_decode_step", rc)
+    return out
+
+
+def kda_decode_tokens(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+                      beta: torch.Tensor, S: torch.Tensor, out: Optional[torch.Tensor] = None,
+                      stream=None) -> torch.Tensor:
+    """L consecutive KDA decode steps in one launch.  q, k [N,L,H,dk]; v [N,L,H,dv];
+    g [N,L,H,dk] f32; beta [N,L,H] f32; S [N,H,dk,dv] f32, updated in place (state
+    after the last token).  Returns out [N,L,H,dv]; identical to L kda_decode_step
+    calls."""
+    if q.dim() != 4:
+        raise ValueError("q must be [N, L, H, dk]")
+    N, L, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = _DTYPES.get(q.dtype)
+    if dt is None:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    _check("q", q)
+    _check("k", k, q.dtype, (N, L, H, dk))
+    _check("v", v, q.dtype, (N, L, H, dv))
+    _check("g", g, torch.float32, (N, L, H, dk))
+    _check("beta", beta, torch.float32, (N, L, H))
+    _check("S", S, torch.float32, (N, H, dk, dv))
+    if out is None:
+        out = torch.empty((N, L, H, dv), dtype=q.dtype, device=q.device)
+    _check("out", out, q.dtype, (N, L, H, dv))
+    rc = lib().kda_decode_tokens(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S),
+                                 _ptr(out), N, L, H, dk, dv, dt, _stream(stream))
+    if rc != KDA_OK:
+        raise KdaError("kda_decode_tokens", rc)
     return out

@@ -80,6 +80,20 @@ int kda_decode_step(const void* q, const void* k, const void* v, const float* g,
   return status_from(kda::launch_decode(q, k, v, g, beta, S, out, N, H, dk, dv, in_dtype, st));
 }
 
+int kda_decode_tokens(const void* q, const void* k, const void* v, const float* g,
+                      const float* beta, float* S, void* out, int N, int L, int H, int dk, int dv,
+                      int in_dtype, void* stream) {
+  if (N < 1 || L < 1 || H < 1) return KDA_ERR_INVALID_ARG;
+  if (in_dtype != KDA_BF16 && in_dtype != KDA_F32) return KDA_ERR_INVALID_ARG;
+  if (!pointers_ok({q, k, v, g, beta, S, out}, {})) return KDA_ERR_INVALID_ARG;
+  if (!head_ok(dk) || !head_ok(dv)) return KDA_ERR_UNSUPPORTED;
+  if ((long long)N * H > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
+  if ((long long)N * L * H * (dk > dv ? dk : dv) > (1LL << 40)) return KDA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return status_from(
+      kda::launch_decode_tokens(q, k, v, g, beta, S, out, N, L, H, dk, dv, in_dtype, st));
+}
+
 const char* kda_status_string(int status) {
   switch (status) {
     case KDA_OK: return "KDA_OK";

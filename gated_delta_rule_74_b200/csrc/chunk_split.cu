@@ -843,7 +843,7 @@ bool set_attrs() {
 // chunk step: pass A runs NH*(2P-3) chains, pass C NH*(P-1), each G chunks
 // long, in waves of one chain per SM; the combine costs kCombine steps per
 // segment.
-constexpr double kCombine = 12.0;
+constexpr double kCombine = 4.5;
 int plan_split(int B, int T, int H, bool varlen, int sms) {
   const long long NH = (long long)B * H;
   const long long nch = ((long long)T + C - 1) / C;

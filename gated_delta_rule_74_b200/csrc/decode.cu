@@ -102,9 +102,12 @@ kda_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
   float u[CPT];
 #pragma unroll
   for (int j = 0; j < CPT; ++j) {
-    float rt = 0.f, pt = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) { rt += s_r[w][col0 + j]; pt += s_p[w][col0 + j]; }
+    // pairwise tree ((0+1)+(2+3))+((4+5)+(6+7)) over the warps' partials
+    const int c = col0 + j;
+    const float rt = ((s_r[0][c] + s_r[1][c]) + (s_r[2][c] + s_r[3][c])) +
+                     ((s_r[4][c] + s_r[5][c]) + (s_r[6][c] + s_r[7][c]));
+    const float pt = ((s_p[0][c] + s_p[1][c]) + (s_p[2][c] + s_p[3][c])) +
+                     ((s_p[4][c] + s_p[5][c]) + (s_p[6][c] + s_p[7][c]));
     u[j] = b * (s_v[col0 + j] - rt);
     if (warp == 0) out[p * DV + col0 + j] = from_f32<Tin>(fmaf(u[j], kq, pt));
   }
@@ -115,6 +118,138 @@ kda_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     for (int j = 0; j < CPT; ++j) x[i][j] = fmaf(kc, u[j], x[i][j]);
     vstore(Sp + (warp * ROWS + i) * DV + col0, x[i]);
   }
+}
+
+// Multi-token decode: L consecutive tokens per (n, h) with the state held in
+// registers, so S is read once and written once for all L tokens.  Warp w owns
+// columns [w DV/8, (w+1) DV/8) of S over all rows, lane (g, c) = (lane / 4,
+// lane % 4) the rows [g DK/8, (g+1) DK/8) and DV/32 of those columns, so the
+// two reductions over dk are a per-lane partial followed by an xor-shuffle tree
+// over the 8 row groups inside the warp: no barrier per token.  The single
+// step above forms its partials over the same rows in the same order and adds
+// the 8 partials in the same pairwise tree, so L tokens here give bit-for-bit
+// the results of L single steps.  Token vectors are staged in shared memory 16
+// tokens at a time (one barrier pair per 16 tokens).
+constexpr int kTile = 16;
+
+template <typename Tin, int DK, int DV>
+__global__ void __launch_bounds__(kThreads, 2)
+kda_decode_tokens_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                         const Tin* __restrict__ v, const float* __restrict__ g,
+                         const float* __restrict__ beta, float* __restrict__ S,
+                         Tin* __restrict__ out, int L, int H) {
+  constexpr int R = DK / 8;           // rows per lane (one row group)
+  constexpr int CPL = DV / 32;        // columns per lane
+  // (a = exp(g), k, q) of row c = grp R + i at [t][i][grp]: the 8 row groups a
+  // warp reads together are consecutive 16-byte words (no bank conflicts)
+  __shared__ float4 s_akq[kTile][R][8];
+  __shared__ float s_v[kTile][DV];
+  __shared__ float s_b[kTile], s_kq[kTile];
+
+  const long long p = blockIdx.x;     // flat (n, h)
+  const long long n = p / H;
+  const int h = (int)(p - n * H);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int grp = lane >> 2;
+  const int col0 = warp * (DV / 8) + (lane & 3) * CPL;
+  float* Sp = S + p * (long long)(DK * DV);
+
+  float x[R][CPL];
+#pragma unroll
+  for (int i = 0; i < R; ++i) vload(Sp + (grp * R + i) * DV + col0, x[i]);
+
+#pragma unroll 1
+  for (int t0 = 0; t0 < L; t0 += kTile) {
+    const int nt = min(kTile, L - t0);
+    __syncthreads();                  // the previous tile's vectors are no longer read
+    for (int e = tid; e < nt * DK; e += kThreads) {
+      const int t = e / DK, c = e - t * DK;
+      const long long row = (n * L + t0 + t) * H + h;
+      s_akq[t][c % R][c / R] =
+          make_float4(expf(g[row * DK + c]), to_f32(k[row * DK + c]), to_f32(q[row * DK + c]), 0.f);
+    }
+    for (int e = tid; e < nt * DV; e += kThreads) {
+      const int t = e / DV, j = e - t * DV;
+      s_v[t][j] = to_f32(v[((n * L + t0 + t) * H + h) * DV + j]);
+    }
+    if (tid < nt) s_b[tid] = beta[(n * L + t0 + tid) * H + h];
+    __syncthreads();
+    // k . q per token, each by one warp, in the single step's order
+    for (int t = warp; t < nt; t += kWarps) {
+      float a = 0.f;
+      for (int c = lane; c < DK; c += 32) a = fmaf(s_akq[t][c % R][c / R].y, s_akq[t][c % R][c / R].z, a);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+      if (lane == 0) s_kq[t] = a;
+    }
+    __syncthreads();
+#pragma unroll 1
+    for (int t = 0; t < nt; ++t) {
+      float r[CPL], pq[CPL];
+#pragma unroll
+      for (int j = 0; j < CPL; ++j) { r[j] = 0.f; pq[j] = 0.f; }
+#pragma unroll
+      for (int i = 0; i < R; ++i) {
+        const float4 akq = s_akq[t][i][grp];
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) {
+          x[i][j] *= akq.x;
+          r[j] = fmaf(x[i][j], akq.y, r[j]);
+          pq[j] = fmaf(x[i][j], akq.z, pq[j]);
+        }
+      }
+      // pairwise tree over the 8 row groups (lanes 4 apart hold neighbouring groups)
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) {
+          r[j] += __shfl_xor_sync(0xffffffffu, r[j], o);
+          pq[j] += __shfl_xor_sync(0xffffffffu, pq[j], o);
+        }
+      }
+      const float b = s_b[t], kq = s_kq[t];
+      float u[CPL];
+#pragma unroll
+      for (int j = 0; j < CPL; ++j) {
+        u[j] = b * (s_v[t][col0 + j] - r[j]);
+        if (grp == 0)
+          out[((n * L + t0 + t) * H + h) * DV + col0 + j] = from_f32<Tin>(fmaf(u[j], kq, pq[j]));
+      }
+#pragma unroll
+      for (int i = 0; i < R; ++i) {
+        const float kc = s_akq[t][i][grp].y;
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) x[i][j] = fmaf(kc, u[j], x[i][j]);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < R; ++i) vstore(Sp + (grp * R + i) * DV + col0, x[i]);
+}
+
+template <typename Tin, int DK, int DV>
+cudaError_t launch_tokens_t(const void* q, const void* k, const void* v, const float* g,
+                            const float* beta, float* S, void* out, long long pairs, int L, int H,
+                            cudaStream_t stream) {
+  KDA_TIMED(KDA_KERNEL_DECODE, stream,
+            kda_decode_tokens_kernel<Tin, DK, DV><<<(unsigned)pairs, kThreads, 0, stream>>>(
+                static_cast<const Tin*>(q), static_cast<const Tin*>(k), static_cast<const Tin*>(v),
+                g, beta, S, static_cast<Tin*>(out), L, H));
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+template <typename Tin>
+cudaError_t launch_tokens_dtype(const void* q, const void* k, const void* v, const float* g,
+                                const float* beta, float* S, void* out, long long pairs, int L,
+                                int H, int dk, int dv, cudaStream_t stream) {
+  if (dk == 128 && dv == 128)
+    return launch_tokens_t<Tin, 128, 128>(q, k, v, g, beta, S, out, pairs, L, H, stream);
+  if (dk == 128 && dv == 64)
+    return launch_tokens_t<Tin, 128, 64>(q, k, v, g, beta, S, out, pairs, L, H, stream);
+  if (dk == 64 && dv == 128)
+    return launch_tokens_t<Tin, 64, 128>(q, k, v, g, beta, S, out, pairs, L, H, stream);
+  return launch_tokens_t<Tin, 64, 64>(q, k, v, g, beta, S, out, pairs, L, H, stream);
 }
 
 template <typename Tin, int DK, int DV>
@@ -141,6 +276,16 @@ cudaError_t launch_dtype(const void* q, const void* k, const void* v, const floa
 }
 
 }  // namespace
+
+cudaError_t launch_decode_tokens(const void* q, const void* k, const void* v, const float* g,
+                                 const float* beta, float* S, void* out, int N, int L, int H,
+                                 int dk, int dv, int in_dtype, cudaStream_t stream) {
+  const long long pairs = (long long)N * H;
+  if (in_dtype == KDA_BF16)
+    return launch_tokens_dtype<__nv_bfloat16>(q, k, v, g, beta, S, out, pairs, L, H, dk, dv,
+                                              stream);
+  return launch_tokens_dtype<float>(q, k, v, g, beta, S, out, pairs, L, H, dk, dv, stream);
+}
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* g,
                           const float* beta, float* S, void* out, int N, int H, int dk,

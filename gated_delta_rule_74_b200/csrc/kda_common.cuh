@@ -38,6 +38,10 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, const flo
                           const float* beta, float* S, void* out, int N, int H, int dk,
                           int dv, int in_dtype, cudaStream_t stream);
 
+cudaError_t launch_decode_tokens(const void* q, const void* k, const void* v, const float* g,
+                                 const float* beta, float* S, void* out, int N, int L, int H,
+                                 int dk, int dv, int in_dtype, cudaStream_t stream);
+
 cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const float* g,
                               const float* beta, const float* h0, const int32_t* cu_seqlens,
                               void* out, float* hT, int B, int T, int H, int dk, int dv,

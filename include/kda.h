@@ -123,6 +123,28 @@ KDA_API int kda_decode_step(const void* q, const void* k, const void* v,
                     int N, int H, int dk, int dv, int in_dtype, void* stream);
 
 /*
+ * kda_decode_tokens -- L consecutive recurrent steps for N independent
+ * sequences in one launch (multi-token decode, e.g. checking L drafted tokens).
+ *
+ * Passage: as for kda_decode_step (miniKimiK3 model card, "Kimi Delta
+ * Attention" bullet; Kimi-K3-Tiny-L13 card, serving paragraph: decode is bound
+ * by the KDA state pool).  The pages give no multi-token interface; this one
+ * applies, per (n, h), exactly the update of kda_decode_step to tokens
+ * 0 .. L-1 in order, with the same arithmetic, so its results are bit-for-bit
+ * those of L successive kda_decode_step calls -- but S is read and written
+ * once for all L tokens instead of once per token.
+ *     q, k, g [N, L, H, dk]   v, out [N, L, H, dv]   beta [N, L, H]
+ *     S [N, H, dk, dv] fp32, in place (the state after token L-1)
+ * out must not alias S or any input.  N, L, H >= 1.
+ *
+ * Returns KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED or KDA_ERR_CUDA.
+ */
+KDA_API int kda_decode_tokens(const void* q, const void* k, const void* v,
+                              const float* g, const float* beta, float* S, void* out,
+                              int N, int L, int H, int dk, int dv, int in_dtype,
+                              void* stream);
+
+/*
  * kda_chunk_fwd_noalloc -- kda_chunk_fwd for callers that cannot allocate.
  *
  * The pages have no counterpart: this is a deployment variant.  Some callers

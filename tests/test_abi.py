@@ -72,3 +72,17 @@ def test_binding_rejects_cpu_tensors(L):
     x = torch.zeros(1, 4, 1, 64)
     with pytest.raises(ValueError):
         kda.kda_chunk_fwd(x, x, x, x, torch.zeros(1, 4, 1))
+
+
+def _tokens(L, q=P, k=P, v=P, g=P, beta=P, S=P, out=P, N=1, Lt=4, H=1, dk=64, dv=64, dt=0):
+    return L.kda_decode_tokens(q, k, v, g, beta, S, out, N, Lt, H, dk, dv, dt, None)
+
+
+@pytest.mark.parametrize("bad", [dict(q=None), dict(g=None), dict(S=None), dict(out=P + 4),
+                                 dict(N=0), dict(Lt=0), dict(Lt=-3), dict(H=0), dict(dt=3)])
+def test_decode_tokens_rejects_invalid(L, bad):
+    assert _tokens(L, **bad) == kda.KDA_ERR_INVALID_ARG
+
+
+def test_decode_tokens_rejects_unsupported_heads(L):
+    assert _tokens(L, dv=80) == kda.KDA_ERR_UNSUPPORTED
