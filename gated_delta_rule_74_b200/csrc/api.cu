@@ -60,7 +60,7 @@ int kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (kda::chunk_split_supported(dk, dv, in_dtype))
     return status_from(kda::launch_chunk_split(q, k, v, g, beta, h0, cu_seqlens, out, hT, B, T,
-                                               H, st));
+                                               H, dk, dv, st));
   if (kda::chunk_tc_supported(dk, dv, in_dtype))
     return status_from(kda::launch_chunk_tc(q, k, v, g, beta, h0, cu_seqlens, out, hT, B, T, H,
                                             st));

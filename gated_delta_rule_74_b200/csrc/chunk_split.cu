@@ -66,10 +66,10 @@ constexpr uint32_t REC_QW = 0;          // [Qbar^T | W^T]: MN-major SW128, N = 1
                                         // 16 KB apart), K = dk
 constexpr uint32_t REC_KA = 32768;      // [Kend^T ; Aqk]: K-major SW128, 192 rows x 64 tokens
 constexpr uint32_t REC_AQK = REC_KA + 16384;
-constexpr uint32_t REC_U = 57344;       // U^T [dv][64 tokens] bf16: 128-byte rows, 16-byte
-                                        // chunks XOR-swizzled with (row % 8)
-constexpr uint32_t REC_DECAY = 73728;   // exp(G_last) per key channel, fp32 [dk]
-constexpr uint32_t REC_BYTES = 74240;
+constexpr uint32_t REC_U = 57344;       // U^T [dv][64 tokens] fp32: 256-byte rows, 16-byte
+                                        // chunks XOR-swizzled with (row % 16)
+constexpr uint32_t REC_DECAY = 90112;   // exp(G_last) per key channel, fp32 [dk]
+constexpr uint32_t REC_BYTES = 90624;
 
 // ---- prep kernel: shared memory (from a 1024-aligned base) and TMEM
 constexpr uint32_t Q_V = 0;             // V: MN-major SW128 A operand of U^T (M = value, K = token)
@@ -92,7 +92,7 @@ constexpr uint32_t PT_U = 64;           // U^T [128 x 64]
 constexpr uint32_t kPrepTmemCols = 256;
 
 // ---- state pass: shared memory and TMEM
-constexpr uint32_t S_BUF = 74752;       // record buffer stride (two buffers)
+constexpr uint32_t S_BUF = 91136;       // record buffer stride (two buffers)
 constexpr uint32_t S_OUT = 2 * S_BUF;   // output tile [64 tokens][128] bf16
 constexpr uint32_t STATE_SMEM = S_OUT + 16384 + 1024;
 // [S^T | O^T] and [O^T | P] are each the accumulator of one MMA, so O^T sits
@@ -124,7 +124,8 @@ __global__ void __launch_bounds__(NT, 2)
 kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
                       const bf16* __restrict__ v, const float* __restrict__ g,
                       const float* __restrict__ beta, const int32_t* __restrict__ cu_seqlens,
-                      uint8_t* __restrict__ rec, int B, int T, int H, long long nslots) {
+                      uint8_t* __restrict__ rec, int B, int T, int H, int dk, int dv,
+                      long long nslots) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   __shared__ uint64_t bar;
@@ -166,8 +167,9 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   for (int it = 0; it < 4; ++it) {
     const int idx = tid + it * NT;
     const int r = idx >> 4, ch = idx & 15;
-    const long long e = ((rbase + min(r, L - 1)) * H + h) * D + ch * 8;
-    cp_async16(sm + Q_V + chunk_mnmajor_sw128(ch, r, C), v + e, r < L ? 16u : 0u);
+    const long long e = ((rbase + min(r, L - 1)) * H + h) * dv + min(ch * 8, dv - 8);
+    cp_async16(sm + Q_V + chunk_mnmajor_sw128(ch, r, C), v + e,
+               (r < L && ch * 8 < dv) ? 16u : 0u);
   }
   cp_async_commit();
   if (tid < C) s_beta[tid] = tid < L ? beta[(rbase + tid) * H + h] : 0.f;
@@ -187,8 +189,8 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
 #pragma unroll
   for (int e = 0; e < 16; ++e) {
     const int r = 16 * a + e;
-    if (r < L) {
-      const long long idx = ((rbase + r) * H + h) * D + c0;
+    if (r < L && c0 < dk) {
+      const long long idx = ((rbase + r) * H + h) * dk + c0;
       gq[e] = __ldg(reinterpret_cast<const float2*>(g + idx));
       kw[e] = __ldg(reinterpret_cast<const unsigned int*>(k + idx));
       qw[e] = __ldg(reinterpret_cast<const unsigned int*>(q + idx));
@@ -491,23 +493,31 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   }
 
   if (alive) {
-    // ---- P5: W^T (lower warpgroup) and U^T (upper) -> bf16 record images
+    // ---- P5: W^T (lower warpgroup) -> bf16 record image; U^T (upper) -> fp32
+    // record rows (Delta = U - W S is formed in fp32 by the state pass)
     const int j = tid & 127;
     uint32_t t[4][16];
     const uint32_t col = tid < 128 ? PT_W : PT_U;
 #pragma unroll
     for (int q4 = 0; q4 < 4; ++q4) tmem_ld16(tb + lane_base + col + 16 * q4, t[q4]);
     tmem_wait_ld();
+    if (tid < 128) {
 #pragma unroll
-    for (int g8 = 0; g8 < 8; ++g8) {
-      const uint32_t* f = t[g8 >> 1] + 8 * (g8 & 1);
-      const uint4 val = make_uint4(pack_bf16(__uint_as_float(f[0]), __uint_as_float(f[1])),
-                                   pack_bf16(__uint_as_float(f[2]), __uint_as_float(f[3])),
-                                   pack_bf16(__uint_as_float(f[4]), __uint_as_float(f[5])),
-                                   pack_bf16(__uint_as_float(f[6]), __uint_as_float(f[7])));
-      const uint32_t o = tid < 128 ? REC_QW + 16384 + chunk_mnmajor_sw128(g8, j, D)
-                                   : REC_U + j * 128 + (((uint32_t)g8 ^ (j & 7u)) << 4);
-      *reinterpret_cast<uint4*>(rc + o) = val;
+      for (int g8 = 0; g8 < 8; ++g8) {
+        const uint32_t* f = t[g8 >> 1] + 8 * (g8 & 1);
+        const uint4 val = make_uint4(pack_bf16(__uint_as_float(f[0]), __uint_as_float(f[1])),
+                                     pack_bf16(__uint_as_float(f[2]), __uint_as_float(f[3])),
+                                     pack_bf16(__uint_as_float(f[4]), __uint_as_float(f[5])),
+                                     pack_bf16(__uint_as_float(f[6]), __uint_as_float(f[7])));
+        *reinterpret_cast<uint4*>(rc + REC_QW + 16384 + chunk_mnmajor_sw128(g8, j, D)) = val;
+      }
+    } else {
+#pragma unroll
+      for (int c4 = 0; c4 < 16; ++c4) {
+        const uint32_t* f = t[c4 >> 2] + 4 * (c4 & 3);
+        *reinterpret_cast<uint4*>(rc + REC_U + j * 256 + (((uint32_t)c4 ^ (j & 15u)) << 4)) =
+            make_uint4(f[0], f[1], f[2], f[3]);
+      }
     }
   }
 
@@ -534,7 +544,7 @@ constexpr int NT_S = 512;
 __global__ void __launch_bounds__(NT_S, 1)
 kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
                       const int32_t* __restrict__ cu_seqlens, bf16* __restrict__ out, float* hT,
-                      int T, int H, long long nslots, SegArgs sa) {
+                      int T, int H, int dk, int dv, long long nslots, SegArgs sa) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   __shared__ uint64_t full[2];
@@ -550,7 +560,7 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
   seq_range(cu_seqlens, s, T, row0, t_beg, t_end);
   const long long seq_t0 = t_beg;
   // what this chain computes: a token range, where its state starts, where it ends
-  const long long hoff = ((long long)s * H + h) * D * D;
+  const long long hoff = ((long long)s * H + h) * dk * dv;
   const float* init = h0 ? h0 + hoff : nullptr;   // nullptr: zero state
   bool init_identity = false;
   float* fin = hT ? hT + hoff : nullptr;          // nullptr: final state not kept
@@ -631,8 +641,8 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
     uint32_t f0[16], f1[16], pk[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
-      float x0 = init ? init[(long long)(c + e) * D + j] : 0.f;
-      float x1 = init ? init[(long long)(c + 16 + e) * D + j] : 0.f;
+      float x0 = init && c + e < dk && j < dv ? init[(long long)(c + e) * dv + j] : 0.f;
+      float x1 = init && c + 16 + e < dk && j < dv ? init[(long long)(c + 16 + e) * dv + j] : 0.f;
       if (init_identity) { x0 = (c + e == j) ? 1.f : 0.f; x1 = (c + 16 + e == j) ? 1.f : 0.f; }
       f0[e] = __float_as_uint(x0);
       f1[e] = __float_as_uint(x1);
@@ -706,21 +716,20 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
     {
       uint32_t tp[16];
       tmem_ld16(tl + ST_P + 16 * wq, tp);
-      uint4 u[2];
+      float4 u[4];
 #pragma unroll
-      for (int c2 = 0; c2 < 2; ++c2)
-        u[c2] = homog ? make_uint4(0u, 0u, 0u, 0u)
-                      : *reinterpret_cast<const uint4*>(
-                            rb + REC_U + j * 128 + ((((uint32_t)(2 * wq + c2)) ^ (j & 7u)) << 4));
+      for (int c4 = 0; c4 < 4; ++c4)
+        u[c4] = homog ? make_float4(0.f, 0.f, 0.f, 0.f)
+                      : *reinterpret_cast<const float4*>(
+                            rb + REC_U + j * 256 + ((((uint32_t)(4 * wq + c4)) ^ (j & 15u)) << 4));
       tmem_wait_ld();
       uint32_t dw[8];
 #pragma unroll
-      for (int c2 = 0; c2 < 2; ++c2) {
-        const uint32_t uw[4] = {u[c2].x, u[c2].y, u[c2].z, u[c2].w};
-#pragma unroll
-        for (int e2 = 0; e2 < 4; ++e2)
-          dw[4 * c2 + e2] = pack_bf16(bf_lo(uw[e2]) - __uint_as_float(tp[8 * c2 + 2 * e2]),
-                                      bf_hi(uw[e2]) - __uint_as_float(tp[8 * c2 + 2 * e2 + 1]));
+      for (int c4 = 0; c4 < 4; ++c4) {
+        dw[2 * c4] = pack_bf16(u[c4].x - __uint_as_float(tp[4 * c4]),
+                               u[c4].y - __uint_as_float(tp[4 * c4 + 1]));
+        dw[2 * c4 + 1] = pack_bf16(u[c4].z - __uint_as_float(tp[4 * c4 + 2]),
+                                   u[c4].w - __uint_as_float(tp[4 * c4 + 3]));
       }
       tmem_st8(tl + ST_D + 8 * wq, dw);
       tmem_wait_st();
@@ -791,9 +800,9 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
       for (int it = 0; it < 2; ++it) {
         const int idx = tid + it * NT_S;
         const int r = idx >> 4, ch = idx & 15;
-        if (r < L) {
+        if (r < L && ch * 8 < dv) {
           const uint4 val = *reinterpret_cast<const uint4*>(sm + S_OUT + r * 256 + ch * 16);
-          *reinterpret_cast<uint4*>(out + ((row0 + t0 + r) * H + h) * D + ch * 8) = val;
+          *reinterpret_cast<uint4*>(out + ((row0 + t0 + r) * H + h) * dv + ch * 8) = val;
         }
       }
     }
@@ -806,8 +815,11 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
     tmem_ld16(tl + ST_S + 32 * wq + 16, t[1]);
     tmem_wait_ld();
 #pragma unroll
-    for (int e = 0; e < 32; ++e)
-      fin[(long long)(32 * wq + e) * D + j] = __uint_as_float(t[e >> 4][e & 15]);
+    if (j < dv) {
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        if (32 * wq + e < dk) fin[(long long)(32 * wq + e) * dv + j] = __uint_as_float(t[e >> 4][e & 15]);
+    }
   }
   if (!alive && tid == 0) {
     atomicExch(&g_chunk_split_timeout, 1);
@@ -867,12 +879,13 @@ int plan_split(int B, int T, int H, bool varlen, int sms) {
 }  // namespace
 
 bool chunk_split_supported(int dk, int dv, int in_dtype) {
-  return in_dtype == KDA_BF16 && dk == D && dv == D;
+  return in_dtype == KDA_BF16 && (dk == 64 || dk == D) && (dv == 64 || dv == D);
 }
 
 cudaError_t launch_chunk_split(const void* q, const void* k, const void* v, const float* g,
                                const float* beta, const float* h0, const int32_t* cu_seqlens,
-                               void* out, float* hT, int B, int T, int H, cudaStream_t stream) {
+                               void* out, float* hT, int B, int T, int H, int dk, int dv,
+                               cudaStream_t stream) {
   int sms = 148;
   cudaMemPool_t pool = nullptr;
   if (!device_ctx(&sms, &pool) || !set_attrs()) return cudaErrorInvalidDevice;
@@ -907,25 +920,25 @@ cudaError_t launch_chunk_split(const void* q, const void* k, const void* v, cons
   if (nslots > 0) {
     KDA_TIMED(KDA_KERNEL_PREP, stream,
               kda_chunk_prep_kernel<<<dim3((unsigned)nslots, H), NT, PREP_SMEM, stream>>>(
-                  qb, kb, vb, g, beta, cu_seqlens, rec, B, T, H, nslots));
+                  qb, kb, vb, g, beta, cu_seqlens, rec, B, T, H, dk, dv, nslots));
     note_launches(1);
   }
   if (P == 0) {
     SegArgs sa{0, 1, 0, 0, nullptr, nullptr};
     KDA_TIMED(KDA_KERNEL_STATE, stream,
               kda_state_pass_kernel<<<dim3(H, B, 1), NT_S, STATE_SMEM, stream>>>(rec, h0, cu_seqlens, ob, hT,
-                                                                               T, H, nslots, sa));
+                                                                               T, H, dk, dv, nslots, sa));
     note_launches(1);
   } else {
     SegArgs sa{G, P, 1, (int)slots, segbuf, segbuf + (size_t)slots * H * D * D};
     KDA_TIMED(KDA_KERNEL_STATE, stream,
               kda_state_pass_kernel<<<dim3(H, B, 2 * P), NT_S, STATE_SMEM, stream>>>(rec, h0, cu_seqlens, ob,
-                                                                                   hT, T, H, nslots, sa));
+                                                                                   hT, T, H, dk, dv, nslots, sa));
     const cudaError_t ec = launch_seg_combine(cu_seqlens, B, T, H, sa, stream);
     sa.pass = 2;
     KDA_TIMED(KDA_KERNEL_STATE, stream,
               kda_state_pass_kernel<<<dim3(H, B, P - 1), NT_S, STATE_SMEM, stream>>>(rec, h0, cu_seqlens, ob,
-                                                                                   hT, T, H, nslots, sa));
+                                                                                   hT, T, H, dk, dv, nslots, sa));
     note_launches(2);
     if (ec != cudaSuccess) e = ec;
   }

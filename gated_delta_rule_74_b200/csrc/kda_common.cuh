@@ -54,11 +54,13 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const f
                             void* out, float* hT, int B, int T, int H, cudaStream_t stream);
 
 // Tensor-core prefill split into a parallel per-chunk kernel and a state pass
-// (bf16, dk = dv = 128); its scratch comes from the library's memory pool.
+// (bf16, dk, dv in {64, 128}: 64-wide heads run zero-padded to 128); its
+// scratch comes from the library's memory pool.
 bool chunk_split_supported(int dk, int dv, int in_dtype);
 cudaError_t launch_chunk_split(const void* q, const void* k, const void* v, const float* g,
                                const float* beta, const float* h0, const int32_t* cu_seqlens,
-                               void* out, float* hT, int B, int T, int H, cudaStream_t stream);
+                               void* out, float* hT, int B, int T, int H, int dk, int dv,
+                               cudaStream_t stream);
 
 // The tensor-core prefill on caller-provided scratch (allocates nothing).
 int run_chunk_tc_static(const void* q, const void* k, const void* v, const float* g,
