@@ -814,8 +814,25 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
     tmem_ld16(tl + ST_S + 32 * wq, t[0]);
     tmem_ld16(tl + ST_S + 32 * wq + 16, t[1]);
     tmem_wait_ld();
+    if (init_identity) {
+      // a transition X_p: bf16 hi / lo images for the segment combine (MN-major
+      // SW128 A operand, M = row of X, K = column; TMEM lane j holds column j of X)
+      uint8_t* xb = reinterpret_cast<uint8_t*>(fin);
 #pragma unroll
-    if (j < dv) {
+      for (int c8 = 0; c8 < 4; ++c8) {
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float x0 = __uint_as_float(t[c8 >> 1][(c8 & 1) * 8 + 2 * e]);
+          const float x1 = __uint_as_float(t[c8 >> 1][(c8 & 1) * 8 + 2 * e + 1]);
+          hw[e] = pack_bf16(x0, x1);
+          lw[e] = pack_bf16(x0 - bf_lo(hw[e]), x1 - bf_hi(hw[e]));
+        }
+        const uint32_t o = chunk_mnmajor_sw128((uint32_t)(4 * wq + c8), (uint32_t)j, D);
+        *reinterpret_cast<uint4*>(xb + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4*>(xb + 32768 + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      }
+    } else if (j < dv) {
 #pragma unroll
       for (int e = 0; e < 32; ++e)
         if (32 * wq + e < dk) fin[(long long)(32 * wq + e) * dv + j] = __uint_as_float(t[e >> 4][e & 15]);
@@ -855,7 +872,7 @@ bool set_attrs() {
 // chunk step: pass A runs NH*(2P-3) chains, pass C NH*(P-1), each G chunks
 // long, in waves of one chain per SM; the combine costs kCombine steps per
 // segment.
-constexpr double kCombine = 4.5;
+constexpr double kCombine = 2.5;
 int plan_split(int B, int T, int H, bool varlen, int sms) {
   const long long NH = (long long)B * H;
   const long long nch = ((long long)T + C - 1) / C;
@@ -934,7 +951,7 @@ cudaError_t launch_chunk_split(const void* q, const void* k, const void* v, cons
     KDA_TIMED(KDA_KERNEL_STATE, stream,
               kda_state_pass_kernel<<<dim3(H, B, 2 * P), NT_S, STATE_SMEM, stream>>>(rec, h0, cu_seqlens, ob,
                                                                                    hT, T, H, dk, dv, nslots, sa));
-    const cudaError_t ec = launch_seg_combine(cu_seqlens, B, T, H, sa, stream);
+    const cudaError_t ec = launch_seg_combine_img(cu_seqlens, B, T, H, dk, dv, sa, stream);
     sa.pass = 2;
     KDA_TIMED(KDA_KERNEL_STATE, stream,
               kda_state_pass_kernel<<<dim3(H, B, P - 1), NT_S, STATE_SMEM, stream>>>(rec, h0, cu_seqlens, ob,

@@ -85,7 +85,12 @@ __host__ __forceinline__ long long chunk_slots(int B, int T, bool varlen) {
 bool device_ctx(int* sms, cudaMemPool_t* pool);
 
 // Segment combine (one launch): S_start,p+1 = X_p S_start,p + Sloc_p in place.
+// launch_seg_combine: X_p and the states as fp32 [128][128] (single-kernel prefill);
+// launch_seg_combine_img: X_p as bf16 hi/lo MMA operand images, states as fp32
+// [dk][dv] rows (split prefill).
 cudaError_t launch_seg_combine(const int32_t* cu_seqlens, int B, int T, int H, const SegArgs& sa,
                                cudaStream_t stream);
+cudaError_t launch_seg_combine_img(const int32_t* cu_seqlens, int B, int T, int H, int dk, int dv,
+                                   const SegArgs& sa, cudaStream_t stream);
 
 }  // namespace kda
