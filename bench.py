@@ -304,6 +304,55 @@ def prefill_leg(args, world, rank, dev, stream, barrier, clocks):
                      "steps": e2e_steps})
 
 
+def grouped_leg(args, world, rank, dev, stream, barrier, hbm, G=64):
+    """The headline prefill with one decay value per group of G key channels
+    (the decay-granularity variant): K timed calls on three resident input sets."""
+    import torch
+
+    import gated_delta_rule_74_b200 as kda
+    import kda_inputs as ki
+
+    spec = ki.PREFILL_SPECS[args.workload]
+    sets = []
+    for i in range(3):
+        x = ki.make_prefill(spec, seed=spec.seed + 1000 * rank + 500 + i)
+        d = {n: (t.to(dev) if isinstance(t, torch.Tensor) else t) for n, t in x.items()}
+        d["g"] = d["g"][..., ::G].contiguous()
+        d["out"] = torch.empty_like(d["v"])
+        d["hT"] = torch.empty(x["B"], x["H"], x["dk"], x["dv"], device=dev)
+        sets.append(d)
+    x0 = sets[0]
+    if x0["dk"] % G:
+        return None
+    rows = x0["T"] if x0["cu_seqlens"] is not None else x0["B"] * x0["T"]
+    s_in = 2 if x0["dtype"] == "bf16" else 4
+    H, dk, dv = x0["H"], x0["dk"], x0["dv"]
+    bytes_call = rows * H * ((2 * dk + dv) * s_in + 4 * (dk // G) + 4 + dv * s_in) + \
+        x0["B"] * H * 4 * dk * dv * (int(x0["h0"] is not None) + 1)
+
+    def call(i):
+        d = sets[i % 3]
+        kda.kda_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], h0=d["h0"],
+                          cu_seqlens=d["cu_seqlens"], out=d["out"], hT=d["hT"], stream=stream)
+
+    for i in range(args.warmup):
+        call(i)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        call(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = _max_over_ranks(e0.elapsed_time(e1), world, dev) / args.steps
+    gbs = bytes_call / (ms / 1e3) / 1e9
+    return {"call": f"kda_chunk_fwd_grouped (G={G})", "decay_group": G,
+            "tokens_per_s": rows * world / (ms / 1e3), "ms_per_call": ms,
+            "algorithmic_bytes_per_call": bytes_call, "gbs": gbs, "frac_of_hbm_peak": gbs / hbm}
+
+
 def decode_leg(args, world, rank, dev, stream, barrier, clocks, hbm, peak_kind):
     """K timed kda_decode_step calls on the config-4 shape (state in HBM)."""
     import torch
@@ -513,6 +562,9 @@ def run_ours(args, world, rank, local):
     pf = None
     if not args.decode_only:
         pf = prefill_leg(args, world, rank, dev, stream, barrier, clocks)
+    grp = None
+    if not args.decode_only and not args.no_grouped:
+        grp = grouped_leg(args, world, rank, dev, stream, barrier, hbm)
     dec = None
     if not args.no_decode:
         dec = decode_leg(args, world, rank, dev, stream, barrier, clocks, hbm, peak_kind)
@@ -540,6 +592,7 @@ def run_ours(args, world, rank, local):
         "data": "synthetic (seeded random inputs shaped like the pages' models)",
         "config": _config(args, pf["x0"], world),
         "roofline": roof,
+        "prefill_decay_g64": grp,
         "decode": dec, "e2e": pf["e2e"], "gpu_launches": pf["launches"],
         "clocks": pf["clocks"], "cpu_baseline": cpu,
     }
@@ -558,6 +611,8 @@ def main():
     ap.add_argument("--workload", default="metric", choices=["metric", "cfg1", "cfg2", "cfg3"])
     ap.add_argument("--decode-steps", type=int, default=100)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-grouped", action="store_true",
+                    help="skip the grouped-decay (G = 64) prefill leg")
     ap.add_argument("--no-fused-decode", action="store_true",
                     help="skip the multi-token decode (kda_decode_tokens) leg")
     ap.add_argument("--decode-only", action="store_true",

@@ -67,6 +67,10 @@ def lib() -> ctypes.CDLL:
         L.kda_decode_step.restype = ctypes.c_int
         L.kda_decode_tokens.argtypes = [vp, vp, vp, fp, fp, fp, vp, ip, ip, ip, ip, ip, ip, vp]
         L.kda_decode_tokens.restype = ctypes.c_int
+        L.kda_decode_tokens_grouped.argtypes = [vp, vp, vp, fp, fp, fp, vp] + [ip] * 7 + [vp]
+        L.kda_decode_tokens_grouped.restype = ctypes.c_int
+        L.kda_chunk_fwd_grouped.argtypes = [vp, vp, vp, fp, fp, fp, vp, vp, fp] + [ip] * 7 + [vp]
+        L.kda_chunk_fwd_grouped.restype = ctypes.c_int
         L.kda_status_string.argtypes = [ctypes.c_int]
         L.kda_status_string.restype = ctypes.c_char_p
         L.kda_version.argtypes = []
@@ -127,6 +131,14 @@ def kda_timing_read() -> dict:
     return res
 
 
+def _decay_group(g: torch.Tensor, dk: int) -> int:
+    """Channels per decay value implied by g's last dimension."""
+    n = g.shape[-1]
+    if n < 1 or dk % n != 0 or (dk // n) & (dk // n - 1):
+        raise ValueError(f"g's last dimension {n} must be dk / G with G a power of two")
+    return dk // n
+
+
 def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
@@ -153,10 +165,11 @@ def kda_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Te
                   cu_seqlens: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
                   hT: Optional[torch.Tensor] = None, output_final_state: bool = True,
                   stream=None):
-    """KDA prefill (chunked form).  q, k [B,T,H,dk]; v [B,T,H,dv]; g [B,T,H,dk] f32;
-    beta [B,T,H] f32; h0 [Nseq,H,dk,dv] f32 or None; cu_seqlens int32 [Nseq+1] on
-    the device, or None.  Returns (out, hT) (hT None if output_final_state is
-    False and no hT buffer was given)."""
+    """KDA prefill (chunked form).  q, k [B,T,H,dk]; v [B,T,H,dv]; g [B,T,H,dk] f32
+    (or [B,T,H,dk/G] for one decay per group of G key channels, G a power of two:
+    kda_chunk_fwd_grouped); beta [B,T,H] f32; h0 [Nseq,H,dk,dv] f32 or None;
+    cu_seqlens int32 [Nseq+1] on the device, or None.  Returns (out, hT) (hT None
+    if output_final_state is False and no hT buffer was given)."""
     if q.dim() != 4:
         raise ValueError("q must be [B, T, H, dk]")
     Bt, T, H, dk = q.shape
@@ -167,7 +180,8 @@ def kda_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Te
     _check("q", q)
     _check("k", k, q.dtype, (Bt, T, H, dk))
     _check("v", v, q.dtype, (Bt, T, H, dv))
-    _check("g", g, torch.float32, (Bt, T, H, dk))
+    G = _decay_group(g, dk)
+    _check("g", g, torch.float32, (Bt, T, H, dk // G))
     _check("beta", beta, torch.float32, (Bt, T, H))
     if cu_seqlens is not None:
         _check("cu_seqlens", cu_seqlens, torch.int32)
@@ -185,9 +199,14 @@ def kda_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Te
         hT = torch.empty((nseq, H, dk, dv), dtype=torch.float32, device=q.device)
     if hT is not None:
         _check("hT", hT, torch.float32, (nseq, H, dk, dv))
-    rc = lib().kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
-                             _ptr(cu_seqlens), _ptr(out), _ptr(hT),
-                             nseq, T, H, dk, dv, dt, _stream(stream))
+    if G == 1:
+        rc = lib().kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
+                                 _ptr(cu_seqlens), _ptr(out), _ptr(hT),
+                                 nseq, T, H, dk, dv, dt, _stream(stream))
+    else:
+        rc = lib().kda_chunk_fwd_grouped(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                         _ptr(h0), _ptr(cu_seqlens), _ptr(out), _ptr(hT),
+                                         nseq, T, H, dk, dv, G, dt, _stream(stream))
     if rc != KDA_OK:
         raise KdaError("kda_chunk_fwd", rc)
     return out, hT
@@ -238,14 +257,20 @@ def kda_decode_tokens(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torc
     _check("q", q)
     _check("k", k, q.dtype, (N, L, H, dk))
     _check("v", v, q.dtype, (N, L, H, dv))
-    _check("g", g, torch.float32, (N, L, H, dk))
+    G = _decay_group(g, dk)
+    _check("g", g, torch.float32, (N, L, H, dk // G))
     _check("beta", beta, torch.float32, (N, L, H))
     _check("S", S, torch.float32, (N, H, dk, dv))
     if out is None:
         out = torch.empty((N, L, H, dv), dtype=q.dtype, device=q.device)
     _check("out", out, q.dtype, (N, L, H, dv))
-    rc = lib().kda_decode_tokens(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S),
-                                 _ptr(out), N, L, H, dk, dv, dt, _stream(stream))
+    if G == 1:
+        rc = lib().kda_decode_tokens(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S),
+                                     _ptr(out), N, L, H, dk, dv, dt, _stream(stream))
+    else:
+        rc = lib().kda_decode_tokens_grouped(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                             _ptr(S), _ptr(out), N, L, H, dk, dv, G, dt,
+                                             _stream(stream))
     if rc != KDA_OK:
         raise KdaError("kda_decode_tokens", rc)
     return out

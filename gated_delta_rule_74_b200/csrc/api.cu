@@ -36,14 +36,19 @@ bool pointers_ok(std::initializer_list<const void*> required,
   return true;
 }
 
-}  // namespace
 
-extern "C" {
+// log2 of a decay group size: 0..log2(dk) for a power of two dividing dk, else -1
+int group_shift(int g_group, int dk) {
+  if (g_group < 1 || g_group > dk || (g_group & (g_group - 1)) != 0) return -1;
+  int sh = 0;
+  while ((1 << sh) < g_group) ++sh;
+  return sh;
+}
 
-int kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
-                  const float* beta, const float* h0, const int32_t* cu_seqlens, void* out,
-                  float* hT, int B, int T, int H, int dk, int dv, int in_dtype,
-                  void* stream) {
+int chunk_fwd_impl(const void* q, const void* k, const void* v, const float* g,
+                   const float* beta, const float* h0, const int32_t* cu_seqlens, void* out,
+                   float* hT, int B, int T, int H, int dk, int dv, int gsh, int in_dtype,
+                   void* stream) {
   if (B < 1 || T < 0 || H < 1) return KDA_ERR_INVALID_ARG;
   if (in_dtype != KDA_BF16 && in_dtype != KDA_F32) return KDA_ERR_INVALID_ARG;
   const long long rows = cu_seqlens ? (long long)T : (long long)B * T;
@@ -54,18 +59,51 @@ int kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
     if (!pointers_ok({}, {q, k, v, g, beta, out, h0, hT, cu_seqlens})) return KDA_ERR_INVALID_ARG;
   }
   if (!head_ok(dk) || !head_ok(dv)) return KDA_ERR_UNSUPPORTED;
+  if (gsh < 0) return KDA_ERR_INVALID_ARG;
   // element counts must fit the kernels' 64-bit indexing and the grid limits
   if (rows * H * (long long)(dk > dv ? dk : dv) > (1LL << 40)) return KDA_ERR_INVALID_ARG;
   if ((long long)B > 65535LL || H > 65535) return KDA_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (kda::chunk_split_supported(dk, dv, in_dtype))
     return status_from(kda::launch_chunk_split(q, k, v, g, beta, h0, cu_seqlens, out, hT, B, T,
-                                               H, dk, dv, st));
-  if (kda::chunk_tc_supported(dk, dv, in_dtype))
-    return status_from(kda::launch_chunk_tc(q, k, v, g, beta, h0, cu_seqlens, out, hT, B, T, H,
-                                            st));
+                                               H, dk, dv, gsh, st));
   return status_from(kda::launch_chunk_simt(q, k, v, g, beta, h0, cu_seqlens, out, hT, B, T,
-                                            H, dk, dv, in_dtype, st));
+                                            H, dk, dv, in_dtype, gsh, st));
+}
+
+int decode_tokens_impl(const void* q, const void* k, const void* v, const float* g,
+                       const float* beta, float* S, void* out, int N, int L, int H, int dk,
+                       int dv, int gsh, int in_dtype, void* stream) {
+  if (N < 1 || L < 1 || H < 1) return KDA_ERR_INVALID_ARG;
+  if (in_dtype != KDA_BF16 && in_dtype != KDA_F32) return KDA_ERR_INVALID_ARG;
+  if (!pointers_ok({q, k, v, g, beta, S, out}, {})) return KDA_ERR_INVALID_ARG;
+  if (!head_ok(dk) || !head_ok(dv)) return KDA_ERR_UNSUPPORTED;
+  if (gsh < 0) return KDA_ERR_INVALID_ARG;
+  if ((long long)N * H > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
+  if ((long long)N * L * H * (dk > dv ? dk : dv) > (1LL << 40)) return KDA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return status_from(
+      kda::launch_decode_tokens(q, k, v, g, beta, S, out, N, L, H, dk, dv, in_dtype, gsh, st));
+}
+
+}  // namespace
+
+extern "C" {
+
+int kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
+                  const float* beta, const float* h0, const int32_t* cu_seqlens, void* out,
+                  float* hT, int B, int T, int H, int dk, int dv, int in_dtype,
+                  void* stream) {
+  return chunk_fwd_impl(q, k, v, g, beta, h0, cu_seqlens, out, hT, B, T, H, dk, dv, 0, in_dtype,
+                        stream);
+}
+
+int kda_chunk_fwd_grouped(const void* q, const void* k, const void* v, const float* g,
+                          const float* beta, const float* h0, const int32_t* cu_seqlens,
+                          void* out, float* hT, int B, int T, int H, int dk, int dv, int g_group,
+                          int in_dtype, void* stream) {
+  return chunk_fwd_impl(q, k, v, g, beta, h0, cu_seqlens, out, hT, B, T, H, dk, dv,
+                        group_shift(g_group, dk), in_dtype, stream);
 }
 
 int kda_decode_step(const void* q, const void* k, const void* v, const float* g,
@@ -83,15 +121,14 @@ int kda_decode_step(const void* q, const void* k, const void* v, const float* g,
 int kda_decode_tokens(const void* q, const void* k, const void* v, const float* g,
                       const float* beta, float* S, void* out, int N, int L, int H, int dk, int dv,
                       int in_dtype, void* stream) {
-  if (N < 1 || L < 1 || H < 1) return KDA_ERR_INVALID_ARG;
-  if (in_dtype != KDA_BF16 && in_dtype != KDA_F32) return KDA_ERR_INVALID_ARG;
-  if (!pointers_ok({q, k, v, g, beta, S, out}, {})) return KDA_ERR_INVALID_ARG;
-  if (!head_ok(dk) || !head_ok(dv)) return KDA_ERR_UNSUPPORTED;
-  if ((long long)N * H > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
-  if ((long long)N * L * H * (dk > dv ? dk : dv) > (1LL << 40)) return KDA_ERR_INVALID_ARG;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return status_from(
-      kda::launch_decode_tokens(q, k, v, g, beta, S, out, N, L, H, dk, dv, in_dtype, st));
+  return decode_tokens_impl(q, k, v, g, beta, S, out, N, L, H, dk, dv, 0, in_dtype, stream);
+}
+
+int kda_decode_tokens_grouped(const void* q, const void* k, const void* v, const float* g,
+                              const float* beta, float* S, void* out, int N, int L, int H, int dk,
+                              int dv, int g_group, int in_dtype, void* stream) {
+  return decode_tokens_impl(q, k, v, g, beta, S, out, N, L, H, dk, dv, group_shift(g_group, dk),
+                            in_dtype, stream);
 }
 
 const char* kda_status_string(int status) {

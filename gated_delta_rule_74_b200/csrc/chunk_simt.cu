@@ -51,7 +51,7 @@ kda_chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                       const Tin* __restrict__ v, const float* __restrict__ g,
                       const float* __restrict__ beta, const float* h0,
                       const int32_t* __restrict__ cu_seqlens, Tin* __restrict__ out,
-                      float* hT, int T, int H, int dv) {
+                      float* hT, int T, int H, int dv, int gsh) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   SimtSmem<DK>& sm = *reinterpret_cast<SimtSmem<DK>*>(smem_raw);
   constexpr int LD = SimtSmem<DK>::LD;
@@ -88,7 +88,7 @@ kda_chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
         const long long tok = ((row0 + t0 + r) * H + h);
         kv = to_f32(k[tok * DK + c]);
         qv = to_f32(q[tok * DK + c]);
-        gv = g[tok * DK + c];
+        gv = g[tok * (DK >> gsh) + (c >> gsh)];
       }
       sm.k[r * LD + c] = kv; sm.q[r * LD + c] = qv; sm.G[r * LD + c] = gv;
     }
@@ -195,7 +195,7 @@ kda_chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
 template <typename Tin, int DK>
 cudaError_t launch_t(const void* q, const void* k, const void* v, const float* g,
                      const float* beta, const float* h0, const int32_t* cu, void* out,
-                     float* hT, int B, int T, int H, int dv, cudaStream_t stream) {
+                     float* hT, int B, int T, int H, int dv, int gsh, cudaStream_t stream) {
   const size_t smem = sizeof(SimtSmem<DK>);
   cudaError_t e = cudaFuncSetAttribute(kda_chunk_simt_kernel<Tin, DK>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -204,7 +204,7 @@ cudaError_t launch_t(const void* q, const void* k, const void* v, const float* g
   KDA_TIMED(KDA_KERNEL_SIMT, stream,
             kda_chunk_simt_kernel<Tin, DK><<<grid, NT, smem, stream>>>(
                 static_cast<const Tin*>(q), static_cast<const Tin*>(k), static_cast<const Tin*>(v), g,
-                beta, h0, cu, static_cast<Tin*>(out), hT, T, H, dv));
+                beta, h0, cu, static_cast<Tin*>(out), hT, T, H, dv, gsh));
   note_launches(1);
   return cudaGetLastError();
 }
@@ -214,15 +214,15 @@ cudaError_t launch_t(const void* q, const void* k, const void* v, const float* g
 cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const float* g,
                               const float* beta, const float* h0, const int32_t* cu_seqlens,
                               void* out, float* hT, int B, int T, int H, int dk, int dv,
-                              int in_dtype, cudaStream_t stream) {
+                              int in_dtype, int gsh, cudaStream_t stream) {
   if (in_dtype == KDA_BF16) {
     if (dk == 128)
-      return launch_t<__nv_bfloat16, 128>(q, k, v, g, beta, h0, cu_seqlens, out, hT, B, T, H, dv, stream);
-    return launch_t<__nv_bfloat16, 64>(q, k, v, g, beta, h0, cu_seqlens, out, hT, B, T, H, dv, stream);
+      return launch_t<__nv_bfloat16, 128>(q, k, v, g, beta, h0, cu_seqlens, out, hT, B, T, H, dv, gsh, stream);
+    return launch_t<__nv_bfloat16, 64>(q, k, v, g, beta, h0, cu_seqlens, out, hT, B, T, H, dv, gsh, stream);
   }
   if (dk == 128)
-    return launch_t<float, 128>(q, k, v, g, beta, h0, cu_seqlens, out, hT, B, T, H, dv, stream);
-  return launch_t<float, 64>(q, k, v, g, beta, h0, cu_seqlens, out, hT, B, T, H, dv, stream);
+    return launch_t<float, 128>(q, k, v, g, beta, h0, cu_seqlens, out, hT, B, T, H, dv, gsh, stream);
+  return launch_t<float, 64>(q, k, v, g, beta, h0, cu_seqlens, out, hT, B, T, H, dv, gsh, stream);
 }
 
 }  // namespace kda

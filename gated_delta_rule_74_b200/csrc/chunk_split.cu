@@ -124,7 +124,7 @@ __global__ void __launch_bounds__(NT, 2)
 kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
                       const bf16* __restrict__ v, const float* __restrict__ g,
                       const float* __restrict__ beta, const int32_t* __restrict__ cu_seqlens,
-                      uint8_t* __restrict__ rec, int B, int T, int H, int dk, int dv,
+                      uint8_t* __restrict__ rec, int B, int T, int H, int dk, int dv, int gsh,
                       long long nslots) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
@@ -191,7 +191,12 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     const int r = 16 * a + e;
     if (r < L && c0 < dk) {
       const long long idx = ((rbase + r) * H + h) * dk + c0;
-      gq[e] = __ldg(reinterpret_cast<const float2*>(g + idx));
+      if (gsh == 0) {
+        gq[e] = __ldg(reinterpret_cast<const float2*>(g + idx));
+      } else {                                   // one decay per group of 2^gsh channels
+        const float gg = __ldg(g + ((rbase + r) * H + h) * (dk >> gsh) + (c0 >> gsh));
+        gq[e] = make_float2(gg, gg);
+      }
       kw[e] = __ldg(reinterpret_cast<const unsigned int*>(k + idx));
       qw[e] = __ldg(reinterpret_cast<const unsigned int*>(q + idx));
     } else {
@@ -902,7 +907,7 @@ bool chunk_split_supported(int dk, int dv, int in_dtype) {
 cudaError_t launch_chunk_split(const void* q, const void* k, const void* v, const float* g,
                                const float* beta, const float* h0, const int32_t* cu_seqlens,
                                void* out, float* hT, int B, int T, int H, int dk, int dv,
-                               cudaStream_t stream) {
+                               int gsh, cudaStream_t stream) {
   int sms = 148;
   cudaMemPool_t pool = nullptr;
   if (!device_ctx(&sms, &pool) || !set_attrs()) return cudaErrorInvalidDevice;
@@ -937,7 +942,7 @@ cudaError_t launch_chunk_split(const void* q, const void* k, const void* v, cons
   if (nslots > 0) {
     KDA_TIMED(KDA_KERNEL_PREP, stream,
               kda_chunk_prep_kernel<<<dim3((unsigned)nslots, H), NT, PREP_SMEM, stream>>>(
-                  qb, kb, vb, g, beta, cu_seqlens, rec, B, T, H, dk, dv, nslots));
+                  qb, kb, vb, g, beta, cu_seqlens, rec, B, T, H, dk, dv, gsh, nslots));
     note_launches(1);
   }
   if (P == 0) {

@@ -137,7 +137,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 kda_decode_tokens_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                          const Tin* __restrict__ v, const float* __restrict__ g,
                          const float* __restrict__ beta, float* __restrict__ S,
-                         Tin* __restrict__ out, int L, int H) {
+                         Tin* __restrict__ out, int L, int H, int gsh) {
   constexpr int R = DK / 8;           // rows per lane (one row group)
   constexpr int CPL = DV / 32;        // columns per lane
   // (a = exp(g), k, q) of row c = grp R + i at [t][i][grp]: the 8 row groups a
@@ -166,7 +166,8 @@ kda_decode_tokens_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
       const int t = e / DK, c = e - t * DK;
       const long long row = (n * L + t0 + t) * H + h;
       s_akq[t][c % R][c / R] =
-          make_float4(expf(g[row * DK + c]), to_f32(k[row * DK + c]), to_f32(q[row * DK + c]), 0.f);
+          make_float4(expf(g[row * (DK >> gsh) + (c >> gsh)]), to_f32(k[row * DK + c]),
+                      to_f32(q[row * DK + c]), 0.f);
     }
     for (int e = tid; e < nt * DV; e += kThreads) {
       const int t = e / DV, j = e - t * DV;
@@ -230,11 +231,11 @@ kda_decode_tokens_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
 template <typename Tin, int DK, int DV>
 cudaError_t launch_tokens_t(const void* q, const void* k, const void* v, const float* g,
                             const float* beta, float* S, void* out, long long pairs, int L, int H,
-                            cudaStream_t stream) {
+                            int gsh, cudaStream_t stream) {
   KDA_TIMED(KDA_KERNEL_DECODE, stream,
             kda_decode_tokens_kernel<Tin, DK, DV><<<(unsigned)pairs, kThreads, 0, stream>>>(
                 static_cast<const Tin*>(q), static_cast<const Tin*>(k), static_cast<const Tin*>(v),
-                g, beta, S, static_cast<Tin*>(out), L, H));
+                g, beta, S, static_cast<Tin*>(out), L, H, gsh));
   note_launches(1);
   return cudaGetLastError();
 }
@@ -242,14 +243,14 @@ cudaError_t launch_tokens_t(const void* q, const void* k, const void* v, const f
 template <typename Tin>
 cudaError_t launch_tokens_dtype(const void* q, const void* k, const void* v, const float* g,
                                 const float* beta, float* S, void* out, long long pairs, int L,
-                                int H, int dk, int dv, cudaStream_t stream) {
+                                int H, int dk, int dv, int gsh, cudaStream_t stream) {
   if (dk == 128 && dv == 128)
-    return launch_tokens_t<Tin, 128, 128>(q, k, v, g, beta, S, out, pairs, L, H, stream);
+    return launch_tokens_t<Tin, 128, 128>(q, k, v, g, beta, S, out, pairs, L, H, gsh, stream);
   if (dk == 128 && dv == 64)
-    return launch_tokens_t<Tin, 128, 64>(q, k, v, g, beta, S, out, pairs, L, H, stream);
+    return launch_tokens_t<Tin, 128, 64>(q, k, v, g, beta, S, out, pairs, L, H, gsh, stream);
   if (dk == 64 && dv == 128)
-    return launch_tokens_t<Tin, 64, 128>(q, k, v, g, beta, S, out, pairs, L, H, stream);
-  return launch_tokens_t<Tin, 64, 64>(q, k, v, g, beta, S, out, pairs, L, H, stream);
+    return launch_tokens_t<Tin, 64, 128>(q, k, v, g, beta, S, out, pairs, L, H, gsh, stream);
+  return launch_tokens_t<Tin, 64, 64>(q, k, v, g, beta, S, out, pairs, L, H, gsh, stream);
 }
 
 template <typename Tin, int DK, int DV>
@@ -279,12 +280,12 @@ cudaError_t launch_dtype(const void* q, const void* k, const void* v, const floa
 
 cudaError_t launch_decode_tokens(const void* q, const void* k, const void* v, const float* g,
                                  const float* beta, float* S, void* out, int N, int L, int H,
-                                 int dk, int dv, int in_dtype, cudaStream_t stream) {
+                                 int dk, int dv, int in_dtype, int gsh, cudaStream_t stream) {
   const long long pairs = (long long)N * H;
   if (in_dtype == KDA_BF16)
     return launch_tokens_dtype<__nv_bfloat16>(q, k, v, g, beta, S, out, pairs, L, H, dk, dv,
-                                              stream);
-  return launch_tokens_dtype<float>(q, k, v, g, beta, S, out, pairs, L, H, dk, dv, stream);
+                                              gsh, stream);
+  return launch_tokens_dtype<float>(q, k, v, g, beta, S, out, pairs, L, H, dk, dv, gsh, stream);
 }
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* g,

@@ -38,14 +38,15 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, const flo
                           const float* beta, float* S, void* out, int N, int H, int dk,
                           int dv, int in_dtype, cudaStream_t stream);
 
+// gsh: log2 of the decay group (g holds one value per 2^gsh key channels).
 cudaError_t launch_decode_tokens(const void* q, const void* k, const void* v, const float* g,
                                  const float* beta, float* S, void* out, int N, int L, int H,
-                                 int dk, int dv, int in_dtype, cudaStream_t stream);
+                                 int dk, int dv, int in_dtype, int gsh, cudaStream_t stream);
 
 cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const float* g,
                               const float* beta, const float* h0, const int32_t* cu_seqlens,
                               void* out, float* hT, int B, int T, int H, int dk, int dv,
-                              int in_dtype, cudaStream_t stream);
+                              int in_dtype, int gsh, cudaStream_t stream);
 
 // Tensor-core chunked prefill (bf16, dk = dv = 128).
 bool chunk_tc_supported(int dk, int dv, int in_dtype);
@@ -60,7 +61,7 @@ bool chunk_split_supported(int dk, int dv, int in_dtype);
 cudaError_t launch_chunk_split(const void* q, const void* k, const void* v, const float* g,
                                const float* beta, const float* h0, const int32_t* cu_seqlens,
                                void* out, float* hT, int B, int T, int H, int dk, int dv,
-                               cudaStream_t stream);
+                               int gsh, cudaStream_t stream);
 
 // The tensor-core prefill on caller-provided scratch (allocates nothing).
 int run_chunk_tc_static(const void* q, const void* k, const void* v, const float* g,

@@ -60,7 +60,7 @@ extern "C" int kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v
   if (!kda::chunk_tc_supported(dk, dv, in_dtype)) {
     // this path keeps everything on chip and needs no scratch
     const cudaError_t e = kda::launch_chunk_simt(q, k, v, g, beta, h0, cu_seqlens, out, hT, B, T,
-                                                 H, dk, dv, in_dtype, st);
+                                                 H, dk, dv, in_dtype, 0, st);
     if (e != cudaSuccess) { (void)cudaGetLastError(); return KDA_ERR_CUDA; }
     return KDA_OK;
   }

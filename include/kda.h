@@ -176,6 +176,27 @@ KDA_API int kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
                                   int B, int T, int H, int dk, int dv,
                                   int in_dtype, void* stream);
 
+/*
+ * Grouped decay ("decay-g64" ablation of the Mini-K3-1H v2 family cards: the
+ * decay granularity is one of the varied architecture choices).  The pages
+ * name the variant but not its definition; the reading taken here: one log-
+ * decay value per group of g_group consecutive key channels, shared by the
+ * channels of the group -- channel c decays by exp(g[..., c / g_group]).  g is
+ * then [B, T, H, dk / g_group] (prefill) or [N, L, H, dk / g_group] (decode);
+ * everything else is as in kda_chunk_fwd / kda_decode_tokens, and g_group = 1
+ * is exactly those calls.  g_group must be a power of two, 1 <= g_group <= dk
+ * (else KDA_ERR_INVALID_ARG).
+ */
+KDA_API int kda_chunk_fwd_grouped(const void* q, const void* k, const void* v,
+                                  const float* g, const float* beta, const float* h0,
+                                  const int32_t* cu_seqlens, void* out, float* hT,
+                                  int B, int T, int H, int dk, int dv, int g_group,
+                                  int in_dtype, void* stream);
+KDA_API int kda_decode_tokens_grouped(const void* q, const void* k, const void* v,
+                                      const float* g, const float* beta, float* S, void* out,
+                                      int N, int L, int H, int dk, int dv, int g_group,
+                                      int in_dtype, void* stream);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 KDA_API const char* kda_status_string(int status);
 

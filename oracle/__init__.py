@@ -95,14 +95,29 @@ def _ptr(a):
     return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
 
 
+def expand_decay_groups(g, dk: int):
+    """Grouped decay (one log-decay per group of G = dk / g.shape[-1] consecutive key
+    channels, the "decay-g64" family card's decay-granularity variant): channel c
+    decays by exp(g[..., c // G]).  Returns the per-channel [..., dk] float64 array."""
+    g = _f64(g)
+    n = g.shape[-1]
+    if n == dk:
+        return g
+    if n < 1 or dk % n != 0:
+        raise ValueError(f"g's last dimension {n} does not divide dk = {dk}")
+    return np.ascontiguousarray(np.repeat(g, dk // n, axis=-1))
+
+
 def prefill(q, k, v, g, beta, h0=None, cu_seqlens=None, heads=None, nthreads: int = 0):
     """Float64 KDA prefill by recurrence.
 
-    q, k [B,T,H,dk]; v [B,T,H,dv]; g [B,T,H,dk]; beta [B,T,H]; h0 [Nseq,H,dk,dv]
+    q, k [B,T,H,dk]; v [B,T,H,dv]; g [B,T,H,dk] (or [B,T,H,dk/G]: one decay per group
+    of G key channels, see expand_decay_groups); beta [B,T,H]; h0 [Nseq,H,dk,dv]
     or None; cu_seqlens int [Nseq+1] or None (then tensors are [1,T,H,*]).
     ``heads``: optional (lo, hi) range; only those heads are computed and returned.
     Returns (out [B,T,H',dv], hT [Nseq,H',dk,dv]) as float64 numpy arrays.
     """
+    g = expand_decay_groups(g, q.shape[-1])
     if heads is not None:
         lo, hi = heads
         q, k, v, g, beta = (x[:, :, lo:hi] for x in (q, k, v, g, beta))
@@ -134,7 +149,8 @@ def prefill(q, k, v, g, beta, h0=None, cu_seqlens=None, heads=None, nthreads: in
 def decode(q, k, v, g, beta, S, nthreads: int = 0):
     """One float64 KDA decode step.  q,k [N,H,dk]; v [N,H,dv]; g [N,H,dk];
     beta [N,H]; S [N,H,dk,dv].  Returns (out [N,H,dv], S_new) as float64 arrays
-    (S is copied, not modified)."""
+    (S is copied, not modified).  g may be grouped ([N,H,dk/G], expand_decay_groups)."""
+    g = expand_decay_groups(g, q.shape[-1])
     q, k, v, g, beta = (_f64(x) for x in (q, k, v, g, beta))
     S = _f64(S).copy()
     N, H, dk = q.shape

@@ -86,3 +86,11 @@ def test_decode_tokens_rejects_invalid(L, bad):
 
 def test_decode_tokens_rejects_unsupported_heads(L):
     assert _tokens(L, dv=80) == kda.KDA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("G", [0, 3, 96, 256])
+def test_grouped_rejects_bad_group(L, G):
+    assert L.kda_chunk_fwd_grouped(P, P, P, P, P, None, None, P, None, 1, 4, 1, 128, 128, G, 0,
+                                   None) == kda.KDA_ERR_INVALID_ARG
+    assert L.kda_decode_tokens_grouped(P, P, P, P, P, P, P, 1, 2, 1, 128, 128, G, 0,
+                                       None) == kda.KDA_ERR_INVALID_ARG

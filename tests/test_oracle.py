@@ -382,3 +382,43 @@ def test_oracle_rejects_bad_cu_seqlens(oracle_lib):
         oracle.prefill(q, k, v, g, b, cu_seqlens=np.array([0, 6, 4, 10], dtype=np.int32))
     with pytest.raises(ValueError):
         oracle.prefill(q, k, v, g, b, cu_seqlens=np.array([0, 6, 9], dtype=np.int32))
+
+
+# ---- grouped decay (decay-granularity variant, "decay-g64" family card) -------
+@pytest.mark.parametrize("G", [2, 4, 8])
+def test_grouped_decay_beta_zero_closed_form(oracle_lib, G):
+    """With beta = 0 only the decay acts: row c of the state decays by
+    exp(sum_t g[t, c // G]) -- consecutive channels share one decay value."""
+    rng = np.random.default_rng(40 + G)
+    T, H, dk, dv = 9, 2, 8, 3
+    q, k, v, _, b = _rand_inputs(rng, T, H, dk, dv, beta=0.0)
+    gg = -0.5 * rng.random((1, T, H, dk // G))
+    h0 = rng.standard_normal((1, H, dk, dv))
+    out, hT = oracle.prefill(q, k, v, gg, b, h0)
+    for h in range(H):
+        for c in range(dk):
+            grp = c // G
+            np.testing.assert_allclose(hT[0, h, c], np.exp(gg[0, :, h, grp].sum()) * h0[0, h, c],
+                                       rtol=1e-12)
+        for t in range(T):
+            decay = np.array([np.exp(gg[0, :t + 1, h, c // G].sum()) for c in range(dk)])
+            np.testing.assert_allclose(out[0, t, h], (decay[:, None] * h0[0, h]).T @ q[0, t, h],
+                                       rtol=1e-10, atol=1e-14)
+
+
+def test_grouped_decay_single_group_is_scalar_gated_delta_rule(oracle_lib):
+    """G = dk: one decay per head and token, i.e. the scalar-gated delta rule
+    S_t = a_t (I - beta k k^T) S_{t-1} + beta k v^T (the scalar commutes with the
+    rank-1 factor), written out here with a matrix product per step."""
+    rng = np.random.default_rng(44)
+    T, H, dk, dv = 7, 1, 4, 3
+    q, k, v, _, b = _rand_inputs(rng, T, H, dk, dv)
+    gg = -0.4 * rng.random((1, T, H, 1))
+    h0 = rng.standard_normal((1, H, dk, dv))
+    out, hT = oracle.prefill(q, k, v, gg, b, h0)
+    S = h0[0, 0].copy()
+    for t in range(T):
+        kt, vt, bt = k[0, t, 0], v[0, t, 0], b[0, t, 0]
+        S = np.exp(gg[0, t, 0, 0]) * (np.eye(dk) - bt * np.outer(kt, kt)) @ S + bt * np.outer(kt, vt)
+        np.testing.assert_allclose(out[0, t, 0], S.T @ q[0, t, 0], rtol=1e-11, atol=1e-14)
+    np.testing.assert_allclose(hT[0, 0], S, rtol=1e-11, atol=1e-14)
