@@ -201,6 +201,17 @@ def cpu_baseline(args):
     return {"value": val, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
 
 
+def whole_job_rate(units_per_rank: int, world: int, steps: int, ms_max: float) -> float:
+    """Units per second over all ranks: every rank processes units_per_rank per
+    step (weak scaling); the job takes the slowest rank's time."""
+    return units_per_rank * world * steps / (ms_max / 1e3)
+
+
+def rank_seed(base: int, rank: int, i: int = 0) -> int:
+    """Seed of input set i on a rank: every rank draws its own shard."""
+    return base + 1000 * rank + i
+
+
 def _max_over_ranks(val, world, dev):
     if world == 1:
         return val
@@ -221,7 +232,7 @@ def prefill_leg(args, world, rank, dev, stream, barrier, clocks):
     spec = ki.PREFILL_SPECS[args.workload]
     sets = []                       # 3 resident input sets (L2 rotation)
     for i in range(3):
-        x = ki.make_prefill(spec, seed=spec.seed + 1000 * rank + i)
+        x = ki.make_prefill(spec, seed=rank_seed(spec.seed, rank, i))
         d = {n: (t.to(dev) if isinstance(t, torch.Tensor) else t) for n, t in x.items()}
         d["out"] = torch.empty_like(d["v"])
         d["hT"] = torch.empty(x["B"], x["H"], x["dk"], x["dv"], device=dev)
@@ -297,9 +308,9 @@ def prefill_leg(args, world, rank, dev, stream, barrier, clocks):
     e2e_ms = _max_over_ranks(e0.elapsed_time(e1), world, dev)
     return dict(x0=x0, rows=rows, s_in=s_in, bytes_call=bytes_call, flops_call=flops_call,
                 ktimes=ktimes,
-                value=rows * world * args.steps / (ms_max / 1e3), ms_max=ms_max,
+                value=whole_job_rate(rows, world, args.steps, ms_max), ms_max=ms_max,
                 call_ms=call_ms, launches=launches, clocks=clocks.summary(mark0, mark1),
-                e2e={"value": rows * world * e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
+                e2e={"value": whole_job_rate(rows, world, e2e_steps, e2e_ms), "unit": UNIT,
                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                      "steps": e2e_steps})
 
