@@ -85,6 +85,9 @@ constexpr uint32_t Q_B32 = 32768;       // diag(beta) A, fp32
 constexpr uint32_t Q_T32 = Q_B32 + 17408;   // T, fp32
 constexpr uint32_t Q_M32 = Q_T32 + 17408;   // T_aa B_am, 6 x 16 x 16 fp32
 constexpr uint32_t Q_TB = 73728;        // T diag(beta): K-major SW128 B operand of W^T / U^T
+// record images on their way out (bulk copies): Aqk after the Gram readout,
+// then W^T and U^T over the dead solve scratch once their MMAs are done
+constexpr uint32_t Q_OAQK = 81920, Q_OW = 32768, Q_OU = 49152;
 constexpr uint32_t PREP_SMEM = 106496 + 1024;
 constexpr uint32_t PT_G = 0;            // Gram D^(0..3) at +0, +16, +48, +96 (160 columns)
 constexpr uint32_t PT_W = 0;            // W^T [128 x 64] (after the Gram is read)
@@ -356,7 +359,7 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
 #pragma unroll
           for (int e = 0; e < 8; ++e)
             w[e] = (c8 * 8 + e <= r) ? __uint_as_float(tv[c8 >> 1][(c8 & 1) * 8 + e]) : 0.f;
-          *reinterpret_cast<uint4*>(rc + REC_AQK + chunk_kmajor_sw128(r, c8, C)) = pack8(w, 1.f);
+          sts16(sm, Q_OAQK + chunk_kmajor_sw128(r, c8, C), pack8(w, 1.f));
         }
       }
     }
@@ -514,15 +517,23 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
                                      pack_bf16(__uint_as_float(f[2]), __uint_as_float(f[3])),
                                      pack_bf16(__uint_as_float(f[4]), __uint_as_float(f[5])),
                                      pack_bf16(__uint_as_float(f[6]), __uint_as_float(f[7])));
-        *reinterpret_cast<uint4*>(rc + REC_QW + 16384 + chunk_mnmajor_sw128(g8, j, D)) = val;
+        sts16(sm, Q_OW + chunk_mnmajor_sw128(g8, j, D), val);
       }
     } else {
 #pragma unroll
       for (int c4 = 0; c4 < 16; ++c4) {
         const uint32_t* f = t[c4 >> 2] + 4 * (c4 & 3);
-        *reinterpret_cast<uint4*>(rc + REC_U + j * 256 + (((uint32_t)c4 ^ (j & 15u)) << 4)) =
-            make_uint4(f[0], f[1], f[2], f[3]);
+        sts16(sm, Q_OU + j * 256 + (((uint32_t)c4 ^ (j & 15u)) << 4), make_uint4(f[0], f[1], f[2], f[3]));
       }
+    }
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {                          // the staged images go out as three bulk copies
+      bulk_s2g(rc + REC_AQK, sm + Q_OAQK, 8192);
+      bulk_s2g(rc + REC_QW + 16384, sm + Q_OW, 16384);
+      bulk_s2g(rc + REC_U, sm + Q_OU, 32768);
+      bulk_commit();
+      bulk_wait_read<0>();                   // shared memory read out before the CTA ends
     }
   }
 
