@@ -437,7 +437,7 @@ def decode_leg(args, world, rank, dev, stream, barrier, clocks, hbm, peak_kind):
 
 
 KERNEL_NAMES = {"prep": "kda_chunk_prep_kernel", "state": "kda_state_pass_kernel",
-                "combine": "kda_seg_combine_kernel", "fused": "kda_chunk_tc_kernel",
+                "combine": "kda_seg_combine_img_kernel", "fused": "kda_chunk_tc_kernel",
                 "simt": "kda_chunk_simt_kernel"}
 
 
