@@ -71,6 +71,9 @@ def _load():
                                               ctypes.c_int, ctypes.c_longlong,
                                               ctypes.c_longlong, ctypes.c_int]
             lib.kda_oracle_decode.restype = ctypes.c_int
+            lib.kda_oracle_backward.argtypes = ([dp] * 6 + [ctypes.POINTER(ctypes.c_int32)] +
+                                                [dp] * 8 + [ctypes.c_int] * 8)
+            lib.kda_oracle_backward.restype = ctypes.c_int
             lib.kda_oracle_max_threads.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -162,3 +165,44 @@ def decode(q, k, v, g, beta, S, nthreads: int = 0):
     if rc != 0:
         raise ValueError(f"kda_oracle_decode rejected its arguments (rc={rc})")
     return out, S
+
+
+def backward(q, k, v, g, beta, dout, h0=None, dhT=None, cu_seqlens=None, heads=None,
+             nthreads: int = 0):
+    """Float64 gradients of L = sum(out * dout) + sum(hT * dhT) for the prefill
+    (reverse-mode differentiation of the recurrence; kda_oracle.cpp).
+
+    Shapes as in ``prefill``; dout [B,T,H,dv]; dhT [Nseq,H,dk,dv] or None.
+    Returns a dict of float64 arrays dq, dk, dv, dg, dbeta, dh0 (dg has g's
+    per-channel shape [B,T,H,dk]; for grouped g sum it over each group).
+    """
+    if heads is not None:
+        lo, hi = heads
+        q, k, v, g, beta, dout = (x[:, :, lo:hi] for x in (q, k, v, g, beta, dout))
+        if h0 is not None:
+            h0 = h0[:, lo:hi]
+        if dhT is not None:
+            dhT = dhT[:, lo:hi]
+    g = expand_decay_groups(g, q.shape[-1])
+    q, k, v, g, beta, h0, dout, dhT = (_f64(x) for x in (q, k, v, g, beta, h0, dout, dhT))
+    Bt, T, H, dk = q.shape
+    dv = v.shape[-1]
+    cu = None
+    if cu_seqlens is not None:
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens.cpu() if hasattr(cu_seqlens, "cpu")
+                                             else cu_seqlens), dtype=np.int32)
+        nseq = cu.shape[0] - 1
+    else:
+        nseq = Bt
+    res = {n: np.zeros(x.shape, dtype=np.float64) for n, x in
+           (("dq", q), ("dk", k), ("dv", v), ("dg", g), ("dbeta", beta))}
+    res["dh0"] = np.zeros((nseq, H, dk, dv), dtype=np.float64)
+    rc = _load().kda_oracle_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
+        None if cu is None else cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+        _ptr(dout), _ptr(dhT), _ptr(res["dq"]), _ptr(res["dk"]), _ptr(res["dv"]),
+        _ptr(res["dg"]), _ptr(res["dbeta"]), _ptr(res["dh0"]), nseq, T, H, dk, dv, 0, H,
+        int(nthreads))
+    if rc != 0:
+        raise ValueError(f"kda_oracle_backward rejected its arguments (rc={rc})")
+    return res

@@ -422,3 +422,83 @@ def test_grouped_decay_single_group_is_scalar_gated_delta_rule(oracle_lib):
         S = np.exp(gg[0, t, 0, 0]) * (np.eye(dk) - bt * np.outer(kt, kt)) @ S + bt * np.outer(kt, vt)
         np.testing.assert_allclose(out[0, t, 0], S.T @ q[0, t, 0], rtol=1e-11, atol=1e-14)
     np.testing.assert_allclose(hT[0, 0], S, rtol=1e-11, atol=1e-14)
+
+
+# ---- backward (the chunked form "trains through"; gradient checks by finite differences) ----
+def _loss_fd(args, dout, dhT, cu=None):
+    o, s = oracle.prefill(args["q"], args["k"], args["v"], args["g"], args["b"], args["h0"], cu)
+    return (o * dout).sum() + (s * dhT).sum()
+
+
+@pytest.mark.parametrize("packed", [False, True])
+def test_backward_matches_finite_differences(oracle_lib, packed):
+    """Central differences of L = <out, dout> + <hT, dhT> on the float64 forward
+    (the course outline's finite-difference gradient checks)."""
+    rng = np.random.default_rng(60 + packed)
+    T, H, dk, dv = 7, 2, 4, 3
+    q, k, v, g, b = _rand_inputs(rng, T, H, dk, dv)
+    cu = np.array([0, 3, 7], dtype=np.int32) if packed else None
+    nseq = 2 if packed else 1
+    h0 = rng.standard_normal((nseq, H, dk, dv))
+    dout = rng.standard_normal((1, T, H, dv))
+    dhT = rng.standard_normal((nseq, H, dk, dv))
+    r = oracle.backward(q, k, v, g, b, dout, h0, dhT, cu)
+    args = dict(q=q, k=k, v=v, g=g, b=b, h0=h0)
+    eps = 1e-6
+    for name, key in (("q", "dq"), ("k", "dk"), ("v", "dv"), ("g", "dg"), ("b", "dbeta"),
+                      ("h0", "dh0")):
+        x = args[name]
+        num = np.zeros_like(x)
+        for i in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[i] += eps
+            xm[i] -= eps
+            num[i] = (_loss_fd({**args, name: xp}, dout, dhT, cu) -
+                      _loss_fd({**args, name: xm}, dout, dhT, cu)) / (2 * eps)
+        np.testing.assert_allclose(r[key], num, rtol=1e-6, atol=1e-7, err_msg=name)
+
+
+def test_backward_matches_autograd_of_literal_recurrence(oracle_lib):
+    """torch autograd through a float64 restatement with the dk x dk factor
+    (I - beta k k^T) Diag(exp g) materialised (recurrence_literal's form)."""
+    rng = np.random.default_rng(70)
+    T, H, dk, dv = 6, 1, 5, 4
+    q, k, v, g, b = _rand_inputs(rng, T, H, dk, dv)
+    h0 = rng.standard_normal((1, H, dk, dv))
+    dout = rng.standard_normal((1, T, H, dv))
+    dhT = rng.standard_normal((1, H, dk, dv))
+    r = oracle.backward(q, k, v, g, b, dout, h0, dhT)
+    tq, tk, tv, tg, tb, th = (torch.tensor(x, dtype=torch.float64, requires_grad=True)
+                              for x in (q, k, v, g, b, h0))
+    S = th[0, 0]
+    loss = 0.0
+    for t in range(T):
+        kt, vt = tk[0, t, 0], tv[0, t, 0]
+        M = (torch.eye(dk, dtype=torch.float64) - tb[0, t, 0] * torch.outer(kt, kt)) @ \
+            torch.diag(torch.exp(tg[0, t, 0]))
+        S = M @ S + tb[0, t, 0] * torch.outer(kt, vt)
+        loss = loss + (S.T @ tq[0, t, 0] * torch.tensor(dout[0, t, 0])).sum()
+    loss = loss + (S * torch.tensor(dhT[0, 0])).sum()
+    loss.backward()
+    for key, t in (("dq", tq), ("dk", tk), ("dv", tv), ("dg", tg), ("dbeta", tb), ("dh0", th)):
+        np.testing.assert_allclose(r[key], t.grad.numpy(), rtol=1e-11, atol=1e-13, err_msg=key)
+
+
+def test_backward_document_isolation_zero_gradient(oracle_lib):
+    """A loss on document 2 only gives exactly zero gradient to every input of
+    document 1 and to its initial state (the packed-document card's zero-gradient
+    isolation gate: state flow resets at every boundary)."""
+    rng = np.random.default_rng(71)
+    T, H, dk, dv = 9, 2, 4, 3
+    q, k, v, g, b = _rand_inputs(rng, T, H, dk, dv)
+    cu = np.array([0, 4, 9], dtype=np.int32)
+    h0 = rng.standard_normal((2, H, dk, dv))
+    dout = rng.standard_normal((1, T, H, dv))
+    dout[:, :4] = 0.0
+    dhT = rng.standard_normal((2, H, dk, dv))
+    dhT[0] = 0.0
+    r = oracle.backward(q, k, v, g, b, dout, h0, dhT, cu)
+    for key in ("dq", "dk", "dv", "dg", "dbeta"):
+        assert np.all(r[key][:, :4] == 0.0), key
+        assert np.any(r[key][:, 4:] != 0.0), key
+    assert np.all(r["dh0"][0] == 0.0) and np.any(r["dh0"][1] != 0.0)
