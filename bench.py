@@ -364,6 +364,61 @@ def grouped_leg(args, world, rank, dev, stream, barrier, hbm, G=64):
             "algorithmic_bytes_per_call": bytes_call, "gbs": gbs, "frac_of_hbm_peak": gbs / hbm}
 
 
+def bwd_leg(args, world, rank, dev, stream, barrier, hbm):
+    """The prefill backward (kda_chunk_bwd) on the headline workload: a few timed
+    calls on two resident input sets, fp32 gradients of sum(out*dout) + sum(hT*dhT)."""
+    import torch
+
+    import gated_delta_rule_74_b200 as kda
+    import kda_inputs as ki
+
+    spec = ki.PREFILL_SPECS[args.workload]
+    sets = []
+    for i in range(2):
+        x = ki.make_prefill(spec, seed=spec.seed + 1000 * rank + 700 + i)
+        d = {n: (t.to(dev) if isinstance(t, torch.Tensor) else t) for n, t in x.items()}
+        gen = torch.Generator().manual_seed(rank_seed(spec.seed + 900, rank, i))
+        d["dout"] = torch.randn(x["v"].shape, generator=gen).to(x["v"].dtype).to(dev)
+        d["dhT"] = (0.1 * torch.randn((x["B"], x["H"], x["dk"], x["dv"]), generator=gen)).to(dev)
+        d["grads"] = {n: torch.empty(x[src].shape, dtype=torch.float32, device=dev)
+                      for n, src in (("dq", "q"), ("dk", "k"), ("dv", "v"), ("dg", "g"),
+                                     ("dbeta", "beta"))}
+        if x["h0"] is not None:
+            d["grads"]["dh0"] = torch.empty_like(d["h0"])
+        sets.append(d)
+    x0 = sets[0]
+    rows = x0["T"] if x0["cu_seqlens"] is not None else x0["B"] * x0["T"]
+    s_in = 2 if x0["dtype"] == "bf16" else 4
+    H, dk, dv = x0["H"], x0["dk"], x0["dv"]
+    nstate = int(x0["h0"] is not None) * 2 + 1
+    bytes_call = rows * H * ((2 * dk + 2 * dv) * s_in + 4 * dk + 4 + 12 * dk + 4 * dv + 4) + \
+        x0["B"] * H * 4 * dk * dv * nstate
+    steps = max(1, min(args.steps, args.bwd_steps))
+
+    def call(i):
+        d = sets[i % 2]
+        kda.kda_chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["dout"], h0=d["h0"],
+                          dhT=d["dhT"], cu_seqlens=d["cu_seqlens"], grads=d["grads"],
+                          stream=stream)
+
+    for i in range(min(args.warmup, 3)):
+        call(i)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        call(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = _max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
+    gbs = bytes_call / (ms / 1e3) / 1e9
+    return {"call": "kda_chunk_bwd", "steps": steps,
+            "tokens_per_s": rows * world / (ms / 1e3), "ms_per_call": ms,
+            "algorithmic_bytes_per_call": bytes_call, "gbs": gbs, "frac_of_hbm_peak": gbs / hbm}
+
+
 def decode_leg(args, world, rank, dev, stream, barrier, clocks, hbm, peak_kind):
     """K timed kda_decode_step calls on the config-4 shape (state in HBM)."""
     import torch
@@ -576,6 +631,9 @@ def run_ours(args, world, rank, local):
     grp = None
     if not args.decode_only and not args.no_grouped:
         grp = grouped_leg(args, world, rank, dev, stream, barrier, hbm)
+    bwd = None
+    if not args.decode_only and not args.no_bwd:
+        bwd = bwd_leg(args, world, rank, dev, stream, barrier, hbm)
     dec = None
     if not args.no_decode:
         dec = decode_leg(args, world, rank, dev, stream, barrier, clocks, hbm, peak_kind)
@@ -604,6 +662,7 @@ def run_ours(args, world, rank, local):
         "config": _config(args, pf["x0"], world),
         "roofline": roof,
         "prefill_decay_g64": grp,
+        "prefill_bwd": bwd,
         "decode": dec, "e2e": pf["e2e"], "gpu_launches": pf["launches"],
         "clocks": pf["clocks"], "cpu_baseline": cpu,
     }
@@ -622,6 +681,10 @@ def main():
     ap.add_argument("--workload", default="metric", choices=["metric", "cfg1", "cfg2", "cfg3"])
     ap.add_argument("--decode-steps", type=int, default=100)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-bwd", action="store_true",
+                    help="skip the prefill backward (kda_chunk_bwd) leg")
+    ap.add_argument("--bwd-steps", type=int, default=5,
+                    help="timed kda_chunk_bwd calls (at most --steps)")
     ap.add_argument("--no-grouped", action="store_true",
                     help="skip the grouped-decay (G = 64) prefill leg")
     ap.add_argument("--no-fused-decode", action="store_true",

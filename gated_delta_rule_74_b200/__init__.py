@@ -8,6 +8,7 @@ call fails, an exception is raised.
 
     out, hT = kda_chunk_fwd(q, k, v, g, beta, h0=None, cu_seqlens=None)
     out     = kda_decode_step(q, k, v, g, beta, S)        # S updated in place
+    grads   = kda_chunk_bwd(q, k, v, g, beta, dout, h0=None, dhT=None, cu_seqlens=None)
 """
 from __future__ import annotations
 
@@ -18,7 +19,7 @@ from typing import Optional
 
 import torch
 
-__all__ = ["kda_chunk_fwd", "kda_decode_step", "kda_status_string", "kda_version",
+__all__ = ["kda_chunk_fwd", "kda_chunk_bwd", "kda_decode_step", "kda_decode_tokens", "kda_status_string", "kda_version",
            "kda_launch_count",
            "lib", "library_path", "header_symbols", "KdaError",
            "KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED", "KDA_ERR_CUDA",
@@ -71,6 +72,9 @@ def lib() -> ctypes.CDLL:
         L.kda_decode_tokens_grouped.restype = ctypes.c_int
         L.kda_chunk_fwd_grouped.argtypes = [vp, vp, vp, fp, fp, fp, vp, vp, fp] + [ip] * 7 + [vp]
         L.kda_chunk_fwd_grouped.restype = ctypes.c_int
+        L.kda_chunk_bwd.argtypes = [vp, vp, vp, fp, fp, fp, vp, vp, fp,
+                                    fp, fp, fp, fp, fp, fp] + [ip] * 6 + [vp]
+        L.kda_chunk_bwd.restype = ctypes.c_int
         L.kda_status_string.argtypes = [ctypes.c_int]
         L.kda_status_string.restype = ctypes.c_char_p
         L.kda_version.argtypes = []
@@ -108,7 +112,8 @@ def kda_launch_count() -> int:
     return int(lib().kda_launch_count())
 
 
-KERNEL_KINDS = {"prep": 0, "state": 1, "combine": 2, "fused": 3, "simt": 4, "decode": 5}
+KERNEL_KINDS = {"prep": 0, "state": 1, "combine": 2, "fused": 3, "simt": 4, "decode": 5,
+                "bwd": 6}
 
 
 def kda_timing_start() -> None:
@@ -210,6 +215,58 @@ def kda_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Te
     if rc != KDA_OK:
         raise KdaError("kda_chunk_fwd", rc)
     return out, hT
+
+
+def kda_chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+                  beta: torch.Tensor, dout: torch.Tensor, h0: Optional[torch.Tensor] = None,
+                  dhT: Optional[torch.Tensor] = None, cu_seqlens: Optional[torch.Tensor] = None,
+                  grads: Optional[dict] = None, stream=None) -> dict:
+    """Gradients of L = sum(out * dout) + sum(hT * dhT) for kda_chunk_fwd with the same
+    inputs (per-channel g only).  dout has out's shape and dtype; dhT [Nseq,H,dk,dv] f32
+    or None.  Returns a dict of fp32 tensors dq, dk, dv, dg, dbeta, dh0 (dh0 None when
+    h0 is None); ``grads`` may hold preallocated outputs under those names."""
+    if q.dim() != 4:
+        raise ValueError("q must be [B, T, H, dk]")
+    Bt, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = _DTYPES.get(q.dtype)
+    if dt is None:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    _check("q", q)
+    _check("k", k, q.dtype, (Bt, T, H, dk))
+    _check("v", v, q.dtype, (Bt, T, H, dv))
+    _check("g", g, torch.float32, (Bt, T, H, dk))
+    _check("beta", beta, torch.float32, (Bt, T, H))
+    _check("dout", dout, q.dtype, (Bt, T, H, dv))
+    if cu_seqlens is not None:
+        _check("cu_seqlens", cu_seqlens, torch.int32)
+        if Bt != 1:
+            raise ValueError("packed inputs (cu_seqlens) must have B == 1")
+        nseq = cu_seqlens.numel() - 1
+    else:
+        nseq = Bt
+    if h0 is not None:
+        _check("h0", h0, torch.float32, (nseq, H, dk, dv))
+    if dhT is not None:
+        _check("dhT", dhT, torch.float32, (nseq, H, dk, dv))
+    shapes = {"dq": (Bt, T, H, dk), "dk": (Bt, T, H, dk), "dv": (Bt, T, H, dv),
+              "dg": (Bt, T, H, dk), "dbeta": (Bt, T, H), "dh0": (nseq, H, dk, dv)}
+    res = dict(grads or {})
+    for name, shp in shapes.items():
+        if name == "dh0" and h0 is None and res.get(name) is None:
+            res[name] = None
+            continue
+        if res.get(name) is None:
+            res[name] = torch.empty(shp, dtype=torch.float32, device=q.device)
+        _check(name, res[name], torch.float32, shp)
+    rc = lib().kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
+                             _ptr(cu_seqlens), _ptr(dout), _ptr(dhT), _ptr(res["dq"]),
+                             _ptr(res["dk"]), _ptr(res["dv"]), _ptr(res["dg"]),
+                             _ptr(res["dbeta"]), _ptr(res["dh0"]), nseq, T, H, dk, dv, dt,
+                             _stream(stream))
+    if rc != KDA_OK:
+        raise KdaError("kda_chunk_bwd", rc)
+    return res
 
 
 def kda_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,

@@ -131,6 +131,32 @@ int kda_decode_tokens_grouped(const void* q, const void* k, const void* v, const
                             in_dtype, stream);
 }
 
+int kda_chunk_bwd(const void* q, const void* k, const void* v, const float* g,
+                  const float* beta, const float* h0, const int32_t* cu_seqlens,
+                  const void* dout, const float* dhT, float* dq, float* dk, float* dv, float* dg,
+                  float* dbeta, float* dh0, int B, int T, int H, int dk_dim, int dv_dim,
+                  int in_dtype, void* stream) {
+  if (B < 1 || T < 0 || H < 1) return KDA_ERR_INVALID_ARG;
+  if (in_dtype != KDA_BF16 && in_dtype != KDA_F32) return KDA_ERR_INVALID_ARG;
+  const long long rows = cu_seqlens ? (long long)T : (long long)B * T;
+  if (rows > 0) {
+    if (!pointers_ok({q, k, v, g, beta, dout, dq, dk, dv, dg, dbeta}, {h0, dhT, dh0, cu_seqlens}))
+      return KDA_ERR_INVALID_ARG;
+  } else {
+    if (!pointers_ok({}, {q, k, v, g, beta, dout, dq, dk, dv, dg, dbeta, h0, dhT, dh0,
+                          cu_seqlens}))
+      return KDA_ERR_INVALID_ARG;
+  }
+  if (!head_ok(dk_dim) || !head_ok(dv_dim)) return KDA_ERR_UNSUPPORTED;
+  if (rows * H * (long long)(dk_dim > dv_dim ? dk_dim : dv_dim) > (1LL << 40))
+    return KDA_ERR_INVALID_ARG;
+  if ((long long)B > 65535LL || H > 0x7fffffff) return KDA_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return status_from(kda::launch_chunk_bwd(q, k, v, g, beta, h0, cu_seqlens, dout, dhT, dq, dk,
+                                           dv, dg, dbeta, dh0, B, T, H, dk_dim, dv_dim,
+                                           in_dtype, st));
+}
+
 const char* kda_status_string(int status) {
   switch (status) {
     case KDA_OK: return "KDA_OK";

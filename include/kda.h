@@ -197,6 +197,40 @@ KDA_API int kda_decode_tokens_grouped(const void* q, const void* k, const void* 
                                       int N, int L, int H, int dk, int dv, int g_group,
                                       int in_dtype, void* stream);
 
+/*
+ * kda_chunk_bwd -- gradients of the KDA prefill (training backward).
+ *
+ * Passage: miniKimiK3 model card, "Kimi Delta Attention" bullet: KDA "trains
+ * through a chunked parallel form"; the chunked form equals the recurrence at
+ * the top of this file, so its gradients are those of the recurrence.  For the
+ * scalar L = sum(out * dout) + sum(hT * dhT) of a kda_chunk_fwd call with the
+ * same inputs, this writes
+ *     dq, dk [B, T, H, dk]   dv [B, T, H, dv]   dg [B, T, H, dk]   dbeta [B, T, H]
+ *     dh0 [B, H, dk, dv]
+ * as fp32 (dL/dq, ..., dL/dh0), whatever in_dtype is.  Inputs, layouts,
+ * packed mode (cu_seqlens) and in_dtype are those of kda_chunk_fwd; dout has
+ * out's shape and dtype; dhT has hT's shape (fp32).  h0 NULL means zeros and
+ * then dh0 may be NULL; dhT NULL means zeros.  No gradient flows across a
+ * document boundary.  Every token gradient buffer is fully written (empty
+ * documents write nothing; their dh0 = dhT).  Output buffers must not alias
+ * each other or any input.  The chunk length (64) does not change the result.
+ *
+ * Method: a recurrent reverse sweep in fp32 on the CUDA cores, one CTA per
+ * (sequence, head); the states are kept at every 64th token and each chunk's
+ * states are recomputed once.  Scratch: 4 * dk * dv bytes per (chunk, head)
+ * plus 65 * 4 * dk * dv bytes per (sequence, head), from the library's
+ * stream-ordered memory pool (released on the stream at the end of the call).
+ *
+ * Returns KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED or KDA_ERR_CUDA
+ * (also when the scratch cannot be allocated).
+ */
+KDA_API int kda_chunk_bwd(const void* q, const void* k, const void* v,
+                          const float* g, const float* beta, const float* h0,
+                          const int32_t* cu_seqlens, const void* dout, const float* dhT,
+                          float* dq, float* dk, float* dv, float* dg, float* dbeta,
+                          float* dh0, int B, int T, int H, int dk_dim, int dv_dim,
+                          int in_dtype, void* stream);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 KDA_API const char* kda_status_string(int status);
 
@@ -226,7 +260,8 @@ typedef enum {
   KDA_KERNEL_FUSED = 3,         /* single-kernel tensor-core prefill              */
   KDA_KERNEL_SIMT = 4,          /* CUDA-core prefill (fp32, d = 64)               */
   KDA_KERNEL_DECODE = 5,        /* decode step                                    */
-  KDA_KERNEL_KINDS = 6
+  KDA_KERNEL_BWD = 6,           /* prefill backward                               */
+  KDA_KERNEL_KINDS = 7
 } kda_kernel_kind_t;
 KDA_API int kda_timing_start(void);
 KDA_API int kda_timing_stop(void);

@@ -94,3 +94,22 @@ def test_grouped_rejects_bad_group(L, G):
                                    None) == kda.KDA_ERR_INVALID_ARG
     assert L.kda_decode_tokens_grouped(P, P, P, P, P, P, P, 1, 2, 1, 128, 128, G, 0,
                                        None) == kda.KDA_ERR_INVALID_ARG
+
+
+def _bwd(L, q=P, k=P, v=P, g=P, beta=P, h0=None, cu=None, dout=P, dhT=None, dq=P, dk_=P,
+         dv_=P, dg=P, dbeta=P, dh0=None, B=1, T=64, H=2, dk=64, dv=64, dt=0):
+    return L.kda_chunk_bwd(q, k, v, g, beta, h0, cu, dout, dhT, dq, dk_, dv_, dg, dbeta, dh0,
+                           B, T, H, dk, dv, dt, None)
+
+
+@pytest.mark.parametrize("bad", [dict(q=None), dict(dout=None), dict(dq=None), dict(dk_=None),
+                                 dict(dv_=None), dict(dg=None), dict(dbeta=None),
+                                 dict(dout=P + 4), dict(dhT=P + 8), dict(dh0=P + 2),
+                                 dict(B=0), dict(T=-1), dict(H=0), dict(dt=5)])
+def test_chunk_bwd_rejects_invalid(L, bad):
+    assert _bwd(L, **bad) == kda.KDA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("dims", [dict(dk=32), dict(dv=96)])
+def test_chunk_bwd_rejects_unsupported_heads(L, dims):
+    assert _bwd(L, **dims) == kda.KDA_ERR_UNSUPPORTED
