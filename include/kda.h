@@ -215,11 +215,15 @@ KDA_API int kda_decode_tokens_grouped(const void* q, const void* k, const void* 
  * documents write nothing; their dh0 = dhT).  Output buffers must not alias
  * each other or any input.  The chunk length (64) does not change the result.
  *
- * Method: a recurrent reverse sweep in fp32 on the CUDA cores, one CTA per
- * (sequence, head); the states are kept at every 64th token and each chunk's
- * states are recomputed once.  Scratch: 4 * dk * dv bytes per (chunk, head)
- * plus 65 * 4 * dk * dv bytes per (sequence, head), from the library's
- * stream-ordered memory pool (released on the stream at the end of the call).
+ * Method: a recurrent reverse sweep in fp32 on the CUDA cores.  The columns of
+ * the state evolve independently, so each warp runs the chain of 8 state
+ * columns for one (sequence, head); the state is kept at every 64th token and
+ * each chunk's states are recomputed once.  dv and dh0 are reproducible bit for
+ * bit; dq, dk, dg and dbeta add the warps' parts with atomics, so repeated calls
+ * may differ in the last bits (fp32 summation order).  Scratch: 4 * dk * dv
+ * bytes per (chunk, head) plus 64 * 4 * dk * dv bytes per (sequence, head), from
+ * the library's stream-ordered memory pool (released on the stream at the end
+ * of the call).
  *
  * Returns KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED or KDA_ERR_CUDA
  * (also when the scratch cannot be allocated).
