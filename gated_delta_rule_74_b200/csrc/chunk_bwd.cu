@@ -13,7 +13,7 @@
 //
 // Column independence.  Every column j of S (and of G) evolves on its own: the
 // sums that couple entries run over the rows (a^T k, G^T k), never over the
-// columns.  So a warp owns NC = 8 columns and all dk rows (lane l: rows
+// columns.  So a warp owns NC = 4 columns and all dk rows (lane l: rows
 // [l R, l R + R), R = dk / 32) and runs its chain with warp shuffles only -- no
 // CTA barrier per token.  Only the per-token row gradients dq, dk, dg and dbeta
 // sum over columns; each warp adds its part with one vector atomic per lane
@@ -37,39 +37,32 @@ namespace {
 
 using namespace sm100;
 
-constexpr int NC = 8;             // state columns per warp
+constexpr int NC = 4;             // state columns per warp
 constexpr int WPC = 4;            // warps per CTA
 constexpr int CPC = NC * WPC;     // state columns per CTA
 constexpr int NTB = 32 * WPC;
 constexpr int RING = 4;           // depth of the reverse sweep's state prefetch
 constexpr unsigned FULL = 0xffffffffu;
 
-// Sum over the 32 lanes of each of the 8 per-lane values p[j]; every lane gets
-// all 8 totals.  Transpose-reduce (the halves exchanged at lane distance 16, 8,
-// 4 leave each lane one column), two butterfly steps, then a gather.
-__device__ __forceinline__ void colsum8(const float (&p)[8], float (&tot)[8], int lane) {
-  const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
-  float x[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float keep = b4 ? p[i + 4] : p[i];
-    const float send = b4 ? p[i] : p[i + 4];
-    x[i] = keep + __shfl_xor_sync(FULL, send, 16);
-  }
-  float y[2];
+// Sum over the 32 lanes of each of the 4 per-lane values p[j]; every lane gets
+// all 4 totals.  Transpose-reduce (the halves exchanged at lane distance 16 and
+// 8 leave each lane one column), three butterfly steps, then a gather.
+__device__ __forceinline__ void colsum4(const float (&p)[4], float (&tot)[4], int lane) {
+  const bool b4 = lane & 16, b3 = lane & 8;
+  float x[2];
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
-    const float keep = b3 ? x[i + 2] : x[i];
-    const float send = b3 ? x[i] : x[i + 2];
-    y[i] = keep + __shfl_xor_sync(FULL, send, 8);
+    const float keep = b4 ? p[i + 2] : p[i];
+    const float send = b4 ? p[i] : p[i + 2];
+    x[i] = keep + __shfl_xor_sync(FULL, send, 16);
   }
-  float z = (b2 ? y[1] : y[0]) + __shfl_xor_sync(FULL, b2 ? y[0] : y[1], 4);
+  float z = (b3 ? x[1] : x[0]) + __shfl_xor_sync(FULL, b3 ? x[0] : x[1], 8);
+  z += __shfl_xor_sync(FULL, z, 4);
   z += __shfl_xor_sync(FULL, z, 2);
   z += __shfl_xor_sync(FULL, z, 1);
-  // lane holds column 4*b4 + 2*b3 + b2
+  // lane holds column 2*b4 + b3
 #pragma unroll
-  for (int j = 0; j < 8; ++j)
-    tot[j] = __shfl_sync(FULL, z, ((j >> 2) & 1) * 16 + ((j >> 1) & 1) * 8 + (j & 1) * 4);
+  for (int j = 0; j < 4; ++j) tot[j] = __shfl_sync(FULL, z, ((j >> 1) & 1) * 16 + (j & 1) * 8);
 }
 
 template <int R> struct Rows;
@@ -92,6 +85,13 @@ template <> struct Rows<2> {
   }
 };
 
+__device__ __forceinline__ void ld4(const float* p, float (&x)[4]) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+}
+__device__ __forceinline__ void st4(float* p, const float (&x)[4]) {
+  *reinterpret_cast<float4*>(p) = make_float4(x[0], x[1], x[2], x[3]);
+}
 __device__ __forceinline__ void ld8(const float* p, float (&x)[8]) {
   const float4 a = *reinterpret_cast<const float4*>(p);
   const float4 b = *reinterpret_cast<const float4*>(p + 4);
@@ -115,60 +115,81 @@ __device__ __forceinline__ void gld8(const __nv_bfloat16* p, float (&x)[8]) {
   }
 }
 
-// Shared-memory layout (floats): per chunk the staged inputs, then per-warp e_t,
-// then the per-warp state ring.
-template <int DK>
+// R (4 or 2) consecutive shared-memory elements as fp32
+__device__ __forceinline__ void lds_n(const float* p, float (&x)[4]) { ld4(p, x); }
+__device__ __forceinline__ void lds_n(const float* p, float (&x)[2]) {
+  const float2 t = *reinterpret_cast<const float2*>(p);
+  x[0] = t.x; x[1] = t.y;
+}
+__device__ __forceinline__ void lds_n(const __nv_bfloat16* p, float (&x)[4]) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  x[0] = __uint_as_float(u.x << 16); x[1] = __uint_as_float(u.x & 0xffff0000u);
+  x[2] = __uint_as_float(u.y << 16); x[3] = __uint_as_float(u.y & 0xffff0000u);
+}
+__device__ __forceinline__ void lds_n(const __nv_bfloat16* p, float (&x)[2]) {
+  const uint32_t u = *reinterpret_cast<const uint32_t*>(p);
+  x[0] = __uint_as_float(u << 16); x[1] = __uint_as_float(u & 0xffff0000u);
+}
+
+__device__ int g_chunk_bwd_timeout = 0;      // set if a chunk's inputs never arrived
+constexpr uint32_t kWaitLimit = 1u << 22;
+
+// Shared-memory layout (bytes).  NBUF chunk buffers of raw inputs, bulk-copied
+// (g in fp32, turned into exp(g) in place once the chunk has landed; k, q, v and
+// dout in their storage type; beta written by threads), then the per-warp e_t,
+// the per-warp state ring and one mbarrier per buffer.  bf16 inputs use two
+// buffers (the next chunk loads while this one is processed), fp32 inputs one.
+template <typename Tin, int DK>
 struct BwdSmem {
-  static constexpr int G = 0;                         // [64][DK] log-decay
-  static constexpr int K = G + kChunk * DK;           // [64][DK]
-  static constexpr int Q = K + kChunk * DK;           // [64][DK]
-  static constexpr int V = Q + kChunk * DK;           // [64][CPC] this CTA's columns
-  static constexpr int DO = V + kChunk * CPC;         // [64][CPC]
-  static constexpr int BETA = DO + kChunk * CPC;      // [64]
-  static constexpr int E = BETA + kChunk;             // [WPC][64][NC]
-  static constexpr int RINGB = E + WPC * kChunk * NC; // [WPC][RING][DK * NC]
-  static constexpr int TOTAL = RINGB + WPC * RING * DK * NC;
-  static constexpr size_t BYTES = (size_t)TOTAL * sizeof(float);
+  static constexpr int NBUF = sizeof(Tin) == 2 ? 2 : 1;
+  static constexpr int SI = (int)sizeof(Tin);
+  static constexpr int G = 0;                                   // fp32 [64][DK]
+  static constexpr int K = G + kChunk * DK * 4;                 // Tin [64][DK]
+  static constexpr int Q = K + kChunk * DK * SI;                // Tin [64][DK]
+  static constexpr int V = Q + kChunk * DK * SI;                // Tin [64][CPC]
+  static constexpr int DO = V + kChunk * CPC * SI;              // Tin [64][CPC]
+  static constexpr int BETA = DO + kChunk * CPC * SI;           // fp32 [64]
+  static constexpr int BUF = BETA + kChunk * 4;                 // bytes per buffer
+  static constexpr int E = NBUF * BUF;                          // fp32 [WPC][64][NC]
+  static constexpr int RINGB = E + WPC * kChunk * NC * 4;       // fp32 [WPC][RING][DK * NC]
+  static constexpr int BAR = RINGB + WPC * RING * DK * NC * 4;  // uint64 [NBUF]
+  static constexpr size_t BYTES = (size_t)BAR + 8 * NBUF;
+  static_assert(BUF % 16 == 0 && CPC * SI % 16 == 0, "bulk copies need 16-byte pieces");
+  static constexpr uint32_t bytes(int L, bool rev) {
+    return (uint32_t)L * (DK * 4 + DK * SI + CPC * SI + (rev ? DK * SI + CPC * SI : 0));
+  }
 };
 
-// Stage tokens [0, L) of a chunk whose first token row is `rowbase` (head h): g, k
-// and this CTA's CPC columns of v; with `rev` also q and dout.
+// Start the bulk copies of tokens [0, L) of a chunk (first token row `rowbase`,
+// head h) into buffer `buf`: g, k and this CTA's CPC columns of v, with `rev`
+// also q and dout; completion on `bar`, whose transaction count the caller has
+// set to BwdSmem::bytes(L, rev).  Two threads per token.  Returns beta of the
+// calling thread's token (threads 0 .. L-1), else 0.
 template <typename Tin, int DK, int DV>
-__device__ __forceinline__ void stage_chunk(float* sm, const Tin* __restrict__ q,
-                                            const Tin* __restrict__ k, const Tin* __restrict__ v,
-                                            const float* __restrict__ g,
-                                            const float* __restrict__ beta,
-                                            const Tin* __restrict__ dout, long long rowbase, int L,
-                                            int H, int h, int cta_c0, bool rev) {
-  using S = BwdSmem<DK>;
-  const int tid = threadIdx.x;
-  constexpr int P8 = DK / 8;                  // 8-element pieces per row
-  for (int i = tid; i < L * P8; i += NTB) {
-    const int t = i / P8, c = (i % P8) * 8;
-    const long long src = ((rowbase + t) * H + h) * (long long)DK + c;
-    float x[8];
-    ld8(g + src, x);
-    st8(sm + S::G + t * DK + c, x);
-    gld8(k + src, x);
-    st8(sm + S::K + t * DK + c, x);
-    if (rev) {
-      gld8(q + src, x);
-      st8(sm + S::Q + t * DK + c, x);
+__device__ __forceinline__ float issue_chunk(char* buf, uint64_t* bar, const Tin* __restrict__ q,
+                                             const Tin* __restrict__ k,
+                                             const Tin* __restrict__ v,
+                                             const float* __restrict__ g,
+                                             const float* __restrict__ beta,
+                                             const Tin* __restrict__ dout, long long rowbase,
+                                             int L, int H, int h, int cta_c0, bool rev) {
+  using S = BwdSmem<Tin, DK>;
+  static_assert(NTB == 2 * kChunk, "two threads per token");
+  const int t = threadIdx.x & (kChunk - 1), part = threadIdx.x / kChunk;
+  float b = 0.f;
+  if (t < L) {
+    const long long row = (rowbase + t) * H + h;
+    if (part == 0) {
+      bulk_g2s(buf + S::G + t * DK * 4, g + row * DK, DK * 4, bar);
+      bulk_g2s(buf + S::K + t * DK * S::SI, k + row * DK, DK * S::SI, bar);
+      if (rev) bulk_g2s(buf + S::Q + t * DK * S::SI, q + row * DK, DK * S::SI, bar);
+      b = beta[row];
+    } else {
+      bulk_g2s(buf + S::V + t * CPC * S::SI, v + row * DV + cta_c0, CPC * S::SI, bar);
+      if (rev) bulk_g2s(buf + S::DO + t * CPC * S::SI, dout + row * DV + cta_c0, CPC * S::SI, bar);
     }
   }
-  constexpr int PV = CPC / 8;
-  for (int i = tid; i < L * PV; i += NTB) {
-    const int t = i / PV, c = (i % PV) * 8;
-    const long long src = ((rowbase + t) * H + h) * (long long)DV + cta_c0 + c;
-    float x[8];
-    gld8(v + src, x);
-    st8(sm + S::V + t * CPC + c, x);
-    if (rev) {
-      gld8(dout + src, x);
-      st8(sm + S::DO + t * CPC + c, x);
-    }
-  }
-  for (int t = tid; t < L; t += NTB) sm[S::BETA + t] = beta[(rowbase + t) * H + h];
+  return b;
 }
 
 // One CTA per (column block of CPC state columns, head, sequence).
@@ -187,17 +208,19 @@ kda_chunk_bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
   constexpr int SLICE = DK * NC;        // floats in a warp's state slice
   constexpr int NB = DV / CPC;          // CTAs per (sequence, head)
   constexpr long long SZ = (long long)DK * DV;
-  using SM = BwdSmem<DK>;
-  extern __shared__ __align__(16) float sm[];
+  using SM = BwdSmem<Tin, DK>;
+  constexpr int NBUF = SM::NBUF;
+  extern __shared__ __align__(16) char smc[];
 
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int bx = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
   const int cta_c0 = bx * CPC, wc = warp * NC;
   const int c0 = cta_c0 + wc;           // this warp's first state column
   const int rl = lane * R;              // this lane's first state row
   long long row0, t_beg, t_end;
   seq_range(cu_seqlens, s, T, row0, t_beg, t_end);
-  const int nch = (int)chunk_count(t_end - t_beg);
+  const long long len = t_end - t_beg;
+  const int nch = (int)chunk_count(len);
   const long long sidx = ((long long)s * H + h) * SZ;
   // checkpoint of chunk c: ckpt + ck0 + c * H * SZ (chunks of all sequences numbered
   // consecutively, heads inside a chunk, warp slices inside a head)
@@ -205,202 +228,239 @@ kda_chunk_bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
       (seq_chunk_base(cu_seqlens, s, T) * H + h) * SZ + (long long)(bx * WPC + warp) * SLICE;
   // pre-token state of token t of the current chunk: cs + t * WPC * SLICE
   float* const cs = cst + ((((long long)s * H + h) * NB + bx) * kChunk * WPC + warp) * SLICE;
-  float* const e_sm = sm + SM::E + warp * kChunk * NC;
-  float* const ring = sm + SM::RINGB + warp * RING * SLICE;
+  float* const e_sm = reinterpret_cast<float*>(smc + SM::E) + warp * kChunk * NC;
+  float* const ring = reinterpret_cast<float*>(smc + SM::RINGB) + warp * RING * SLICE;
+  uint64_t* const bars = reinterpret_cast<uint64_t*>(smc + SM::BAR);
 
-  // a warp's state slice: lane element (i, j) in float4 m = 2 i + j / 4, at (m * 32 + lane) * 4
+  // a warp's state slice: lane row i (NC = 4 columns) is float4 number i, at (i * 32 + lane) * 4
   auto st_slice = [&](float* base, const float (&X)[R][NC]) {
 #pragma unroll
-    for (int i = 0; i < R; ++i)
-#pragma unroll
-      for (int jq = 0; jq < 2; ++jq)
-        *reinterpret_cast<float4*>(base + ((i * 2 + jq) * 32 + lane) * 4) =
-            make_float4(X[i][jq * 4], X[i][jq * 4 + 1], X[i][jq * 4 + 2], X[i][jq * 4 + 3]);
+    for (int i = 0; i < R; ++i) st4(base + (i * 32 + lane) * 4, X[i]);
   };
   auto ld_slice = [&](const float* base, float (&X)[R][NC]) {
 #pragma unroll
-    for (int i = 0; i < R; ++i)
-#pragma unroll
-      for (int jq = 0; jq < 2; ++jq) {
-        const float4 t4 = *reinterpret_cast<const float4*>(base + ((i * 2 + jq) * 32 + lane) * 4);
-        X[i][jq * 4] = t4.x; X[i][jq * 4 + 1] = t4.y;
-        X[i][jq * 4 + 2] = t4.z; X[i][jq * 4 + 3] = t4.w;
-      }
-  };
-  // one forward step on staged token t: S <- a + beta k e^T, e = v - a^T k
-  auto fwd = [&](float (&S)[R][NC], int t, float (&e)[NC]) {
-    float gl[R], kr[R];
-    Rows<R>::ld(sm + SM::G + t * DK + rl, gl);
-    Rows<R>::ld(sm + SM::K + t * DK + rl, kr);
-    float p[NC];
-#pragma unroll
-    for (int j = 0; j < NC; ++j) p[j] = 0.f;
-#pragma unroll
-    for (int i = 0; i < R; ++i) {
-      const float al = __expf(gl[i]);
-#pragma unroll
-      for (int j = 0; j < NC; ++j) {
-        S[i][j] *= al;
-        p[j] = fmaf(S[i][j], kr[i], p[j]);
-      }
-    }
-    float tot[NC];
-    colsum8(p, tot, lane);
-    float vv[NC];
-    ld8(sm + SM::V + t * CPC + wc, vv);
-    const float b = sm[SM::BETA + t];
-#pragma unroll
-    for (int j = 0; j < NC; ++j) {
-      e[j] = vv[j] - tot[j];
-      const float u = b * e[j];
-#pragma unroll
-      for (int i = 0; i < R; ++i) S[i][j] = fmaf(kr[i], u, S[i][j]);
-    }
+    for (int i = 0; i < R; ++i) ld4(base + (i * 32 + lane) * 4, X[i]);
   };
 
-  // ---- forward sweep: the warp's slice of S at every chunk start
-  float S[R][NC], e[NC];
+  // Jobs: the forward sweep's chunks 0 .. nch-2, then the reverse sweep's chunks
+  // nch-1 .. 0.  Job j's inputs sit in buffer j % NBUF.
+  const int nf = nch > 0 ? nch - 1 : 0;
+  const int njobs = nf + nch;
+  auto job_chunk = [&](int j) { return j < nf ? j : nch - 1 - (j - nf); };
+  auto job_len = [&](int j) {
+    return (int)min((long long)kChunk, len - (long long)job_chunk(j) * kChunk);
+  };
+  auto job_row = [&](int j) { return row0 + t_beg + (long long)job_chunk(j) * kChunk; };
+  auto issue = [&](int j) {
+    const int b = j % NBUF;
+    return issue_chunk<Tin, DK, DV>(smc + b * SM::BUF, &bars[b], q, k, v, g, beta, dout,
+                                    job_row(j), job_len(j), H, h, cta_c0, j >= nf);
+  };
+
+  if (tid == 0) {
+#pragma unroll
+    for (int b = 0; b < NBUF; ++b) mbar_init(&bars[b], 1);
+    fence_mbar_init();
+    if (njobs > 0) mbar_arrive_expect_tx(&bars[0], SM::bytes(job_len(0), 0 >= nf));
+  }
+  __syncthreads();
+  float bnext = njobs > 0 ? issue(0) : 0.f;
+  uint32_t parity = 0;                  // bit b: parity of buffer b's next completion
+  bool stalled = false;                 // a wait expired (diagnostic flag set)
+
+  float S[R][NC], e[NC], G[R][NC];
 #pragma unroll
   for (int i = 0; i < R; ++i) {
     if (h0) {
-      ld8(h0 + sidx + (long long)(rl + i) * DV + c0, S[i]);
+      ld4(h0 + sidx + (long long)(rl + i) * DV + c0, S[i]);
     } else {
 #pragma unroll
       for (int j = 0; j < NC; ++j) S[i][j] = 0.f;
     }
-  }
-#pragma unroll 1
-  for (int c = 0; c < nch; ++c) {
-    st_slice(ckpt + ck0 + (long long)c * H * SZ, S);
-    if (c == nch - 1) break;            // the last chunk is re-run by the reverse sweep
-    const long long rb = row0 + t_beg + (long long)c * kChunk;
-    __syncthreads();                    // the previous chunk's staged inputs are consumed
-    stage_chunk<Tin, DK, DV>(sm, q, k, v, g, beta, dout, rb, kChunk, H, h, cta_c0, false);
-    __syncthreads();
-#pragma unroll 1
-    for (int t = 0; t < kChunk; ++t) fwd(S, t, e);
-  }
-
-  // ---- reverse sweep
-  float G[R][NC];
-#pragma unroll
-  for (int i = 0; i < R; ++i) {
     if (dhT) {
-      ld8(dhT + sidx + (long long)(rl + i) * DV + c0, G[i]);
+      ld4(dhT + sidx + (long long)(rl + i) * DV + c0, G[i]);
     } else {
 #pragma unroll
       for (int j = 0; j < NC; ++j) G[i][j] = 0.f;
     }
   }
+
 #pragma unroll 1
-  for (int c = nch - 1; c >= 0; --c) {
-    const long long rb = row0 + t_beg + (long long)c * kChunk;
-    const int L = (int)min((long long)kChunk, t_end - t_beg - (long long)c * kChunk);
+  for (int j = 0; j < njobs; ++j) {
+    const int b = j % NBUF;
+    char* const buf = smc + b * SM::BUF;
+    const int c = job_chunk(j), L = job_len(j);
+    const bool rev = j >= nf;
+    const long long rb = job_row(j);
+    // wait for the chunk, publish beta and exp(g), start the next chunk's copies
+    if (!stalled && !mbar_wait(&bars[b], (parity >> b) & 1u, kWaitLimit)) {
+      stalled = true;                   // wait no more: finish without blocking
+      atomicExch(&g_chunk_bwd_timeout, 1);
+    }
+    parity ^= 1u << b;
+    float* const al_s = reinterpret_cast<float*>(buf + SM::G);
+    float* const beta_s = reinterpret_cast<float*>(buf + SM::BETA);
+    if (tid < L) beta_s[tid] = bnext;
+    for (int i = tid; i < L * DK / 4; i += NTB) {
+      float4 x = reinterpret_cast<float4*>(al_s)[i];
+      x.x = __expf(x.x); x.y = __expf(x.y); x.z = __expf(x.z); x.w = __expf(x.w);
+      reinterpret_cast<float4*>(al_s)[i] = x;
+    }
+    if (NBUF == 2 && tid == 0 && j + 1 < njobs)
+      mbar_arrive_expect_tx(&bars[b ^ 1], SM::bytes(job_len(j + 1), j + 1 >= nf));
     __syncthreads();
-    stage_chunk<Tin, DK, DV>(sm, q, k, v, g, beta, dout, rb, L, H, h, cta_c0, true);
-    __syncthreads();
-    ld_slice(ckpt + ck0 + (long long)c * H * SZ, S);
-    // re-run the chunk: pre-token states to scratch, e_t to shared, dq_t = S_t do_t
-#pragma unroll 1
-    for (int t = 0; t < L; ++t) {
-      st_slice(cs + (long long)t * WPC * SLICE, S);
-      fwd(S, t, e);
-      if (lane == 0) st8(e_sm + t * NC, e);
-      float dov[NC];
-      ld8(sm + SM::DO + t * CPC + wc, dov);
-      float dqp[R];
+    if (NBUF == 2 && j + 1 < njobs) bnext = issue(j + 1);
+
+    const Tin* const k_s = reinterpret_cast<const Tin*>(buf + SM::K);
+    const Tin* const q_s = reinterpret_cast<const Tin*>(buf + SM::Q);
+    const Tin* const v_s = reinterpret_cast<const Tin*>(buf + SM::V);
+    const Tin* const do_s = reinterpret_cast<const Tin*>(buf + SM::DO);
+    // one forward step on token t: S <- a + beta k e^T, e = v - a^T k
+    auto fwd = [&](int t) {
+      float al[R], kr[R];
+      lds_n(al_s + t * DK + rl, al);
+      lds_n(k_s + t * DK + rl, kr);
+      float p[NC];
 #pragma unroll
-      for (int i = 0; i < R; ++i) {
-        float acc = 0.f;
+      for (int jj = 0; jj < NC; ++jj) p[jj] = 0.f;
 #pragma unroll
-        for (int j = 0; j < NC; ++j) acc = fmaf(S[i][j], dov[j], acc);
-        dqp[i] = acc;
-      }
-      Rows<R>::add(dq + ((rb + t) * H + h) * DK + rl, dqp);
-    }
-    __syncwarp();
-    // walk the chunk backwards; pre-token states arrive through the ring
+      for (int i = 0; i < R; ++i)
 #pragma unroll
-    for (int d = 0; d < RING; ++d) {
-      const int t = L - 1 - d;
-      if (t >= 0) {
-#pragma unroll
-        for (int m = 0; m < NV; ++m)
-          cp_async16(ring + (t % RING) * SLICE + (m * 32 + lane) * 4,
-                     cs + (long long)t * WPC * SLICE + (m * 32 + lane) * 4, 16);
-      }
-      cp_async_commit();
-    }
-#pragma unroll 1
-    for (int t = L - 1; t >= 0; --t) {
-      cp_async_wait_group<RING - 1>();
-      float A[R][NC];
-      ld_slice(ring + (t % RING) * SLICE, A);
-      float gl[R], kr[R], qr[R], dov[NC], ee[NC];
-      Rows<R>::ld(sm + SM::G + t * DK + rl, gl);
-      Rows<R>::ld(sm + SM::K + t * DK + rl, kr);
-      Rows<R>::ld(sm + SM::Q + t * DK + rl, qr);
-      ld8(sm + SM::DO + t * CPC + wc, dov);
-      ld8(e_sm + t * NC, ee);
-      const float b = sm[SM::BETA + t];
-      float al[R], pw[NC];
-#pragma unroll
-      for (int j = 0; j < NC; ++j) pw[j] = 0.f;
-#pragma unroll
-      for (int i = 0; i < R; ++i) {
-        al[i] = __expf(gl[i]);
-#pragma unroll
-        for (int j = 0; j < NC; ++j) {
-          A[i][j] *= al[i];
-          G[i][j] = fmaf(qr[i], dov[j], G[i][j]);
-          pw[j] = fmaf(G[i][j], kr[i], pw[j]);
+        for (int jj = 0; jj < NC; ++jj) {
+          S[i][jj] *= al[i];
+          p[jj] = fmaf(S[i][jj], kr[i], p[jj]);
         }
-      }
-      float w[NC];
-      colsum8(pw, w, lane);
-      float de[NC], dbp = 0.f;
+      float tot[NC];
+      colsum4(p, tot, lane);
+      float vv[NC];
+      lds_n(v_s + t * CPC + wc, vv);
+      const float bt = beta_s[t];
 #pragma unroll
-      for (int j = 0; j < NC; ++j) {
-        de[j] = b * w[j];
-        dbp = fmaf(w[j], ee[j], dbp);
-      }
-      const long long tok = (rb + t) * H + h;
-      if (lane == 0) {
-        st8(dvo + tok * DV + c0, de);
-        atomicAdd(dbeta + tok, dbp);
-      }
-      float dkp[R], dgp[R];
+      for (int jj = 0; jj < NC; ++jj) {
+        e[jj] = vv[jj] - tot[jj];
+        const float u = bt * e[jj];
 #pragma unroll
-      for (int i = 0; i < R; ++i) {
-        float a1 = 0.f, a2 = 0.f, a3 = 0.f;
+        for (int i = 0; i < R; ++i) S[i][jj] = fmaf(kr[i], u, S[i][jj]);
+      }
+    };
+
+    if (!rev) {
+      // forward sweep: checkpoint, then the chunk's 64 tokens
+      st_slice(ckpt + ck0 + (long long)c * H * SZ, S);
+#pragma unroll 1
+      for (int t = 0; t < L; ++t) fwd(t);
+    } else {
+      // the last chunk starts from the state the forward sweep ended with
+      if (c != nch - 1) ld_slice(ckpt + ck0 + (long long)c * H * SZ, S);
+      // re-run the chunk: pre-token states to scratch, e_t to shared, dq_t = S_t do_t
+#pragma unroll 1
+      for (int t = 0; t < L; ++t) {
+        st_slice(cs + (long long)t * WPC * SLICE, S);
+        fwd(t);
+        if (lane == 0) st4(e_sm + t * NC, e);
+        float dov[NC];
+        lds_n(do_s + t * CPC + wc, dov);
+        float dqp[R];
 #pragma unroll
-        for (int j = 0; j < NC; ++j) {
-          a1 = fmaf(G[i][j], ee[j], a1);
-          a2 = fmaf(A[i][j], de[j], a2);
-          const float da = fmaf(-kr[i], de[j], G[i][j]);
-          a3 = fmaf(da, A[i][j], a3);
-          G[i][j] = al[i] * da;
+        for (int i = 0; i < R; ++i) {
+          float acc = 0.f;
+#pragma unroll
+          for (int jj = 0; jj < NC; ++jj) acc = fmaf(S[i][jj], dov[jj], acc);
+          dqp[i] = acc;
         }
-        dkp[i] = b * a1 - a2;
-        dgp[i] = a3;
+        Rows<R>::add(dq + ((rb + t) * H + h) * DK + rl, dqp);
       }
-      Rows<R>::add(dk + tok * DK + rl, dkp);
-      Rows<R>::add(dg + tok * DK + rl, dgp);
-      const int tn = t - RING;
-      if (tn >= 0) {
+      __syncwarp();
+      // walk the chunk backwards; pre-token states arrive through the ring
 #pragma unroll
-        for (int m = 0; m < NV; ++m)
-          cp_async16(ring + (tn % RING) * SLICE + (m * 32 + lane) * 4,
-                     cs + (long long)tn * WPC * SLICE + (m * 32 + lane) * 4, 16);
+      for (int d = 0; d < RING; ++d) {
+        const int t = L - 1 - d;
+        if (t >= 0) {
+#pragma unroll
+          for (int m = 0; m < NV; ++m)
+            cp_async16(ring + (t % RING) * SLICE + (m * 32 + lane) * 4,
+                       cs + (long long)t * WPC * SLICE + (m * 32 + lane) * 4, 16);
+        }
+        cp_async_commit();
       }
-      cp_async_commit();
+#pragma unroll 1
+      for (int t = L - 1; t >= 0; --t) {
+        cp_async_wait_group<RING - 1>();
+        float A[R][NC];                 // pre-token state S_{t-1} (a = Diag(alpha) A)
+        ld_slice(ring + (t % RING) * SLICE, A);
+        float al[R], kr[R], qr[R], dov[NC], ee[NC];
+        lds_n(al_s + t * DK + rl, al);
+        lds_n(k_s + t * DK + rl, kr);
+        lds_n(q_s + t * DK + rl, qr);
+        lds_n(do_s + t * CPC + wc, dov);
+        ld4(e_sm + t * NC, ee);
+        const float bt = beta_s[t];
+        float pw[NC];
+#pragma unroll
+        for (int jj = 0; jj < NC; ++jj) pw[jj] = 0.f;
+#pragma unroll
+        for (int i = 0; i < R; ++i)
+#pragma unroll
+          for (int jj = 0; jj < NC; ++jj) {
+            G[i][jj] = fmaf(qr[i], dov[jj], G[i][jj]);
+            pw[jj] = fmaf(G[i][jj], kr[i], pw[jj]);
+          }
+        float w[NC];
+        colsum4(pw, w, lane);
+        float de[NC], dbp = 0.f;
+#pragma unroll
+        for (int jj = 0; jj < NC; ++jj) {
+          de[jj] = bt * w[jj];
+          dbp = fmaf(w[jj], ee[jj], dbp);
+        }
+        const long long tok = (rb + t) * H + h;
+        if (lane == 0) {
+          st4(dvo + tok * DV + c0, de);
+          atomicAdd(dbeta + tok, dbp);
+        }
+        // dk = beta G e - a de;  dg = rowsum((G - k de^T) * a);  G <- Diag(alpha)(G - k de^T),
+        // with a = alpha_i A_ij: the row factor alpha_i is applied to the row sums
+        float dkp[R], dgp[R];
+#pragma unroll
+        for (int i = 0; i < R; ++i) {
+          float a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+          for (int jj = 0; jj < NC; ++jj) {
+            a1 = fmaf(G[i][jj], ee[jj], a1);
+            a2 = fmaf(A[i][jj], de[jj], a2);
+            const float da = fmaf(-kr[i], de[jj], G[i][jj]);
+            a3 = fmaf(da, A[i][jj], a3);
+            G[i][jj] = al[i] * da;
+          }
+          dkp[i] = fmaf(bt, a1, -al[i] * a2);
+          dgp[i] = al[i] * a3;
+        }
+        Rows<R>::add(dk + tok * DK + rl, dkp);
+        Rows<R>::add(dg + tok * DK + rl, dgp);
+        const int tn = t - RING;
+        if (tn >= 0) {
+#pragma unroll
+          for (int m = 0; m < NV; ++m)
+            cp_async16(ring + (tn % RING) * SLICE + (m * 32 + lane) * 4,
+                       cs + (long long)tn * WPC * SLICE + (m * 32 + lane) * 4, 16);
+        }
+        cp_async_commit();
+      }
+      __syncwarp();
     }
-    __syncwarp();
+    // this buffer is refilled by bulk copies (async proxy) after the next barrier
+    fence_async_smem();
+    if (NBUF == 1 && j + 1 < njobs) {
+      __syncthreads();
+      if (tid == 0) mbar_arrive_expect_tx(&bars[0], SM::bytes(job_len(j + 1), j + 1 >= nf));
+      __syncthreads();
+      bnext = issue(j + 1);
+    }
   }
   cp_async_wait_all();
   if (dh0) {
 #pragma unroll
-    for (int i = 0; i < R; ++i) st8(dh0 + sidx + (long long)(rl + i) * DV + c0, G[i]);
+    for (int i = 0; i < R; ++i) st4(dh0 + sidx + (long long)(rl + i) * DV + c0, G[i]);
   }
 }
 
@@ -410,7 +470,7 @@ cudaError_t launch_t(const void* q, const void* k, const void* v, const float* g
                      const float* dhT, float* dq, float* dk, float* dv, float* dg, float* dbeta,
                      float* dh0, float* ckpt, float* cst, int B, int T, int H,
                      cudaStream_t stream) {
-  constexpr size_t smem = BwdSmem<DK>::BYTES;
+  constexpr size_t smem = BwdSmem<Tin, DK>::BYTES;
   const cudaError_t ea = cudaFuncSetAttribute(kda_chunk_bwd_kernel<Tin, DK, DV>,
                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                                               (int)smem);
