@@ -364,6 +364,56 @@ def grouped_leg(args, world, rank, dev, stream, barrier, hbm, G=64):
             "algorithmic_bytes_per_call": bytes_call, "gbs": gbs, "frac_of_hbm_peak": gbs / hbm}
 
 
+def fused_leg(args, world, rank, dev, stream, barrier, hbm, W=4):
+    """The headline prefill with the q/k short convolution + L2 norm and the output
+    gate fused (kda_chunk_fwd_fused): K timed calls on three resident input sets."""
+    import torch
+
+    import gated_delta_rule_74_b200 as kda
+    import kda_inputs as ki
+
+    spec = ki.PREFILL_SPECS[args.workload]
+    if spec.dtype != "bf16":
+        return None
+    sets = []
+    for i in range(3):
+        x = ki.make_fused_prefill(spec, W=W, seed=spec.seed + 1000 * rank + 800 + i)
+        d = {n: (t.to(dev) if isinstance(t, torch.Tensor) else t) for n, t in x.items()}
+        d["out"] = torch.empty_like(d["v"])
+        d["hT"] = torch.empty(x["B"], x["H"], x["dk"], x["dv"], device=dev)
+        sets.append(d)
+    x0 = sets[0]
+    rows = x0["T"] if x0["cu_seqlens"] is not None else x0["B"] * x0["T"]
+    H, dk, dv = x0["H"], x0["dk"], x0["dv"]
+    # raw q, k, v, gate in; g, beta; out; taps and states
+    bytes_call = rows * H * ((2 * dk + 2 * dv) * 2 + 4 * dk + 4 + dv * 2) + \
+        2 * H * dk * W * 4 + x0["B"] * H * 4 * dk * dv * (int(x0["h0"] is not None) + 1)
+
+    def call(i):
+        d = sets[i % 3]
+        kda.kda_chunk_fwd_fused(d["q_raw"], d["k_raw"], d["v"], d["g"], d["beta"],
+                                conv_q=d["conv_q"], conv_k=d["conv_k"], gate=d["gate"],
+                                h0=d["h0"], cu_seqlens=d["cu_seqlens"], out=d["out"], hT=d["hT"],
+                                stream=stream)
+
+    for i in range(args.warmup):
+        call(i)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        call(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = _max_over_ranks(e0.elapsed_time(e1), world, dev) / args.steps
+    gbs = bytes_call / (ms / 1e3) / 1e9
+    return {"call": f"kda_chunk_fwd_fused (conv W={W}, L2 norm, output gate)",
+            "tokens_per_s": rows * world / (ms / 1e3), "ms_per_call": ms,
+            "algorithmic_bytes_per_call": bytes_call, "gbs": gbs, "frac_of_hbm_peak": gbs / hbm}
+
+
 def bwd_leg(args, world, rank, dev, stream, barrier, hbm):
     """The prefill backward (kda_chunk_bwd) on the headline workload: a few timed
     calls on two resident input sets, fp32 gradients of sum(out*dout) + sum(hT*dhT)."""
@@ -631,6 +681,9 @@ def run_ours(args, world, rank, local):
     grp = None
     if not args.decode_only and not args.no_grouped:
         grp = grouped_leg(args, world, rank, dev, stream, barrier, hbm)
+    fzd = None
+    if not args.decode_only and not args.no_fused_prep:
+        fzd = fused_leg(args, world, rank, dev, stream, barrier, hbm)
     bwd = None
     if not args.decode_only and not args.no_bwd:
         bwd = bwd_leg(args, world, rank, dev, stream, barrier, hbm)
@@ -662,6 +715,7 @@ def run_ours(args, world, rank, local):
         "config": _config(args, pf["x0"], world),
         "roofline": roof,
         "prefill_decay_g64": grp,
+        "prefill_fused_prep": fzd,
         "prefill_bwd": bwd,
         "decode": dec, "e2e": pf["e2e"], "gpu_launches": pf["launches"],
         "clocks": pf["clocks"], "cpu_baseline": cpu,
@@ -681,6 +735,8 @@ def main():
     ap.add_argument("--workload", default="metric", choices=["metric", "cfg1", "cfg2", "cfg3"])
     ap.add_argument("--decode-steps", type=int, default=100)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-fused-prep", action="store_true",
+                    help="skip the fused conv + norm + gate prefill (kda_chunk_fwd_fused) leg")
     ap.add_argument("--no-bwd", action="store_true",
                     help="skip the prefill backward (kda_chunk_bwd) leg")
     ap.add_argument("--bwd-steps", type=int, default=5,

@@ -19,7 +19,7 @@ from typing import Optional
 
 import torch
 
-__all__ = ["kda_chunk_fwd", "kda_chunk_bwd", "kda_decode_step", "kda_decode_tokens", "kda_status_string", "kda_version",
+__all__ = ["kda_chunk_fwd", "kda_chunk_fwd_fused", "kda_chunk_bwd", "kda_decode_step", "kda_decode_tokens", "kda_status_string", "kda_version",
            "kda_launch_count",
            "lib", "library_path", "header_symbols", "KdaError",
            "KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED", "KDA_ERR_CUDA",
@@ -72,6 +72,9 @@ def lib() -> ctypes.CDLL:
         L.kda_decode_tokens_grouped.restype = ctypes.c_int
         L.kda_chunk_fwd_grouped.argtypes = [vp, vp, vp, fp, fp, fp, vp, vp, fp] + [ip] * 7 + [vp]
         L.kda_chunk_fwd_grouped.restype = ctypes.c_int
+        L.kda_chunk_fwd_fused.argtypes = [vp, vp, vp, fp, fp, ip, fp, fp, vp, fp, vp, vp, fp] + \
+            [ip] * 6 + [vp]
+        L.kda_chunk_fwd_fused.restype = ctypes.c_int
         L.kda_chunk_bwd.argtypes = [vp, vp, vp, fp, fp, fp, vp, vp, fp,
                                     fp, fp, fp, fp, fp, fp] + [ip] * 6 + [vp]
         L.kda_chunk_bwd.restype = ctypes.c_int
@@ -214,6 +217,64 @@ def kda_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Te
                                          nseq, T, H, dk, dv, G, dt, _stream(stream))
     if rc != KDA_OK:
         raise KdaError("kda_chunk_fwd", rc)
+    return out, hT
+
+
+def kda_chunk_fwd_fused(q_raw: torch.Tensor, k_raw: torch.Tensor, v: torch.Tensor,
+                        g: torch.Tensor, beta: torch.Tensor,
+                        conv_q: Optional[torch.Tensor] = None,
+                        conv_k: Optional[torch.Tensor] = None,
+                        gate: Optional[torch.Tensor] = None, h0: Optional[torch.Tensor] = None,
+                        cu_seqlens: Optional[torch.Tensor] = None,
+                        out: Optional[torch.Tensor] = None, hT: Optional[torch.Tensor] = None,
+                        output_final_state: bool = True, stream=None):
+    """KDA prefill with the q/k prep and the output gate fused (bf16 only):
+    q = dk^-1/2 n(conv_q * q_raw), k = n(conv_k * k_raw) (causal per-channel convolutions
+    of width W, conv_* [H, dk, W] f32, n = L2 normalisation per token and head),
+    out = o * sigmoid(gate) (gate [B,T,H,dv] bf16 or None).  Returns (out, hT)."""
+    if q_raw.dim() != 4:
+        raise ValueError("q_raw must be [B, T, H, dk]")
+    Bt, T, H, dk = q_raw.shape
+    dv = v.shape[-1]
+    dt = _DTYPES.get(q_raw.dtype)
+    if dt is None:
+        raise ValueError(f"unsupported dtype {q_raw.dtype}")
+    _check("q_raw", q_raw)
+    _check("k_raw", k_raw, q_raw.dtype, (Bt, T, H, dk))
+    _check("v", v, q_raw.dtype, (Bt, T, H, dv))
+    _check("g", g, torch.float32, (Bt, T, H, dk))
+    _check("beta", beta, torch.float32, (Bt, T, H))
+    W = 0
+    if (conv_q is None) != (conv_k is None):
+        raise ValueError("give both conv_q and conv_k, or neither")
+    if conv_q is not None:
+        W = conv_q.shape[-1]
+        _check("conv_q", conv_q, torch.float32, (H, dk, W))
+        _check("conv_k", conv_k, torch.float32, (H, dk, W))
+    if gate is not None:
+        _check("gate", gate, q_raw.dtype, (Bt, T, H, dv))
+    if cu_seqlens is not None:
+        _check("cu_seqlens", cu_seqlens, torch.int32)
+        if Bt != 1:
+            raise ValueError("packed inputs (cu_seqlens) must have B == 1")
+        nseq = cu_seqlens.numel() - 1
+    else:
+        nseq = Bt
+    if h0 is not None:
+        _check("h0", h0, torch.float32, (nseq, H, dk, dv))
+    if out is None:
+        out = torch.empty((Bt, T, H, dv), dtype=q_raw.dtype, device=q_raw.device)
+    _check("out", out, q_raw.dtype, (Bt, T, H, dv))
+    if hT is None and output_final_state:
+        hT = torch.empty((nseq, H, dk, dv), dtype=torch.float32, device=q_raw.device)
+    if hT is not None:
+        _check("hT", hT, torch.float32, (nseq, H, dk, dv))
+    rc = lib().kda_chunk_fwd_fused(_ptr(q_raw), _ptr(k_raw), _ptr(v), _ptr(conv_q), _ptr(conv_k),
+                                   W, _ptr(g), _ptr(beta), _ptr(gate), _ptr(h0),
+                                   _ptr(cu_seqlens), _ptr(out), _ptr(hT), nseq, T, H, dk, dv, dt,
+                                   _stream(stream))
+    if rc != KDA_OK:
+        raise KdaError("kda_chunk_fwd_fused", rc)
     return out, hT
 
 

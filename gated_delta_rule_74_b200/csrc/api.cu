@@ -131,6 +131,34 @@ int kda_decode_tokens_grouped(const void* q, const void* k, const void* v, const
                             in_dtype, stream);
 }
 
+int kda_chunk_fwd_fused(const void* q_raw, const void* k_raw, const void* v, const float* conv_q,
+                        const float* conv_k, int conv_w, const float* g, const float* beta,
+                        const void* gate, const float* h0, const int32_t* cu_seqlens, void* out,
+                        float* hT, int B, int T, int H, int dk, int dv, int in_dtype,
+                        void* stream) {
+  if (B < 1 || T < 0 || H < 1) return KDA_ERR_INVALID_ARG;
+  if (in_dtype != KDA_BF16 && in_dtype != KDA_F32) return KDA_ERR_INVALID_ARG;
+  if ((conv_q == nullptr) != (conv_k == nullptr)) return KDA_ERR_INVALID_ARG;
+  if (conv_q && (conv_w < 1 || conv_w > 4)) return KDA_ERR_INVALID_ARG;
+  const long long rows = cu_seqlens ? (long long)T : (long long)B * T;
+  if (rows > 0) {
+    if (!pointers_ok({q_raw, k_raw, v, g, beta, out}, {conv_q, conv_k, gate, h0, hT, cu_seqlens}))
+      return KDA_ERR_INVALID_ARG;
+  } else {
+    if (!pointers_ok({}, {q_raw, k_raw, v, g, beta, out, conv_q, conv_k, gate, h0, hT,
+                          cu_seqlens}))
+      return KDA_ERR_INVALID_ARG;
+  }
+  if (!head_ok(dk) || !head_ok(dv)) return KDA_ERR_UNSUPPORTED;
+  if (!kda::chunk_split_supported(dk, dv, in_dtype)) return KDA_ERR_UNSUPPORTED;
+  if (rows * H * (long long)(dk > dv ? dk : dv) > (1LL << 40)) return KDA_ERR_INVALID_ARG;
+  if ((long long)B > 65535LL || H > 65535) return KDA_ERR_UNSUPPORTED;
+  const kda::InputFusion fz{conv_q, conv_k, conv_q ? conv_w : 0, gate};
+  return status_from(kda::launch_chunk_split(q_raw, k_raw, v, g, beta, h0, cu_seqlens, out, hT, B,
+                                             T, H, dk, dv, 0, static_cast<cudaStream_t>(stream),
+                                             &fz));
+}
+
 int kda_chunk_bwd(const void* q, const void* k, const void* v, const float* g,
                   const float* beta, const float* h0, const int32_t* cu_seqlens,
                   const void* dout, const float* dhT, float* dq, float* dk, float* dv, float* dg,

@@ -97,7 +97,8 @@ constexpr uint32_t kPrepTmemCols = 256;
 // ---- state pass: shared memory and TMEM
 constexpr uint32_t S_BUF = 91136;       // record buffer stride (two buffers)
 constexpr uint32_t S_OUT = 2 * S_BUF;   // output tile [64 tokens][128] bf16
-constexpr uint32_t STATE_SMEM = S_OUT + 16384 + 1024;
+constexpr uint32_t S_GATE = S_OUT + 16384;   // output-gate tile [64 tokens][128] bf16
+constexpr uint32_t STATE_SMEM = S_GATE + 16384 + 1024;
 // [S^T | O^T] and [O^T | P] are each the accumulator of one MMA, so O^T sits
 // between S^T and P.
 constexpr uint32_t ST_S = 0;            // S^T fp32        [128 lanes x 128]
@@ -120,15 +121,40 @@ __device__ __forceinline__ void sts16(uint8_t* base, uint32_t off, uint4 v) {
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
+// Sum over the warp's 32 lanes of each of 16 per-lane values; lane l returns the
+// total of value l / 2 (transpose-reduce: halves exchanged at lane distance 16,
+// 8, 4, 2, then one butterfly step).
+__device__ __forceinline__ float rowsum16(const float (&v)[16], int lane) {
+  float x8[8], x4[4], x2[2];
+  const bool b16 = lane & 16, b8 = lane & 8, b4 = lane & 4, b2 = lane & 2;
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    x8[i] = (b16 ? v[i + 8] : v[i]) + __shfl_xor_sync(0xffffffffu, b16 ? v[i] : v[i + 8], 16);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    x4[i] = (b8 ? x8[i + 4] : x8[i]) + __shfl_xor_sync(0xffffffffu, b8 ? x8[i] : x8[i + 4], 8);
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+    x2[i] = (b4 ? x4[i + 2] : x4[i]) + __shfl_xor_sync(0xffffffffu, b4 ? x4[i] : x4[i + 2], 4);
+  float x = (b2 ? x2[1] : x2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? x2[0] : x2[1], 2);
+  return x + __shfl_xor_sync(0xffffffffu, x, 1);
+}
+
+constexpr float kNormEps2 = 1e-24f;     // (1e-12)^2: L2 norm floor of the fused q/k prep
+
 // ============================================================================
-// Prep kernel: one CTA per (chunk slot, head).
+// Prep kernel: one CTA per (chunk slot, head).  CONV: q and k are the raw
+// projections; each is convolved causally per channel (width convW <= 4, history
+// reset at the document start), L2-normalised per token, and q scaled by dk^-1/2.
 // ============================================================================
+template <bool CONV>
 __global__ void __launch_bounds__(NT, 2)
 kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
                       const bf16* __restrict__ v, const float* __restrict__ g,
                       const float* __restrict__ beta, const int32_t* __restrict__ cu_seqlens,
                       uint8_t* __restrict__ rec, int B, int T, int H, int dk, int dv, int gsh,
-                      long long nslots) {
+                      long long nslots, const float* __restrict__ conv_q,
+                      const float* __restrict__ conv_k, int convW) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   __shared__ uint64_t bar;
@@ -136,6 +162,7 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   __shared__ float s_beta[C];
   __shared__ float2 s_sum[4][64];       // per 16-row block: its total log-decay (channel pair)
   __shared__ float2 s_first[4][64];     // per 16-row block: g at its first row
+  __shared__ float s_ss[CONV ? 4 * 2 * 2 * 16 : 1];   // [block][warp][k|q][row]: sums of squares
 
   const int tid = threadIdx.x, warp = tid >> 5;
   const long long slot = blockIdx.x;
@@ -189,6 +216,7 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   const int cp = tid & 63, a = tid >> 6, c0 = 2 * cp;
   float2 gq[16];
   uint32_t kw[16], qw[16];
+  float2 kf[CONV ? 16 : 1], qf[CONV ? 16 : 1];   // CONV: fp32 convolution outputs
 #pragma unroll
   for (int e = 0; e < 16; ++e) {
     const int r = 16 * a + e;
@@ -200,13 +228,57 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
         const float gg = __ldg(g + ((rbase + r) * H + h) * (dk >> gsh) + (c0 >> gsh));
         gq[e] = make_float2(gg, gg);
       }
-      kw[e] = __ldg(reinterpret_cast<const unsigned int*>(k + idx));
-      qw[e] = __ldg(reinterpret_cast<const unsigned int*>(q + idx));
+      if constexpr (!CONV) {
+        kw[e] = __ldg(reinterpret_cast<const unsigned int*>(k + idx));
+        qw[e] = __ldg(reinterpret_cast<const unsigned int*>(q + idx));
+      }
     } else {
       gq[e] = make_float2(0.f, 0.f);
       kw[e] = 0u;
       qw[e] = 0u;
     }
+  }
+  if constexpr (CONV) {
+    // x_conv[r] = sum_i w[i] x[r - (W-1) + i]: a 4-tap window whose first 4 - W taps
+    // are zero; rows before the document start and at or after L read as zero.
+    const long long doc0 = row0 + t_beg;
+    auto conv = [&](const bf16* __restrict__ x, const float* __restrict__ w,
+                    float2 (&o)[16], int which) {
+      float2 wt[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i = j - (4 - convW);
+        wt[j] = make_float2(0.f, 0.f);
+        if (i >= 0 && c0 < dk)
+          wt[j] = make_float2(__ldg(w + ((long long)h * dk + c0) * convW + i),
+                              __ldg(w + ((long long)h * dk + c0 + 1) * convW + i));
+      }
+      // rows 16 a - 3 .. 16 a + 15, all loads issued before any use
+      uint32_t u[19];
+#pragma unroll
+      for (int m = 0; m < 19; ++m) {
+        const int r = 16 * a - 3 + m;
+        const bool ok = c0 < dk && r < L && rbase + r >= doc0;
+        u[m] = ok ? __ldg(reinterpret_cast<const unsigned int*>(x + ((rbase + r) * H + h) * dk + c0))
+                  : 0u;
+      }
+      auto raw = [&](int m) { return make_float2(bf_lo(u[m]), bf_hi(u[m])); };
+      float2 w0 = raw(0), w1 = raw(1), w2 = raw(2);
+      float ss[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float2 cur = raw(e + 3);
+        const float ox = fmaf(wt[3].x, cur.x, fmaf(wt[2].x, w2.x, fmaf(wt[1].x, w1.x, wt[0].x * w0.x)));
+        const float oy = fmaf(wt[3].y, cur.y, fmaf(wt[2].y, w2.y, fmaf(wt[1].y, w1.y, wt[0].y * w0.y)));
+        o[e] = 16 * a + e < L ? make_float2(ox, oy) : make_float2(0.f, 0.f);
+        ss[e] = fmaf(o[e].x, o[e].x, o[e].y * o[e].y);
+        w0 = w1; w1 = w2; w2 = cur;
+      }
+      const float tot = rowsum16(ss, tid & 31);
+      if ((tid & 1) == 0) s_ss[((a * 2 + (warp & 1)) * 2 + which) * 16 + ((tid & 31) >> 1)] = tot;
+    };
+    conv(k, conv_k, kf, 0);
+    conv(q, conv_q, qf, 1);
   }
 #pragma unroll
   for (int e = 1; e < 16; ++e) {
@@ -220,6 +292,19 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   tc_fence_after();
   const uint32_t tb = tmem_base_sh;
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+  if constexpr (CONV) {                 // L2 norms of this block's rows (two warps' sums)
+    const float qs = 1.f / sqrtf((float)dk);
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float ik = rsqrtf(fmaxf(s_ss[((a * 2) * 2) * 16 + e] + s_ss[((a * 2 + 1) * 2) * 16 + e],
+                                    kNormEps2));
+      const float iq = rsqrtf(fmaxf(s_ss[((a * 2) * 2 + 1) * 16 + e] +
+                                        s_ss[((a * 2 + 1) * 2 + 1) * 16 + e],
+                                    kNormEps2)) * qs;
+      kf[e].x *= ik; kf[e].y *= ik;
+      qf[e].x *= iq; qf[e].y *= iq;
+    }
+  }
 
   float2 Pr[4], Pown = make_float2(0.f, 0.f), off = make_float2(0.f, 0.f),
                run = make_float2(0.f, 0.f);
@@ -259,8 +344,14 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
         const float x = (ch ? gq[idx].y : gq[idx].x) - Pa;
         const float ell = __expf(x);
         const float rho = __expf(fminf(-x, 80.f));
-        const float kv = ch ? bf_hi(kw[idx]) : bf_lo(kw[idx]);
-        const float qv = ch ? bf_hi(qw[idx]) : bf_lo(qw[idx]);
+        float kv, qv;
+        if constexpr (!CONV) {
+          kv = ch ? bf_hi(kw[idx]) : bf_lo(kw[idx]);
+          qv = ch ? bf_hi(qw[idx]) : bf_lo(qw[idx]);
+        } else {                       // normalised above
+          kv = ch ? kf[idx].y : kf[idx].x;
+          qv = ch ? qf[idx].y : qf[idx].x;
+        }
         lk[e] = kv * ell;
         lq[e] = qv * ell;
         kr[e] = kv * rho;                      // k_i e^{P_a - G_i}
@@ -556,11 +647,33 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
 // the MMAs and the record copies (two records ahead).
 // ============================================================================
 constexpr int NT_S = 512;
+constexpr int kStorePieces = (C * 16 + NT_S - 32 - 1) / (NT_S - 32);   // 16-byte pieces per thread
+
+// hardware tanh approximation (one MUFU op; relative error about 2^-11)
+__device__ __forceinline__ float tanh_fast(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// 8 bf16 outputs times sigmoid of the 8 bf16 gate values, rounded to bf16;
+// o * sigmoid(z) = o/2 + (o/2) tanh(z/2)
+__device__ __forceinline__ uint4 apply_gate(uint4 o, uint4 z) {
+  uint32_t ow[4] = {o.x, o.y, o.z, o.w};
+  const uint32_t zw[4] = {z.x, z.y, z.z, z.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float lo = 0.5f * bf_lo(ow[i]), hi = 0.5f * bf_hi(ow[i]);
+    ow[i] = pack_bf16(fmaf(lo, tanh_fast(0.5f * bf_lo(zw[i])), lo),
+                      fmaf(hi, tanh_fast(0.5f * bf_hi(zw[i])), hi));
+  }
+  return make_uint4(ow[0], ow[1], ow[2], ow[3]);
+}
 
 __global__ void __launch_bounds__(NT_S, 1)
 kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
                       const int32_t* __restrict__ cu_seqlens, bf16* __restrict__ out, float* hT,
-                      int T, int H, int dk, int dv, long long nslots, SegArgs sa) {
+                      int T, int H, int dk, int dv, long long nslots, SegArgs sa,
+                      const bf16* __restrict__ gate) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   __shared__ uint64_t full[2];
@@ -686,6 +799,18 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
     uint8_t* rb = sm + buf * S_BUF;
     const long long t0 = t_beg + (long long)i * C;
     const int L = (int)min((long long)C, t_end - t0);
+    // the output gate's tile of this chunk: each thread fetches the pieces it stores
+    if (gate && outputs && warp > 0) {
+#pragma unroll
+      for (int it = 0; it < kStorePieces; ++it) {
+        const int idx = (tid - 32) + it * (NT_S - 32);
+        const int r = idx >> 4, ch = idx & 15;
+        if (idx < C * 16 && r < L && ch * 8 < dv)
+          cp_async16(sm + S_GATE + r * 256 + ch * 16,
+                     gate + ((row0 + t0 + r) * H + h) * dv + ch * 8, 16u);
+      }
+      cp_async_commit();
+    }
 
     // ---- [O^T | P] = S^T [Qbar^T | W^T]^T   (P only when no outputs are kept)
     if (tid == 0) {
@@ -811,18 +936,24 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
     if (__syncthreads_or(!good)) { alive = false; break; }
     tc_fence_after();
     // coalesced 16-byte stores of the tile (overlap the next MMA)
-    if (outputs) {
+    // (warps 1 .. 15: thread 0 is free to issue the next chunk's MMAs)
+    if (outputs && warp > 0) {
+      if (gate) cp_async_wait_all();
 #pragma unroll
-      for (int it = 0; it < 2; ++it) {
-        const int idx = tid + it * NT_S;
+      for (int it = 0; it < kStorePieces; ++it) {
+        const int idx = (tid - 32) + it * (NT_S - 32);
         const int r = idx >> 4, ch = idx & 15;
-        if (r < L && ch * 8 < dv) {
-          const uint4 val = *reinterpret_cast<const uint4*>(sm + S_OUT + r * 256 + ch * 16);
+        if (idx < C * 16 && r < L && ch * 8 < dv) {
+          uint4 val = *reinterpret_cast<const uint4*>(sm + S_OUT + r * 256 + ch * 16);
+          if (gate)
+            val = apply_gate(val, *reinterpret_cast<const uint4*>(sm + S_GATE + r * 256 + ch * 16));
           *reinterpret_cast<uint4*>(out + ((row0 + t0 + r) * H + h) * dv + ch * 8) = val;
         }
       }
     }
   }
+
+  if (gate) cp_async_wait_all();          // no gate copy outlives the loop (early exit)
 
   // ---- final state
   if (alive && fin) {
@@ -874,8 +1005,10 @@ bool set_attrs() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
   if (!done[dev]) {
-    if (cudaFuncSetAttribute(kda_chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             PREP_SMEM) != cudaSuccess ||
+    if (cudaFuncSetAttribute(kda_chunk_prep_kernel<false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, PREP_SMEM) != cudaSuccess ||
+        cudaFuncSetAttribute(kda_chunk_prep_kernel<true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, PREP_SMEM) != cudaSuccess ||
         cudaFuncSetAttribute(kda_state_pass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              STATE_SMEM) != cudaSuccess)
       return false;
@@ -918,7 +1051,7 @@ bool chunk_split_supported(int dk, int dv, int in_dtype) {
 cudaError_t launch_chunk_split(const void* q, const void* k, const void* v, const float* g,
                                const float* beta, const float* h0, const int32_t* cu_seqlens,
                                void* out, float* hT, int B, int T, int H, int dk, int dv,
-                               int gsh, cudaStream_t stream) {
+                               int gsh, cudaStream_t stream, const InputFusion* fz) {
   int sms = 148;
   cudaMemPool_t pool = nullptr;
   if (!device_ctx(&sms, &pool) || !set_attrs()) return cudaErrorInvalidDevice;
@@ -927,6 +1060,7 @@ cudaError_t launch_chunk_split(const void* q, const void* k, const void* v, cons
   const bf16* kb = static_cast<const bf16*>(k);
   const bf16* vb = static_cast<const bf16*>(v);
   bf16* ob = static_cast<bf16*>(out);
+  const bf16* gt = fz ? static_cast<const bf16*>(fz->gate) : nullptr;
   const bool varlen = cu_seqlens != nullptr;
 
   const long long nslots = chunk_slots(B, T, varlen);
@@ -951,27 +1085,35 @@ cudaError_t launch_chunk_split(const void* q, const void* k, const void* v, cons
 
   cudaError_t e = cudaSuccess;
   if (nslots > 0) {
-    KDA_TIMED(KDA_KERNEL_PREP, stream,
-              kda_chunk_prep_kernel<<<dim3((unsigned)nslots, H), NT, PREP_SMEM, stream>>>(
-                  qb, kb, vb, g, beta, cu_seqlens, rec, B, T, H, dk, dv, gsh, nslots));
+    if (fz && fz->conv_q) {
+      KDA_TIMED(KDA_KERNEL_PREP, stream,
+                kda_chunk_prep_kernel<true><<<dim3((unsigned)nslots, H), NT, PREP_SMEM, stream>>>(
+                    qb, kb, vb, g, beta, cu_seqlens, rec, B, T, H, dk, dv, gsh, nslots,
+                    fz->conv_q, fz->conv_k, fz->W));
+    } else {
+      KDA_TIMED(KDA_KERNEL_PREP, stream,
+                kda_chunk_prep_kernel<false><<<dim3((unsigned)nslots, H), NT, PREP_SMEM, stream>>>(
+                    qb, kb, vb, g, beta, cu_seqlens, rec, B, T, H, dk, dv, gsh, nslots, nullptr,
+                    nullptr, 0));
+    }
     note_launches(1);
   }
   if (P == 0) {
     SegArgs sa{0, 1, 0, 0, nullptr, nullptr};
     KDA_TIMED(KDA_KERNEL_STATE, stream,
               kda_state_pass_kernel<<<dim3(H, B, 1), NT_S, STATE_SMEM, stream>>>(rec, h0, cu_seqlens, ob, hT,
-                                                                               T, H, dk, dv, nslots, sa));
+                                                                               T, H, dk, dv, nslots, sa, gt));
     note_launches(1);
   } else {
     SegArgs sa{G, P, 1, (int)slots, segbuf, segbuf + (size_t)slots * H * D * D};
     KDA_TIMED(KDA_KERNEL_STATE, stream,
               kda_state_pass_kernel<<<dim3(H, B, 2 * P), NT_S, STATE_SMEM, stream>>>(rec, h0, cu_seqlens, ob,
-                                                                                   hT, T, H, dk, dv, nslots, sa));
+                                                                                   hT, T, H, dk, dv, nslots, sa, gt));
     const cudaError_t ec = launch_seg_combine_img(cu_seqlens, B, T, H, dk, dv, sa, stream);
     sa.pass = 2;
     KDA_TIMED(KDA_KERNEL_STATE, stream,
               kda_state_pass_kernel<<<dim3(H, B, P - 1), NT_S, STATE_SMEM, stream>>>(rec, h0, cu_seqlens, ob,
-                                                                                   hT, T, H, dk, dv, nslots, sa));
+                                                                                   hT, T, H, dk, dv, nslots, sa, gt));
     note_launches(2);
     if (ec != cudaSuccess) e = ec;
   }

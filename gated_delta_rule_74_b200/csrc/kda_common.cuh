@@ -54,6 +54,16 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const f
                             const float* beta, const float* h0, const int32_t* cu_seqlens,
                             void* out, float* hT, int B, int T, int H, cudaStream_t stream);
 
+// Fused input prep and output gate (kda_chunk_fwd_fused; split path only):
+// q, k <- L2-normalised causal per-channel convolutions of the raw q, k (q also
+// scaled by dk^-1/2), out <- out * sigmoid(gate).
+struct InputFusion {
+  const float* conv_q;   // [H, dk, W] fp32, or nullptr: q, k used as given
+  const float* conv_k;   // [H, dk, W] fp32
+  int W;                 // convolution width, 1 .. 4
+  const void* gate;      // [rows, H, dv] in the input dtype, or nullptr: no gate
+};
+
 // Tensor-core prefill split into a parallel per-chunk kernel and a state pass
 // (bf16, dk, dv in {64, 128}: 64-wide heads run zero-padded to 128); its
 // scratch comes from the library's memory pool.
@@ -61,7 +71,7 @@ bool chunk_split_supported(int dk, int dv, int in_dtype);
 cudaError_t launch_chunk_split(const void* q, const void* k, const void* v, const float* g,
                                const float* beta, const float* h0, const int32_t* cu_seqlens,
                                void* out, float* hT, int B, int T, int H, int dk, int dv,
-                               int gsh, cudaStream_t stream);
+                               int gsh, cudaStream_t stream, const InputFusion* fz = nullptr);
 
 // Prefill backward (recurrent, fp32): gradients of sum(out*dout) + sum(hT*dhT).
 cudaError_t launch_chunk_bwd(const void* q, const void* k, const void* v, const float* g,

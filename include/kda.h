@@ -198,6 +198,43 @@ KDA_API int kda_decode_tokens_grouped(const void* q, const void* k, const void* 
                                       int in_dtype, void* stream);
 
 /*
+ * kda_chunk_fwd_fused -- kda_chunk_fwd with its input prep and output gate fused.
+ *
+ * Passages: Mini-K3-1H v2 family cards (model architecture: KDA with short
+ * convolutions, output gates, decay granularity and convolution length among
+ * the varied choices); miniKimiK3 model card (no positional encoding: order
+ * enters only through KDA's decay and the short convolutions); Mini-K3-1H-mamba2
+ * card, packed-document paragraph (convolution history and recurrent state are
+ * reset at every document boundary).  The pages name these pieces but do not
+ * define them; the reading taken here (the plainest one):
+ *   q_t = dk^-1/2 * n(cq * q_raw)_t,   k_t = n(ck * k_raw)_t,   v_t as given,
+ *   (c * x)_t[i] = sum_{j<W} c[h][i][j] x_{t-W+1+j}[i]   (causal, per channel,
+ *                  x before the document's first token = 0, no activation),
+ *   n(x) = x / max(||x||_2, 1e-12)                       (per token and head),
+ *   out_t = o_t * sigmoid(z_t)                           (elementwise, z = gate),
+ * with o_t the KDA output of kda_chunk_fwd on (q, k, v, g, beta, h0).
+ *     q_raw, k_raw [B, T, H, dk]   v, gate, out [B, T, H, dv]   (in_dtype)
+ *     conv_q, conv_k [H, dk, conv_w] fp32 (tap conv_w - 1 multiplies the current
+ *     token); conv_w in 1 .. 4.  conv_q = conv_k = NULL: q_raw, k_raw are used as
+ *     q, k unchanged (no convolution, normalisation or scaling).  gate NULL: no
+ *     gate.  Everything else as in kda_chunk_fwd.
+ * The convolution and the normalisation run inside the per-chunk prep kernel
+ * (each chunk reads conv_w - 1 rows before it), the gate in the output store:
+ * the normalised q, k and the ungated output never reach memory.  Precision:
+ * the convolution output is rounded to bf16 before normalisation.
+ * Supported: in_dtype KDA_BF16 (KDA_F32: KDA_ERR_UNSUPPORTED).
+ *
+ * Returns KDA_OK, KDA_ERR_INVALID_ARG (also for only one of conv_q, conv_k, or
+ * conv_w out of range), KDA_ERR_UNSUPPORTED or KDA_ERR_CUDA.
+ */
+KDA_API int kda_chunk_fwd_fused(const void* q_raw, const void* k_raw, const void* v,
+                                const float* conv_q, const float* conv_k, int conv_w,
+                                const float* g, const float* beta, const void* gate,
+                                const float* h0, const int32_t* cu_seqlens, void* out,
+                                float* hT, int B, int T, int H, int dk, int dv,
+                                int in_dtype, void* stream);
+
+/*
  * kda_chunk_bwd -- gradients of the KDA prefill (training backward).
  *
  * Passage: miniKimiK3 model card, "Kimi Delta Attention" bullet: KDA "trains

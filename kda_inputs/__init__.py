@@ -26,6 +26,9 @@ Distributions (N(mu, s): s is the standard deviation):
     Kimi-K3-Tiny-L13 card mentions for its real KDA weights).
   * beta = sigmoid(N(0, 1)).
   * initial state, where used: N(0, 0.02), float32, layout [Nseq, H, dk, dv].
+  * fused prep workloads (make_fused_prefill): raw q, k projections ~ N(0, 1)
+    (not normalised), convolution taps ~ N(0, 0.5) of shape [H, dk, W], output
+    gate pre-activations ~ N(0, 1).
 """
 from __future__ import annotations
 
@@ -36,7 +39,7 @@ import torch
 
 __all__ = [
     "PrefillSpec", "DecodeSpec", "PREFILL_SPECS", "DECODE_SPECS",
-    "make_prefill", "make_decode", "doc_lengths", "spec_by_name",
+    "make_prefill", "make_fused_prefill", "make_decode", "doc_lengths", "spec_by_name",
 ]
 
 
@@ -188,6 +191,30 @@ def make_prefill(spec: PrefillSpec | str, *, T: Optional[int] = None, B: Optiona
                 h0=None if h0 is None else h0.float().contiguous(),
                 cu_seqlens=cu, B=nseq, T=T, H=H, dk=dk, dv=dv, dtype=spec.dtype,
                 name=spec.name)
+
+
+def make_fused_prefill(spec: PrefillSpec | str, *, W: int = 4, gate: bool = True,
+                       T: Optional[int] = None, B: Optional[int] = None, H: Optional[int] = None,
+                       seed: Optional[int] = None, doc_lens: Optional[list[int]] = None) -> dict:
+    """Inputs for one ``kda_chunk_fwd_fused`` call: ``make_prefill``'s tensors
+    (v, g, beta, h0, cu_seqlens) plus raw q, k projections (q_raw, k_raw, storage
+    dtype), convolution taps conv_q, conv_k ([H, dk, W] f32) and, with ``gate``,
+    the gate pre-activations gate ([B, T, H, dv], storage dtype)."""
+    if isinstance(spec, str):
+        spec = PREFILL_SPECS[spec]
+    x = make_prefill(spec, T=T, B=B, H=H, seed=seed, doc_lens=doc_lens)
+    gen = torch.Generator().manual_seed((spec.seed if seed is None else seed) + 7919)
+    dt = _torch_dtype(spec.dtype)
+    Bt, Tt, Hh, dk = x["q"].shape
+    dv = x["v"].shape[-1]
+    x["q_raw"] = torch.randn(Bt, Tt, Hh, dk, generator=gen).to(dt).contiguous()
+    x["k_raw"] = torch.randn(Bt, Tt, Hh, dk, generator=gen).to(dt).contiguous()
+    x["conv_q"] = (torch.randn(Hh, dk, W, generator=gen) * 0.5).float().contiguous()
+    x["conv_k"] = (torch.randn(Hh, dk, W, generator=gen) * 0.5).float().contiguous()
+    x["gate"] = (torch.randn(Bt, Tt, Hh, dv, generator=gen).to(dt).contiguous() if gate
+                 else None)
+    x["W"] = W
+    return x
 
 
 def make_decode(spec: DecodeSpec | str, *, N: Optional[int] = None, H: Optional[int] = None,

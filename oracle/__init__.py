@@ -20,6 +20,12 @@ Contents
     recurrence in float64 numpy, for checking the chunked algebra the GPU
     kernels implement ("trains through a chunked parallel form", same bullet).
 
+  * ``prefill_fused`` (with ``short_conv``, ``l2_normalize``, ``output_gate``):
+    the input prep and output gate around KDA that the Mini-K3-1H v2 family
+    cards name (short convolutions, output gates) but do not define; the reading
+    taken is stated in ``prefill_fused``.
+  * ``backward``: float64 reverse-mode gradients of the recurrence.
+
 Pins: tests/test_oracle.py checks these routines against closed forms,
 invariants, a hand-worked example (tests/golden/) and brute force.
 """
@@ -40,7 +46,8 @@ _SO = os.path.join(_HERE, "libkda_oracle.so")
 _lib = None
 _lock = threading.Lock()
 
-__all__ = ["build", "prefill", "decode", "max_threads", "reference"]
+__all__ = ["build", "prefill", "decode", "backward", "prefill_fused", "short_conv",
+           "l2_normalize", "output_gate", "max_threads", "reference"]
 
 
 def build(force: bool = False) -> str:
@@ -206,3 +213,74 @@ def backward(q, k, v, g, beta, dout, h0=None, dhT=None, cu_seqlens=None, heads=N
     if rc != 0:
         raise ValueError(f"kda_oracle_backward rejected its arguments (rc={rc})")
     return res
+
+
+def _doc_ranges(T: int, Bt: int, cu_seqlens):
+    """(batch row, first token, end token) of every document."""
+    if cu_seqlens is None:
+        return [(b, 0, T) for b in range(Bt)]
+    cu = np.asarray(cu_seqlens.cpu() if hasattr(cu_seqlens, "cpu") else cu_seqlens,
+                    dtype=np.int64)
+    return [(0, int(cu[d]), int(cu[d + 1])) for d in range(cu.shape[0] - 1)]
+
+
+def short_conv(x, w, cu_seqlens=None):
+    """Causal per-channel convolution over tokens, restarting at every document:
+    y_t[h, i] = sum_{j<W} w[h, i, j] * x_{t-W+1+j}[h, i], with x = 0 before the
+    document's first token (Mini-K3-1H-mamba2 card: convolution history is reset
+    at every document boundary).  x [B,T,H,d]; w [H,d,W].  float64 result."""
+    x, w = _f64(x), _f64(w)
+    Bt, T = x.shape[:2]
+    W = w.shape[-1]
+    y = np.zeros_like(x)
+    for b, t0, t1 in _doc_ranges(T, Bt, cu_seqlens):
+        for t in range(t0, t1):
+            for j in range(W):
+                src = t - (W - 1) + j
+                if src >= t0:
+                    y[b, t] += w[:, :, j] * x[b, src]
+    return y
+
+
+def l2_normalize(x, eps: float = 1e-12):
+    """x / max(||x||_2, eps) over the last axis (per token and head)."""
+    x = _f64(x)
+    n = np.sqrt(np.sum(x * x, axis=-1, keepdims=True))
+    return x / np.maximum(n, eps)
+
+
+def output_gate(o, z):
+    """o * sigmoid(z), elementwise (the output gate of the family cards)."""
+    o, z = _f64(o), _f64(z)
+    return o / (1.0 + np.exp(-z))
+
+
+def prefill_fused(q_raw, k_raw, v, g, beta, conv_q=None, conv_k=None, gate=None, h0=None,
+                  cu_seqlens=None, heads=None, nthreads: int = 0):
+    """KDA prefill with its input prep and output gate, in float64.
+
+    Reading (the pages name short convolutions, q/k normalisation and output
+    gates without defining them): q = dk^-1/2 * l2_normalize(short_conv(q_raw, conv_q)),
+    k = l2_normalize(short_conv(k_raw, conv_k)), v unchanged; with conv_q = conv_k =
+    None, q = q_raw and k = k_raw.  out = output_gate(o, gate) when gate is given.
+    Returns (out, hT) as ``prefill`` does (``heads`` selects a head range).
+    """
+    if heads is not None:
+        lo, hi = heads
+        q_raw, k_raw, v, g, beta = (x[:, :, lo:hi] for x in (q_raw, k_raw, v, g, beta))
+        conv_q = None if conv_q is None else conv_q[lo:hi]
+        conv_k = None if conv_k is None else conv_k[lo:hi]
+        gate = None if gate is None else gate[:, :, lo:hi]
+        h0 = None if h0 is None else h0[:, lo:hi]
+    if (conv_q is None) != (conv_k is None):
+        raise ValueError("give both conv_q and conv_k, or neither")
+    if conv_q is not None:
+        dk = q_raw.shape[-1]
+        q = l2_normalize(short_conv(q_raw, conv_q, cu_seqlens)) / np.sqrt(dk)
+        k = l2_normalize(short_conv(k_raw, conv_k, cu_seqlens))
+    else:
+        q, k = _f64(q_raw), _f64(k_raw)
+    out, hT = prefill(q, k, v, g, beta, h0, cu_seqlens, nthreads=nthreads)
+    if gate is not None:
+        out = output_gate(out, gate)
+    return out, hT

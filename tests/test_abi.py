@@ -113,3 +113,21 @@ def test_chunk_bwd_rejects_invalid(L, bad):
 @pytest.mark.parametrize("dims", [dict(dk=32), dict(dv=96)])
 def test_chunk_bwd_rejects_unsupported_heads(L, dims):
     assert _bwd(L, **dims) == kda.KDA_ERR_UNSUPPORTED
+
+
+def _fused(L, qr=P, kr=P, v=P, cq=P, ck=P, W=4, g=P, beta=P, gate=None, h0=None, cu=None,
+           out=P, hT=None, B=1, T=64, H=2, dk=128, dv=128, dt=0):
+    return L.kda_chunk_fwd_fused(qr, kr, v, cq, ck, W, g, beta, gate, h0, cu, out, hT,
+                                 B, T, H, dk, dv, dt, None)
+
+
+@pytest.mark.parametrize("bad", [dict(qr=None), dict(v=None), dict(out=None), dict(cq=None),
+                                 dict(ck=None), dict(W=0), dict(W=5), dict(gate=P + 4),
+                                 dict(cq=P + 4), dict(B=0), dict(H=0), dict(dt=2)])
+def test_chunk_fwd_fused_rejects_invalid(L, bad):
+    assert _fused(L, **bad) == kda.KDA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("dims", [dict(dk=32), dict(dt=1)])
+def test_chunk_fwd_fused_rejects_unsupported(L, dims):
+    assert _fused(L, **dims) == kda.KDA_ERR_UNSUPPORTED

@@ -502,3 +502,96 @@ def test_backward_document_isolation_zero_gradient(oracle_lib):
         assert np.all(r[key][:, :4] == 0.0), key
         assert np.any(r[key][:, 4:] != 0.0), key
     assert np.all(r["dh0"][0] == 0.0) and np.any(r["dh0"][1] != 0.0)
+
+
+# ---- fused input prep and output gate (short convolution, L2 norm, sigmoid gate) ----
+
+def test_short_conv_matches_numpy_convolve():
+    """Per channel, the causal convolution of one document is numpy's full
+    convolution with the taps reversed, cut to the document's length."""
+    rng = np.random.default_rng(80)
+    x = rng.standard_normal((2, 11, 3, 5))
+    w = rng.standard_normal((3, 5, 4))
+    y = oracle.short_conv(x, w)
+    for b in range(2):
+        for h in range(3):
+            for c in range(5):
+                ref = np.convolve(x[b, :, h, c], w[h, c, ::-1])[:11]
+                np.testing.assert_allclose(y[b, :, h, c], ref, rtol=1e-13, atol=1e-13)
+
+
+@pytest.mark.parametrize("tap", [0, 1, 2, 3])
+def test_short_conv_delta_taps_shift(tap):
+    """A single unit tap j of a width-4 convolution delays the sequence by 3 - j
+    tokens, with zeros shifted in at the document start."""
+    rng = np.random.default_rng(81 + tap)
+    x = rng.standard_normal((1, 9, 2, 3))
+    w = np.zeros((2, 3, 4))
+    w[..., tap] = 1.0
+    y = oracle.short_conv(x, w)
+    s = 3 - tap
+    assert np.array_equal(y[0, s:], x[0, :9 - s])
+    assert np.all(y[0, :s] == 0)
+
+
+def test_short_conv_restarts_at_document_boundaries():
+    """Packed documents: each document's convolution equals that document run
+    alone, and perturbing one document leaves the others unchanged."""
+    rng = np.random.default_rng(85)
+    lens = [5, 1, 0, 7, 2]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T = int(cu[-1])
+    x = rng.standard_normal((1, T, 2, 3))
+    w = rng.standard_normal((2, 3, 3))
+    y = oracle.short_conv(x, w, cu)
+    for d in range(len(lens)):
+        a, b = cu[d], cu[d + 1]
+        alone = oracle.short_conv(x[:, a:b], w)
+        assert np.array_equal(y[:, a:b], alone)
+    x2 = x.copy()
+    x2[:, cu[3]:cu[4]] += 5.0
+    y2 = oracle.short_conv(x2, w, cu)
+    assert np.array_equal(np.delete(y2, np.s_[cu[3]:cu[4]], axis=1),
+                          np.delete(y, np.s_[cu[3]:cu[4]], axis=1))
+
+
+def test_l2_normalize_properties():
+    rng = np.random.default_rng(86)
+    x = rng.standard_normal((3, 4, 2, 16))
+    n = oracle.l2_normalize(x)
+    np.testing.assert_allclose(np.linalg.norm(n, axis=-1), 1.0, rtol=1e-14)
+    np.testing.assert_allclose(oracle.l2_normalize(7.5 * x), n, rtol=1e-14)   # scale-free
+    z = np.zeros((1, 2, 1, 8))
+    assert np.array_equal(oracle.l2_normalize(z), z)                        # no NaN at 0
+
+
+def test_output_gate_special_values():
+    rng = np.random.default_rng(87)
+    o = rng.standard_normal((2, 5, 3, 4))
+    z = rng.standard_normal((2, 5, 3, 4))
+    assert np.array_equal(oracle.output_gate(o, np.zeros_like(o)), o / 2)    # sigmoid(0) = 1/2
+    np.testing.assert_allclose(oracle.output_gate(o, z) + oracle.output_gate(o, -z), o,
+                               rtol=1e-14, atol=1e-15)                        # s(z) + s(-z) = 1
+    np.testing.assert_allclose(oracle.output_gate(o, np.full_like(o, 60.0)), o, rtol=1e-15)
+
+
+def test_prefill_fused_identity_prep_reduces_to_prefill(oracle_lib):
+    """A width-1 unit convolution on inputs that are already unit-norm leaves k
+    unchanged and scales q by dk^-1/2: the fused prefill is then the plain one."""
+    rng = np.random.default_rng(88)
+    T, H, dk, dv = 40, 2, 8, 6
+    qr = rng.standard_normal((1, T, H, dk))
+    kr = rng.standard_normal((1, T, H, dk))
+    qr /= np.linalg.norm(qr, axis=-1, keepdims=True)
+    kr /= np.linalg.norm(kr, axis=-1, keepdims=True)
+    v = rng.standard_normal((1, T, H, dv))
+    g = -np.abs(rng.standard_normal((1, T, H, dk))) * 0.1
+    b = 1 / (1 + np.exp(-rng.standard_normal((1, T, H))))
+    w = np.ones((H, dk, 1))
+    o1, s1 = oracle.prefill_fused(qr, kr, v, g, b, w, w)
+    o2, s2 = oracle.prefill(qr / np.sqrt(dk), kr, v, g, b)
+    np.testing.assert_allclose(o1, o2, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(s1, s2, rtol=1e-12, atol=1e-14)
+    o3, _ = oracle.prefill_fused(qr, kr, v, g, b)                     # no prep: q, k as given
+    o4, _ = oracle.prefill(qr, kr, v, g, b)
+    assert np.array_equal(o3, o4)
