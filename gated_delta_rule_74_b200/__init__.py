@@ -78,6 +78,9 @@ def lib() -> ctypes.CDLL:
         L.kda_chunk_bwd.argtypes = [vp, vp, vp, fp, fp, fp, vp, vp, fp,
                                     fp, fp, fp, fp, fp, fp] + [ip] * 6 + [vp]
         L.kda_chunk_bwd.restype = ctypes.c_int
+        L.kda_chunk_bwd_grouped.argtypes = [vp, vp, vp, fp, fp, fp, vp, vp, fp,
+                                            fp, fp, fp, fp, fp, fp] + [ip] * 7 + [vp]
+        L.kda_chunk_bwd_grouped.restype = ctypes.c_int
         L.kda_status_string.argtypes = [ctypes.c_int]
         L.kda_status_string.restype = ctypes.c_char_p
         L.kda_version.argtypes = []
@@ -283,9 +286,10 @@ def kda_chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Te
                   dhT: Optional[torch.Tensor] = None, cu_seqlens: Optional[torch.Tensor] = None,
                   grads: Optional[dict] = None, stream=None) -> dict:
     """Gradients of L = sum(out * dout) + sum(hT * dhT) for kda_chunk_fwd with the same
-    inputs (per-channel g only).  dout has out's shape and dtype; dhT [Nseq,H,dk,dv] f32
-    or None.  Returns a dict of fp32 tensors dq, dk, dv, dg, dbeta, dh0 (dh0 None when
-    h0 is None); ``grads`` may hold preallocated outputs under those names."""
+    inputs.  g [B,T,H,dk] f32, or [B,T,H,dk/G] for one decay per group of G key channels
+    (kda_chunk_bwd_grouped; dg then has g's shape).  dout has out's shape and dtype; dhT
+    [Nseq,H,dk,dv] f32 or None.  Returns a dict of fp32 tensors dq, dk, dv, dg, dbeta, dh0
+    (dh0 None when h0 is None); ``grads`` may hold preallocated outputs under those names."""
     if q.dim() != 4:
         raise ValueError("q must be [B, T, H, dk]")
     Bt, T, H, dk = q.shape
@@ -296,7 +300,8 @@ def kda_chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Te
     _check("q", q)
     _check("k", k, q.dtype, (Bt, T, H, dk))
     _check("v", v, q.dtype, (Bt, T, H, dv))
-    _check("g", g, torch.float32, (Bt, T, H, dk))
+    G = _decay_group(g, dk)
+    _check("g", g, torch.float32, (Bt, T, H, dk // G))
     _check("beta", beta, torch.float32, (Bt, T, H))
     _check("dout", dout, q.dtype, (Bt, T, H, dv))
     if cu_seqlens is not None:
@@ -311,7 +316,7 @@ def kda_chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Te
     if dhT is not None:
         _check("dhT", dhT, torch.float32, (nseq, H, dk, dv))
     shapes = {"dq": (Bt, T, H, dk), "dk": (Bt, T, H, dk), "dv": (Bt, T, H, dv),
-              "dg": (Bt, T, H, dk), "dbeta": (Bt, T, H), "dh0": (nseq, H, dk, dv)}
+              "dg": (Bt, T, H, dk // G), "dbeta": (Bt, T, H), "dh0": (nseq, H, dk, dv)}
     res = dict(grads or {})
     for name, shp in shapes.items():
         if name == "dh0" and h0 is None and res.get(name) is None:
@@ -320,11 +325,13 @@ def kda_chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Te
         if res.get(name) is None:
             res[name] = torch.empty(shp, dtype=torch.float32, device=q.device)
         _check(name, res[name], torch.float32, shp)
-    rc = lib().kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
-                             _ptr(cu_seqlens), _ptr(dout), _ptr(dhT), _ptr(res["dq"]),
-                             _ptr(res["dk"]), _ptr(res["dv"]), _ptr(res["dg"]),
-                             _ptr(res["dbeta"]), _ptr(res["dh0"]), nseq, T, H, dk, dv, dt,
-                             _stream(stream))
+    args = [_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0), _ptr(cu_seqlens),
+            _ptr(dout), _ptr(dhT), _ptr(res["dq"]), _ptr(res["dk"]), _ptr(res["dv"]),
+            _ptr(res["dg"]), _ptr(res["dbeta"]), _ptr(res["dh0"]), nseq, T, H, dk, dv]
+    if G == 1:
+        rc = lib().kda_chunk_bwd(*args, dt, _stream(stream))
+    else:
+        rc = lib().kda_chunk_bwd_grouped(*args, G, dt, _stream(stream))
     if rc != KDA_OK:
         raise KdaError("kda_chunk_bwd", rc)
     return res

@@ -159,11 +159,13 @@ int kda_chunk_fwd_fused(const void* q_raw, const void* k_raw, const void* v, con
                                              &fz));
 }
 
-int kda_chunk_bwd(const void* q, const void* k, const void* v, const float* g,
-                  const float* beta, const float* h0, const int32_t* cu_seqlens,
-                  const void* dout, const float* dhT, float* dq, float* dk, float* dv, float* dg,
-                  float* dbeta, float* dh0, int B, int T, int H, int dk_dim, int dv_dim,
-                  int in_dtype, void* stream) {
+namespace {
+int chunk_bwd_impl(const void* q, const void* k, const void* v, const float* g,
+                   const float* beta, const float* h0, const int32_t* cu_seqlens,
+                   const void* dout, const float* dhT, float* dq, float* dk, float* dv, float* dg,
+                   float* dbeta, float* dh0, int B, int T, int H, int dk_dim, int dv_dim, int gsh,
+                   int in_dtype, void* stream) {
+  if (gsh < 0) return KDA_ERR_INVALID_ARG;
   if (B < 1 || T < 0 || H < 1) return KDA_ERR_INVALID_ARG;
   if (in_dtype != KDA_BF16 && in_dtype != KDA_F32) return KDA_ERR_INVALID_ARG;
   const long long rows = cu_seqlens ? (long long)T : (long long)B * T;
@@ -181,8 +183,27 @@ int kda_chunk_bwd(const void* q, const void* k, const void* v, const float* g,
   if ((long long)B > 65535LL || H > 0x7fffffff) return KDA_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return status_from(kda::launch_chunk_bwd(q, k, v, g, beta, h0, cu_seqlens, dout, dhT, dq, dk,
-                                           dv, dg, dbeta, dh0, B, T, H, dk_dim, dv_dim,
+                                           dv, dg, dbeta, dh0, B, T, H, dk_dim, dv_dim, gsh,
                                            in_dtype, st));
+}
+}  // namespace
+
+int kda_chunk_bwd(const void* q, const void* k, const void* v, const float* g,
+                  const float* beta, const float* h0, const int32_t* cu_seqlens,
+                  const void* dout, const float* dhT, float* dq, float* dk, float* dv, float* dg,
+                  float* dbeta, float* dh0, int B, int T, int H, int dk_dim, int dv_dim,
+                  int in_dtype, void* stream) {
+  return chunk_bwd_impl(q, k, v, g, beta, h0, cu_seqlens, dout, dhT, dq, dk, dv, dg, dbeta, dh0,
+                        B, T, H, dk_dim, dv_dim, 0, in_dtype, stream);
+}
+
+int kda_chunk_bwd_grouped(const void* q, const void* k, const void* v, const float* g,
+                          const float* beta, const float* h0, const int32_t* cu_seqlens,
+                          const void* dout, const float* dhT, float* dq, float* dk, float* dv,
+                          float* dg, float* dbeta, float* dh0, int B, int T, int H, int dk_dim,
+                          int dv_dim, int g_group, int in_dtype, void* stream) {
+  return chunk_bwd_impl(q, k, v, g, beta, h0, cu_seqlens, dout, dhT, dq, dk, dv, dg, dbeta, dh0,
+                        B, T, H, dk_dim, dv_dim, group_shift(g_group, dk_dim), in_dtype, stream);
 }
 
 const char* kda_status_string(int status) {

@@ -143,7 +143,7 @@ template <typename Tin, int DK>
 struct BwdSmem {
   static constexpr int NBUF = sizeof(Tin) == 2 ? 2 : 1;
   static constexpr int SI = (int)sizeof(Tin);
-  static constexpr int G = 0;                                   // fp32 [64][DK]
+  static constexpr int G = 0;                                   // fp32 [64][DK >> gsh]
   static constexpr int K = G + kChunk * DK * 4;                 // Tin [64][DK]
   static constexpr int Q = K + kChunk * DK * SI;                // Tin [64][DK]
   static constexpr int V = Q + kChunk * DK * SI;                // Tin [64][CPC]
@@ -155,32 +155,47 @@ struct BwdSmem {
   static constexpr int BAR = RINGB + WPC * RING * DK * NC * 4;  // uint64 [NBUF]
   static constexpr size_t BYTES = (size_t)BAR + 8 * NBUF;
   static_assert(BUF % 16 == 0 && CPC * SI % 16 == 0, "bulk copies need 16-byte pieces");
-  static constexpr uint32_t bytes(int L, bool rev) {
-    return (uint32_t)L * (DK * 4 + DK * SI + CPC * SI + (rev ? DK * SI + CPC * SI : 0));
+  // g rows of NG = DK >> gsh values go by bulk copy when 16-byte multiples
+  static __device__ __forceinline__ bool g_bulk(int gsh) { return ((DK >> gsh) & 3) == 0; }
+  static __device__ __forceinline__ uint32_t bytes(int L, bool rev, int gsh) {
+    return (uint32_t)L * ((g_bulk(gsh) ? (DK >> gsh) * 4 : 0) + DK * SI + CPC * SI +
+                          (rev ? DK * SI + CPC * SI : 0));
   }
 };
 
 // Start the bulk copies of tokens [0, L) of a chunk (first token row `rowbase`,
 // head h) into buffer `buf`: g, k and this CTA's CPC columns of v, with `rev`
 // also q and dout; completion on `bar`, whose transaction count the caller has
-// set to BwdSmem::bytes(L, rev).  Two threads per token.  Returns beta of the
-// calling thread's token (threads 0 .. L-1), else 0.
+// set to BwdSmem::bytes(L, rev, gsh).  Two threads per token.  Returns, for the
+// calling thread's token (threads 0 .. L-1): beta, and the token's g row when it
+// is too short for a bulk copy (DK >> gsh <= 2 values); else zeros.
+struct Staged {
+  float beta, g0, g1;
+};
 template <typename Tin, int DK, int DV>
-__device__ __forceinline__ float issue_chunk(char* buf, uint64_t* bar, const Tin* __restrict__ q,
-                                             const Tin* __restrict__ k,
-                                             const Tin* __restrict__ v,
-                                             const float* __restrict__ g,
-                                             const float* __restrict__ beta,
-                                             const Tin* __restrict__ dout, long long rowbase,
-                                             int L, int H, int h, int cta_c0, bool rev) {
+__device__ __forceinline__ Staged issue_chunk(char* buf, uint64_t* bar, const Tin* __restrict__ q,
+                                              const Tin* __restrict__ k,
+                                              const Tin* __restrict__ v,
+                                              const float* __restrict__ g,
+                                              const float* __restrict__ beta,
+                                              const Tin* __restrict__ dout, long long rowbase,
+                                              int L, int H, int h, int cta_c0, bool rev,
+                                              int gsh) {
   using S = BwdSmem<Tin, DK>;
   static_assert(NTB == 2 * kChunk, "two threads per token");
   const int t = threadIdx.x & (kChunk - 1), part = threadIdx.x / kChunk;
-  float b = 0.f;
+  const int ng = DK >> gsh;
+  Staged st{0.f, 0.f, 0.f};
+  float& b = st.beta;
   if (t < L) {
     const long long row = (rowbase + t) * H + h;
     if (part == 0) {
-      bulk_g2s(buf + S::G + t * DK * 4, g + row * DK, DK * 4, bar);
+      if (S::g_bulk(gsh)) {
+        bulk_g2s(buf + S::G + t * ng * 4, g + row * ng, ng * 4, bar);
+      } else {
+        st.g0 = g[row * ng];
+        if (ng > 1) st.g1 = g[row * ng + 1];
+      }
       bulk_g2s(buf + S::K + t * DK * S::SI, k + row * DK, DK * S::SI, bar);
       if (rev) bulk_g2s(buf + S::Q + t * DK * S::SI, q + row * DK, DK * S::SI, bar);
       b = beta[row];
@@ -189,11 +204,12 @@ __device__ __forceinline__ float issue_chunk(char* buf, uint64_t* bar, const Tin
       if (rev) bulk_g2s(buf + S::DO + t * CPC * S::SI, dout + row * DV + cta_c0, CPC * S::SI, bar);
     }
   }
-  return b;
+  return st;
 }
 
-// One CTA per (column block of CPC state columns, head, sequence).
-template <typename Tin, int DK, int DV>
+// One CTA per (column block of CPC state columns, head, sequence).  GRP: grouped
+// decay (gsh > 0); without it the kernel is compiled for per-channel g.
+template <typename Tin, int DK, int DV, bool GRP>
 __global__ void __launch_bounds__(NTB, 1)
 kda_chunk_bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                      const Tin* __restrict__ v, const float* __restrict__ g,
@@ -202,7 +218,9 @@ kda_chunk_bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                      const float* __restrict__ dhT, float* __restrict__ dq,
                      float* __restrict__ dk, float* __restrict__ dvo, float* __restrict__ dg,
                      float* __restrict__ dbeta, float* __restrict__ dh0,
-                     float* __restrict__ ckpt, float* __restrict__ cst, int T, int H) {
+                     float* __restrict__ ckpt, float* __restrict__ cst, int T, int H,
+                     int gsh_arg) {
+  const int gsh = GRP ? gsh_arg : 0;
   constexpr int R = DK / 32;            // state rows per lane
   constexpr int NV = R * NC / 4;        // float4 per lane in a warp's state slice
   constexpr int SLICE = DK * NC;        // floats in a warp's state slice
@@ -254,17 +272,27 @@ kda_chunk_bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
   auto issue = [&](int j) {
     const int b = j % NBUF;
     return issue_chunk<Tin, DK, DV>(smc + b * SM::BUF, &bars[b], q, k, v, g, beta, dout,
-                                    job_row(j), job_len(j), H, h, cta_c0, j >= nf);
+                                    job_row(j), job_len(j), H, h, cta_c0, j >= nf, gsh);
+  };
+  const int ng = DK >> gsh;             // decay values per token (groups of 2^gsh channels)
+  // the decay of this lane's rows at staged token t
+  auto decay_rows = [&](const float* al_s, int t, float (&al)[R]) {
+    if (!GRP) {
+      lds_n(al_s + t * DK + rl, al);
+    } else {
+#pragma unroll
+      for (int i = 0; i < R; ++i) al[i] = al_s[t * ng + ((rl + i) >> gsh)];
+    }
   };
 
   if (tid == 0) {
 #pragma unroll
     for (int b = 0; b < NBUF; ++b) mbar_init(&bars[b], 1);
     fence_mbar_init();
-    if (njobs > 0) mbar_arrive_expect_tx(&bars[0], SM::bytes(job_len(0), 0 >= nf));
+    if (njobs > 0) mbar_arrive_expect_tx(&bars[0], SM::bytes(job_len(0), 0 >= nf, gsh));
   }
   __syncthreads();
-  float bnext = njobs > 0 ? issue(0) : 0.f;
+  Staged bnext = njobs > 0 ? issue(0) : Staged{0.f, 0.f, 0.f};
   uint32_t parity = 0;                  // bit b: parity of buffer b's next completion
   bool stalled = false;                 // a wait expired (diagnostic flag set)
 
@@ -300,14 +328,22 @@ kda_chunk_bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     parity ^= 1u << b;
     float* const al_s = reinterpret_cast<float*>(buf + SM::G);
     float* const beta_s = reinterpret_cast<float*>(buf + SM::BETA);
-    if (tid < L) beta_s[tid] = bnext;
-    for (int i = tid; i < L * DK / 4; i += NTB) {
-      float4 x = reinterpret_cast<float4*>(al_s)[i];
-      x.x = __expf(x.x); x.y = __expf(x.y); x.z = __expf(x.z); x.w = __expf(x.w);
-      reinterpret_cast<float4*>(al_s)[i] = x;
+    if (tid < L) {
+      beta_s[tid] = bnext.beta;
+      if (!SM::g_bulk(gsh)) {
+        al_s[tid * ng] = __expf(bnext.g0);
+        if (ng > 1) al_s[tid * ng + 1] = __expf(bnext.g1);
+      }
+    }
+    if (SM::g_bulk(gsh)) {
+      for (int i = tid; i < L * ng / 4; i += NTB) {
+        float4 x = reinterpret_cast<float4*>(al_s)[i];
+        x.x = __expf(x.x); x.y = __expf(x.y); x.z = __expf(x.z); x.w = __expf(x.w);
+        reinterpret_cast<float4*>(al_s)[i] = x;
+      }
     }
     if (NBUF == 2 && tid == 0 && j + 1 < njobs)
-      mbar_arrive_expect_tx(&bars[b ^ 1], SM::bytes(job_len(j + 1), j + 1 >= nf));
+      mbar_arrive_expect_tx(&bars[b ^ 1], SM::bytes(job_len(j + 1), j + 1 >= nf, gsh));
     __syncthreads();
     if (NBUF == 2 && j + 1 < njobs) bnext = issue(j + 1);
 
@@ -318,7 +354,7 @@ kda_chunk_bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     // one forward step on token t: S <- a + beta k e^T, e = v - a^T k
     auto fwd = [&](int t) {
       float al[R], kr[R];
-      lds_n(al_s + t * DK + rl, al);
+      decay_rows(al_s, t, al);
       lds_n(k_s + t * DK + rl, kr);
       float p[NC];
 #pragma unroll
@@ -389,7 +425,7 @@ kda_chunk_bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
         float A[R][NC];                 // pre-token state S_{t-1} (a = Diag(alpha) A)
         ld_slice(ring + (t % RING) * SLICE, A);
         float al[R], kr[R], qr[R], dov[NC], ee[NC];
-        lds_n(al_s + t * DK + rl, al);
+        decay_rows(al_s, t, al);
         lds_n(k_s + t * DK + rl, kr);
         lds_n(q_s + t * DK + rl, qr);
         lds_n(do_s + t * CPC + wc, dov);
@@ -436,7 +472,19 @@ kda_chunk_bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
           dgp[i] = al[i] * a3;
         }
         Rows<R>::add(dk + tok * DK + rl, dkp);
-        Rows<R>::add(dg + tok * DK + rl, dgp);
+        if (!GRP) {
+          Rows<R>::add(dg + tok * DK + rl, dgp);
+        } else {                        // rows of one group add into one value
+          float acc = 0.f;
+#pragma unroll
+          for (int i = 0; i < R; ++i) {
+            acc += dgp[i];
+            if (i == R - 1 || ((rl + i + 1) >> gsh) != ((rl + i) >> gsh)) {
+              atomicAdd(dg + tok * ng + ((rl + i) >> gsh), acc);
+              acc = 0.f;
+            }
+          }
+        }
         const int tn = t - RING;
         if (tn >= 0) {
 #pragma unroll
@@ -452,7 +500,7 @@ kda_chunk_bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     fence_async_smem();
     if (NBUF == 1 && j + 1 < njobs) {
       __syncthreads();
-      if (tid == 0) mbar_arrive_expect_tx(&bars[0], SM::bytes(job_len(j + 1), j + 1 >= nf));
+      if (tid == 0) mbar_arrive_expect_tx(&bars[0], SM::bytes(job_len(j + 1), j + 1 >= nf, gsh));
       __syncthreads();
       bnext = issue(j + 1);
     }
@@ -468,18 +516,20 @@ template <typename Tin, int DK, int DV>
 cudaError_t launch_t(const void* q, const void* k, const void* v, const float* g,
                      const float* beta, const float* h0, const int32_t* cu, const void* dout,
                      const float* dhT, float* dq, float* dk, float* dv, float* dg, float* dbeta,
-                     float* dh0, float* ckpt, float* cst, int B, int T, int H,
+                     float* dh0, float* ckpt, float* cst, int B, int T, int H, int gsh,
                      cudaStream_t stream) {
   constexpr size_t smem = BwdSmem<Tin, DK>::BYTES;
-  const cudaError_t ea = cudaFuncSetAttribute(kda_chunk_bwd_kernel<Tin, DK, DV>,
+  auto kern = gsh > 0 ? kda_chunk_bwd_kernel<Tin, DK, DV, true>
+                     : kda_chunk_bwd_kernel<Tin, DK, DV, false>;
+  const cudaError_t ea = cudaFuncSetAttribute(kern,
                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                                               (int)smem);
   if (ea != cudaSuccess) return ea;
   KDA_TIMED(KDA_KERNEL_BWD, stream,
-            kda_chunk_bwd_kernel<Tin, DK, DV><<<dim3(DV / CPC, H, B), NTB, smem, stream>>>(
+            kern<<<dim3(DV / CPC, H, B), NTB, smem, stream>>>(
                 static_cast<const Tin*>(q), static_cast<const Tin*>(k), static_cast<const Tin*>(v),
                 g, beta, h0, cu, static_cast<const Tin*>(dout), dhT, dq, dk, dv, dg, dbeta, dh0,
-                ckpt, cst, T, H));
+                ckpt, cst, T, H, gsh));
   note_launches(1);
   return cudaGetLastError();
 }
@@ -489,11 +539,11 @@ cudaError_t launch_dtype(const void* q, const void* k, const void* v, const floa
                          const float* beta, const float* h0, const int32_t* cu, const void* dout,
                          const float* dhT, float* dq, float* dk, float* dv, float* dg,
                          float* dbeta, float* dh0, float* ckpt, float* cst, int B, int T, int H,
-                         int dkk, int dvv, cudaStream_t stream) {
+                         int dkk, int dvv, int gsh, cudaStream_t stream) {
 #define KDA_BWD_CASE(A, Bv)                                                                   \
   if (dkk == A && dvv == Bv)                                                                 \
     return launch_t<Tin, A, Bv>(q, k, v, g, beta, h0, cu, dout, dhT, dq, dk, dv, dg, dbeta, \
-                                dh0, ckpt, cst, B, T, H, stream);
+                                dh0, ckpt, cst, B, T, H, gsh, stream);
   KDA_BWD_CASE(128, 128)
   KDA_BWD_CASE(128, 64)
   KDA_BWD_CASE(64, 128)
@@ -508,7 +558,7 @@ cudaError_t launch_chunk_bwd(const void* q, const void* k, const void* v, const 
                              const float* beta, const float* h0, const int32_t* cu_seqlens,
                              const void* dout, const float* dhT, float* dq, float* dkk,
                              float* dvv, float* dg, float* dbeta, float* dh0, int B, int T, int H,
-                             int dk, int dv, int in_dtype, cudaStream_t stream) {
+                             int dk, int dv, int gsh, int in_dtype, cudaStream_t stream) {
   int sms = 148;
   cudaMemPool_t pool = nullptr;
   if (!device_ctx(&sms, &pool)) return cudaErrorInvalidDevice;
@@ -520,7 +570,7 @@ cudaError_t launch_chunk_bwd(const void* q, const void* k, const void* v, const 
     const size_t n = rows * H * dk * sizeof(float);
     if ((e = cudaMemsetAsync(dq, 0, n, stream)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(dkk, 0, n, stream)) != cudaSuccess) return e;
-    if ((e = cudaMemsetAsync(dg, 0, n, stream)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(dg, 0, n >> gsh, stream)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(dbeta, 0, rows * H * sizeof(float), stream)) != cudaSuccess)
       return e;
   }
@@ -536,10 +586,10 @@ cudaError_t launch_chunk_bwd(const void* q, const void* k, const void* v, const 
   float* cst = ckpt + nck * sz;
   if (in_dtype == KDA_BF16)
     e = launch_dtype<__nv_bfloat16>(q, k, v, g, beta, h0, cu_seqlens, dout, dhT, dq, dkk, dvv, dg,
-                                    dbeta, dh0, ckpt, cst, B, T, H, dk, dv, stream);
+                                    dbeta, dh0, ckpt, cst, B, T, H, dk, dv, gsh, stream);
   else
     e = launch_dtype<float>(q, k, v, g, beta, h0, cu_seqlens, dout, dhT, dq, dkk, dvv, dg, dbeta,
-                            dh0, ckpt, cst, B, T, H, dk, dv, stream);
+                            dh0, ckpt, cst, B, T, H, dk, dv, gsh, stream);
   cudaFreeAsync(scratch, stream);
   return e;
 }

@@ -78,7 +78,7 @@ cudaError_t launch_chunk_bwd(const void* q, const void* k, const void* v, const 
                              const float* beta, const float* h0, const int32_t* cu_seqlens,
                              const void* dout, const float* dhT, float* dq, float* dk, float* dv,
                              float* dg, float* dbeta, float* dh0, int B, int T, int H, int dkd,
-                             int dvd, int in_dtype, cudaStream_t stream);
+                             int dvd, int gsh, int in_dtype, cudaStream_t stream);
 
 // The tensor-core prefill on caller-provided scratch (allocates nothing).
 int run_chunk_tc_static(const void* q, const void* k, const void* v, const float* g,

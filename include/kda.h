@@ -272,6 +272,21 @@ KDA_API int kda_chunk_bwd(const void* q, const void* k, const void* v,
                           float* dh0, int B, int T, int H, int dk_dim, int dv_dim,
                           int in_dtype, void* stream);
 
+/*
+ * kda_chunk_bwd_grouped -- kda_chunk_bwd for grouped decay (one log-decay per
+ * group of g_group consecutive key channels, the reading documented at
+ * kda_chunk_fwd_grouped).  g and dg are [B, T, H, dk / g_group]; dg[.., m] is
+ * the gradient of the shared value, i.e. the sum over the group's channels.
+ * Everything else as in kda_chunk_bwd; g_group = 1 is exactly that call.
+ * g_group must be a power of two, 1 <= g_group <= dk (else KDA_ERR_INVALID_ARG).
+ */
+KDA_API int kda_chunk_bwd_grouped(const void* q, const void* k, const void* v,
+                                  const float* g, const float* beta, const float* h0,
+                                  const int32_t* cu_seqlens, const void* dout,
+                                  const float* dhT, float* dq, float* dk, float* dv, float* dg,
+                                  float* dbeta, float* dh0, int B, int T, int H, int dk_dim,
+                                  int dv_dim, int g_group, int in_dtype, void* stream);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 KDA_API const char* kda_status_string(int status);
 

@@ -131,3 +131,9 @@ def test_chunk_fwd_fused_rejects_invalid(L, bad):
 @pytest.mark.parametrize("dims", [dict(dk=32), dict(dt=1)])
 def test_chunk_fwd_fused_rejects_unsupported(L, dims):
     assert _fused(L, **dims) == kda.KDA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("G", [0, 3, 96, 256])
+def test_bwd_grouped_rejects_bad_group(L, G):
+    assert L.kda_chunk_bwd_grouped(P, P, P, P, P, None, None, P, None, P, P, P, P, P, None,
+                                   1, 4, 1, 128, 128, G, 0, None) == kda.KDA_ERR_INVALID_ARG

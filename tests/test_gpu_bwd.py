@@ -137,3 +137,24 @@ def test_bwd_repeatable():
         assert torch.equal(a[n], b[n]), n
     for n in ("dq", "dk", "dg", "dbeta"):
         assert rel_err(a[n], b[n].double().cpu().numpy()) <= 1e-6, n
+
+
+@pytest.mark.parametrize("dtype,dk,dv,G", [("bf16", 128, 128, 64), ("bf16", 128, 128, 2),
+                                           ("f32", 64, 64, 16), ("bf16", 64, 128, 64),
+                                           ("f32", 128, 64, 4)])
+def test_bwd_grouped_decay_matches_oracle(dtype, dk, dv, G):
+    """One decay per group of G key channels: dg of a shared value is the sum of
+    the per-channel gradients over its group (chain rule of the expansion)."""
+    spec = ki.PrefillSpec("bwd", B=2, T=150, H=2, dk=dk, dv=dv, dtype=dtype, decay="alog",
+                          seed=G + dk, h0=True)
+    x = ki.make_prefill(spec)
+    gg = x["g"][..., ::G].contiguous()
+    dout, dhT = _cotangents(x, 61 + G, 2)
+    d = to_dev(x)
+    r = kda.kda_chunk_bwd(d["q"], d["k"], d["v"], gg.cuda(), d["beta"], dout.cuda(),
+                          h0=d["h0"], dhT=dhT.cuda())
+    torch.cuda.synchronize()
+    ref = oracle.backward(x["q"], x["k"], x["v"], gg, x["beta"], dout, x["h0"], dhT)
+    assert tuple(r["dg"].shape) == tuple(gg.shape)
+    ref["dg"] = ref["dg"].reshape(*gg.shape, G).sum(-1)
+    _assert_close(r, ref)
