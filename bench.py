@@ -69,6 +69,70 @@ def decode_bytes(N: int, H: int, dk: int, dv: int, s_in: int) -> int:
 # ---------------------------------------------------------------------------
 # clocks sampled during the timed region
 # ---------------------------------------------------------------------------
+class NvmlClockSampler:
+    """Polls the GPU's SM clock, max clock, power and clock-event reasons every 2 ms
+    through NVML (read-only queries) and keeps them as ClockSampler-style rows."""
+    FIELDS = None
+
+    def __init__(self, gpu_index: int):
+        import pynvml
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        self.h = pynvml.nvmlDeviceGetHandleByIndex(gpu_index)
+        self.max_sm = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        g = lambda *names, d: next((getattr(pynvml, n) for n in names if hasattr(pynvml, n)), d)
+        self.bits = [g("nvmlClocksEventReasonHwSlowdown", "nvmlClocksThrottleReasonHwSlowdown",
+                       d=0x8),
+                     g("nvmlClocksEventReasonHwThermalSlowdown",
+                       "nvmlClocksThrottleReasonHwThermalSlowdown", d=0x40),
+                     g("nvmlClocksEventReasonSwThermalSlowdown",
+                       "nvmlClocksThrottleReasonSwThermalSlowdown", d=0x20),
+                     g("nvmlClocksEventReasonSwPowerCap", "nvmlClocksThrottleReasonSwPowerCap",
+                       d=0x4)]
+        self.lines: list[str] = []
+        self.stop_ev = threading.Event()
+        self.t = None
+
+    def start(self):
+        self.t = threading.Thread(target=self._poll, daemon=True)
+        self.t.start()
+
+    def _poll(self):
+        nv = self.nv
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self.stop_ev.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                pw = nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+                rs = get_reasons(self.h)
+                flags = ["Active" if rs & b else "Not Active" for b in self.bits]
+                self.lines.append(", ".join([str(sm), str(self.max_sm), f"{pw:.1f}"] + flags))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def mark(self) -> int:
+        return len(self.lines)
+
+    def stop(self):
+        self.stop_ev.set()
+        if self.t is not None:
+            self.t.join(timeout=2)
+
+    def summary(self, lo: int, hi: int) -> dict:
+        return ClockSampler.summarize(self.lines[lo:hi] or self.lines[-3:])
+
+
+def make_clock_sampler(gpu_index: int):
+    """NVML polling when available (dense samples even in short timed regions), else
+    nvidia-smi's loop mode."""
+    try:
+        return NvmlClockSampler(gpu_index)
+    except Exception:
+        return ClockSampler(gpu_index)
+
+
 class ClockSampler:
     FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw",
               "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
@@ -110,10 +174,14 @@ class ClockSampler:
                 self.t.join(timeout=2)
 
     def summary(self, lo: int, hi: int) -> dict:
+        return ClockSampler.summarize(self.lines[lo:hi] or self.lines[-3:])
+
+    @staticmethod
+    def summarize(lines) -> dict:
         rows = []
-        for line in self.lines[lo:hi] or self.lines[-3:]:
+        for line in lines:
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) == len(self.FIELDS):
+            if len(parts) == len(ClockSampler.FIELDS):
                 rows.append(parts)
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
@@ -672,7 +740,7 @@ def run_ours(args, world, rank, local):
     hbm, tf_burst, tf_sust, peak_kind = _peaks()
     stream = torch.cuda.current_stream()
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
-    clocks = ClockSampler(int(vis.split(",")[local]) if vis else local)
+    clocks = make_clock_sampler(int(vis.split(",")[local]) if vis else local)
     clocks.start()
     time.sleep(0.3)
     pf = None
