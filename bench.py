@@ -202,15 +202,38 @@ def _dist():
 
 
 def run_reference(args, world, rank):
-    """The float64 oracle on the host cores, bounded sample of the workload."""
+    """The float64 oracle on the host cores: W untimed and K timed steps, each step one
+    pass over a bounded sample of the workload (its first --ref-tokens tokens, default
+    1024, all heads), so that the whole run ends within minutes."""
     if rank != 0:
         return 0
     import kda_inputs as ki
-    val, threads, desc, times = _oracle_timing(args)
+    import oracle
+    oracle.build()
     x = ki.make_prefill(args.workload)
+    Tb = min(x["T"], args.ref_tokens if args.ref_tokens > 0 else 1024)
+    q, k, v, g, b = (x[n][:, :Tb] for n in ("q", "k", "v", "g", "beta"))
+    cu = None
+    if x["cu_seqlens"] is not None:
+        import torch
+        cu = torch.clamp(x["cu_seqlens"], max=Tb)
+    pairs = (q.shape[0] if cu is None else cu.numel() - 1) * x["H"]
+    threads = max(1, min(oracle.max_threads(), pairs))
+    step = lambda: oracle.prefill(q, k, v, g, b, None, cu, nthreads=threads)
+    for _ in range(args.warmup):
+        step()
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        step()
+        times.append(time.perf_counter() - t0)
+    tok = Tb * q.shape[0]
+    val = tok * len(times) / sum(times)
+    desc = (f"first {Tb} tokens x {x['H']} heads of the {args.workload} workload per step, "
+            f"float64 recurrence, {threads} threads")
     line = {
         "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus,
-        "steps": len(times), "warmup": 0, "ms_per_step": 1e3 * statistics.median(times),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / len(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": _config(args, x, world),
         "cpu_baseline": {"value": val, "unit": UNIT, "cores": threads, "kind": "oracle",
@@ -819,9 +842,10 @@ def main():
                     help="sequences in the decode leg (0 = the config-4 value, 256)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-tokens", type=int, default=0,
-                    help="tokens of the workload the oracle processes per pass (0 = all)")
+                    help="tokens of the workload the oracle processes per pass (0: all for "
+                         "the cpu_baseline leg, 1024 per step for --impl reference)")
     ap.add_argument("--ref-seconds", type=float, default=10.0,
-                    help="repeat oracle passes until this much time has passed")
+                    help="cpu_baseline leg: repeat oracle passes until this much time has passed")
     ap.add_argument("--ingest-ncu", default="",
                     help="write profiles/traffic.json from this ncu --csv launch list (no GPU run)")
     args = ap.parse_args()
