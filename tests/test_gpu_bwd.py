@@ -158,3 +158,21 @@ def test_bwd_grouped_decay_matches_oracle(dtype, dk, dv, G):
     assert tuple(r["dg"].shape) == tuple(gg.shape)
     ref["dg"] = ref["dg"].reshape(*gg.shape, G).sum(-1)
     _assert_close(r, ref)
+
+
+def test_bwd_grouped_packed_documents():
+    spec = ki.PrefillSpec("varlen", B=0, T=0, H=2, dk=128, dv=128, dtype="bf16", decay="alog",
+                          seed=71, h0=True, varlen=True)
+    x = ki.make_prefill(spec, doc_lens=[100, 0, 64, 33])
+    G = 64
+    gg = x["g"][..., ::G].contiguous()
+    nseq = x["cu_seqlens"].numel() - 1
+    dout, dhT = _cotangents(x, 72, nseq)
+    d = to_dev(x)
+    r = kda.kda_chunk_bwd(d["q"], d["k"], d["v"], gg.cuda(), d["beta"], dout.cuda(),
+                          h0=d["h0"], dhT=dhT.cuda(), cu_seqlens=d["cu_seqlens"])
+    torch.cuda.synchronize()
+    ref = oracle.backward(x["q"], x["k"], x["v"], gg, x["beta"], dout, x["h0"], dhT,
+                          x["cu_seqlens"])
+    ref["dg"] = ref["dg"].reshape(*gg.shape, G).sum(-1)
+    _assert_close(r, ref)

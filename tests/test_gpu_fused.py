@@ -103,3 +103,15 @@ def test_fused_rejects_f32_and_half_conv():
     with pytest.raises(ValueError):
         kda.kda_chunk_fwd_fused(d["q_raw"], d["k_raw"], d["v"], d["g"], d["beta"],
                                 conv_q=d["conv_q"])
+
+
+def test_fused_packed_long_documents_segmented():
+    """Packed documents long enough for the segmented state pass (16-chunk segments):
+    the gate applies in both passes, the convolution restarts per document."""
+    spec = ki.PrefillSpec("varlen", B=0, T=0, H=2, dk=128, dv=128, dtype="bf16", decay="alog",
+                          seed=43, h0=True, varlen=True)
+    x = ki.make_fused_prefill(spec, W=4, doc_lens=[1500, 70, 1100, 700])
+    out, hT = _run(x)
+    o_ref, s_ref = _ref(x)
+    assert rel_err(out, o_ref) <= TOL["bf16"]
+    assert rel_err(hT, s_ref) <= TOL["bf16"]
