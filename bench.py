@@ -367,32 +367,56 @@ def prefill_leg(args, world, rank, dev, stream, barrier, clocks):
     ms_max = _max_over_ranks(t_start.elapsed_time(t_end), world, dev)
     call_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
 
-    # e2e: pinned host buffers -> device -> kda_chunk_fwd -> host, all timed
+    # e2e: pinned host buffers -> device -> kda_chunk_fwd -> host, all timed.  Steps are
+    # pipelined over three streams with two device buffer sets: while step i computes,
+    # step i+1's inputs are copied in and step i-1's outputs copied out (events order
+    # every reuse of a buffer); every step's copies are inside the timed region.
     hx = {n: x0[n].cpu().pin_memory() for n in ("q", "k", "v", "g", "beta")}
-    h_out = torch.empty(x0["out"].shape, dtype=x0["out"].dtype).pin_memory()
-    h_hT = torch.empty(x0["hT"].shape, dtype=torch.float32).pin_memory()
-    dx = {n: torch.empty_like(x0[n]) for n in hx}
+    h_out = [torch.empty(x0["out"].shape, dtype=x0["out"].dtype).pin_memory() for _ in range(2)]
+    h_hT = [torch.empty(x0["hT"].shape, dtype=torch.float32).pin_memory() for _ in range(2)]
+    dx = [{n: torch.empty_like(x0[n]) for n in hx} for _ in range(2)]
+    dout = [torch.empty_like(x0["out"]) for _ in range(2)]
+    dhT = [torch.empty_like(x0["hT"]) for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in hx.values())
-    d2h = h_out.numel() * h_out.element_size() + h_hT.numel() * 4
+    d2h = h_out[0].numel() * h_out[0].element_size() + h_hT[0].numel() * 4
     e2e_steps = max(3, args.steps // 4)
+    cp_in, cp_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    for e in ev_comp + ev_out:
+        e.record(stream)
 
-    def e2e_step():
-        for n in hx:
-            dx[n].copy_(hx[n], non_blocking=True)
-        kda.kda_chunk_fwd(dx["q"], dx["k"], dx["v"], dx["g"], dx["beta"], h0=x0["h0"],
-                          cu_seqlens=x0["cu_seqlens"], out=x0["out"], hT=x0["hT"],
+    def e2e_step(i):
+        b = i & 1
+        cp_in.wait_event(ev_comp[b])            # step i-2 no longer reads dx[b]
+        with torch.cuda.stream(cp_in):
+            for n in hx:
+                dx[b][n].copy_(hx[n], non_blocking=True)
+        ev_in[b].record(cp_in)
+        stream.wait_event(ev_in[b])
+        stream.wait_event(ev_out[b])           # step i-2's outputs have left dout[b], dhT[b]
+        kda.kda_chunk_fwd(dx[b]["q"], dx[b]["k"], dx[b]["v"], dx[b]["g"], dx[b]["beta"],
+                          h0=x0["h0"], cu_seqlens=x0["cu_seqlens"], out=dout[b], hT=dhT[b],
                           stream=stream)
-        h_out.copy_(x0["out"], non_blocking=True)
-        h_hT.copy_(x0["hT"], non_blocking=True)
+        ev_comp[b].record(stream)
+        cp_out.wait_event(ev_comp[b])
+        with torch.cuda.stream(cp_out):
+            h_out[b].copy_(dout[b], non_blocking=True)
+            h_hT[b].copy_(dhT[b], non_blocking=True)
+        ev_out[b].record(cp_out)
 
-    for _ in range(2):
-        e2e_step()
+    for i in range(2):
+        e2e_step(i)
     torch.cuda.synchronize()
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
+    cp_in.wait_event(e0)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    stream.wait_event(ev_out[(e2e_steps - 1) & 1])
+    stream.wait_event(ev_out[e2e_steps & 1])
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
