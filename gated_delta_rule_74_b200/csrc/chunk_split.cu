@@ -253,14 +253,17 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
           wt[j] = make_float2(__ldg(w + ((long long)h * dk + c0) * convW + i),
                               __ldg(w + ((long long)h * dk + c0 + 1) * convW + i));
       }
-      // rows 16 a - 3 .. 16 a + 15, all loads issued before any use
+      // rows 16 a - 3 .. 16 a + 15, all loads issued before any use; one pointer walks
+      // the rows (stride H dk), rows outside [doc0 - rbase, L) read as zero
       uint32_t u[19];
+      const int rlo = (int)max(doc0 - rbase, -3LL) - (16 * a - 3);   // first valid m
+      const int rhi = L - (16 * a - 3);                              // first invalid m
+      const long long stride = (long long)H * dk;
+      const bf16* px = x + ((rbase + 16 * a - 3) * H + h) * dk + c0;
 #pragma unroll
       for (int m = 0; m < 19; ++m) {
-        const int r = 16 * a - 3 + m;
-        const bool ok = c0 < dk && r < L && rbase + r >= doc0;
-        u[m] = ok ? __ldg(reinterpret_cast<const unsigned int*>(x + ((rbase + r) * H + h) * dk + c0))
-                  : 0u;
+        const bool ok = c0 < dk && m >= rlo && m < rhi;
+        u[m] = ok ? __ldg(reinterpret_cast<const unsigned int*>(px + m * stride)) : 0u;
       }
       auto raw = [&](int m) { return make_float2(bf_lo(u[m]), bf_hi(u[m])); };
       float2 w0 = raw(0), w1 = raw(1), w2 = raw(2);
@@ -293,14 +296,18 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   const uint32_t tb = tmem_base_sh;
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
   if constexpr (CONV) {                 // L2 norms of this block's rows (two warps' sums)
-    const float qs = 1.f / sqrtf((float)dk);
+    // lane l < 16 forms row l's inverse norms; the other lanes take them by shuffle
+    const int lr = (tid & 31) & 15;
+    const float ik_l = rsqrtf(fmaxf(s_ss[((a * 2) * 2) * 16 + lr] +
+                                        s_ss[((a * 2 + 1) * 2) * 16 + lr],
+                                    kNormEps2));
+    const float iq_l = rsqrtf(fmaxf(s_ss[((a * 2) * 2 + 1) * 16 + lr] +
+                                        s_ss[((a * 2 + 1) * 2 + 1) * 16 + lr],
+                                    kNormEps2) * (float)dk);
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
-      const float ik = rsqrtf(fmaxf(s_ss[((a * 2) * 2) * 16 + e] + s_ss[((a * 2 + 1) * 2) * 16 + e],
-                                    kNormEps2));
-      const float iq = rsqrtf(fmaxf(s_ss[((a * 2) * 2 + 1) * 16 + e] +
-                                        s_ss[((a * 2 + 1) * 2 + 1) * 16 + e],
-                                    kNormEps2)) * qs;
+      const float ik = __shfl_sync(0xffffffffu, ik_l, e);
+      const float iq = __shfl_sync(0xffffffffu, iq_l, e);
       kf[e].x *= ik; kf[e].y *= ik;
       qf[e].x *= iq; qf[e].y *= iq;
     }
