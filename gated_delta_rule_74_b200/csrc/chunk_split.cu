@@ -25,8 +25,11 @@
 //     [O^T | P]   [dv x 128] = S^T [Qbar^T | W^T]^T      (S^T bf16 copy in TMEM)
 //     Delta^T = U^T - P
 //     [S^T | O^T] [dv x 192] += Delta^T [Kend^T ; Aqk]^T  (after S^T <- S^T Diag(exp(G_last)))
-// with one bulk copy per record, two records ahead.  S^T stays in TMEM in fp32
-// for the whole chain.  Packed documents restart the state from their own h0
+// with one bulk copy per record, two records ahead.  The first product runs on bf16
+// operands; the second on f16 ones (Delta, Kend and Aqk are bounded -- |Kend|,
+// |Aqk| <= 1 for unit-norm keys -- and f16's 11-bit significand halves the
+// output error against bf16's 8 bits; conversions saturate at the f16 range).
+// S^T stays in TMEM in fp32 for the whole chain.  Packed documents restart the state from their own h0
 // slot and restart chunking at the document start (Mini-K3-1H-mamba2 card,
 // packed-document paragraph: state flow resets at every boundary).
 //
@@ -64,7 +67,7 @@ constexpr uint32_t kWaitLimit = 1u << 22;
 // ---- chunk record (one per (head, chunk)), byte offsets
 constexpr uint32_t REC_QW = 0;          // [Qbar^T | W^T]: MN-major SW128, N = 128 (2 x 64 tokens,
                                         // 16 KB apart), K = dk
-constexpr uint32_t REC_KA = 32768;      // [Kend^T ; Aqk]: K-major SW128, 192 rows x 64 tokens
+constexpr uint32_t REC_KA = 32768;      // [Kend^T ; Aqk] (f16): K-major SW128, 192 rows x 64 tokens
 constexpr uint32_t REC_AQK = REC_KA + 16384;
 constexpr uint32_t REC_U = 57344;       // U^T [dv][64 tokens] fp32: 256-byte rows, 16-byte
                                         // chunks XOR-swizzled with (row % 16)
@@ -105,7 +108,7 @@ constexpr uint32_t ST_S = 0;            // S^T fp32        [128 lanes x 128]
 constexpr uint32_t ST_O = 128;          // O^T             [128 x 64]
 constexpr uint32_t ST_P = 192;          // P               [128 x 64]
 constexpr uint32_t ST_SB = 256;         // S^T bf16 (A)    [128 x 64]
-constexpr uint32_t ST_D = 320;          // Delta^T bf16 (A) [128 x 32]
+constexpr uint32_t ST_D = 320;          // Delta^T f16 (A)  [128 x 32]
 constexpr uint32_t kStateTmemCols = 512;
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -114,6 +117,12 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 __device__ __forceinline__ uint4 pack8(const float (&x)[8], float s) {
   return make_uint4(pack_bf16(x[0] * s, x[1] * s), pack_bf16(x[2] * s, x[3] * s),
                     pack_bf16(x[4] * s, x[5] * s), pack_bf16(x[6] * s, x[7] * s));
+}
+// the same as f16 (the [Kend^T ; Aqk] operand and Delta^T are f16: the second MMA
+// of the state step runs in kind::f16 with f16 A and B)
+__device__ __forceinline__ uint4 pack8_f16(const float (&x)[8], float s) {
+  return make_uint4(pack_f16(x[0] * s, x[1] * s), pack_f16(x[2] * s, x[3] * s),
+                    pack_f16(x[4] * s, x[5] * s), pack_f16(x[6] * s, x[7] * s));
 }
 __device__ __forceinline__ void sts16(uint8_t* base, uint32_t off, uint4 v) {
   *reinterpret_cast<uint4*>(base + off) = v;
@@ -371,7 +380,7 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
         if (a2 >= a) sts16(sm, q_r(a2) + chunk_mnmajor_sw32(g8, c, D), pack8(kr, f[a2]));
       // record: Qbar^T (MN-major, N = tokens, K = channels) and Kend^T (K-major)
       *reinterpret_cast<uint4*>(rc + REC_QW + chunk_mnmajor_sw128(g8, c, D)) = pack8(lq, eP);
-      *reinterpret_cast<uint4*>(rc + REC_KA + chunk_kmajor_sw128(c, g8, D)) = pack8(kr, eE);
+      *reinterpret_cast<uint4*>(rc + REC_KA + chunk_kmajor_sw128(c, g8, D)) = pack8_f16(kr, eE);
     }
   }
   if (a == 3)
@@ -457,7 +466,7 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
 #pragma unroll
           for (int e = 0; e < 8; ++e)
             w[e] = (c8 * 8 + e <= r) ? __uint_as_float(tv[c8 >> 1][(c8 & 1) * 8 + e]) : 0.f;
-          sts16(sm, Q_OAQK + chunk_kmajor_sw128(r, c8, C), pack8(w, 1.f));
+          sts16(sm, Q_OAQK + chunk_kmajor_sw128(r, c8, C), pack8_f16(w, 1.f));
         }
       }
     }
@@ -860,7 +869,7 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
     tc_fence_after();
     if (__syncthreads_or(!good)) { alive = false; break; }
 
-    // ---- Delta^T = U^T - P for tokens [16 wq, 16 wq + 16) -> bf16 TMEM
+    // ---- Delta^T = U^T - P for tokens [16 wq, 16 wq + 16) -> f16 TMEM
     {
       uint32_t tp[16];
       tmem_ld16(tl + ST_P + 16 * wq, tp);
@@ -874,10 +883,10 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
       uint32_t dw[8];
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) {
-        dw[2 * c4] = pack_bf16(u[c4].x - __uint_as_float(tp[4 * c4]),
-                               u[c4].y - __uint_as_float(tp[4 * c4 + 1]));
-        dw[2 * c4 + 1] = pack_bf16(u[c4].z - __uint_as_float(tp[4 * c4 + 2]),
-                                   u[c4].w - __uint_as_float(tp[4 * c4 + 3]));
+        dw[2 * c4] = pack_f16(u[c4].x - __uint_as_float(tp[4 * c4]),
+                              u[c4].y - __uint_as_float(tp[4 * c4 + 1]));
+        dw[2 * c4 + 1] = pack_f16(u[c4].z - __uint_as_float(tp[4 * c4 + 2]),
+                                  u[c4].w - __uint_as_float(tp[4 * c4 + 3]));
       }
       tmem_st8(tl + ST_D + 8 * wq, dw);
       tmem_wait_st();
@@ -890,7 +899,7 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
       tc_fence_after();
       const uint32_t ka = smem_u32(rb + REC_KA);
       const int n = outputs ? D + C : D;
-      const uint32_t id = idesc_bf16(128, n, false, false);
+      const uint32_t id = idesc_f16(128, n, false, false);   // f16 A (Delta^T) and B
 #pragma unroll
       for (int kk = 0; kk < C / 16; ++kk)
         mma_ts(tb + ST_S, tb + ST_D + kk * 8, desc_kmajor_sw128(ka, n, kk), id, 1);

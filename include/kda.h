@@ -94,8 +94,10 @@ typedef enum {
  * unsplit instead.
  *
  * Precision: g, beta and the state are fp32.  With KDA_BF16 inputs the chunk
- * contractions run on the tensor cores with bf16 operands and fp32
- * accumulation; with KDA_F32 inputs every step runs in fp32 on the CUDA cores.
+ * contractions run on the tensor cores with fp32 accumulation, on bf16 operands
+ * except the state update's second product (Delta, Kend, Aqk), which runs on
+ * f16 operands (finer rounding; values beyond +-65504 saturate there); with
+ * KDA_F32 inputs every step runs in fp32 on the CUDA cores.
  *
  * Returns KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED or KDA_ERR_CUDA.
  */
