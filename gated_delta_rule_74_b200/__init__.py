@@ -19,7 +19,7 @@ from typing import Optional
 
 import torch
 
-__all__ = ["kda_chunk_fwd", "kda_chunk_fwd_fused", "kda_chunk_bwd", "kda_decode_step", "kda_decode_tokens", "kda_status_string", "kda_version",
+__all__ = ["kda_chunk_fwd", "kda_chunk_fwd_fused", "kda_chunk_bwd", "kda_device_status", "kda_decode_step", "kda_decode_tokens", "kda_status_string", "kda_version",
            "kda_launch_count",
            "lib", "library_path", "header_symbols", "KdaError",
            "KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED", "KDA_ERR_CUDA",
@@ -81,6 +81,10 @@ def lib() -> ctypes.CDLL:
         L.kda_chunk_bwd_grouped.argtypes = [vp, vp, vp, fp, fp, fp, vp, vp, fp,
                                             fp, fp, fp, fp, fp, fp] + [ip] * 7 + [vp]
         L.kda_chunk_bwd_grouped.restype = ctypes.c_int
+        L.kda_device_status.argtypes = [ip]
+        L.kda_device_status.restype = ctypes.c_int
+        L.kda_selftest_bounded_wait.argtypes = [ctypes.c_uint, vp]
+        L.kda_selftest_bounded_wait.restype = ctypes.c_int
         L.kda_status_string.argtypes = [ctypes.c_int]
         L.kda_status_string.restype = ctypes.c_char_p
         L.kda_version.argtypes = []
@@ -111,6 +115,22 @@ def kda_status_string(status: int) -> str:
 
 def kda_version() -> int:
     return int(lib().kda_version())
+
+
+def kda_device_status(reset: bool = True) -> int:
+    """KDA_OK, or KDA_ERR_TIMEOUT if a bounded device-side wait of the library's kernels
+    gave up since the last reset (synchronizes the device; see include/kda.h)."""
+    rc = int(lib().kda_device_status(1 if reset else 0))
+    if rc not in (KDA_OK, KDA_ERR_TIMEOUT):
+        raise KdaError("kda_device_status", rc)
+    return rc
+
+
+def kda_selftest_bounded_wait(polls: int = 1000, stream=None) -> None:
+    """Launch the self-test whose wait nothing completes (see include/kda.h)."""
+    rc = lib().kda_selftest_bounded_wait(int(polls), _stream(stream))
+    if rc != KDA_OK:
+        raise KdaError("kda_selftest_bounded_wait", rc)
 
 
 def kda_launch_count() -> int:

@@ -206,6 +206,23 @@ int kda_chunk_bwd_grouped(const void* q, const void* k, const void* v, const flo
                         B, T, H, dk_dim, dv_dim, group_shift(g_group, dk_dim), in_dtype, stream);
 }
 
+int kda_device_status(int reset) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return status_from(cudaErrorUnknown);
+  int any = 0;
+  for (auto take : {kda::take_split_timeout, kda::take_tc_timeout, kda::take_bwd_timeout,
+                    kda::take_combine_timeout, kda::take_selftest_timeout}) {
+    int f = 0;
+    if (take(&f, reset != 0) != cudaSuccess) return status_from(cudaErrorUnknown);
+    any |= f;
+  }
+  return any ? KDA_ERR_TIMEOUT : KDA_OK;
+}
+
+int kda_selftest_bounded_wait(unsigned polls, void* stream) {
+  if (polls < 1 || polls > (1u << 20)) return KDA_ERR_INVALID_ARG;
+  return status_from(kda::launch_selftest_wait(polls, static_cast<cudaStream_t>(stream)));
+}
+
 const char* kda_status_string(int status) {
   switch (status) {
     case KDA_OK: return "KDA_OK";

@@ -1139,4 +1139,16 @@ cudaError_t launch_chunk_split(const void* q, const void* k, const void* v, cons
   return e;
 }
 
+// Reads (and with reset clears) g_chunk_split_timeout; host side of kda_device_status.
+cudaError_t take_split_timeout(int* flag, bool reset) {
+  int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_chunk_split_timeout, sizeof(int));
+  if (e == cudaSuccess && reset && v != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_chunk_split_timeout, &zero, sizeof(int));
+  }
+  *flag = v;
+  return e;
+}
+
 }  // namespace kda

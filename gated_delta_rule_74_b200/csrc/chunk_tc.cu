@@ -931,4 +931,16 @@ int run_chunk_tc_static(const void* q, const void* k, const void* v, const float
   return KDA_OK;
 }
 
+// Reads (and with reset clears) g_chunk_tc_timeout; host side of kda_device_status.
+cudaError_t take_tc_timeout(int* flag, bool reset) {
+  int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_chunk_tc_timeout, sizeof(int));
+  if (e == cudaSuccess && reset && v != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_chunk_tc_timeout, &zero, sizeof(int));
+  }
+  *flag = v;
+  return e;
+}
+
 }  // namespace kda

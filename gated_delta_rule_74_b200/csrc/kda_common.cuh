@@ -80,6 +80,16 @@ cudaError_t launch_chunk_bwd(const void* q, const void* k, const void* v, const 
                              float* dg, float* dbeta, float* dh0, int B, int T, int H, int dkd,
                              int dvd, int gsh, int in_dtype, cudaStream_t stream);
 
+// Bounded-wait flags (one per kernel file): read, and with reset clear, the flag a
+// kernel raises when one of its bounded waits gives up.
+cudaError_t take_split_timeout(int* flag, bool reset);
+cudaError_t take_tc_timeout(int* flag, bool reset);
+cudaError_t take_bwd_timeout(int* flag, bool reset);
+cudaError_t take_combine_timeout(int* flag, bool reset);
+cudaError_t take_selftest_timeout(int* flag, bool reset);
+// One thread waits, at most `polls` polls, on an mbarrier phase nothing completes.
+cudaError_t launch_selftest_wait(uint32_t polls, cudaStream_t stream);
+
 // The tensor-core prefill on caller-provided scratch (allocates nothing).
 int run_chunk_tc_static(const void* q, const void* k, const void* v, const float* g,
                         const float* beta, const float* h0, const int32_t* cu_seqlens, void* out,

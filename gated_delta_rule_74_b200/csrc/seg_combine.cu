@@ -6,6 +6,10 @@
 #include "sm100.cuh"
 
 namespace kda {
+
+// Set when a bounded wait of the segment combine gives up (diagnostic).
+__device__ int g_seg_combine_timeout = 0;
+
 namespace {
 using namespace sm100;
 constexpr int D = kHead;
@@ -174,7 +178,10 @@ kda_seg_combine_kernel(const int32_t* __restrict__ cu_seqlens, int T, int H, Seg
     tc_fence_before();
     __syncthreads();
   }
-  if (!ok && tid == 0) mbar_wait(&bar, phase, 1u << 22);
+  if (!ok && tid == 0) {
+    atomicExch(&g_seg_combine_timeout, 1);
+    mbar_wait(&bar, phase, 1u << 22);
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -330,6 +337,7 @@ kda_seg_combine_img_kernel(const int32_t* __restrict__ cu_seqlens, int T, int H,
     __syncthreads();
   }
   if (!ok && tid == 0) {
+    atomicExch(&g_seg_combine_timeout, 1);
     mbar_wait(&mbar, mphase ^ 1u, kWait2);
     for (int r = waited + 1; r <= issued; ++r) mbar_wait(&xfull[(r - 1) & 1], (uint32_t)((r - 1) >> 1) & 1u, kWait2);
   }
@@ -382,6 +390,18 @@ cudaError_t launch_seg_combine_img(const int32_t* cu_seqlens, int B, int T, int 
                                          stream>>>(cu_seqlens, T, H, dk, dv, sa));
   note_launches(1);
   return cudaGetLastError();
+}
+
+// Reads (and with reset clears) g_seg_combine_timeout; host side of kda_device_status.
+cudaError_t take_combine_timeout(int* flag, bool reset) {
+  int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_seg_combine_timeout, sizeof(int));
+  if (e == cudaSuccess && reset && v != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_seg_combine_timeout, &zero, sizeof(int));
+  }
+  *flag = v;
+  return e;
 }
 
 }  // namespace kda

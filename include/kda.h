@@ -49,7 +49,7 @@ typedef enum {
   KDA_ERR_INVALID_ARG = -1,   /* null required pointer, bad size, misalignment */
   KDA_ERR_UNSUPPORTED = -2,   /* valid request this build does not implement   */
   KDA_ERR_CUDA = -3,          /* a CUDA runtime call or kernel launch failed    */
-  KDA_ERR_TIMEOUT = -4        /* reserved: a bounded device-side wait expired   */
+  KDA_ERR_TIMEOUT = -4        /* a bounded device-side wait expired (see kda_device_status) */
 } kda_status_t;
 
 typedef enum {
@@ -288,6 +288,29 @@ KDA_API int kda_chunk_bwd_grouped(const void* q, const void* k, const void* v,
                                   const float* dhT, float* dq, float* dk, float* dv, float* dg,
                                   float* dbeta, float* dh0, int B, int T, int H, int dk_dim,
                                   int dv_dim, int g_group, int in_dtype, void* stream);
+
+/*
+ * kda_device_status -- did a bounded device-side wait give up?
+ *
+ * Every wait of the library's kernels on an asynchronous copy or a tensor-core
+ * operation polls a bounded number of times.  If a limit runs out (a completion
+ * that never arrives), the kernel stops waiting -- its results are then invalid --
+ * raises a device flag and finishes, so the GPU never hangs on the library.  This
+ * call synchronizes the current device (cudaDeviceSynchronize), reads the flags and,
+ * with reset != 0, clears them.  Returns KDA_OK (no wait gave up since the library
+ * was loaded or since the last reset), KDA_ERR_TIMEOUT (at least one did) or
+ * KDA_ERR_CUDA (the device could not be synchronized or read).
+ */
+KDA_API int kda_device_status(int reset);
+
+/*
+ * kda_selftest_bounded_wait -- exercise the path above: launch one thread that
+ * waits, at most `polls` polls (1 .. 2^20), on an mbarrier phase that nothing
+ * completes, and raises the flag kda_device_status reports.  Asynchronous on
+ * `stream`; the device stays usable.  Returns KDA_OK, KDA_ERR_INVALID_ARG or
+ * KDA_ERR_CUDA.
+ */
+KDA_API int kda_selftest_bounded_wait(unsigned polls, void* stream);
 
 /* Human-readable name of a status code (static storage, never NULL). */
 KDA_API const char* kda_status_string(int status);

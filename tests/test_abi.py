@@ -137,3 +137,8 @@ def test_chunk_fwd_fused_rejects_unsupported(L, dims):
 def test_bwd_grouped_rejects_bad_group(L, G):
     assert L.kda_chunk_bwd_grouped(P, P, P, P, P, None, None, P, None, P, P, P, P, P, None,
                                    1, 4, 1, 128, 128, G, 0, None) == kda.KDA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("polls", [0, (1 << 20) + 1])
+def test_selftest_rejects_poll_counts(L, polls):
+    assert L.kda_selftest_bounded_wait(polls, None) == kda.KDA_ERR_INVALID_ARG
