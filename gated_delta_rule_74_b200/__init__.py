@@ -19,7 +19,8 @@ from typing import Optional
 
 import torch
 
-__all__ = ["kda_chunk_fwd", "kda_chunk_fwd_fused", "kda_chunk_bwd", "kda_device_status", "kda_decode_step", "kda_decode_tokens", "kda_status_string", "kda_version",
+__all__ = ["kda_chunk_fwd", "kda_chunk_fwd_fused", "kda_chunk_bwd", "kda_device_status",
+           "kda_decode_chunk", "kda_decode_step", "kda_decode_tokens", "kda_status_string", "kda_version",
            "kda_launch_count",
            "lib", "library_path", "header_symbols", "KdaError",
            "KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED", "KDA_ERR_CUDA",
@@ -68,6 +69,8 @@ def lib() -> ctypes.CDLL:
         L.kda_decode_step.restype = ctypes.c_int
         L.kda_decode_tokens.argtypes = [vp, vp, vp, fp, fp, fp, vp, ip, ip, ip, ip, ip, ip, vp]
         L.kda_decode_tokens.restype = ctypes.c_int
+        L.kda_decode_chunk.argtypes = [vp, vp, vp, fp, fp, fp, vp, ip, ip, ip, ip, ip, ip, vp]
+        L.kda_decode_chunk.restype = ctypes.c_int
         L.kda_decode_tokens_grouped.argtypes = [vp, vp, vp, fp, fp, fp, vp] + [ip] * 7 + [vp]
         L.kda_decode_tokens_grouped.restype = ctypes.c_int
         L.kda_chunk_fwd_grouped.argtypes = [vp, vp, vp, fp, fp, fp, vp, vp, fp] + [ip] * 7 + [vp]
@@ -418,4 +421,33 @@ def kda_decode_tokens(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torc
                                              _stream(stream))
     if rc != KDA_OK:
         raise KdaError("kda_decode_tokens", rc)
+    return out
+
+
+def kda_decode_chunk(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+                     beta: torch.Tensor, S: torch.Tensor, out: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """L <= 16 tokens per (sequence, head) as one chunk of the chunked form on the tensor
+    cores (bf16, dk = dv = 128).  Same layout and in-place S update as kda_decode_tokens;
+    equal to L single steps up to the tensor-core rounding.  Returns out [N,L,H,dv]."""
+    if q.dim() != 4:
+        raise ValueError("q must be [N, L, H, dk]")
+    N, L, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = _DTYPES.get(q.dtype)
+    if dt is None:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    _check("q", q)
+    _check("k", k, q.dtype, (N, L, H, dk))
+    _check("v", v, q.dtype, (N, L, H, dv))
+    _check("g", g, torch.float32, (N, L, H, dk))
+    _check("beta", beta, torch.float32, (N, L, H))
+    _check("S", S, torch.float32, (N, H, dk, dv))
+    if out is None:
+        out = torch.empty((N, L, H, dv), dtype=q.dtype, device=q.device)
+    _check("out", out, q.dtype, (N, L, H, dv))
+    rc = lib().kda_decode_chunk(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S),
+                                _ptr(out), N, L, H, dk, dv, dt, _stream(stream))
+    if rc != KDA_OK:
+        raise KdaError("kda_decode_chunk", rc)
     return out

@@ -124,6 +124,20 @@ int kda_decode_tokens(const void* q, const void* k, const void* v, const float* 
   return decode_tokens_impl(q, k, v, g, beta, S, out, N, L, H, dk, dv, 0, in_dtype, stream);
 }
 
+int kda_decode_chunk(const void* q, const void* k, const void* v, const float* g,
+                     const float* beta, float* S, void* out, int N, int L, int H, int dk, int dv,
+                     int in_dtype, void* stream) {
+  if (N < 1 || L < 1 || H < 1) return KDA_ERR_INVALID_ARG;
+  if (in_dtype != KDA_BF16 && in_dtype != KDA_F32) return KDA_ERR_INVALID_ARG;
+  if (!pointers_ok({q, k, v, g, beta, S, out}, {})) return KDA_ERR_INVALID_ARG;
+  if (!head_ok(dk) || !head_ok(dv)) return KDA_ERR_UNSUPPORTED;
+  if (!kda::decode_chunk_supported(dk, dv, in_dtype, L)) return KDA_ERR_UNSUPPORTED;
+  if ((long long)N * H > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
+  if ((long long)N * L * H * (dk > dv ? dk : dv) > (1LL << 40)) return KDA_ERR_INVALID_ARG;
+  return status_from(kda::launch_decode_chunk(q, k, v, g, beta, S, out, N, L, H,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
 int kda_decode_tokens_grouped(const void* q, const void* k, const void* v, const float* g,
                               const float* beta, float* S, void* out, int N, int L, int H, int dk,
                               int dv, int g_group, int in_dtype, void* stream) {
@@ -210,7 +224,8 @@ int kda_device_status(int reset) {
   if (cudaDeviceSynchronize() != cudaSuccess) return status_from(cudaErrorUnknown);
   int any = 0;
   for (auto take : {kda::take_split_timeout, kda::take_tc_timeout, kda::take_bwd_timeout,
-                    kda::take_combine_timeout, kda::take_selftest_timeout}) {
+                    kda::take_combine_timeout, kda::take_selftest_timeout,
+                    kda::take_decode_chunk_timeout}) {
     int f = 0;
     if (take(&f, reset != 0) != cudaSuccess) return status_from(cudaErrorUnknown);
     any |= f;

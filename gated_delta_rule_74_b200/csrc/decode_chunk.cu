@@ -1,0 +1,438 @@
+// Multi-token decode in the chunked form on the tensor cores (kda_decode_chunk).
+//
+// For each (sequence n, head h) the L <= 16 new tokens form one chunk of the
+// chunked form (miniKimiK3 model card, "Kimi Delta Attention" bullet: the chunked
+// parallel form equals the recurrence), applied to the stored state S:
+//     Gamma = cumsum g;  Qbar = q e^Gamma;  Kbar = k e^Gamma;  Kend_i = k_i e^(Gamma_last - Gamma_i)
+//     A_ri   = sum_c k_rc k_ic e^(Gamma_rc - Gamma_ic)   (i < r),   T = (I + diag(beta) A)^-1
+//     Aqk_ri = sum_c q_rc k_ic e^(Gamma_rc - Gamma_ic)   (i <= r)
+//     W = T diag(beta) Kbar,  U = T diag(beta) V,  Delta = U - W S
+//     O = Qbar S + Aqk Delta,  S' = Diag(e^Gamma_last) S + Kend^T Delta.
+// One CTA per (n, h), 256 threads.  The chunk-local quantities (16 tokens) are
+// formed on the CUDA cores in fp32, with the decay differences split through token
+// 8 (factors e^(+-(Gamma - Gamma_8)), clamped at e^80); the three products with
+// the state run on the tensor cores with S^T resident in TMEM:
+//     [O^T | P]   (128 x 32)  = S^T [Qbar ; W]^T          bf16 operands
+//     S^T        (128 x 128) += Delta^T Kend              f16 operands
+//     O^T        (128 x 16)  += Delta^T Aqk^T             f16 operands
+// S is read from and written back to HBM once for all L tokens.  Tokens L .. 15
+// are zero (q = k = v = g = beta = 0) and contribute nothing.
+//
+// TMEM (256 columns, two CTAs per SM): S^T fp32 [0, 128), [O^T | P] fp32
+// [128, 160), S^T as bf16 pairs [160, 224), Delta^T as f16 pairs [224, 232).
+#include "kda_common.cuh"
+#include "sm100.cuh"
+
+namespace kda {
+
+// Set when a bounded wait of the chunked decode gives up (diagnostic).
+__device__ int g_decode_chunk_timeout = 0;
+
+namespace {
+using namespace sm100;
+using bf16 = __nv_bfloat16;
+
+constexpr int D = 128;                 // dk = dv
+constexpr int LT = 16;                 // tokens per call (padded)
+constexpr int NT = 256;
+constexpr int LDF = D + 4;             // fp32 row stride of the token tiles (bank spread)
+constexpr uint32_t kWaitLimit = 1u << 22;
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t T_S = 0, T_OP = 128, T_SB = 160, T_D = 224;
+
+// shared memory (bytes, from a 1024-aligned base)
+constexpr uint32_t M_B1 = 0;                      // [Qbar ; W] bf16, MN-major SW32, N 32 x K 128 (8 KB)
+constexpr uint32_t M_KE = M_B1 + 8192;            // Kend f16, MN-major SW128, N 128 x K 16 (4 KB)
+constexpr uint32_t M_AQ = M_KE + 4096;            // Aqk^T f16, MN-major SW32, N 16 x K 16 (512 B)
+constexpr uint32_t M_F = M_AQ + 1024;             // fp32 tiles [16][LDF]
+// q, k, v, Gamma, U = T beta V, and the Gram factors k e^(G - G_8), k e^(G_8 - G),
+// q e^(G - G_8) (the first and last later hold Kbar = k e^G and W)
+constexpr uint32_t F_Q = 0, F_K = 1, F_V = 2, F_G = 3, F_U = 4, F_KP = 5, F_KM = 6, F_QP = 7;
+constexpr uint32_t M_SMALL = M_F + 8 * LT * LDF * 4;   // A, Aqk, T (16 x 16 fp32 each), beta, gamma_last
+constexpr uint32_t DC_SMEM = M_SMALL + 3 * 256 * 4 + 64 + D * 4 + 1024;
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+__device__ __forceinline__ uint4 pack8_bf16(const float (&x)[8]) {
+  return make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
+                    pack_bf16(x[6], x[7]));
+}
+__device__ __forceinline__ uint4 pack8_f16v(const float (&x)[8]) {
+  return make_uint4(pack_f16(x[0], x[1]), pack_f16(x[2], x[3]), pack_f16(x[4], x[5]),
+                    pack_f16(x[6], x[7]));
+}
+
+__global__ void __launch_bounds__(NT, 2)
+kda_decode_chunk_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
+                        const bf16* __restrict__ v, const float* __restrict__ g,
+                        const float* __restrict__ beta, float* __restrict__ S,
+                        bf16* __restrict__ out, int L, int H) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = align1024(smem_raw);
+  __shared__ uint64_t mbar;
+  __shared__ uint32_t tmem_base_sh;
+  float* const F = reinterpret_cast<float*>(sm + M_F);
+  float* const fq = F + F_Q * LT * LDF;          // q, later Qbar-ready raw q
+  float* const fk = F + F_K * LT * LDF;          // k
+  float* const fv = F + F_V * LT * LDF;          // v
+  float* const fG = F + F_G * LT * LDF;          // g, then Gamma
+  float* const fU = F + F_U * LT * LDF;          // U = T beta V
+  float* const fKP = F + F_KP * LT * LDF;        // k e^(G - G_8), then Kbar = k e^G
+  float* const fKM = F + F_KM * LT * LDF;        // k e^(G_8 - G)
+  float* const fQP = F + F_QP * LT * LDF;        // q e^(G - G_8), then W
+  float* const sA = reinterpret_cast<float*>(sm + M_SMALL);   // A [16][16] (row r, column i)
+  float* const sAqk = sA + 256;                               // Aqk [16][16]
+  float* const sT = sAqk + 256;                               // T beta [16][16]
+  float* const sBeta = sT + 256;                              // [16]
+  float* const sGl = sBeta + 16;                              // exp(Gamma_last) [128]
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long long pr = blockIdx.x;               // flat (n, h)
+  const long long n = pr / H;
+  const int h = (int)(pr - n * H);
+  float* const Sp = S + pr * (long long)(D * D);
+
+  if (warp == 0) {
+    tmem_alloc(&tmem_base_sh, kTmemCols);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(&mbar, 1);
+    fence_mbar_init();
+  }
+  // ---- stage the tokens (zeros beyond L) as fp32; clear A and Aqk
+  {
+    const int t = tid >> 4, c8 = tid & 15;      // token, 8-channel piece
+    float xq[8], xk[8], xv[8], xg[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) xq[e] = xk[e] = xv[e] = xg[e] = 0.f;
+    if (t < L) {
+      const long long row = (n * L + t) * H + h;
+      const uint4 uq = __ldg(reinterpret_cast<const uint4*>(q + row * D + c8 * 8));
+      const uint4 uk = __ldg(reinterpret_cast<const uint4*>(k + row * D + c8 * 8));
+      const uint4 uv = __ldg(reinterpret_cast<const uint4*>(v + row * D + c8 * 8));
+      const uint32_t wq4[4] = {uq.x, uq.y, uq.z, uq.w}, wk4[4] = {uk.x, uk.y, uk.z, uk.w},
+                     wv4[4] = {uv.x, uv.y, uv.z, uv.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        xq[2 * e] = __uint_as_float(wq4[e] << 16); xq[2 * e + 1] = __uint_as_float(wq4[e] & 0xffff0000u);
+        xk[2 * e] = __uint_as_float(wk4[e] << 16); xk[2 * e + 1] = __uint_as_float(wk4[e] & 0xffff0000u);
+        xv[2 * e] = __uint_as_float(wv4[e] << 16); xv[2 * e + 1] = __uint_as_float(wv4[e] & 0xffff0000u);
+      }
+      const float4 g0 = __ldg(reinterpret_cast<const float4*>(g + row * D + c8 * 8));
+      const float4 g1 = __ldg(reinterpret_cast<const float4*>(g + row * D + c8 * 8 + 4));
+      xg[0] = g0.x; xg[1] = g0.y; xg[2] = g0.z; xg[3] = g0.w;
+      xg[4] = g1.x; xg[5] = g1.y; xg[6] = g1.z; xg[7] = g1.w;
+    }
+    float* dq = fq + t * LDF + c8 * 8;
+    float* dk = fk + t * LDF + c8 * 8;
+    float* dv = fv + t * LDF + c8 * 8;
+    float* dg = fG + t * LDF + c8 * 8;
+    *reinterpret_cast<float4*>(dq) = make_float4(xq[0], xq[1], xq[2], xq[3]);
+    *reinterpret_cast<float4*>(dq + 4) = make_float4(xq[4], xq[5], xq[6], xq[7]);
+    *reinterpret_cast<float4*>(dk) = make_float4(xk[0], xk[1], xk[2], xk[3]);
+    *reinterpret_cast<float4*>(dk + 4) = make_float4(xk[4], xk[5], xk[6], xk[7]);
+    *reinterpret_cast<float4*>(dv) = make_float4(xv[0], xv[1], xv[2], xv[3]);
+    *reinterpret_cast<float4*>(dv + 4) = make_float4(xv[4], xv[5], xv[6], xv[7]);
+    *reinterpret_cast<float4*>(dg) = make_float4(xg[0], xg[1], xg[2], xg[3]);
+    *reinterpret_cast<float4*>(dg + 4) = make_float4(xg[4], xg[5], xg[6], xg[7]);
+    if (tid < LT) sBeta[tid] = tid < L ? beta[(n * L + tid) * H + h] : 0.f;
+    sA[tid] = 0.f;
+    sAqk[tid] = 0.f;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = tmem_base_sh;
+  const int wq = warp >> 2;                       // column half of the TMEM tiles
+  const int j = 32 * (warp & 3) + lane;           // TMEM lane = dv index
+  const uint32_t tl = tb + ((uint32_t)((warp & 3) * 32) << 16);
+
+  // ---- S (fp32 [dk][dv] in HBM) -> S^T in TMEM, and its bf16 copy: channels
+  //      [64 wq, 64 wq + 64) of lane j (coalesced: lanes read consecutive j)
+#pragma unroll 1
+  for (int q4 = 0; q4 < 4; ++q4) {
+    uint32_t f[16], pk[8];
+    const int c0 = 64 * wq + 16 * q4;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) f[e] = __float_as_uint(Sp[(long long)(c0 + e) * D + j]);
+    tmem_st16(tl + T_S + c0, f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      pk[e] = pack_bf16(__uint_as_float(f[2 * e]), __uint_as_float(f[2 * e + 1]));
+    tmem_st8(tl + T_SB + c0 / 2, pk);
+  }
+  tmem_wait_st();
+
+  // ---- Gamma = cumsum g over the 16 tokens, per channel; exp(Gamma_last)
+  if (tid < D) {
+    float acc = 0.f;
+#pragma unroll
+    for (int t = 0; t < LT; ++t) {
+      acc += fG[t * LDF + tid];
+      fG[t * LDF + tid] = acc;
+    }
+    sGl[tid] = __expf(acc);
+  }
+  __syncthreads();
+
+  // ---- Gram factors: e^(G - G_8) and e^(G_8 - G), each clamped at e^80, so that
+  //      e^(G_r - G_i) = e^(G_r - G_8) e^(G_8 - G_i) never overflows
+  {
+    const int t = tid >> 4, c8 = tid & 15;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int c = c8 * 8 + e;
+      const float dG = fG[t * LDF + c] - fG[8 * LDF + c];
+      const float up = __expf(fminf(dG, 80.f)), dn = __expf(fminf(-dG, 80.f));
+      fKP[t * LDF + c] = fk[t * LDF + c] * up;
+      fKM[t * LDF + c] = fk[t * LDF + c] * dn;
+      fQP[t * LDF + c] = fq[t * LDF + c] * up;
+    }
+  }
+  __syncthreads();
+
+  // ---- Gram pairs: thread tid < 136 -> Aqk(r, i <= r), else A(r, i < r) with
+  //      x = tid - 136; row r starts at r(r+1)/2 resp. r(r-1)/2
+  {
+    const bool isq = tid < 136;
+    const int x = isq ? tid : tid - 136;
+    int r = isq ? 0 : 1;
+#pragma unroll 1
+    while (r + 1 < LT && (isq ? (r + 1) * (r + 2) / 2 : (r + 1) * r / 2) <= x) ++r;
+    const int i = isq ? x - r * (r + 1) / 2 : x - r * (r - 1) / 2;
+    const float* xr = (isq ? fQP : fKP) + r * LDF;
+    const float* ki = fKM + i * LDF;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+    for (int c = 0; c < D; c += 4) {
+      const float4 u = *reinterpret_cast<const float4*>(xr + c);
+      const float4 w = *reinterpret_cast<const float4*>(ki + c);
+      a.x = fmaf(u.x, w.x, a.x); a.y = fmaf(u.y, w.y, a.y);
+      a.z = fmaf(u.z, w.z, a.z); a.w = fmaf(u.w, w.w, a.w);
+    }
+    (isq ? sAqk : sA)[r * LT + i] = (a.x + a.y) + (a.z + a.w);
+  }
+  __syncthreads();
+
+  // ---- T = (I + diag(beta) A)^-1 by forward substitution (column jj per thread),
+  //      stored as T diag(beta)
+  if (tid < LT) {
+    const int jj = tid;
+    float x[LT];
+#pragma unroll
+    for (int r = 0; r < LT; ++r) x[r] = (r == jj) ? 1.f : 0.f;
+#pragma unroll
+    for (int r = 1; r < LT; ++r) {
+      float acc = 0.f;
+#pragma unroll
+      for (int m = 0; m < r; ++m) acc = fmaf(sA[r * LT + m], x[m], acc);
+      if (r > jj) x[r] = -sBeta[r] * acc;
+    }
+    const float bj = sBeta[jj];
+#pragma unroll
+    for (int r = 0; r < LT; ++r) sT[r * LT + jj] = x[r] * bj;
+  }
+  __syncthreads();
+  // ---- Kbar = k e^G (into the first factor tile, free now)
+  {
+    const int t = tid >> 4, c8 = tid & 15;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int c = c8 * 8 + e;
+      fKP[t * LDF + c] = fk[t * LDF + c] * __expf(fG[t * LDF + c]);
+    }
+  }
+  __syncthreads();
+  // ---- W = (T beta) Kbar and U = (T beta) V: row r, channels [8 c8, 8 c8 + 8)
+  {
+    const int r = tid >> 4, c8 = tid & 15;
+    float w[8], u[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) { w[e] = 0.f; u[e] = 0.f; }
+#pragma unroll 1
+    for (int i = 0; i <= r; ++i) {
+      const float tb_ri = sT[r * LT + i];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        w[e] = fmaf(tb_ri, fKP[i * LDF + c8 * 8 + e], w[e]);
+        u[e] = fmaf(tb_ri, fv[i * LDF + c8 * 8 + e], u[e]);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      fQP[r * LDF + c8 * 8 + e] = w[e];             // W
+      fU[r * LDF + c8 * 8 + e] = u[e];
+    }
+  }
+  __syncthreads();
+
+  // ---- operand images
+  // [Qbar ; W]: bf16, MN-major SW32, N = 32 (tokens of Qbar, then of W), K = 128 channels
+#pragma unroll
+  for (int it = 0; it < 2; ++it) {
+    const int id = tid + it * NT;
+    const int c8 = id >> 7, kc = id & 127;
+    float x[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int t = 8 * (c8 & 1) + e;
+      x[e] = c8 < 2 ? fq[t * LDF + kc] * __expf(fG[t * LDF + kc]) : fQP[t * LDF + kc];
+    }
+    *reinterpret_cast<uint4*>(sm + M_B1 + chunk_mnmajor_sw32(c8, kc, D)) = pack8_bf16(x);
+  }
+  // Kend: f16, MN-major SW128, N = 128 channels, K = 16 tokens
+  {
+    const int t = tid >> 4, c8 = tid & 15;
+    float x[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int c = c8 * 8 + e;
+      x[e] = fk[t * LDF + c] * __expf(fG[(LT - 1) * LDF + c] - fG[t * LDF + c]);
+    }
+    *reinterpret_cast<uint4*>(sm + M_KE + chunk_mnmajor_sw128(c8, t, LT)) = pack8_f16v(x);
+  }
+  // Aqk^T: f16, MN-major SW32, N = 16 (r), K = 16 (i)
+  if (tid < 32) {
+    const int c8 = tid >> 4, i = tid & 15;
+    float x[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) x[e] = sAqk[(8 * c8 + e) * LT + i];
+    *reinterpret_cast<uint4*>(sm + M_AQ + chunk_mnmajor_sw32(c8, i, LT)) = pack8_f16v(x);
+  }
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  bool alive = true;
+  do {
+    // ---- [O^T | P] = S^T [Qbar ; W]^T
+    if (tid == 0) {
+      const uint32_t id1 = idesc_bf16(128, 2 * LT, false, true);
+      const uint32_t b1 = smem_u32(sm + M_B1);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk)
+        mma_ts(tb + T_OP, tb + T_SB + kk * 8, desc_mnmajor_sw32(b1, D, kk), id1, kk > 0);
+      mma_commit(&mbar);
+    }
+    __syncwarp();
+    // meanwhile S^T <- S^T Diag(exp(Gamma_last))
+#pragma unroll 1
+    for (int q4 = 0; q4 < 4; ++q4) {
+      uint32_t f[16];
+      const int c0 = 64 * wq + 16 * q4;
+      tmem_ld16(tl + T_S + c0, f);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 16; ++e) f[e] = __float_as_uint(__uint_as_float(f[e]) * sGl[c0 + e]);
+      tmem_st16(tl + T_S + c0, f);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    bool good = mbar_wait(&mbar, 0, kWaitLimit);
+    tc_fence_after();
+    if (__syncthreads_or(!good)) { alive = false; break; }
+
+    // ---- Delta^T = U^T - P (lane j, 16 tokens) -> f16 pairs in TMEM
+    if (wq == 0) {
+      uint32_t pp[16];
+      tmem_ld16(tl + T_OP + LT, pp);
+      tmem_wait_ld();
+      uint32_t dw[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        dw[e] = pack_f16(fU[(2 * e) * LDF + j] - __uint_as_float(pp[2 * e]),
+                         fU[(2 * e + 1) * LDF + j] - __uint_as_float(pp[2 * e + 1]));
+      tmem_st8(tl + T_D, dw);
+      tmem_wait_st();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    // ---- S^T += Delta^T Kend;  O^T += Delta^T Aqk^T   (f16 A and B)
+    if (tid == 0) {
+      mma_ts(tb + T_S, tb + T_D, desc_mnmajor_sw128(smem_u32(sm + M_KE), LT, 0),
+             idesc_f16(128, D, false, true), 1);
+      mma_ts(tb + T_OP, tb + T_D, desc_mnmajor_sw32(smem_u32(sm + M_AQ), LT, 0),
+             idesc_f16(128, LT, false, true), 1);
+      mma_commit(&mbar);
+    }
+    __syncwarp();
+    good = mbar_wait(&mbar, 1, kWaitLimit);
+    tc_fence_after();
+    if (__syncthreads_or(!good)) { alive = false; break; }
+
+    // ---- outputs (tokens < L) and the new state
+    if (wq == 0) {
+      uint32_t o[16];
+      tmem_ld16(tl + T_OP, o);
+      tmem_wait_ld();
+#pragma unroll
+      for (int t = 0; t < LT; ++t)
+        if (t < L) out[((n * L + t) * H + h) * D + j] = __float2bfloat16_rn(__uint_as_float(o[t]));
+    }
+#pragma unroll 1
+    for (int q4 = 0; q4 < 4; ++q4) {
+      uint32_t f[16];
+      const int c0 = 64 * wq + 16 * q4;
+      tmem_ld16(tl + T_S + c0, f);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 16; ++e) Sp[(long long)(c0 + e) * D + j] = __uint_as_float(f[e]);
+    }
+  } while (false);
+  if (!alive && tid == 0) {
+    atomicExch(&g_decode_chunk_timeout, 1);
+    mbar_wait(&mbar, 1, kWaitLimit);          // let an MMA still in flight finish
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tb, kTmemCols);
+  }
+}
+
+}  // namespace
+
+bool decode_chunk_supported(int dk, int dv, int in_dtype, int L) {
+  return in_dtype == KDA_BF16 && dk == D && dv == D && L >= 1 && L <= LT;
+}
+
+cudaError_t launch_decode_chunk(const void* q, const void* k, const void* v, const float* g,
+                                const float* beta, float* S, void* out, int N, int L, int H,
+                                cudaStream_t stream) {
+  static bool attr_done[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_done[dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(
+        kda_decode_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DC_SMEM);
+    if (e != cudaSuccess) return e;
+    attr_done[dev] = true;
+  }
+  const long long pairs = (long long)N * H;
+  KDA_TIMED(KDA_KERNEL_DECODE, stream,
+            kda_decode_chunk_kernel<<<(unsigned)pairs, NT, DC_SMEM, stream>>>(
+                static_cast<const bf16*>(q), static_cast<const bf16*>(k),
+                static_cast<const bf16*>(v), g, beta, S, static_cast<bf16*>(out), L, H));
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+// Reads (and with reset clears) g_decode_chunk_timeout; host side of kda_device_status.
+cudaError_t take_decode_chunk_timeout(int* flag, bool reset) {
+  int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_decode_chunk_timeout, sizeof(int));
+  if (e == cudaSuccess && reset && v != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_decode_chunk_timeout, &zero, sizeof(int));
+  }
+  *flag = v;
+  return e;
+}
+
+}  // namespace kda

@@ -87,6 +87,14 @@ cudaError_t take_tc_timeout(int* flag, bool reset);
 cudaError_t take_bwd_timeout(int* flag, bool reset);
 cudaError_t take_combine_timeout(int* flag, bool reset);
 cudaError_t take_selftest_timeout(int* flag, bool reset);
+cudaError_t take_decode_chunk_timeout(int* flag, bool reset);
+
+// Multi-token decode in the chunked form on the tensor cores (bf16, dk = dv = 128,
+// 1 <= L <= 16 tokens per (sequence, head)).
+bool decode_chunk_supported(int dk, int dv, int in_dtype, int L);
+cudaError_t launch_decode_chunk(const void* q, const void* k, const void* v, const float* g,
+                                const float* beta, float* S, void* out, int N, int L, int H,
+                                cudaStream_t stream);
 // One thread waits, at most `polls` polls, on an mbarrier phase nothing completes.
 cudaError_t launch_selftest_wait(uint32_t polls, cudaStream_t stream);
 

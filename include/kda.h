@@ -147,6 +147,31 @@ KDA_API int kda_decode_tokens(const void* q, const void* k, const void* v,
                               void* stream);
 
 /*
+ * kda_decode_chunk -- L <= 16 new tokens per (sequence, head) as one chunk of the
+ * chunked form, on the tensor cores (speculative verification of drafted tokens,
+ * multi-token decode).
+ *
+ * Passage: as for kda_decode_tokens (miniKimiK3 model card, "Kimi Delta Attention"
+ * bullet: the recurrence for decoding and the chunked parallel form, which equal
+ * each other).  Same arguments, layouts and in-place state update as
+ * kda_decode_tokens:
+ *     q, k, g [N, L, H, dk]   v, out [N, L, H, dv]   beta [N, L, H]   S [N, H, dk, dv]
+ * The state is read from and written back to HBM once; the chunk-local quantities
+ * (16 x 16 Gram, its triangular inverse, W, U) are formed in fp32 on the CUDA
+ * cores and the three products with the state run on the tensor cores (S in bf16
+ * for the first, f16 operands for the state update), so the results equal L single
+ * steps up to that rounding -- not bit for bit, unlike kda_decode_tokens.
+ * Supported: KDA_BF16, dk = dv = 128, 1 <= L <= 16 (else KDA_ERR_UNSUPPORTED).
+ * out must not alias S or any input.  N, L, H >= 1.
+ *
+ * Returns KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED or KDA_ERR_CUDA.
+ */
+KDA_API int kda_decode_chunk(const void* q, const void* k, const void* v,
+                             const float* g, const float* beta, float* S, void* out,
+                             int N, int L, int H, int dk, int dv, int in_dtype,
+                             void* stream);
+
+/*
  * kda_chunk_fwd_noalloc -- kda_chunk_fwd for callers that cannot allocate.
  *
  * The pages have no counterpart: this is a deployment variant.  Some callers

@@ -142,3 +142,18 @@ def test_bwd_grouped_rejects_bad_group(L, G):
 @pytest.mark.parametrize("polls", [0, (1 << 20) + 1])
 def test_selftest_rejects_poll_counts(L, polls):
     assert L.kda_selftest_bounded_wait(polls, None) == kda.KDA_ERR_INVALID_ARG
+
+
+def _dchunk(L_, q=P, S=P, out=P, N=1, Lt=4, H=1, dk=128, dv=128, dt=0):
+    return L_.kda_decode_chunk(q, P, P, P, P, S, out, N, Lt, H, dk, dv, dt, None)
+
+
+@pytest.mark.parametrize("bad", [dict(q=None), dict(S=None), dict(out=P + 4), dict(N=0),
+                                 dict(Lt=0), dict(H=0), dict(dt=4)])
+def test_decode_chunk_rejects_invalid(L, bad):
+    assert _dchunk(L, **bad) == kda.KDA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("dims", [dict(Lt=17), dict(dk=64), dict(dv=64), dict(dt=1)])
+def test_decode_chunk_rejects_unsupported(L, dims):
+    assert _dchunk(L, **dims) == kda.KDA_ERR_UNSUPPORTED
