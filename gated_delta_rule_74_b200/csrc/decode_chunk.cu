@@ -20,6 +20,8 @@
 //
 // TMEM (256 columns, two CTAs per SM): S^T fp32 [0, 128), [O^T | P] fp32
 // [128, 160), S^T as bf16 pairs [160, 224), Delta^T as f16 pairs [224, 232).
+#include <cuda_fp16.h>
+
 #include "kda_common.cuh"
 #include "sm100.cuh"
 
@@ -70,9 +72,10 @@ kda_decode_chunk_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
                         bf16* __restrict__ out, int L, int H) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
-  __shared__ uint64_t mbar;
+  __shared__ uint64_t mbar, sbar;
   __shared__ uint32_t tmem_base_sh;
   float* const F = reinterpret_cast<float*>(sm + M_F);
+  float* const Sf = F;                          // S [dk][dv] fp32 staged through the tile region
   float* const fq = F + F_Q * LT * LDF;          // q, later Qbar-ready raw q
   float* const fk = F + F_K * LT * LDF;          // k
   float* const fv = F + F_V * LT * LDF;          // v
@@ -99,12 +102,17 @@ kda_decode_chunk_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   }
   if (tid == 0) {
     mbar_init(&mbar, 1);
+    mbar_init(&sbar, 1);
     fence_mbar_init();
+    // S (64 KB contiguous) in one bulk copy into the tile region
+    mbar_arrive_expect_tx(&sbar, D * D * 4);
+    bulk_g2s(Sf, Sp, D * D * 4, &sbar);
   }
-  // ---- stage the tokens (zeros beyond L) as fp32; clear A and Aqk
+  // ---- the tokens (zeros beyond L) into registers meanwhile
+  const int st_t = tid >> 4, st_c8 = tid & 15;   // token, 8-channel piece
+  float xq[8], xk[8], xv[8], xg[8], xb = 0.f;
   {
-    const int t = tid >> 4, c8 = tid & 15;      // token, 8-channel piece
-    float xq[8], xk[8], xv[8], xg[8];
+    const int t = st_t, c8 = st_c8;
 #pragma unroll
     for (int e = 0; e < 8; ++e) xq[e] = xk[e] = xv[e] = xg[e] = 0.f;
     if (t < L) {
@@ -125,6 +133,37 @@ kda_decode_chunk_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       xg[0] = g0.x; xg[1] = g0.y; xg[2] = g0.z; xg[3] = g0.w;
       xg[4] = g1.x; xg[5] = g1.y; xg[6] = g1.z; xg[7] = g1.w;
     }
+    if (tid < LT && tid < L) xb = beta[(n * L + tid) * H + h];
+    sA[tid] = 0.f;
+    sAqk[tid] = 0.f;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = tmem_base_sh;
+  const int wq = warp >> 2;                       // column half of the TMEM tiles
+  const int j = 32 * (warp & 3) + lane;           // TMEM lane = dv index
+  const uint32_t tl = tb + ((uint32_t)((warp & 3) * 32) << 16);
+
+  // ---- S -> S^T in TMEM and its bf16 copy: channels [64 wq, 64 wq + 64) of lane j,
+  //      read from the staged copy (lanes read consecutive words: no bank conflict)
+  bool s_ok = mbar_wait(&sbar, 0, kWaitLimit);
+#pragma unroll 1
+  for (int q4 = 0; q4 < 4; ++q4) {
+    uint32_t f[16], pk[8];
+    const int c0 = 64 * wq + 16 * q4;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) f[e] = __float_as_uint(Sf[(c0 + e) * D + j]);
+    tmem_st16(tl + T_S + c0, f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      pk[e] = pack_bf16(__uint_as_float(f[2 * e]), __uint_as_float(f[2 * e + 1]));
+    tmem_st8(tl + T_SB + c0 / 2, pk);
+  }
+  tmem_wait_st();
+  __syncthreads();                                // the staged S is consumed
+  {
+    const int t = st_t, c8 = st_c8;
     float* dq = fq + t * LDF + c8 * 8;
     float* dk = fk + t * LDF + c8 * 8;
     float* dv = fv + t * LDF + c8 * 8;
@@ -137,58 +176,37 @@ kda_decode_chunk_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     *reinterpret_cast<float4*>(dv + 4) = make_float4(xv[4], xv[5], xv[6], xv[7]);
     *reinterpret_cast<float4*>(dg) = make_float4(xg[0], xg[1], xg[2], xg[3]);
     *reinterpret_cast<float4*>(dg + 4) = make_float4(xg[4], xg[5], xg[6], xg[7]);
-    if (tid < LT) sBeta[tid] = tid < L ? beta[(n * L + tid) * H + h] : 0.f;
-    sA[tid] = 0.f;
-    sAqk[tid] = 0.f;
+    if (tid < LT) sBeta[tid] = xb;
   }
-  tc_fence_before();
   __syncthreads();
-  tc_fence_after();
-  const uint32_t tb = tmem_base_sh;
-  const int wq = warp >> 2;                       // column half of the TMEM tiles
-  const int j = 32 * (warp & 3) + lane;           // TMEM lane = dv index
-  const uint32_t tl = tb + ((uint32_t)((warp & 3) * 32) << 16);
 
-  // ---- S (fp32 [dk][dv] in HBM) -> S^T in TMEM, and its bf16 copy: channels
-  //      [64 wq, 64 wq + 64) of lane j (coalesced: lanes read consecutive j)
-#pragma unroll 1
-  for (int q4 = 0; q4 < 4; ++q4) {
-    uint32_t f[16], pk[8];
-    const int c0 = 64 * wq + 16 * q4;
-#pragma unroll
-    for (int e = 0; e < 16; ++e) f[e] = __float_as_uint(Sp[(long long)(c0 + e) * D + j]);
-    tmem_st16(tl + T_S + c0, f);
-#pragma unroll
-    for (int e = 0; e < 8; ++e)
-      pk[e] = pack_bf16(__uint_as_float(f[2 * e]), __uint_as_float(f[2 * e + 1]));
-    tmem_st8(tl + T_SB + c0 / 2, pk);
-  }
-  tmem_wait_st();
-
-  // ---- Gamma = cumsum g over the 16 tokens, per channel; exp(Gamma_last)
+  // ---- per channel c (thread c < 128): Gamma = cumsum g; exp(Gamma_last); the Gram
+  //      factors k e^(G - G_8), k e^(G_8 - G), q e^(G - G_8) (each e^ clamped at 80);
+  //      Kbar = k e^G (into the Gamma tile); the Qbar and Kend operand images
   if (tid < D) {
+    const int c = tid;
+    float G[LT];
     float acc = 0.f;
 #pragma unroll
     for (int t = 0; t < LT; ++t) {
-      acc += fG[t * LDF + tid];
-      fG[t * LDF + tid] = acc;
+      acc += fG[t * LDF + c];
+      G[t] = acc;
     }
-    sGl[tid] = __expf(acc);
-  }
-  __syncthreads();
-
-  // ---- Gram factors: e^(G - G_8) and e^(G_8 - G), each clamped at e^80, so that
-  //      e^(G_r - G_i) = e^(G_r - G_8) e^(G_8 - G_i) never overflows
-  {
-    const int t = tid >> 4, c8 = tid & 15;
+    const float gl = acc;
+    sGl[c] = __expf(gl);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int c = c8 * 8 + e;
-      const float dG = fG[t * LDF + c] - fG[8 * LDF + c];
+    for (int t = 0; t < LT; ++t) {
+      const float kt = fk[t * LDF + c], qt = fq[t * LDF + c];
+      const float dG = G[t] - G[8];
       const float up = __expf(fminf(dG, 80.f)), dn = __expf(fminf(-dG, 80.f));
-      fKP[t * LDF + c] = fk[t * LDF + c] * up;
-      fKM[t * LDF + c] = fk[t * LDF + c] * dn;
-      fQP[t * LDF + c] = fq[t * LDF + c] * up;
+      const float eg = __expf(G[t]);
+      fKP[t * LDF + c] = kt * up;
+      fKM[t * LDF + c] = kt * dn;
+      fQP[t * LDF + c] = qt * up;
+      fG[t * LDF + c] = kt * eg;                  // Kbar
+      *reinterpret_cast<bf16*>(sm + M_B1 + off_mnmajor_sw32(t, c, D)) = __float2bfloat16_rn(qt * eg);
+      *reinterpret_cast<__half*>(sm + M_KE + off_mnmajor_sw128(c, t, LT)) =
+          __float2half_rn(kt * __expf(gl - G[t]));
     }
   }
   __syncthreads();
@@ -216,84 +234,10 @@ kda_decode_chunk_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   }
   __syncthreads();
 
-  // ---- T = (I + diag(beta) A)^-1 by forward substitution (column jj per thread),
-  //      stored as T diag(beta)
-  if (tid < LT) {
-    const int jj = tid;
-    float x[LT];
-#pragma unroll
-    for (int r = 0; r < LT; ++r) x[r] = (r == jj) ? 1.f : 0.f;
-#pragma unroll
-    for (int r = 1; r < LT; ++r) {
-      float acc = 0.f;
-#pragma unroll
-      for (int m = 0; m < r; ++m) acc = fmaf(sA[r * LT + m], x[m], acc);
-      if (r > jj) x[r] = -sBeta[r] * acc;
-    }
-    const float bj = sBeta[jj];
-#pragma unroll
-    for (int r = 0; r < LT; ++r) sT[r * LT + jj] = x[r] * bj;
-  }
-  __syncthreads();
-  // ---- Kbar = k e^G (into the first factor tile, free now)
-  {
-    const int t = tid >> 4, c8 = tid & 15;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int c = c8 * 8 + e;
-      fKP[t * LDF + c] = fk[t * LDF + c] * __expf(fG[t * LDF + c]);
-    }
-  }
-  __syncthreads();
-  // ---- W = (T beta) Kbar and U = (T beta) V: row r, channels [8 c8, 8 c8 + 8)
-  {
-    const int r = tid >> 4, c8 = tid & 15;
-    float w[8], u[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) { w[e] = 0.f; u[e] = 0.f; }
-#pragma unroll 1
-    for (int i = 0; i <= r; ++i) {
-      const float tb_ri = sT[r * LT + i];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        w[e] = fmaf(tb_ri, fKP[i * LDF + c8 * 8 + e], w[e]);
-        u[e] = fmaf(tb_ri, fv[i * LDF + c8 * 8 + e], u[e]);
-      }
-    }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      fQP[r * LDF + c8 * 8 + e] = w[e];             // W
-      fU[r * LDF + c8 * 8 + e] = u[e];
-    }
-  }
-  __syncthreads();
-
-  // ---- operand images
-  // [Qbar ; W]: bf16, MN-major SW32, N = 32 (tokens of Qbar, then of W), K = 128 channels
-#pragma unroll
-  for (int it = 0; it < 2; ++it) {
-    const int id = tid + it * NT;
-    const int c8 = id >> 7, kc = id & 127;
-    float x[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int t = 8 * (c8 & 1) + e;
-      x[e] = c8 < 2 ? fq[t * LDF + kc] * __expf(fG[t * LDF + kc]) : fQP[t * LDF + kc];
-    }
-    *reinterpret_cast<uint4*>(sm + M_B1 + chunk_mnmajor_sw32(c8, kc, D)) = pack8_bf16(x);
-  }
-  // Kend: f16, MN-major SW128, N = 128 channels, K = 16 tokens
-  {
-    const int t = tid >> 4, c8 = tid & 15;
-    float x[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int c = c8 * 8 + e;
-      x[e] = fk[t * LDF + c] * __expf(fG[(LT - 1) * LDF + c] - fG[t * LDF + c]);
-    }
-    *reinterpret_cast<uint4*>(sm + M_KE + chunk_mnmajor_sw128(c8, t, LT)) = pack8_f16v(x);
-  }
-  // Aqk^T: f16, MN-major SW32, N = 16 (r), K = 16 (i)
+  // ---- U = (I + diag(beta) A)^-1 diag(beta) V and W likewise with Kbar, by forward
+  //      substitution, one column per thread: U_r = beta_r (V_r - sum_{i<r} A_ri U_i).
+  //      Threads 0..127: U (kept in fp32 for Delta); 128..255: W (the bf16 operand
+  //      image).  Threads 0..31 first write the Aqk^T operand image.
   if (tid < 32) {
     const int c8 = tid >> 4, i = tid & 15;
     float x[8];
@@ -301,13 +245,35 @@ kda_decode_chunk_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     for (int e = 0; e < 8; ++e) x[e] = sAqk[(8 * c8 + e) * LT + i];
     *reinterpret_cast<uint4*>(sm + M_AQ + chunk_mnmajor_sw32(c8, i, LT)) = pack8_f16v(x);
   }
+  {
+    const bool isw = tid >= D;
+    const int c = tid & (D - 1);
+    const float* src = isw ? fG : fv;             // Kbar or V
+    float y[LT];
+#pragma unroll
+    for (int r = 0; r < LT; ++r) {
+      float acc = src[r * LDF + c];
+#pragma unroll
+      for (int i = 0; i < r; ++i) acc = fmaf(-sA[r * LT + i], y[i], acc);
+      y[r] = sBeta[r] * acc;
+    }
+    if (isw) {
+#pragma unroll
+      for (int r = 0; r < LT; ++r)
+        *reinterpret_cast<bf16*>(sm + M_B1 + off_mnmajor_sw32(LT + r, c, D)) = __float2bfloat16_rn(y[r]);
+    } else {
+#pragma unroll
+      for (int r = 0; r < LT; ++r) fU[r * LDF + c] = y[r];
+    }
+  }
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
 
-  bool alive = true;
+  bool alive = __syncthreads_or(!s_ok) == 0;
   do {
+    if (!alive) break;
     // ---- [O^T | P] = S^T [Qbar ; W]^T
     if (tid == 0) {
       const uint32_t id1 = idesc_bf16(128, 2 * LT, false, true);
@@ -374,6 +340,7 @@ kda_decode_chunk_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       for (int t = 0; t < LT; ++t)
         if (t < L) out[((n * L + t) * H + h) * D + j] = __float2bfloat16_rn(__uint_as_float(o[t]));
     }
+    // the new state: TMEM -> the tile region (free again) -> one bulk copy to HBM
 #pragma unroll 1
     for (int q4 = 0; q4 < 4; ++q4) {
       uint32_t f[16];
@@ -381,12 +348,19 @@ kda_decode_chunk_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       tmem_ld16(tl + T_S + c0, f);
       tmem_wait_ld();
 #pragma unroll
-      for (int e = 0; e < 16; ++e) Sp[(long long)(c0 + e) * D + j] = __uint_as_float(f[e]);
+      for (int e = 0; e < 16; ++e) Sf[(c0 + e) * D + j] = __uint_as_float(f[e]);
+    }
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      bulk_s2g(Sp, Sf, D * D * 4);
+      bulk_commit();
+      bulk_wait_read<0>();
     }
   } while (false);
   if (!alive && tid == 0) {
     atomicExch(&g_decode_chunk_timeout, 1);
-    mbar_wait(&mbar, 1, kWaitLimit);          // let an MMA still in flight finish
+    if (s_ok) mbar_wait(&mbar, 1, kWaitLimit);   // let an MMA still in flight finish
   }
   tc_fence_before();
   __syncthreads();
