@@ -622,30 +622,35 @@ def decode_leg(args, world, rank, dev, stream, barrier, clocks, hbm, peak_kind):
         tq = {n: dt[n].transpose(0, 1).contiguous().to(dev) for n in ("q", "k", "v", "g", "beta")}
         del dt
         tout = torch.empty(dd["N"], L, dd["H"], dd["dv"], dtype=q.dtype, device=dev)
-        for _ in range(3):
-            kda.kda_decode_tokens(tq["q"], tq["k"], tq["v"], tq["g"], tq["beta"], S, out=tout,
-                                  stream=stream)
-        torch.cuda.synchronize()
-        barrier()
-        nf = max(3, args.decode_steps // 8)
-        n1 = kda.kda_launch_count()
-        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        f0.record(stream)
-        for _ in range(nf):
-            kda.kda_decode_tokens(tq["q"], tq["k"], tq["v"], tq["g"], tq["beta"], S, out=tout,
-                                  stream=stream)
-        f1.record(stream)
-        torch.cuda.synchronize()
-        barrier()
-        fl = kda.kda_launch_count() - n1
-        fms = _max_over_ranks(f0.elapsed_time(f1), world, dev) / nf
         fbytes = dd["N"] * dd["H"] * (8 * dd["dk"] * dd["dv"] + L * ((2 * dd["dk"] + dd["dv"]) * 2
                                                                    + 4 * dd["dk"] + 4 + dd["dv"] * 2))
-        fgbs = fbytes / (fms / 1e3) / 1e9
-        fused = {"call": "kda_decode_tokens", "tokens_per_launch_per_sequence": L,
-                 "ms_per_launch": fms, "tokens_per_s": dd["N"] * L * world * 1e3 / fms,
-                 "bytes_per_launch": fbytes, "gbs": fgbs, "frac_of_hbm_peak": fgbs / hbm,
-                 "speedup_vs_single_steps": (step_ms * L) / fms, "launches": fl}
+
+        def time_tokens(fn, name):
+            for _ in range(3):
+                fn(tq["q"], tq["k"], tq["v"], tq["g"], tq["beta"], S, out=tout, stream=stream)
+            torch.cuda.synchronize()
+            barrier()
+            nf = max(3, args.decode_steps // 8)
+            n1 = kda.kda_launch_count()
+            f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            f0.record(stream)
+            for _ in range(nf):
+                fn(tq["q"], tq["k"], tq["v"], tq["g"], tq["beta"], S, out=tout, stream=stream)
+            f1.record(stream)
+            torch.cuda.synchronize()
+            barrier()
+            fl = kda.kda_launch_count() - n1
+            fms = _max_over_ranks(f0.elapsed_time(f1), world, dev) / nf
+            fgbs = fbytes / (fms / 1e3) / 1e9
+            return {"call": name, "tokens_per_launch_per_sequence": L,
+                    "ms_per_launch": fms, "tokens_per_s": dd["N"] * L * world * 1e3 / fms,
+                    "bytes_per_launch": fbytes, "gbs": fgbs, "frac_of_hbm_peak": fgbs / hbm,
+                    "speedup_vs_single_steps": (step_ms * L) / fms, "launches": fl}
+
+        fused = time_tokens(kda.kda_decode_tokens, "kda_decode_tokens")
+        if L <= 16 and dd["dk"] == 128 and dd["dv"] == 128 and q.dtype == torch.bfloat16:
+            fused["chunk_form"] = time_tokens(
+                kda.kda_decode_chunk, "kda_decode_chunk (one chunk on the tensor cores)")
         del tq, tout
     return {"metric": "decode state GB/s vs HBM peak", "fused_tokens": fused, "workload":
             f"cfg4 shape: N={dd['N']} H={dd['H']} dk=dv=128 bf16 q/k/v, fp32 state "
