@@ -102,7 +102,7 @@ constexpr uint32_t TM_S = 0;        // S^T fp32        [128 lanes x 128]
 constexpr uint32_t TM_O = 128;      // O^T             [128 x 64]
 constexpr uint32_t TM_P = 192;      // P               [128 x 64]
 constexpr uint32_t TM_SB = 256;     // S^T bf16 (A)    [128 x 64]
-constexpr uint32_t TM_KB = 320;     // Kbar^T bf16 (A) [128 x 32], later Delta^T bf16 (A)
+constexpr uint32_t TM_KB = 320;     // Kbar^T bf16 (A) [128 x 32], later Delta^T f16 (A)
 constexpr uint32_t TM_G = 352;      // Gram D^(0..3) at +0, +16, +48, +96 (160 columns)
 constexpr uint32_t TM_W = 352;      // W^T [128 x 64]  (after the Gram is read)
 constexpr uint32_t TM_U = 416;      // U^T [128 x 64]
@@ -116,6 +116,12 @@ __device__ __forceinline__ void st_v4(uint8_t* base, uint32_t off, uint32_t a, u
 __device__ __forceinline__ void st_v4f(uint8_t* base, uint32_t off, const float (&x)[8], float s) {
   st_v4(base, off, pack_bf16(x[0] * s, x[1] * s), pack_bf16(x[2] * s, x[3] * s),
         pack_bf16(x[4] * s, x[5] * s), pack_bf16(x[6] * s, x[7] * s));
+}
+// the same as f16: [Kend^T ; Aqk] and Delta^T are f16 (the state update runs in
+// kind::f16 with f16 A and B, for the finer rounding)
+__device__ __forceinline__ void st_v4h(uint8_t* base, uint32_t off, const float (&x)[8], float s) {
+  st_v4(base, off, pack_f16(x[0] * s, x[1] * s), pack_f16(x[2] * s, x[3] * s),
+        pack_f16(x[4] * s, x[5] * s), pack_f16(x[6] * s, x[7] * s));
 }
 
 // Issue the cp.async loads of one chunk's q, k, g into the staging region
@@ -191,7 +197,7 @@ __device__ __forceinline__ void build_half(uint8_t* sm, const float (&gv)[32], c
       // Qbar^T: B operand of O^T, MN-major SW128 (N = tokens, K = channels)
       st_v4f(sm, OFF_QB + chunk_mnmajor_sw128(g8, c, D), lq, eP);
       // Kend^T: B operand of the state update, K-major SW128 (N = channels, K = tokens)
-      st_v4f(sm, OFF_KE + chunk_kmajor_sw128(c, g8, D), kr, eE);
+      st_v4h(sm, OFF_KE + chunk_kmajor_sw128(c, g8, D), kr, eE);
       // R^(a'), a' >= a: B operands of the Gram, MN-major SW32 (N = 16(a'+1), K = channels)
       st_v4f(sm, off_r(a) + chunk_mnmajor_sw32(g8, c, D), kr, 1.f);
       if (a + 1 <= 3) st_v4f(sm, off_r(a + 1 <= 3 ? a + 1 : 3) + chunk_mnmajor_sw32(g8, c, D), kr, f1);
@@ -476,7 +482,7 @@ kda_chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
             float w[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) w[e] = (c8 * 8 + e <= r) ? vals[c8 * 8 + e] : 0.f;
-            st_v4f(sm, OFF_AQK + chunk_kmajor_sw128(r, c8, C), w, 1.f);
+            st_v4h(sm, OFF_AQK + chunk_kmajor_sw128(r, c8, C), w, 1.f);
           }
         }
       }
@@ -661,7 +667,7 @@ kda_chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     __syncwarp();
     if (!mma_wait()) { alive = false; break; }
 
-    // ================= P7: Delta^T = U^T - P -> bf16 TMEM (upper threads) =====
+    // ================= P7: Delta^T = U^T - P -> f16 TMEM (upper threads) ======
     if (upper) {
       uint32_t dw[32];
 #pragma unroll
@@ -682,8 +688,8 @@ kda_chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
 #pragma unroll
           for (int e = 0; e < 8; ++e)
             dw[(r0 + 16 * q2) / 2 + e] =
-                pack_bf16(__uint_as_float(tu[q2][2 * e]) - __uint_as_float(tp[q2][2 * e]),
-                          __uint_as_float(tu[q2][2 * e + 1]) - __uint_as_float(tp[q2][2 * e + 1]));
+                pack_f16(__uint_as_float(tu[q2][2 * e]) - __uint_as_float(tp[q2][2 * e]),
+                         __uint_as_float(tu[q2][2 * e + 1]) - __uint_as_float(tp[q2][2 * e + 1]));
         }
       }
       uint32_t w0[16], w1[16];
@@ -702,7 +708,7 @@ kda_chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       // Kend^T (128 rows) and Aqk (64 rows) form one K-major B operand of 192 rows
       const uint32_t ke_base = smem_u32(sm + OFF_KE);
       const int n = outputs ? D + C : D;
-      const uint32_t id_s = idesc_bf16(128, n, false, false);
+      const uint32_t id_s = idesc_f16(128, n, false, false);    // f16 A (Delta^T) and B
 #pragma unroll
       for (int kk = 0; kk < C / 16; ++kk)
         mma_ts(tb + TM_S, tb + TM_KB + kk * 8, desc_kmajor_sw128(ke_base, n, kk), id_s, 1);
