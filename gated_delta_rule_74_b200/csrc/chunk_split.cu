@@ -44,6 +44,7 @@
 // 16-token block the cumulative log-decay must stay above -80 per channel.
 // All four products (A and Aqk rows for all blocks) are one MMA of N = 160:
 //   [D^(0) .. D^(3)] [128 x 160] = [Lk ; Lq] [R^(0); ..; R^(3)]^T
+#include <algorithm>
 #include <type_traits>
 
 #include "kda_common.cuh"
@@ -109,6 +110,7 @@ constexpr uint32_t ST_O = 128;          // O^T             [128 x 64]
 constexpr uint32_t ST_P = 192;          // P               [128 x 64]
 constexpr uint32_t ST_SB = 256;         // S^T bf16 (A)    [128 x 64]
 constexpr uint32_t ST_D = 320;          // Delta^T f16 (A)  [128 x 32]
+constexpr uint32_t ST_LO = 384;         // from a half point: bf16 lo part of S_start^T [128 x 64]
 constexpr uint32_t kStateTmemCols = 512;
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -685,6 +687,43 @@ __device__ __forceinline__ uint4 apply_gate(uint4 o, uint4 z) {
   return make_uint4(ow[0], ow[1], ow[2], ow[3]);
 }
 
+// A state in TMEM (this thread: columns [32 wq, 32 wq + 32) of row j of S^T, from
+// taddr) -> dst.  A transition X (identity start) goes out as bf16 hi / lo images for
+// the segment combine (MN-major SW128 A operand, M = row of X, K = column; TMEM lane
+// j holds column j of X); any other state as fp32 [dk][dv] rows.  Called once or
+// twice per chain, out of line so the chunk loop keeps its registers.
+__device__ __noinline__ void store_state_cols(float* dst, uint32_t taddr, bool ximg, int wq, int j,
+                                              int dk, int dv) {
+  uint32_t t[2][16];
+  tmem_ld16(taddr, t[0]);
+  tmem_ld16(taddr + 16, t[1]);
+  tmem_wait_ld();
+  if (ximg) {
+    uint8_t* xb = reinterpret_cast<uint8_t*>(dst);
+#pragma unroll
+    for (int c8 = 0; c8 < 4; ++c8) {
+      uint32_t hw[4], lw[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float x0 = __uint_as_float(t[c8 >> 1][(c8 & 1) * 8 + 2 * e]);
+        const float x1 = __uint_as_float(t[c8 >> 1][(c8 & 1) * 8 + 2 * e + 1]);
+        hw[e] = pack_bf16(x0, x1);
+        lw[e] = pack_bf16(x0 - bf_lo(hw[e]), x1 - bf_hi(hw[e]));
+      }
+      const uint32_t o = chunk_mnmajor_sw128((uint32_t)(4 * wq + c8), (uint32_t)j, D);
+      *reinterpret_cast<uint4*>(xb + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      *reinterpret_cast<uint4*>(xb + 32768 + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    }
+  } else if (j < dv) {
+#pragma unroll
+    for (int e = 0; e < 32; ++e)
+      if (32 * wq + e < dk) dst[(long long)(32 * wq + e) * dv + j] = __uint_as_float(t[e >> 4][e & 15]);
+  }
+}
+
+// HALF: the split has half points (pass A keeps its half-way state, pass C's
+// second-half chains form S_mid first); otherwise that code is compiled out.
+template <bool HALF>
 __global__ void __launch_bounds__(NT_S, 1)
 kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
                       const int32_t* __restrict__ cu_seqlens, bf16* __restrict__ out, float* hT,
@@ -693,7 +732,7 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   __shared__ uint64_t full[2];
-  __shared__ uint64_t mbar;
+  __shared__ uint64_t mbar, xbar;
   __shared__ uint32_t tmem_base_sh;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -710,6 +749,10 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
   bool init_identity = false;
   float* fin = hT ? hT + hoff : nullptr;          // nullptr: final state not kept
   bool outputs = true, homog = false;
+  int mid = 0;                                    // pass A: after `mid` chunks the state
+  float* mid_dst = nullptr;                       // is also kept here
+  const float* mid_src = nullptr;                 // pass C from a half point: S_start,p and
+  const uint8_t* mid_x = nullptr;                 // the X_half,p images (init = Sloc_half,p)
   if (sa.pass != 0) {
     const int Ps = seg_count(t_end - t_beg, sa.G);
     const int z = blockIdx.z;
@@ -727,7 +770,10 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
         if (p > Ps - 2) return;
         const long long o = slot_off(p);
         if (o < 0) return;
-        if (p > 0) { init = nullptr; outputs = false; }
+        if (p > 0) {
+          init = nullptr; outputs = false;
+          if (HALF) { mid = sa.half; mid_dst = sa.sbuf_h + o; }
+        }
         fin = sa.sbuf + o;
         t_beg += p * seg_tok;
         t_end = min(t_end, t_beg + seg_tok);
@@ -737,18 +783,36 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
         if (o < 0) return;
         init = nullptr; init_identity = true; outputs = false; homog = true;
         fin = sa.xbuf + o;
+        if (HALF) { mid = sa.half; mid_dst = sa.xbuf_h + o; }
         t_beg += p * seg_tok;
         t_end = min(t_end, t_beg + seg_tok);
       }
     } else {
-      const int p = z + 1;
+      // z = p - 1 (one chain per segment), or 2 (p - 1) + q with half points: q = 0
+      // runs the segment's first Gh chunks, q = 1 the rest from S_mid,p
+      const int p = (HALF ? z / 2 : z) + 1, q = HALF ? z % 2 : 0;
       if (Ps <= 1 || p > Ps - 1) return;
-      const long long o = slot_off(p - 1);
+      const bool split = HALF && p <= Ps - 2;
+      if (q == 1 && !split) return;
+      const long long o = q == 0 ? slot_off(p - 1) : slot_off(p);
       if (o < 0) return;
-      init = sa.sbuf + o;
+      init = q == 0 ? sa.sbuf + o : sa.sbuf_h + o;
+      if (q == 1) {                               // S_mid,p = X_half,p S_start,p + Sloc_half,p
+        const long long o0 = slot_off(p - 1);
+        if (o0 < 0) return;
+        mid_src = sa.sbuf + o0;
+        mid_x = reinterpret_cast<const uint8_t*>(sa.xbuf_h + o);
+      }
       if (p != Ps - 1) fin = nullptr;
       t_beg += p * seg_tok;
-      t_end = min(t_end, t_beg + seg_tok);
+      const long long seg_end = min(t_end, t_beg + seg_tok);
+      if (split) {
+        const long long half_tok = (long long)sa.half * C;
+        if (q == 0) t_end = min(seg_end, t_beg + half_tok);
+        else { t_beg += half_tok; t_end = seg_end; }
+      } else {
+        t_end = seg_end;
+      }
     }
   }
   const int nch = (int)chunk_count(t_end - t_beg);
@@ -764,14 +828,23 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
     mbar_init(&full[0], 1);
     mbar_init(&full[1], 1);
     mbar_init(&mbar, 1);
+    mbar_init(&xbar, 1);
     fence_mbar_init();
   }
   __syncthreads();
-  int issued = nch < 2 ? nch : 2;                    // thread 0: records requested
+  // records requested (thread 0); from a half point, record buffer 1 first takes the
+  // X_half images and record 1 follows once they are consumed
+  int issued = nch < 2 ? nch : (HALF && mid_x ? 1 : 2);
+  int xstate = 0;                                    // thread 0: 1 images requested, 2 MMAs issued
   if (tid == 0) {
     for (int i = 0; i < issued; ++i) {
       mbar_arrive_expect_tx(&full[i], REC_BYTES);
       bulk_g2s(sm + i * S_BUF, rec_ptr(i), REC_BYTES, &full[i]);
+    }
+    if (HALF && mid_x) {
+      mbar_arrive_expect_tx(&xbar, 65536);
+      bulk_g2s(sm + S_BUF, mid_x, 65536, &xbar);
+      xstate = 1;
     }
   }
   tc_fence_before();
@@ -792,17 +865,84 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
       f0[e] = __float_as_uint(x0);
       f1[e] = __float_as_uint(x1);
     }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      pk[e] = pack_bf16(__uint_as_float(f0[2 * e]), __uint_as_float(f0[2 * e + 1]));
-      pk[8 + e] = pack_bf16(__uint_as_float(f1[2 * e]), __uint_as_float(f1[2 * e + 1]));
-    }
     tmem_st16(tl + ST_S + c, f0);
     tmem_st16(tl + ST_S + c + 16, f1);
+    if (HALF && mid_src) {              // bf16 hi / lo parts of S_start^T (A operands)
+      uint32_t lo[16];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int r0 = c + 2 * e, r1 = c + 16 + 2 * e;
+        const bool ok = j < dv;
+        const float a0 = ok && r0 < dk ? mid_src[(long long)r0 * dv + j] : 0.f;
+        const float a1 = ok && r0 + 1 < dk ? mid_src[(long long)(r0 + 1) * dv + j] : 0.f;
+        const float b0 = ok && r1 < dk ? mid_src[(long long)r1 * dv + j] : 0.f;
+        const float b1 = ok && r1 + 1 < dk ? mid_src[(long long)(r1 + 1) * dv + j] : 0.f;
+        pk[e] = pack_bf16(a0, a1);
+        pk[8 + e] = pack_bf16(b0, b1);
+        lo[e] = pack_bf16(a0 - bf_lo(pk[e]), a1 - bf_hi(pk[e]));
+        lo[8 + e] = pack_bf16(b0 - bf_lo(pk[8 + e]), b1 - bf_hi(pk[8 + e]));
+      }
+      tmem_st16(tl + ST_LO + c / 2, lo);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        pk[e] = pack_bf16(__uint_as_float(f0[2 * e]), __uint_as_float(f0[2 * e + 1]));
+        pk[8 + e] = pack_bf16(__uint_as_float(f1[2 * e]), __uint_as_float(f1[2 * e + 1]));
+      }
+    }
     tmem_st16(tl + ST_SB + c / 2, pk);
     tmem_wait_st();
   }
-  bool good = nch == 0 || mbar_wait(&full[0], 0, kWaitLimit);
+  bool good = true;
+  if (HALF && mid_x) {
+    // S_mid^T = Sloc_half^T + S_start^T X_half^T (three bf16 products: hi hi, hi lo,
+    // lo hi; fp32 accumulation onto Sloc_half^T in TMEM); X_half is the B operand
+    // (N = row of X, K = column, MN-major images)
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0) {
+      good = mbar_wait(&xbar, 0, kWaitLimit);
+      if (good) {
+        tc_fence_after();
+        const uint32_t xh = smem_u32(sm + S_BUF), xl = xh + 32768u;
+        const uint32_t id = idesc_bf16(128, 128, false, true);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t bh = desc_mnmajor_sw128(xh, D, kk), bl = desc_mnmajor_sw128(xl, D, kk);
+          mma_ts(tb + ST_S, tb + ST_SB + kk * 8, bh, id, 1);
+          mma_ts(tb + ST_S, tb + ST_SB + kk * 8, bl, id, 1);
+          mma_ts(tb + ST_S, tb + ST_LO + kk * 8, bh, id, 1);
+        }
+        mma_commit(&xbar);
+        xstate = 2;
+      }
+    }
+    __syncwarp();
+    good = __syncthreads_or(!good) == 0;
+    if (good) good = mbar_wait(&xbar, 1, kWaitLimit);
+    tc_fence_after();
+    good = __syncthreads_or(!good) == 0;
+    if (good) {                         // the bf16 copy of S_mid for the first product
+      uint32_t t[2][16], pk[16];
+      tmem_ld16(tl + ST_S + 32 * wq, t[0]);
+      tmem_ld16(tl + ST_S + 32 * wq + 16, t[1]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        pk[e] = pack_bf16(__uint_as_float(t[0][2 * e]), __uint_as_float(t[0][2 * e + 1]));
+        pk[8 + e] = pack_bf16(__uint_as_float(t[1][2 * e]), __uint_as_float(t[1][2 * e + 1]));
+      }
+      tmem_st16(tl + ST_SB + 16 * wq, pk);
+      tmem_wait_st();
+      if (tid == 0 && nch >= 2) {       // the images are consumed: record 1 into buffer 1
+        mbar_arrive_expect_tx(&full[1], REC_BYTES);
+        bulk_g2s(sm + S_BUF, rec_ptr(1), REC_BYTES, &full[1]);
+        issued = 2;
+      }
+    }
+  }
+  good = good && (nch == 0 || mbar_wait(&full[0], 0, kWaitLimit));
   tc_fence_before();
   bool alive = __syncthreads_or(!good) == 0;
   tc_fence_after();
@@ -951,6 +1091,8 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
     }
     if (__syncthreads_or(!good)) { alive = false; break; }
     tc_fence_after();
+    if (HALF && i + 1 == mid)           // the state after the first `mid` chunks (once)
+      store_state_cols(mid_dst, tl + ST_S + 32 * wq, init_identity, wq, j, dk, dv);
     // coalesced 16-byte stores of the tile (overlap the next MMA)
     // (warps 1 .. 15: thread 0 is free to issue the next chunk's MMAs)
     if (outputs && warp > 0) {
@@ -973,38 +1115,43 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
 
   // ---- final state
   if (alive && fin) {
-    uint32_t t[2][16];
-    tmem_ld16(tl + ST_S + 32 * wq, t[0]);
-    tmem_ld16(tl + ST_S + 32 * wq + 16, t[1]);
-    tmem_wait_ld();
-    if (init_identity) {
-      // a transition X_p: bf16 hi / lo images for the segment combine (MN-major
-      // SW128 A operand, M = row of X, K = column; TMEM lane j holds column j of X)
-      uint8_t* xb = reinterpret_cast<uint8_t*>(fin);
+    if (HALF) {
+      store_state_cols(fin, tl + ST_S + 32 * wq, init_identity, wq, j, dk, dv);
+    } else {
+      uint32_t t[2][16];
+      tmem_ld16(tl + ST_S + 32 * wq, t[0]);
+      tmem_ld16(tl + ST_S + 32 * wq + 16, t[1]);
+      tmem_wait_ld();
+      if (init_identity) {
+        // a transition X_p: bf16 hi / lo images for the segment combine (MN-major
+        // SW128 A operand, M = row of X, K = column; TMEM lane j holds column j of X)
+        uint8_t* xb = reinterpret_cast<uint8_t*>(fin);
 #pragma unroll
-      for (int c8 = 0; c8 < 4; ++c8) {
-        uint32_t hw[4], lw[4];
+        for (int c8 = 0; c8 < 4; ++c8) {
+          uint32_t hw[4], lw[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float x0 = __uint_as_float(t[c8 >> 1][(c8 & 1) * 8 + 2 * e]);
-          const float x1 = __uint_as_float(t[c8 >> 1][(c8 & 1) * 8 + 2 * e + 1]);
-          hw[e] = pack_bf16(x0, x1);
-          lw[e] = pack_bf16(x0 - bf_lo(hw[e]), x1 - bf_hi(hw[e]));
+          for (int e = 0; e < 4; ++e) {
+            const float x0 = __uint_as_float(t[c8 >> 1][(c8 & 1) * 8 + 2 * e]);
+            const float x1 = __uint_as_float(t[c8 >> 1][(c8 & 1) * 8 + 2 * e + 1]);
+            hw[e] = pack_bf16(x0, x1);
+            lw[e] = pack_bf16(x0 - bf_lo(hw[e]), x1 - bf_hi(hw[e]));
+          }
+          const uint32_t o = chunk_mnmajor_sw128((uint32_t)(4 * wq + c8), (uint32_t)j, D);
+          *reinterpret_cast<uint4*>(xb + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          *reinterpret_cast<uint4*>(xb + 32768 + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
         }
-        const uint32_t o = chunk_mnmajor_sw128((uint32_t)(4 * wq + c8), (uint32_t)j, D);
-        *reinterpret_cast<uint4*>(xb + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-        *reinterpret_cast<uint4*>(xb + 32768 + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-      }
-    } else if (j < dv) {
+      } else if (j < dv) {
 #pragma unroll
-      for (int e = 0; e < 32; ++e)
-        if (32 * wq + e < dk) fin[(long long)(32 * wq + e) * dv + j] = __uint_as_float(t[e >> 4][e & 15]);
+        for (int e = 0; e < 32; ++e)
+          if (32 * wq + e < dk) fin[(long long)(32 * wq + e) * dv + j] = __uint_as_float(t[e >> 4][e & 15]);
+      }
     }
   }
   if (!alive && tid == 0) {
     atomicExch(&g_chunk_split_timeout, 1);
     // let the MMA and the copies still in flight finish before the CTA exits
     mbar_wait(&mbar, mphase ^ 1u, kWaitLimit);
+    if (HALF && xstate >= 1) mbar_wait(&xbar, xstate - 1, kWaitLimit);   // images, or MMAs on them
     for (int r = waited; r < issued; ++r) mbar_wait(&full[r & 1], (r >> 1) & 1, kWaitLimit);
   }
   tc_fence_before();
@@ -1025,37 +1172,51 @@ bool set_attrs() {
                              cudaFuncAttributeMaxDynamicSharedMemorySize, PREP_SMEM) != cudaSuccess ||
         cudaFuncSetAttribute(kda_chunk_prep_kernel<true>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, PREP_SMEM) != cudaSuccess ||
-        cudaFuncSetAttribute(kda_state_pass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             STATE_SMEM) != cudaSuccess)
+        cudaFuncSetAttribute(kda_state_pass_kernel<false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, STATE_SMEM) != cudaSuccess ||
+        cudaFuncSetAttribute(kda_state_pass_kernel<true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, STATE_SMEM) != cudaSuccess)
       return false;
     done[dev] = true;
   }
   return true;
 }
 
-// Chunks per segment (0: no split).  Cost model in units of one state-pass
-// chunk step: pass A runs NH*(2P-3) chains, pass C NH*(P-1), each G chunks
-// long, in waves of one chain per SM; the combine costs kCombine steps per
-// segment.
+// Chunks per segment (G = 0: no split) and the half point of pass C (0: none).
+// Cost model in units of one state-pass chunk step: pass A runs NH*(2P-3)
+// chains, each G chunks long, in waves of one chain per SM; pass C runs NH*(P-1)
+// chains of G chunks, or with half points NH*(2(P-2)+1) chains of at most
+// max(Gh, last segment) chunks; the combine costs kCombine steps per segment and
+// a second-half chain's start (its S_mid product) kMid steps.
 constexpr double kCombine = 2.5;
-int plan_split(int B, int T, int H, bool varlen, int sms) {
+constexpr double kMid = 1.0;
+struct SplitPlan {
+  int G, half;
+};
+SplitPlan plan_split(int B, int T, int H, bool varlen, int sms) {
   const long long NH = (long long)B * H;
   const long long nch = ((long long)T + C - 1) / C;
-  if (NH >= sms || nch < 8) return 0;
-  if (varlen) return nch >= 2 * 16 ? 16 : 0;
+  if (NH >= sms || nch < 8) return {0, 0};
+  if (varlen) return {nch >= 2 * 16 ? 16 : 0, 0};
   const long long w1 = (NH + sms - 1) / sms;
   double best = (double)(nch * w1);
-  int bestG = 0;
-  for (int P = 2; P <= 64 && P <= nch; ++P) {
-    const long long G = (nch + P - 1) / P;
+  SplitPlan plan{0, 0};
+  for (long long G = 2; G < nch; ++G) {
     const long long Pe = (nch + G - 1) / G;
-    if (Pe < 2) continue;
+    if (Pe < 2 || Pe > 64) continue;
     const long long wA = (NH * (2 * Pe - 3) + sms - 1) / sms;
     const long long wC = (NH * (Pe - 1) + sms - 1) / sms;
     const double cost = (double)G * (double)(wA + wC) + kCombine * (double)(Pe - 2) + 2.0;
-    if (cost < best) { best = cost; bestG = (int)G; }
+    if (cost < best) { best = cost; plan = {(int)G, 0}; }
+    if (Pe >= 3) {
+      const long long Gh = (G + 1) / 2, last = nch - (Pe - 1) * G;
+      const long long wCh = (NH * (2 * (Pe - 2) + 1) + sms - 1) / sms;
+      const double costh = (double)G * (double)wA + (double)std::max(Gh, last) * (double)wCh +
+                           kCombine * (double)(Pe - 2) + kMid + 2.0;
+      if (costh < best) { best = costh; plan = {(int)G, (int)Gh}; }
+    }
   }
-  return bestG;
+  return plan;
 }
 
 }  // namespace
@@ -1081,7 +1242,8 @@ cudaError_t launch_chunk_split(const void* q, const void* k, const void* v, cons
 
   const long long nslots = chunk_slots(B, T, varlen);
   const size_t rec_bytes = (size_t)nslots * H * REC_BYTES;
-  const int G = plan_split(B, T, H, varlen, sms);
+  const SplitPlan plan = plan_split(B, T, H, varlen, sms);
+  const int G = plan.G;
   const long long nch_all = ((long long)T + C - 1) / C;
   int P = 0;
   long long slots = 0;
@@ -1089,7 +1251,7 @@ cudaError_t launch_chunk_split(const void* q, const void* k, const void* v, cons
   if (G > 0 && (nch_all + G - 1) / G >= 2) {
     P = (int)((nch_all + G - 1) / G);
     slots = varlen ? (long long)P + B : (long long)B * P;
-    seg_bytes = (size_t)2 * slots * H * D * D * sizeof(float);
+    seg_bytes = (size_t)(plan.half > 0 ? 4 : 2) * slots * H * D * D * sizeof(float);
   }
   void* scratch = nullptr;
   if (rec_bytes + seg_bytes > 0) {
@@ -1117,19 +1279,30 @@ cudaError_t launch_chunk_split(const void* q, const void* k, const void* v, cons
   if (P == 0) {
     SegArgs sa{0, 1, 0, 0, nullptr, nullptr};
     KDA_TIMED(KDA_KERNEL_STATE, stream,
-              kda_state_pass_kernel<<<dim3(H, B, 1), NT_S, STATE_SMEM, stream>>>(rec, h0, cu_seqlens, ob, hT,
-                                                                               T, H, dk, dv, nslots, sa, gt));
+              kda_state_pass_kernel<false><<<dim3(H, B, 1), NT_S, STATE_SMEM, stream>>>(
+                  rec, h0, cu_seqlens, ob, hT, T, H, dk, dv, nslots, sa, gt));
     note_launches(1);
   } else {
-    SegArgs sa{G, P, 1, (int)slots, segbuf, segbuf + (size_t)slots * H * D * D};
-    KDA_TIMED(KDA_KERNEL_STATE, stream,
-              kda_state_pass_kernel<<<dim3(H, B, 2 * P), NT_S, STATE_SMEM, stream>>>(rec, h0, cu_seqlens, ob,
-                                                                                   hT, T, H, dk, dv, nslots, sa, gt));
+    const size_t per = (size_t)slots * H * D * D;
+    SegArgs sa{G, P, 1, (int)slots, segbuf, segbuf + per};
+    if (plan.half > 0) {
+      sa.half = plan.half;
+      sa.sbuf_h = segbuf + 2 * per;
+      sa.xbuf_h = segbuf + 3 * per;
+    }
+    auto state_pass = [&](dim3 grid) {
+      if (sa.half > 0)
+        kda_state_pass_kernel<true><<<grid, NT_S, STATE_SMEM, stream>>>(rec, h0, cu_seqlens, ob, hT, T, H, dk,
+                                                                        dv, nslots, sa, gt);
+      else
+        kda_state_pass_kernel<false><<<grid, NT_S, STATE_SMEM, stream>>>(rec, h0, cu_seqlens, ob, hT, T, H, dk,
+                                                                         dv, nslots, sa, gt);
+    };
+    KDA_TIMED(KDA_KERNEL_STATE, stream, state_pass(dim3(H, B, 2 * P)));
     const cudaError_t ec = launch_seg_combine_img(cu_seqlens, B, T, H, dk, dv, sa, stream);
     sa.pass = 2;
-    KDA_TIMED(KDA_KERNEL_STATE, stream,
-              kda_state_pass_kernel<<<dim3(H, B, P - 1), NT_S, STATE_SMEM, stream>>>(rec, h0, cu_seqlens, ob,
-                                                                                   hT, T, H, dk, dv, nslots, sa, gt));
+    const unsigned zc = (unsigned)(sa.half > 0 ? 2 * (P - 1) : P - 1);
+    KDA_TIMED(KDA_KERNEL_STATE, stream, state_pass(dim3(H, B, zc)));
     note_launches(2);
     if (ec != cudaSuccess) e = ec;
   }

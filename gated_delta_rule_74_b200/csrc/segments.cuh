@@ -21,6 +21,11 @@ constexpr int kHead = 128;     // dk = dv handled by the tensor-core kernels
 //   combine S_start,1 = S_end,0 and S_start,p+1 = X_p S_start,p + Sloc_p (fp32);
 //   pass C  segments p >= 1 run again from S_start,p and write their outputs;
 //           the last one writes hT.
+// With a half point Gh (split prefill), the pass A chains of segments 1 .. Ps-2
+// also keep their state after the first Gh chunks (Sloc_half,p and X_half,p), and
+// pass C runs each of those segments as two chains: [0, Gh) from S_start,p and
+// [Gh, G) from S_mid,p = X_half,p S_start,p + Sloc_half,p, which that chain forms
+// on the tensor cores before its first chunk.  This halves pass C's serial length.
 // This is the chunked recurrence's own affine structure over chunks, grouped.
 struct SegArgs {
   int G;          // chunks per segment; 0 = one chain walks the whole sequence
@@ -29,6 +34,9 @@ struct SegArgs {
   int slots;      // number of (segment) slots the scratch holds per head
   float* sbuf;    // [slots][H][D][D] fp32: Sloc_p, then S_start,p+1
   float* xbuf;    // [slots][H][D][D] fp32: X_p
+  int half;       // Gh: chunks of the first pass C chain of a split segment (0 = no split)
+  float* sbuf_h;  // [slots][H][D][D] fp32: Sloc_half,p
+  float* xbuf_h;  // [slots][H][D][D] fp32: X_half,p
 };
 
 // Token range of sequence s: rows [row0 + t_beg, row0 + t_end) of the token axis.

@@ -229,3 +229,13 @@ def test_split_slow_decay_carries_state_across_segments(T):
     decides the later segments' outputs; they must match the recurrence."""
     _check(ki.make_prefill(_spec("bf16", 128, 128, decay="logsigmoid", T=T, B=1, H=2,
                                  h0=True, seed=T + 1)))
+
+
+@pytest.mark.parametrize("T,decay", [(4100, "alog"), (8000, "logsigmoid"), (20000, "logsigmoid")])
+def test_split_half_points(T, decay):
+    """Shapes whose split runs pass C as two chains per segment (B=1, H=2: 4100
+    tokens -> segments of 10 chunks split at 5, 8000 -> 12 at 6, 20000 -> 22 at 11):
+    the half-point states S_mid = X_half S_start + Sloc_half start the second chains,
+    and the last, shorter segment runs whole."""
+    _check(ki.make_prefill(_spec("bf16", 128, 128, decay=decay, T=T, B=1, H=2, h0=True,
+                                 seed=T + 7)))
