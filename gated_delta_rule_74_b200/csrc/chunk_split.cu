@@ -178,6 +178,7 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   const int tid = threadIdx.x, warp = tid >> 5;
   const long long slot = blockIdx.x;
   const int h = blockIdx.y;
+  grid_dep_launch();          // the state pass may take SMs this grid no longer needs
 
   // which chunk of which sequence this slot is (uniform over the CTA)
   long long row0 = 0, t_beg = 0, t_end = 0, n = 0;
@@ -836,7 +837,11 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
   // X_half images and record 1 follows once they are consumed
   int issued = nch < 2 ? nch : (HALF && mid_x ? 1 : 2);
   int xstate = 0;                                    // thread 0: 1 images requested, 2 MMAs issued
+  // Launched right behind the kernel before it: the records come from the prep
+  // kernel, which has ended before pass C starts (pass A does not let its
+  // successor start early); the combine's output is read only after the wait below.
   if (tid == 0) {
+    if (sa.pass != 2) grid_dep_wait();
     for (int i = 0; i < issued; ++i) {
       mbar_arrive_expect_tx(&full[i], REC_BYTES);
       bulk_g2s(sm + i * S_BUF, rec_ptr(i), REC_BYTES, &full[i]);
@@ -853,6 +858,7 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
   const uint32_t tb = tmem_base_sh;
   const uint32_t tl = tb + lane_base;
 
+  if (sa.pass == 2) grid_dep_wait();     // S_start comes from the segment combine
   // ---- initial state: columns [32 wq, 32 wq + 32) of row j of S^T, and its bf16 copy
   {
     const int c = 32 * wq;
@@ -1279,8 +1285,8 @@ cudaError_t launch_chunk_split(const void* q, const void* k, const void* v, cons
   if (P == 0) {
     SegArgs sa{0, 1, 0, 0, nullptr, nullptr};
     KDA_TIMED(KDA_KERNEL_STATE, stream,
-              kda_state_pass_kernel<false><<<dim3(H, B, 1), NT_S, STATE_SMEM, stream>>>(
-                  rec, h0, cu_seqlens, ob, hT, T, H, dk, dv, nslots, sa, gt));
+              e = launch_after(kda_state_pass_kernel<false>, dim3(H, B, 1), dim3(NT_S), STATE_SMEM,
+                               stream, rec, h0, cu_seqlens, ob, hT, T, H, dk, dv, nslots, sa, gt));
     note_launches(1);
   } else {
     const size_t per = (size_t)slots * H * D * D;
@@ -1291,20 +1297,21 @@ cudaError_t launch_chunk_split(const void* q, const void* k, const void* v, cons
       sa.xbuf_h = segbuf + 3 * per;
     }
     auto state_pass = [&](dim3 grid) {
-      if (sa.half > 0)
-        kda_state_pass_kernel<true><<<grid, NT_S, STATE_SMEM, stream>>>(rec, h0, cu_seqlens, ob, hT, T, H, dk,
-                                                                        dv, nslots, sa, gt);
-      else
-        kda_state_pass_kernel<false><<<grid, NT_S, STATE_SMEM, stream>>>(rec, h0, cu_seqlens, ob, hT, T, H, dk,
-                                                                         dv, nslots, sa, gt);
+      return launch_after(sa.half > 0 ? kda_state_pass_kernel<true> : kda_state_pass_kernel<false>,
+                          grid, dim3(NT_S), STATE_SMEM, stream, rec, h0, cu_seqlens, ob, hT, T, H, dk,
+                          dv, nslots, sa, gt);
     };
-    KDA_TIMED(KDA_KERNEL_STATE, stream, state_pass(dim3(H, B, 2 * P)));
+    cudaError_t es = cudaSuccess;
+    KDA_TIMED(KDA_KERNEL_STATE, stream, es = state_pass(dim3(H, B, 2 * P)));
     const cudaError_t ec = launch_seg_combine_img(cu_seqlens, B, T, H, dk, dv, sa, stream);
     sa.pass = 2;
     const unsigned zc = (unsigned)(sa.half > 0 ? 2 * (P - 1) : P - 1);
-    KDA_TIMED(KDA_KERNEL_STATE, stream, state_pass(dim3(H, B, zc)));
+    const cudaError_t es2 = es;
+    KDA_TIMED(KDA_KERNEL_STATE, stream, es = state_pass(dim3(H, B, zc)));
     note_launches(2);
     if (ec != cudaSuccess) e = ec;
+    if (es2 != cudaSuccess) e = es2;
+    if (es != cudaSuccess) e = es;
   }
   const cudaError_t el = cudaGetLastError();
   if (e == cudaSuccess) e = el;

@@ -32,6 +32,25 @@ void timing_end(int handle, cudaStream_t stream);
     timing_end(kda_th_, stream);                      \
   } while (0)
 
+// Launch `kern` with programmatic stream serialization: it may start while the
+// kernel before it on `stream` is still running, and must call grid_dep_wait()
+// before touching anything that kernel writes (see sm100.cuh).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_after(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                         cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // Launchers implemented in the kernel translation units.  Each returns a
 // cudaError_t from the launch (cudaSuccess when the launch was accepted).
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* g,

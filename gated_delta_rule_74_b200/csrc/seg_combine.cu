@@ -212,6 +212,10 @@ kda_seg_combine_img_kernel(const int32_t* __restrict__ cu_seqlens, int T, int H,
                                            ~uintptr_t(1023));
   __shared__ uint64_t xfull[2], mbar;
   __shared__ uint32_t tmem_base_sh;
+  // launched right behind pass A: wait for its X_p and Sloc_p; pass C may start
+  // taking free SMs (it reads the combine's output only after its own wait)
+  grid_dep_launch();
+  grid_dep_wait();
   const int h = blockIdx.x, s = blockIdx.y, col0 = kQCols * blockIdx.z;
   if (col0 >= dv) return;
   long long r0, a, b;
@@ -385,11 +389,12 @@ cudaError_t launch_seg_combine_img(const int32_t* cu_seqlens, int B, int T, int 
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
+  cudaError_t e = cudaSuccess;
   KDA_TIMED(KDA_KERNEL_COMBINE, stream,
-            kda_seg_combine_img_kernel<<<dim3(H, B, dv / kQCols), kCombineThreads, kCombine2Smem,
-                                         stream>>>(cu_seqlens, T, H, dk, dv, sa));
+            e = launch_after(kda_seg_combine_img_kernel, dim3(H, B, dv / kQCols), dim3(kCombineThreads),
+                             kCombine2Smem, stream, cu_seqlens, T, H, dk, dv, sa));
   note_launches(1);
-  return cudaGetLastError();
+  return e;
 }
 
 // Reads (and with reset clears) g_seg_combine_timeout; host side of kda_device_status.

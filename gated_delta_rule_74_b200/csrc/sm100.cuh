@@ -131,6 +131,20 @@ __device__ __forceinline__ void named_arrive(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// ------------------------------------------- programmatic dependent launch
+// Kernels of one call that follow each other on a stream may be launched with
+// programmatic stream serialization: the next grid can start before this one
+// ends.  grid_dep_wait() blocks the calling thread until the preceding grid has
+// completed and its memory writes are visible (it returns at once when there is no
+// such grid); grid_dep_launch() lets the next grid start once every CTA of this
+// grid has executed it or exited.
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // -------------------------------------------------------------------- TMEM
 // Warp-collective.  Writes the allocated TMEM base address to *dst (smem).
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
