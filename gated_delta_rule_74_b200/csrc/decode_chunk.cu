@@ -340,7 +340,8 @@ kda_decode_chunk_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       for (int t = 0; t < LT; ++t)
         if (t < L) out[((n * L + t) * H + h) * D + j] = __float2bfloat16_rn(__uint_as_float(o[t]));
     }
-    // the new state: TMEM -> the tile region (free again) -> one bulk copy to HBM
+    // the new state straight to HBM: lane j holds column j of S, so each warp's store
+    // of one row of S covers 128 contiguous bytes
 #pragma unroll 1
     for (int q4 = 0; q4 < 4; ++q4) {
       uint32_t f[16];
@@ -348,14 +349,7 @@ kda_decode_chunk_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       tmem_ld16(tl + T_S + c0, f);
       tmem_wait_ld();
 #pragma unroll
-      for (int e = 0; e < 16; ++e) Sf[(c0 + e) * D + j] = __uint_as_float(f[e]);
-    }
-    fence_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-      bulk_s2g(Sp, Sf, D * D * 4);
-      bulk_commit();
-      bulk_wait_read<0>();
+      for (int e = 0; e < 16; ++e) Sp[(long long)(c0 + e) * D + j] = __uint_as_float(f[e]);
     }
   } while (false);
   if (!alive && tid == 0) {
