@@ -56,6 +56,17 @@ constexpr uint32_t DC_SMEM = M_SMALL + 3 * 256 * 4 + 64 + D * 4 + 1024;
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
+// D (16 x 8, fp32) += A (16 x 16) B (16 x 8), bf16 operands: lane l holds A rows l/4 and
+// l/4 + 8, columns 2 (l%4) + {0, 1} and + 8; B rows 2 (l%4) + {0, 1} and + 8, column l/4;
+// D rows l/4 and l/4 + 8, columns 2 (l%4) + {0, 1}.
+__device__ __forceinline__ void mma_bf16_16x8x16(float (&d)[4], const uint32_t (&a)[4],
+                                                 const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
 __device__ __forceinline__ uint4 pack8_bf16(const float (&x)[8]) {
   return make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
                     pack_bf16(x[6], x[7]));
@@ -211,26 +222,36 @@ kda_decode_chunk_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   }
   __syncthreads();
 
-  // ---- Gram pairs: thread tid < 136 -> Aqk(r, i <= r), else A(r, i < r) with
-  //      x = tid - 136; row r starts at r(r+1)/2 resp. r(r-1)/2
-  {
-    const bool isq = tid < 136;
-    const int x = isq ? tid : tid - 136;
-    int r = isq ? 0 : 1;
-#pragma unroll 1
-    while (r + 1 < LT && (isq ? (r + 1) * (r + 2) / 2 : (r + 1) * r / 2) <= x) ++r;
-    const int i = isq ? x - r * (r + 1) / 2 : x - r * (r - 1) / 2;
-    const float* xr = (isq ? fQP : fKP) + r * LDF;
-    const float* ki = fKM + i * LDF;
-    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-    for (int c = 0; c < D; c += 4) {
-      const float4 u = *reinterpret_cast<const float4*>(xr + c);
-      const float4 w = *reinterpret_cast<const float4*>(ki + c);
-      a.x = fmaf(u.x, w.x, a.x); a.y = fmaf(u.y, w.y, a.y);
-      a.z = fmaf(u.z, w.z, a.z); a.w = fmaf(u.w, w.w, a.w);
+  // ---- Gram on warp-level tensor-core tiles (mma.sync m16n8k16, bf16 operands as in the
+  //      prefill's Gram, fp32 accumulation): [q e^(G - G_8) ; k e^(G - G_8)] (32 x 128)
+  //      against the rows of k e^(G_8 - G) (16 x 128).  Warp w < 4 takes the 16 x 8 tile
+  //      (w >> 1, w & 1) and keeps Aqk(r, i <= r) resp. A(r, i < r); the products above
+  //      the diagonal are not used.
+  if (warp < 4) {
+    const int gq = lane >> 2, tq = lane & 3;
+    const float* X = (warp >> 1) ? fKP : fQP;
+    const int n0 = 8 * (warp & 1);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int k0 = 0; k0 < D; k0 += 16) {
+      const float2 a0 = *reinterpret_cast<const float2*>(X + gq * LDF + k0 + 2 * tq);
+      const float2 a1 = *reinterpret_cast<const float2*>(X + (gq + 8) * LDF + k0 + 2 * tq);
+      const float2 a2 = *reinterpret_cast<const float2*>(X + gq * LDF + k0 + 2 * tq + 8);
+      const float2 a3 = *reinterpret_cast<const float2*>(X + (gq + 8) * LDF + k0 + 2 * tq + 8);
+      const float2 b0 = *reinterpret_cast<const float2*>(fKM + (n0 + gq) * LDF + k0 + 2 * tq);
+      const float2 b1 = *reinterpret_cast<const float2*>(fKM + (n0 + gq) * LDF + k0 + 2 * tq + 8);
+      const uint32_t af[4] = {pack_bf16(a0.x, a0.y), pack_bf16(a1.x, a1.y), pack_bf16(a2.x, a2.y),
+                              pack_bf16(a3.x, a3.y)};
+      const uint32_t bfr[2] = {pack_bf16(b0.x, b0.y), pack_bf16(b1.x, b1.y)};
+      mma_bf16_16x8x16(acc, af, bfr);
     }
-    (isq ? sAqk : sA)[r * LT + i] = (a.x + a.y) + (a.z + a.w);
+    const bool isq = (warp >> 1) == 0;
+    float* dst = isq ? sAqk : sA;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int r = gq + 8 * (e >> 1), i = n0 + 2 * tq + (e & 1);
+      if (isq ? i <= r : i < r) dst[r * LT + i] = acc[e];
+    }
   }
   __syncthreads();
 
