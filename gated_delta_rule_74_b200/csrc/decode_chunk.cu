@@ -67,10 +67,6 @@ __device__ __forceinline__ void mma_bf16_16x8x16(float (&d)[4], const uint32_t (
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
-__device__ __forceinline__ uint4 pack8_bf16(const float (&x)[8]) {
-  return make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
-                    pack_bf16(x[6], x[7]));
-}
 __device__ __forceinline__ uint4 pack8_f16v(const float (&x)[8]) {
   return make_uint4(pack_f16(x[0], x[1]), pack_f16(x[2], x[3]), pack_f16(x[4], x[5]),
                     pack_f16(x[6], x[7]));
@@ -191,11 +187,12 @@ kda_decode_chunk_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   }
   __syncthreads();
 
-  // ---- per channel c (thread c < 128): Gamma = cumsum g; exp(Gamma_last); the Gram
-  //      factors k e^(G - G_8), k e^(G_8 - G), q e^(G - G_8) (each e^ clamped at 80);
-  //      Kbar = k e^G (into the Gamma tile); the Qbar and Kend operand images
-  if (tid < D) {
-    const int c = tid;
+  // ---- per channel c, two threads (tokens [0, 8) and [8, 16)): Gamma = cumsum g;
+  //      exp(Gamma_last); the Gram factors k e^(G - G_8), k e^(G_8 - G), q e^(G - G_8)
+  //      (each e^ clamped at 80); Kbar = k e^G (into the Gamma tile, once both threads
+  //      have read g); the Qbar and Kend operand images
+  {
+    const int c = tid & (D - 1), t0 = 8 * (tid >> 7);
     float G[LT];
     float acc = 0.f;
 #pragma unroll
@@ -204,20 +201,23 @@ kda_decode_chunk_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       G[t] = acc;
     }
     const float gl = acc;
-    sGl[c] = __expf(gl);
+    if (t0 == 0) sGl[c] = __expf(gl);
+    __syncthreads();
 #pragma unroll
-    for (int t = 0; t < LT; ++t) {
+    for (int i = 0; i < 8; ++i) {
+      const int t = t0 + i;
+      const float Gt = t0 ? G[8 + i] : G[i];      // register-resident either way
       const float kt = fk[t * LDF + c], qt = fq[t * LDF + c];
-      const float dG = G[t] - G[8];
+      const float dG = Gt - G[8];
       const float up = __expf(fminf(dG, 80.f)), dn = __expf(fminf(-dG, 80.f));
-      const float eg = __expf(G[t]);
+      const float eg = __expf(Gt);
       fKP[t * LDF + c] = kt * up;
       fKM[t * LDF + c] = kt * dn;
       fQP[t * LDF + c] = qt * up;
       fG[t * LDF + c] = kt * eg;                  // Kbar
       *reinterpret_cast<bf16*>(sm + M_B1 + off_mnmajor_sw32(t, c, D)) = __float2bfloat16_rn(qt * eg);
       *reinterpret_cast<__half*>(sm + M_KE + off_mnmajor_sw128(c, t, LT)) =
-          __float2half_rn(kt * __expf(gl - G[t]));
+          __float2half_rn(kt * __expf(gl - Gt));
     }
   }
   __syncthreads();
@@ -275,7 +275,13 @@ kda_decode_chunk_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     for (int r = 0; r < LT; ++r) {
       float acc = src[r * LDF + c];
 #pragma unroll
-      for (int i = 0; i < r; ++i) acc = fmaf(-sA[r * LT + i], y[i], acc);
+      for (int i4 = 0; i4 < (r + 3) / 4; ++i4) {          // row r of A, four at a time
+        const float4 a4 = *reinterpret_cast<const float4*>(sA + r * LT + 4 * i4);
+        const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (4 * i4 + e < r) acc = fmaf(-av[e], y[4 * i4 + e], acc);
+      }
       y[r] = sBeta[r] * acc;
     }
     if (isw) {
