@@ -87,11 +87,21 @@ typedef enum {
  * out must not alias any input.  hT may alias h0 (in-place state update).
  * B >= 1, T >= 0, H >= 1.  T == 0 writes hT = h0 (or zeros) and nothing else.
  *
- * Scratch: when a call splits sequences into segments (dk = dv = 128, bf16,
- * few (sequence, head) pairs) it takes 2 * 64 KB per segment and head from a
- * library-owned, stream-ordered memory pool of the current device; the pool
- * keeps its memory for later calls.  If that allocation fails the call runs
- * unsplit instead.
+ * Scratch (KDA_BF16): the call takes its working memory from a library-owned,
+ * stream-ordered memory pool of the current device, which keeps its memory for
+ * later calls; it is released on the stream when the call's kernels end:
+ *   - the chunk records, 90,624 B per (head, chunk), with ceil(T/64) * B chunks
+ *     (ceil(T/64) + B in packed mode);
+ *   - when few (sequence, head) pairs leave SMs idle and sequences are split into
+ *     segments: 2 * 64 KB per segment and head, 4 * 64 KB when the split also
+ *     keeps half-way states.
+ * If the scratch cannot be allocated nothing is launched and the call returns
+ * KDA_ERR_CUDA; kda_chunk_fwd_noalloc runs without allocating.
+ * The call's kernels follow each other on `stream` with programmatic stream
+ * serialization (a kernel may start while its predecessor in the call drains and
+ * waits for it on the device); its first kernel starts after the work queued
+ * before it, and work queued after the call sees all of its results, as for a
+ * plain launch.  The call can be captured into a CUDA graph.
  *
  * Precision: g, beta and the state are fp32.  With KDA_BF16 inputs the chunk
  * contractions run on the tensor cores with fp32 accumulation, on bf16 operands
