@@ -239,3 +239,12 @@ def test_split_half_points(T, decay):
     and the last, shorter segment runs whole."""
     _check(ki.make_prefill(_spec("bf16", 128, 128, decay=decay, T=T, B=1, H=2, h0=True,
                                  seed=T + 7)))
+
+
+@pytest.mark.parametrize("B,T,H", [(1, 131072, 1), (2, 32768, 4)])
+def test_split_long_sequences(B, T, H):
+    """Very long sequences over few heads: the split runs dozens of segments with half
+    points (131072 tokens, one head: 36 segments of 58 chunks, halves of 29), with slow
+    decay so state crosses every segment boundary."""
+    _check(ki.make_prefill(_spec("bf16", 128, 128, decay="logsigmoid", T=T, B=B, H=H, h0=True,
+                                 seed=T + H)))
