@@ -1,10 +1,10 @@
 """Benchmark of the KDA hot path on B200: chunked prefill and recurrent decode.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload metric|cfg1|cfg2|cfg3]
+                    [--workload t8k_h12|b16_t512_d64|packed_16k|t32k_h96]
 
 One JSON line on rank 0.  `value` is prefill tokens/s over all ranks for the
-headline prefill shape (B=1, T=8192, H=12, dk=dv=128, bf16; "metric" workload),
+headline prefill shape (B=1, T=8192, H=12, dk=dv=128, bf16; workload "t8k_h12"),
 measured over K timed calls of kda_chunk_fwd with the inputs already in HBM.
 Each rank runs its own shard (independent sequences, no collective: weak
 scaling).  The `decode` object is the second half of the metric: K timed
@@ -251,7 +251,7 @@ def _config(args, x, world):
             "head_dim": x["dk"], "parallelism": f"dp{world} (independent sequences per rank)",
             "l2": "prefill rotates 3 resident input sets (3 x inputs > 126 MB L2); decode "
                   "state 1.61 GB > L2",
-            "decode_workload": "cfg4: N=256 H=96 d=128 bf16, fp32 state 1.61 GB"}
+            "decode_workload": "decode_n256_h96: N=256 H=96 d=128 bf16, fp32 state 1.61 GB"}
 
 
 def _oracle_timing(args):
@@ -595,7 +595,7 @@ def decode_leg(args, world, rank, dev, stream, barrier, clocks, hbm, peak_kind):
     import gated_delta_rule_74_b200 as kda
     import kda_inputs as ki
 
-    dspec = ki.DECODE_SPECS["cfg4"]
+    dspec = ki.DECODE_SPECS["decode_n256_h96"]
     dd = ki.make_decode(dspec, steps=1, seed=dspec.seed + 1000 * rank, N=args.decode_n or None)
     S = dd["S0"].to(dev)
     q, k, v, g, b = (dd[n][0].to(dev) for n in ("q", "k", "v", "g", "beta"))
@@ -657,7 +657,7 @@ def decode_leg(args, world, rank, dev, stream, barrier, clocks, hbm, peak_kind):
                 kda.kda_decode_chunk, "kda_decode_chunk (one chunk on the tensor cores)")
         del tq, tout
     return {"metric": "decode state GB/s vs HBM peak", "fused_tokens": fused, "workload":
-            f"cfg4 shape: N={dd['N']} H={dd['H']} dk=dv=128 bf16 q/k/v, fp32 state "
+            f"decode_n256_h96 shape: N={dd['N']} H={dd['H']} dk=dv=128 bf16 q/k/v, fp32 state "
             f"{dd['N'] * dd['H'] * 65536 / 1e9:.2f} GB", "gbs": gbs,
             "frac_of_hbm_peak": gbs / hbm, "peak_gbs": hbm, "peak_kind": peak_kind,
             "steps_per_s": 1e3 / step_ms, "tokens_per_s": dd["N"] * world * 1e3 / step_ms,
@@ -857,7 +857,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="metric", choices=["metric", "cfg1", "cfg2", "cfg3"])
+    ap.add_argument("--workload", default="t8k_h12", choices=["t8k_h12", "b16_t512_d64", "packed_16k", "t32k_h96"])
     ap.add_argument("--decode-steps", type=int, default=100)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-fused-prep", action="store_true",

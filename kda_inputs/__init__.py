@@ -75,28 +75,28 @@ class DecodeSpec:
     desc: str = ""
 
 
-# The five workloads plus the headline prefill shape.
+# The workloads: four prefill shapes, the headline prefill shape, the decode shape.
 PREFILL_SPECS = {
-    "cfg0": PrefillSpec("cfg0", B=1, T=256, H=2, dk=64, dv=64, dtype="f32",
+    "fp32_t256": PrefillSpec("fp32_t256", B=1, T=256, H=2, dk=64, dv=64, dtype="f32",
                         decay="logsigmoid", seed=0,
                         desc="fp32 KDA forward, B=1 T=256 H=2 d=64"),
-    "cfg1": PrefillSpec("cfg1", B=16, T=512, H=8, dk=64, dv=64, dtype="bf16",
+    "b16_t512_d64": PrefillSpec("b16_t512_d64", B=16, T=512, H=8, dk=64, dv=64, dtype="bf16",
                         decay="logsigmoid", seed=1,
                         desc="miniKimiK3-shaped prefill, B=16 T=512 H=8 d=64"),
-    "cfg2": PrefillSpec("cfg2", B=0, T=16384, H=12, dk=128, dv=128, dtype="bf16",
+    "packed_16k": PrefillSpec("packed_16k", B=0, T=16384, H=12, dk=128, dv=128, dtype="bf16",
                         decay="alog", seed=2, varlen=True,
                         desc="Mini-K3-1H-shaped packed varlen prefill, 16384 tokens, "
                              "docs ~ U[128, 4096], H=12 d=128"),
-    "cfg3": PrefillSpec("cfg3", B=1, T=32768, H=96, dk=128, dv=128, dtype="bf16",
+    "t32k_h96": PrefillSpec("t32k_h96", B=1, T=32768, H=96, dk=128, dv=128, dtype="bf16",
                         decay="alog", seed=3, h0=True,
                         desc="Kimi-K3-width long prefill, B=1 T=32768 H=96 d=128, h0 ~ N(0,0.02)"),
-    "metric": PrefillSpec("metric", B=1, T=8192, H=12, dk=128, dv=128, dtype="bf16",
+    "t8k_h12": PrefillSpec("t8k_h12", B=1, T=8192, H=12, dk=128, dv=128, dtype="bf16",
                           decay="alog", seed=100,
                           desc="headline prefill, B=1 T=8192 H=12 d=128 bf16"),
 }
 
 DECODE_SPECS = {
-    "cfg4": DecodeSpec("cfg4", N=256, H=96, dk=128, dv=128, steps=16, dtype="bf16",
+    "decode_n256_h96": DecodeSpec("decode_n256_h96", N=256, H=96, dk=128, dv=128, steps=16, dtype="bf16",
                        decay="alog", seed=4,
                        desc="recurrent decode, N=256 x 16 tokens, H=96 d=128, "
                             "fp32 state ~ N(0,0.02) (1.61 GB)"),

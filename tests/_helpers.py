@@ -1,5 +1,5 @@
 """Shared helpers for the GPU parity tests: run the CUDA path and the oracle on the
-same seeded inputs and compare with the benchmark spec's metric
+same seeded inputs and compare them by the relative error
 max|x - x_ref| / max|x_ref| (computed separately for the output and the state)."""
 from __future__ import annotations
 

@@ -37,7 +37,7 @@ def _worker(rank, world, port, q):
         seeds = [bench.rank_seed(100, r, i) for i in range(3)]
         # the reference arm: only rank 0 runs it; the others return at once
         class A:  # noqa: E701 - minimal argument namespace
-            workload, ref_tokens, ref_seconds, gpus = "metric", 64, 0.0, w
+            workload, ref_tokens, ref_seconds, gpus = "t8k_h12", 64, 0.0, w
         rc = bench.run_reference(A, w, r) if r != 0 else 0
         q.put((r, w, l, ms, seeds, rc))
         dist.destroy_process_group()

@@ -38,7 +38,7 @@ def test_decode_small(dtype, dk, dv):
 def test_decode_cfg4_sampled():
     """Full config-4 shape (N=256, H=96, d=128, 16 consecutive tokens, 1.61 GB of
     fp32 state) on the GPU; the oracle checks 96 sampled (n, h) pairs."""
-    d = ki.make_decode("cfg4")
+    d = ki.make_decode("decode_n256_h96")
     N, H = d["N"], d["H"]
     rng = np.random.default_rng(0)
     pairs = np.sort(rng.choice(N * H, size=96, replace=False))
@@ -102,7 +102,7 @@ def test_decode_tokens_cfg4_sampled():
     """The config-4 workload (N=256, H=96, d=128, 16 tokens) as one launch; the
     oracle checks 64 sampled (n, h) pairs over all 16 tokens."""
     import gated_delta_rule_74_b200 as kda
-    d = ki.make_decode("cfg4")
+    d = ki.make_decode("decode_n256_h96")
     N, H, L = d["N"], d["H"], d["steps"]
     x = _tokens_inputs(d)
     S = d["S0"].cuda()

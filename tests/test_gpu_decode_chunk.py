@@ -43,7 +43,7 @@ def test_decode_chunk_close_to_single_steps():
 
 def test_decode_chunk_cfg4_sampled():
     """The config-4 shape (N = 256, H = 96, 16 tokens), 200 sampled (n, h) pairs."""
-    d = ki.make_decode("cfg4")
+    d = ki.make_decode("decode_n256_h96")
     x = {n: d[n].transpose(0, 1).contiguous() for n in ("q", "k", "v", "g", "beta")}
     S = d["S0"].cuda()
     out = kda.kda_decode_chunk(*(x[n].cuda() for n in ("q", "k", "v", "g", "beta")), S)

@@ -85,7 +85,7 @@ def test_fused_without_prep_or_gate_is_kda_chunk_fwd():
 def test_fused_long_sequence_sampled_heads():
     """The headline shape (T = 8192, 12 heads of 128, segmented state pass), two
     heads against the oracle."""
-    x = ki.make_fused_prefill("metric", W=4)
+    x = ki.make_fused_prefill("t8k_h12", W=4)
     out, hT = _run(x)
     heads = (3, 5)
     o_ref, s_ref = _ref(x, heads=heads)

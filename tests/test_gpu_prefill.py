@@ -24,26 +24,26 @@ def _check(x, heads=None, with_h0=True):
 
 
 # ---- the five workloads and the headline shape -------------------------------
-def test_cfg0_fp32():
-    _check(ki.make_prefill("cfg0"))
+def test_fp32_t256_fp32():
+    _check(ki.make_prefill("fp32_t256"))
 
 
-def test_cfg1_bf16():
-    _check(ki.make_prefill("cfg1"))
+def test_b16_t512_d64_bf16():
+    _check(ki.make_prefill("b16_t512_d64"))
 
 
-def test_cfg2_varlen():
-    _check(ki.make_prefill("cfg2"))
+def test_packed_16k_varlen():
+    _check(ki.make_prefill("packed_16k"))
 
 
-def test_metric_shape():
-    _check(ki.make_prefill("metric"))
+def test_t8k_h12_shape():
+    _check(ki.make_prefill("t8k_h12"))
 
 
-def test_cfg3_sampled_heads():
+def test_t32k_h96_sampled_heads():
     """B=1, T=32768, H=96, d=128 with h0 ~ N(0, 0.02) on the GPU; the oracle
     checks heads 0, 1 and 95 over the whole sequence."""
-    x = ki.make_prefill("cfg3")
+    x = ki.make_prefill("t32k_h96")
     out, hT = gpu_prefill(x)
     for lo, hi in ((0, 2), (95, 96)):
         o_ref, s_ref = oracle_prefill(x, heads=(lo, hi))

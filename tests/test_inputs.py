@@ -5,7 +5,7 @@ import kda_inputs as ki
 
 
 def test_prefill_shapes_and_ranges():
-    x = ki.make_prefill("cfg1", T=64, B=2)
+    x = ki.make_prefill("b16_t512_d64", T=64, B=2)
     assert x["q"].shape == (2, 64, 8, 64) and x["q"].dtype == torch.bfloat16
     assert x["g"].dtype == torch.float32 and (x["g"] <= 0).all()
     assert ((x["beta"] > 0) & (x["beta"] < 1)).all()
@@ -17,15 +17,15 @@ def test_prefill_shapes_and_ranges():
 
 
 def test_prefill_deterministic():
-    a = ki.make_prefill("cfg0")
-    b = ki.make_prefill("cfg0")
+    a = ki.make_prefill("fp32_t256")
+    b = ki.make_prefill("fp32_t256")
     for key in ("q", "k", "v", "g", "beta"):
         assert torch.equal(a[key], b[key])
     assert a["q"].dtype == torch.float32
 
 
 def test_varlen_doc_lengths():
-    x = ki.make_prefill("cfg2")
+    x = ki.make_prefill("packed_16k")
     cu = x["cu_seqlens"]
     assert int(cu[0]) == 0 and int(cu[-1]) == 16384 == x["T"]
     lens = (cu[1:] - cu[:-1]).tolist()
@@ -34,13 +34,13 @@ def test_varlen_doc_lengths():
 
 
 def test_alog_decay_and_h0():
-    x = ki.make_prefill("cfg3", T=128, H=4)
+    x = ki.make_prefill("t32k_h96", T=128, H=4)
     assert x["h0"].shape == (1, 4, 128, 128)
     assert abs(float(x["h0"].std()) - 0.02) < 2e-3
     assert (x["g"] <= 0).all()
 
 
 def test_decode_inputs():
-    d = ki.make_decode("cfg4", N=4, H=3, steps=2)
+    d = ki.make_decode("decode_n256_h96", N=4, H=3, steps=2)
     assert d["q"].shape == (2, 4, 3, 128) and d["S0"].shape == (4, 3, 128, 128)
     assert d["beta"].shape == (2, 4, 3)

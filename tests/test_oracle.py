@@ -137,7 +137,7 @@ def test_hand_example_catches_mutations(mutation):
 
 # ----------------------------------------------------------------------------
 # beta = 0: the write vanishes and the state only decays per channel
-# (north-star update with beta = 0; "Inside Kimi" outline, KDA gating lesson:
+# (the KDA update with beta = 0; "Inside Kimi" outline, KDA gating lesson:
 # channel-wise decay).  Closed form S_T = Diag(exp(sum_t g_t)) h0.
 # ----------------------------------------------------------------------------
 def test_beta_zero_pure_channel_decay(oracle_lib):

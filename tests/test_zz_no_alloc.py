@@ -42,7 +42,7 @@ def _call_noalloc(d, out, hT):
 def test_noalloc_matches_chunk_fwd_twice(shape):
     if shape == "fixed":
         # B*H = 12 with 128 chunks: the call is split into segments (uses scratch)
-        x = ki.make_prefill("metric", H=6, T=4096)
+        x = ki.make_prefill("t8k_h12", H=6, T=4096)
     else:
         spec = ki.PrefillSpec("varlen", B=0, T=0, H=3, dk=128, dv=128, dtype="bf16",
                               decay="alog", seed=12, h0=True, varlen=True)
