@@ -44,6 +44,8 @@
 // 16-token block the cumulative log-decay must stay above -80 per channel.
 // All four products (A and Aqk rows for all blocks) are one MMA of N = 160:
 //   [D^(0) .. D^(3)] [128 x 160] = [Lk ; Lq] [R^(0); ..; R^(3)]^T
+#include <cuda_fp16.h>
+
 #include <algorithm>
 #include <type_traits>
 
@@ -70,10 +72,10 @@ constexpr uint32_t REC_QW = 0;          // [Qbar^T | W^T]: MN-major SW128, N = 1
                                         // 16 KB apart), K = dk
 constexpr uint32_t REC_KA = 32768;      // [Kend^T ; Aqk] (f16): K-major SW128, 192 rows x 64 tokens
 constexpr uint32_t REC_AQK = REC_KA + 16384;
-constexpr uint32_t REC_U = 57344;       // U^T [dv][64 tokens] fp32: 256-byte rows, 16-byte
-                                        // chunks XOR-swizzled with (row % 16)
-constexpr uint32_t REC_DECAY = 90112;   // exp(G_last) per key channel, fp32 [dk]
-constexpr uint32_t REC_BYTES = 90624;
+constexpr uint32_t REC_U = 57344;       // U^T [dv][64 tokens] f16: 128-byte rows, 16-byte
+                                        // chunks (8 tokens) XOR-swizzled with (row % 8)
+constexpr uint32_t REC_DECAY = 73728;   // exp(G_last) per key channel, fp32 [dk]
+constexpr uint32_t REC_BYTES = 74240;
 
 // ---- prep kernel: shared memory (from a 1024-aligned base) and TMEM
 constexpr uint32_t Q_V = 0;             // V: MN-major SW128 A operand of U^T (M = value, K = token)
@@ -99,7 +101,7 @@ constexpr uint32_t PT_U = 64;           // U^T [128 x 64]
 constexpr uint32_t kPrepTmemCols = 256;
 
 // ---- state pass: shared memory and TMEM
-constexpr uint32_t S_BUF = 91136;       // record buffer stride (two buffers)
+constexpr uint32_t S_BUF = 74752;       // record buffer stride (two buffers)
 constexpr uint32_t S_OUT = 2 * S_BUF;   // output tile [64 tokens][128] bf16
 constexpr uint32_t S_GATE = S_OUT + 16384;   // output-gate tile [64 tokens][128] bf16
 constexpr uint32_t STATE_SMEM = S_GATE + 16384 + 1024;
@@ -131,6 +133,12 @@ __device__ __forceinline__ void sts16(uint8_t* base, uint32_t off, uint4 v) {
 }
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+__device__ __forceinline__ float h_lo(uint32_t w) {
+  return __half2float(__ushort_as_half((unsigned short)(w & 0xffffu)));
+}
+__device__ __forceinline__ float h_hi(uint32_t w) {
+  return __half2float(__ushort_as_half((unsigned short)(w >> 16)));
+}
 
 // Sum over the warp's 32 lanes of each of 16 per-lane values; lane l returns the
 // total of value l / 2 (transpose-reduce: halves exchanged at lane distance 16,
@@ -611,7 +619,7 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   }
 
   if (alive) {
-    // ---- P5: W^T (lower warpgroup) -> bf16 record image; U^T (upper) -> fp32
+    // ---- P5: W^T (lower warpgroup) -> bf16 record image; U^T (upper) -> f16
     // record rows (Delta = U - W S is formed in fp32 by the state pass)
     const int j = tid & 127;
     uint32_t t[4][16];
@@ -631,9 +639,13 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       }
     } else {
 #pragma unroll
-      for (int c4 = 0; c4 < 16; ++c4) {
-        const uint32_t* f = t[c4 >> 2] + 4 * (c4 & 3);
-        sts16(sm, Q_OU + j * 256 + (((uint32_t)c4 ^ (j & 15u)) << 4), make_uint4(f[0], f[1], f[2], f[3]));
+      for (int c8 = 0; c8 < 8; ++c8) {
+        const uint32_t* f = t[c8 >> 1] + 8 * (c8 & 1);
+        const uint4 val = make_uint4(pack_f16(__uint_as_float(f[0]), __uint_as_float(f[1])),
+                                     pack_f16(__uint_as_float(f[2]), __uint_as_float(f[3])),
+                                     pack_f16(__uint_as_float(f[4]), __uint_as_float(f[5])),
+                                     pack_f16(__uint_as_float(f[6]), __uint_as_float(f[7])));
+        sts16(sm, Q_OU + j * 128 + (((uint32_t)c8 ^ (j & 7u)) << 4), val);
       }
     }
     fence_async_smem();
@@ -641,7 +653,7 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     if (tid == 0) {                          // the staged images go out as three bulk copies
       bulk_s2g(rc + REC_AQK, sm + Q_OAQK, 8192);
       bulk_s2g(rc + REC_QW + 16384, sm + Q_OW, 16384);
-      bulk_s2g(rc + REC_U, sm + Q_OU, 32768);
+      bulk_s2g(rc + REC_U, sm + Q_OU, 16384);
       bulk_commit();
       bulk_wait_read<0>();                   // shared memory read out before the CTA ends
     }
@@ -1019,21 +1031,20 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
     {
       uint32_t tp[16];
       tmem_ld16(tl + ST_P + 16 * wq, tp);
-      float4 u[4];
+      uint32_t uw[8];                  // U^T row j, tokens [16 wq, 16 wq + 16), f16 pairs
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4)
-        u[c4] = homog ? make_float4(0.f, 0.f, 0.f, 0.f)
-                      : *reinterpret_cast<const float4*>(
-                            rb + REC_U + j * 256 + ((((uint32_t)(4 * wq + c4)) ^ (j & 15u)) << 4));
+      for (int c = 0; c < 2; ++c) {
+        const uint4 v4 = homog ? make_uint4(0u, 0u, 0u, 0u)
+                               : *reinterpret_cast<const uint4*>(
+                                     rb + REC_U + j * 128 + ((((uint32_t)(2 * wq + c)) ^ (j & 7u)) << 4));
+        uw[4 * c] = v4.x; uw[4 * c + 1] = v4.y; uw[4 * c + 2] = v4.z; uw[4 * c + 3] = v4.w;
+      }
       tmem_wait_ld();
       uint32_t dw[8];
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        dw[2 * c4] = pack_f16(u[c4].x - __uint_as_float(tp[4 * c4]),
-                              u[c4].y - __uint_as_float(tp[4 * c4 + 1]));
-        dw[2 * c4 + 1] = pack_f16(u[c4].z - __uint_as_float(tp[4 * c4 + 2]),
-                                  u[c4].w - __uint_as_float(tp[4 * c4 + 3]));
-      }
+      for (int e = 0; e < 8; ++e)
+        dw[e] = pack_f16(h_lo(uw[e]) - __uint_as_float(tp[2 * e]),
+                         h_hi(uw[e]) - __uint_as_float(tp[2 * e + 1]));
       tmem_st8(tl + ST_D + 8 * wq, dw);
       tmem_wait_st();
     }

@@ -90,7 +90,7 @@ typedef enum {
  * Scratch (KDA_BF16): the call takes its working memory from a library-owned,
  * stream-ordered memory pool of the current device, which keeps its memory for
  * later calls; it is released on the stream when the call's kernels end:
- *   - the chunk records, 90,624 B per (head, chunk), with ceil(T/64) * B chunks
+ *   - the chunk records, 74,240 B per (head, chunk), with ceil(T/64) * B chunks
  *     (ceil(T/64) + B in packed mode);
  *   - when few (sequence, head) pairs leave SMs idle and sequences are split into
  *     segments: 2 * 64 KB per segment and head, 4 * 64 KB when the split also
