@@ -365,30 +365,36 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     for (int gg = 0; gg < 2; ++gg) {
       const int g8 = 2 * a + gg;               // group of 8 rows
       float lk[8], lq[8], kr[8];
+      if (c0 < dk) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int idx = 8 * gg + e;
-        const float x = (ch ? gq[idx].y : gq[idx].x) - Pa;
-        const float ell = __expf(x);
-        const float rho = __expf(fminf(-x, 80.f));
-        float kv, qv;
-        if constexpr (!CONV) {
-          kv = ch ? bf_hi(kw[idx]) : bf_lo(kw[idx]);
-          qv = ch ? bf_hi(qw[idx]) : bf_lo(qw[idx]);
-        } else {                       // normalised above
-          kv = ch ? kf[idx].y : kf[idx].x;
-          qv = ch ? qf[idx].y : qf[idx].x;
+        for (int e = 0; e < 8; ++e) {
+          const int idx = 8 * gg + e;
+          const float x = (ch ? gq[idx].y : gq[idx].x) - Pa;
+          const float ell = __expf(x);
+          const float rho = __expf(fminf(-x, 80.f));
+          float kv, qv;
+          if constexpr (!CONV) {
+            kv = ch ? bf_hi(kw[idx]) : bf_lo(kw[idx]);
+            qv = ch ? bf_hi(qw[idx]) : bf_lo(qw[idx]);
+          } else {                     // normalised above
+            kv = ch ? kf[idx].y : kf[idx].x;
+            qv = ch ? qf[idx].y : qf[idx].x;
+          }
+          lk[e] = kv * ell;
+          lq[e] = qv * ell;
+          kr[e] = kv * rho;                    // k_i e^{P_a - G_i}
         }
-        lk[e] = kv * ell;
-        lq[e] = qv * ell;
-        kr[e] = kv * rho;                      // k_i e^{P_a - G_i}
-      }
-      sts16(sm, Q_L + chunk_mnmajor_sw128(g8, c, D), pack8(lk, 1.f));
-      sts16(sm, Q_L + chunk_mnmajor_sw128(8 + g8, c, D), pack8(lq, 1.f));
-      sts16(sm, Q_KB + chunk_kmajor_sw128(c, g8, D), pack8(lk, eP));
+        // the Gram operands (its K loop covers channels < dk only)
+        sts16(sm, Q_L + chunk_mnmajor_sw128(g8, c, D), pack8(lk, 1.f));
+        sts16(sm, Q_L + chunk_mnmajor_sw128(8 + g8, c, D), pack8(lq, 1.f));
 #pragma unroll
-      for (int a2 = 0; a2 < 4; ++a2)
-        if (a2 >= a) sts16(sm, q_r(a2) + chunk_mnmajor_sw32(g8, c, D), pack8(kr, f[a2]));
+        for (int a2 = 0; a2 < 4; ++a2)
+          if (a2 >= a) sts16(sm, q_r(a2) + chunk_mnmajor_sw32(g8, c, D), pack8(kr, f[a2]));
+      } else {                         // padded channels (dk = 64; whole warps): zeros
+#pragma unroll
+        for (int e = 0; e < 8; ++e) lk[e] = lq[e] = kr[e] = 0.f;
+      }
+      sts16(sm, Q_KB + chunk_kmajor_sw128(c, g8, D), pack8(lk, eP));
       // record: Qbar^T (MN-major, N = tokens, K = channels) and Kend^T (K-major)
       *reinterpret_cast<uint4*>(rc + REC_QW + chunk_mnmajor_sw128(g8, c, D)) = pack8(lq, eP);
       *reinterpret_cast<uint4*>(rc + REC_KA + chunk_kmajor_sw128(c, g8, D)) = pack8_f16(kr, eE);
@@ -420,8 +426,7 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     tc_fence_after();
     const uint32_t l_base = smem_u32(sm + Q_L), r_base = smem_u32(sm + q_r(0));
     const uint32_t idesc = idesc_bf16(128, 160, true, true);
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk)
+    for (int kk = 0; kk < dk / 16; ++kk)       // channels < dk (64-wide heads: half the steps)
       mma_ss(tb + PT_G, desc_mnmajor_sw128(l_base, D, kk), desc_mnmajor_sw32(r_base, D, kk), idesc,
              kk > 0);
     mma_commit(&bar);
@@ -992,13 +997,11 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
       const uint32_t qw = smem_u32(rb + REC_QW);
       if (outputs) {
         const uint32_t id = idesc_bf16(128, 128, false, true);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
+        for (int kk = 0; kk < dk / 16; ++kk)   // channels < dk
           mma_ts(tb + ST_O, tb + ST_SB + kk * 8, desc_mnmajor_sw128(qw, D, kk), id, kk > 0);
       } else {
         const uint32_t id = idesc_bf16(128, 64, false, true);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
+        for (int kk = 0; kk < dk / 16; ++kk)
           mma_ts(tb + ST_P, tb + ST_SB + kk * 8, desc_mnmajor_sw128(qw + 16384, D, kk), id,
                  kk > 0);
       }
