@@ -671,12 +671,19 @@ KERNEL_NAMES = {"prep": "kda_chunk_prep_kernel", "state": "kda_state_pass_kernel
 
 
 def _source_hash() -> str:
+    """Hash of the kernel sources with comments and whitespace removed: DRAM traffic
+    depends on the code, so a comment edit keeps a capture valid."""
     import hashlib
+    import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_delta_rule_74_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)        # block comments
+        text = re.sub(r"//[^\n]*", " ", text)                      # line comments
+        text = re.sub(r"\s+", " ", text)
+        h.update(name.encode() + text.encode())
     return h.hexdigest()[:16]
 
 

@@ -854,9 +854,12 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
   // X_half images and record 1 follows once they are consumed
   int issued = nch < 2 ? nch : (HALF && mid_x ? 1 : 2);
   int xstate = 0;                                    // thread 0: 1 images requested, 2 MMAs issued
-  // Launched right behind the kernel before it: the records come from the prep
-  // kernel, which has ended before pass C starts (pass A does not let its
-  // successor start early); the combine's output is read only after the wait below.
+  // Launched right behind the kernel before it (programmatic stream serialization).
+  // Passes 0 and A wait for the prep kernel before the first record copy.  Pass C
+  // needs no wait for the records (prep) or a second-half chain's X_half images
+  // (pass A): pass A does not let its successor start early, so the combine, and pass
+  // C after it, start only once pass A, and prep before it, have ended.  The combine's
+  // output (S_start) is read only after the wait below the copies.
   if (tid == 0) {
     if (sa.pass != 2) grid_dep_wait();
     for (int i = 0; i < issued; ++i) {
