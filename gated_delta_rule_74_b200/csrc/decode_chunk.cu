@@ -203,6 +203,7 @@ kda_decode_chunk_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     const float gl = acc;
     if (t0 == 0) sGl[c] = __expf(gl);
     __syncthreads();
+    float qb[8];                          // Qbar of these 8 tokens: one 16-byte chunk
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int t = t0 + i;
@@ -215,10 +216,13 @@ kda_decode_chunk_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       fKM[t * LDF + c] = kt * dn;
       fQP[t * LDF + c] = qt * up;
       fG[t * LDF + c] = kt * eg;                  // Kbar
-      *reinterpret_cast<bf16*>(sm + M_B1 + off_mnmajor_sw32(t, c, D)) = __float2bfloat16_rn(qt * eg);
+      qb[i] = qt * eg;
       *reinterpret_cast<__half*>(sm + M_KE + off_mnmajor_sw128(c, t, LT)) =
           __float2half_rn(kt * __expf(gl - Gt));
     }
+    *reinterpret_cast<uint4*>(sm + M_B1 + chunk_mnmajor_sw32(t0 >> 3, c, D)) =
+        make_uint4(pack_bf16(qb[0], qb[1]), pack_bf16(qb[2], qb[3]), pack_bf16(qb[4], qb[5]),
+                   pack_bf16(qb[6], qb[7]));
   }
   __syncthreads();
 
@@ -284,10 +288,12 @@ kda_decode_chunk_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       }
       y[r] = sBeta[r] * acc;
     }
-    if (isw) {
+    if (isw) {                          // tokens 0..7 and 8..15 of W: one 16-byte chunk each
 #pragma unroll
-      for (int r = 0; r < LT; ++r)
-        *reinterpret_cast<bf16*>(sm + M_B1 + off_mnmajor_sw32(LT + r, c, D)) = __float2bfloat16_rn(y[r]);
+      for (int h8 = 0; h8 < 2; ++h8)
+        *reinterpret_cast<uint4*>(sm + M_B1 + chunk_mnmajor_sw32(2 + h8, c, D)) =
+            make_uint4(pack_bf16(y[8 * h8], y[8 * h8 + 1]), pack_bf16(y[8 * h8 + 2], y[8 * h8 + 3]),
+                       pack_bf16(y[8 * h8 + 4], y[8 * h8 + 5]), pack_bf16(y[8 * h8 + 6], y[8 * h8 + 7]));
     } else {
 #pragma unroll
       for (int r = 0; r < LT; ++r) fU[r * LDF + c] = y[r];
