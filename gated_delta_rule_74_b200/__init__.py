@@ -94,6 +94,8 @@ def lib() -> ctypes.CDLL:
         L.kda_version.restype = ctypes.c_int
         L.kda_launch_count.argtypes = []
         L.kda_launch_count.restype = ctypes.c_ulonglong
+        L.kda_prefill_plan.argtypes = [ctypes.c_int] * 5 + [ctypes.POINTER(ctypes.c_int)] * 2
+        L.kda_prefill_plan.restype = ctypes.c_int
         L.kda_timing_start.argtypes = []
         L.kda_timing_start.restype = ctypes.c_int
         L.kda_timing_stop.argtypes = []
@@ -139,6 +141,17 @@ def kda_selftest_bounded_wait(polls: int = 1000, stream=None) -> None:
 def kda_launch_count() -> int:
     """Kernels launched by libkda in this process so far."""
     return int(lib().kda_launch_count())
+
+
+def kda_prefill_plan(B: int, T: int, H: int, packed: bool = False, sms: int = 148) -> tuple:
+    """(chunks per segment, chunks of a half point) that kda_chunk_fwd's split takes for
+    B sequences of T tokens (packed: T tokens in B documents) over H heads on `sms` SMs;
+    (0, 0) when sequences are not split.  Host only."""
+    G, half = ctypes.c_int(0), ctypes.c_int(0)
+    rc = lib().kda_prefill_plan(B, T, H, int(bool(packed)), sms, ctypes.byref(G),
+                                ctypes.byref(half))
+    _check_status(rc, "kda_prefill_plan")
+    return int(G.value), int(half.value)
 
 
 KERNEL_KINDS = {"prep": 0, "state": 1, "combine": 2, "fused": 3, "simt": 4, "decode": 5,

@@ -255,4 +255,12 @@ unsigned long long kda_launch_count(void) {
   return kda::g_launches.load(std::memory_order_relaxed);
 }
 
+int kda_prefill_plan(int B, int T, int H, int packed, int sms, int* segment_chunks,
+                     int* half_chunks) {
+  if (B < 1 || T < 0 || H < 1 || sms < 1 || !segment_chunks || !half_chunks)
+    return KDA_ERR_INVALID_ARG;
+  kda::chunk_split_plan(B, T, H, packed != 0, sms, segment_chunks, half_chunks);
+  return KDA_OK;
+}
+
 }  // extern "C"

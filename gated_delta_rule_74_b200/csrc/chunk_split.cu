@@ -1248,6 +1248,12 @@ bool chunk_split_supported(int dk, int dv, int in_dtype) {
   return in_dtype == KDA_BF16 && (dk == 64 || dk == D) && (dv == 64 || dv == D);
 }
 
+void chunk_split_plan(int B, int T, int H, bool varlen, int sms, int* G, int* half) {
+  const SplitPlan p = plan_split(B, T, H, varlen, sms);
+  *G = p.G;
+  *half = p.half;
+}
+
 cudaError_t launch_chunk_split(const void* q, const void* k, const void* v, const float* g,
                                const float* beta, const float* h0, const int32_t* cu_seqlens,
                                void* out, float* hT, int B, int T, int H, int dk, int dv,

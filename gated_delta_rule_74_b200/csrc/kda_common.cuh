@@ -87,6 +87,8 @@ struct InputFusion {
 // (bf16, dk, dv in {64, 128}: 64-wide heads run zero-padded to 128); its
 // scratch comes from the library's memory pool.
 bool chunk_split_supported(int dk, int dv, int in_dtype);
+// The split prefill's plan (host only): chunks per segment, chunks of a half point.
+void chunk_split_plan(int B, int T, int H, bool varlen, int sms, int* G, int* half);
 cudaError_t launch_chunk_split(const void* q, const void* k, const void* v, const float* g,
                                const float* beta, const float* h0, const int32_t* cu_seqlens,
                                void* out, float* hT, int B, int T, int H, int dk, int dv,

@@ -357,6 +357,19 @@ KDA_API int kda_version(void);
  * since it was loaded (all threads, all devices).  Diagnostic only. */
 KDA_API unsigned long long kda_launch_count(void);
 
+/*
+ * kda_prefill_plan -- the sequence split kda_chunk_fwd (KDA_BF16, dk, dv in
+ * {64, 128}) chooses for B sequences of T tokens (packed != 0: T packed tokens in
+ * B documents) over H heads on a device with `sms` streaming multiprocessors.
+ * Host-only (no device access); diagnostic.  Writes *segment_chunks = G, the
+ * chunks (of 64 tokens) per segment, 0 when sequences are not split, and
+ * *half_chunks = Gh, the chunks of the first pass-C chain of a split middle
+ * segment, 0 without half points.  Returns KDA_OK, or KDA_ERR_INVALID_ARG for
+ * B, H or sms < 1, T < 0 or a NULL output pointer.
+ */
+KDA_API int kda_prefill_plan(int B, int T, int H, int packed, int sms, int* segment_chunks,
+                             int* half_chunks);
+
 /* Per-kernel timing (diagnostic; this library's own facility, with no
  * counterpart on the pages).  Between kda_timing_start() and
  * kda_timing_stop(), every kernel the library launches is bracketed by two CUDA
