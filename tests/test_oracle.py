@@ -280,6 +280,66 @@ def test_chunked_form_strong_decay(oracle_lib):
 
 
 # ----------------------------------------------------------------------------
+# The chunked form's backward (reference.chunked_backward: the adjoint of each
+# chunk's WY step, chunks in reverse) gives the gradients of the recurrence: the
+# C++ oracle's reverse-mode sweep, itself pinned by finite differences and
+# autograd below.  Ragged last chunks, C = 1 (one token per chunk) and strong decay.
+# ----------------------------------------------------------------------------
+def _bwd_pair(rng, T, dk, dv, C, g_scale=1.5):
+    q, k, v, g, b = _rand_inputs(rng, T, 1, dk, dv, g_scale=g_scale)
+    h0 = rng.standard_normal((1, 1, dk, dv))
+    dout = rng.standard_normal((1, T, 1, dv))
+    dhT = rng.standard_normal((1, 1, dk, dv))
+    rec = oracle.backward(q, k, v, g, b, dout, h0, dhT)
+    chk = ref.chunked_backward(q[0, :, 0], k[0, :, 0], v[0, :, 0], g[0, :, 0], b[0, :, 0],
+                               dout[0, :, 0], h0[0, 0], dhT[0, 0], C=C)
+    return (q, k, v, g, b, h0, dout, dhT), rec, chk
+
+
+def _assert_grads_equal(rec, chk, tol):
+    for key in ("dq", "dk", "dv", "dg", "dbeta"):
+        a = rec[key][0, :, 0]
+        assert np.abs(chk[key] - a).max() <= tol * max(np.abs(a).max(), 1e-30), key
+    a = rec["dh0"][0, 0]
+    assert np.abs(chk["dh0"] - a).max() <= tol * max(np.abs(a).max(), 1e-30), "dh0"
+
+
+@pytest.mark.parametrize("C", [1, 2, 4, 5, 64])
+@pytest.mark.parametrize("T", [1, 7, 63, 64, 65, 130])
+def test_chunked_backward_equals_recurrent_backward(oracle_lib, C, T):
+    rng = np.random.default_rng(500 + 7 * C + T)
+    _, rec, chk = _bwd_pair(rng, T, 8, 6, C)
+    _assert_grads_equal(rec, chk, 1e-11)
+
+
+def test_chunked_backward_strong_decay(oracle_lib):
+    """Chunk-wide decay down to about exp(-300): the pairwise exponents keep every
+    gradient term finite and exact in float64."""
+    _, rec, chk = _bwd_pair(np.random.default_rng(8), 150, 8, 8, 64, g_scale=2.5)
+    assert all(np.isfinite(chk[key]).all() for key in ("dq", "dk", "dv", "dg", "dbeta", "dh0"))
+    _assert_grads_equal(rec, chk, 1e-11)
+
+
+def test_chunked_backward_state_gradient_at_chunk_starts(oracle_lib):
+    """dS_start[c] is the gradient of the loss with respect to the state entering
+    chunk c: the recurrent backward of the suffix from chunk c, started from the
+    forward state there, returns it as its dh0."""
+    rng = np.random.default_rng(9)
+    T, dk, dv, C = 150, 6, 5, 32
+    (q, k, v, g, b, h0, dout, dhT), _, chk = _bwd_pair(rng, T, dk, dv, C)
+    for c in range(chk["dS_start"].shape[0]):
+        t0 = c * C
+        S_c = h0
+        if t0 > 0:
+            _, S_c = oracle.prefill(q[:, :t0], k[:, :t0], v[:, :t0], g[:, :t0], b[:, :t0], h0)
+        suf = oracle.backward(q[:, t0:], k[:, t0:], v[:, t0:], g[:, t0:], b[:, t0:],
+                              dout[:, t0:], S_c, dhT)
+        ref_ds = suf["dh0"][0, 0]
+        assert np.abs(chk["dS_start"][c] - ref_ds).max() <= 1e-11 * np.abs(ref_ds).max(), c
+    assert np.array_equal(chk["dS_start"][0], chk["dh0"])
+
+
+# ----------------------------------------------------------------------------
 # Packed documents are isolated (Mini-K3-1H-mamba2 card, packed-document
 # paragraph: state flow resets at every boundary; a later document gets exactly
 # nothing from earlier ones).  Forward analogue of the zero-gradient gate, over
