@@ -46,12 +46,20 @@ Kend, A and Aqk; dg is the reverse cumulative sum of dGamma inside the chunk.
 dS0 is the state gradient at the chunk's start, which the previous chunk takes
 as its dS.  It is pinned against the reverse-mode recurrence of the C++ oracle,
 which finite differences and autograd pin in turn.
+
+``reverse_state_segments``: the same chunk-start state gradients without the
+forward states.  Substituting dDelta into dS0 gives dS_n = Y_n dS_{n+1} + c_n
+with Y_n = Diag(exp(Gamma_last)) - W^T Kend and c_n = (Qbar - Aqk W)^T dO_n,
+neither of which depends on the state.  The reverse recurrence is affine, so
+it splits into segments of G chunks: each segment is run from its end once
+from zero (its local part) and once as the product of its Y_n (its
+transition), and the segments are then chained from the last.
 """
 from __future__ import annotations
 
 import numpy as np
 
-__all__ = ["recurrence_literal", "chunked", "chunked_backward"]
+__all__ = ["recurrence_literal", "chunked", "chunked_backward", "reverse_state_segments"]
 
 
 def recurrence_literal(q, k, v, g, beta, h0=None):
@@ -198,3 +206,45 @@ def chunked_backward(q, k, v, g, beta, dout, h0=None, dhT=None, C: int = 64):
         dS = dS0
     res["dh0"] = dS
     return res
+
+
+def reverse_state_segments(q, k, v, g, beta, dout, dhT=None, C: int = 64, G: int = 4):
+    """One sequence, one head: the gradient with respect to the state at every chunk
+    start ([nchunks, dk, dv], as ``chunked_backward``'s dS_start), computed from
+    per-chunk affine maps dS_n = Y_n dS_{n+1} + c_n grouped in segments of G chunks."""
+    q, k, v, g, dout = (np.asarray(x, dtype=np.float64) for x in (q, k, v, g, dout))
+    beta = np.asarray(beta, dtype=np.float64)
+    T, dk = k.shape
+    dv = v.shape[1]
+    Y, c = [], []
+    zero = np.zeros((dk, dv))
+    for t0 in range(0, T, C):                                   # per chunk, independent
+        t1 = min(t0 + C, T)
+        ct = _chunk_terms(q[t0:t1], k[t0:t1], v[t0:t1], g[t0:t1], beta[t0:t1], zero)
+        Y.append(np.diag(np.exp(ct["gam"][-1])) - ct["W"].T @ ct["kend"])
+        c.append((ct["qbar"] - ct["Aqk"] @ ct["W"]).T @ dout[t0:t1])
+    n = len(Y)
+    segs = [(a, min(a + G, n)) for a in range(0, n, G)]
+    # per segment, from its end: local part (from zero) and transition (product of Y)
+    loc, trans = [], []
+    for a, b in segs:
+        Lp, Xp = np.zeros((dk, dv)), np.eye(dk)
+        for i in reversed(range(a, b)):
+            Lp = Y[i] @ Lp + c[i]
+            Xp = Y[i] @ Xp
+        loc.append(Lp)
+        trans.append(Xp)
+    # chain the segments from the last: gradient entering each segment's end
+    end = np.zeros((dk, dv)) if dhT is None else np.array(dhT, dtype=np.float64)
+    seg_end = [None] * len(segs)
+    for p in reversed(range(len(segs))):
+        seg_end[p] = end
+        end = trans[p] @ end + loc[p]
+    # rerun each segment from its end gradient for the chunk starts inside it
+    out = np.zeros((n, dk, dv))
+    for p, (a, b) in enumerate(segs):
+        d = seg_end[p]
+        for i in reversed(range(a, b)):
+            d = Y[i] @ d + c[i]
+            out[i] = d
+    return out

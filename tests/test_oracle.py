@@ -339,6 +339,19 @@ def test_chunked_backward_state_gradient_at_chunk_starts(oracle_lib):
     assert np.array_equal(chk["dS_start"][0], chk["dh0"])
 
 
+@pytest.mark.parametrize("T,C,G", [(150, 32, 2), (130, 64, 1), (400, 16, 7), (64, 64, 3)])
+def test_reverse_state_segments_equal_chunk_start_gradients(oracle_lib, T, C, G):
+    """The reverse state recurrence needs no forward state and splits into segments:
+    its chunk-start gradients equal chunked_backward's, whose dS_start the suffix
+    pin above ties to the recurrent backward."""
+    rng = np.random.default_rng(T + C + G)
+    (q, k, v, g, b, h0, dout, dhT), _, chk = _bwd_pair(rng, T, 6, 5, C)
+    seg = ref.reverse_state_segments(q[0, :, 0], k[0, :, 0], v[0, :, 0], g[0, :, 0], b[0, :, 0],
+                                     dout[0, :, 0], dhT[0, 0], C=C, G=G)
+    assert seg.shape == chk["dS_start"].shape
+    assert np.abs(seg - chk["dS_start"]).max() <= 1e-11 * np.abs(chk["dS_start"]).max()
+
+
 # ----------------------------------------------------------------------------
 # Packed documents are isolated (Mini-K3-1H-mamba2 card, packed-document
 # paragraph: state flow resets at every boundary; a later document gets exactly
