@@ -339,6 +339,36 @@ def test_chunked_backward_state_gradient_at_chunk_starts(oracle_lib):
     assert np.array_equal(chk["dS_start"][0], chk["dh0"])
 
 
+def _pair_terms_einsum(dA, dAqk, q, k, gam):
+    """The pairwise terms exactly as chunked_backward forms them (full E tensor)."""
+    L = k.shape[0]
+    lower = np.tril(np.ones((L, L), dtype=bool))[:, :, None]
+    E = np.exp(np.where(lower, gam[:, None, :] - gam[None, :, :], -np.inf))
+    PA, PQ = np.tril(dA, -1)[:, :, None] * E, np.tril(dAqk)[:, :, None] * E
+    dk = np.einsum("ric,ic->rc", PA, k) + np.einsum("ric,rc->ic", PA, k) + \
+        np.einsum("ric,rc->ic", PQ, q)
+    dq = np.einsum("ric,ic->rc", PQ, k)
+    tA, tQ = PA * k[:, None, :] * k[None, :, :], PQ * q[:, None, :] * k[None, :, :]
+    dgam = tA.sum(1) - tA.sum(0) + tQ.sum(1) - tQ.sum(0)
+    return dq, dk, dgam
+
+
+@pytest.mark.parametrize("L,g_scale", [(64, 0.3), (64, 2.5), (45, 1.0), (16, 0.5), (7, 0.5)])
+def test_pair_grads_blocked_equal_pairwise_terms(L, g_scale):
+    """Splitting the exponents at 16-token reference points changes nothing but
+    rounding; with strong decay (Gamma down to about -160 in one chunk) every
+    factor stays finite."""
+    rng = np.random.default_rng(L + int(10 * g_scale))
+    q, k, _, g, _ = _rand_inputs(rng, L, 1, 8, 4, g_scale=g_scale)
+    q, k, gam = q[0, :, 0], k[0, :, 0], np.cumsum(g[0, :, 0], axis=0)
+    dA, dAqk = rng.standard_normal((L, L)), rng.standard_normal((L, L))
+    want = _pair_terms_einsum(dA, dAqk, q, k, gam)
+    got = ref.pair_grads_blocked(dA, dAqk, q, k, gam)
+    for w, x, name in zip(want, got, ("dq", "dk", "dgam")):
+        assert np.isfinite(x).all(), name
+        assert np.abs(x - w).max() <= 1e-12 * max(np.abs(w).max(), 1e-30), name
+
+
 @pytest.mark.parametrize("T,C,G", [(150, 32, 2), (130, 64, 1), (400, 16, 7), (64, 64, 3)])
 def test_reverse_state_segments_equal_chunk_start_gradients(oracle_lib, T, C, G):
     """The reverse state recurrence needs no forward state and splits into segments:
