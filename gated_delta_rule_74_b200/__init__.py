@@ -65,6 +65,9 @@ def lib() -> ctypes.CDLL:
         L.kda_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, fp, vp, vp, fp,
                                     ip, ip, ip, ip, ip, ip, vp]
         L.kda_chunk_fwd.restype = ctypes.c_int
+        L.kda_chunk_fwd_noalloc.argtypes = [vp, vp, vp, fp, fp, fp, vp, vp, fp,
+                                            ip, ip, ip, ip, ip, ip, vp]
+        L.kda_chunk_fwd_noalloc.restype = ctypes.c_int
         L.kda_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, vp, ip, ip, ip, ip, ip, vp]
         L.kda_decode_step.restype = ctypes.c_int
         L.kda_decode_tokens.argtypes = [vp, vp, vp, fp, fp, fp, vp, ip, ip, ip, ip, ip, ip, vp]
@@ -211,12 +214,13 @@ def kda_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Te
                   beta: torch.Tensor, h0: Optional[torch.Tensor] = None,
                   cu_seqlens: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
                   hT: Optional[torch.Tensor] = None, output_final_state: bool = True,
-                  stream=None):
+                  stream=None, noalloc: bool = False):
     """KDA prefill (chunked form).  q, k [B,T,H,dk]; v [B,T,H,dv]; g [B,T,H,dk] f32
     (or [B,T,H,dk/G] for one decay per group of G key channels, G a power of two:
     kda_chunk_fwd_grouped); beta [B,T,H] f32; h0 [Nseq,H,dk,dv] f32 or None;
     cu_seqlens int32 [Nseq+1] on the device, or None.  Returns (out, hT) (hT None
-    if output_final_state is False and no hT buffer was given)."""
+    if output_final_state is False and no hT buffer was given).  noalloc=True calls
+    kda_chunk_fwd_noalloc instead (per-channel decay only)."""
     if q.dim() != 4:
         raise ValueError("q must be [B, T, H, dk]")
     Bt, T, H, dk = q.shape
@@ -246,16 +250,18 @@ def kda_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Te
         hT = torch.empty((nseq, H, dk, dv), dtype=torch.float32, device=q.device)
     if hT is not None:
         _check("hT", hT, torch.float32, (nseq, H, dk, dv))
+    if noalloc and G != 1:
+        raise ValueError("kda_chunk_fwd_noalloc takes one decay per key channel")
     if G == 1:
-        rc = lib().kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
-                                 _ptr(cu_seqlens), _ptr(out), _ptr(hT),
-                                 nseq, T, H, dk, dv, dt, _stream(stream))
+        fn = lib().kda_chunk_fwd_noalloc if noalloc else lib().kda_chunk_fwd
+        rc = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
+                _ptr(cu_seqlens), _ptr(out), _ptr(hT), nseq, T, H, dk, dv, dt, _stream(stream))
     else:
         rc = lib().kda_chunk_fwd_grouped(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
                                          _ptr(h0), _ptr(cu_seqlens), _ptr(out), _ptr(hT),
                                          nseq, T, H, dk, dv, G, dt, _stream(stream))
     if rc != KDA_OK:
-        raise KdaError("kda_chunk_fwd", rc)
+        raise KdaError("kda_chunk_fwd_noalloc" if noalloc else "kda_chunk_fwd", rc)
     return out, hT
 
 

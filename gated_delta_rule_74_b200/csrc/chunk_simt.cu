@@ -35,7 +35,9 @@ struct SimtSmem {
   static constexpr int LD = DK + 1;            // padded row stride (bank spread)
   float k[C * LD];
   float q[C * LD];                             // q, later reused for Kend
-  float G[C * LD];                             // cumulative log-decay
+  double G[C * LD];                            // cumulative log-decay (fp64: exponents are
+                                               // differences G_r - G_i, exact to fp32
+                                               // rounding however large |G| grows)
   float E[C * LD];                             // exp(G)
   float A[C * (C + 1)];
   float Aqk[C * (C + 1)];
@@ -102,11 +104,11 @@ kda_chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     __syncthreads();
     // ---- cumulative log-decay along the chunk, one thread per channel
     if (tid < DK) {
-      float acc = 0.f;
+      double acc = 0.0;
       for (int r = 0; r < C; ++r) {
         acc += sm.G[r * LD + tid];
         sm.G[r * LD + tid] = acc;
-        sm.E[r * LD + tid] = expf(acc);
+        sm.E[r * LD + tid] = expf((float)acc);
       }
     }
     __syncthreads();
@@ -118,10 +120,10 @@ kda_chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
         const float* kr = sm.k + r * LD;
         const float* qr = sm.q + r * LD;
         const float* ki = sm.k + i * LD;
-        const float* Gr = sm.G + r * LD;
-        const float* Gi = sm.G + i * LD;
+        const double* Gr = sm.G + r * LD;
+        const double* Gi = sm.G + i * LD;
         for (int c = 0; c < DK; ++c) {
-          const float e = expf(Gr[c] - Gi[c]);
+          const float e = expf((float)(Gr[c] - Gi[c]));
           const float kie = ki[c] * e;
           a = fmaf(kr[c], kie, a);
           aq = fmaf(qr[c], kie, aq);
@@ -172,7 +174,7 @@ kda_chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     //      G of padded rows equals G_{L-1} because their g is 0)
     for (int idx = tid; idx < C * DK; idx += NT) {
       const int r = idx / DK, c = idx % DK;
-      sm.q[r * LD + c] = sm.k[r * LD + c] * expf(sm.G[(C - 1) * LD + c] - sm.G[r * LD + c]);
+      sm.q[r * LD + c] = sm.k[r * LD + c] * expf((float)(sm.G[(C - 1) * LD + c] - sm.G[r * LD + c]));
     }
     __syncthreads();
     // ---- S_next = Diag(exp(G_{L-1})) S + Kend^T D

@@ -37,18 +37,24 @@
 // points so no factor overflows): rows are grouped in 16-token blocks a with
 // P_a = G at row 16a.
 //   i, r in block a:   (k_r e^{G_r - P_a}) (k_i e^{P_a - G_i})
-//       first factor <= 1; second <= e^{decay over <= 15 tokens}, clamped at e^80
-//   i in block b < a:  (k_r e^{G_r - P_a}) (k_i e^{P_b - G_i} e^{P_a - P_b})
+//       first factor <= 1; second <= e^{decay inside the block}
+//   i in block b < a:  (k_r e^{G_r - P_a}) (k_i e^{P_a - G_i}),  e^{P_a - G_i} <= 1
 // so the Gram of row block a is one product against R^(a) = [k_i e^{P_a - G_i}]
-// over i < 16(a+1): two exponentials per element.  Range limit: within one
-// 16-token block the cumulative log-decay must stay above -80 per channel.
-// All four products (A and Aqk rows for all blocks) are one MMA of N = 160:
+// over i < 16(a+1).  All four products (A and Aqk rows for all blocks) are one
+// MMA of N = 160:
 //   [D^(0) .. D^(3)] [128 x 160] = [Lk ; Lq] [R^(0); ..; R^(3)]^T
+// A channel whose decay inside block a exceeds kUnsafeDecay (strong decay, or a
+// gate that closes) has its within-block entries of R^(a) zeroed; those pairs are
+// then added exactly by a CUDA-core pass (decay_pairs.cuh), and its other factors
+// (R^(a') for a' > a, Kend) are formed directly, each <= 1.  Exponents are taken
+// as differences of per-block sums, never of chunk-wide sums, so a closed gate
+// (g -> -1e4) early in the chunk costs no precision later in it.
 #include <cuda_fp16.h>
 
 #include <algorithm>
 #include <type_traits>
 
+#include "decay_pairs.cuh"
 #include "kda_common.cuh"
 #include "segments.cuh"
 #include "sm100.cuh"
@@ -94,6 +100,8 @@ constexpr uint32_t Q_TB = 73728;        // T diag(beta): K-major SW128 B operand
 // record images on their way out (bulk copies): Aqk after the Gram readout,
 // then W^T and U^T over the dead solve scratch once their MMAs are done
 constexpr uint32_t Q_OAQK = 81920, Q_OW = 32768, Q_OU = 49152;
+// corrections of unsafe channels (8 KB, between the Gram readout and the solve)
+constexpr uint32_t Q_CORR = 90112;
 constexpr uint32_t PREP_SMEM = 106496 + 1024;
 constexpr uint32_t PT_G = 0;            // Gram D^(0..3) at +0, +16, +48, +96 (160 columns)
 constexpr uint32_t PT_W = 0;            // W^T [128 x 64] (after the Gram is read)
@@ -140,26 +148,89 @@ __device__ __forceinline__ float h_hi(uint32_t w) {
   return __half2float(__ushort_as_half((unsigned short)(w >> 16)));
 }
 
-// Sum over the warp's 32 lanes of each of 16 per-lane values; lane l returns the
-// total of value l / 2 (transpose-reduce: halves exchanged at lane distance 16,
-// 8, 4, 2, then one butterfly step).
-__device__ __forceinline__ float rowsum16(const float (&v)[16], int lane) {
-  float x8[8], x4[4], x2[2];
-  const bool b16 = lane & 16, b8 = lane & 8, b4 = lane & 4, b2 = lane & 2;
+constexpr float kNormEps2 = 1e-24f;     // (1e-12)^2: L2 norm floor of the fused q/k prep
+
+// Per-row values of one thread's two channels in its 16-row block a: x = G_r - P_a,
+// k and q; per channel d[a2] = P_{a2} - P_a and tl = G_last - P_a.
+struct UnsafeRows {
+  float x[2][16], k[2][16], q[2][16], d[2][4], tl[2];
+};
+
+// Operands of this thread's unsafe channels (bit 0 / 1 of `uns`: c0, c0 + 1): no
+// within-block entries in R^(a); R^(a2), a2 > a, and Kend formed directly as
+// k e^{P_{a2} - G_i} and k e^{G_last - G_i} (exponents <= 0).  With conv, also
+// stages the normalised k, q as bf16 [row][128] in the record's U^T and W^T areas
+// for the exact pair pass (the record's own images overwrite them at the end).
+__device__ __noinline__ void prep_unsafe_direct(uint8_t* sm, uint8_t* rc, int a, int c0, int uns,
+                                                bool conv, const UnsafeRows& ur) {
+#pragma unroll 1
+  for (int ch = 0; ch < 2; ++ch) {
+    if (!((uns >> ch) & 1)) continue;
+    const int c = c0 + ch;
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
-    x8[i] = (b16 ? v[i + 8] : v[i]) + __shfl_xor_sync(0xffffffffu, b16 ? v[i] : v[i + 8], 16);
+    for (int gg = 0; gg < 2; ++gg) {
+      const int g8 = 2 * a + gg;
+      sts16(sm, q_r(a) + chunk_mnmajor_sw32(g8, c, D), make_uint4(0u, 0u, 0u, 0u));
+      float v[8];
+#pragma unroll 1
+      for (int a2 = a + 1; a2 < 4; ++a2) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
-    x4[i] = (b8 ? x8[i + 4] : x8[i]) + __shfl_xor_sync(0xffffffffu, b8 ? x8[i] : x8[i + 4], 8);
+        for (int e = 0; e < 8; ++e)
+          v[e] = ur.k[ch][8 * gg + e] * __expf(fminf(ur.d[ch][a2] - ur.x[ch][8 * gg + e], 0.f));
+        sts16(sm, q_r(a2) + chunk_mnmajor_sw32(g8, c, D), pack8(v, 1.f));
+      }
 #pragma unroll
-  for (int i = 0; i < 2; ++i)
-    x2[i] = (b4 ? x4[i + 2] : x4[i]) + __shfl_xor_sync(0xffffffffu, b4 ? x4[i] : x4[i + 2], 4);
-  float x = (b2 ? x2[1] : x2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? x2[0] : x2[1], 2);
-  return x + __shfl_xor_sync(0xffffffffu, x, 1);
+      for (int e = 0; e < 8; ++e)
+        v[e] = ur.k[ch][8 * gg + e] * __expf(fminf(ur.tl[ch] - ur.x[ch][8 * gg + e], 0.f));
+      *reinterpret_cast<uint4*>(rc + REC_KA + chunk_kmajor_sw128(c, g8, D)) = pack8_f16(v, 1.f);
+      if (conv) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int row = 16 * a + 8 * gg + e;
+          reinterpret_cast<bf16*>(rc + REC_U)[row * D + c] = __float2bfloat16_rn(ur.k[ch][8 * gg + e]);
+          reinterpret_cast<bf16*>(rc + REC_QW + 16384)[row * D + c] =
+              __float2bfloat16_rn(ur.q[ch][8 * gg + e]);
+        }
+      }
+    }
+  }
 }
 
-constexpr float kNormEps2 = 1e-24f;     // (1e-12)^2: L2 norm floor of the fused q/k prep
+// The exact within-block pair terms of this thread's unsafe channels (c0, c0 + 1;
+// flags ux, uy) of one 16-row block, added to the block's corrections (A, Aqk:
+// [r][i], row stride 16).  Warp-cooperative.  Reloads the block's rows: g (one
+// value per channel, or per group of 2^gsh channels; `gst` apart), k and q (bf16
+// channel pairs, `kst` apart); rows >= nrows are not read.  Out of line: it runs
+// only for chunks with unsafe channels and keeps its registers to itself.
+__device__ __noinline__ void prep_unsafe_pairs(const float* __restrict__ g, long long gix,
+                                               long long gst, int gsh, const bf16* kp,
+                                               const bf16* qp, long long kst, int nrows, bool ux,
+                                               bool uy, float* corrA, float* corrQ, int lane) {
+  if (!__any_sync(0xffffffffu, ux || uy)) return;
+  float al[16][2], kv[16][2], qv[16][2];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    float2 gg = make_float2(0.f, 0.f);
+    uint32_t kw = 0u, qw = 0u;
+    if (e < nrows && (ux || uy)) {
+      if (gsh == 0) {
+        gg = *reinterpret_cast<const float2*>(g + gix + e * gst);
+      } else {
+        const float t = g[gix + e * gst];
+        gg = make_float2(t, t);
+      }
+      kw = *reinterpret_cast<const uint32_t*>(kp + e * kst);
+      qw = *reinterpret_cast<const uint32_t*>(qp + e * kst);
+    }
+    al[e][0] = __expf(gg.x);
+    al[e][1] = __expf(gg.y);
+    kv[e][0] = ux ? bf_lo(kw) : 0.f;
+    kv[e][1] = uy ? bf_hi(kw) : 0.f;
+    qv[e][0] = ux ? bf_lo(qw) : 0.f;
+    qv[e][1] = uy ? bf_hi(qw) : 0.f;
+  }
+  add_pair_terms<2, 16>(al, kv, qv, corrA, corrQ, lane);
+}
 
 // ============================================================================
 // Prep kernel: one CTA per (chunk slot, head).  CONV: q and k are the raw
@@ -182,6 +253,9 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   __shared__ float2 s_sum[4][64];       // per 16-row block: its total log-decay (channel pair)
   __shared__ float2 s_first[4][64];     // per 16-row block: g at its first row
   __shared__ float s_ss[CONV ? 4 * 2 * 2 * 16 : 1];   // [block][warp][k|q][row]: sums of squares
+  __shared__ uint8_t s_uns[NT];         // per thread: bit 0 / 1 = channel c0 / c0 + 1 unsafe
+  __shared__ long long s_rbase;
+  __shared__ int s_L;
 
   const int tid = threadIdx.x, warp = tid >> 5;
   const long long slot = blockIdx.x;
@@ -310,8 +384,17 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   }
   s_sum[a][cp] = gq[15];
   s_first[a][cp] = gq[0];
+  // a channel whose decay inside this block is too strong for the reference-point
+  // split: its within-block pairs are added exactly after the Gram (decay_pairs.cuh)
+  const bool ux = c0 < dk && gq[0].x - gq[15].x > kUnsafeDecay;
+  const bool uy = c0 < dk && gq[0].y - gq[15].y > kUnsafeDecay;
+  s_uns[tid] = (uint8_t)((ux ? 1 : 0) | (uy ? 2 : 0));
+  if (tid == 0) {
+    s_rbase = rbase;
+    s_L = L;
+  }
   tc_fence_before();
-  __syncthreads();
+  const bool fix = __syncthreads_or(ux || uy) != 0;
   tc_fence_after();
   const uint32_t tb = tmem_base_sh;
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
@@ -333,34 +416,63 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     }
   }
 
-  float2 Pr[4], Pown = make_float2(0.f, 0.f), off = make_float2(0.f, 0.f),
-               run = make_float2(0.f, 0.f);
+  // Per channel, from per-block sums only: off = P_a - g_{16a} (the blocks before
+  // this one), rel = the decay of blocks a..3, d[a2] = P_{a2} - P_a + g_{16a}.
+  float2 d[4], off = make_float2(0.f, 0.f), rel = make_float2(0.f, 0.f);
 #pragma unroll
   for (int a2 = 0; a2 < 4; ++a2) {
     const float2 f = s_first[a2][cp], sm2 = s_sum[a2][cp];
-    Pr[a2] = make_float2(run.x + f.x, run.y + f.y);
-    if (a2 == a) { off = run; Pown = Pr[a2]; }
-    run.x += sm2.x;
-    run.y += sm2.y;
+    d[a2] = make_float2(rel.x + f.x, rel.y + f.y);
+    if (a2 < a) {
+      off.x += sm2.x;
+      off.y += sm2.y;
+    } else {
+      rel.x += sm2.x;
+      rel.y += sm2.y;
+    }
   }
-  const float2 Glast = run;
+  const float2 fo = gq[0];                     // g at the block's first row
+  auto kval = [&](int idx, int ch) -> float {
+    if constexpr (!CONV) return ch ? bf_hi(kw[idx]) : bf_lo(kw[idx]);
+    else return ch ? kf[idx].y : kf[idx].x;              // normalised above
+  };
+  auto qval = [&](int idx, int ch) -> float {
+    if constexpr (!CONV) return ch ? bf_hi(qw[idx]) : bf_lo(qw[idx]);
+    else return ch ? qf[idx].y : qf[idx].x;
+  };
+
+  if (ux || uy) {
+    // unsafe channels: their operands are formed out of line (the loop below skips
+    // their R and Kend stores); the values go over on the stack, so the common
+    // path's registers are untouched
+    UnsafeRows ur;
 #pragma unroll
-  for (int e = 0; e < 16; ++e) {
-    gq[e].x += off.x;
-    gq[e].y += off.y;
+    for (int ch = 0; ch < 2; ++ch) {
+      const float first = ch ? fo.y : fo.x;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        ur.x[ch][e] = (ch ? gq[e].y : gq[e].x) - first;
+        ur.k[ch][e] = kval(e, ch);
+        ur.q[ch][e] = qval(e, ch);
+      }
+#pragma unroll
+      for (int a2 = 0; a2 < 4; ++a2) ur.d[ch][a2] = (ch ? d[a2].y : d[a2].x) - first;
+      ur.tl[ch] = (ch ? rel.y : rel.x) - first;
+    }
+    prep_unsafe_direct(sm, rc, a, c0, (ux ? 1 : 0) | (uy ? 2 : 0), CONV, ur);
   }
 
 #pragma unroll
   for (int ch = 0; ch < 2; ++ch) {
     const int c = c0 + ch;
-    const float Pa = ch ? Pown.y : Pown.x;
-    const float Gl = ch ? Glast.y : Glast.x;
-    const float eP = __expf(Pa);               // Kbar, Qbar: e^{G_r} = e^{G_r - P_a} e^{P_a}
-    const float eE = __expf(Gl - Pa);          // Kend: e^{G_last - G_i} = e^{P_a - G_i} e^{G_last - P_a}
+    const float first = ch ? fo.y : fo.x;
+    const bool uns = ch ? uy : ux;
+    const float eP = __expf((ch ? off.y : off.x) + first);   // Kbar, Qbar: e^{G_r} = e^{G_r - P_a} e^{P_a}
+    const float eE = __expf((ch ? rel.y : rel.x) - first);   // Kend: e^{G_last - G_i} = e^{P_a - G_i} e^{G_last - P_a}
     float f[4];
 #pragma unroll
     for (int a2 = 0; a2 < 4; ++a2)
-      f[a2] = a2 > a ? __expf((ch ? Pr[a2].y : Pr[a2].x) - Pa) : 1.f;
+      f[a2] = a2 > a ? __expf((ch ? d[a2].y : d[a2].x) - first) : 1.f;   // e^{P_{a2} - P_a}
 #pragma unroll
     for (int gg = 0; gg < 2; ++gg) {
       const int g8 = 2 * a + gg;               // group of 8 rows
@@ -369,17 +481,10 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int idx = 8 * gg + e;
-          const float x = (ch ? gq[idx].y : gq[idx].x) - Pa;
+          const float x = (ch ? gq[idx].y : gq[idx].x) - first;   // G_r - P_a
           const float ell = __expf(x);
           const float rho = __expf(fminf(-x, 80.f));
-          float kv, qv;
-          if constexpr (!CONV) {
-            kv = ch ? bf_hi(kw[idx]) : bf_lo(kw[idx]);
-            qv = ch ? bf_hi(qw[idx]) : bf_lo(qw[idx]);
-          } else {                     // normalised above
-            kv = ch ? kf[idx].y : kf[idx].x;
-            qv = ch ? qf[idx].y : qf[idx].x;
-          }
+          const float kv = kval(idx, ch), qv = qval(idx, ch);
           lk[e] = kv * ell;
           lq[e] = qv * ell;
           kr[e] = kv * rho;                    // k_i e^{P_a - G_i}
@@ -387,9 +492,11 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
         // the Gram operands (its K loop covers channels < dk only)
         sts16(sm, Q_L + chunk_mnmajor_sw128(g8, c, D), pack8(lk, 1.f));
         sts16(sm, Q_L + chunk_mnmajor_sw128(8 + g8, c, D), pack8(lq, 1.f));
+        if (!uns) {
 #pragma unroll
-        for (int a2 = 0; a2 < 4; ++a2)
-          if (a2 >= a) sts16(sm, q_r(a2) + chunk_mnmajor_sw32(g8, c, D), pack8(kr, f[a2]));
+          for (int a2 = 0; a2 < 4; ++a2)
+            if (a2 >= a) sts16(sm, q_r(a2) + chunk_mnmajor_sw32(g8, c, D), pack8(kr, f[a2]));
+        }
       } else {                         // padded channels (dk = 64; whole warps): zeros
 #pragma unroll
         for (int e = 0; e < 8; ++e) lk[e] = lq[e] = kr[e] = 0.f;
@@ -397,12 +504,13 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       sts16(sm, Q_KB + chunk_kmajor_sw128(c, g8, D), pack8(lk, eP));
       // record: Qbar^T (MN-major, N = tokens, K = channels) and Kend^T (K-major)
       *reinterpret_cast<uint4*>(rc + REC_QW + chunk_mnmajor_sw128(g8, c, D)) = pack8(lq, eP);
-      *reinterpret_cast<uint4*>(rc + REC_KA + chunk_kmajor_sw128(c, g8, D)) = pack8_f16(kr, eE);
+      if (!uns)
+        *reinterpret_cast<uint4*>(rc + REC_KA + chunk_kmajor_sw128(c, g8, D)) = pack8_f16(kr, eE);
     }
   }
-  if (a == 3)
+  if (a == 3)                                  // exp(G_last), G_last = off + rel
     *reinterpret_cast<float2*>(rc + REC_DECAY + 4 * c0) =
-        make_float2(__expf(Glast.x), __expf(Glast.y));
+        make_float2(__expf(off.x + rel.x), __expf(off.y + rel.y));
   cp_async_wait_all();
   fence_async_smem();
   tc_fence_before();
@@ -434,6 +542,39 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   __syncwarp();
   if (!mma_wait()) alive = false;
 
+  if (alive && fix) {
+    // exact within-block pairs of the unsafe channels into the corrections (R^(3)'s
+    // area, free once the Gram has completed): A at [block][r][i], Aqk 4 KB above
+    float4* cz = reinterpret_cast<float4*>(sm + Q_CORR);
+    cz[tid] = make_float4(0.f, 0.f, 0.f, 0.f);
+    cz[tid + NT] = make_float4(0.f, 0.f, 0.f, 0.f);
+    __syncthreads();
+    // (rbase, L and the flags come back from shared memory: nothing of this stays
+    // live in registers across the common path)
+    const long long rb = s_rbase;
+    const int u = s_uns[tid];
+    const int ta = tid >> 6, tc0 = 2 * (tid & 63);
+    const int nrows = max(0, min(16, s_L - 16 * ta));
+    const long long gst = (long long)H * (dk >> gsh);
+    const long long gix = ((rb + 16 * ta) * H + h) * (dk >> gsh) + (tc0 >> gsh);
+    const bf16 *kp, *qp;
+    long long kst;
+    if constexpr (CONV) {
+      kp = reinterpret_cast<const bf16*>(rc + REC_U) + 16 * ta * D + tc0;
+      qp = reinterpret_cast<const bf16*>(rc + REC_QW + 16384) + 16 * ta * D + tc0;
+      kst = D;
+    } else {
+      kp = k + ((rb + 16 * ta) * H + h) * dk + tc0;
+      qp = q + ((rb + 16 * ta) * H + h) * dk + tc0;
+      kst = (long long)H * dk;
+    }
+    float* corr = reinterpret_cast<float*>(sm + Q_CORR);
+    prep_unsafe_pairs(g, gix, gst, gsh, kp, qp, kst, nrows, (u & 1) != 0, (u & 2) != 0,
+                      corr + 256 * ta, corr + 1024 + 256 * ta, tid & 31);
+    if constexpr (CONV) fence_async_global();   // the staged rows are overwritten by bulk copies
+    __syncthreads();
+  }
+
   float* B32 = reinterpret_cast<float*>(sm + Q_B32);
   float* T32 = reinterpret_cast<float*>(sm + Q_T32);
   float* M32 = reinterpret_cast<float*>(sm + Q_M32);
@@ -462,6 +603,17 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       }
     }
     tmem_wait_ld();
+    if (fix && mine) {               // the exact within-block pairs of unsafe channels
+      const float* cr = reinterpret_cast<const float*>(sm + Q_CORR) + (isA ? 0 : 1024) +
+                        256 * ab + 16 * (r - 16 * ab);
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4)
+        if (q4 == ab) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            tv[q4][e] = __float_as_uint(__uint_as_float(tv[q4][e]) + cr[e]);
+        }
+    }
     if (mine) {
       if (isA) {
         const float br = s_beta[r];

@@ -19,14 +19,15 @@
 // Decay factoring.  exp(G_r - G_i) is split through reference points so that no
 // factor overflows: rows are grouped in 16-token blocks a; P_a = G at row 16a.
 //   i, r in block a:   (k_r e^{G_r - P_a}) (k_i e^{P_a - G_i})
-//       first factor <= 1; second <= e^{decay over <= 15 tokens}, clamped at e^80
-//   i in block b < a:  (k_r e^{G_r - P_a}) (k_i e^{P_b - G_i} e^{P_a - P_b})
-//       with e^{P_a - G_i} <= 1.
-// So the Gram of row block a is one MMA against R^(a) = [k_i e^{P_a - G_i}]_{i<16(a+1)},
-// and every other operand is one of these factors times a per-(block, channel)
-// constant: two exponentials per element in all.  The only range limit: within
-// one 16-token block the cumulative log-decay must stay above -80 per channel
-// (|g| below about 5 per token on average).
+//       first factor <= 1; second <= e^{decay inside the block}
+//   i in block b < a:  (k_r e^{G_r - P_a}) (k_i e^{P_a - G_i}),  e^{P_a - G_i} <= 1
+// So the Gram of row block a is one MMA against R^(a) = [k_i e^{P_a - G_i}]_{i<16(a+1)}.
+// A channel whose decay inside block a exceeds kUnsafeDecay (strong decay, or a
+// gate that closes) has its within-block entries of R^(a) zeroed; those pairs are
+// added exactly on the CUDA cores (decay_pairs.cuh), and its other factors
+// (R^(a') for a' > a, Kend) are formed directly, each <= 1.  Exponents are taken as
+// differences of per-half sums, so a closed gate (g -> -1e4) in the first half of
+// the chunk costs no precision in the second.
 //
 // Everything is computed transposed so that every MMA has M = 128 (the channel
 // or value index on the TMEM lanes):
@@ -54,6 +55,7 @@
 #include <mutex>
 #include <type_traits>
 
+#include "decay_pairs.cuh"
 #include "kda_common.cuh"
 #include "segments.cuh"
 #include "sm100.cuh"
@@ -158,51 +160,72 @@ __device__ __forceinline__ void prefetch_v(uint8_t* sm, const bf16* v, long long
   }
 }
 
-// Operand build for rows [32*HF, 32*HF + 32) of the chunk, key channel c;
-// gv holds the cumulative log-decay of those rows.
+// Per 16-row block lb of a thread's half (block a = 2 HF + lb), channel c: the
+// reference P_a in the half's local frame (x = gv[r] - ref), e^{P_a}, G_63 - P_a and
+// its exponential, P_{a2} - P_a and its exponential for a2 > a, and whether the
+// block's decay is too strong for the split.
+struct BlockRefs {
+  float ref[2], eP[2], tl[2], eE[2], dd[2][4], f[2][4];
+  bool uns[2];
+};
+
+// Operand build for rows [32*HF, 32*HF + 32) of the chunk, key channel c; gv holds
+// the cumulative log-decay of those rows from the start of the half.
 template <int HF>
 __device__ __forceinline__ void build_half(uint8_t* sm, const float (&gv)[32], const bf16* kc,
-                                           const bf16* qc, int c, float P0, float P1, float P2,
-                                           float P3, float G63, uint32_t tm_kb) {
-  const float P[4] = {P0, P1, P2, P3};
+                                           const bf16* qc, int c, const BlockRefs& br,
+                                           uint32_t tm_kb) {
   uint32_t kbw[16];
 #pragma unroll
   for (int lb = 0; lb < 2; ++lb) {
     const int a = 2 * HF + lb;
-    const float Pa = P[a];
-    const float eP = __expf(Pa);                 // Kbar, Qbar: e^{G_r} = e^{G_r - P_a} e^{P_a}
-    const float eE = __expf(G63 - Pa);           // Kend: e^{G63 - G_i} = e^{P_a - G_i} e^{G63 - P_a}
-    const float f1 = a + 1 <= 3 ? __expf(P[a + 1 <= 3 ? a + 1 : 3] - Pa) : 0.f;
-    const float f2 = a + 2 <= 3 ? __expf(P[a + 2 <= 3 ? a + 2 : 3] - Pa) : 0.f;
-    const float f3 = a + 3 <= 3 ? __expf(P[3] - Pa) : 0.f;
+    const float eP = br.eP[lb];                  // Kbar, Qbar: e^{G_r} = e^{G_r - P_a} e^{P_a}
+    const float eE = br.eE[lb];                  // Kend: e^{G63 - G_i} = e^{P_a - G_i} e^{G63 - P_a}
+    const bool uns = br.uns[lb];
 #pragma unroll
     for (int gg = 0; gg < 2; ++gg) {
       const int g8 = 2 * a + gg;                 // global group of 8 rows
-      float lk[8], lq[8], kr[8];
+      float lk[8], lq[8], kr[8], kv[8], xs[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const int r = g8 * 8 + e;
-        const float x = gv[r - 32 * HF] - Pa;
+        const float x = gv[r - 32 * HF] - br.ref[lb];
         const float ell = __expf(x);
         const float rho = __expf(fminf(-x, 80.f));
-        const float kv = __bfloat162float(kc[r * D]);
+        kv[e] = __bfloat162float(kc[r * D]);
         const float qv = __bfloat162float(qc[r * D]);
-        lk[e] = kv * ell;
+        xs[e] = x;
+        lk[e] = kv[e] * ell;
         lq[e] = qv * ell;
-        kr[e] = kv * rho;                        // k_i e^{P_a - G_i}
+        kr[e] = kv[e] * rho;                     // k_i e^{P_a - G_i}
       }
       // L = [Lk ; Lq]: A operand of the Gram, MN-major SW128 (M = 128, K = channels)
       st_v4f(sm, OFF_L + chunk_mnmajor_sw128(g8, c, D), lk, 1.f);
       st_v4f(sm, OFF_L + chunk_mnmajor_sw128(8 + g8, c, D), lq, 1.f);
       // Qbar^T: B operand of O^T, MN-major SW128 (N = tokens, K = channels)
       st_v4f(sm, OFF_QB + chunk_mnmajor_sw128(g8, c, D), lq, eP);
-      // Kend^T: B operand of the state update, K-major SW128 (N = channels, K = tokens)
-      st_v4h(sm, OFF_KE + chunk_kmajor_sw128(c, g8, D), kr, eE);
-      // R^(a'), a' >= a: B operands of the Gram, MN-major SW32 (N = 16(a'+1), K = channels)
-      st_v4f(sm, off_r(a) + chunk_mnmajor_sw32(g8, c, D), kr, 1.f);
-      if (a + 1 <= 3) st_v4f(sm, off_r(a + 1 <= 3 ? a + 1 : 3) + chunk_mnmajor_sw32(g8, c, D), kr, f1);
-      if (a + 2 <= 3) st_v4f(sm, off_r(a + 2 <= 3 ? a + 2 : 3) + chunk_mnmajor_sw32(g8, c, D), kr, f2);
-      if (a + 3 <= 3) st_v4f(sm, off_r(3) + chunk_mnmajor_sw32(g8, c, D), kr, f3);
+      if (!uns) {
+        // Kend^T: B operand of the state update, K-major SW128 (N = channels, K = tokens)
+        st_v4h(sm, OFF_KE + chunk_kmajor_sw128(c, g8, D), kr, eE);
+        // R^(a'), a' >= a: B operands of the Gram, MN-major SW32 (N = 16(a'+1), K = channels)
+#pragma unroll
+        for (int a2 = a; a2 < 4; ++a2)
+          st_v4f(sm, off_r(a2) + chunk_mnmajor_sw32(g8, c, D), kr, br.f[lb][a2]);
+      } else {
+        // unsafe: no within-block entries; later blocks' factors and Kend directly
+        st_v4(sm, off_r(a) + chunk_mnmajor_sw32(g8, c, D), 0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int a2 = a + 1; a2 < 4; ++a2) {
+          float r2[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) r2[e] = kv[e] * __expf(fminf(br.dd[lb][a2] - xs[e], 0.f));
+          st_v4f(sm, off_r(a2) + chunk_mnmajor_sw32(g8, c, D), r2, 1.f);
+        }
+        float ke[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ke[e] = kv[e] * __expf(fminf(br.tl[lb] - xs[e], 0.f));
+        st_v4h(sm, OFF_KE + chunk_kmajor_sw128(c, g8, D), ke, 1.f);
+      }
       // Kbar^T: A operand in TMEM, lane c, two tokens per 32-bit column
 #pragma unroll
       for (int e = 0; e < 4; ++e)
@@ -225,7 +248,10 @@ kda_chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   __shared__ uint32_t tmem_base_sh;
   __shared__ float s_beta[C];
   __shared__ float s_gamma[D];
-  __shared__ float s_pref[5][D];       // P0, P1, P2, P3, G63 per channel
+  // per channel, each half's local cumulative log-decay at its rows 0, 16, 31
+  __shared__ float s_pref[6][D];
+  // exact within-block pairs of unsafe channels: A at [block][r][i], then Aqk
+  __shared__ __align__(16) float s_corr[2 * 4 * 256];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = blockIdx.x, s = blockIdx.y;
@@ -290,6 +316,9 @@ kda_chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     mbar_init(&bar, 1);
     fence_mbar_init();
   }
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+    reinterpret_cast<float4*>(s_corr)[tid + i * NT] = make_float4(0.f, 0.f, 0.f, 0.f);
   // first chunk's inputs
   float beta_next = 0.f;
   if (t_beg < t_end) {
@@ -354,6 +383,7 @@ kda_chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     __syncthreads();
 
     // ================= P1: decay scan and operand build (all threads) ========
+    bool unsafe_any = false;
     {
       const int c = tid & 127, hf = tid >> 7;
       const float* Gc = reinterpret_cast<const float*>(sm + OFF_SG) + c;   // column c
@@ -362,33 +392,71 @@ kda_chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       for (int r = 0; r < 32; ++r) gv[r] = Gc[(32 * hf + r) * D];
 #pragma unroll
       for (int r = 1; r < 32; ++r) gv[r] += gv[r - 1];
-      if (hf == 0) {
-        s_pref[0][c] = gv[0];
-        s_pref[1][c] = gv[16];
-        s_pref[4][c] = gv[31];                                  // G_31 for the upper half
-      }
+      s_pref[3 * hf][c] = gv[0];
+      s_pref[3 * hf + 1][c] = gv[16];
+      s_pref[3 * hf + 2][c] = gv[31];
       __syncthreads();
-      if (hf == 1) {
-        const float off = s_pref[4][c];
+      // P_a and G_63 from per-half sums: s0 = G_0, s1 = G_16, s2 = G_31 (first half),
+      // s3, s4, s5 = G_32, G_48, G_63 minus G_31 (second half)
+      const float s0 = s_pref[0][c], s1 = s_pref[1][c], s2 = s_pref[2][c];
+      const float s3 = s_pref[3][c], s4 = s_pref[4][c], s5 = s_pref[5][c];
+      if (hf == 1) s_gamma[c] = __expf(s2 + s5);
+      BlockRefs br;
+      {
+        // dP[a][a2] = P_{a2} - P_a (a2 > a), tg[a] = G_63 - P_a, Pabs[a] = P_a
+        const float Pabs[4] = {s0, s1, s2 + s3, s2 + s4};
+        const float ref[4] = {s0, s1, s3, s4};            // P_a in the half's frame
+        const float tg[4] = {(s2 - s0) + s5, (s2 - s1) + s5, s5 - s3, s5 - s4};
+        const float dP[4][4] = {{0.f, s1 - s0, (s2 - s0) + s3, (s2 - s0) + s4},
+                                {0.f, 0.f, (s2 - s1) + s3, (s2 - s1) + s4},
+                                {0.f, 0.f, 0.f, s4 - s3},
+                                {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-        for (int r = 0; r < 32; ++r) gv[r] += off;
-        s_pref[2][c] = gv[0];
-        s_pref[3][c] = gv[16];
-        s_pref[4][c] = gv[31];                                  // G_63
-        s_gamma[c] = __expf(gv[31]);
+        for (int lb = 0; lb < 2; ++lb) {
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            if (hh != hf) continue;
+            const int a = 2 * hh + lb;
+            br.ref[lb] = ref[a];
+            br.eP[lb] = __expf(Pabs[a]);
+            br.tl[lb] = tg[a];
+            br.eE[lb] = __expf(tg[a]);
+#pragma unroll
+            for (int a2 = 0; a2 < 4; ++a2) {
+              br.dd[lb][a2] = dP[a][a2];
+              br.f[lb][a2] = a2 > a ? __expf(dP[a][a2]) : 1.f;
+            }
+            br.uns[lb] = gv[16 * lb] - gv[16 * lb + 15] > kUnsafeDecay;
+          }
+        }
       }
-      __syncthreads();
-      const float P0 = s_pref[0][c], P1 = s_pref[1][c], P2 = s_pref[2][c], P3 = s_pref[3][c];
-      const float G63 = s_pref[4][c];
       const bf16* kc = reinterpret_cast<const bf16*>(sm + OFF_SK) + c;
       const bf16* qc = reinterpret_cast<const bf16*>(sm + OFF_SQ) + c;
-      if (hf == 0) build_half<0>(sm, gv, kc, qc, c, P0, P1, P2, P3, G63, tb + lane_base + TM_KB);
-      else build_half<1>(sm, gv, kc, qc, c, P0, P1, P2, P3, G63, tb + lane_base + TM_KB);
+      if (hf == 0) build_half<0>(sm, gv, kc, qc, c, br, tb + lane_base + TM_KB);
+      else build_half<1>(sm, gv, kc, qc, c, br, tb + lane_base + TM_KB);
+      // exact within-block pairs of the unsafe channels, from the staged rows
+#pragma unroll
+      for (int lb = 0; lb < 2; ++lb) {
+        if (__any_sync(0xffffffffu, br.uns[lb])) {
+          const int a = 2 * hf + lb;
+          float al[16][1], kv[16][1], qv[16][1];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int r = 16 * a + e;
+            const bool u = br.uns[lb];
+            al[e][0] = u ? __expf(Gc[r * D]) : 1.f;
+            kv[e][0] = u ? __bfloat162float(kc[r * D]) : 0.f;
+            qv[e][0] = u ? __bfloat162float(qc[r * D]) : 0.f;
+          }
+          add_pair_terms<1, 16>(al, kv, qv, s_corr + 256 * a, s_corr + 1024 + 256 * a, lane);
+        }
+      }
+      unsafe_any = br.uns[0] || br.uns[1];
       tmem_wait_st();
       fence_async_smem();
     }
     tc_fence_before();
-    __syncthreads();
+    const bool fix = __syncthreads_or(unsafe_any) != 0;
 
     // staging is free: fetch the next chunk's q, k, g (and beta) behind the MMAs
     if (has_next) {
@@ -460,6 +528,18 @@ kda_chunk_tc_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
         }
       }
       tmem_wait_ld();
+      if (fix && mine) {             // the exact within-block pairs of unsafe channels
+        float* cr = s_corr + (isA ? 0 : 1024) + 256 * ab + 16 * (r - 16 * ab);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4)
+          if (q4 == ab) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              tv[q4][e] = __float_as_uint(__uint_as_float(tv[q4][e]) + cr[e]);
+              cr[e] = 0.f;             // cleared for the next chunk
+            }
+          }
+      }
       float vals[64];
 #pragma unroll
       for (int i = 0; i < 64; ++i) vals[i] = __uint_as_float(tv[i >> 4][i & 15]);

@@ -10,7 +10,10 @@
 //     O = Qbar S + Aqk Delta,  S' = Diag(e^Gamma_last) S + Kend^T Delta.
 // One CTA per (n, h), 256 threads.  The chunk-local quantities (16 tokens) are
 // formed on the CUDA cores in fp32, with the decay differences split through token
-// 8 (factors e^(+-(Gamma - Gamma_8)), clamped at e^80); the three products with
+// 8 (factors e^(+-(Gamma - Gamma_8))); a channel whose decay within tokens 0..8 or
+// 8..15 exceeds kUnsafeDecay has that half's growing factor zeroed and the half's
+// pairs added exactly (decay_pairs.cuh), so strong decay and closed gates stay
+// exact.  The three products with
 // the state run on the tensor cores with S^T resident in TMEM:
 //     [O^T | P]   (128 x 32)  = S^T [Qbar ; W]^T          bf16 operands
 //     S^T        (128 x 128) += Delta^T Kend              f16 operands
@@ -22,6 +25,7 @@
 // [128, 160), S^T as bf16 pairs [160, 224), Delta^T as f16 pairs [224, 232).
 #include <cuda_fp16.h>
 
+#include "decay_pairs.cuh"
 #include "kda_common.cuh"
 #include "sm100.cuh"
 
@@ -81,6 +85,8 @@ kda_decode_chunk_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   uint8_t* sm = align1024(smem_raw);
   __shared__ uint64_t mbar, sbar;
   __shared__ uint32_t tmem_base_sh;
+  // exact within-half pairs of unsafe channels (A, Aqk: [r][i], 16 x 16)
+  __shared__ __align__(16) float s_cA[LT * LT], s_cQ[LT * LT];
   float* const F = reinterpret_cast<float*>(sm + M_F);
   float* const Sf = F;                          // S [dk][dv] fp32 staged through the tile region
   float* const fq = F + F_Q * LT * LDF;          // q, later Qbar-ready raw q
@@ -143,6 +149,8 @@ kda_decode_chunk_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     if (tid < LT && tid < L) xb = beta[(n * L + tid) * H + h];
     sA[tid] = 0.f;
     sAqk[tid] = 0.f;
+    s_cA[tid] = 0.f;
+    s_cQ[tid] = 0.f;
   }
   tc_fence_before();
   __syncthreads();
@@ -191,17 +199,32 @@ kda_decode_chunk_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   //      exp(Gamma_last); the Gram factors k e^(G - G_8), k e^(G_8 - G), q e^(G - G_8)
   //      (each e^ clamped at 80); Kbar = k e^G (into the Gamma tile, once both threads
   //      have read g); the Qbar and Kend operand images
+  bool unsafe = false;
   {
     const int c = tid & (D - 1), t0 = 8 * (tid >> 7);
-    float G[LT];
+    float G[LT], al[8][1];
     float acc = 0.f;
 #pragma unroll
     for (int t = 0; t < LT; ++t) {
-      acc += fG[t * LDF + c];
+      const float gt = fG[t * LDF + c];
+      if (t >= t0 && t < t0 + 8) al[t - t0][0] = __expf(gt);   // this thread's half
+      acc += gt;
       G[t] = acc;
     }
     const float gl = acc;
     if (t0 == 0) sGl[c] = __expf(gl);
+    // this half's growing factor: e^(G - G_8) over tokens 0..7, e^(G_8 - G) over 8..15
+    unsafe = (t0 == 0 ? G[0] - G[8] : G[8] - G[15]) > kUnsafeDecay;
+    if (__any_sync(0xffffffffu, unsafe)) {
+      // its pairs exactly (the factors below are zeroed for them)
+      float kv[8][1], qv[8][1];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        kv[e][0] = unsafe ? fk[(t0 + e) * LDF + c] : 0.f;
+        qv[e][0] = unsafe ? fq[(t0 + e) * LDF + c] : 0.f;
+      }
+      add_pair_terms<1, 8>(al, kv, qv, s_cA + t0 * LT + t0, s_cQ + t0 * LT + t0, lane);
+    }
     __syncthreads();
     float qb[8];                          // Qbar of these 8 tokens: one 16-byte chunk
 #pragma unroll
@@ -210,7 +233,11 @@ kda_decode_chunk_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       const float Gt = t0 ? G[8 + i] : G[i];      // register-resident either way
       const float kt = fk[t * LDF + c], qt = fq[t * LDF + c];
       const float dG = Gt - G[8];
-      const float up = __expf(fminf(dG, 80.f)), dn = __expf(fminf(-dG, 80.f));
+      float up = __expf(fminf(dG, 80.f)), dn = __expf(fminf(-dG, 80.f));
+      if (unsafe) {                       // the growing factor of this half: zero
+        if (t0 == 0) up = 0.f;
+        else dn = 0.f;
+      }
       const float eg = __expf(Gt);
       fKP[t * LDF + c] = kt * up;
       fKM[t * LDF + c] = kt * dn;
@@ -251,10 +278,11 @@ kda_decode_chunk_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     }
     const bool isq = (warp >> 1) == 0;
     float* dst = isq ? sAqk : sA;
+    const float* cor = isq ? s_cQ : s_cA;   // exact pairs of unsafe channels (else zero)
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int r = gq + 8 * (e >> 1), i = n0 + 2 * tq + (e & 1);
-      if (isq ? i <= r : i < r) dst[r * LT + i] = acc[e];
+      if (isq ? i <= r : i < r) dst[r * LT + i] = acc[e] + cor[r * LT + i];
     }
   }
   __syncthreads();

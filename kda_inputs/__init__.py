@@ -40,6 +40,7 @@ import torch
 __all__ = [
     "PrefillSpec", "DecodeSpec", "PREFILL_SPECS", "DECODE_SPECS",
     "make_prefill", "make_fused_prefill", "make_decode", "doc_lengths", "spec_by_name",
+    "strong_decay", "STRONG_DECAY_KINDS",
 ]
 
 
@@ -240,3 +241,52 @@ def make_decode(spec: DecodeSpec | str, *, N: Optional[int] = None, H: Optional[
                 g=g.float().contiguous(), beta=beta.float().contiguous(),
                 S0=S0.float().contiguous(), N=N, H=H, dk=dk, dv=dv, steps=steps,
                 dtype=spec.dtype, name=spec.name)
+
+
+STRONG_DECAY_KINDS = ("channels", "spikes", "both")
+
+
+def strong_decay(g: torch.Tensor, kind: str, *, token_dim: int, seed: int = 0) -> torch.Tensor:
+    """A copy of the log-decay ``g`` (float32, key channels on the last axis, tokens on
+    ``token_dim``) with strong and complete-forgetting decay planted in it.
+
+    These are the decay inputs at the edge of any factoring of exp(G_r - G_i)
+    through per-block reference points: a 16-token block whose cumulative log-decay
+    on a channel falls far below -80.
+
+      "channels": key channels 1, 5, dk/2 + 3 and dk - 2 of every head decay by
+                  g ~ U(-6.5, -5.5) at every token (about -96 over 16 tokens);
+      "spikes":   isolated tokens whose gate closes on every channel: g = -20 at
+                  tokens t = 5 (mod 23) and g = -1e4 at t = 11 (mod 37) (alpha = 0
+                  in float32: complete forgetting), plus g = -1e4 on every other
+                  channel at t = 2 (mod 29) -- all of them inside 16-token blocks,
+                  not only at their first rows;
+      "both":     the two together.
+    Where two rules hit one element the later one in this list wins.
+    """
+    if kind not in STRONG_DECAY_KINDS:
+        raise ValueError(kind)
+    out = g.clone()
+    dk = g.shape[-1]
+    nt = g.shape[token_dim]
+    gen = torch.Generator().manual_seed(seed + 104729)
+    tok = torch.arange(nt)
+
+    def at_tokens(mask: torch.Tensor) -> torch.Tensor:
+        # index tuple selecting the tokens in ``mask`` along token_dim
+        idx = [slice(None)] * g.dim()
+        idx[token_dim] = mask.nonzero().flatten()
+        return tuple(idx)
+
+    if kind in ("channels", "both"):
+        chans = sorted({1, 5, dk // 2 + 3, dk - 2})
+        noise = torch.rand(*g.shape[:-1], len(chans), generator=gen)
+        out[..., chans] = -6.5 + noise
+    if kind in ("spikes", "both"):
+        out[at_tokens(tok % 23 == 5)] = -20.0
+        out[at_tokens(tok % 37 == 11)] = -1.0e4
+        sel = list(at_tokens(tok % 29 == 2))
+        sub = out[tuple(sel)]
+        sub[..., 0::2] = -1.0e4
+        out[tuple(sel)] = sub
+    return out.contiguous()

@@ -1,0 +1,187 @@
+"""Strong and complete-forgetting decay on every prefill and decode path, against
+the float64 oracle.
+
+The tensor-core paths factor exp(G_r - G_i) through per-block reference points.
+A 16-token block whose cumulative log-decay on a channel falls far below -80 is
+the edge of that factoring: per-token g about -6 on a few channels throughout,
+or one token whose gate closes (g = -20, g = -1e4: complete forgetting).  Such
+inputs are real -- a closed gate forgets everything (miniKimiK3 model card, the
+per-channel gated decay of the "Kimi Delta Attention" bullet) -- so every path
+must match the oracle on them within the bf16 bound, with every value finite."""
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_74_b200 as kda
+import kda_inputs as ki
+import oracle
+from _helpers import TOL, rel_err, to_dev
+
+pytestmark = pytest.mark.gpu
+
+KINDS = list(ki.STRONG_DECAY_KINDS)
+
+
+def _strong(x: dict, kind: str, seed: int = 0) -> dict:
+    y = dict(x)
+    y["g"] = ki.strong_decay(x["g"], kind, token_dim=1, seed=seed)
+    return y
+
+
+def _check(x, out, hT, heads=None):
+    assert torch.isfinite(out.float()).all() and torch.isfinite(hT).all()
+    o_ref, s_ref = oracle.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], x["h0"],
+                                  x["cu_seqlens"], heads=heads)
+    if heads is not None:
+        out, hT = out[:, :, heads[0]:heads[1]], hT[:, heads[0]:heads[1]]
+    tol = TOL[x["dtype"]]
+    eo, es = rel_err(out, o_ref), rel_err(hT, s_ref)
+    assert eo <= tol and es <= tol, (x.get("name"), eo, es)
+
+
+def _run(x, **kw):
+    d = to_dev(x)
+    out, hT = kda.kda_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], h0=d["h0"],
+                                cu_seqlens=d["cu_seqlens"], **kw)
+    torch.cuda.synchronize()
+    return out, hT
+
+
+def _spec(dtype="bf16", dk=128, dv=128, B=2, T=300, H=3, seed=5, varlen=False):
+    return ki.PrefillSpec("strong", B=B, T=T, H=H, dk=dk, dv=dv, dtype=dtype, decay="alog",
+                          seed=seed, h0=True, varlen=varlen)
+
+
+@pytest.mark.parametrize("kind", KINDS)
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 64), (128, 64), (64, 128)])
+def test_split_prefill(kind, dk, dv):
+    x = _strong(ki.make_prefill(_spec(dk=dk, dv=dv)), kind)
+    _check(x, *_run(x))
+
+
+@pytest.mark.parametrize("kind", KINDS)
+def test_split_prefill_segmented(kind):
+    """Few (sequence, head) pairs: the sequence is cut into segments whose states
+    are chained afterwards (with half points)."""
+    G, half = kda.kda_prefill_plan(1, 4000, 2)
+    assert G > 0 and half > 0
+    x = _strong(ki.make_prefill(_spec(B=1, T=4000, H=2, seed=6)), kind)
+    _check(x, *_run(x))
+
+
+@pytest.mark.parametrize("kind", KINDS)
+def test_packed_documents(kind):
+    spec = _spec(varlen=True, seed=7)
+    x = _strong(ki.make_prefill(spec, doc_lens=[130, 2, 0, 65, 300, 17]), kind)
+    _check(x, *_run(x))
+
+
+@pytest.mark.parametrize("kind", KINDS)
+def test_fp32_prefill(kind):
+    x = _strong(ki.make_prefill(_spec(dtype="f32", dk=64, dv=64, T=200)), kind)
+    _check(x, *_run(x))
+
+
+@pytest.mark.parametrize("kind", KINDS)
+@pytest.mark.parametrize("shape", ["fixed", "segmented", "packed"])
+def test_noalloc(kind, shape):
+    if shape == "fixed":
+        x = ki.make_prefill(_spec(seed=8))
+    elif shape == "segmented":
+        x = ki.make_prefill(_spec(B=1, T=3000, H=2, seed=9))
+    else:
+        x = ki.make_prefill(_spec(varlen=True, seed=10), doc_lens=[700, 3, 250])
+    x = _strong(x, kind)
+    _check(x, *_run(x, noalloc=True))
+
+
+def test_grouped_decay():
+    """One decay per group of 64 key channels: group 0 at g about -6 throughout,
+    closed gates (g = -1e4) on every group at a few tokens."""
+    x = ki.make_prefill(_spec(seed=11))
+    gc = x["g"].view(*x["g"].shape[:-1], 2, 64)[..., 0].contiguous()   # [B, T, H, 2]
+    gc = ki.strong_decay(gc, "spikes", token_dim=1, seed=11)
+    gc[..., 0] = torch.minimum(gc[..., 0], torch.full_like(gc[..., 0], -6.0))
+    d = to_dev(x)
+    out, hT = kda.kda_chunk_fwd(d["q"], d["k"], d["v"], gc.cuda(), d["beta"], h0=d["h0"])
+    torch.cuda.synchronize()
+    y = dict(x)
+    y["g"] = gc.repeat_interleave(64, dim=-1).contiguous()
+    _check(y, out, hT)
+
+
+@pytest.mark.parametrize("kind", KINDS)
+def test_fused_prep(kind):
+    spec = _spec(seed=12)
+    x = ki.make_fused_prefill(spec, W=4, gate=True)
+    x["g"] = ki.strong_decay(x["g"], kind, token_dim=1, seed=12)
+    d = to_dev(x)
+    out, hT = kda.kda_chunk_fwd_fused(d["q_raw"], d["k_raw"], d["v"], d["g"], d["beta"],
+                                      conv_q=d["conv_q"], conv_k=d["conv_k"], gate=d["gate"],
+                                      h0=d["h0"])
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all() and torch.isfinite(hT).all()
+    o_ref, s_ref = oracle.prefill_fused(x["q_raw"], x["k_raw"], x["v"], x["g"], x["beta"],
+                                        x["conv_q"], x["conv_k"], x["gate"], x["h0"], None)
+    assert rel_err(out, o_ref) <= TOL["bf16"]
+    assert rel_err(hT, s_ref) <= TOL["bf16"]
+
+
+def _decode_inputs(kind, N=3, H=4, L=16, seed=13):
+    d = ki.make_decode(ki.DecodeSpec("c", N=N, H=H, dk=128, dv=128, steps=L, dtype="bf16",
+                                     decay="alog", seed=seed))
+    d["g"] = ki.strong_decay(d["g"], kind, token_dim=0, seed=seed)
+    x = {n: d[n].transpose(0, 1).contiguous() for n in ("q", "k", "v", "g", "beta")}
+    return d, x
+
+
+@pytest.mark.parametrize("kind", KINDS)
+@pytest.mark.parametrize("L", [12, 16])
+def test_decode_chunk(kind, L):
+    d, x = _decode_inputs(kind, L=L)
+    S = d["S0"].cuda()
+    out = kda.kda_decode_chunk(*(x[n].cuda() for n in ("q", "k", "v", "g", "beta")), S)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all() and torch.isfinite(S).all()
+    o_ref, s_ref = oracle.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], d["S0"])
+    assert rel_err(out, o_ref) <= TOL["bf16"]
+    assert rel_err(S, s_ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("kind", KINDS)
+def test_decode_tokens_and_steps(kind):
+    d, x = _decode_inputs(kind, L=16, seed=14)
+    S = d["S0"].cuda()
+    out = kda.kda_decode_tokens(*(x[n].cuda() for n in ("q", "k", "v", "g", "beta")), S)
+    torch.cuda.synchronize()
+    o_ref, s_ref = oracle.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], d["S0"])
+    assert rel_err(out, o_ref) <= TOL["bf16"]
+    assert rel_err(S, s_ref) <= TOL["bf16"]
+    S2 = d["S0"].cuda()
+    outs = []
+    for t in range(16):
+        outs.append(kda.kda_decode_step(*(d[n][t].cuda() for n in ("q", "k", "v", "g", "beta")),
+                                        S2))
+    torch.cuda.synchronize()
+    o2 = torch.stack(outs, 1)
+    assert rel_err(o2, o_ref) <= TOL["bf16"]
+    assert rel_err(S2, s_ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("kind", ["spikes", "both"])
+def test_backward(kind):
+    """The backward's gradients with closed gates, against the oracle's float64
+    backward (bound 1e-4: the backward runs in fp32)."""
+    x = _strong(ki.make_prefill(_spec(B=1, T=200, H=2, seed=15)), kind)
+    gen = torch.Generator().manual_seed(15)
+    dout = torch.randn(x["v"].shape, generator=gen).to(x["v"].dtype)
+    dhT = torch.randn(x["h0"].shape, generator=gen) * 0.1
+    d = to_dev(x)
+    grads = kda.kda_chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], dout.cuda(),
+                              h0=d["h0"], dhT=dhT.cuda())
+    torch.cuda.synchronize()
+    ref = oracle.backward(x["q"], x["k"], x["v"], x["g"], x["beta"], dout, x["h0"], dhT)
+    for name in ("dq", "dk", "dv", "dg", "dbeta", "dh0"):
+        got = grads[name]
+        assert torch.isfinite(got).all(), name
+        assert rel_err(got, ref[name]) <= 1e-4, name
