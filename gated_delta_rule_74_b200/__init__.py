@@ -24,7 +24,8 @@ __all__ = ["kda_chunk_fwd", "kda_chunk_fwd_fused", "kda_chunk_bwd", "kda_device_
            "kda_launch_count",
            "lib", "library_path", "header_symbols", "KdaError",
            "KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED", "KDA_ERR_CUDA",
-           "KDA_ERR_TIMEOUT", "KDA_BF16", "KDA_F32"]
+           "KDA_ERR_TIMEOUT", "KDA_BF16", "KDA_F32", "KDA_OP_CHUNK_FWD", "KDA_OP_CHUNK_BWD",
+           "kda_workspace_size", "kda_pool_usage"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _ROOT = os.path.dirname(_PKG)
@@ -33,6 +34,7 @@ _HEADER = os.path.join(_ROOT, "include", "kda.h")
 
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = 0, -1, -2, -3, -4
 KDA_BF16, KDA_F32 = 0, 1
+KDA_OP_CHUNK_FWD, KDA_OP_CHUNK_BWD = 0, 1
 
 _DTYPES = {torch.bfloat16: KDA_BF16, torch.float32: KDA_F32}
 _lib = None
@@ -106,6 +108,16 @@ def lib() -> ctypes.CDLL:
         L.kda_timing_read.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_ulonglong),
                                       ctypes.POINTER(ctypes.c_double)]
         L.kda_timing_read.restype = ctypes.c_int
+        sz = ctypes.c_size_t
+        L.kda_workspace_size.argtypes = [ctypes.c_int] * 9 + [ctypes.POINTER(sz)]
+        L.kda_workspace_size.restype = ctypes.c_int
+        L.kda_chunk_fwd_ws.argtypes = [vp, vp, vp, fp, fp, fp, vp, vp, fp] + [ip] * 7 + [vp, sz, vp]
+        L.kda_chunk_fwd_ws.restype = ctypes.c_int
+        L.kda_chunk_bwd_ws.argtypes = [vp, vp, vp, fp, fp, fp, vp, vp, fp,
+                                       fp, fp, fp, fp, fp, fp] + [ip] * 7 + [vp, sz, vp]
+        L.kda_chunk_bwd_ws.restype = ctypes.c_int
+        L.kda_pool_usage.argtypes = [ip, ctypes.POINTER(ctypes.c_ulonglong)]
+        L.kda_pool_usage.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -115,6 +127,35 @@ def header_symbols() -> list[str]:
     with open(_HEADER) as f:
         text = f.read()
     return re.findall(r"^KDA_API\s+[\w\s\*]*?\b(kda_\w+)\s*\(", text, flags=re.M)
+
+
+def kda_workspace_size(op: int, B: int, T: int, H: int, dk: int, dv: int, packed: bool = False,
+                       dtype: int = KDA_BF16, sms: int = 0) -> int:
+    """Workspace bytes of one kda_chunk_fwd_ws (op KDA_OP_CHUNK_FWD) or kda_chunk_bwd_ws
+    (KDA_OP_CHUNK_BWD) call; sms = 0 asks the current device."""
+    out = ctypes.c_size_t(0)
+    rc = lib().kda_workspace_size(int(op), int(B), int(T), int(H), int(dk), int(dv),
+                                  1 if packed else 0, int(dtype), int(sms), ctypes.byref(out))
+    if rc != KDA_OK:
+        raise KdaError("kda_workspace_size", rc)
+    return int(out.value)
+
+
+def kda_pool_usage(reset: bool = False) -> int:
+    """Most bytes the library pool of the current device has had in use at once."""
+    out = ctypes.c_ulonglong(0)
+    rc = lib().kda_pool_usage(1 if reset else 0, ctypes.byref(out))
+    if rc != KDA_OK:
+        raise KdaError("kda_pool_usage", rc)
+    return int(out.value)
+
+
+def _workspace_args(workspace: Optional[torch.Tensor]):
+    if workspace is None:
+        return None, 0
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    return _ptr(workspace), workspace.numel() * workspace.element_size()
 
 
 def kda_status_string(status: int) -> str:
@@ -214,13 +255,14 @@ def kda_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Te
                   beta: torch.Tensor, h0: Optional[torch.Tensor] = None,
                   cu_seqlens: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
                   hT: Optional[torch.Tensor] = None, output_final_state: bool = True,
-                  stream=None, noalloc: bool = False):
+                  stream=None, noalloc: bool = False, workspace: Optional[torch.Tensor] = None):
     """KDA prefill (chunked form).  q, k [B,T,H,dk]; v [B,T,H,dv]; g [B,T,H,dk] f32
     (or [B,T,H,dk/G] for one decay per group of G key channels, G a power of two:
     kda_chunk_fwd_grouped); beta [B,T,H] f32; h0 [Nseq,H,dk,dv] f32 or None;
     cu_seqlens int32 [Nseq+1] on the device, or None.  Returns (out, hT) (hT None
     if output_final_state is False and no hT buffer was given).  noalloc=True calls
-    kda_chunk_fwd_noalloc instead (per-channel decay only)."""
+    kda_chunk_fwd_noalloc instead (per-channel decay only); a ``workspace`` tensor
+    (kda_workspace_size bytes, e.g. torch.uint8) calls kda_chunk_fwd_ws on it."""
     if q.dim() != 4:
         raise ValueError("q must be [B, T, H, dk]")
     Bt, T, H, dk = q.shape
@@ -252,6 +294,14 @@ def kda_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Te
         _check("hT", hT, torch.float32, (nseq, H, dk, dv))
     if noalloc and G != 1:
         raise ValueError("kda_chunk_fwd_noalloc takes one decay per key channel")
+    if workspace is not None:
+        wp, wb = _workspace_args(workspace)
+        rc = lib().kda_chunk_fwd_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
+                                    _ptr(cu_seqlens), _ptr(out), _ptr(hT), nseq, T, H, dk, dv, G,
+                                    dt, wp, wb, _stream(stream))
+        if rc != KDA_OK:
+            raise KdaError("kda_chunk_fwd_ws", rc)
+        return out, hT
     if G == 1:
         fn = lib().kda_chunk_fwd_noalloc if noalloc else lib().kda_chunk_fwd
         rc = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
@@ -326,12 +376,14 @@ def kda_chunk_fwd_fused(q_raw: torch.Tensor, k_raw: torch.Tensor, v: torch.Tenso
 def kda_chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
                   beta: torch.Tensor, dout: torch.Tensor, h0: Optional[torch.Tensor] = None,
                   dhT: Optional[torch.Tensor] = None, cu_seqlens: Optional[torch.Tensor] = None,
-                  grads: Optional[dict] = None, stream=None) -> dict:
+                  grads: Optional[dict] = None, stream=None,
+                  workspace: Optional[torch.Tensor] = None) -> dict:
     """Gradients of L = sum(out * dout) + sum(hT * dhT) for kda_chunk_fwd with the same
     inputs.  g [B,T,H,dk] f32, or [B,T,H,dk/G] for one decay per group of G key channels
     (kda_chunk_bwd_grouped; dg then has g's shape).  dout has out's shape and dtype; dhT
     [Nseq,H,dk,dv] f32 or None.  Returns a dict of fp32 tensors dq, dk, dv, dg, dbeta, dh0
-    (dh0 None when h0 is None); ``grads`` may hold preallocated outputs under those names."""
+    (dh0 None when h0 is None); ``grads`` may hold preallocated outputs under those names;
+    a ``workspace`` tensor (kda_workspace_size bytes) calls kda_chunk_bwd_ws on it."""
     if q.dim() != 4:
         raise ValueError("q must be [B, T, H, dk]")
     Bt, T, H, dk = q.shape
@@ -370,6 +422,12 @@ def kda_chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Te
     args = [_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0), _ptr(cu_seqlens),
             _ptr(dout), _ptr(dhT), _ptr(res["dq"]), _ptr(res["dk"]), _ptr(res["dv"]),
             _ptr(res["dg"]), _ptr(res["dbeta"]), _ptr(res["dh0"]), nseq, T, H, dk, dv]
+    if workspace is not None:
+        wp, wb = _workspace_args(workspace)
+        rc = lib().kda_chunk_bwd_ws(*args, G, dt, wp, wb, _stream(stream))
+        if rc != KDA_OK:
+            raise KdaError("kda_chunk_bwd_ws", rc)
+        return res
     if G == 1:
         rc = lib().kda_chunk_bwd(*args, dt, _stream(stream))
     else:

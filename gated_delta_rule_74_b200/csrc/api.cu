@@ -45,10 +45,22 @@ int group_shift(int g_group, int dk) {
   return sh;
 }
 
+bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+
+// SM count of the current device (no allocation, no pool).
+bool current_sms(int* sms) { return kda::device_ctx(sms, nullptr); }
+
+// A caller workspace that is 256-byte aligned and holds `need` bytes (a NULL or
+// empty workspace is fine when nothing is needed).
+bool workspace_ok(const kda::Workspace* ws, size_t need) {
+  if (need == 0) return ws->ptr == nullptr || aligned256(ws->ptr);
+  return ws->ptr != nullptr && aligned256(ws->ptr) && ws->bytes >= need;
+}
+
 int chunk_fwd_impl(const void* q, const void* k, const void* v, const float* g,
                    const float* beta, const float* h0, const int32_t* cu_seqlens, void* out,
                    float* hT, int B, int T, int H, int dk, int dv, int gsh, int in_dtype,
-                   void* stream) {
+                   void* stream, const kda::Workspace* ws = nullptr) {
   if (B < 1 || T < 0 || H < 1) return KDA_ERR_INVALID_ARG;
   if (in_dtype != KDA_BF16 && in_dtype != KDA_F32) return KDA_ERR_INVALID_ARG;
   const long long rows = cu_seqlens ? (long long)T : (long long)B * T;
@@ -64,9 +76,17 @@ int chunk_fwd_impl(const void* q, const void* k, const void* v, const float* g,
   if (rows * H * (long long)(dk > dv ? dk : dv) > (1LL << 40)) return KDA_ERR_INVALID_ARG;
   if ((long long)B > 65535LL || H > 65535) return KDA_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (kda::chunk_split_supported(dk, dv, in_dtype))
+  if (kda::chunk_split_supported(dk, dv, in_dtype)) {
+    if (ws) {
+      int sms = 0;
+      if (!current_sms(&sms)) return KDA_ERR_CUDA;
+      if (!workspace_ok(ws, kda::chunk_split_scratch_bytes(B, T, H, cu_seqlens != nullptr, sms)))
+        return KDA_ERR_INVALID_ARG;
+    }
     return status_from(kda::launch_chunk_split(q, k, v, g, beta, h0, cu_seqlens, out, hT, B, T,
-                                               H, dk, dv, gsh, st));
+                                               H, dk, dv, gsh, st, nullptr, ws));
+  }
+  if (ws && !workspace_ok(ws, 0)) return KDA_ERR_INVALID_ARG;
   return status_from(kda::launch_chunk_simt(q, k, v, g, beta, h0, cu_seqlens, out, hT, B, T,
                                             H, dk, dv, in_dtype, gsh, st));
 }
@@ -178,7 +198,7 @@ int chunk_bwd_impl(const void* q, const void* k, const void* v, const float* g,
                    const float* beta, const float* h0, const int32_t* cu_seqlens,
                    const void* dout, const float* dhT, float* dq, float* dk, float* dv, float* dg,
                    float* dbeta, float* dh0, int B, int T, int H, int dk_dim, int dv_dim, int gsh,
-                   int in_dtype, void* stream) {
+                   int in_dtype, void* stream, const kda::Workspace* ws = nullptr) {
   if (gsh < 0) return KDA_ERR_INVALID_ARG;
   if (B < 1 || T < 0 || H < 1) return KDA_ERR_INVALID_ARG;
   if (in_dtype != KDA_BF16 && in_dtype != KDA_F32) return KDA_ERR_INVALID_ARG;
@@ -195,10 +215,13 @@ int chunk_bwd_impl(const void* q, const void* k, const void* v, const float* g,
   if (rows * H * (long long)(dk_dim > dv_dim ? dk_dim : dv_dim) > (1LL << 40))
     return KDA_ERR_INVALID_ARG;
   if ((long long)B > 65535LL || H > 0x7fffffff) return KDA_ERR_UNSUPPORTED;
+  if (ws && !workspace_ok(ws, kda::chunk_bwd_scratch_bytes(B, T, H, dk_dim, dv_dim,
+                                                            cu_seqlens != nullptr)))
+    return KDA_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return status_from(kda::launch_chunk_bwd(q, k, v, g, beta, h0, cu_seqlens, dout, dhT, dq, dk,
                                            dv, dg, dbeta, dh0, B, T, H, dk_dim, dv_dim, gsh,
-                                           in_dtype, st));
+                                           in_dtype, st, ws));
 }
 }  // namespace
 
@@ -218,6 +241,51 @@ int kda_chunk_bwd_grouped(const void* q, const void* k, const void* v, const flo
                           int dv_dim, int g_group, int in_dtype, void* stream) {
   return chunk_bwd_impl(q, k, v, g, beta, h0, cu_seqlens, dout, dhT, dq, dk, dv, dg, dbeta, dh0,
                         B, T, H, dk_dim, dv_dim, group_shift(g_group, dk_dim), in_dtype, stream);
+}
+
+int kda_workspace_size(int op, int B, int T, int H, int dk, int dv, int packed, int in_dtype,
+                       int sms, size_t* bytes) {
+  if (!bytes || B < 1 || T < 0 || H < 1 || sms < 0) return KDA_ERR_INVALID_ARG;
+  if (op != KDA_OP_CHUNK_FWD && op != KDA_OP_CHUNK_BWD) return KDA_ERR_INVALID_ARG;
+  if (in_dtype != KDA_BF16 && in_dtype != KDA_F32) return KDA_ERR_INVALID_ARG;
+  if (!head_ok(dk) || !head_ok(dv)) return KDA_ERR_UNSUPPORTED;
+  if (op == KDA_OP_CHUNK_BWD) {
+    *bytes = kda::chunk_bwd_scratch_bytes(B, T, H, dk, dv, packed != 0);
+    return KDA_OK;
+  }
+  if (!kda::chunk_split_supported(dk, dv, in_dtype)) {
+    *bytes = 0;                                     // the fp32 path keeps everything on chip
+    return KDA_OK;
+  }
+  if (sms == 0 && !current_sms(&sms)) return KDA_ERR_CUDA;
+  *bytes = kda::chunk_split_scratch_bytes(B, T, H, packed != 0, sms);
+  return KDA_OK;
+}
+
+int kda_chunk_fwd_ws(const void* q, const void* k, const void* v, const float* g,
+                     const float* beta, const float* h0, const int32_t* cu_seqlens, void* out,
+                     float* hT, int B, int T, int H, int dk, int dv, int g_group, int in_dtype,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  const kda::Workspace ws{workspace, workspace_bytes};
+  return chunk_fwd_impl(q, k, v, g, beta, h0, cu_seqlens, out, hT, B, T, H, dk, dv,
+                        group_shift(g_group, dk), in_dtype, stream, &ws);
+}
+
+int kda_chunk_bwd_ws(const void* q, const void* k, const void* v, const float* g,
+                     const float* beta, const float* h0, const int32_t* cu_seqlens,
+                     const void* dout, const float* dhT, float* dq, float* dk, float* dv,
+                     float* dg, float* dbeta, float* dh0, int B, int T, int H, int dk_dim,
+                     int dv_dim, int g_group, int in_dtype, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+  const kda::Workspace ws{workspace, workspace_bytes};
+  return chunk_bwd_impl(q, k, v, g, beta, h0, cu_seqlens, dout, dhT, dq, dk, dv, dg, dbeta, dh0,
+                        B, T, H, dk_dim, dv_dim, group_shift(g_group, dk_dim), in_dtype, stream,
+                        &ws);
+}
+
+int kda_pool_usage(int reset, unsigned long long* used_high_bytes) {
+  if (!used_high_bytes) return KDA_ERR_INVALID_ARG;
+  return kda::pool_used_high(reset != 0, used_high_bytes);
 }
 
 int kda_device_status(int reset) {

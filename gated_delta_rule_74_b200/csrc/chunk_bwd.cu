@@ -554,15 +554,26 @@ cudaError_t launch_dtype(const void* q, const void* k, const void* v, const floa
 
 }  // namespace
 
+// Checkpoints: one state per chunk of every sequence, per head; and the pre-token
+// states of one chunk per (sequence, head).
+size_t chunk_bwd_scratch_bytes(int B, int T, int H, int dk, int dv, bool varlen) {
+  const size_t nck = (size_t)(chunk_slots(B, T, varlen) + B) * H;
+  const size_t ncs = (size_t)B * H * kChunk;
+  return (nck + ncs) * (size_t)dk * dv * sizeof(float);
+}
+
 cudaError_t launch_chunk_bwd(const void* q, const void* k, const void* v, const float* g,
                              const float* beta, const float* h0, const int32_t* cu_seqlens,
                              const void* dout, const float* dhT, float* dq, float* dkk,
                              float* dvv, float* dg, float* dbeta, float* dh0, int B, int T, int H,
-                             int dk, int dv, int gsh, int in_dtype, cudaStream_t stream) {
+                             int dk, int dv, int gsh, int in_dtype, cudaStream_t stream,
+                             const Workspace* ws) {
   int sms = 148;
   cudaMemPool_t pool = nullptr;
-  if (!device_ctx(&sms, &pool)) return cudaErrorInvalidDevice;
-  if (!pool) return cudaErrorMemoryAllocation;
+  if (!device_ctx(&sms, ws ? nullptr : &pool)) return cudaErrorInvalidDevice;
+  if (!ws && !pool) return cudaErrorMemoryAllocation;
+  const size_t need = chunk_bwd_scratch_bytes(B, T, H, dk, dv, cu_seqlens != nullptr);
+  if (ws && (!ws->ptr || ws->bytes < need)) return cudaErrorInvalidValue;
   // dq, dk, dg and dbeta are sums of per-warp parts
   const size_t rows = cu_seqlens ? (size_t)T : (size_t)B * T;
   cudaError_t e = cudaSuccess;
@@ -575,13 +586,12 @@ cudaError_t launch_chunk_bwd(const void* q, const void* k, const void* v, const 
       return e;
   }
   const size_t sz = (size_t)dk * dv;
-  // checkpoints: one state per chunk of every sequence, per head; the pre-token
-  // states of one chunk per (sequence, head)
   const size_t nck = (size_t)(chunk_slots(B, T, cu_seqlens != nullptr) + B) * H;
-  const size_t ncs = (size_t)B * H * kChunk;
-  void* scratch = nullptr;
-  e = cudaMallocFromPoolAsync(&scratch, (nck + ncs) * sz * sizeof(float), pool, stream);
-  if (e != cudaSuccess) return e;
+  void* scratch = ws ? ws->ptr : nullptr;
+  if (!ws) {
+    e = cudaMallocFromPoolAsync(&scratch, need, pool, stream);
+    if (e != cudaSuccess) return e;
+  }
   float* ckpt = static_cast<float*>(scratch);
   float* cst = ckpt + nck * sz;
   if (in_dtype == KDA_BF16)
@@ -590,7 +600,7 @@ cudaError_t launch_chunk_bwd(const void* q, const void* k, const void* v, const 
   else
     e = launch_dtype<float>(q, k, v, g, beta, h0, cu_seqlens, dout, dhT, dq, dkk, dvv, dg, dbeta,
                             dh0, ckpt, cst, B, T, H, dk, dv, gsh, stream);
-  cudaFreeAsync(scratch, stream);
+  if (!ws) cudaFreeAsync(scratch, stream);
   return e;
 }
 

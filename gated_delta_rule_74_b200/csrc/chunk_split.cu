@@ -1339,22 +1339,16 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
 
 // Dynamic shared memory of the kernels, set once per device.
 bool set_attrs() {
-  static bool done[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
-  if (!done[dev]) {
-    if (cudaFuncSetAttribute(kda_chunk_prep_kernel<false>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, PREP_SMEM) != cudaSuccess ||
-        cudaFuncSetAttribute(kda_chunk_prep_kernel<true>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, PREP_SMEM) != cudaSuccess ||
-        cudaFuncSetAttribute(kda_state_pass_kernel<false>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, STATE_SMEM) != cudaSuccess ||
-        cudaFuncSetAttribute(kda_state_pass_kernel<true>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, STATE_SMEM) != cudaSuccess)
-      return false;
-    done[dev] = true;
-  }
-  return true;
+  return once_per_device(kOnceSplit, []() {
+    return cudaFuncSetAttribute(kda_chunk_prep_kernel<false>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, PREP_SMEM) == cudaSuccess &&
+           cudaFuncSetAttribute(kda_chunk_prep_kernel<true>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, PREP_SMEM) == cudaSuccess &&
+           cudaFuncSetAttribute(kda_state_pass_kernel<false>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, STATE_SMEM) == cudaSuccess &&
+           cudaFuncSetAttribute(kda_state_pass_kernel<true>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, STATE_SMEM) == cudaSuccess;
+  });
 }
 
 // Chunks per segment (G = 0: no split) and the half point of pass C (0: none).
@@ -1406,14 +1400,46 @@ void chunk_split_plan(int B, int T, int H, bool varlen, int sms, int* G, int* ha
   *half = p.half;
 }
 
+namespace {
+// Chunk records (nslots per head) and, when sequences are split, the segment
+// states: the one layout both the size query and the launcher use.
+struct SplitScratch {
+  long long nslots;
+  size_t rec_bytes, seg_bytes;
+  SplitPlan plan;
+  int P;
+  long long slots;
+};
+SplitScratch split_scratch(int B, int T, int H, bool varlen, int sms) {
+  SplitScratch r{};
+  r.nslots = chunk_slots(B, T, varlen);
+  r.rec_bytes = (size_t)r.nslots * H * REC_BYTES;
+  r.plan = plan_split(B, T, H, varlen, sms);
+  const long long nch_all = ((long long)T + C - 1) / C;
+  if (r.plan.G > 0 && (nch_all + r.plan.G - 1) / r.plan.G >= 2) {
+    r.P = (int)((nch_all + r.plan.G - 1) / r.plan.G);
+    r.slots = varlen ? (long long)r.P + B : (long long)B * r.P;
+    r.seg_bytes = (size_t)(r.plan.half > 0 ? 4 : 2) * r.slots * H * D * D * sizeof(float);
+  }
+  return r;
+}
+
+}  // namespace
+
+size_t chunk_split_scratch_bytes(int B, int T, int H, bool varlen, int sms) {
+  const SplitScratch r = split_scratch(B, T, H, varlen, sms);
+  return r.rec_bytes + r.seg_bytes;
+}
+
 cudaError_t launch_chunk_split(const void* q, const void* k, const void* v, const float* g,
                                const float* beta, const float* h0, const int32_t* cu_seqlens,
                                void* out, float* hT, int B, int T, int H, int dk, int dv,
-                               int gsh, cudaStream_t stream, const InputFusion* fz) {
+                               int gsh, cudaStream_t stream, const InputFusion* fz,
+                               const Workspace* ws) {
   int sms = 148;
   cudaMemPool_t pool = nullptr;
-  if (!device_ctx(&sms, &pool) || !set_attrs()) return cudaErrorInvalidDevice;
-  if (!pool) return cudaErrorMemoryAllocation;
+  if (!device_ctx(&sms, ws ? nullptr : &pool) || !set_attrs()) return cudaErrorInvalidDevice;
+  if (!ws && !pool) return cudaErrorMemoryAllocation;
   const bf16* qb = static_cast<const bf16*>(q);
   const bf16* kb = static_cast<const bf16*>(k);
   const bf16* vb = static_cast<const bf16*>(v);
@@ -1421,23 +1447,23 @@ cudaError_t launch_chunk_split(const void* q, const void* k, const void* v, cons
   const bf16* gt = fz ? static_cast<const bf16*>(fz->gate) : nullptr;
   const bool varlen = cu_seqlens != nullptr;
 
-  const long long nslots = chunk_slots(B, T, varlen);
-  const size_t rec_bytes = (size_t)nslots * H * REC_BYTES;
-  const SplitPlan plan = plan_split(B, T, H, varlen, sms);
-  const int G = plan.G;
-  const long long nch_all = ((long long)T + C - 1) / C;
-  int P = 0;
-  long long slots = 0;
-  size_t seg_bytes = 0;
-  if (G > 0 && (nch_all + G - 1) / G >= 2) {
-    P = (int)((nch_all + G - 1) / G);
-    slots = varlen ? (long long)P + B : (long long)B * P;
-    seg_bytes = (size_t)(plan.half > 0 ? 4 : 2) * slots * H * D * D * sizeof(float);
-  }
+  const SplitScratch sc = split_scratch(B, T, H, varlen, sms);
+  const long long nslots = sc.nslots;
+  const size_t rec_bytes = sc.rec_bytes, seg_bytes = sc.seg_bytes;
+  const SplitPlan plan = sc.plan;
+  const int G = plan.G, P = sc.P;
+  const long long slots = sc.slots;
   void* scratch = nullptr;
+  bool pooled = false;
   if (rec_bytes + seg_bytes > 0) {
-    const cudaError_t e = cudaMallocFromPoolAsync(&scratch, rec_bytes + seg_bytes, pool, stream);
-    if (e != cudaSuccess) return e;
+    if (ws) {
+      if (!ws->ptr || ws->bytes < rec_bytes + seg_bytes) return cudaErrorInvalidValue;
+      scratch = ws->ptr;
+    } else {
+      const cudaError_t e = cudaMallocFromPoolAsync(&scratch, rec_bytes + seg_bytes, pool, stream);
+      if (e != cudaSuccess) return e;
+      pooled = true;
+    }
   }
   uint8_t* rec = static_cast<uint8_t*>(scratch);
   float* segbuf = reinterpret_cast<float*>(rec + rec_bytes);
@@ -1490,7 +1516,7 @@ cudaError_t launch_chunk_split(const void* q, const void* k, const void* v, cons
   }
   const cudaError_t el = cudaGetLastError();
   if (e == cudaSuccess) e = el;
-  if (scratch) cudaFreeAsync(scratch, stream);
+  if (pooled) cudaFreeAsync(scratch, stream);
   return e;
 }
 

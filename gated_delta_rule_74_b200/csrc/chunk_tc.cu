@@ -883,16 +883,10 @@ namespace {
 
 // Dynamic shared memory of the kernel, set once per device.
 bool set_attrs() {
-  static bool done[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
-  if (!done[dev]) {
-    if (cudaFuncSetAttribute(kda_chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SMEM_BYTES) != cudaSuccess)
-      return false;
-    done[dev] = true;
-  }
-  return true;
+  return once_per_device(kOnceTc, []() {
+    return cudaFuncSetAttribute(kda_chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                SMEM_BYTES) == cudaSuccess;
+  });
 }
 
 // Chunks per segment (0: no split).  Cost model in units of one chunk step:
@@ -919,58 +913,8 @@ int plan_segments(int B, int T, int H, bool varlen, int sms) {
 
 }  // namespace
 
-cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const float* g,
-                            const float* beta, const float* h0, const int32_t* cu_seqlens,
-                            void* out, float* hT, int B, int T, int H, cudaStream_t stream) {
-  int sms = 148;
-  cudaMemPool_t pool = nullptr;
-  if (!device_ctx(&sms, &pool) || !set_attrs()) return cudaErrorInvalidDevice;
-  const bf16* qb = static_cast<const bf16*>(q);
-  const bf16* kb = static_cast<const bf16*>(k);
-  const bf16* vb = static_cast<const bf16*>(v);
-  bf16* ob = static_cast<bf16*>(out);
-
-  SegArgs sa{0, 1, 0, 0, nullptr, nullptr};
-  const int G = plan_segments(B, T, H, cu_seqlens != nullptr, sms);
-  void* scratch = nullptr;
-  const long long nch_all = ((long long)T + C - 1) / C;
-  if (G > 0 && pool && (nch_all + G - 1) / G >= 2) {
-    const long long nch = nch_all;
-    const int P = (int)((nch + G - 1) / G);
-    const long long slots = cu_seqlens ? (long long)P + B : (long long)B * P;
-    const size_t bytes = (size_t)2 * slots * H * D * D * sizeof(float);
-    if (cudaMallocFromPoolAsync(&scratch, bytes, pool, stream) == cudaSuccess) {
-      sa = SegArgs{G, P, 1, (int)slots, static_cast<float*>(scratch),
-                   static_cast<float*>(scratch) + (size_t)slots * H * D * D};
-    } else {
-      (void)cudaGetLastError();
-      scratch = nullptr;
-    }
-  }
-  if (sa.pass == 0) {
-    KDA_TIMED(KDA_KERNEL_FUSED, stream,
-              kda_chunk_tc_kernel<<<dim3(H, B, 1), NT, SMEM_BYTES, stream>>>(qb, kb, vb, g, beta, h0,
-                                                                            cu_seqlens, ob, hT, T, H, sa));
-    note_launches(1);
-    return cudaGetLastError();
-  }
-  KDA_TIMED(KDA_KERNEL_FUSED, stream,
-            kda_chunk_tc_kernel<<<dim3(H, B, 2 * sa.P), NT, SMEM_BYTES, stream>>>(
-                qb, kb, vb, g, beta, h0, cu_seqlens, ob, hT, T, H, sa));
-  cudaError_t ec = launch_seg_combine(cu_seqlens, B, T, H, sa, stream);
-  sa.pass = 2;
-  KDA_TIMED(KDA_KERNEL_FUSED, stream,
-            kda_chunk_tc_kernel<<<dim3(H, B, sa.P - 1), NT, SMEM_BYTES, stream>>>(
-                qb, kb, vb, g, beta, h0, cu_seqlens, ob, hT, T, H, sa));
-  note_launches(2);
-  cudaError_t e = cudaGetLastError();
-  if (e == cudaSuccess) e = ec;
-  cudaFreeAsync(scratch, stream);
-  return e;
-}
-
-// Same plan as launch_chunk_tc, run on caller-provided scratch: no pool, no
-// allocation of any kind.  Returns a kda_status_t: KDA_ERR_INVALID_ARG when the
+// The single-kernel prefill on caller-provided scratch: no pool, no allocation
+// of any kind.  Returns a kda_status_t: KDA_ERR_INVALID_ARG when the
 // split this call would use needs more than `capacity` bytes of scratch.
 int run_chunk_tc_static(const void* q, const void* k, const void* v, const float* g,
                         const float* beta, const float* h0, const int32_t* cu_seqlens, void* out,

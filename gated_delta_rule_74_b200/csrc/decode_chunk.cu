@@ -202,13 +202,11 @@ kda_decode_chunk_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   bool unsafe = false;
   {
     const int c = tid & (D - 1), t0 = 8 * (tid >> 7);
-    float G[LT], al[8][1];
+    float G[LT];
     float acc = 0.f;
 #pragma unroll
     for (int t = 0; t < LT; ++t) {
-      const float gt = fG[t * LDF + c];
-      if (t >= t0 && t < t0 + 8) al[t - t0][0] = __expf(gt);   // this thread's half
-      acc += gt;
+      acc += fG[t * LDF + c];
       G[t] = acc;
     }
     const float gl = acc;
@@ -216,10 +214,11 @@ kda_decode_chunk_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     // this half's growing factor: e^(G - G_8) over tokens 0..7, e^(G_8 - G) over 8..15
     unsafe = (t0 == 0 ? G[0] - G[8] : G[8] - G[15]) > kUnsafeDecay;
     if (__any_sync(0xffffffffu, unsafe)) {
-      // its pairs exactly (the factors below are zeroed for them)
-      float kv[8][1], qv[8][1];
+      // its pairs exactly (the factors below are zeroed for them); fG still holds g
+      float al[8][1], kv[8][1], qv[8][1];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
+        al[e][0] = __expf(fG[(t0 + e) * LDF + c]);
         kv[e][0] = unsafe ? fk[(t0 + e) * LDF + c] : 0.f;
         qv[e][0] = unsafe ? fq[(t0 + e) * LDF + c] : 0.f;
       }
@@ -434,15 +433,12 @@ bool decode_chunk_supported(int dk, int dv, int in_dtype, int L) {
 cudaError_t launch_decode_chunk(const void* q, const void* k, const void* v, const float* g,
                                 const float* beta, float* S, void* out, int N, int L, int H,
                                 cudaStream_t stream) {
-  static bool attr_done[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!attr_done[dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(
-        kda_decode_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DC_SMEM);
-    if (e != cudaSuccess) return e;
-    attr_done[dev] = true;
-  }
+  if (!once_per_device(kOnceDecodeChunk, []() {
+        return cudaFuncSetAttribute(kda_decode_chunk_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)DC_SMEM) == cudaSuccess;
+      }))
+    return cudaErrorInvalidDevice;
   const long long pairs = (long long)N * H;
   KDA_TIMED(KDA_KERNEL_DECODE, stream,
             kda_decode_chunk_kernel<<<(unsigned)pairs, NT, DC_SMEM, stream>>>(

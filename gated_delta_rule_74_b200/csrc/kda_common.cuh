@@ -18,6 +18,17 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
   return __float2bfloat16_rn(x);
 }
 
+// Runs setup() (kernel attributes and the like) once per call site and device, with
+// that device current; thread-safe.  A setup that fails is retried on the next call.
+enum OnceSite { kOnceSplit = 0, kOnceTc, kOnceDecodeChunk, kOnceCombine, kOnceCombineImg, kOnceSites };
+bool once_per_device(int site, bool (*setup)());
+
+// Most bytes the library pool of the current device has had in use at once; with
+// reset, the count restarts (kda_pool_usage).
+int pool_used_high(bool reset, unsigned long long* used_high);
+// SM count (and, when pool != nullptr, the library's memory pool) of the current device.
+bool device_ctx(int* sms, cudaMemPool_t* pool);
+
 // Count of kernel launches made by the library (see kda_launch_count()).
 void note_launches(unsigned long long n);
 
@@ -67,11 +78,9 @@ cudaError_t launch_chunk_simt(const void* q, const void* k, const void* v, const
                               void* out, float* hT, int B, int T, int H, int dk, int dv,
                               int in_dtype, int gsh, cudaStream_t stream);
 
-// Tensor-core chunked prefill (bf16, dk = dv = 128).
+// Tensor-core chunked prefill (bf16, dk = dv = 128) in one kernel per sequence
+// (kda_chunk_fwd_noalloc; see run_chunk_tc_static below).
 bool chunk_tc_supported(int dk, int dv, int in_dtype);
-cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const float* g,
-                            const float* beta, const float* h0, const int32_t* cu_seqlens,
-                            void* out, float* hT, int B, int T, int H, cudaStream_t stream);
 
 // Fused input prep and output gate (kda_chunk_fwd_fused; split path only):
 // q, k <- L2-normalised causal per-channel convolutions of the raw q, k (q also
@@ -83,23 +92,36 @@ struct InputFusion {
   const void* gate;      // [rows, H, dv] in the input dtype, or nullptr: no gate
 };
 
+// Scratch the caller provides for one call (kda_chunk_fwd_ws / kda_chunk_bwd_ws);
+// a launcher given one takes nothing from the library pool.
+struct Workspace {
+  void* ptr;
+  size_t bytes;
+};
+
 // Tensor-core prefill split into a parallel per-chunk kernel and a state pass
 // (bf16, dk, dv in {64, 128}: 64-wide heads run zero-padded to 128); its
 // scratch comes from the library's memory pool.
 bool chunk_split_supported(int dk, int dv, int in_dtype);
 // The split prefill's plan (host only): chunks per segment, chunks of a half point.
 void chunk_split_plan(int B, int T, int H, bool varlen, int sms, int* G, int* half);
+// Scratch bytes of one split prefill call on a device with `sms` SMs.
+size_t chunk_split_scratch_bytes(int B, int T, int H, bool varlen, int sms);
 cudaError_t launch_chunk_split(const void* q, const void* k, const void* v, const float* g,
                                const float* beta, const float* h0, const int32_t* cu_seqlens,
                                void* out, float* hT, int B, int T, int H, int dk, int dv,
-                               int gsh, cudaStream_t stream, const InputFusion* fz = nullptr);
+                               int gsh, cudaStream_t stream, const InputFusion* fz = nullptr,
+                               const Workspace* ws = nullptr);
 
 // Prefill backward (recurrent, fp32): gradients of sum(out*dout) + sum(hT*dhT).
+// Scratch bytes of one backward call.
+size_t chunk_bwd_scratch_bytes(int B, int T, int H, int dk, int dv, bool varlen);
 cudaError_t launch_chunk_bwd(const void* q, const void* k, const void* v, const float* g,
                              const float* beta, const float* h0, const int32_t* cu_seqlens,
                              const void* dout, const float* dhT, float* dq, float* dk, float* dv,
                              float* dg, float* dbeta, float* dh0, int B, int T, int H, int dkd,
-                             int dvd, int gsh, int in_dtype, cudaStream_t stream);
+                             int dvd, int gsh, int in_dtype, cudaStream_t stream,
+                             const Workspace* ws = nullptr);
 
 // Bounded-wait flags (one per kernel file): read, and with reset clear, the flag a
 // kernel raises when one of its bounded waits gives up.

@@ -12,7 +12,7 @@ namespace kda {
 namespace {
 
 struct DeviceCtx {
-  bool init = false;
+  bool init = false, pool_init = false;
   int sms = 148;
   cudaMemPool_t pool = nullptr;
 };
@@ -29,6 +29,9 @@ bool device_ctx(int* sms, cudaMemPool_t* pool) {
   if (!d.init) {
     if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return false;
+    d.init = true;
+  }
+  if (pool && !d.pool_init) {     // the pool is created on first use
     cudaMemPoolProps props = {};
     props.allocType = cudaMemAllocationTypePinned;
     props.location.type = cudaMemLocationTypeDevice;
@@ -40,10 +43,47 @@ bool device_ctx(int* sms, cudaMemPool_t* pool) {
       d.pool = nullptr;
       (void)cudaGetLastError();
     }
-    d.init = true;
+    d.pool_init = true;
   }
   if (sms) *sms = d.sms;
   if (pool) *pool = d.pool;
+  return true;
+}
+
+int pool_used_high(bool reset, unsigned long long* used_high) {
+  int sms = 0;
+  cudaMemPool_t pool = nullptr;
+  if (!device_ctx(&sms, &pool) || !pool) return KDA_ERR_CUDA;
+  uint64_t v = 0;
+  if (cudaMemPoolGetAttribute(pool, cudaMemPoolAttrUsedMemHigh, &v) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return KDA_ERR_CUDA;
+  }
+  *used_high = (unsigned long long)v;
+  if (reset) {
+    uint64_t zero = 0;
+    if (cudaMemPoolSetAttribute(pool, cudaMemPoolAttrUsedMemHigh, &zero) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return KDA_ERR_CUDA;
+    }
+  }
+  return KDA_OK;
+}
+
+bool once_per_device(int site, bool (*setup)()) {
+  static std::mutex mu;
+  static bool done[kOnceSites][64] = {};
+  int dev = 0;
+  if (site < 0 || site >= kOnceSites || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+    return false;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!done[site][dev]) {
+    if (!setup()) {
+      (void)cudaGetLastError();
+      return false;
+    }
+    done[site][dev] = true;
+  }
   return true;
 }
 

@@ -357,15 +357,12 @@ kda_seg_combine_img_kernel(const int32_t* __restrict__ cu_seqlens, int T, int H,
 
 cudaError_t launch_seg_combine(const int32_t* cu_seqlens, int B, int T, int H, const SegArgs& sa,
                                cudaStream_t stream) {
-  static bool attr_set[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!attr_set[dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(
-        kda_seg_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kCombineSmem);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  if (!once_per_device(kOnceCombine, []() {
+        return cudaFuncSetAttribute(kda_seg_combine_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)kCombineSmem) == cudaSuccess;
+      }))
+    return cudaErrorInvalidDevice;
   KDA_TIMED(KDA_KERNEL_COMBINE, stream,
             kda_seg_combine_kernel<<<dim3(H, B), kCombineThreads, kCombineSmem, stream>>>(cu_seqlens, T, H,
                                                                                           sa));
@@ -379,16 +376,12 @@ namespace kda {
 
 cudaError_t launch_seg_combine_img(const int32_t* cu_seqlens, int B, int T, int H, int dk, int dv,
                                    const SegArgs& sa, cudaStream_t stream) {
-  static bool attr_set[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!attr_set[dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(kda_seg_combine_img_kernel,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               (int)kCombine2Smem);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  if (!once_per_device(kOnceCombineImg, []() {
+        return cudaFuncSetAttribute(kda_seg_combine_img_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)kCombine2Smem) == cudaSuccess;
+      }))
+    return cudaErrorInvalidDevice;
   cudaError_t e = cudaSuccess;
   KDA_TIMED(KDA_KERNEL_COMBINE, stream,
             e = launch_after(kda_seg_combine_img_kernel, dim3(H, B, dv / kQCols), dim3(kCombineThreads),

@@ -201,8 +201,10 @@ KDA_API int kda_decode_chunk(const void* q, const void* k, const void* v,
  *   - Every GPU that loads the library holds the array (KDA_NOALLOC_SCRATCH_BYTES)
  *     until the process exits.
  *   - The first call on a device looks up the array's device address (one
- *     cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture.
+ *     cudaGetSymbolAddress, with that device current) and keeps it for the life
+ *     of the process; make that first call before any stream capture.  Do not
+ *     call this entry point again on a device after cudaDeviceReset: the kept
+ *     address would be stale.
  *   - All calls on a device share the one array: calls that overlap on the GPU
  *     (different streams without ordering) race on it.  Serialize them.
  */
@@ -323,6 +325,77 @@ KDA_API int kda_chunk_bwd_grouped(const void* q, const void* k, const void* v,
                                   const float* dhT, float* dq, float* dk, float* dv, float* dg,
                                   float* dbeta, float* dh0, int B, int T, int H, int dk_dim,
                                   int dv_dim, int g_group, int in_dtype, void* stream);
+
+/*
+ * Caller-owned workspace.  kda_chunk_fwd and kda_chunk_bwd take their scratch from
+ * a library-owned memory pool (see their Scratch notes).  The entry points below
+ * take it from the caller instead and allocate nothing at all, so that the caller
+ * owns every buffer: query the size, allocate it with the caller's allocator, and
+ * pass it in.
+ *
+ * kda_workspace_size -- the workspace bytes one call needs.  Host only: no device
+ * memory is read or allocated.
+ *   op        KDA_OP_CHUNK_FWD (kda_chunk_fwd_ws) or KDA_OP_CHUNK_BWD (kda_chunk_bwd_ws)
+ *   B, T, H, dk, dv, in_dtype   as the call will pass them
+ *   packed    != 0 when the call passes cu_seqlens
+ *   sms       streaming multiprocessors of the device the call will run on (the
+ *             prefill splits long sequences into segments by it), or 0 for the
+ *             current device (then the device's attribute is queried)
+ *   *bytes    the size in bytes; 0 means the call needs no workspace
+ * The forward's workspace is the chunk records, 74,240 B per (head, chunk slot)
+ * with ceil(T/64) * B slots (ceil(T/64) + B when packed), followed, when the call
+ * splits sequences into segments, by 2 * 64 KB per (segment slot, head), or
+ * 4 * 64 KB when the split keeps half-way states (kda_prefill_plan gives the split;
+ * segment slots = B * ceil(ceil(T/64) / G), or that count + B when packed).  KDA_F32
+ * forward calls need none.  The backward's is 4 * dk * dv B per (chunk slot +
+ * sequence, head) plus 64 * 4 * dk * dv B per (sequence, head).
+ * Returns KDA_OK, KDA_ERR_INVALID_ARG (unknown op, bad sizes, NULL bytes),
+ * KDA_ERR_UNSUPPORTED (head sizes) or KDA_ERR_CUDA (sms = 0 and no device).
+ */
+typedef enum {
+  KDA_OP_CHUNK_FWD = 0,
+  KDA_OP_CHUNK_BWD = 1
+} kda_op_t;
+KDA_API int kda_workspace_size(int op, int B, int T, int H, int dk, int dv, int packed,
+                               int in_dtype, int sms, size_t* bytes);
+
+/*
+ * kda_chunk_fwd_ws -- kda_chunk_fwd (g_group = 1) or kda_chunk_fwd_grouped (g_group
+ * channels per decay value, as documented there) on caller workspace.
+ * kda_chunk_bwd_ws -- kda_chunk_bwd / kda_chunk_bwd_grouped likewise.
+ * Passages, arguments, layouts and results: those of the calls named, plus
+ *   workspace        DEVICE memory of at least kda_workspace_size(op, ..., sms = 0)
+ *                    bytes, 256-byte aligned (NULL when that size is 0), owned by
+ *                    the caller.  Its contents on entry do not matter and are
+ *                    undefined afterwards; it must not be used by anything else
+ *                    until the call's work on `stream` has finished (calls that share
+ *                    one workspace must be ordered on the device).
+ *   workspace_bytes  its size.
+ * These calls allocate nothing and take nothing from the library pool.  A
+ * workspace that is too small or misaligned gives KDA_ERR_INVALID_ARG with
+ * nothing launched.  Otherwise as the calls named.
+ */
+KDA_API int kda_chunk_fwd_ws(const void* q, const void* k, const void* v,
+                             const float* g, const float* beta, const float* h0,
+                             const int32_t* cu_seqlens, void* out, float* hT,
+                             int B, int T, int H, int dk, int dv, int g_group, int in_dtype,
+                             void* workspace, size_t workspace_bytes, void* stream);
+KDA_API int kda_chunk_bwd_ws(const void* q, const void* k, const void* v,
+                             const float* g, const float* beta, const float* h0,
+                             const int32_t* cu_seqlens, const void* dout, const float* dhT,
+                             float* dq, float* dk, float* dv, float* dg, float* dbeta,
+                             float* dh0, int B, int T, int H, int dk_dim, int dv_dim,
+                             int g_group, int in_dtype, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
+/*
+ * kda_pool_usage -- the most bytes the library's memory pool on the current device
+ * has had in use at once, since the pool was created or since the last reset
+ * (diagnostic).  reset != 0 restarts the count after reading it.  Creates the pool
+ * if it does not exist yet (which allocates no memory).  Returns KDA_OK,
+ * KDA_ERR_INVALID_ARG (NULL output) or KDA_ERR_CUDA.
+ */
+KDA_API int kda_pool_usage(int reset, unsigned long long* used_high_bytes);
 
 /*
  * kda_device_status -- did a bounded device-side wait give up?

@@ -15,6 +15,8 @@ import torch
 import oracle
 from oracle import reference as ref
 
+import kernel_forms as kf
+
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
 
@@ -363,7 +365,7 @@ def test_pair_grads_blocked_equal_pairwise_terms(L, g_scale):
     q, k, gam = q[0, :, 0], k[0, :, 0], np.cumsum(g[0, :, 0], axis=0)
     dA, dAqk = rng.standard_normal((L, L)), rng.standard_normal((L, L))
     want = _pair_terms_einsum(dA, dAqk, q, k, gam)
-    got = ref.pair_grads_blocked(dA, dAqk, q, k, gam)
+    got = kf.pair_grads_blocked(dA, dAqk, q, k, gam)
     for w, x, name in zip(want, got, ("dq", "dk", "dgam")):
         assert np.isfinite(x).all(), name
         assert np.abs(x - w).max() <= 1e-12 * max(np.abs(w).max(), 1e-30), name
@@ -376,7 +378,7 @@ def test_reverse_state_segments_equal_chunk_start_gradients(oracle_lib, T, C, G)
     pin above ties to the recurrent backward."""
     rng = np.random.default_rng(T + C + G)
     (q, k, v, g, b, h0, dout, dhT), _, chk = _bwd_pair(rng, T, 6, 5, C)
-    seg = ref.reverse_state_segments(q[0, :, 0], k[0, :, 0], v[0, :, 0], g[0, :, 0], b[0, :, 0],
+    seg = kf.reverse_state_segments(q[0, :, 0], k[0, :, 0], v[0, :, 0], g[0, :, 0], b[0, :, 0],
                                      dout[0, :, 0], dhT[0, 0], C=C, G=G)
     assert seg.shape == chk["dS_start"].shape
     assert np.abs(seg - chk["dS_start"]).max() <= 1e-11 * np.abs(chk["dS_start"]).max()

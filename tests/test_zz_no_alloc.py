@@ -11,6 +11,7 @@ import torch
 
 import gated_delta_rule_74_b200 as kda
 import kda_inputs as ki
+import oracle
 from _helpers import TOL, rel_err, to_dev
 
 pytestmark = pytest.mark.gpu
@@ -29,11 +30,12 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _call_noalloc(d, out, hT):
+def _call_noalloc(d, out, hT, dtype=None):
     nseq = d["B"]
+    dt = kda.KDA_BF16 if dtype in (None, "bf16") else kda.KDA_F32
     rc = _noalloc()(_ptr(d["q"]), _ptr(d["k"]), _ptr(d["v"]), _ptr(d["g"]), _ptr(d["beta"]),
                     _ptr(d["h0"]), _ptr(d["cu_seqlens"]), _ptr(out), _ptr(hT),
-                    nseq, d["T"], d["H"], d["dk"], d["dv"], kda.KDA_BF16,
+                    nseq, d["T"], d["H"], d["dk"], d["dv"], dt,
                     ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     return rc
 
@@ -41,7 +43,7 @@ def _call_noalloc(d, out, hT):
 @pytest.mark.parametrize("shape", ["fixed", "packed"])
 def test_noalloc_matches_chunk_fwd_twice(shape):
     if shape == "fixed":
-        # B*H = 12 with 128 chunks: the call is split into segments (uses scratch)
+        # B*H = 6 with 64 chunks: the call is split into segments (uses scratch)
         x = ki.make_prefill("t8k_h12", H=6, T=4096)
     else:
         spec = ki.PrefillSpec("varlen", B=0, T=0, H=3, dk=128, dv=128, dtype="bf16",
@@ -57,6 +59,39 @@ def test_noalloc_matches_chunk_fwd_twice(shape):
         torch.cuda.synchronize()
         assert rel_err(out, ref_out.double().cpu().numpy()) <= TOL["bf16"]
         assert rel_err(hT, ref_hT.double().cpu().numpy()) <= TOL["bf16"]
+    # and against the float64 oracle directly, on the same inputs
+    o_ref, s_ref = oracle.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], x["h0"],
+                                  x["cu_seqlens"])
+    assert rel_err(out, o_ref) <= TOL["bf16"]
+    assert rel_err(hT, s_ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("dtype,dk,dv", [("bf16", 64, 64), ("f32", 64, 64), ("f32", 128, 128),
+                                         ("bf16", 128, 64)])
+def test_noalloc_other_shapes_match_oracle(dtype, dk, dv):
+    """64-wide heads and fp32 inputs run on the CUDA-core path (no scratch at all)."""
+    spec = ki.PrefillSpec("na", B=2, T=200, H=3, dk=dk, dv=dv, dtype=dtype, decay="alog",
+                          seed=dk + dv, h0=True)
+    x = ki.make_prefill(spec)
+    d = to_dev(x)
+    for _ in range(2):
+        out = torch.full_like(d["v"], float("nan"))
+        hT = torch.full_like(d["h0"], float("nan"))
+        assert _call_noalloc(d, out, hT, dtype) == kda.KDA_OK
+        torch.cuda.synchronize()
+        o_ref, s_ref = oracle.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], x["h0"])
+        assert rel_err(out, o_ref) <= TOL[dtype]
+        assert rel_err(hT, s_ref) <= TOL[dtype]
+
+
+def test_noalloc_empty_sequence_without_hT():
+    """T = 0 with no final state: nothing to write, and the call succeeds."""
+    spec = ki.PrefillSpec("na0", B=2, T=0, H=2, dk=128, dv=128, dtype="bf16", decay="alog",
+                          seed=3, h0=True)
+    d = to_dev(ki.make_prefill(spec))
+    out = torch.empty_like(d["v"])
+    assert _call_noalloc(d, out, None) == kda.KDA_OK
+    torch.cuda.synchronize()
 
 
 def test_noalloc_rejects_scratch_beyond_its_array():
