@@ -12,6 +12,12 @@ kda_decode_step calls on the config-4 shape (N=256 sequences x H=96 heads,
 d=128, 1.61 GB of fp32 state), reported as GB/s of algorithmic traffic and as a
 fraction of the measured HBM peak.
 
+`configs` times the other prefill workloads the same way (configs 0-3 of the
+workload table: fp32_t256, b16_t512_d64, packed_16k, t32k_h96), each with its
+fraction of the HBM roofline and the oracle timed on a bounded sample of it;
+`decode.cpu_baseline` is the oracle's decode step on 8 of the 256 sequences,
+scaled to whole steps/s.
+
 L2: every prefill step reads a different one of three resident input sets
 (3 x 152 MB > 126 MB L2), so no step finds its inputs in L2; the decode state
 (1.61 GB) is far larger than L2.
@@ -665,6 +671,106 @@ def decode_leg(args, world, rank, dev, stream, barrier, clocks, hbm, peak_kind):
             "gpu_launches": launches, "clocks": clocks.summary(mark0, clocks.mark())}
 
 
+CONFIG_WORKLOADS = ("fp32_t256", "b16_t512_d64", "packed_16k", "t32k_h96")
+L2_BYTES = 126 * 1024 * 1024
+
+
+def configs_leg(args, world, rank, dev, stream, barrier, hbm, tf_sust):
+    """Every other prefill workload: K timed kda_chunk_fwd calls each (three resident
+    input sets when one set is smaller than twice the L2, else one set larger than
+    L2), its fraction of the HBM roofline, and -- on rank 0 at N = 1 -- the float64
+    oracle timed on a bounded sample of the same workload."""
+    import torch
+
+    import gated_delta_rule_74_b200 as kda
+    import kda_inputs as ki
+
+    res = {}
+    for name in CONFIG_WORKLOADS:
+        if name == args.workload:
+            continue
+        spec = ki.PREFILL_SPECS[name]
+        x = ki.make_prefill(spec, seed=rank_seed(spec.seed, rank))
+        s_in = 2 if x["dtype"] == "bf16" else 4
+        rows = x["T"] if x["cu_seqlens"] is not None else x["B"] * x["T"]
+        bytes_call = prefill_bytes(rows, x["H"], x["dk"], x["dv"], s_in, x["B"],
+                                   x["h0"] is not None, True)
+        nsets = 3 if bytes_call < 2 * L2_BYTES else 1
+        sets = []
+        for i in range(nsets):
+            xi = x if i == 0 else ki.make_prefill(spec, seed=rank_seed(spec.seed, rank, i))
+            d = {n: (t.to(dev) if isinstance(t, torch.Tensor) else t) for n, t in xi.items()}
+            d["out"] = torch.empty_like(d["v"])
+            d["hT"] = torch.empty(xi["B"], xi["H"], xi["dk"], xi["dv"], device=dev)
+            sets.append(d)
+        del x
+
+        def call(i):
+            d = sets[i % nsets]
+            kda.kda_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], h0=d["h0"],
+                              cu_seqlens=d["cu_seqlens"], out=d["out"], hT=d["hT"], stream=stream)
+
+        steps = max(3, min(args.steps, 50))
+        for i in range(args.warmup):
+            call(i)
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(steps):
+            call(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms = _max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
+        gbs = bytes_call / (ms / 1e3) / 1e9
+        flops = prefill_flops(rows, sets[0]["H"], sets[0]["dk"], sets[0]["dv"])
+        t_roof = max(bytes_call / (hbm * 1e9), flops / (tf_sust * 1e12) if s_in == 2 else 0.0)
+        entry = {"workload": f"{name}: {spec.desc}", "tokens_per_s": rows * world / (ms / 1e3),
+                 "ms_per_call": ms, "steps": steps, "algorithmic_bytes_per_call": bytes_call,
+                 "gbs": gbs, "frac_of_hbm_peak": gbs / hbm,
+                 "roofline_ms": 1e3 * t_roof, "frac_of_roofline": 1e3 * t_roof / ms,
+                 "l2": (f"{nsets} resident input sets rotated" if nsets > 1 else
+                        "one input set, larger than L2")}
+        del sets
+        torch.cuda.empty_cache()
+        if world == 1 and not args.no_cpu_baseline and rank == 0:
+            sub = argparse.Namespace(**vars(args))
+            sub.workload = name
+            sub.ref_tokens = {"t32k_h96": 256, "packed_16k": 2048}.get(name, 0)
+            sub.ref_seconds = 3.0
+            val, threads, desc, _ = _oracle_timing(sub)
+            entry["cpu_baseline"] = {"value": val, "unit": UNIT, "cores": threads,
+                                     "kind": "oracle", "sample": desc}
+        res[name] = entry
+    return res
+
+
+def decode_oracle(args, N_sample=8):
+    """The float64 oracle's decode step on a bounded sample of the config-4 shape
+    (N_sample of the 256 sequences, all 96 heads), scaled to whole steps."""
+    import kda_inputs as ki
+    import oracle
+    oracle.build()
+    dspec = ki.DECODE_SPECS["decode_n256_h96"]
+    dd = ki.make_decode(dspec, steps=1, N=N_sample)
+    q, k, v, g, b = (dd[n][0] for n in ("q", "k", "v", "g", "beta"))
+    threads = max(1, min(oracle.max_threads(), N_sample * dd["H"]))
+    S = dd["S0"]
+    times = []
+    t_all = time.perf_counter()
+    while time.perf_counter() - t_all < 3.0 and len(times) < 50:
+        t0 = time.perf_counter()
+        oracle.decode(q, k, v, g, b, S, nthreads=threads)
+        times.append(time.perf_counter() - t0)
+    med = statistics.median(times)
+    scale = dspec.N / N_sample
+    return {"value": 1.0 / (med * scale), "unit": "steps/s", "cores": threads, "kind": "oracle",
+            "sample": f"{N_sample} of the {dspec.N} sequences x {dd['H']} heads per step, "
+                      f"float64 recurrence, median of {len(times)} steps, scaled to all "
+                      f"{dspec.N} sequences"}
+
+
 KERNEL_NAMES = {"prep": "kda_chunk_prep_kernel", "state": "kda_state_pass_kernel",
                 "combine": "kda_seg_combine_img_kernel", "fused": "kda_chunk_tc_kernel",
                 "simt": "kda_chunk_simt_kernel"}
@@ -819,9 +925,14 @@ def run_ours(args, world, rank, local):
     bwd = None
     if not args.decode_only and not args.no_bwd:
         bwd = bwd_leg(args, world, rank, dev, stream, barrier, hbm)
+    cfg = None
+    if not args.decode_only and not args.no_configs:
+        cfg = configs_leg(args, world, rank, dev, stream, barrier, hbm, tf_sust)
     dec = None
     if not args.no_decode:
         dec = decode_leg(args, world, rank, dev, stream, barrier, clocks, hbm, peak_kind)
+        if dec is not None and world == 1 and rank == 0 and not args.no_cpu_baseline:
+            dec["cpu_baseline"] = decode_oracle(args)
     clocks.stop()
 
     if rank != 0:
@@ -849,6 +960,7 @@ def run_ours(args, world, rank, local):
         "prefill_decay_g64": grp,
         "prefill_fused_prep": fzd,
         "prefill_bwd": bwd,
+        "configs": cfg,
         "decode": dec, "e2e": pf["e2e"], "gpu_launches": pf["launches"],
         "clocks": pf["clocks"], "cpu_baseline": cpu,
     }
@@ -882,6 +994,8 @@ def main():
     ap.add_argument("--decode-n", type=int, default=0,
                     help="sequences in the decode leg (0 = the config-4 value, 256)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other prefill workloads (configs leg)")
     ap.add_argument("--ref-tokens", type=int, default=0,
                     help="tokens of the workload the oracle processes per pass (0: all for "
                          "the cpu_baseline leg, 1024 per step for --impl reference)")

@@ -52,12 +52,14 @@
 #include <cuda_fp16.h>
 
 #include <algorithm>
+#include <cstring>
 #include <type_traits>
 
 #include "decay_pairs.cuh"
 #include "kda_common.cuh"
 #include "segments.cuh"
 #include "sm100.cuh"
+#include "tma.cuh"
 
 namespace kda {
 
@@ -82,6 +84,12 @@ constexpr uint32_t REC_U = 57344;       // U^T [dv][64 tokens] f16: 128-byte row
                                         // chunks (8 tokens) XOR-swizzled with (row % 8)
 constexpr uint32_t REC_DECAY = 73728;   // exp(G_last) per key channel, fp32 [dk]
 constexpr uint32_t REC_BYTES = 74240;
+
+// TMA maps of the prep kernel's tiles: q, k, g [rows, H, dk] and v [rows, H, dv]
+// (3-D: channel, head, token row), boxes of 64 token rows of one head.
+struct PrepMaps {
+  CUtensorMap q, k, g, v;
+};
 
 // ---- prep kernel: shared memory (from a 1024-aligned base) and TMEM
 constexpr uint32_t Q_V = 0;             // V: MN-major SW128 A operand of U^T (M = value, K = token)
@@ -244,10 +252,11 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
                       const float* __restrict__ beta, const int32_t* __restrict__ cu_seqlens,
                       uint8_t* __restrict__ rec, int B, int T, int H, int dk, int dv, int gsh,
                       long long nslots, const float* __restrict__ conv_q,
-                      const float* __restrict__ conv_k, int convW) {
+                      const float* __restrict__ conv_k, int convW,
+                      const __grid_constant__ PrepMaps maps, int tma) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
-  __shared__ uint64_t bar;
+  __shared__ uint64_t bar, in_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ float s_beta[C];
   __shared__ float2 s_sum[4][64];       // per 16-row block: its total log-decay (channel pair)
@@ -286,24 +295,76 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   const long long rbase = row0 + t0;                   // first token row of the chunk
   uint8_t* rc = rec + ((size_t)h * (size_t)nslots + (size_t)slot) * REC_BYTES;
 
-  // v goes straight into the MN-major operand of U^T (rows >= L zero-filled)
+  // The chunk's tiles.  TMA (tma != 0; not with the fused convolution): v straight
+  // into the MN-major operand of U^T (two 64-value boxes, 128-byte swizzle), q and k
+  // row-major into the Gram operand area and g into the R area (both free until the
+  // operand build), all on one mbarrier.  Otherwise v by cp.async and q, k, g by
+  // per-thread loads below.  Rows >= L are never used from the staged tiles; the v
+  // rows >= L are zeroed once the tile has landed.
+  const bool use_tma = !CONV && tma != 0;
+  if (use_tma) {
+    if (tid == 0) {
+      mbar_init(&in_bar, 1);
+      mbar_init(&bar, 1);
+      fence_mbar_init();
+      const uint32_t bytes =
+          (uint32_t)(C * dv * 2 + 2 * C * dk * 2 + (gsh == 0 ? C * dk * 4 : 0));
+      mbar_arrive_expect_tx(&in_bar, bytes);
+      const int row = (int)rbase;               // < 2^31 - 64 (checked on the host)
+      tma_load_3d(sm + Q_V, &maps.v, 0, h, row, &in_bar);
+      if (dv > 64) tma_load_3d(sm + Q_V + 8192, &maps.v, 64, h, row, &in_bar);
+      tma_load_3d(sm + Q_L, &maps.q, 0, h, row, &in_bar);
+      tma_load_3d(sm + Q_L + 16384, &maps.k, 0, h, row, &in_bar);
+      if (gsh == 0) tma_load_3d(sm + Q_R, &maps.g, 0, h, row, &in_bar);
+    }
+  } else {
 #pragma unroll
-  for (int it = 0; it < 4; ++it) {
-    const int idx = tid + it * NT;
-    const int r = idx >> 4, ch = idx & 15;
-    const long long e = ((rbase + min(r, L - 1)) * H + h) * dv + min(ch * 8, dv - 8);
-    cp_async16(sm + Q_V + chunk_mnmajor_sw128(ch, r, C), v + e,
-               (r < L && ch * 8 < dv) ? 16u : 0u);
+    for (int it = 0; it < 4; ++it) {
+      const int idx = tid + it * NT;
+      const int r = idx >> 4, ch = idx & 15;
+      const long long e = ((rbase + min(r, L - 1)) * H + h) * dv + min(ch * 8, dv - 8);
+      cp_async16(sm + Q_V + chunk_mnmajor_sw128(ch, r, C), v + e,
+                 (r < L && ch * 8 < dv) ? 16u : 0u);
+    }
+    cp_async_commit();
   }
-  cp_async_commit();
   if (tid < C) s_beta[tid] = tid < L ? beta[(rbase + tid) * H + h] : 0.f;
   if (warp == 0) {
     tmem_alloc(&tmem_base_sh, kPrepTmemCols);
     tmem_relinquish();
   }
-  if (tid == 0) {
+  if (!use_tma && tid == 0) {
     mbar_init(&bar, 1);
     fence_mbar_init();
+  }
+  if (use_tma) {
+    tc_fence_before();
+    __syncthreads();                            // in_bar is initialised
+    tc_fence_after();
+    bool got = true;
+    if (warp == 0) got = mbar_wait(&in_bar, 0, kWaitLimit);
+    if (__syncthreads_or(!got)) {
+      // the tiles never arrived: raise the flag, let the copies finish, free TMEM
+      if (tid == 0) {
+        atomicExch(&g_chunk_split_timeout, 1);
+        mbar_wait(&in_bar, 0, kWaitLimit);
+      }
+      tc_fence_before();
+      __syncthreads();
+      if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base_sh, kPrepTmemCols);
+      }
+      return;
+    }
+    // v: rows >= L, and values >= dv, to zero
+    if (L < C || dv < D) {
+      for (int i = tid; i < C * 16; i += NT) {
+        const int r = i >> 4, ch = i & 15;
+        if (r >= L || ch * 8 >= dv) sts16(sm, Q_V + chunk_mnmajor_sw128(ch, r, C),
+                                           make_uint4(0u, 0u, 0u, 0u));
+      }
+    }
   }
 
   // ---- P1: per thread a channel pair (2cp, 2cp+1) and a 16-row block a
@@ -316,15 +377,25 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     const int r = 16 * a + e;
     if (r < L && c0 < dk) {
       const long long idx = ((rbase + r) * H + h) * dk + c0;
-      if (gsh == 0) {
-        gq[e] = __ldg(reinterpret_cast<const float2*>(g + idx));
-      } else {                                   // one decay per group of 2^gsh channels
-        const float gg = __ldg(g + ((rbase + r) * H + h) * (dk >> gsh) + (c0 >> gsh));
-        gq[e] = make_float2(gg, gg);
+      if (use_tma) {                             // staged tiles: row stride dk
+        const int si = r * dk + c0;
+        if (gsh == 0) gq[e] = *reinterpret_cast<const float2*>(sm + Q_R + 4 * si);
+        kw[e] = *reinterpret_cast<const uint32_t*>(sm + Q_L + 16384 + 2 * si);
+        qw[e] = *reinterpret_cast<const uint32_t*>(sm + Q_L + 2 * si);
+      }
+      if (!use_tma || gsh != 0) {
+        if (gsh == 0) {
+          gq[e] = __ldg(reinterpret_cast<const float2*>(g + idx));
+        } else {                                 // one decay per group of 2^gsh channels
+          const float gg = __ldg(g + ((rbase + r) * H + h) * (dk >> gsh) + (c0 >> gsh));
+          gq[e] = make_float2(gg, gg);
+        }
       }
       if constexpr (!CONV) {
-        kw[e] = __ldg(reinterpret_cast<const unsigned int*>(k + idx));
-        qw[e] = __ldg(reinterpret_cast<const unsigned int*>(q + idx));
+        if (!use_tma) {
+          kw[e] = __ldg(reinterpret_cast<const unsigned int*>(k + idx));
+          qw[e] = __ldg(reinterpret_cast<const unsigned int*>(q + idx));
+        }
       }
     } else {
       gq[e] = make_float2(0.f, 0.f);
@@ -1470,16 +1541,34 @@ cudaError_t launch_chunk_split(const void* q, const void* k, const void* v, cons
 
   cudaError_t e = cudaSuccess;
   if (nslots > 0) {
-    if (fz && fz->conv_q) {
+    // TMA maps of the tiles (rows addressed by int32 coordinates)
+    PrepMaps maps;
+    const long long rows = varlen ? (long long)T : (long long)B * T;
+    const bool conv = fz && fz->conv_q;
+    int tma = 0;
+    if (!conv && rows > 0 && rows < (1LL << 31) - 2 * C) {
+      const uint64_t hh = (uint64_t)H, nr = (uint64_t)rows;
+      tma = make_tile_map_3d(&maps.q, false, qb, dk, hh, nr, dk * 2ull, hh * dk * 2, dk, C,
+                             false) &&
+            make_tile_map_3d(&maps.k, false, kb, dk, hh, nr, dk * 2ull, hh * dk * 2, dk, C,
+                             false) &&
+            make_tile_map_3d(&maps.v, false, vb, dv, hh, nr, dv * 2ull, hh * dv * 2, 64, C,
+                             true) &&
+            (gsh != 0 || make_tile_map_3d(&maps.g, true, g, dk, hh, nr, dk * 4ull, hh * dk * 4,
+                                          dk, C, false));
+      if (gsh != 0) maps.g = maps.q;             // not read
+    }
+    if (!tma) memset(&maps, 0, sizeof(maps));
+    if (conv) {
       KDA_TIMED(KDA_KERNEL_PREP, stream,
                 kda_chunk_prep_kernel<true><<<dim3((unsigned)nslots, H), NT, PREP_SMEM, stream>>>(
                     qb, kb, vb, g, beta, cu_seqlens, rec, B, T, H, dk, dv, gsh, nslots,
-                    fz->conv_q, fz->conv_k, fz->W));
+                    fz->conv_q, fz->conv_k, fz->W, maps, 0));
     } else {
       KDA_TIMED(KDA_KERNEL_PREP, stream,
                 kda_chunk_prep_kernel<false><<<dim3((unsigned)nslots, H), NT, PREP_SMEM, stream>>>(
                     qb, kb, vb, g, beta, cu_seqlens, rec, B, T, H, dk, dv, gsh, nslots, nullptr,
-                    nullptr, 0));
+                    nullptr, 0, maps, tma));
     }
     note_launches(1);
   }

@@ -76,6 +76,18 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
+// 3-D tiled TMA load of one box into shared memory, completing on `bar` (which
+// counts the box's bytes).  `tmap` is the address of a CUtensorMap kernel
+// parameter (__grid_constant__).  Plain load: no cluster multicast.
+__device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* tmap, int c0, int c1,
+                                            int c2, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // ------------------------------------------------- async global -> smem copies
 // 16-byte cp.async (L2 only); src_bytes = 0 zero-fills the destination and reads
 // nothing (the caller still passes an in-bounds address).
