@@ -930,7 +930,7 @@ __device__ __forceinline__ uint4 apply_gate(uint4 o, uint4 z) {
 
 // A state in TMEM (this thread: columns [32 wq, 32 wq + 32) of row j of S^T, from
 // taddr) -> dst.  A transition X (identity start) goes out as bf16 hi / lo images for
-// the segment combine (MN-major SW128 A operand, M = row of X, K = column; TMEM lane
+// pass C's hops (MN-major SW128 B operand, N = row of X, K = column; TMEM lane
 // j holds column j of X); any other state as fp32 [dk][dv] rows.  Called once or
 // twice per chain, out of line so the chunk loop keeps its registers.
 __device__ __noinline__ void store_state_cols(float* dst, uint32_t taddr, bool ximg, int wq, int j,
@@ -973,7 +973,7 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   __shared__ uint64_t full[2];
-  __shared__ uint64_t mbar, xbar;
+  __shared__ uint64_t mbar;
   __shared__ uint32_t tmem_base_sh;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -992,8 +992,8 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
   bool outputs = true, homog = false;
   int mid = 0;                                    // pass A: after `mid` chunks the state
   float* mid_dst = nullptr;                       // is also kept here
-  const float* mid_src = nullptr;                 // pass C from a half point: S_start,p and
-  const uint8_t* mid_x = nullptr;                 // the X_half,p images (init = Sloc_half,p)
+  int nhop = 0, hop_p = 0;                        // pass C: hops that form the start state
+  const float* hop0 = nullptr;                    // (from hop0, see below)
   if (sa.pass != 0) {
     const int Ps = seg_count(t_end - t_beg, sa.G);
     const int z = blockIdx.z;
@@ -1030,20 +1030,19 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
       }
     } else {
       // z = p - 1 (one chain per segment), or 2 (p - 1) + q with half points: q = 0
-      // runs the segment's first Gh chunks, q = 1 the rest from S_mid,p
+      // runs the segment's first Gh chunks, q = 1 the rest from S_mid,p.  The chain
+      // forms its own start state from pass A's results, hop by hop:
+      //   S_start,1 = S_end,0 (= Sloc_0),  S_start,k+1 = X_k S_start,k + Sloc_k,
+      //   and for q = 1  S_mid,p = X_half,p S_start,p + Sloc_half,p.
       const int p = (HALF ? z / 2 : z) + 1, q = HALF ? z % 2 : 0;
       if (Ps <= 1 || p > Ps - 1) return;
       const bool split = HALF && p <= Ps - 2;
       if (q == 1 && !split) return;
-      const long long o = q == 0 ? slot_off(p - 1) : slot_off(p);
-      if (o < 0) return;
-      init = q == 0 ? sa.sbuf + o : sa.sbuf_h + o;
-      if (q == 1) {                               // S_mid,p = X_half,p S_start,p + Sloc_half,p
-        const long long o0 = slot_off(p - 1);
-        if (o0 < 0) return;
-        mid_src = sa.sbuf + o0;
-        mid_x = reinterpret_cast<const uint8_t*>(sa.xbuf_h + o);
-      }
+      if (slot_off(q == 1 ? p : p - 1) < 0) return;     // slots beyond the planned scratch
+      nhop = p - 1 + q;
+      hop0 = sa.sbuf + slot_off(0);
+      init = nhop == 0 ? hop0 : nullptr;
+      hop_p = p;
       if (p != Ps - 1) fin = nullptr;
       t_beg += p * seg_tok;
       const long long seg_end = min(t_end, t_beg + seg_tok);
@@ -1069,31 +1068,37 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
     mbar_init(&full[0], 1);
     mbar_init(&full[1], 1);
     mbar_init(&mbar, 1);
-    mbar_init(&xbar, 1);
     fence_mbar_init();
   }
   __syncthreads();
-  // records requested (thread 0); from a half point, record buffer 1 first takes the
-  // X_half images and record 1 follows once they are consumed
-  int issued = nch < 2 ? nch : (HALF && mid_x ? 1 : 2);
-  int xstate = 0;                                    // thread 0: 1 images requested, 2 MMAs issued
-  // Launched right behind the kernel before it (programmatic stream serialization).
-  // Passes 0 and A wait for the prep kernel before the first record copy.  Pass C
-  // needs no wait for the records (prep) or a second-half chain's X_half images
-  // (pass A): pass A does not let its successor start early, so the combine, and pass
-  // C after it, start only once pass A, and prep before it, have ended.  The combine's
-  // output (S_start) is read only after the wait below the copies.
+  // Hop h (pass C): X images and Sloc of the hop.  Loads go through the two record
+  // buffers in one sequence -- the hops' X images first, then the records -- load li
+  // into buffer li & 1 on barrier full[li & 1], phase (li >> 1) & 1.
+  const long long seq_slot = seg_slot_base(cu_seqlens, s, T, sa.G);
+  auto hop_off = [&](int hh) -> long long {
+    return ((seq_slot + (hh < hop_p - 1 ? hh + 1 : hop_p)) * H + h) * D * D;
+  };
+  auto hop_x = [&](int hh) -> const uint8_t* {
+    return reinterpret_cast<const uint8_t*>((hh < hop_p - 1 ? sa.xbuf : sa.xbuf_h) + hop_off(hh));
+  };
+  auto hop_l = [&](int hh) -> const float* {
+    return (hh < hop_p - 1 ? sa.sbuf : sa.sbuf_h) + hop_off(hh);
+  };
+  const int nload = nhop + nch;
+  auto issue_load = [&](int li) {                  // thread 0
+    const uint32_t bytes = li < nhop ? 65536u : REC_BYTES;
+    mbar_arrive_expect_tx(&full[li & 1], bytes);
+    bulk_g2s(sm + (li & 1) * S_BUF, li < nhop ? hop_x(li) : rec_ptr(li - nhop), bytes,
+             &full[li & 1]);
+  };
+  int issued = min(nload, 2);                      // loads requested (thread 0)
+  int waited = 0;                                  // loads whose arrival thread 0 has seen
+  // Launched right behind the kernel before it (programmatic stream serialization):
+  // everything it reads from that kernel (prep's records, pass A's states and
+  // transitions) is read after the wait.
   if (tid == 0) {
-    if (sa.pass != 2) grid_dep_wait();
-    for (int i = 0; i < issued; ++i) {
-      mbar_arrive_expect_tx(&full[i], REC_BYTES);
-      bulk_g2s(sm + i * S_BUF, rec_ptr(i), REC_BYTES, &full[i]);
-    }
-    if (HALF && mid_x) {
-      mbar_arrive_expect_tx(&xbar, 65536);
-      bulk_g2s(sm + S_BUF, mid_x, 65536, &xbar);
-      xstate = 1;
-    }
+    grid_dep_wait();
+    for (int li = 0; li < issued; ++li) issue_load(li);
   }
   tc_fence_before();
   __syncthreads();
@@ -1101,9 +1106,9 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
   const uint32_t tb = tmem_base_sh;
   const uint32_t tl = tb + lane_base;
 
-  if (sa.pass == 2) grid_dep_wait();     // S_start comes from the segment combine
+  if (sa.pass == 2) grid_dep_wait();
   // ---- initial state: columns [32 wq, 32 wq + 32) of row j of S^T, and its bf16 copy
-  {
+  if (nhop == 0) {
     const int c = 32 * wq;
     uint32_t f0[16], f1[16], pk[16];
 #pragma unroll
@@ -1116,45 +1121,61 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
     }
     tmem_st16(tl + ST_S + c, f0);
     tmem_st16(tl + ST_S + c + 16, f1);
-    if (HALF && mid_src) {              // bf16 hi / lo parts of S_start^T (A operands)
-      uint32_t lo[16];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int r0 = c + 2 * e, r1 = c + 16 + 2 * e;
-        const bool ok = j < dv;
-        const float a0 = ok && r0 < dk ? mid_src[(long long)r0 * dv + j] : 0.f;
-        const float a1 = ok && r0 + 1 < dk ? mid_src[(long long)(r0 + 1) * dv + j] : 0.f;
-        const float b0 = ok && r1 < dk ? mid_src[(long long)r1 * dv + j] : 0.f;
-        const float b1 = ok && r1 + 1 < dk ? mid_src[(long long)(r1 + 1) * dv + j] : 0.f;
-        pk[e] = pack_bf16(a0, a1);
-        pk[8 + e] = pack_bf16(b0, b1);
-        lo[e] = pack_bf16(a0 - bf_lo(pk[e]), a1 - bf_hi(pk[e]));
-        lo[8 + e] = pack_bf16(b0 - bf_lo(pk[8 + e]), b1 - bf_hi(pk[8 + e]));
-      }
-      tmem_st16(tl + ST_LO + c / 2, lo);
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        pk[e] = pack_bf16(__uint_as_float(f0[2 * e]), __uint_as_float(f0[2 * e + 1]));
-        pk[8 + e] = pack_bf16(__uint_as_float(f1[2 * e]), __uint_as_float(f1[2 * e + 1]));
-      }
+    for (int e = 0; e < 8; ++e) {
+      pk[e] = pack_bf16(__uint_as_float(f0[2 * e]), __uint_as_float(f0[2 * e + 1]));
+      pk[8 + e] = pack_bf16(__uint_as_float(f1[2 * e]), __uint_as_float(f1[2 * e + 1]));
     }
     tmem_st16(tl + ST_SB + c / 2, pk);
     tmem_wait_st();
   }
   bool good = true;
-  if (HALF && mid_x) {
-    // S_mid^T = Sloc_half^T + S_start^T X_half^T (three bf16 products: hi hi, hi lo,
-    // lo hi; fp32 accumulation onto Sloc_half^T in TMEM); X_half is the B operand
-    // (N = row of X, K = column, MN-major images)
+  uint32_t mphase = 0;
+  // ---- pass C hops: S^T <- Sloc^T + S^T X^T (three bf16 products: hi hi, hi lo, lo hi;
+  // fp32 accumulation onto Sloc^T in TMEM); X is the B operand (N = row of X, K =
+  // column, MN-major images), S^T's hi / lo parts the A operands
+#pragma unroll 1
+  for (int hh = 0; hh < nhop && good; ++hh) {
+    const float* lp = hop_l(hh);
+#pragma unroll 1
+    for (int hf = 0; hf < 2; ++hf) {                 // 16 of this thread's 32 columns at a time
+      const int c = 32 * wq + 16 * hf;
+      float cur[16];
+      if (hh == 0) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          cur[e] = c + e < dk && j < dv ? hop0[(long long)(c + e) * dv + j] : 0.f;
+      } else {
+        uint32_t t[16];
+        tmem_ld16(tl + ST_S + c, t);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) cur[e] = __uint_as_float(t[e]);
+      }
+      uint32_t hi[8], lo[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        hi[e] = pack_bf16(cur[2 * e], cur[2 * e + 1]);
+        lo[e] = pack_bf16(cur[2 * e] - bf_lo(hi[e]), cur[2 * e + 1] - bf_hi(hi[e]));
+      }
+      tmem_st8(tl + ST_SB + c / 2, hi);
+      tmem_st8(tl + ST_LO + c / 2, lo);
+      uint32_t f[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        f[e] = __float_as_uint(c + e < dk && j < dv ? lp[(long long)(c + e) * dv + j] : 0.f);
+      tmem_st16(tl + ST_S + c, f);
+      tmem_wait_st();
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (tid == 0) {
-      good = mbar_wait(&xbar, 0, kWaitLimit);
+      good = mbar_wait(&full[hh & 1], (hh >> 1) & 1, kWaitLimit);
       if (good) {
+        waited = hh + 1;
         tc_fence_after();
-        const uint32_t xh = smem_u32(sm + S_BUF), xl = xh + 32768u;
+        const uint32_t xh = smem_u32(sm + (hh & 1) * S_BUF), xl = xh + 32768u;
         const uint32_t id = idesc_bf16(128, 128, false, true);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -1163,44 +1184,46 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
           mma_ts(tb + ST_S, tb + ST_SB + kk * 8, bl, id, 1);
           mma_ts(tb + ST_S, tb + ST_LO + kk * 8, bh, id, 1);
         }
-        mma_commit(&xbar);
-        xstate = 2;
+        mma_commit(&mbar);
       }
     }
     __syncwarp();
-    good = __syncthreads_or(!good) == 0;
-    if (good) good = mbar_wait(&xbar, 1, kWaitLimit);
+    if (__syncthreads_or(!good)) { good = false; break; }
+    good = warp != 0 || mbar_wait(&mbar, mphase, kWaitLimit);
+    mphase ^= 1u;
+    if (__syncthreads_or(!good)) { good = false; break; }
     tc_fence_after();
-    good = __syncthreads_or(!good) == 0;
-    if (good) {                         // the bf16 copy of S_mid for the first product
-      uint32_t t[2][16], pk[16];
-      tmem_ld16(tl + ST_S + 32 * wq, t[0]);
-      tmem_ld16(tl + ST_S + 32 * wq + 16, t[1]);
-      tmem_wait_ld();
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        pk[e] = pack_bf16(__uint_as_float(t[0][2 * e]), __uint_as_float(t[0][2 * e + 1]));
-        pk[8 + e] = pack_bf16(__uint_as_float(t[1][2 * e]), __uint_as_float(t[1][2 * e + 1]));
-      }
-      tmem_st16(tl + ST_SB + 16 * wq, pk);
-      tmem_wait_st();
-      if (tid == 0 && nch >= 2) {       // the images are consumed: record 1 into buffer 1
-        mbar_arrive_expect_tx(&full[1], REC_BYTES);
-        bulk_g2s(sm + S_BUF, rec_ptr(1), REC_BYTES, &full[1]);
-        issued = 2;
-      }
+    // this hop's buffer is consumed: the next load into it
+    if (tid == 0 && issued < nload) {
+      fence_async_smem();
+      issue_load(issued);
+      ++issued;
     }
   }
-  good = good && (nch == 0 || mbar_wait(&full[0], 0, kWaitLimit));
+  if (nhop > 0 && good) {               // the bf16 copy of the start state for the first product
+    uint32_t t[2][16], pk[16];
+    tmem_ld16(tl + ST_S + 32 * wq, t[0]);
+    tmem_ld16(tl + ST_S + 32 * wq + 16, t[1]);
+    tmem_wait_ld();
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      pk[e] = pack_bf16(__uint_as_float(t[0][2 * e]), __uint_as_float(t[0][2 * e + 1]));
+      pk[8 + e] = pack_bf16(__uint_as_float(t[1][2 * e]), __uint_as_float(t[1][2 * e + 1]));
+    }
+    tmem_st16(tl + ST_SB + 16 * wq, pk);
+    tmem_wait_st();
+  }
+  if (good && nch > 0 && warp == 0) {
+    good = mbar_wait(&full[nhop & 1], (nhop >> 1) & 1, kWaitLimit);
+    if (good) waited = nhop + 1;
+  }
   tc_fence_before();
   bool alive = __syncthreads_or(!good) == 0;
   tc_fence_after();
 
-  uint32_t mphase = 0;
-  int waited = alive && nch > 0 ? 1 : 0;             // records whose arrival has been seen
 #pragma unroll 1
   for (int i = 0; i < nch && alive; ++i) {
-    const int buf = i & 1;
+    const int buf = (nhop + i) & 1;               // load nhop + i (see above)
     uint8_t* rb = sm + buf * S_BUF;
     const long long t0 = t_beg + (long long)i * C;
     const int L = (int)min((long long)C, t_end - t0);
@@ -1250,11 +1273,13 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
       }
       tmem_wait_st();
     }
+    // warp 0 (whose thread 0 issued the MMAs) polls; the other warps wait in the CTA
+    // barrier, so no spinning warp takes issue slots from the MMA issue
     tc_fence_before();
-    good = mbar_wait(&mbar, mphase, kWaitLimit);
+    good = warp != 0 || mbar_wait(&mbar, mphase, kWaitLimit);
     mphase ^= 1u;
-    tc_fence_after();
     if (__syncthreads_or(!good)) { alive = false; break; }
+    tc_fence_after();
 
     // ---- Delta^T = U^T - P for tokens [16 wq, 16 wq + 16) -> f16 TMEM
     {
@@ -1292,10 +1317,10 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
       mma_commit(&mbar);
     }
     __syncwarp();
-    good = mbar_wait(&mbar, mphase, kWaitLimit);
+    good = warp != 0 || mbar_wait(&mbar, mphase, kWaitLimit);
     mphase ^= 1u;
-    tc_fence_after();
     if (__syncthreads_or(!good)) { alive = false; break; }
+    tc_fence_after();
 
     // the record in this buffer is consumed: fetch record i + 2 into it
     if (i + 2 < nch) {
@@ -1331,9 +1356,10 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
     }
     tc_fence_before();
     good = true;
-    if (i + 1 < nch) {
-      good = mbar_wait(&full[(i + 1) & 1], ((i + 1) >> 1) & 1, kWaitLimit);
-      if (good) waited = i + 2;
+    if (i + 1 < nch && warp == 0) {
+      const int li = nhop + i + 1;
+      good = mbar_wait(&full[li & 1], (li >> 1) & 1, kWaitLimit);
+      if (good) waited = li + 1;
     }
     if (__syncthreads_or(!good)) { alive = false; break; }
     tc_fence_after();
@@ -1369,8 +1395,8 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
       tmem_ld16(tl + ST_S + 32 * wq + 16, t[1]);
       tmem_wait_ld();
       if (init_identity) {
-        // a transition X_p: bf16 hi / lo images for the segment combine (MN-major
-        // SW128 A operand, M = row of X, K = column; TMEM lane j holds column j of X)
+        // a transition X_p: bf16 hi / lo images for pass C's hops (MN-major SW128
+        // B operand, N = row of X, K = column; TMEM lane j holds column j of X)
         uint8_t* xb = reinterpret_cast<uint8_t*>(fin);
 #pragma unroll
         for (int c8 = 0; c8 < 4; ++c8) {
@@ -1397,7 +1423,6 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
     atomicExch(&g_chunk_split_timeout, 1);
     // let the MMA and the copies still in flight finish before the CTA exits
     mbar_wait(&mbar, mphase ^ 1u, kWaitLimit);
-    if (HALF && xstate >= 1) mbar_wait(&xbar, xstate - 1, kWaitLimit);   // images, or MMAs on them
     for (int r = waited; r < issued; ++r) mbar_wait(&full[r & 1], (r >> 1) & 1, kWaitLimit);
   }
   tc_fence_before();
@@ -1426,8 +1451,9 @@ bool set_attrs() {
 // Cost model in units of one state-pass chunk step: pass A runs NH*(2P-3)
 // chains, each G chunks long, in waves of one chain per SM; pass C runs NH*(P-1)
 // chains of G chunks, or with half points NH*(2(P-2)+1) chains of at most
-// max(Gh, last segment) chunks; the combine costs kCombine steps per segment and
-// a second-half chain's start (its S_mid product) kMid steps.
+// max(Gh, last segment) chunks; chaining the segments' states (pass C's hops, about
+// one chunk step each, on the deepest chain) is charged kCombine steps per segment
+// and a second-half chain's extra hop (to S_mid) kMid steps.
 constexpr double kCombine = 2.5;
 constexpr double kMid = 1.0;
 struct SplitPlan {
@@ -1591,15 +1617,14 @@ cudaError_t launch_chunk_split(const void* q, const void* k, const void* v, cons
                           grid, dim3(NT_S), STATE_SMEM, stream, rec, h0, cu_seqlens, ob, hT, T, H, dk,
                           dv, nslots, sa, gt);
     };
+    // pass A, then pass C, whose chains chain the segments' states themselves
     cudaError_t es = cudaSuccess;
     KDA_TIMED(KDA_KERNEL_STATE, stream, es = state_pass(dim3(H, B, 2 * P)));
-    const cudaError_t ec = launch_seg_combine_img(cu_seqlens, B, T, H, dk, dv, sa, stream);
     sa.pass = 2;
     const unsigned zc = (unsigned)(sa.half > 0 ? 2 * (P - 1) : P - 1);
     const cudaError_t es2 = es;
     KDA_TIMED(KDA_KERNEL_STATE, stream, es = state_pass(dim3(H, B, zc)));
     note_launches(2);
-    if (ec != cudaSuccess) e = ec;
     if (es2 != cudaSuccess) e = es2;
     if (es != cudaSuccess) e = es;
   }

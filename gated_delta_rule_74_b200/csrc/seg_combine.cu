@@ -190,169 +190,6 @@ kda_seg_combine_kernel(const int32_t* __restrict__ cu_seqlens, int T, int H, Seg
   }
 }
 
-// The same chain for the split prefill, where the transition chains leave X_p
-// as ready tensor-core operands: bf16 hi and lo images of X_p (32 KB each,
-// MN-major SW128, M = row i of X, K = column) in X_p's scratch slot, and
-// S_start / Sloc as fp32 [dk][dv] rows.  The dv columns are independent, so
-// each (sequence, head) runs four CTAs (blockIdx.z), each owning 32 columns:
-//   D [128 x 32] = (Xh Sh + Xh Sl + Xl Sh)[:, cols] + Sloc_p[:, cols]
-// with the next X_p bulk-copied into shared memory while the current step runs.
-constexpr int kQCols = 32;
-constexpr uint32_t C2_X = 0;                 // two buffers of [Xhi | Xlo], 64 KB each
-constexpr uint32_t C2_BH = 131072;           // S_start[:, cols] hi, MN-major SW32 (K = 128, N = 32)
-constexpr uint32_t C2_BL = C2_BH + 8192;     // ... lo
-constexpr size_t kCombine2Smem = 131072 + 16384 + 1024;
-constexpr uint32_t kWait2 = 1u << 22;
-
-__global__ void __launch_bounds__(kCombineThreads, 1)
-kda_seg_combine_img_kernel(const int32_t* __restrict__ cu_seqlens, int T, int H, int dk, int dv,
-                           SegArgs sa) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                           ~uintptr_t(1023));
-  __shared__ uint64_t xfull[2], mbar;
-  __shared__ uint32_t tmem_base_sh;
-  // launched right behind pass A: wait for its X_p and Sloc_p; pass C may start
-  // taking free SMs (it reads the combine's output only after its own wait)
-  grid_dep_launch();
-  grid_dep_wait();
-  const int h = blockIdx.x, s = blockIdx.y, col0 = kQCols * blockIdx.z;
-  if (col0 >= dv) return;
-  long long r0, a, b;
-  seq_range(cu_seqlens, s, T, r0, a, b);
-  const int Ps = seg_count(b - a, sa.G);
-  if (Ps <= 2) return;
-  const int base = seg_slot_base(cu_seqlens, s, T, sa.G);
-  if (base + Ps - 1 > sa.slots) return;                    // offsets beyond the planned scratch
-  const int tid = threadIdx.x, warp = tid >> 5, i = tid;    // thread i: row i of S / lane i
-  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-  auto slot = [&](int p) { return ((long long)(base + p) * H + h) * D * D; };
-  const bool row_ok = i < dk;
-
-  // S rows are fp32 [dk][dv]; thread i holds S[i][col0 .. col0 + 31]
-  auto load_row = [&](const float* src, float (&x)[kQCols]) {
-#pragma unroll
-    for (int c4 = 0; c4 < kQCols / 4; ++c4) {
-      const float4 v = row_ok ? *reinterpret_cast<const float4*>(src + (long long)i * dv + col0 + 4 * c4)
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
-      x[4 * c4] = v.x; x[4 * c4 + 1] = v.y; x[4 * c4 + 2] = v.z; x[4 * c4 + 3] = v.w;
-    }
-  };
-  // B operand (K = row i of S, N = the 32 columns): hi / lo parts, MN-major SW32
-  auto store_b = [&](const float (&x)[kQCols]) {
-#pragma unroll
-    for (int c8 = 0; c8 < kQCols / 8; ++c8) {
-      uint32_t hw[4], lw[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) split2(x[8 * c8 + 2 * e], x[8 * c8 + 2 * e + 1], hw[e], lw[e]);
-      const uint32_t o = chunk_mnmajor_sw32(c8, i, D);
-      *reinterpret_cast<uint4*>(sm + C2_BH + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-      *reinterpret_cast<uint4*>(sm + C2_BL + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-    }
-  };
-
-  if (warp == 0) {
-    tmem_alloc(&tmem_base_sh, kQCols);
-    tmem_relinquish();
-  }
-  if (tid == 0) {
-    mbar_init(&xfull[0], 1);
-    mbar_init(&xfull[1], 1);
-    mbar_init(&mbar, 1);
-    fence_mbar_init();
-  }
-  __syncthreads();
-  const uint8_t* xsrc = reinterpret_cast<const uint8_t*>(sa.xbuf);
-  if (tid == 0) {
-    mbar_arrive_expect_tx(&xfull[0], 65536);
-    bulk_g2s(sm + C2_X, xsrc + slot(1) * 4, 65536, &xfull[0]);
-  }
-  {
-    float x[kQCols];
-    load_row(sa.sbuf + slot(0), x);                        // S_start,1 = S_end,0
-    store_b(x);
-  }
-  fence_async_smem();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tb = tmem_base_sh;
-  const uint32_t idesc = idesc_bf16(128, kQCols, true, true);
-  uint32_t mphase = 0;
-  int waited = 0, issued = 1;                              // X copies seen / requested
-  bool ok = true;
-#pragma unroll 1
-  for (int p = 1; p <= Ps - 2; ++p) {
-    const int buf = (p - 1) & 1;
-    // the other buffer held X_{p-1}, consumed by the previous step's MMAs
-    if (tid == 0 && p + 1 <= Ps - 2) {
-      mbar_arrive_expect_tx(&xfull[p & 1], 65536);
-      bulk_g2s(sm + C2_X + (uint32_t)(p & 1) * 65536u, xsrc + slot(p + 1) * 4, 65536,
-               &xfull[p & 1]);
-      ++issued;
-    }
-    float loc[kQCols];
-    float* Sp = sa.sbuf + slot(p);
-    load_row(Sp, loc);                                     // Sloc_p
-    bool good = mbar_wait(&xfull[buf], (uint32_t)((p - 1) >> 1) & 1u, kWait2);
-    if (good) waited = p;
-    if (__syncthreads_or(!good)) { ok = false; break; }
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t ah = smem_u32(sm + C2_X + (uint32_t)buf * 65536u), al = ah + 32768u;
-      const uint32_t bh = smem_u32(sm + C2_BH), bl = smem_u32(sm + C2_BL);
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint64_t dah = desc_mnmajor_sw128(ah, D, kk), dal = desc_mnmajor_sw128(al, D, kk);
-        const uint64_t dbh = desc_mnmajor_sw32(bh, D, kk), dbl = desc_mnmajor_sw32(bl, D, kk);
-        mma_ss(tb, dah, dbh, idesc, kk > 0);
-        mma_ss(tb, dah, dbl, idesc, 1);
-        mma_ss(tb, dal, dbh, idesc, 1);
-      }
-      mma_commit(&mbar);
-    }
-    __syncwarp();
-    good = mbar_wait(&mbar, mphase, kWait2);
-    mphase ^= 1u;
-    tc_fence_after();
-    if (__syncthreads_or(!good)) { ok = false; break; }
-    // S_start,p+1 = X_p S_start,p + Sloc_p: row i from TMEM lane i
-    float x[kQCols];
-    {
-      uint32_t t0[16], t1[16];
-      tmem_ld16(tb + lane_base, t0);
-      tmem_ld16(tb + lane_base + 16, t1);
-      tmem_wait_ld();
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        x[e] = __uint_as_float(t0[e]) + loc[e];
-        x[16 + e] = __uint_as_float(t1[e]) + loc[16 + e];
-      }
-    }
-    if (row_ok) {
-#pragma unroll
-      for (int c4 = 0; c4 < kQCols / 4; ++c4)
-        *reinterpret_cast<float4*>(Sp + (long long)i * dv + col0 + 4 * c4) =
-            make_float4(x[4 * c4], x[4 * c4 + 1], x[4 * c4 + 2], x[4 * c4 + 3]);
-    }
-    if (p + 1 <= Ps - 2) store_b(x);
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-  }
-  if (!ok && tid == 0) {
-    atomicExch(&g_seg_combine_timeout, 1);
-    mbar_wait(&mbar, mphase ^ 1u, kWait2);
-    for (int r = waited + 1; r <= issued; ++r) mbar_wait(&xfull[(r - 1) & 1], (uint32_t)((r - 1) >> 1) & 1u, kWait2);
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) {
-    tc_fence_after();
-    tmem_dealloc(tb, kQCols);
-  }
-}
-
 }  // namespace
 
 cudaError_t launch_seg_combine(const int32_t* cu_seqlens, int B, int T, int H, const SegArgs& sa,
@@ -373,22 +210,6 @@ cudaError_t launch_seg_combine(const int32_t* cu_seqlens, int B, int T, int H, c
 }  // namespace kda
 
 namespace kda {
-
-cudaError_t launch_seg_combine_img(const int32_t* cu_seqlens, int B, int T, int H, int dk, int dv,
-                                   const SegArgs& sa, cudaStream_t stream) {
-  if (!once_per_device(kOnceCombineImg, []() {
-        return cudaFuncSetAttribute(kda_seg_combine_img_kernel,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)kCombine2Smem) == cudaSuccess;
-      }))
-    return cudaErrorInvalidDevice;
-  cudaError_t e = cudaSuccess;
-  KDA_TIMED(KDA_KERNEL_COMBINE, stream,
-            e = launch_after(kda_seg_combine_img_kernel, dim3(H, B, dv / kQCols), dim3(kCombineThreads),
-                             kCombine2Smem, stream, cu_seqlens, T, H, dk, dv, sa));
-  note_launches(1);
-  return e;
-}
 
 // Reads (and with reset clears) g_seg_combine_timeout; host side of kda_device_status.
 cudaError_t take_combine_timeout(int* flag, bool reset) {

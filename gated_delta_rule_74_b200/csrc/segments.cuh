@@ -18,7 +18,9 @@ constexpr int kHead = 128;     // dk = dv handled by the tensor-core kernels
 //           Sloc_p; further chains run segments 1 <= p <= Ps-2 from the
 //           identity with the write term dropped (U = 0), which yields the
 //           segment's transition X_p (S_end = X_p S_start + Sloc_p);
-//   combine S_start,1 = S_end,0 and S_start,p+1 = X_p S_start,p + Sloc_p (fp32);
+//   combine S_start,1 = S_end,0 and S_start,p+1 = X_p S_start,p + Sloc_p (fp32):
+//           a separate launch in the single-kernel prefill; in the split prefill
+//           each pass C chain forms its own S_start,p from pass A's results;
 //   pass C  segments p >= 1 run again from S_start,p and write their outputs;
 //           the last one writes hT.
 // With a half point Gh (split prefill), the pass A chains of segments 1 .. Ps-2
@@ -32,7 +34,8 @@ struct SegArgs {
   int P;          // segment slots per sequence in the grid (z extent of pass C)
   int pass;       // 0 = single pass, 1 = pass A, 2 = pass C
   int slots;      // number of (segment) slots the scratch holds per head
-  float* sbuf;    // [slots][H][D][D] fp32: Sloc_p, then S_start,p+1
+  float* sbuf;    // [slots][H][D][D] fp32: Sloc_p (the single-kernel prefill's combine
+                  // then overwrites it with S_start,p+1)
   float* xbuf;    // [slots][H][D][D] fp32: X_p
   int half;       // Gh: chunks of the first pass C chain of a split segment (0 = no split)
   float* sbuf_h;  // [slots][H][D][D] fp32: Sloc_half,p
@@ -92,13 +95,10 @@ __host__ __forceinline__ long long chunk_slots(int B, int T, bool varlen) {
 // that keeps its memory between calls.  Returns false without a usable device.
 bool device_ctx(int* sms, cudaMemPool_t* pool);
 
-// Segment combine (one launch): S_start,p+1 = X_p S_start,p + Sloc_p in place.
-// launch_seg_combine: X_p and the states as fp32 [128][128] (single-kernel prefill);
-// launch_seg_combine_img: X_p as bf16 hi/lo MMA operand images, states as fp32
-// [dk][dv] rows (split prefill).
+// Segment combine of the single-kernel prefill (one launch):
+// S_start,p+1 = X_p S_start,p + Sloc_p in place, with X_p and the states as fp32
+// [128][128].  (The split prefill chains the segments inside its pass C instead.)
 cudaError_t launch_seg_combine(const int32_t* cu_seqlens, int B, int T, int H, const SegArgs& sa,
                                cudaStream_t stream);
-cudaError_t launch_seg_combine_img(const int32_t* cu_seqlens, int B, int T, int H, int dk, int dv,
-                                   const SegArgs& sa, cudaStream_t stream);
 
 }  // namespace kda
