@@ -204,6 +204,57 @@ __device__ __noinline__ void prep_unsafe_direct(uint8_t* sm, uint8_t* rc, int a,
   }
 }
 
+// UnsafeRows of this thread's channel pair and block a, re-read from the inputs in
+// global memory (other warps may already be overwriting the staged tiles), with
+// the cumulative decay summed in the prep kernel's order; d1..d3, rel: P_{a2} - P_a
+// + g_{16a} and the decay of blocks a..3 (per channel); gsh: one decay per group of
+// 2^gsh channels.
+__device__ __noinline__ void fill_unsafe_rows(UnsafeRows& ur, const float* __restrict__ g,
+                                              const bf16* __restrict__ k,
+                                              const bf16* __restrict__ q, long long rbase, int H,
+                                              int h, int dk, int gsh, int L, int a, int c0,
+                                              float2 d1, float2 d2, float2 d3, float2 rel) {
+  float2 loc = make_float2(0.f, 0.f), first = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const int r = 16 * a + e;
+    float2 gv = make_float2(0.f, 0.f);
+    uint32_t kv = 0u, qv = 0u;
+    if (r < L && c0 < dk) {
+      const long long idx = ((rbase + r) * H + h) * dk + c0;
+      kv = *reinterpret_cast<const uint32_t*>(k + idx);
+      qv = *reinterpret_cast<const uint32_t*>(q + idx);
+      if (gsh != 0) {                          // g [rows, H, dk >> gsh]
+        const float t = g[((rbase + r) * H + h) * (dk >> gsh) + (c0 >> gsh)];
+        gv = make_float2(t, t);
+      } else {
+        gv = *reinterpret_cast<const float2*>(g + idx);
+      }
+    }
+    if (e == 0) {
+      loc = gv;
+      first = gv;
+    } else {
+      loc.x += gv.x;
+      loc.y += gv.y;
+    }
+    ur.x[0][e] = loc.x - first.x;
+    ur.x[1][e] = loc.y - first.y;
+    ur.k[0][e] = bf_lo(kv);
+    ur.k[1][e] = bf_hi(kv);
+    ur.q[0][e] = bf_lo(qv);
+    ur.q[1][e] = bf_hi(qv);
+  }
+  const float2 dd[4] = {make_float2(0.f, 0.f), d1, d2, d3};
+#pragma unroll
+  for (int a2 = 0; a2 < 4; ++a2) {
+    ur.d[0][a2] = dd[a2].x - first.x;
+    ur.d[1][a2] = dd[a2].y - first.y;
+  }
+  ur.tl[0] = rel.x - first.x;
+  ur.tl[1] = rel.y - first.y;
+}
+
 // The exact within-block pair terms of this thread's unsafe channels (c0, c0 + 1;
 // flags ux, uy) of one 16-row block, added to the block's corrections (A, Aqk:
 // [r][i], row stride 16).  Warp-cooperative.  Reloads the block's rows: g (one
@@ -372,35 +423,45 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   float2 gq[16];
   uint32_t kw[16], qw[16];
   float2 kf[CONV ? 16 : 1], qf[CONV ? 16 : 1];   // CONV: fp32 convolution outputs
+  // branch-free loops per source, so that all of a thread's loads issue back to back
+  if (use_tma) {                                 // staged tiles: row stride dk
 #pragma unroll
-  for (int e = 0; e < 16; ++e) {
-    const int r = 16 * a + e;
-    if (r < L && c0 < dk) {
-      const long long idx = ((rbase + r) * H + h) * dk + c0;
-      if (use_tma) {                             // staged tiles: row stride dk
-        const int si = r * dk + c0;
-        if (gsh == 0) gq[e] = *reinterpret_cast<const float2*>(sm + Q_R + 4 * si);
-        kw[e] = *reinterpret_cast<const uint32_t*>(sm + Q_L + 16384 + 2 * si);
-        qw[e] = *reinterpret_cast<const uint32_t*>(sm + Q_L + 2 * si);
-      }
-      if (!use_tma || gsh != 0) {
-        if (gsh == 0) {
-          gq[e] = __ldg(reinterpret_cast<const float2*>(g + idx));
-        } else {                                 // one decay per group of 2^gsh channels
-          const float gg = __ldg(g + ((rbase + r) * H + h) * (dk >> gsh) + (c0 >> gsh));
-          gq[e] = make_float2(gg, gg);
-        }
-      }
-      if constexpr (!CONV) {
-        if (!use_tma) {
+    for (int e = 0; e < 16; ++e) {
+      const int r = 16 * a + e;
+      const bool ok = r < L && c0 < dk;
+      const int si = ok ? r * dk + c0 : 0;
+      const float2 gv = *reinterpret_cast<const float2*>(sm + Q_R + 4 * si);
+      const uint32_t kv = *reinterpret_cast<const uint32_t*>(sm + Q_L + 16384 + 2 * si);
+      const uint32_t qv = *reinterpret_cast<const uint32_t*>(sm + Q_L + 2 * si);
+      gq[e] = ok ? gv : make_float2(0.f, 0.f);
+      kw[e] = ok ? kv : 0u;
+      qw[e] = ok ? qv : 0u;
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const int r = 16 * a + e;
+      if (r < L && c0 < dk) {
+        const long long idx = ((rbase + r) * H + h) * dk + c0;
+        if (gsh == 0) gq[e] = __ldg(reinterpret_cast<const float2*>(g + idx));
+        if constexpr (!CONV) {
           kw[e] = __ldg(reinterpret_cast<const unsigned int*>(k + idx));
           qw[e] = __ldg(reinterpret_cast<const unsigned int*>(q + idx));
         }
+      } else {
+        gq[e] = make_float2(0.f, 0.f);
+        kw[e] = 0u;
+        qw[e] = 0u;
       }
-    } else {
-      gq[e] = make_float2(0.f, 0.f);
-      kw[e] = 0u;
-      qw[e] = 0u;
+    }
+  }
+  if (gsh != 0) {                                // one decay per group of 2^gsh channels
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const int r = 16 * a + e;
+      float gg = 0.f;
+      if (r < L && c0 < dk) gg = __ldg(g + ((rbase + r) * H + h) * (dk >> gsh) + (c0 >> gsh));
+      gq[e] = make_float2(gg, gg);
     }
   }
   if constexpr (CONV) {
@@ -512,10 +573,17 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     else return ch ? qf[idx].y : qf[idx].x;
   };
 
-  if (ux || uy) {
-    // unsafe channels: their operands are formed out of line (the loop below skips
-    // their R and Kend stores); the values go over on the stack, so the common
-    // path's registers are untouched
+  if (!CONV && (ux || uy)) {
+    // unsafe channels: their operands are formed out of line from the block's rows,
+    // re-read from global memory (the loop below skips their R and Kend stores);
+    // nothing of this stays in the common path
+    UnsafeRows ur;
+    fill_unsafe_rows(ur, g, k, q, rbase, H, h, dk, gsh, L, a, c0, d[1], d[2], d[3], rel);
+    prep_unsafe_direct(sm, rc, a, c0, (ux ? 1 : 0) | (uy ? 2 : 0), false, ur);
+  }
+  if (CONV && (ux || uy)) {
+    // fused convolution: the normalised q, k exist only in registers, so they go
+    // over on the stack
     UnsafeRows ur;
 #pragma unroll
     for (int ch = 0; ch < 2; ++ch) {
