@@ -671,11 +671,15 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   // ---- P2: Gram (one MMA per K step, N = 160)
   if (tid == 0) {
     tc_fence_after();
-    const uint32_t l_base = smem_u32(sm + Q_L), r_base = smem_u32(sm + q_r(0));
     const uint32_t idesc = idesc_bf16(128, 160, true, true);
-    for (int kk = 0; kk < dk / 16; ++kk)       // channels < dk (64-wide heads: half the steps)
-      mma_ss(tb + PT_G, desc_mnmajor_sw128(l_base, D, kk), desc_mnmajor_sw32(r_base, D, kk), idesc,
-             kk > 0);
+    // K step kk: 2048 bytes further in L, 512 in R (descriptor address fields)
+    const uint64_t a0 = desc_mnmajor_sw128(smem_u32(sm + Q_L), D, 0);
+    const uint64_t b0 = desc_mnmajor_sw32(smem_u32(sm + q_r(0)), D, 0);
+    const int nk = dk / 16;                    // channels < dk (64-wide heads: half the steps)
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk)
+      if (kk < nk)
+        mma_ss(tb + PT_G, a0 + (uint64_t)(kk * 128), b0 + (uint64_t)(kk * 32), idesc, kk > 0);
     mma_commit(&bar);
   }
   __syncwarp();
@@ -902,11 +906,14 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       const uint32_t v_base = smem_u32(sm + Q_V);
       const uint32_t id_w = idesc_bf16(128, 64, false, false);
       const uint32_t id_u = idesc_bf16(128, 64, true, false);
+      // K step kk: 32 bytes further along the K-major rows, 2048 in the MN-major V
+      const uint64_t bt0 = desc_kmajor_sw128(tb_base, C, 0), kb0 = desc_kmajor_sw128(kb_base, D, 0);
+      const uint64_t v0 = desc_mnmajor_sw128(v_base, C, 0);
 #pragma unroll
       for (int kk = 0; kk < C / 16; ++kk) {
-        const uint64_t bt = desc_kmajor_sw128(tb_base, C, kk);
-        mma_ss(tb + PT_W, desc_kmajor_sw128(kb_base, D, kk), bt, id_w, kk > 0);
-        mma_ss(tb + PT_U, desc_mnmajor_sw128(v_base, C, kk), bt, id_u, kk > 0);
+        const uint64_t bt = bt0 + (uint64_t)(kk * 2);
+        mma_ss(tb + PT_W, kb0 + (uint64_t)(kk * 2), bt, id_w, kk > 0);
+        mma_ss(tb + PT_U, v0 + (uint64_t)(kk * 128), bt, id_u, kk > 0);
       }
       mma_commit(&bar);
     }
@@ -1245,9 +1252,10 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
         tc_fence_after();
         const uint32_t xh = smem_u32(sm + (hh & 1) * S_BUF), xl = xh + 32768u;
         const uint32_t id = idesc_bf16(128, 128, false, true);
+        const uint64_t bh0 = desc_mnmajor_sw128(xh, D, 0), bl0 = desc_mnmajor_sw128(xl, D, 0);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t bh = desc_mnmajor_sw128(xh, D, kk), bl = desc_mnmajor_sw128(xl, D, kk);
+        for (int kk = 0; kk < D / 16; ++kk) {   // K step kk: 2048 bytes further
+          const uint64_t bh = bh0 + (uint64_t)(kk * 128), bl = bl0 + (uint64_t)(kk * 128);
           mma_ts(tb + ST_S, tb + ST_SB + kk * 8, bh, id, 1);
           mma_ts(tb + ST_S, tb + ST_SB + kk * 8, bl, id, 1);
           mma_ts(tb + ST_S, tb + ST_LO + kk * 8, bh, id, 1);
@@ -1309,19 +1317,18 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
     }
 
     // ---- [O^T | P] = S^T [Qbar^T | W^T]^T   (P only when no outputs are kept)
+    // The issue loop is kept to the MMA instructions alone: the descriptor of K step
+    // kk is the first one plus kk * 2048 bytes in its address field.
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t qw = smem_u32(rb + REC_QW);
-      if (outputs) {
-        const uint32_t id = idesc_bf16(128, 128, false, true);
-        for (int kk = 0; kk < dk / 16; ++kk)   // channels < dk
-          mma_ts(tb + ST_O, tb + ST_SB + kk * 8, desc_mnmajor_sw128(qw, D, kk), id, kk > 0);
-      } else {
-        const uint32_t id = idesc_bf16(128, 64, false, true);
-        for (int kk = 0; kk < dk / 16; ++kk)
-          mma_ts(tb + ST_P, tb + ST_SB + kk * 8, desc_mnmajor_sw128(qw + 16384, D, kk), id,
-                 kk > 0);
-      }
+      const uint64_t b0 = desc_mnmajor_sw128(smem_u32(rb + REC_QW) + (outputs ? 0u : 16384u), D, 0);
+      const uint32_t dst = tb + (outputs ? ST_O : ST_P);
+      const uint32_t id = outputs ? idesc_bf16(128, 128, false, true) : idesc_bf16(128, 64, false, true);
+      const int nk = dk / 16;                  // channels < dk
+      mma_ts(dst, tb + ST_SB, b0, id, 0);
+#pragma unroll
+      for (int kk = 1; kk < D / 16; ++kk)
+        if (kk < nk) mma_ts(dst, tb + ST_SB + kk * 8, b0 + (uint64_t)(kk * 128), id, 1);
       mma_commit(&mbar);
     }
     __syncwarp();
@@ -1376,12 +1383,13 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
     // ---- [S^T | O^T] += Delta^T [Kend^T ; Aqk]^T
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t ka = smem_u32(rb + REC_KA);
       const int n = outputs ? D + C : D;
       const uint32_t id = idesc_f16(128, n, false, false);   // f16 A (Delta^T) and B
+      // K step kk: 32 bytes further along the 128-byte rows
+      const uint64_t b0 = desc_kmajor_sw128(smem_u32(rb + REC_KA), n, 0);
 #pragma unroll
       for (int kk = 0; kk < C / 16; ++kk)
-        mma_ts(tb + ST_S, tb + ST_D + kk * 8, desc_kmajor_sw128(ka, n, kk), id, 1);
+        mma_ts(tb + ST_S, tb + ST_D + kk * 8, b0 + (uint64_t)(kk * 2), id, 1);
       mma_commit(&mbar);
     }
     __syncwarp();
