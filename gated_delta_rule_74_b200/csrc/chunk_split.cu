@@ -296,7 +296,7 @@ __device__ __noinline__ void prep_unsafe_pairs(const float* __restrict__ g, long
 // projections; each is convolved causally per channel (width convW <= 4, history
 // reset at the document start), L2-normalised per token, and q scaled by dk^-1/2.
 // ============================================================================
-template <bool CONV>
+template <bool CONV, bool GRPD>
 __global__ void __launch_bounds__(NT, 2)
 kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
                       const bf16* __restrict__ v, const float* __restrict__ g,
@@ -380,6 +380,18 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     cp_async_commit();
   }
   if (tid < C) s_beta[tid] = tid < L ? beta[(rbase + tid) * H + h] : 0.f;
+  // ---- P1: per thread a channel pair (2cp, 2cp+1) and a 16-row block a
+  const int cp = tid & 63, a = tid >> 6, c0 = 2 * cp;
+  float2 gq[16];
+  if constexpr (GRPD) {                          // one decay per group of 2^gsh channels: its
+#pragma unroll                                   // loads go out before the tiles are waited for
+    for (int e = 0; e < 16; ++e) {
+      const int r = 16 * a + e;
+      float gg = 0.f;
+      if (r < L && c0 < dk) gg = __ldg(g + ((rbase + r) * H + h) * (dk >> gsh) + (c0 >> gsh));
+      gq[e] = make_float2(gg, gg);
+    }
+  }
   if (warp == 0) {
     tmem_alloc(&tmem_base_sh, kPrepTmemCols);
     tmem_relinquish();
@@ -418,9 +430,6 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     }
   }
 
-  // ---- P1: per thread a channel pair (2cp, 2cp+1) and a 16-row block a
-  const int cp = tid & 63, a = tid >> 6, c0 = 2 * cp;
-  float2 gq[16];
   uint32_t kw[16], qw[16];
   float2 kf[CONV ? 16 : 1], qf[CONV ? 16 : 1];   // CONV: fp32 convolution outputs
   // branch-free loops per source, so that all of a thread's loads issue back to back
@@ -430,10 +439,12 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       const int r = 16 * a + e;
       const bool ok = r < L && c0 < dk;
       const int si = ok ? r * dk + c0 : 0;
-      const float2 gv = *reinterpret_cast<const float2*>(sm + Q_R + 4 * si);
       const uint32_t kv = *reinterpret_cast<const uint32_t*>(sm + Q_L + 16384 + 2 * si);
       const uint32_t qv = *reinterpret_cast<const uint32_t*>(sm + Q_L + 2 * si);
-      gq[e] = ok ? gv : make_float2(0.f, 0.f);
+      if constexpr (!GRPD) {
+        const float2 gv = *reinterpret_cast<const float2*>(sm + Q_R + 4 * si);
+        gq[e] = ok ? gv : make_float2(0.f, 0.f);
+      }
       kw[e] = ok ? kv : 0u;
       qw[e] = ok ? qv : 0u;
     }
@@ -443,25 +454,16 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       const int r = 16 * a + e;
       if (r < L && c0 < dk) {
         const long long idx = ((rbase + r) * H + h) * dk + c0;
-        if (gsh == 0) gq[e] = __ldg(reinterpret_cast<const float2*>(g + idx));
+        if constexpr (!GRPD) gq[e] = __ldg(reinterpret_cast<const float2*>(g + idx));
         if constexpr (!CONV) {
           kw[e] = __ldg(reinterpret_cast<const unsigned int*>(k + idx));
           qw[e] = __ldg(reinterpret_cast<const unsigned int*>(q + idx));
         }
       } else {
-        gq[e] = make_float2(0.f, 0.f);
+        if constexpr (!GRPD) gq[e] = make_float2(0.f, 0.f);
         kw[e] = 0u;
         qw[e] = 0u;
       }
-    }
-  }
-  if (gsh != 0) {                                // one decay per group of 2^gsh channels
-#pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const int r = 16 * a + e;
-      float gg = 0.f;
-      if (r < L && c0 < dk) gg = __ldg(g + ((rbase + r) * H + h) * (dk >> gsh) + (c0 >> gsh));
-      gq[e] = make_float2(gg, gg);
     }
   }
   if constexpr (CONV) {
@@ -1512,9 +1514,11 @@ kda_state_pass_kernel(const uint8_t* __restrict__ rec, const float* h0,
 // Dynamic shared memory of the kernels, set once per device.
 bool set_attrs() {
   return once_per_device(kOnceSplit, []() {
-    return cudaFuncSetAttribute(kda_chunk_prep_kernel<false>,
+    return cudaFuncSetAttribute(kda_chunk_prep_kernel<false, false>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, PREP_SMEM) == cudaSuccess &&
-           cudaFuncSetAttribute(kda_chunk_prep_kernel<true>,
+           cudaFuncSetAttribute(kda_chunk_prep_kernel<false, true>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, PREP_SMEM) == cudaSuccess &&
+           cudaFuncSetAttribute(kda_chunk_prep_kernel<true, false>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, PREP_SMEM) == cudaSuccess &&
            cudaFuncSetAttribute(kda_state_pass_kernel<false>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, STATE_SMEM) == cudaSuccess &&
@@ -1663,12 +1667,13 @@ cudaError_t launch_chunk_split(const void* q, const void* k, const void* v, cons
     if (!tma) memset(&maps, 0, sizeof(maps));
     if (conv) {
       KDA_TIMED(KDA_KERNEL_PREP, stream,
-                kda_chunk_prep_kernel<true><<<dim3((unsigned)nslots, H), NT, PREP_SMEM, stream>>>(
+                kda_chunk_prep_kernel<true, false><<<dim3((unsigned)nslots, H), NT, PREP_SMEM, stream>>>(
                     qb, kb, vb, g, beta, cu_seqlens, rec, B, T, H, dk, dv, gsh, nslots,
                     fz->conv_q, fz->conv_k, fz->W, maps, 0));
     } else {
+      auto prep = gsh != 0 ? kda_chunk_prep_kernel<false, true> : kda_chunk_prep_kernel<false, false>;
       KDA_TIMED(KDA_KERNEL_PREP, stream,
-                kda_chunk_prep_kernel<false><<<dim3((unsigned)nslots, H), NT, PREP_SMEM, stream>>>(
+                prep<<<dim3((unsigned)nslots, H), NT, PREP_SMEM, stream>>>(
                     qb, kb, vb, g, beta, cu_seqlens, rec, B, T, H, dk, dv, gsh, nslots, nullptr,
                     nullptr, 0, maps, tma));
     }
