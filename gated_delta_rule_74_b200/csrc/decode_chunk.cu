@@ -57,6 +57,23 @@ constexpr uint32_t F_Q = 0, F_K = 1, F_V = 2, F_G = 3, F_U = 4, F_KP = 5, F_KM =
 constexpr uint32_t M_SMALL = M_F + 8 * LT * LDF * 4;   // A, Aqk, T (16 x 16 fp32 each), beta, gamma_last
 constexpr uint32_t DC_SMEM = M_SMALL + 3 * 256 * 4 + 64 + D * 4 + 1024;
 
+// The exact pairs of one half (tokens t0 .. t0 + 7) of channel c, when `unsafe`,
+// summed over the warp into the half's corrections (decay_pairs.cuh); the tiles
+// hold k, q and g (row stride LDF).  Out of line: it runs only for inputs with
+// strong decay and keeps its registers to itself.  Warp-cooperative.
+__device__ __noinline__ void decode_unsafe_pairs(const float* fk, const float* fq, const float* fg,
+                                                 int t0, int c, bool unsafe, float* cA, float* cQ,
+                                                 int lane) {
+  float al[8][1], kv[8][1], qv[8][1];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    al[e][0] = __expf(fg[(t0 + e) * LDF + c]);
+    kv[e][0] = unsafe ? fk[(t0 + e) * LDF + c] : 0.f;
+    qv[e][0] = unsafe ? fq[(t0 + e) * LDF + c] : 0.f;
+  }
+  add_pair_terms<1, 8>(al, kv, qv, cA, cQ, lane);
+}
+
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
@@ -213,17 +230,9 @@ kda_decode_chunk_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     if (t0 == 0) sGl[c] = __expf(gl);
     // this half's growing factor: e^(G - G_8) over tokens 0..7, e^(G_8 - G) over 8..15
     unsafe = (t0 == 0 ? G[0] - G[8] : G[8] - G[15]) > kUnsafeDecay;
-    if (__any_sync(0xffffffffu, unsafe)) {
-      // its pairs exactly (the factors below are zeroed for them); fG still holds g
-      float al[8][1], kv[8][1], qv[8][1];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        al[e][0] = __expf(fG[(t0 + e) * LDF + c]);
-        kv[e][0] = unsafe ? fk[(t0 + e) * LDF + c] : 0.f;
-        qv[e][0] = unsafe ? fq[(t0 + e) * LDF + c] : 0.f;
-      }
-      add_pair_terms<1, 8>(al, kv, qv, s_cA + t0 * LT + t0, s_cQ + t0 * LT + t0, lane);
-    }
+    // its pairs exactly (the factors below are zeroed for them); fG still holds g
+    if (__any_sync(0xffffffffu, unsafe))
+      decode_unsafe_pairs(fk, fq, fG, t0, c, unsafe, s_cA + t0 * LT + t0, s_cQ + t0 * LT + t0, lane);
     __syncthreads();
     float qb[8];                          // Qbar of these 8 tokens: one 16-byte chunk
 #pragma unroll
