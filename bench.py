@@ -12,6 +12,8 @@ kda_decode_step calls on the config-4 shape (N=256 sequences x H=96 heads,
 d=128, 1.61 GB of fp32 state), reported as GB/s of algorithmic traffic and as a
 fraction of the measured HBM peak.
 
+`prefill_noalloc` times the same prefill through kda_chunk_fwd_noalloc (the single-kernel
+path on the library's fixed scratch array) with its error against the oracle on two heads.
 `configs` times the other prefill workloads the same way (configs 0-3 of the
 workload table: fp32_t256, b16_t512_d64, packed_16k, t32k_h96), each with its
 fraction of the HBM roofline and the oracle timed on a bounded sample of it;
@@ -671,6 +673,73 @@ def decode_leg(args, world, rank, dev, stream, barrier, clocks, hbm, peak_kind):
             "gpu_launches": launches, "clocks": clocks.summary(mark0, clocks.mark())}
 
 
+def noalloc_leg(args, world, rank, dev, stream, barrier, hbm):
+    """The headline prefill through kda_chunk_fwd_noalloc (the single-kernel prefill on the
+    library's fixed scratch array): K timed calls on three resident input sets, and its
+    error against the float64 oracle on heads 0 and H-1 (rank 0)."""
+    import torch
+
+    import gated_delta_rule_74_b200 as kda
+    import kda_inputs as ki
+
+    spec = ki.PREFILL_SPECS[args.workload]
+    sets, xs = [], []
+    for i in range(3):
+        x = ki.make_prefill(spec, seed=rank_seed(spec.seed, rank, i))
+        d = {n: (t.to(dev) if isinstance(t, torch.Tensor) else t) for n, t in x.items()}
+        d["out"] = torch.empty_like(d["v"])
+        d["hT"] = torch.empty(x["B"], x["H"], x["dk"], x["dv"], device=dev)
+        sets.append(d)
+        xs.append(x)
+    x0 = sets[0]
+    rows = x0["T"] if x0["cu_seqlens"] is not None else x0["B"] * x0["T"]
+    s_in = 2 if x0["dtype"] == "bf16" else 4
+    bytes_call = prefill_bytes(rows, x0["H"], x0["dk"], x0["dv"], s_in, x0["B"],
+                               x0["h0"] is not None, True)
+
+    def call(i):
+        d = sets[i % 3]
+        kda.kda_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], h0=d["h0"],
+                          cu_seqlens=d["cu_seqlens"], out=d["out"], hT=d["hT"], stream=stream,
+                          noalloc=True)
+
+    for i in range(args.warmup):
+        call(i)
+    torch.cuda.synchronize()
+    barrier()
+    steps = max(3, min(args.steps, 50))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        call(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = _max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
+    gbs = bytes_call / (ms / 1e3) / 1e9
+    res = {"call": "kda_chunk_fwd_noalloc", "tokens_per_s": rows * world / (ms / 1e3),
+           "ms_per_call": ms, "algorithmic_bytes_per_call": bytes_call, "gbs": gbs,
+           "frac_of_hbm_peak": gbs / hbm}
+    if rank == 0 and not args.no_cpu_baseline:
+        import numpy as np
+        import oracle
+        oracle.build()
+        call(0)
+        torch.cuda.synchronize()
+        x, d = xs[0], sets[0]
+        H = x["H"]
+        err = {"out": 0.0, "hT": 0.0}
+        for lo, hi in ((0, 1), (H - 1, H)):
+            o_ref, s_ref = oracle.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], x["h0"],
+                                          x["cu_seqlens"], heads=(lo, hi))
+            got_o = d["out"][:, :, lo:hi].double().cpu().numpy()
+            got_s = d["hT"][:, lo:hi].double().cpu().numpy()
+            err["out"] = max(err["out"], float(np.abs(got_o - o_ref).max() / np.abs(o_ref).max()))
+            err["hT"] = max(err["hT"], float(np.abs(got_s - s_ref).max() / np.abs(s_ref).max()))
+        res["parity_vs_oracle"] = {"heads": [0, H - 1], "max_rel_err": err, "bound": 1e-2}
+    return res
+
+
 CONFIG_WORKLOADS = ("fp32_t256", "b16_t512_d64", "packed_16k", "t32k_h96")
 L2_BYTES = 126 * 1024 * 1024
 
@@ -925,6 +994,9 @@ def run_ours(args, world, rank, local):
     bwd = None
     if not args.decode_only and not args.no_bwd:
         bwd = bwd_leg(args, world, rank, dev, stream, barrier, hbm)
+    nal = None
+    if not args.decode_only and not args.no_noalloc:
+        nal = noalloc_leg(args, world, rank, dev, stream, barrier, hbm)
     cfg = None
     if not args.decode_only and not args.no_configs:
         cfg = configs_leg(args, world, rank, dev, stream, barrier, hbm, tf_sust)
@@ -960,6 +1032,7 @@ def run_ours(args, world, rank, local):
         "prefill_decay_g64": grp,
         "prefill_fused_prep": fzd,
         "prefill_bwd": bwd,
+        "prefill_noalloc": nal,
         "configs": cfg,
         "decode": dec, "e2e": pf["e2e"], "gpu_launches": pf["launches"],
         "clocks": pf["clocks"], "cpu_baseline": cpu,
@@ -994,6 +1067,8 @@ def main():
     ap.add_argument("--decode-n", type=int, default=0,
                     help="sequences in the decode leg (0 = the config-4 value, 256)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-noalloc", action="store_true",
+                    help="skip the kda_chunk_fwd_noalloc leg")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the other prefill workloads (configs leg)")
     ap.add_argument("--ref-tokens", type=int, default=0,
