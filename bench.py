@@ -841,7 +841,7 @@ def decode_oracle(args, N_sample=8):
 
 
 KERNEL_NAMES = {"prep": "kda_chunk_prep_kernel", "state": "kda_state_pass_kernel",
-                "combine": "kda_seg_combine_img_kernel", "fused": "kda_chunk_tc_kernel",
+                "fused": "kda_chunk_tc_kernel",
                 "simt": "kda_chunk_simt_kernel"}
 
 
@@ -878,25 +878,53 @@ def _traffic(workload: str) -> dict:
     return w
 
 
-def ingest_ncu(csv_path: str, workload: str) -> int:
-    """Write profiles/traffic.json from an ncu --csv launch list that holds
-    dram__bytes_read.sum and dram__bytes_write.sum per launch: the average DRAM
-    bytes per launch of each kernel kind, tagged with the hash of the kernel
-    sources it was taken on."""
+_BYTE_UNITS = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "KB": 1e3, "MB": 1e6,
+               "GB": 1e9, "": 1}
+
+
+def _ncu_dram_bytes(csv_path: str) -> dict:
+    """DRAM bytes (read + write) per captured launch of each kernel kind, from an
+    ncu --csv export: either a launch list (one row per launch and metric) or the
+    raw page of a report (`ncu -i rep --page raw --csv`: one row per launch, a
+    column per metric, a row of units under the header)."""
     import csv
     rows = list(csv.reader(open(csv_path)))
     hdr = next(i for i, r in enumerate(rows) if r and r[0] == "ID")
     H = rows[hdr]
-    ki, mi, vi, ii = H.index("Kernel Name"), H.index("Metric Name"), H.index("Metric Value"), 0
+    ki = H.index("Kernel Name")
     per = {}
-    for r in rows[hdr + 1:]:
-        if len(r) <= vi or not r[mi].startswith("dram__bytes_"):
+    if "Metric Name" in H:
+        mi, vi, ui = H.index("Metric Name"), H.index("Metric Value"), H.index("Metric Unit")
+        for r in rows[hdr + 1:]:
+            if len(r) <= vi or r[mi] not in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+                continue
+            kind = next((k for k, n in KERNEL_NAMES.items() if n in r[ki]), None)
+            if kind is not None:
+                b = float(r[vi].replace(",", "")) * _BYTE_UNITS[r[ui]]
+                per.setdefault(kind, {}).setdefault(r[0], 0.0)
+                per[kind][r[0]] += b
+        return per
+    cols = [H.index(m) for m in ("dram__bytes_read.sum", "dram__bytes_write.sum")]
+    units = rows[hdr + 1]
+    for r in rows[hdr + 2:]:
+        if len(r) <= max(cols):
             continue
         kind = next((k for k, n in KERNEL_NAMES.items() if n in r[ki]), None)
-        if kind is None:
-            continue
-        per.setdefault(kind, {}).setdefault(r[ii], 0)
-        per[kind][r[ii]] += int(float(r[vi].replace(",", "")))
+        if kind is not None:
+            per.setdefault(kind, {})[csv_path + ":" + r[0]] = sum(
+                float(r[c].replace(",", "")) * _BYTE_UNITS[units[c]] for c in cols)
+    return per
+
+
+def ingest_ncu(csv_paths, workload: str) -> int:
+    """Write profiles/traffic.json from ncu --csv exports (launch lists or raw
+    pages) that hold dram__bytes_read.sum and dram__bytes_write.sum per launch:
+    the average DRAM bytes per launch of each kernel kind, tagged with the hash of
+    the kernel sources it was taken on."""
+    per = {}
+    for path in csv_paths:
+        for kind, launches in _ncu_dram_bytes(path).items():
+            per.setdefault(kind, {}).update(launches)
     tpath = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(tpath) as f:
@@ -924,7 +952,7 @@ def _roofline(args, pf, hbm, tf_sust, peak_kind) -> dict:
     reads = rows * H * ((2 * dk + dv) * s_in + 4 * dk + 4)          # q, k, v, g, beta
     writes = rows * H * dv * s_in                                   # out
     algo = {"prep": reads, "state": writes + states, "fused": pf["bytes_call"],
-            "simt": pf["bytes_call"], "combine": 0}
+            "simt": pf["bytes_call"]}
     kt = {k: v for k, v in pf["ktimes"].items() if v[0] > 0 and k != "decode"}
     total_ms = sum(v[1] for v in kt.values()) or 1e-9
     traffic = _traffic(args.workload)
@@ -1076,8 +1104,9 @@ def main():
                          "the cpu_baseline leg, 1024 per step for --impl reference)")
     ap.add_argument("--ref-seconds", type=float, default=10.0,
                     help="cpu_baseline leg: repeat oracle passes until this much time has passed")
-    ap.add_argument("--ingest-ncu", default="",
-                    help="write profiles/traffic.json from this ncu --csv launch list (no GPU run)")
+    ap.add_argument("--ingest-ncu", nargs="+", default=[],
+                    help="write profiles/traffic.json from these ncu --csv exports (launch "
+                         "lists or raw pages of reports; no GPU run)")
     args = ap.parse_args()
     if args.ingest_ncu:
         return ingest_ncu(args.ingest_ncu, args.workload)

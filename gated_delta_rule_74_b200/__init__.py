@@ -89,6 +89,8 @@ def lib() -> ctypes.CDLL:
         L.kda_chunk_bwd_grouped.argtypes = [vp, vp, vp, fp, fp, fp, vp, vp, fp,
                                             fp, fp, fp, fp, fp, fp] + [ip] * 7 + [vp]
         L.kda_chunk_bwd_grouped.restype = ctypes.c_int
+        L.kda_chunk_bwd_recurrent.argtypes = L.kda_chunk_bwd_grouped.argtypes
+        L.kda_chunk_bwd_recurrent.restype = ctypes.c_int
         L.kda_device_status.argtypes = [ip]
         L.kda_device_status.restype = ctypes.c_int
         L.kda_selftest_bounded_wait.argtypes = [ctypes.c_uint, vp]
@@ -199,7 +201,7 @@ def kda_prefill_plan(B: int, T: int, H: int, packed: bool = False, sms: int = 14
 
 
 KERNEL_KINDS = {"prep": 0, "state": 1, "combine": 2, "fused": 3, "simt": 4, "decode": 5,
-                "bwd": 6}
+                "bwd": 6, "bwd_prep": 7, "bwd_chain": 8, "bwd_grad": 9}
 
 
 def kda_timing_start() -> None:
@@ -377,13 +379,14 @@ def kda_chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Te
                   beta: torch.Tensor, dout: torch.Tensor, h0: Optional[torch.Tensor] = None,
                   dhT: Optional[torch.Tensor] = None, cu_seqlens: Optional[torch.Tensor] = None,
                   grads: Optional[dict] = None, stream=None,
-                  workspace: Optional[torch.Tensor] = None) -> dict:
+                  workspace: Optional[torch.Tensor] = None, recurrent: bool = False) -> dict:
     """Gradients of L = sum(out * dout) + sum(hT * dhT) for kda_chunk_fwd with the same
     inputs.  g [B,T,H,dk] f32, or [B,T,H,dk/G] for one decay per group of G key channels
     (kda_chunk_bwd_grouped; dg then has g's shape).  dout has out's shape and dtype; dhT
     [Nseq,H,dk,dv] f32 or None.  Returns a dict of fp32 tensors dq, dk, dv, dg, dbeta, dh0
     (dh0 None when h0 is None); ``grads`` may hold preallocated outputs under those names;
-    a ``workspace`` tensor (kda_workspace_size bytes) calls kda_chunk_bwd_ws on it."""
+    a ``workspace`` tensor (kda_workspace_size bytes) calls kda_chunk_bwd_ws on it;
+    ``recurrent`` calls kda_chunk_bwd_recurrent (the fp32 reverse sweep) instead."""
     if q.dim() != 4:
         raise ValueError("q must be [B, T, H, dk]")
     Bt, T, H, dk = q.shape
@@ -422,6 +425,13 @@ def kda_chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Te
     args = [_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0), _ptr(cu_seqlens),
             _ptr(dout), _ptr(dhT), _ptr(res["dq"]), _ptr(res["dk"]), _ptr(res["dv"]),
             _ptr(res["dg"]), _ptr(res["dbeta"]), _ptr(res["dh0"]), nseq, T, H, dk, dv]
+    if recurrent:
+        if workspace is not None:
+            raise ValueError("the recurrent backward takes no workspace")
+        rc = lib().kda_chunk_bwd_recurrent(*args, G, dt, _stream(stream))
+        if rc != KDA_OK:
+            raise KdaError("kda_chunk_bwd_recurrent", rc)
+        return res
     if workspace is not None:
         wp, wb = _workspace_args(workspace)
         rc = lib().kda_chunk_bwd_ws(*args, G, dt, wp, wb, _stream(stream))

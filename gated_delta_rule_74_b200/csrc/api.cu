@@ -194,11 +194,20 @@ int kda_chunk_fwd_fused(const void* q_raw, const void* k_raw, const void* v, con
 }
 
 namespace {
+// Scratch of a kda_chunk_bwd call: the chunked form's (bf16, 128-wide heads) or the
+// recurrent sweep's.
+size_t bwd_scratch(int B, int T, int H, int dk, int dv, bool varlen, int in_dtype) {
+  if (kda::chunk_bwd_tc_supported(dk, dv, in_dtype))
+    return kda::chunk_bwd_tc_scratch_bytes(B, T, H, varlen);
+  return kda::chunk_bwd_scratch_bytes(B, T, H, dk, dv, varlen);
+}
+
 int chunk_bwd_impl(const void* q, const void* k, const void* v, const float* g,
                    const float* beta, const float* h0, const int32_t* cu_seqlens,
                    const void* dout, const float* dhT, float* dq, float* dk, float* dv, float* dg,
                    float* dbeta, float* dh0, int B, int T, int H, int dk_dim, int dv_dim, int gsh,
-                   int in_dtype, void* stream, const kda::Workspace* ws = nullptr) {
+                   int in_dtype, void* stream, const kda::Workspace* ws = nullptr,
+                   bool recurrent = false) {
   if (gsh < 0) return KDA_ERR_INVALID_ARG;
   if (B < 1 || T < 0 || H < 1) return KDA_ERR_INVALID_ARG;
   if (in_dtype != KDA_BF16 && in_dtype != KDA_F32) return KDA_ERR_INVALID_ARG;
@@ -215,10 +224,14 @@ int chunk_bwd_impl(const void* q, const void* k, const void* v, const float* g,
   if (rows * H * (long long)(dk_dim > dv_dim ? dk_dim : dv_dim) > (1LL << 40))
     return KDA_ERR_INVALID_ARG;
   if ((long long)B > 65535LL || H > 0x7fffffff) return KDA_ERR_UNSUPPORTED;
-  if (ws && !workspace_ok(ws, kda::chunk_bwd_scratch_bytes(B, T, H, dk_dim, dv_dim,
-                                                            cu_seqlens != nullptr)))
+  const bool chunked = !recurrent && kda::chunk_bwd_tc_supported(dk_dim, dv_dim, in_dtype);
+  if (ws && !workspace_ok(ws, bwd_scratch(B, T, H, dk_dim, dv_dim, cu_seqlens != nullptr,
+                                          in_dtype)))
     return KDA_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (chunked)
+    return status_from(kda::launch_chunk_bwd_tc(q, k, v, g, beta, h0, cu_seqlens, dout, dhT, dq,
+                                                dk, dv, dg, dbeta, dh0, B, T, H, gsh, st, ws));
   return status_from(kda::launch_chunk_bwd(q, k, v, g, beta, h0, cu_seqlens, dout, dhT, dq, dk,
                                            dv, dg, dbeta, dh0, B, T, H, dk_dim, dv_dim, gsh,
                                            in_dtype, st, ws));
@@ -243,6 +256,16 @@ int kda_chunk_bwd_grouped(const void* q, const void* k, const void* v, const flo
                         B, T, H, dk_dim, dv_dim, group_shift(g_group, dk_dim), in_dtype, stream);
 }
 
+int kda_chunk_bwd_recurrent(const void* q, const void* k, const void* v, const float* g,
+                            const float* beta, const float* h0, const int32_t* cu_seqlens,
+                            const void* dout, const float* dhT, float* dq, float* dk, float* dv,
+                            float* dg, float* dbeta, float* dh0, int B, int T, int H, int dk_dim,
+                            int dv_dim, int g_group, int in_dtype, void* stream) {
+  return chunk_bwd_impl(q, k, v, g, beta, h0, cu_seqlens, dout, dhT, dq, dk, dv, dg, dbeta, dh0,
+                        B, T, H, dk_dim, dv_dim, group_shift(g_group, dk_dim), in_dtype, stream,
+                        nullptr, true);
+}
+
 int kda_workspace_size(int op, int B, int T, int H, int dk, int dv, int packed, int in_dtype,
                        int sms, size_t* bytes) {
   if (!bytes || B < 1 || T < 0 || H < 1 || sms < 0) return KDA_ERR_INVALID_ARG;
@@ -250,7 +273,7 @@ int kda_workspace_size(int op, int B, int T, int H, int dk, int dv, int packed, 
   if (in_dtype != KDA_BF16 && in_dtype != KDA_F32) return KDA_ERR_INVALID_ARG;
   if (!head_ok(dk) || !head_ok(dv)) return KDA_ERR_UNSUPPORTED;
   if (op == KDA_OP_CHUNK_BWD) {
-    *bytes = kda::chunk_bwd_scratch_bytes(B, T, H, dk, dv, packed != 0);
+    *bytes = bwd_scratch(B, T, H, dk, dv, packed != 0, in_dtype);
     return KDA_OK;
   }
   if (!kda::chunk_split_supported(dk, dv, in_dtype)) {

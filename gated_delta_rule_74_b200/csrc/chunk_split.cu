@@ -55,6 +55,7 @@
 #include <cstring>
 #include <type_traits>
 
+#include "chunk_record.cuh"
 #include "decay_pairs.cuh"
 #include "kda_common.cuh"
 #include "segments.cuh"
@@ -75,15 +76,18 @@ constexpr int D = kHead;
 constexpr int NT = 256;
 constexpr uint32_t kWaitLimit = 1u << 22;
 
-// ---- chunk record (one per (head, chunk)), byte offsets
-constexpr uint32_t REC_QW = 0;          // [Qbar^T | W^T]: MN-major SW128, N = 128 (2 x 64 tokens,
+// ---- chunk record (one per (head, chunk)), byte offsets (chunk_record.cuh)
+constexpr uint32_t REC_QW = rec::QW;    // [Qbar^T | W^T]: MN-major SW128, N = 128 (2 x 64 tokens,
                                         // 16 KB apart), K = dk
-constexpr uint32_t REC_KA = 32768;      // [Kend^T ; Aqk] (f16): K-major SW128, 192 rows x 64 tokens
-constexpr uint32_t REC_AQK = REC_KA + 16384;
-constexpr uint32_t REC_U = 57344;       // U^T [dv][64 tokens] f16: 128-byte rows, 16-byte
+constexpr uint32_t REC_KA = rec::KA;    // [Kend^T ; Aqk] (f16): K-major SW128, 192 rows x 64 tokens
+constexpr uint32_t REC_AQK = rec::AQK;
+constexpr uint32_t REC_U = rec::U;      // U^T [dv][64 tokens] f16: 128-byte rows, 16-byte
                                         // chunks (8 tokens) XOR-swizzled with (row % 8)
-constexpr uint32_t REC_DECAY = 73728;   // exp(G_last) per key channel, fp32 [dk]
-constexpr uint32_t REC_BYTES = 74240;
+constexpr uint32_t REC_DECAY = rec::DECAY;   // exp(G_last) per key channel, fp32 [dk]
+constexpr uint32_t REC_BYTES = rec::BYTES;
+// The backward's records (BWD instantiation): the same images, but Kend^T, Aqk and
+// U^T in bf16 (gradients can be far below f16's normal range), followed by T and A
+// in fp32.
 
 // TMA maps of the prep kernel's tiles: q, k, g [rows, H, dk] and v [rows, H, dv]
 // (3-D: channel, head, token row), boxes of 64 token rows of one head.
@@ -170,7 +174,7 @@ struct UnsafeRows {
 // stages the normalised k, q as bf16 [row][128] in the record's U^T and W^T areas
 // for the exact pair pass (the record's own images overwrite them at the end).
 __device__ __noinline__ void prep_unsafe_direct(uint8_t* sm, uint8_t* rc, int a, int c0, int uns,
-                                                bool conv, const UnsafeRows& ur) {
+                                                bool conv, bool bf, const UnsafeRows& ur) {
 #pragma unroll 1
   for (int ch = 0; ch < 2; ++ch) {
     if (!((uns >> ch) & 1)) continue;
@@ -190,7 +194,8 @@ __device__ __noinline__ void prep_unsafe_direct(uint8_t* sm, uint8_t* rc, int a,
 #pragma unroll
       for (int e = 0; e < 8; ++e)
         v[e] = ur.k[ch][8 * gg + e] * __expf(fminf(ur.tl[ch] - ur.x[ch][8 * gg + e], 0.f));
-      *reinterpret_cast<uint4*>(rc + REC_KA + chunk_kmajor_sw128(c, g8, D)) = pack8_f16(v, 1.f);
+      *reinterpret_cast<uint4*>(rc + REC_KA + chunk_kmajor_sw128(c, g8, D)) =
+          bf ? pack8(v, 1.f) : pack8_f16(v, 1.f);
       if (conv) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -295,8 +300,9 @@ __device__ __noinline__ void prep_unsafe_pairs(const float* __restrict__ g, long
 // Prep kernel: one CTA per (chunk slot, head).  CONV: q and k are the raw
 // projections; each is convolved causally per channel (width convW <= 4, history
 // reset at the document start), L2-normalised per token, and q scaled by dk^-1/2.
+// BWD: the backward's record (bf16 images, plus T and A in fp32).
 // ============================================================================
-template <bool CONV, bool GRPD>
+template <bool CONV, bool GRPD, bool BWD = false>
 __global__ void __launch_bounds__(NT, 2)
 kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
                       const bf16* __restrict__ v, const float* __restrict__ g,
@@ -344,7 +350,7 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   const long long t0 = t_beg + n * C;
   const int L = (int)min((long long)C, t_end - t0);
   const long long rbase = row0 + t0;                   // first token row of the chunk
-  uint8_t* rc = rec + ((size_t)h * (size_t)nslots + (size_t)slot) * REC_BYTES;
+  uint8_t* rc = rec + ((size_t)h * (size_t)nslots + (size_t)slot) * (BWD ? rec::BYTES_BWD : REC_BYTES);
 
   // The chunk's tiles.  TMA (tma != 0; not with the fused convolution): v straight
   // into the MN-major operand of U^T (two 64-value boxes, 128-byte swizzle), q and k
@@ -581,7 +587,7 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     // nothing of this stays in the common path
     UnsafeRows ur;
     fill_unsafe_rows(ur, g, k, q, rbase, H, h, dk, gsh, L, a, c0, d[1], d[2], d[3], rel);
-    prep_unsafe_direct(sm, rc, a, c0, (ux ? 1 : 0) | (uy ? 2 : 0), false, ur);
+    prep_unsafe_direct(sm, rc, a, c0, (ux ? 1 : 0) | (uy ? 2 : 0), false, BWD, ur);
   }
   if (CONV && (ux || uy)) {
     // fused convolution: the normalised q, k exist only in registers, so they go
@@ -600,7 +606,7 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       for (int a2 = 0; a2 < 4; ++a2) ur.d[ch][a2] = (ch ? d[a2].y : d[a2].x) - first;
       ur.tl[ch] = (ch ? rel.y : rel.x) - first;
     }
-    prep_unsafe_direct(sm, rc, a, c0, (ux ? 1 : 0) | (uy ? 2 : 0), CONV, ur);
+    prep_unsafe_direct(sm, rc, a, c0, (ux ? 1 : 0) | (uy ? 2 : 0), CONV, BWD, ur);
   }
 
 #pragma unroll
@@ -646,7 +652,8 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       // record: Qbar^T (MN-major, N = tokens, K = channels) and Kend^T (K-major)
       *reinterpret_cast<uint4*>(rc + REC_QW + chunk_mnmajor_sw128(g8, c, D)) = pack8(lq, eP);
       if (!uns)
-        *reinterpret_cast<uint4*>(rc + REC_KA + chunk_kmajor_sw128(c, g8, D)) = pack8_f16(kr, eE);
+        *reinterpret_cast<uint4*>(rc + REC_KA + chunk_kmajor_sw128(c, g8, D)) =
+            BWD ? pack8(kr, eE) : pack8_f16(kr, eE);
     }
   }
   if (a == 3)                                  // exp(G_last), G_last = off + rel
@@ -762,6 +769,18 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     if (mine) {
       if (isA) {
         const float br = s_beta[r];
+        if constexpr (BWD) {                 // A itself, strictly lower, for the backward
+          float4* ar = reinterpret_cast<float4*>(rc + rec::AMAT) + 16 * r;
+#pragma unroll
+          for (int i4 = 0; i4 < 16; ++i4) {
+            float4 w;
+            w.x = (4 * i4 + 0 < r) ? __uint_as_float(tv[i4 >> 2][(4 * i4 + 0) & 15]) : 0.f;
+            w.y = (4 * i4 + 1 < r) ? __uint_as_float(tv[i4 >> 2][(4 * i4 + 1) & 15]) : 0.f;
+            w.z = (4 * i4 + 2 < r) ? __uint_as_float(tv[i4 >> 2][(4 * i4 + 2) & 15]) : 0.f;
+            w.w = (4 * i4 + 3 < r) ? __uint_as_float(tv[i4 >> 2][(4 * i4 + 3) & 15]) : 0.f;
+            ar[i4] = w;
+          }
+        }
 #pragma unroll
         for (int i4 = 0; i4 < 16; ++i4) {
           float4 w;
@@ -779,7 +798,7 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
 #pragma unroll
           for (int e = 0; e < 8; ++e)
             w[e] = (c8 * 8 + e <= r) ? __uint_as_float(tv[c8 >> 1][(c8 & 1) * 8 + e]) : 0.f;
-          sts16(sm, Q_OAQK + chunk_kmajor_sw128(r, c8, C), pack8_f16(w, 1.f));
+          sts16(sm, Q_OAQK + chunk_kmajor_sw128(r, c8, C), BWD ? pack8(w, 1.f) : pack8_f16(w, 1.f));
         }
       }
     }
@@ -883,6 +902,17 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       put(48 + i, col, x);
     }
     __syncthreads();
+    if constexpr (BWD) {                       // T for the backward, fp32 [64][64]
+      // (the blocks above the diagonal were never written: zeros)
+      float4* tr = reinterpret_cast<float4*>(rc + rec::TMAT);
+#pragma unroll
+      for (int it = 0; it < 4; ++it) {
+        const int idx = tid + it * NT, row = idx >> 4, c4 = idx & 15;
+        const float4 x = *reinterpret_cast<const float4*>(T32 + row * LDA + 4 * c4);
+        tr[idx] = make_float4(4 * c4 + 0 <= row ? x.x : 0.f, 4 * c4 + 1 <= row ? x.y : 0.f,
+                              4 * c4 + 2 <= row ? x.z : 0.f, 4 * c4 + 3 <= row ? x.w : 0.f);
+      }
+    }
     // T diag(beta) as bf16: B operand of W^T / U^T, K-major SW128, N = 64 (r'), K = 64 (r)
 #pragma unroll
     for (int it = 0; it < 2; ++it) {
@@ -946,11 +976,11 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
 #pragma unroll
       for (int c8 = 0; c8 < 8; ++c8) {
         const uint32_t* f = t[c8 >> 1] + 8 * (c8 & 1);
-        const uint4 val = make_uint4(pack_f16(__uint_as_float(f[0]), __uint_as_float(f[1])),
-                                     pack_f16(__uint_as_float(f[2]), __uint_as_float(f[3])),
-                                     pack_f16(__uint_as_float(f[4]), __uint_as_float(f[5])),
-                                     pack_f16(__uint_as_float(f[6]), __uint_as_float(f[7])));
-        sts16(sm, Q_OU + j * 128 + (((uint32_t)c8 ^ (j & 7u)) << 4), val);
+        float x[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = __uint_as_float(f[e]);
+        sts16(sm, Q_OU + j * 128 + (((uint32_t)c8 ^ (j & 7u)) << 4),
+              BWD ? pack8(x, 1.f) : pack8_f16(x, 1.f));
       }
     }
     fence_async_smem();
@@ -1520,6 +1550,10 @@ bool set_attrs() {
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, PREP_SMEM) == cudaSuccess &&
            cudaFuncSetAttribute(kda_chunk_prep_kernel<true, false>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, PREP_SMEM) == cudaSuccess &&
+           cudaFuncSetAttribute(kda_chunk_prep_kernel<false, false, true>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, PREP_SMEM) == cudaSuccess &&
+           cudaFuncSetAttribute(kda_chunk_prep_kernel<false, true, true>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, PREP_SMEM) == cudaSuccess &&
            cudaFuncSetAttribute(kda_state_pass_kernel<false>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, STATE_SMEM) == cudaSuccess &&
            cudaFuncSetAttribute(kda_state_pass_kernel<true>,
@@ -1578,6 +1612,27 @@ void chunk_split_plan(int B, int T, int H, bool varlen, int sms, int* G, int* ha
 }
 
 namespace {
+// TMA maps of the prep kernel's tiles (rows addressed by int32 coordinates); 0 when
+// the tiles are loaded without TMA (the maps are then zeroed and not read).
+int prep_maps(PrepMaps* maps, const bf16* qb, const bf16* kb, const bf16* vb, const float* g,
+              long long rows, int H, int dk, int dv, int gsh) {
+  int tma = 0;
+  if (rows > 0 && rows < (1LL << 31) - 2 * C) {
+    const uint64_t hh = (uint64_t)H, nr = (uint64_t)rows;
+    tma = make_tile_map_3d(&maps->q, false, qb, dk, hh, nr, dk * 2ull, hh * dk * 2, dk, C,
+                           false) &&
+          make_tile_map_3d(&maps->k, false, kb, dk, hh, nr, dk * 2ull, hh * dk * 2, dk, C,
+                           false) &&
+          make_tile_map_3d(&maps->v, false, vb, dv, hh, nr, dv * 2ull, hh * dv * 2, 64, C,
+                           true) &&
+          (gsh != 0 || make_tile_map_3d(&maps->g, true, g, dk, hh, nr, dk * 4ull, hh * dk * 4,
+                                        dk, C, false));
+    if (gsh != 0) maps->g = maps->q;             // not read
+  }
+  if (!tma) memset(maps, 0, sizeof(*maps));
+  return tma;
+}
+
 // Chunk records (nslots per head) and, when sequences are split, the segment
 // states: the one layout both the size query and the launcher use.
 struct SplitScratch {
@@ -1647,24 +1702,10 @@ cudaError_t launch_chunk_split(const void* q, const void* k, const void* v, cons
 
   cudaError_t e = cudaSuccess;
   if (nslots > 0) {
-    // TMA maps of the tiles (rows addressed by int32 coordinates)
     PrepMaps maps;
     const long long rows = varlen ? (long long)T : (long long)B * T;
     const bool conv = fz && fz->conv_q;
-    int tma = 0;
-    if (!conv && rows > 0 && rows < (1LL << 31) - 2 * C) {
-      const uint64_t hh = (uint64_t)H, nr = (uint64_t)rows;
-      tma = make_tile_map_3d(&maps.q, false, qb, dk, hh, nr, dk * 2ull, hh * dk * 2, dk, C,
-                             false) &&
-            make_tile_map_3d(&maps.k, false, kb, dk, hh, nr, dk * 2ull, hh * dk * 2, dk, C,
-                             false) &&
-            make_tile_map_3d(&maps.v, false, vb, dv, hh, nr, dv * 2ull, hh * dv * 2, 64, C,
-                             true) &&
-            (gsh != 0 || make_tile_map_3d(&maps.g, true, g, dk, hh, nr, dk * 4ull, hh * dk * 4,
-                                          dk, C, false));
-      if (gsh != 0) maps.g = maps.q;             // not read
-    }
-    if (!tma) memset(&maps, 0, sizeof(maps));
+    const int tma = conv ? 0 : prep_maps(&maps, qb, kb, vb, g, rows, H, dk, dv, gsh);
     if (conv) {
       KDA_TIMED(KDA_KERNEL_PREP, stream,
                 kda_chunk_prep_kernel<true, false><<<dim3((unsigned)nslots, H), NT, PREP_SMEM, stream>>>(
@@ -1713,6 +1754,30 @@ cudaError_t launch_chunk_split(const void* q, const void* k, const void* v, cons
   if (e == cudaSuccess) e = el;
   if (pooled) cudaFreeAsync(scratch, stream);
   return e;
+}
+
+// The prep kernel for the backward (dk = dv = 128): nslots records of
+// rec::BYTES_BWD bytes per head at `rec`, numbered as the prefill numbers them.
+cudaError_t launch_chunk_prep_bwd(const void* q, const void* k, const void* v, const float* g,
+                                  const float* beta, const int32_t* cu_seqlens, uint8_t* rec,
+                                  int B, int T, int H, int gsh, long long nslots,
+                                  cudaStream_t stream) {
+  if (!set_attrs()) return cudaErrorInvalidDevice;
+  if (nslots == 0) return cudaSuccess;
+  const bf16* qb = static_cast<const bf16*>(q);
+  const bf16* kb = static_cast<const bf16*>(k);
+  const bf16* vb = static_cast<const bf16*>(v);
+  PrepMaps maps;
+  const long long rows = cu_seqlens ? (long long)T : (long long)B * T;
+  const int tma = prep_maps(&maps, qb, kb, vb, g, rows, H, D, D, gsh);
+  auto prep = gsh != 0 ? kda_chunk_prep_kernel<false, true, true>
+                       : kda_chunk_prep_kernel<false, false, true>;
+  KDA_TIMED(KDA_KERNEL_BWD_PREP, stream,
+            prep<<<dim3((unsigned)nslots, H), NT, PREP_SMEM, stream>>>(
+                qb, kb, vb, g, beta, cu_seqlens, rec, B, T, H, D, D, gsh, nslots, nullptr,
+                nullptr, 0, maps, tma));
+  note_launches(1);
+  return cudaGetLastError();
 }
 
 // Reads (and with reset clears) g_chunk_split_timeout; host side of kda_device_status.

@@ -20,7 +20,9 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 
 // Runs setup() (kernel attributes and the like) once per call site and device, with
 // that device current; thread-safe.  A setup that fails is retried on the next call.
-enum OnceSite { kOnceSplit = 0, kOnceTc, kOnceDecodeChunk, kOnceCombine, kOnceCombineImg, kOnceSites };
+enum OnceSite {
+  kOnceSplit = 0, kOnceTc, kOnceDecodeChunk, kOnceCombine, kOnceCombineImg, kOnceBwdTc, kOnceSites
+};
 bool once_per_device(int site, bool (*setup)());
 
 // Most bytes the library pool of the current device has had in use at once; with
@@ -122,6 +124,18 @@ cudaError_t launch_chunk_bwd(const void* q, const void* k, const void* v, const 
                              float* dg, float* dbeta, float* dh0, int B, int T, int H, int dkd,
                              int dvd, int gsh, int in_dtype, cudaStream_t stream,
                              const Workspace* ws = nullptr);
+
+// Chunked backward on the tensor cores (bf16, dk = dv = 128): the prep kernel's
+// backward form, the state chains and the per-chunk gradient kernel.  Scratch:
+// chunk_bwd_tc_scratch_bytes() (records, states, Delta and their gradients).
+bool chunk_bwd_tc_supported(int dk, int dv, int in_dtype);
+size_t chunk_bwd_tc_scratch_bytes(int B, int T, int H, bool varlen);
+cudaError_t launch_chunk_bwd_tc(const void* q, const void* k, const void* v, const float* g,
+                                const float* beta, const float* h0, const int32_t* cu_seqlens,
+                                const void* dout, const float* dhT, float* dq, float* dk,
+                                float* dv, float* dg, float* dbeta, float* dh0, int B, int T,
+                                int H, int gsh, cudaStream_t stream,
+                                const Workspace* ws = nullptr);
 
 // Bounded-wait flags (one per kernel file): read, and with reset clear, the flag a
 // kernel raises when one of its bounded waits gives up.

@@ -291,15 +291,20 @@ KDA_API int kda_chunk_fwd_fused(const void* q_raw, const void* k_raw, const void
  * documents write nothing; their dh0 = dhT).  Output buffers must not alias
  * each other or any input.  The chunk length (64) does not change the result.
  *
- * Method: a recurrent reverse sweep in fp32 on the CUDA cores.  The columns of
- * the state evolve independently, so each warp runs the chain of 8 state
- * columns for one (sequence, head); the state is kept at every 64th token and
- * each chunk's states are recomputed once.  dv and dh0 are reproducible bit for
- * bit; dq, dk, dg and dbeta add the warps' parts with atomics, so repeated calls
- * may differ in the last bits (fp32 summation order).  Scratch: 4 * dk * dv
- * bytes per (chunk, head) plus 64 * 4 * dk * dv bytes per (sequence, head), from
- * the library's stream-ordered memory pool (released on the stream at the end
- * of the call).
+ * Method.  KDA_BF16 with dk = dv = 128: the chunked form on the tensor cores
+ * (chunks of 64 tokens; the chain rule through the chunked form's equations).
+ * Its matrix products take bf16 operands with fp32 accumulation, as the forward's
+ * do, so the gradients carry the bf16 bound of the forward (relative error
+ * max|x - x_ref| / max|x_ref| of a few 1e-3, at most 1e-2).  The state and its
+ * gradient are carried across chunks in fp32.  dq, dk, dv and dh0 are
+ * reproducible bit for bit; dg and dbeta add a few per-chunk sums with
+ * shared-memory atomics, so repeated calls may differ in their last bits.  Scratch:
+ * 205,312 B per (chunk slot, head) (ceil(T/64) * B slots, ceil(T/64) + B when
+ * packed).
+ * Otherwise (KDA_F32, or a 64-wide head): the recurrent reverse sweep of
+ * kda_chunk_bwd_recurrent below.
+ * Scratch comes from the library's stream-ordered memory pool (released on the
+ * stream at the end of the call).
  *
  * Returns KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED or KDA_ERR_CUDA
  * (also when the scratch cannot be allocated).
@@ -310,6 +315,26 @@ KDA_API int kda_chunk_bwd(const void* q, const void* k, const void* v,
                           float* dq, float* dk, float* dv, float* dg, float* dbeta,
                           float* dh0, int B, int T, int H, int dk_dim, int dv_dim,
                           int in_dtype, void* stream);
+
+/*
+ * kda_chunk_bwd_recurrent -- the same gradients (g_group as in
+ * kda_chunk_bwd_grouped; 1 = one decay per channel) by a recurrent reverse sweep
+ * in fp32 on the CUDA cores, for any in_dtype and head size: accurate to fp32
+ * rounding (relative error about 1e-6) where the chunked form is bf16-bounded.
+ * The columns of the state evolve independently, so each warp runs the chain of
+ * 4 state columns for one (sequence, head); the state is kept at every 64th token
+ * and each chunk's states are recomputed once.  dv and dh0 are reproducible bit for
+ * bit; dq, dk, dg and dbeta add the warps' parts with atomics, so repeated calls may
+ * differ in the last bits (fp32 summation order).  Scratch: 4 * dk * dv bytes per
+ * (chunk, head) plus 64 * 4 * dk * dv bytes per (sequence, head), from the library
+ * pool.  Returns as kda_chunk_bwd.
+ */
+KDA_API int kda_chunk_bwd_recurrent(const void* q, const void* k, const void* v,
+                                    const float* g, const float* beta, const float* h0,
+                                    const int32_t* cu_seqlens, const void* dout,
+                                    const float* dhT, float* dq, float* dk, float* dv, float* dg,
+                                    float* dbeta, float* dh0, int B, int T, int H, int dk_dim,
+                                    int dv_dim, int g_group, int in_dtype, void* stream);
 
 /*
  * kda_chunk_bwd_grouped -- kda_chunk_bwd for grouped decay (one log-decay per
@@ -347,8 +372,9 @@ KDA_API int kda_chunk_bwd_grouped(const void* q, const void* k, const void* v,
  * splits sequences into segments, by 2 * 64 KB per (segment slot, head), or
  * 4 * 64 KB when the split keeps half-way states (kda_prefill_plan gives the split;
  * segment slots = B * ceil(ceil(T/64) / G), or that count + B when packed).  KDA_F32
- * forward calls need none.  The backward's is 4 * dk * dv B per (chunk slot +
- * sequence, head) plus 64 * 4 * dk * dv B per (sequence, head).
+ * forward calls need none.  The backward's is, in its chunked form (KDA_BF16,
+ * dk = dv = 128), 205,312 B per (chunk slot, head); otherwise 4 * dk * dv B per
+ * (chunk slot + sequence, head) plus 64 * 4 * dk * dv B per (sequence, head).
  * Returns KDA_OK, KDA_ERR_INVALID_ARG (unknown op, bad sizes, NULL bytes),
  * KDA_ERR_UNSUPPORTED (head sizes) or KDA_ERR_CUDA (sms = 0 and no device).
  */
@@ -462,8 +488,11 @@ typedef enum {
   KDA_KERNEL_FUSED = 3,         /* single-kernel tensor-core prefill              */
   KDA_KERNEL_SIMT = 4,          /* CUDA-core prefill (fp32, d = 64)               */
   KDA_KERNEL_DECODE = 5,        /* decode step                                    */
-  KDA_KERNEL_BWD = 6,           /* prefill backward                               */
-  KDA_KERNEL_KINDS = 7
+  KDA_KERNEL_BWD = 6,           /* prefill backward, recurrent sweep              */
+  KDA_KERNEL_BWD_PREP = 7,      /* chunked backward: per-chunk prep               */
+  KDA_KERNEL_BWD_CHAIN = 8,     /* chunked backward: forward and reverse chains   */
+  KDA_KERNEL_BWD_GRAD = 9,      /* chunked backward: per-chunk gradients          */
+  KDA_KERNEL_KINDS = 10
 } kda_kernel_kind_t;
 KDA_API int kda_timing_start(void);
 KDA_API int kda_timing_stop(void);
