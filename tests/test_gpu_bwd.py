@@ -1,9 +1,12 @@
-"""Prefill backward on the GPU (kda_chunk_bwd) against the oracle's float64
-reverse-mode differentiation of the recurrence, on the same seeded inputs.
+"""The recurrent prefill backward on the GPU (kda_chunk_bwd_recurrent, and
+kda_chunk_bwd for the inputs it sends there: fp32 or 64-wide heads) against the
+oracle's float64 reverse-mode differentiation of the recurrence, on the same
+seeded inputs.
 
-The kernel computes in fp32 on the exact values of the (bf16 or fp32) inputs, so
+The sweep computes in fp32 on the exact values of the (bf16 or fp32) inputs, so
 every gradient is held to the fp32 bound max|d - d_ref| / max|d_ref| <= 1e-4,
-whatever the storage dtype."""
+whatever the storage dtype.  The chunked form (bf16, 128-wide heads) has its own
+tests in test_gpu_bwd_chunked.py."""
 import pytest
 import torch
 
@@ -33,7 +36,8 @@ def _run(x, dout, dhT, with_h0=True, heads=None):
     d = to_dev(x)
     h0 = d["h0"] if with_h0 else None
     r = kda.kda_chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], dout.cuda(), h0=h0,
-                          dhT=None if dhT is None else dhT.cuda(), cu_seqlens=d["cu_seqlens"])
+                          dhT=None if dhT is None else dhT.cuda(), cu_seqlens=d["cu_seqlens"],
+                          recurrent=True)
     torch.cuda.synchronize()
     ref = oracle.backward(x["q"], x["k"], x["v"], x["g"], x["beta"], dout,
                           x["h0"] if with_h0 else None, dhT, x["cu_seqlens"], heads=heads)
@@ -97,7 +101,7 @@ def test_bwd_zero_tokens():
     dhT = torch.randn((2, 2, 64, 64))
     d = to_dev(x)
     r = kda.kda_chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], dout.cuda(), h0=d["h0"],
-                          dhT=dhT.cuda())
+                          dhT=dhT.cuda(), recurrent=True)
     torch.cuda.synchronize()
     assert torch.equal(r["dh0"].cpu(), dhT)
 
@@ -110,7 +114,8 @@ def test_bwd_long_sequence_sampled_heads():
     x = ki.make_prefill(spec)
     dout, dhT = _cotangents(x, 8193, 1)
     d = to_dev(x)
-    r = kda.kda_chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], dout.cuda(), dhT=dhT.cuda())
+    r = kda.kda_chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], dout.cuda(), dhT=dhT.cuda(),
+                          recurrent=True)
     torch.cuda.synchronize()
     heads = (5, 7)
     ref = oracle.backward(x["q"], x["k"], x["v"], x["g"], x["beta"], dout, None, dhT,
@@ -127,9 +132,9 @@ def test_bwd_repeatable():
     dout, dhT = _cotangents(x, 42, 1)
     d = to_dev(x)
     a = kda.kda_chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], dout.cuda(), h0=d["h0"],
-                          dhT=dhT.cuda())
+                          dhT=dhT.cuda(), recurrent=True)
     b = kda.kda_chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], dout.cuda(), h0=d["h0"],
-                          dhT=dhT.cuda())
+                          dhT=dhT.cuda(), recurrent=True)
     torch.cuda.synchronize()
     # dv and dh0 are column-local: reproducible bit for bit; dq, dk, dg and dbeta
     # sum per-warp parts in arrival order: equal up to fp32 rounding
@@ -152,7 +157,7 @@ def test_bwd_grouped_decay_matches_oracle(dtype, dk, dv, G):
     dout, dhT = _cotangents(x, 61 + G, 2)
     d = to_dev(x)
     r = kda.kda_chunk_bwd(d["q"], d["k"], d["v"], gg.cuda(), d["beta"], dout.cuda(),
-                          h0=d["h0"], dhT=dhT.cuda())
+                          h0=d["h0"], dhT=dhT.cuda(), recurrent=True)
     torch.cuda.synchronize()
     ref = oracle.backward(x["q"], x["k"], x["v"], gg, x["beta"], dout, x["h0"], dhT)
     assert tuple(r["dg"].shape) == tuple(gg.shape)
@@ -170,7 +175,7 @@ def test_bwd_grouped_packed_documents():
     dout, dhT = _cotangents(x, 72, nseq)
     d = to_dev(x)
     r = kda.kda_chunk_bwd(d["q"], d["k"], d["v"], gg.cuda(), d["beta"], dout.cuda(),
-                          h0=d["h0"], dhT=dhT.cuda(), cu_seqlens=d["cu_seqlens"])
+                          h0=d["h0"], dhT=dhT.cuda(), cu_seqlens=d["cu_seqlens"], recurrent=True)
     torch.cuda.synchronize()
     ref = oracle.backward(x["q"], x["k"], x["v"], gg, x["beta"], dout, x["h0"], dhT,
                           x["cu_seqlens"])

@@ -92,8 +92,9 @@ def test_too_small_or_misaligned_workspace_is_rejected():
     assert bool((out == 3.0).all())
 
 
-@pytest.mark.parametrize("dtype,packed", [("bf16", False), ("f32", True)])
+@pytest.mark.parametrize("dtype,packed", [("bf16", False), ("bf16", True), ("f32", True)])
 def test_backward_on_caller_workspace(dtype, packed):
+    """bf16 runs the chunked form (bf16 bound), fp32 the recurrent sweep (fp32 bound)."""
     spec = ki.PrefillSpec("wsb", B=0 if packed else 2, T=0 if packed else 200, H=2, dk=128,
                           dv=128, dtype=dtype, decay="alog", seed=24, h0=True, varlen=packed)
     x = ki.make_prefill(spec, doc_lens=[150, 2, 90] if packed else None)
@@ -113,5 +114,6 @@ def test_backward_on_caller_workspace(dtype, packed):
     assert kda.kda_pool_usage() == 0
     ref = oracle.backward(x["q"], x["k"], x["v"], x["g"], x["beta"], dout, x["h0"], dhT,
                           x["cu_seqlens"])
+    tol = TOL["bf16"] if dtype == "bf16" else 1e-4
     for n in ("dq", "dk", "dv", "dg", "dbeta", "dh0"):
-        assert rel_err(r[n], ref[n]) <= 1e-4, n
+        assert rel_err(r[n], ref[n]) <= tol, n
