@@ -315,8 +315,8 @@ int kda_device_status(int reset) {
   if (cudaDeviceSynchronize() != cudaSuccess) return status_from(cudaErrorUnknown);
   int any = 0;
   for (auto take : {kda::take_split_timeout, kda::take_tc_timeout, kda::take_bwd_timeout,
-                    kda::take_combine_timeout, kda::take_selftest_timeout,
-                    kda::take_decode_chunk_timeout}) {
+                    kda::take_bwd_tc_timeout, kda::take_combine_timeout,
+                    kda::take_selftest_timeout, kda::take_decode_chunk_timeout}) {
     int f = 0;
     if (take(&f, reset != 0) != cudaSuccess) return status_from(cudaErrorUnknown);
     any |= f;

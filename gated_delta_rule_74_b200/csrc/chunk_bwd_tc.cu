@@ -47,6 +47,9 @@
 
 namespace kda {
 
+// Set when a bounded wait of the chunked backward gives up (diagnostic).
+__device__ int g_bwd_tc_timeout = 0;
+
 cudaError_t launch_chunk_prep_bwd(const void* q, const void* k, const void* v, const float* g,
                                   const float* beta, const int32_t* cu_seqlens, uint8_t* rec,
                                   int B, int T, int H, int gsh, long long nslots,
@@ -58,9 +61,10 @@ using bf16 = __nv_bfloat16;
 
 constexpr int C = kChunk;
 constexpr int D = kHead;
-constexpr int NTH = 256;
+constexpr int NTC = 256;               // threads of the chain kernel
 constexpr uint32_t kImgS = 32768;      // S / dS image per (chunk, head): [128 j][128 c] bf16
 constexpr uint32_t kImgD = 16384;      // Delta / dDelta image: [64 t][128 j] bf16
+constexpr uint32_t kWaitLimit = 1u << 22;
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -190,21 +194,22 @@ struct Chain {
   static constexpr int STG = 3;            // record stages in flight
   // forward stage: W^T (16 KB), Kend^T (16 KB), U^T rows of the block, exp(Gamma_last)
   static constexpr uint32_t F_W = 0, F_K = 16384, F_U = 32768, F_DEC = F_U + NB * 128,
-                            F_STAGE = F_DEC + 512;
+                            F_STAGE = F_DEC + 512, F_BYTES = F_STAGE;
   static constexpr uint32_t F_S = STG * F_STAGE;        // S tile [NB j][128 c]
   static constexpr uint32_t F_DL = F_S + NB * 256;      // Delta tile [64 t][NB j] (64-column panel)
   static constexpr uint32_t F_SMEM = F_DL + 8192;
   // reverse stage: [Qbar^T | W^T] (32 KB), [Kend^T ; Aqk] (24 KB), exp(Gamma_last), dO tile
   static constexpr uint32_t R_QW = 0, R_KA = 32768, R_DEC = 57344, R_DO = 57856,
-                            R_STAGE = R_DO + 8192;
+                            R_STAGE = R_DO + 8192, R_BYTES = R_DO;
   static constexpr uint32_t R_Y = STG * R_STAGE;        // dS tile [NB j][128 c]
   static constexpr uint32_t R_DD = R_Y + NB * 256;      // -dDelta tile [64 t][NB j]
   static constexpr uint32_t R_SMEM = R_DD + 8192;
   static constexpr uint32_t SMEM = (F_SMEM > R_SMEM ? F_SMEM : R_SMEM) + 1024;
+  static_assert(F_STAGE % 128 == 0 && R_STAGE % 128 == 0, "tiles stay 128-byte aligned");
 };
 
 template <int NB>
-__global__ void __launch_bounds__(NTH, 1)
+__global__ void __launch_bounds__(NTC, 1)
 kda_bwd_chain_kernel(const uint8_t* __restrict__ rec, const float* __restrict__ h0,
                      const int32_t* __restrict__ cu_seqlens, const bf16* __restrict__ dout,
                      const float* __restrict__ dhT, float* __restrict__ dh0,
@@ -212,9 +217,11 @@ kda_bwd_chain_kernel(const uint8_t* __restrict__ rec, const float* __restrict__ 
                      uint8_t* __restrict__ dsimg, uint8_t* __restrict__ ddimg, int T, int H,
                      long long nslots) {
   using CF = Chain<NB>;
-  constexpr int NJ = CF::NJ, STG = CF::STG;
+  constexpr int STG = CF::STG;
+  static_assert(NB == 32, "8 warps: 8 row blocks of the state, all 4 n8 tiles");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
+  __shared__ uint64_t full[STG];           // record stage landed (bulk copies)
   const uint32_t sb = smem_u32(sm);
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31, g = lane >> 2, qd = lane & 3;
   const bool fwd = (int)blockIdx.x < CF::NJB;
@@ -225,50 +232,85 @@ kda_bwd_chain_kernel(const uint8_t* __restrict__ rec, const float* __restrict__ 
   const int nch = (int)chunk_count(t_end - t_beg);
   const size_t base = (size_t)h * (size_t)nslots + (size_t)seq_chunk_base(cu_seqlens, s, T);
   const size_t st_off = ((size_t)s * H + h) * D * D;
+  if (tid == 0) {
+#pragma unroll
+    for (int i = 0; i < STG; ++i) mbar_init(&full[i], 1);
+    fence_mbar_init();
+  }
+  grid_dep_launch();                       // the gradient kernel may start preloading its inputs
 
-  float X[NJ][4];
+  // the state (or its gradient): warp w holds rows cr = 16 w .. cr + 15 and the block's
+  // four n8 tiles of columns
+  const int cr = 16 * w;
+  float X[4][4];
   {
     const float* init = fwd ? h0 : dhT;
 #pragma unroll
-    for (int nt = 0; nt < NJ; ++nt)
+    for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int c = 16 * w + g + ((e >> 1) << 3), j = j0 + 8 * nt + 2 * qd + (e & 1);
+        const int c = cr + g + ((e >> 1) << 3), j = j0 + 8 * nt + 2 * qd + (e & 1);
         X[nt][e] = init ? init[st_off + (size_t)c * D + j] : 0.f;
       }
   }
-  const int tb = w & 3, jh = w >> 2;       // Delta / dDelta tiles: token block, half of the n8 tiles
-  constexpr int NH = NJ / 2;
+  __syncthreads();                         // the barriers are initialised
+  grid_dep_wait();                         // the records are complete
+  const int tb = w & 3, jh = w >> 2;       // Delta / dDelta tiles: token block, n8 tiles 2 jh, 2 jh + 1
 
-  // the S (or dS) tile as bf16 [j][c], then copied out as rows j0.. of the chunk's image
-  auto put_state = [&](uint32_t tile) {
+  // The S (or dS) tile as bf16 [j][c]; each warp then copies its own 16 channels of the
+  // tile's NB rows j out to rows j0.. of the chunk's image (no barrier needed).
+  auto put_state = [&](uint32_t tile_off, uint8_t* img) {
+    st_nm(sb + tile_off, NB, cr, 0, lane, X[0], X[1], 1.f);
+    st_nm(sb + tile_off, NB, cr, 16, lane, X[2], X[3], 1.f);
+    __syncwarp();
 #pragma unroll
-    for (int p = 0; p < NH; ++p) st_nm(tile, NB, 16 * w, 16 * p, lane, X[2 * p], X[2 * p + 1], 1.f);
-  };
-  auto copy_state = [&](uint32_t tile_off, uint8_t* img) {
-    for (int i = tid; i < NB * 16; i += NTH) {
-      const int pnl = i / (NB * 8), rr = (i >> 3) % NB, ck = i & 7;
-      *reinterpret_cast<uint4*>(img + pnl * 16384 + (j0 + rr) * 128 + ck * 16) =
-          *reinterpret_cast<const uint4*>(sm + tile_off + pnl * NB * 128 + rr * 128 + ck * 16);
+    for (int i = lane; i < 2 * NB; i += 32) {
+      const int rr = i >> 1, ck = (cr >> 3) + (i & 1);          // row j, 16-byte chunk
+      const uint32_t sw = (uint32_t)(((ck & 7) ^ (rr & 7)) << 4);
+      *reinterpret_cast<uint4*>(img + (ck >> 3) * 16384 + (j0 + rr) * 128 + sw) =
+          *reinterpret_cast<const uint4*>(sm + tile_off + (ck >> 3) * NB * 128 + rr * 128 + sw);
     }
+  };
+  // a bounded wait for a stage failed: raise the flag and let the copies in flight land
+  auto give_up = [&](int n_first, int n_last, bool ascending) {
+    if (tid == 0) {
+      atomicExch(&g_bwd_tc_timeout, 1);
+      for (int m = n_first; ascending ? m <= n_last : m >= n_last; m += ascending ? 1 : -1) {
+        const uint32_t use = ascending ? (uint32_t)(m / STG) : (uint32_t)((nch - 1 - m) / STG);
+        mbar_wait(&full[m % STG], use & 1u, kWaitLimit);
+      }
+    }
+    cp_async_wait_all();
+  };
+  // state update: one K step (16 tokens) of A B into X, or into Y (a second accumulator)
+  auto update = [&](uint32_t a_img, uint32_t b_img, float (&Y)[4][4], int ks, bool into_y) {
+    uint32_t a[4], b[4], b2[4];
+    a_mk(a_img, 128, cr, 16 * ks, lane, a);                       // [c][t] image
+    b_kn(b_img, 64, 0, 16 * ks, lane, b);                         // [t][j] tile
+    b_kn(b_img, 64, 16, 16 * ks, lane, b2);
+    float (&u0)[4] = into_y ? Y[0] : X[0];
+    float (&u1)[4] = into_y ? Y[1] : X[1];
+    float (&u2)[4] = into_y ? Y[2] : X[2];
+    float (&u3)[4] = into_y ? Y[3] : X[3];
+    mma(u0, a, b[0], b[1]);
+    mma(u1, a, b[2], b[3]);
+    mma(u2, a, b2[0], b2[1]);
+    mma(u3, a, b2[2], b2[3]);
   };
 
   if (fwd) {
     auto issue = [&](int n) {
-      if (n < nch) {
+      if (tid == NTC - 32 && n < nch) {
         const uint8_t* rc = rec + (base + n) * rec::BYTES_BWD;
         uint8_t* st = sm + (n % STG) * CF::F_STAGE;
-        constexpr int NP = 2048 + NB * 8 + 32;
-        for (int i = tid; i < NP; i += NTH) {
-          uint32_t d, o;
-          if (i < 1024) { d = CF::F_W + 16 * i; o = rec::QW + 16384 + 16 * i; }
-          else if (i < 2048) { d = CF::F_K + 16 * (i - 1024); o = rec::KA + 16 * (i - 1024); }
-          else if (i < 2048 + NB * 8) { d = CF::F_U + 16 * (i - 2048); o = rec::U + j0 * 128 + 16 * (i - 2048); }
-          else { d = CF::F_DEC + 16 * (i - 2048 - NB * 8); o = rec::DECAY + 16 * (i - 2048 - NB * 8); }
-          cp_async16(st + d, rc + o, 16u);
-        }
+        uint64_t* bar = &full[n % STG];
+        fence_async_smem();
+        mbar_arrive_expect_tx(bar, CF::F_BYTES);
+        bulk_g2s(st + CF::F_W, rc + rec::QW + 16384, 16384, bar);
+        bulk_g2s(st + CF::F_K, rc + rec::KA, 16384, bar);
+        bulk_g2s(st + CF::F_U, rc + rec::U + j0 * 128, NB * 128, bar);
+        bulk_g2s(st + CF::F_DEC, rc + rec::DECAY, 512, bar);
       }
-      cp_async_commit();
     };
     const uint32_t uS = sb + CF::F_S, uDL = sb + CF::F_DL;
 #pragma unroll 1
@@ -276,37 +318,31 @@ kda_bwd_chain_kernel(const uint8_t* __restrict__ rec, const float* __restrict__ 
 #pragma unroll 1
     for (int n = 0; n < nch; ++n) {
       const uint32_t so = (uint32_t)(n % STG) * CF::F_STAGE;
-      put_state(uS);                                   // S at the start of chunk n
-      cp_async_wait_group<STG - 2>();
-      __syncthreads();
-      issue(n + STG - 1);
-      copy_state(CF::F_S, simg + (base + n) * kImgS);
-      // Delta = U - W S: token block tb, n8 tiles jh * NH ..
-      float acc[NH][4];
-#pragma unroll
-      for (int p = 0; p < NH; ++p)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[p][e] = 0.f;
+      put_state(CF::F_S, simg + (base + n) * kImgS);   // S at the start of chunk n
+      const bool ok = mbar_wait(&full[n % STG], (uint32_t)(n / STG) & 1u, kWaitLimit);
+      if (__syncthreads_or(!ok)) {
+        give_up(n, min(n + STG - 2, nch - 1), true);
+        return;
+      }
+      // Delta = U - W S: token block tb, n8 tiles 2 jh, 2 jh + 1 (two accumulators each)
+      float acc[2][2][4] = {};
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
-        uint32_t a[4];
+        uint32_t a[4], b[4];
         a_km(sb + so + CF::F_W, 128, 16 * tb, 16 * ks, lane, a);      // W [t][c] from W^T
-#pragma unroll
-        for (int p = 0; p < NH; ++p) {
-          uint32_t b[2];
-          b_nk1(uS, NB, 8 * (jh * NH + p), 16 * ks, lane, b);           // S [c][j] from [j][c]
-          mma(acc[p], a, b[0], b[1]);
-        }
+        b_nk(uS, NB, 16 * jh, 16 * ks, lane, b);                      // S [c][j] from [j][c]
+        mma(acc[0][ks & 1], a, b[0], b[1]);
+        mma(acc[1][ks & 1], a, b[2], b[3]);
       }
       uint8_t* gD = dlimg + (base + n) * kImgD;
 #pragma unroll
-      for (int p = 0; p < NH; ++p) {
-        const int n0 = 8 * (jh * NH + p), jl = n0 + 2 * qd;
+      for (int p = 0; p < 2; ++p) {
+        const int n0 = 16 * jh + 8 * p, jl = n0 + 2 * qd;
         float dl[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int t = 16 * tb + g + ((e >> 1) << 3);
-          dl[e] = bf_at(sm + so + CF::F_U + io(jl + (e & 1), t, NB)) - acc[p][e];
+          dl[e] = bf_at(sm + so + CF::F_U + io(jl + (e & 1), t, NB)) - acc[p][0][e] - acc[p][1][e];
         }
         st_mn1(uDL, 64, 16 * tb, n0, lane, dl, 1.f);
 #pragma unroll
@@ -317,25 +353,20 @@ kda_bwd_chain_kernel(const uint8_t* __restrict__ rec, const float* __restrict__ 
       __syncthreads();
       // S <- Diag(exp(Gamma_last)) S + Kend^T Delta
       const float* dec = reinterpret_cast<const float*>(sm + so + CF::F_DEC);
-      const float d0 = dec[16 * w + g], d1 = dec[16 * w + g + 8];
+      const float d0 = dec[cr + g], d1 = dec[cr + g + 8];
+      float Y[4][4] = {};
 #pragma unroll
-      for (int nt = 0; nt < NJ; ++nt) {
+      for (int nt = 0; nt < 4; ++nt) {
         X[nt][0] *= d0; X[nt][1] *= d0; X[nt][2] *= d1; X[nt][3] *= d1;
       }
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
-        uint32_t a[4];
-        a_mk(sb + so + CF::F_K, 128, 16 * w, 16 * ks, lane, a);       // Kend^T [c][t]
+      for (int ks = 0; ks < 4; ++ks) update(sb + so + CF::F_K, uDL, Y, ks, ks & 1);
 #pragma unroll
-        for (int p = 0; p < NH; ++p) {
-          uint32_t b[4];
-          b_kn(uDL, 64, 16 * p, 16 * ks, lane, b);                    // Delta [t][j]
-          mma(X[2 * p], a, b[0], b[1]);
-          mma(X[2 * p + 1], a, b[2], b[3]);
-        }
-      }
+      for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) X[nt][e] += Y[nt][e];
+      issue(n + STG - 1);               // into chunk n - 1's stage, read before this step's barrier
     }
-    cp_async_wait_all();
     return;
   }
 
@@ -344,21 +375,20 @@ kda_bwd_chain_kernel(const uint8_t* __restrict__ rec, const float* __restrict__ 
     if (n >= 0) {
       const uint8_t* rc = rec + (base + n) * rec::BYTES_BWD;
       uint8_t* st = sm + (n % STG) * CF::R_STAGE;
+      if (tid == NTC - 32) {
+        uint64_t* bar = &full[n % STG];
+        fence_async_smem();
+        mbar_arrive_expect_tx(bar, CF::R_BYTES);
+        bulk_g2s(st + CF::R_QW, rc + rec::QW, 32768, bar);
+        bulk_g2s(st + CF::R_KA, rc + rec::KA, 24576, bar);
+        bulk_g2s(st + CF::R_DEC, rc + rec::DECAY, 512, bar);
+      }
       const long long t0 = t_beg + (long long)n * C;
       const int L = (int)min((long long)C, t_end - t0);
-      constexpr int NP = 2048 + 1536 + 32 + 64 * NJ;
-      for (int i = tid; i < NP; i += NTH) {
-        if (i < 2048) {
-          cp_async16(st + CF::R_QW + 16 * i, rc + rec::QW + 16 * i, 16u);
-        } else if (i < 3584) {
-          cp_async16(st + CF::R_KA + 16 * (i - 2048), rc + rec::KA + 16 * (i - 2048), 16u);
-        } else if (i < 3616) {
-          cp_async16(st + CF::R_DEC + 16 * (i - 3584), rc + rec::DECAY + 16 * (i - 3584), 16u);
-        } else {
-          const int kk = i - 3616, t = kk / NJ, ck = kk % NJ;
-          const bf16* src = dout + ((row0 + t0 + min(t, L - 1)) * H + h) * D + j0 + 8 * ck;
-          cp_async16(st + CF::R_DO + io(t, 8 * ck, 64), src, t < L ? 16u : 0u);
-        }
+      for (int i = tid; i < 64 * CF::NJ; i += NTC) {
+        const int t = i / CF::NJ, ck = i % CF::NJ;
+        const bf16* src = dout + ((row0 + t0 + min(t, L - 1)) * H + h) * D + j0 + 8 * ck;
+        cp_async16(st + CF::R_DO + io(t, 8 * ck, 64), src, t < L ? 16u : 0u);
       }
     }
     cp_async_commit();
@@ -369,93 +399,84 @@ kda_bwd_chain_kernel(const uint8_t* __restrict__ rec, const float* __restrict__ 
 #pragma unroll 1
   for (int n = nch - 1; n >= 0; --n) {
     const uint32_t so = (uint32_t)(n % STG) * CF::R_STAGE;
-    put_state(uY);                                       // dS after chunk n
+    put_state(CF::R_Y, dsimg + (base + n) * kImgS);      // dS after chunk n
     cp_async_wait_group<STG - 2>();
-    __syncthreads();
-    issue(n - (STG - 1));
-    copy_state(CF::R_Y, dsimg + (base + n) * kImgS);
-    // dDelta = Kend dS + Aqk^T dO
-    float acc[NH][4];
-#pragma unroll
-    for (int p = 0; p < NH; ++p)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[p][e] = 0.f;
+    const bool ok = mbar_wait(&full[n % STG], (uint32_t)((nch - 1 - n) / STG) & 1u, kWaitLimit);
+    if (__syncthreads_or(!ok)) {
+      give_up(n, max(n - (STG - 2), 0), false);
+      return;
+    }
+    // dDelta = Kend dS + Aqk^T dO: token block tb, n8 tiles 2 jh, 2 jh + 1
+    float acc[2][2][4] = {};
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
-      uint32_t a[4];
+      uint32_t a[4], b[4];
       a_km(sb + so + CF::R_KA, 128, 16 * tb, 16 * ks, lane, a);          // Kend [t][c] from Kend^T
-#pragma unroll
-      for (int p = 0; p < NH; ++p) {
-        uint32_t b[2];
-        b_nk1(uY, NB, 8 * (jh * NH + p), 16 * ks, lane, b);               // dS [c][j] from [j][c]
-        mma(acc[p], a, b[0], b[1]);
-      }
+      b_nk(uY, NB, 16 * jh, 16 * ks, lane, b);                           // dS [c][j] from [j][c]
+      mma(acc[0][ks & 1], a, b[0], b[1]);
+      mma(acc[1][ks & 1], a, b[2], b[3]);
     }
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) {
-      uint32_t a[4];
+      uint32_t a[4], b[4];
       a_km(sb + so + CF::R_KA + 16384, 64, 16 * tb, 16 * ks, lane, a);   // Aqk^T [t][r] from Aqk
-#pragma unroll
-      for (int p = 0; p < NH; ++p) {
-        uint32_t b[2];
-        b_kn1(sb + so + CF::R_DO, 64, 8 * (jh * NH + p), 16 * ks, lane, b);   // dO [r][j]
-        mma(acc[p], a, b[0], b[1]);
-      }
+      b_kn(sb + so + CF::R_DO, 64, 16 * jh, 16 * ks, lane, b);           // dO [r][j]
+      mma(acc[0][ks & 1], a, b[0], b[1]);
+      mma(acc[1][ks & 1], a, b[2], b[3]);
     }
     uint8_t* gD = ddimg + (base + n) * kImgD;
 #pragma unroll
-    for (int p = 0; p < NH; ++p) {
-      const int n0 = 8 * (jh * NH + p), jl = n0 + 2 * qd;
-      st_mn1(uDD, 64, 16 * tb, n0, lane, acc[p], -1.f);
+    for (int p = 0; p < 2; ++p) {
+      const int n0 = 16 * jh + 8 * p, jl = n0 + 2 * qd;
+      float dd[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) dd[e] = acc[p][0][e] + acc[p][1][e];
+      st_mn1(uDD, 64, 16 * tb, n0, lane, dd, -1.f);
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf)
         *reinterpret_cast<uint32_t*>(gD + io(16 * tb + g + 8 * hf, j0 + jl, 64)) =
-            pack_bf16(acc[p][2 * hf], acc[p][2 * hf + 1]);
+            pack_bf16(dd[2 * hf], dd[2 * hf + 1]);
     }
     __syncthreads();
     // dS <- Diag(exp(Gamma_last)) dS + Qbar^T dO - W^T dDelta
     const float* dec = reinterpret_cast<const float*>(sm + so + CF::R_DEC);
-    const float d0 = dec[16 * w + g], d1 = dec[16 * w + g + 8];
+    const float d0 = dec[cr + g], d1 = dec[cr + g + 8];
+    float Y[4][4] = {};
 #pragma unroll
-    for (int nt = 0; nt < NJ; ++nt) {
+    for (int nt = 0; nt < 4; ++nt) {
       X[nt][0] *= d0; X[nt][1] *= d0; X[nt][2] *= d1; X[nt][3] *= d1;
     }
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) {
-      uint32_t a[4], a2[4];
-      a_mk(sb + so + CF::R_QW, 128, 16 * w, 16 * ks, lane, a);            // Qbar^T [c][t]
-      a_mk(sb + so + CF::R_QW + 16384, 128, 16 * w, 16 * ks, lane, a2);   // W^T [c][t]
-#pragma unroll
-      for (int p = 0; p < NH; ++p) {
-        uint32_t b[4], b2[4];
-        b_kn(sb + so + CF::R_DO, 64, 16 * p, 16 * ks, lane, b);           // dO [t][j]
-        b_kn(uDD, 64, 16 * p, 16 * ks, lane, b2);                         // -dDelta [t][j]
-        mma(X[2 * p], a, b[0], b[1]);
-        mma(X[2 * p + 1], a, b[2], b[3]);
-        mma(X[2 * p], a2, b2[0], b2[1]);
-        mma(X[2 * p + 1], a2, b2[2], b2[3]);
-      }
+      update(sb + so + CF::R_QW, sb + so + CF::R_DO, Y, ks, ks & 1);         // Qbar^T dO
+      update(sb + so + CF::R_QW + 16384, uDD, Y, ks, !(ks & 1));             // W^T (-dDelta)
     }
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) X[nt][e] += Y[nt][e];
+    issue(n - (STG - 1));               // into chunk n + 1's stage, read before this step's barrier
   }
   cp_async_wait_all();
   if (dh0) {
 #pragma unroll
-    for (int nt = 0; nt < NJ; ++nt)
+    for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int c = 16 * w + g + ((e >> 1) << 3), j = j0 + 8 * nt + 2 * qd + (e & 1);
+        const int c = cr + g + ((e >> 1) << 3), j = j0 + 8 * nt + 2 * qd + (e & 1);
         dh0[st_off + (size_t)c * D + j] = X[nt][e];
       }
   }
 }
 
 // ============================================================================
-// Gradient kernel: one CTA per (chunk slot, head), 8 warps.  Warp w owns token
+// Gradient kernel: one CTA per (chunk slot, head), 16 warps.  Warp w owns token
 // rows r0 = 16 tb .. r0 + 15 (tb = w % 4: one decay block) and channels
-// c0 = 64 ch .. c0 + 63 (ch = w / 4) of dq, dk and dGamma in registers: lane
+// c0 = 32 cq .. c0 + 31 (cq = w / 4) of dq, dk and dGamma in registers: lane
 // (g, qd) holds rows r0 + g + 8 hf (hf = 0, 1) and channels c0 + 8 nt + 2 qd + e1
-// (nt = 0..7, e1 = 0, 1), element [nt][2 hf + e1] -- the m16n8 accumulator layout.
+// (nt = 0..3, e1 = 0, 1), element [nt][2 hf + e1] -- the m16n8 accumulator layout.
 // ============================================================================
+constexpr int NTG = 512;                       // threads of the gradient kernel
 constexpr int LDG = 136;                       // Gamma / dGamma row stride (floats)
 constexpr uint32_t G_Q = 0;                    // q image [t][c]
 constexpr uint32_t G_K = 16384;                // k image [t][c]
@@ -477,12 +498,14 @@ __host__ __device__ constexpr uint32_t r_col(int b) {
   return b == 0 ? 0u : b == 1 ? 16384u : b == 2 ? 28672u : 36864u;
 }
 constexpr uint32_t G_RR = G_S0, G_RK = G_S0 + 40960, G_RQ = G_S0 + 81920;
+// factors between the blocks' reference points, fp32 [6][128] each (after the R images)
+constexpr uint32_t G_F1 = G_S0 + 122880, G_F2 = G_F1 + 3072;
 // exact within-block corrections of unsafe channels (phase 4, after the products):
 // fp32 [64][128] each
 constexpr uint32_t G_CYA = G_S0, G_CYQ = G_S0 + 32768, G_CZ = G_S0 + 65536;
 
 template <bool GRPD>
-__global__ void __launch_bounds__(NTH, 1)
+__global__ void __launch_bounds__(NTG, 1)
 kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
                     const bf16* __restrict__ v, const float* __restrict__ g,
                     const float* __restrict__ beta, const bf16* __restrict__ dout,
@@ -495,8 +518,8 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   const uint32_t sb = smem_u32(sm);
-  __shared__ float s_beta[C], s_dbeta[C], s_dgl[D], s_half[D];
-  __shared__ uint8_t s_uns[4][D];
+  __shared__ float s_beta[C], s_dbeta[C], s_dgl[D], s_part[4][D];
+  __shared__ __align__(16) uint8_t s_uns[4][D];
 
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31, g8 = lane >> 2, qd = lane & 3;
   const long long slot = blockIdx.x;
@@ -528,14 +551,8 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   const uint8_t* rc = rec + ix * rec::BYTES_BWD;
   float* G = reinterpret_cast<float*>(sm + G_G);
 
-  // ---- phase 0: loads
-  for (int i = tid; i < 2048; i += NTH) {
-    cp_async16(sm + G_S0 + 16 * i, simg + ix * kImgS + 16 * i, 16u);
-    cp_async16(sm + G_DS + 16 * i, dsimg + ix * kImgS + 16 * i, 16u);
-  }
-  for (int i = tid; i < 1024; i += NTH) {
-    cp_async16(sm + G_DL + 16 * i, dlimg + ix * kImgD + 16 * i, 16u);
-    cp_async16(sm + G_DD + 16 * i, ddimg + ix * kImgD + 16 * i, 16u);
+  // ---- phase 0: loads (the inputs first; the chains' images once the chains are done)
+  for (int i = tid; i < 1024; i += NTG) {
     const int t = i >> 4, c8 = i & 15;
     const long long src = ((rb + min(t, L - 1)) * H + h) * D + 8 * c8;
     const uint32_t ok = t < L ? 16u : 0u;
@@ -544,11 +561,21 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     cp_async16(sm + G_K + io(t, 8 * c8, 64), k + src, ok);
   }
   if constexpr (!GRPD) {
-    for (int i = tid; i < 2048; i += NTH) {
+    for (int i = tid; i < 2048; i += NTG) {
       const int t = i >> 5, c4 = i & 31;
       cp_async16(G + t * LDG + 4 * c4, g + ((rb + min(t, L - 1)) * H + h) * D + 4 * c4,
                  t < L ? 16u : 0u);
     }
+  }
+  cp_async_commit();
+  grid_dep_wait();
+  for (int i = tid; i < 2048; i += NTG) {
+    cp_async16(sm + G_S0 + 16 * i, simg + ix * kImgS + 16 * i, 16u);
+    cp_async16(sm + G_DS + 16 * i, dsimg + ix * kImgS + 16 * i, 16u);
+  }
+  for (int i = tid; i < 1024; i += NTG) {
+    cp_async16(sm + G_DL + 16 * i, dlimg + ix * kImgD + 16 * i, 16u);
+    cp_async16(sm + G_DD + 16 * i, ddimg + ix * kImgD + 16 * i, 16u);
   }
   cp_async_commit();
   if (tid < C) {
@@ -558,61 +585,84 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   if (tid < D) s_dgl[tid] = 0.f;
   if constexpr (GRPD) {
     const int ng = D >> gsh;
-    for (int i = tid; i < C * D; i += NTH) {
+    for (int i = tid; i < C * D; i += NTG) {
       const int t = i >> 7, c = i & 127;
       G[t * LDG + c] = t < L ? g[((rb + t) * H + h) * ng + (c >> gsh)] : 0.f;
     }
   }
+  cp_async_wait_group<1>();             // the inputs (the images may still be in flight)
+  __syncthreads();
+  // Gamma = cumsum g per channel: four threads per channel, 16 rows each
+  {
+    const int c = tid & 127, part = tid >> 7;
+    float x[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) x[e] = G[(16 * part + e) * LDG + c];
+#pragma unroll
+    for (int e = 1; e < 16; ++e) x[e] += x[e - 1];
+    s_part[part][c] = x[15];
+    __syncthreads();
+    float add = 0.f;
+    for (int p2 = 0; p2 < part; ++p2) add += s_part[p2][c];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) G[(16 * part + e) * LDG + c] = x[e] + add;
+  }
   cp_async_wait_all();
   __syncthreads();
-  // Gamma = cumsum g per channel: two threads per channel, 32 rows each
-  {
-    const int c = tid & 127, part = tid >> 7;
-    float x[32];
-#pragma unroll
-    for (int e = 0; e < 32; ++e) x[e] = G[(32 * part + e) * LDG + c];
-#pragma unroll
-    for (int e = 1; e < 32; ++e) x[e] += x[e - 1];
-    if (part == 0) s_half[c] = x[31];
-    __syncthreads();
-    const float add = part ? s_half[c] : 0.f;
-#pragma unroll
-    for (int e = 0; e < 32; ++e) G[(32 * part + e) * LDG + c] = x[e] + add;
-  }
-  __syncthreads();
-  // unsafe (block, channel) pairs; and dGamma_last's state term e^Gamma_last sum_j S dS
+  // unsafe (block, channel) pairs; dGamma_last's state term e^Gamma_last sum_j S dS
   bool any_uns = false;
   {
-    const int c = tid & 127, part = tid >> 7;
+    const int c = tid & 127, a = tid >> 7;
+    const bool u = G[16 * a * LDG + c] - G[(16 * a + 15) * LDG + c] > kUnsafeDecay;
+    s_uns[a][c] = u ? 1 : 0;
+    any_uns = u;
+    const int c8 = tid & 15, jg = tid >> 4;           // 32 groups of 4 rows j
+    float acc[8];
 #pragma unroll
-    for (int a2 = 0; a2 < 2; ++a2) {
-      const int a = 2 * part + a2;
-      const bool u = G[16 * a * LDG + c] - G[(16 * a + 15) * LDG + c] > kUnsafeDecay;
-      s_uns[a][c] = u ? 1 : 0;
-      any_uns |= u;
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      const int j = 4 * jg + jj;
+      const uint4 a4 = *reinterpret_cast<const uint4*>(sm + G_S0 + io(j, 8 * c8, 128));
+      const uint4 b4 = *reinterpret_cast<const uint4*>(sm + G_DS + io(j, 8 * c8, 128));
+      const uint32_t aw[4] = {a4.x, a4.y, a4.z, a4.w}, bw[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        acc[2 * e] = fmaf(__uint_as_float(aw[e] << 16), __uint_as_float(bw[e] << 16), acc[2 * e]);
+        acc[2 * e + 1] = fmaf(__uint_as_float(aw[e] & 0xffff0000u),
+                              __uint_as_float(bw[e] & 0xffff0000u), acc[2 * e + 1]);
+      }
     }
-    float acc = 0.f;
-#pragma unroll 8
-    for (int j = 64 * part; j < 64 * part + 64; ++j)
-      acc = fmaf(bf_at(sm + G_S0 + io(j, c, 128)), bf_at(sm + G_DS + io(j, c, 128)), acc);
-    atomicAdd(&s_dgl[c], acc * __expf(G[63 * LDG + c]));
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 16);
+    if (lane < 16) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        atomicAdd(&s_dgl[8 * c8 + e], acc[e] * __expf(G[63 * LDG + 8 * c8 + e]));
+    }
   }
   const bool fix = __syncthreads_or(any_uns) != 0;
 
-  const int tb = w & 3, ch = w >> 2, r0 = 16 * tb, c0 = 64 * ch;
-  float dQ[8][4], dK[8][4], dG[8][4];
+  const int tb = w & 3, cq = w >> 2, r0 = 16 * tb, c0 = 32 * cq;
+  float dQ[4][4], dK[4][4], dG[4][4];
 #pragma unroll
-  for (int nt = 0; nt < 8; ++nt)
+  for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
     for (int e = 0; e < 4; ++e) dQ[nt][e] = dK[nt][e] = dG[nt][e] = 0.f;
-  // element helpers: row, column of accumulator element e of n8 tile nt (this warp's tile)
-  auto erow = [&](int e) { return r0 + g8 + ((e >> 1) << 3); };
-  auto ecol = [&](int nt, int e) { return c0 + 8 * nt + 2 * qd + (e & 1); };
-  auto qk = [&](uint32_t img, int r, int c) { return bf_at(sm + img + io(r, c, 64)); };
+  // The element pair (e = 2 hf, 2 hf + 1) of n8 tile nt: row r0 + g8 + 8 hf, columns
+  // c0 + 8 nt + 2 qd (+1).  Its values in a [t][c] image and in Gamma:
+  const uint32_t prow = (uint32_t)(cq >> 1) * 8192u + (uint32_t)(r0 + g8) * 128u + (uint32_t)qd * 4u;
+  const int cb = 4 * (cq & 1);                 // the tile's first 16-byte chunk in its panel
+  auto img2 = [&](uint32_t img, int hf, int nt) -> float2 {
+    return bf2_at(sm + img + prow + hf * 1024 + (((cb + nt) ^ g8) << 4));
+  };
+  auto gam2 = [&](int row, int nt) -> float2 {
+    return *reinterpret_cast<const float2*>(G + row * LDG + c0 + 8 * nt + 2 * qd);
+  };
 
   // ---- phase 1: dQbar and dW (against S^T), dKend (dS^T), dAqk
 #pragma unroll
-  for (int np = 0; np < 4; ++np) {
+  for (int np = 0; np < 2; ++np) {
     float aq[2][4] = {}, aw[2][4] = {};
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
@@ -629,20 +679,23 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     for (int sub = 0; sub < 2; ++sub) {
       const int nt = 2 * np + sub;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int r = erow(e), c = ecol(nt, e);
-        const float eg = __expf(G[r * LDG + c]);
-        dQ[nt][e] = fmaf(aq[sub][e], eg, dQ[nt][e]);
-        dG[nt][e] = fmaf(aq[sub][e] * qk(G_Q, r, c), eg, dG[nt][e]);
+      for (int hf = 0; hf < 2; ++hf) {
+        const float2 gp = gam2(r0 + g8 + 8 * hf, nt), qv = img2(G_Q, hf, nt);
+        const float e0 = __expf(gp.x), e1 = __expf(gp.y);
+        const float x0 = aq[sub][2 * hf], x1 = aq[sub][2 * hf + 1];
+        dQ[nt][2 * hf] = fmaf(x0, e0, dQ[nt][2 * hf]);
+        dQ[nt][2 * hf + 1] = fmaf(x1, e1, dQ[nt][2 * hf + 1]);
+        dG[nt][2 * hf] = fmaf(x0 * qv.x, e0, dG[nt][2 * hf]);
+        dG[nt][2 * hf + 1] = fmaf(x1 * qv.y, e1, dG[nt][2 * hf + 1]);
       }
     }
     st_mn(sb + G_DW, 64, r0, c0 + 16 * np, lane, aw[0], aw[1], -1.f);   // dW = -dDelta S^T
   }
   __syncthreads();                      // S image no longer read: T and A go there
-  for (int i = tid; i < 2048; i += NTH) cp_async16(sm + G_S0 + 16 * i, rc + rec::TMAT + 16 * i, 16u);
+  for (int i = tid; i < 2048; i += NTG) cp_async16(sm + G_S0 + 16 * i, rc + rec::TMAT + 16 * i, 16u);
   cp_async_commit();
 #pragma unroll
-  for (int np = 0; np < 4; ++np) {
+  for (int np = 0; np < 2; ++np) {
     float ak[2][4] = {};
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
@@ -655,67 +708,75 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
 #pragma unroll
     for (int sub = 0; sub < 2; ++sub) {
       const int nt = 2 * np + sub;
-      float cs[2] = {0.f, 0.f};
+      const float2 gl = gam2(63, nt);
+      float cs0 = 0.f, cs1 = 0.f;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int r = erow(e), c = ecol(nt, e);
-        const float ee = __expf(G[63 * LDG + c] - G[r * LDG + c]);
-        dK[nt][e] = fmaf(ak[sub][e], ee, dK[nt][e]);
-        const float tk = ak[sub][e] * qk(G_K, r, c) * ee;
-        dG[nt][e] -= tk;
-        cs[e & 1] += tk;
+      for (int hf = 0; hf < 2; ++hf) {
+        const float2 gp = gam2(r0 + g8 + 8 * hf, nt), kv = img2(G_K, hf, nt);
+        const float e0 = __expf(gl.x - gp.x), e1 = __expf(gl.y - gp.y);
+        const float x0 = ak[sub][2 * hf], x1 = ak[sub][2 * hf + 1];
+        dK[nt][2 * hf] = fmaf(x0, e0, dK[nt][2 * hf]);
+        dK[nt][2 * hf + 1] = fmaf(x1, e1, dK[nt][2 * hf + 1]);
+        const float t0v = x0 * kv.x * e0, t1v = x1 * kv.y * e1;
+        dG[nt][2 * hf] -= t0v;
+        dG[nt][2 * hf + 1] -= t1v;
+        cs0 += t0v;
+        cs1 += t1v;
       }
 #pragma unroll
-      for (int e1 = 0; e1 < 2; ++e1) {
-        float x = cs[e1];
-        x += __shfl_xor_sync(0xffffffffu, x, 4);
-        x += __shfl_xor_sync(0xffffffffu, x, 8);
-        x += __shfl_xor_sync(0xffffffffu, x, 16);
-        if (g8 == 0) atomicAdd(&s_dgl[c0 + 8 * nt + 2 * qd + e1], x);
+      for (int m = 4; m < 32; m <<= 1) {
+        cs0 += __shfl_xor_sync(0xffffffffu, cs0, m);
+        cs1 += __shfl_xor_sync(0xffffffffu, cs1, m);
+      }
+      if (g8 == 0) {
+        atomicAdd(&s_dgl[c0 + 8 * nt + 2 * qd], cs0);
+        atomicAdd(&s_dgl[c0 + 8 * nt + 2 * qd + 1], cs1);
       }
     }
   }
-  {   // dAqk (rows r0.., columns 32 ch ..), lower triangle
-    const bool live = ch == 0 || tb >= 2;
+  {   // dAqk (rows r0.., columns 16 cq ..), lower triangle
+    float aa[2][4] = {};
+    if (cq <= tb) {
 #pragma unroll
-    for (int np = 0; np < 2; ++np) {
-      float aa[2][4] = {};
-      if (live) {
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          uint32_t a[4], b[4];
-          a_mk(sb + G_DO, 64, r0, 16 * ks, lane, a);
-          b_nk(sb + G_DL, 64, 32 * ch + 16 * np, 16 * ks, lane, b);   // Delta^T from Delta [i][j]
-          mma(aa[0], a, b[0], b[1]);
-          mma(aa[1], a, b[2], b[3]);
-        }
-#pragma unroll
-        for (int sub = 0; sub < 2; ++sub)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int r = erow(e), i = 32 * ch + 16 * np + 8 * sub + 2 * qd + (e & 1);
-            if (i > r) aa[sub][e] = 0.f;
-          }
+      for (int ks = 0; ks < 8; ++ks) {
+        uint32_t a[4], b[4];
+        a_mk(sb + G_DO, 64, r0, 16 * ks, lane, a);
+        b_nk(sb + G_DL, 64, 16 * cq, 16 * ks, lane, b);             // Delta^T from Delta [i][j]
+        mma(aa[0], a, b[0], b[1]);
+        mma(aa[1], a, b[2], b[3]);
       }
-      st_mn(sb + G_AQK, 64, r0, 32 * ch + 16 * np, lane, aa[0], aa[1], 1.f);
+#pragma unroll
+      for (int sub = 0; sub < 2; ++sub)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int r = r0 + g8 + ((e >> 1) << 3);
+          const int i = 16 * cq + 8 * sub + 2 * qd + (e & 1);
+          if (i > r) aa[sub][e] = 0.f;
+        }
     }
+    st_mn(sb + G_AQK, 64, r0, 16 * cq, lane, aa[0], aa[1], 1.f);
   }
   __syncthreads();                      // dO, Delta, dS no longer read
-  for (int i = tid; i < 1024; i += NTH) {
+  for (int i = tid; i < 1024; i += NTG) {
     const int t = i >> 4, c8 = i & 15;
     cp_async16(sm + G_DO + io(t, 8 * c8, 64), v + ((rb + min(t, L - 1)) * H + h) * D + 8 * c8,
                t < L ? 16u : 0u);
   }
   cp_async_commit();
   // Kb = diag(beta) Kbar = beta k e^Gamma (image [i][c] at G_DS)
-  for (int i = tid; i < 1024; i += NTH) {
+  for (int i = tid; i < 1024; i += NTG) {
     const int t = i >> 4, c8 = i & 15;
     const float bt = s_beta[t];
+    const float4 ga = *reinterpret_cast<const float4*>(G + t * LDG + 8 * c8);
+    const float4 gb = *reinterpret_cast<const float4*>(G + t * LDG + 8 * c8 + 4);
+    const uint4 kw = *reinterpret_cast<const uint4*>(sm + G_K + io(t, 8 * c8, 64));
+    const float gv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+    const uint32_t kk[4] = {kw.x, kw.y, kw.z, kw.w};
     float x[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int c = 8 * c8 + e;
-      x[e] = bt * qk(G_K, t, c) * __expf(G[t * LDG + c]);
+    for (int e = 0; e < 4; ++e) {
+      x[2 * e] = bt * __uint_as_float(kk[e] << 16) * __expf(gv[2 * e]);
+      x[2 * e + 1] = bt * __uint_as_float(kk[e] & 0xffff0000u) * __expf(gv[2 * e + 1]);
     }
     *reinterpret_cast<uint4*>(sm + G_DS + io(t, 8 * c8, 64)) =
         make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
@@ -726,23 +787,25 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   const float* Tm = reinterpret_cast<const float*>(sm + G_S0);           // T [r][i]
   const float* Am = reinterpret_cast<const float*>(sm + G_S0 + 16384);   // A [r][i]
   // T image (bf16 [r][i] at G_DL) and Vb = diag(beta) V (image [i][j] at G_DS + 16384)
-  for (int i = tid; i < 1536; i += NTH) {
-    float x[8];
+  for (int i = tid; i < 1536; i += NTG) {
     if (i < 512) {
       const int r = i >> 3, c8 = i & 7;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) x[e] = Tm[r * 64 + 8 * c8 + e];
+      const float4 a4 = *reinterpret_cast<const float4*>(Tm + r * 64 + 8 * c8);
+      const float4 b4 = *reinterpret_cast<const float4*>(Tm + r * 64 + 8 * c8 + 4);
       *reinterpret_cast<uint4*>(sm + G_DL + io(r, 8 * c8, 64)) =
-          make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
-                     pack_bf16(x[6], x[7]));
+          make_uint4(pack_bf16(a4.x, a4.y), pack_bf16(a4.z, a4.w), pack_bf16(b4.x, b4.y),
+                     pack_bf16(b4.z, b4.w));
     } else {
       const int t = (i - 512) >> 4, c8 = (i - 512) & 15;
       const float bt = s_beta[t];
+      const uint4 vw = *reinterpret_cast<const uint4*>(sm + G_DO + io(t, 8 * c8, 64));
+      const uint32_t vv[4] = {vw.x, vw.y, vw.z, vw.w};
+      uint32_t o[4];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) x[e] = bt * qk(G_DO, t, 8 * c8 + e);
+      for (int e = 0; e < 4; ++e)
+        o[e] = pack_bf16(bt * __uint_as_float(vv[e] << 16), bt * __uint_as_float(vv[e] & 0xffff0000u));
       *reinterpret_cast<uint4*>(sm + G_DS + 16384 + io(t, 8 * c8, 64)) =
-          make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
-                     pack_bf16(x[6], x[7]));
+          make_uint4(o[0], o[1], o[2], o[3]);
     }
   }
   __syncthreads();
@@ -751,7 +814,7 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   {
     float dbp[2] = {0.f, 0.f};                 // dbeta parts of rows r0 + g8 (+8)
 #pragma unroll
-    for (int np = 0; np < 4; ++np) {
+    for (int np = 0; np < 2; ++np) {
       float av[2][4] = {}, ak[2][4] = {};
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks) {
@@ -772,22 +835,19 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
         for (int hf = 0; hf < 2; ++hf) {
           const int i = r0 + g8 + 8 * hf, c = c0 + 8 * nt + 2 * qd;
           const float bi = s_beta[i];
-          const float2 vv = bf2_at(sm + G_DO + io(i, c, 64));
+          const float2 vv = img2(G_DO, hf, nt), kv = img2(G_K, hf, nt), gp = gam2(i, nt);
           const float x0 = av[sub][2 * hf], x1 = av[sub][2 * hf + 1];
           if (i < L)
             *reinterpret_cast<float2*>(dv + ((rb + i) * H + h) * D + c) =
                 make_float2(bi * x0, bi * x1);
-          dbp[hf] += x0 * vv.x + x1 * vv.y;
-#pragma unroll
-          for (int e1 = 0; e1 < 2; ++e1) {
-            const int e = 2 * hf + e1;
-            const float eg = __expf(G[i * LDG + c + e1]);
-            const float kb = qk(G_K, i, c + e1) * eg;          // Kbar
-            const float y = ak[sub][e];
-            dK[nt][e] = fmaf(bi * y, eg, dK[nt][e]);
-            dG[nt][e] = fmaf(bi * y, kb, dG[nt][e]);
-            dbp[hf] = fmaf(y, kb, dbp[hf]);
-          }
+          const float e0 = __expf(gp.x), e1 = __expf(gp.y);
+          const float kb0 = kv.x * e0, kb1 = kv.y * e1;             // Kbar
+          const float y0 = ak[sub][2 * hf], y1 = ak[sub][2 * hf + 1];
+          dK[nt][2 * hf] = fmaf(bi * y0, e0, dK[nt][2 * hf]);
+          dK[nt][2 * hf + 1] = fmaf(bi * y1, e1, dK[nt][2 * hf + 1]);
+          dG[nt][2 * hf] = fmaf(bi * y0, kb0, dG[nt][2 * hf]);
+          dG[nt][2 * hf + 1] = fmaf(bi * y1, kb1, dG[nt][2 * hf + 1]);
+          dbp[hf] += x0 * vv.x + x1 * vv.y + y0 * kb0 + y1 * kb1;
         }
       }
     }
@@ -799,163 +859,231 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       if (qd == 0) atomicAdd(&s_dbeta[r0 + g8 + 8 * hf], x);
     }
   }
-  __syncthreads();                      // V and the T image no longer read
+  __syncthreads();                      // V no longer read
 
-  // ---- phase 3: dT = dDelta Vb^T + dW Kb^T (strictly lower part), stored as dT^T
-  float* dTt = reinterpret_cast<float*>(sm + G_DO);    // [i][r], stride 68
-  if (ch == 0 || tb >= 2) {
-#pragma unroll
-    for (int np = 0; np < 2; ++np) {
-      float at[2][4] = {};
+  // ---- phase 3: dT = dDelta Vb^T + dW Kb^T, X = dT T^T, dM = -T^T X (strictly lower),
+  // on the tensor cores: dT and X as bf16 images [r][i], [r][b] at G_DO, G_DO + 8192
+  {                                     // dT tile: rows r0 .., columns i = 16 cq ..
+    float at[2][2][4] = {};             // two accumulator pairs: even / odd K steps
+    if (cq <= tb) {                     // (tiles above the diagonal are never read: zeros)
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
         uint32_t a[4], b[4];
         a_mk(sb + G_DD, 64, r0, 16 * ks, lane, a);
-        b_nk(sb + G_DS + 16384, 64, 32 * ch + 16 * np, 16 * ks, lane, b);   // Vb^T from Vb [i][j]
-        mma(at[0], a, b[0], b[1]);
-        mma(at[1], a, b[2], b[3]);
+        b_nk(sb + G_DS + 16384, 64, 16 * cq, 16 * ks, lane, b);   // Vb^T from Vb [i][j]
+        mma(at[ks & 1][0], a, b[0], b[1]);
+        mma(at[ks & 1][1], a, b[2], b[3]);
       }
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
         uint32_t a[4], b[4];
         a_mk(sb + G_DW, 64, r0, 16 * ks, lane, a);
-        b_nk(sb + G_DS, 64, 32 * ch + 16 * np, 16 * ks, lane, b);           // Kb^T from Kb [i][c]
-        mma(at[0], a, b[0], b[1]);
-        mma(at[1], a, b[2], b[3]);
+        b_nk(sb + G_DS, 64, 16 * cq, 16 * ks, lane, b);           // Kb^T from Kb [i][c]
+        mma(at[ks & 1][0], a, b[0], b[1]);
+        mma(at[ks & 1][1], a, b[2], b[3]);
+      }
+#pragma unroll
+      for (int sub = 0; sub < 2; ++sub)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) at[0][sub][e] += at[1][sub][e];
+    }
+    st_mn(sb + G_DO, 64, r0, 16 * cq, lane, at[0][0], at[0][1], 1.f);
+  }
+  __syncthreads();
+  {                                     // X tile: rows r0 .., columns b = 16 cq .. (r > b only)
+    float ax[2][4] = {};
+    if (cq <= tb) {
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        if (ks > cq) continue;          // T[b][i] = 0 for i > b
+        uint32_t a[4], b[4];
+        a_mk(sb + G_DO, 64, r0, 16 * ks, lane, a);                  // dT [r][i]
+        b_nk(sb + G_DL, 64, 16 * cq, 16 * ks, lane, b);             // T^T from T [b][i]
+        mma(ax[0], a, b[0], b[1]);
+        mma(ax[1], a, b[2], b[3]);
       }
 #pragma unroll
       for (int sub = 0; sub < 2; ++sub)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int r = erow(e), i = 32 * ch + 16 * np + 8 * sub + 2 * qd + (e & 1);
-          dTt[i * 68 + r] = at[sub][e];
+          const int r = r0 + g8 + ((e >> 1) << 3), bb = 16 * cq + 8 * sub + 2 * qd + (e & 1);
+          if (r <= bb) ax[sub][e] = 0.f;
         }
     }
-  }
-  __syncthreads();                      // dDelta, dW, Kb, Vb no longer read
-  float* Tt = reinterpret_cast<float*>(sm + G_DD);     // T^T [i][b], stride 68
-  for (int i = tid; i < 4096; i += NTH) {
-    const int b = i >> 6, ii = i & 63;
-    Tt[ii * 68 + b] = Tm[b * 64 + ii];
+    st_mn(sb + G_DO + 8192, 64, r0, 16 * cq, lane, ax[0], ax[1], 1.f);
   }
   __syncthreads();
-  // X[r][b] = sum_i dT[r][i] T[b][i] (needed for r > b; i <= b < r) -> G_DS, stride 68
-  float* Xm = reinterpret_cast<float*>(sm + G_DS);
-  {
-    const int rt = tid >> 4, bt = tid & 15;
-    float acc[4][4] = {};
-    if (rt >= bt) {
-#pragma unroll 4
-      for (int i = 0; i < 4 * bt + 4; ++i) {
-        const float4 x4 = *reinterpret_cast<const float4*>(dTt + i * 68 + 4 * rt);
-        const float4 t4 = *reinterpret_cast<const float4*>(Tt + i * 68 + 4 * bt);
-        const float xv[4] = {x4.x, x4.y, x4.z, x4.w}, tv[4] = {t4.x, t4.y, t4.z, t4.w};
+  {                                     // dM tile: rows a = r0 .., columns b = 16 cq ..
+    float am[2][4] = {};
+    if (cq <= tb) {
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-          for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(xv[a], tv[b], acc[a][b]);
+      for (int ks = 0; ks < 4; ++ks) {
+        if (ks < tb) continue;          // T[r][a] = 0 for r < a
+        uint32_t a[4], b[4];
+        a_km(sb + G_DL, 64, r0, 16 * ks, lane, a);                  // T^T [a][r] from T [r][a]
+        b_kn(sb + G_DO + 8192, 64, 16 * cq, 16 * ks, lane, b);      // X [r][b]
+        mma(am[0], a, b[0], b[1]);
+        mma(am[1], a, b[2], b[3]);
       }
     }
+    float dbp[2] = {0.f, 0.f};
 #pragma unroll
-    for (int a = 0; a < 4; ++a) {
-      float4 o;
-      o.x = (4 * rt + a > 4 * bt + 0) ? acc[a][0] : 0.f;
-      o.y = (4 * rt + a > 4 * bt + 1) ? acc[a][1] : 0.f;
-      o.z = (4 * rt + a > 4 * bt + 2) ? acc[a][2] : 0.f;
-      o.w = (4 * rt + a > 4 * bt + 3) ? acc[a][3] : 0.f;
-      *reinterpret_cast<float4*>(Xm + (4 * rt + a) * 68 + 4 * bt) = o;
-    }
-  }
-  __syncthreads();
-  // dM[a][b] = -sum_{r >= a} T[r][a] X[r][b] (a > b); dA = diag(beta) dM (image);
-  // dbeta_a += sum_b dM[a][b] A[a][b]
-  {
-    const int at = tid >> 4, bt = tid & 15;
-    float acc[4][4] = {};
-    if (at >= bt) {
-#pragma unroll 4
-      for (int r = 4 * at; r < 64; ++r) {
-        const float4 t4 = *reinterpret_cast<const float4*>(Tm + r * 64 + 4 * at);
-        const float4 x4 = *reinterpret_cast<const float4*>(Xm + r * 68 + 4 * bt);
-        const float tv[4] = {t4.x, t4.y, t4.z, t4.w}, xv[4] = {x4.x, x4.y, x4.z, x4.w};
+    for (int sub = 0; sub < 2; ++sub)
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-          for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(tv[a], xv[b], acc[a][b]);
+      for (int hf = 0; hf < 2; ++hf) {
+        const int ra = r0 + g8 + 8 * hf, bb = 16 * cq + 8 * sub + 2 * qd;
+        const float m0 = ra > bb ? -am[sub][2 * hf] : 0.f;
+        const float m1 = ra > bb + 1 ? -am[sub][2 * hf + 1] : 0.f;
+        const float2 a2 = *reinterpret_cast<const float2*>(Am + ra * 64 + bb);
+        dbp[hf] += m0 * a2.x + m1 * a2.y;
+        am[sub][2 * hf] = s_beta[ra] * m0;
+        am[sub][2 * hf + 1] = s_beta[ra] * m1;
       }
-    }
-    float dbp[4];
+    st_mn(sb + G_DA, 64, r0, 16 * cq, lane, am[0], am[1], 1.f);   // dA = diag(beta) dM
 #pragma unroll
-    for (int a = 0; a < 4; ++a) {
-      const int ra = 4 * at + a;
-      const float ba = s_beta[ra];
-      float m[4];
-      dbp[a] = 0.f;
-#pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        m[b] = (ra > 4 * bt + b) ? -acc[a][b] : 0.f;
-        dbp[a] = fmaf(m[b], Am[ra * 64 + 4 * bt + b], dbp[a]);
-      }
-      *reinterpret_cast<uint2*>(sm + G_DA + io(ra, 4 * bt, 64)) =
-          make_uint2(pack_bf16(ba * m[0], ba * m[1]), pack_bf16(ba * m[2], ba * m[3]));
-    }
-#pragma unroll
-    for (int a = 0; a < 4; ++a) {
-      float x = dbp[a];
+    for (int hf = 0; hf < 2; ++hf) {
+      float x = dbp[hf];
       x += __shfl_xor_sync(0xffffffffu, x, 1);
       x += __shfl_xor_sync(0xffffffffu, x, 2);
-      x += __shfl_xor_sync(0xffffffffu, x, 4);
-      x += __shfl_xor_sync(0xffffffffu, x, 8);
-      if (bt == 0) atomicAdd(&s_dbeta[4 * at + a], x);
+      if (qd == 0) atomicAdd(&s_dbeta[r0 + g8 + 8 * hf], x);
     }
   }
-  __syncthreads();                      // T, A, X, dT^T no longer read
+  __syncthreads();                      // T, A, dT, X no longer read
 
   // ---- phase 4: the decay-weighted Gram products
   // R^(a)[i][c] = k_ic e^{G_16a,c - G_ic}, i < 16(a+1) (block a's own rows zero where
-  // unsafe); R'x^(b)[r - 16b][c] = x_rc e^{G_rc - G_16b+15,c}, r >= 16b (likewise)
-  for (int i = tid; i < 160 * 16; i += NTH) {
-    const int row = i >> 4, c8 = i & 15;
-    int a = 0;
-    while (row >= (a + 1) * (a + 2) * 8) ++a;         // rows of R^(0..3): 16, 32, 48, 64
-    const int ii = row - a * (a + 1) * 8;
-    float x[8];
+  // unsafe); R'x^(b)[r - 16b][c] = x_rc e^{G_rc - G_16b+15,c}, r >= 16b (likewise).
+  // One item: 8 channels of one row of one image.
+  auto build_r = [&](bool flags) {
+    for (int i = tid; i < 160 * 16; i += NTG) {
+      const int x = i >> 4, c8 = i & 15;
+      const int a = x >= 96 ? 3 : x >= 48 ? 2 : x >= 16 ? 1 : 0;
+      const int ii = x - 8 * a * (a + 1);
+      const float* gi = G + ii * LDG + 8 * c8;
+      const float* ga = G + 16 * a * LDG + 8 * c8;
+      const float4 i0 = *reinterpret_cast<const float4*>(gi), i1 = *reinterpret_cast<const float4*>(gi + 4);
+      const float4 a0 = *reinterpret_cast<const float4*>(ga), a1 = *reinterpret_cast<const float4*>(ga + 4);
+      const uint4 kw = *reinterpret_cast<const uint4*>(sm + G_K + io(ii, 8 * c8, 64));
+      const float dgv[8] = {a0.x - i0.x, a0.y - i0.y, a0.z - i0.z, a0.w - i0.w,
+                            a1.x - i1.x, a1.y - i1.y, a1.z - i1.z, a1.w - i1.w};
+      const uint32_t kk[4] = {kw.x, kw.y, kw.z, kw.w};
+      uint32_t zm = 0;                  // channels whose within-block entries are zero
+      if (flags && ii >= 16 * a) {
+        const uint2 un = *reinterpret_cast<const uint2*>(&s_uns[a][8 * c8]);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int c = 8 * c8 + e;
-      const bool zero = ii >= 16 * a && s_uns[a][c];
-      const float ex = fminf(G[16 * a * LDG + c] - G[ii * LDG + c], 80.f);
-      x[e] = zero ? 0.f : qk(G_K, ii, c) * __expf(ex);
-    }
-    *reinterpret_cast<uint4*>(sm + G_RR + r_row(a) + io(ii, 8 * c8, 16 * (a + 1))) =
-        make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
-                   pack_bf16(x[6], x[7]));
-  }
-  for (int i = tid; i < 160 * 16; i += NTH) {
-    const int row = i >> 4, c8 = i & 15;
-    int b = 0, acc_rows = 0;
-    while (row >= acc_rows + (64 - 16 * b)) { acc_rows += 64 - 16 * b; ++b; }
-    const int rr = row - acc_rows, r = 16 * b + rr, nrows = 64 - 16 * b;
-    float xk[8], xq[8];
+        for (int e = 0; e < 8; ++e) zm |= (((e < 4 ? un.x : un.y) >> (8 * (e & 3))) & 1u) << e;
+      }
+      uint32_t o[4];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int c = 8 * c8 + e;
-      const bool zero = rr < 16 && s_uns[b][c];
-      const float f = __expf(fminf(G[r * LDG + c] - G[(16 * b + 15) * LDG + c], 80.f));
-      xk[e] = zero ? 0.f : qk(G_K, r, c) * f;
-      xq[e] = zero ? 0.f : qk(G_Q, r, c) * f;
+      for (int e = 0; e < 4; ++e) {
+        const float v0 = __uint_as_float(kk[e] << 16) * __expf(fminf(dgv[2 * e], 80.f));
+        const float v1 = __uint_as_float(kk[e] & 0xffff0000u) * __expf(fminf(dgv[2 * e + 1], 80.f));
+        o[e] = pack_bf16(((zm >> (2 * e)) & 1u) ? 0.f : v0, ((zm >> (2 * e + 1)) & 1u) ? 0.f : v1);
+      }
+      *reinterpret_cast<uint4*>(sm + G_RR + r_row(a) + io(ii, 8 * c8, 16 * (a + 1))) =
+          make_uint4(o[0], o[1], o[2], o[3]);
     }
-    *reinterpret_cast<uint4*>(sm + G_RK + r_col(b) + io(rr, 8 * c8, nrows)) =
-        make_uint4(pack_bf16(xk[0], xk[1]), pack_bf16(xk[2], xk[3]), pack_bf16(xk[4], xk[5]),
-                   pack_bf16(xk[6], xk[7]));
-    *reinterpret_cast<uint4*>(sm + G_RQ + r_col(b) + io(rr, 8 * c8, nrows)) =
-        make_uint4(pack_bf16(xq[0], xq[1]), pack_bf16(xq[2], xq[3]), pack_bf16(xq[4], xq[5]),
-                   pack_bf16(xq[6], xq[7]));
+    for (int i = tid; i < 160 * 16; i += NTG) {
+      const int x = i >> 4, c8 = i & 15;
+      const int b = x >= 144 ? 3 : x >= 112 ? 2 : x >= 64 ? 1 : 0;
+      const int start = b == 0 ? 0 : b == 1 ? 64 : b == 2 ? 112 : 144;
+      const int rr = x - start, r = 16 * b + rr, nrows = 64 - 16 * b;
+      const float* gr = G + r * LDG + 8 * c8;
+      const float* gb = G + (16 * b + 15) * LDG + 8 * c8;
+      const float4 r0v = *reinterpret_cast<const float4*>(gr), r1v = *reinterpret_cast<const float4*>(gr + 4);
+      const float4 b0v = *reinterpret_cast<const float4*>(gb), b1v = *reinterpret_cast<const float4*>(gb + 4);
+      const uint4 kw = *reinterpret_cast<const uint4*>(sm + G_K + io(r, 8 * c8, 64));
+      const uint4 qw = *reinterpret_cast<const uint4*>(sm + G_Q + io(r, 8 * c8, 64));
+      const float dgv[8] = {r0v.x - b0v.x, r0v.y - b0v.y, r0v.z - b0v.z, r0v.w - b0v.w,
+                            r1v.x - b1v.x, r1v.y - b1v.y, r1v.z - b1v.z, r1v.w - b1v.w};
+      const uint32_t kk[4] = {kw.x, kw.y, kw.z, kw.w}, qq[4] = {qw.x, qw.y, qw.z, qw.w};
+      uint32_t zm = 0;
+      if (flags && rr < 16) {
+        const uint2 un = *reinterpret_cast<const uint2*>(&s_uns[b][8 * c8]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) zm |= (((e < 4 ? un.x : un.y) >> (8 * (e & 3))) & 1u) << e;
+      }
+      uint32_t ok_[4], oq[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float f0 = ((zm >> (2 * e)) & 1u) ? 0.f : __expf(fminf(dgv[2 * e], 80.f));
+        const float f1 = ((zm >> (2 * e + 1)) & 1u) ? 0.f : __expf(fminf(dgv[2 * e + 1], 80.f));
+        ok_[e] = pack_bf16(__uint_as_float(kk[e] << 16) * f0, __uint_as_float(kk[e] & 0xffff0000u) * f1);
+        oq[e] = pack_bf16(__uint_as_float(qq[e] << 16) * f0, __uint_as_float(qq[e] & 0xffff0000u) * f1);
+      }
+      const uint32_t o = r_col(b) + io(rr, 8 * c8, nrows);
+      *reinterpret_cast<uint4*>(sm + G_RK + o) = make_uint4(ok_[0], ok_[1], ok_[2], ok_[3]);
+      *reinterpret_cast<uint4*>(sm + G_RQ + o) = make_uint4(oq[0], oq[1], oq[2], oq[3]);
+    }
+  };
+  if (fix) {
+    build_r(true);
+  } else {
+    // No unsafe channel: each row's within-block factor is formed once and scaled by
+    // factors between block references (all <= 1):
+    //   R^(a)[x]  = k_x e^{G_16i - G_x} F1(a, i),        F1(a, i) = e^{G_16a - G_16i},  a > i
+    //   R'^(b)[x] = x_x e^{G_x - G_16i+15} F2(i, b),     F2(i, b) = e^{G_16i+15 - G_16b+15}, b < i
+    // (i = block of row x; pair index hi (hi - 1) / 2 + lo).
+    float* F1 = reinterpret_cast<float*>(sm + G_F1);
+    float* F2 = reinterpret_cast<float*>(sm + G_F2);
+    for (int i = tid; i < 6 * D; i += NTG) {
+      const int pr = i >> 7, c = i & 127;
+      const int hi = pr == 0 ? 1 : pr < 3 ? 2 : 3, lo = pr - hi * (hi - 1) / 2;
+      F1[i] = __expf(G[16 * hi * LDG + c] - G[16 * lo * LDG + c]);
+      F2[i] = __expf(G[(16 * hi + 15) * LDG + c] - G[(16 * lo + 15) * LDG + c]);
+    }
+    __syncthreads();
+    for (int i = tid; i < C * 16; i += NTG) {
+      const int x = i >> 4, c8 = i & 15, blk = x >> 4;
+      const float* gx = G + x * LDG + 8 * c8;
+      const float* gs = G + 16 * blk * LDG + 8 * c8;
+      const float* ge = G + (16 * blk + 15) * LDG + 8 * c8;
+      const float4 x0 = *reinterpret_cast<const float4*>(gx), x1 = *reinterpret_cast<const float4*>(gx + 4);
+      const float4 s0 = *reinterpret_cast<const float4*>(gs), s1 = *reinterpret_cast<const float4*>(gs + 4);
+      const float4 e0 = *reinterpret_cast<const float4*>(ge), e1 = *reinterpret_cast<const float4*>(ge + 4);
+      const uint4 kw = *reinterpret_cast<const uint4*>(sm + G_K + io(x, 8 * c8, 64));
+      const uint4 qw = *reinterpret_cast<const uint4*>(sm + G_Q + io(x, 8 * c8, 64));
+      const float gxv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+      const float gsv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+      const float gev[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
+      const uint32_t kk[4] = {kw.x, kw.y, kw.z, kw.w}, qq[4] = {qw.x, qw.y, qw.z, qw.w};
+      float rk[8], ck[8], cqv[8];                // k e^{G_16i - G_x}; k, q e^{G_x - G_16i+15}
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float kv = __uint_as_float((e & 1) ? (kk[e >> 1] & 0xffff0000u) : (kk[e >> 1] << 16));
+        const float qv = __uint_as_float((e & 1) ? (qq[e >> 1] & 0xffff0000u) : (qq[e >> 1] << 16));
+        const float up = __expf(fminf(gsv[e] - gxv[e], 80.f)), dn = __expf(fminf(gxv[e] - gev[e], 80.f));
+        rk[e] = kv * up;
+        ck[e] = kv * dn;
+        cqv[e] = qv * dn;
+      }
+      auto put8 = [&](uint32_t off, const float (&v)[8], const float* f) {
+        float y[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) y[e] = f ? v[e] * f[8 * c8 + e] : v[e];
+        *reinterpret_cast<uint4*>(sm + off) =
+            make_uint4(pack_bf16(y[0], y[1]), pack_bf16(y[2], y[3]), pack_bf16(y[4], y[5]),
+                       pack_bf16(y[6], y[7]));
+      };
+#pragma unroll
+      for (int a = 0; a < 4; ++a)              // row x of R^(a), a >= blk
+        if (a >= blk)
+          put8(G_RR + r_row(a) + io(x, 8 * c8, 16 * (a + 1)), rk,
+               a == blk ? nullptr : F1 + (a * (a - 1) / 2 + blk) * D);
+#pragma unroll
+      for (int b = 0; b < 4; ++b)              // row x - 16 b of R'k^(b), R'q^(b), b <= blk
+        if (b <= blk) {
+          const float* f = b == blk ? nullptr : F2 + (blk * (blk - 1) / 2 + b) * D;
+          const uint32_t o = r_col(b) + io(x - 16 * b, 8 * c8, 64 - 16 * b);
+          put8(G_RK + o, ck, f);
+          put8(G_RQ + o, cqv, f);
+        }
+    }
   }
   __syncthreads();
   // row side: [YA | YQ] = [dA | dAqk] R^(tb) for rows r0.. (times e^{G_r - G_16tb})
 #pragma unroll
-  for (int np = 0; np < 4; ++np) {
+  for (int np = 0; np < 2; ++np) {
     float ya[2][4] = {}, yq[2][4] = {};
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) {
@@ -972,20 +1100,26 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
 #pragma unroll
     for (int sub = 0; sub < 2; ++sub) {
       const int nt = 2 * np + sub;
+      const float2 gref = gam2(r0, nt);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int r = erow(e), c = ecol(nt, e);
-        const float f = __expf(fminf(G[r * LDG + c] - G[r0 * LDG + c], 80.f));
-        const float yA = ya[sub][e] * f, yQ = yq[sub][e] * f;
-        dK[nt][e] += yA;
-        dQ[nt][e] += yQ;
-        dG[nt][e] += yA * qk(G_K, r, c) + yQ * qk(G_Q, r, c);
+      for (int hf = 0; hf < 2; ++hf) {
+        const float2 gp = gam2(r0 + g8 + 8 * hf, nt);
+        const float2 kv = img2(G_K, hf, nt), qv = img2(G_Q, hf, nt);
+        const float f0 = __expf(fminf(gp.x - gref.x, 80.f)), f1 = __expf(fminf(gp.y - gref.y, 80.f));
+        const float yA0 = ya[sub][2 * hf] * f0, yA1 = ya[sub][2 * hf + 1] * f1;
+        const float yQ0 = yq[sub][2 * hf] * f0, yQ1 = yq[sub][2 * hf + 1] * f1;
+        dK[nt][2 * hf] += yA0;
+        dK[nt][2 * hf + 1] += yA1;
+        dQ[nt][2 * hf] += yQ0;
+        dQ[nt][2 * hf + 1] += yQ1;
+        dG[nt][2 * hf] += yA0 * kv.x + yQ0 * qv.x;
+        dG[nt][2 * hf + 1] += yA1 * kv.y + yQ1 * qv.y;
       }
     }
   }
   // column side: Z = dA^T R'k^(tb) + dAqk^T R'q^(tb) for rows i = r0.. (times e^{G_16tb+15 - G_i})
 #pragma unroll
-  for (int np = 0; np < 4; ++np) {
+  for (int np = 0; np < 2; ++np) {
     float z[2][4] = {};
 #pragma unroll
     for (int rho = 0; rho < 4; ++rho) {
@@ -1003,26 +1137,30 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
 #pragma unroll
     for (int sub = 0; sub < 2; ++sub) {
       const int nt = 2 * np + sub;
+      const float2 gref = gam2(r0 + 15, nt);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int r = erow(e), c = ecol(nt, e);
-        const float f = __expf(fminf(G[(r0 + 15) * LDG + c] - G[r * LDG + c], 80.f));
-        const float zz = z[sub][e] * f;
-        dK[nt][e] += zz;
-        dG[nt][e] -= zz * qk(G_K, r, c);
+      for (int hf = 0; hf < 2; ++hf) {
+        const float2 gp = gam2(r0 + g8 + 8 * hf, nt), kv = img2(G_K, hf, nt);
+        const float z0 = z[sub][2 * hf] * __expf(fminf(gref.x - gp.x, 80.f));
+        const float z1 = z[sub][2 * hf + 1] * __expf(fminf(gref.y - gp.y, 80.f));
+        dK[nt][2 * hf] += z0;
+        dK[nt][2 * hf + 1] += z1;
+        dG[nt][2 * hf] -= z0 * kv.x;
+        dG[nt][2 * hf + 1] -= z1 * kv.y;
       }
     }
   }
   if (fix) {
     // exact within-block pairs of unsafe (block, channel) pairs, by running products
     // of alpha_j = e^{g_j} (exponents from the block's own g, never from Gamma)
+    auto qk = [&](uint32_t img, int r, int c) { return bf_at(sm + img + io(r, c, 64)); };
     __syncthreads();                    // R images no longer read
     float* cya = reinterpret_cast<float*>(sm + G_CYA);
     float* cyq = reinterpret_cast<float*>(sm + G_CYQ);
     float* cz = reinterpret_cast<float*>(sm + G_CZ);
-    for (int i = tid; i < 3 * 64 * 128; i += NTH) cya[i] = 0.f;   // the three are contiguous
+    for (int i = tid; i < 3 * 64 * 128; i += NTG) cya[i] = 0.f;   // the three are contiguous
     __syncthreads();
-    for (int item = tid; item < 4 * D; item += NTH) {
+    for (int item = tid; item < 4 * D; item += NTG) {
       const int a = item >> 7, c = item & 127;
       if (!s_uns[a][c]) continue;
       const int ra = 16 * a;
@@ -1058,10 +1196,10 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     }
     __syncthreads();
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
+    for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int r = erow(e), c = ecol(nt, e);
+        const int r = r0 + g8 + ((e >> 1) << 3), c = c0 + 8 * nt + 2 * qd + (e & 1);
         if (!s_uns[tb][c]) continue;
         const float yA = cya[r * 128 + c], yQ = cyq[r * 128 + c], zz = cz[r * 128 + c];
         const float kv = qk(G_K, r, c), qv = qk(G_Q, r, c);
@@ -1071,47 +1209,49 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       }
   }
 
-  // ---- phase 5: outputs
-#pragma unroll
-  for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-      const int r = r0 + g8 + 8 * hf, c = c0 + 8 * nt + 2 * qd;
-      if (r < L) {
-        const long long o = ((rb + r) * H + h) * D + c;
-        *reinterpret_cast<float2*>(dq + o) = make_float2(dQ[nt][2 * hf], dQ[nt][2 * hf + 1]);
-        *reinterpret_cast<float2*>(dk + o) = make_float2(dK[nt][2 * hf], dK[nt][2 * hf + 1]);
-      }
-    }
+  // ---- phase 5: outputs (dq, dk and dGamma through shared memory, [64][LDG] fp32 each)
   __syncthreads();                      // R images / corrections no longer read
-  float* dGs = reinterpret_cast<float*>(sm + G_S0);    // dGamma [64][LDG]
+  float* dGs = reinterpret_cast<float*>(sm + G_S0);
+  float* dQs = dGs + 64 * LDG;
+  float* dKs = dQs + 64 * LDG;
 #pragma unroll
-  for (int nt = 0; nt < 8; ++nt)
+  for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
-      const int r = r0 + g8 + 8 * hf, c = c0 + 8 * nt + 2 * qd;
-      *reinterpret_cast<float2*>(dGs + r * LDG + c) = make_float2(dG[nt][2 * hf], dG[nt][2 * hf + 1]);
+      const int o = (r0 + g8 + 8 * hf) * LDG + c0 + 8 * nt + 2 * qd;
+      *reinterpret_cast<float2*>(dGs + o) = make_float2(dG[nt][2 * hf], dG[nt][2 * hf + 1]);
+      *reinterpret_cast<float2*>(dQs + o) = make_float2(dQ[nt][2 * hf], dQ[nt][2 * hf + 1]);
+      *reinterpret_cast<float2*>(dKs + o) = make_float2(dK[nt][2 * hf], dK[nt][2 * hf + 1]);
     }
   __syncthreads();
+  for (int i = tid; i < C * 32; i += NTG) {
+    const int r = i >> 5, c4 = i & 31;
+    if (r < L) {
+      const long long o = ((rb + r) * H + h) * D + 4 * c4;
+      *reinterpret_cast<float4*>(dq + o) = *reinterpret_cast<const float4*>(dQs + r * LDG + 4 * c4);
+      *reinterpret_cast<float4*>(dk + o) = *reinterpret_cast<const float4*>(dKs + r * LDG + 4 * c4);
+    }
+  }
   if (tid < D) dGs[63 * LDG + tid] += s_dgl[tid];
   __syncthreads();
-  // dg = reverse cumulative sum of dGamma: two threads per channel, 32 rows each
+  // dg = reverse cumulative sum of dGamma: four threads per channel, 16 rows each
   {
     const int c = tid & 127, part = tid >> 7;
-    float x[32];
+    float x[16];
 #pragma unroll
-    for (int e = 0; e < 32; ++e) x[e] = dGs[(32 * part + e) * LDG + c];
+    for (int e = 0; e < 16; ++e) x[e] = dGs[(16 * part + e) * LDG + c];
 #pragma unroll
-    for (int e = 30; e >= 0; --e) x[e] += x[e + 1];
-    if (part == 1) s_half[c] = x[0];
+    for (int e = 14; e >= 0; --e) x[e] += x[e + 1];
+    s_part[part][c] = x[0];
     __syncthreads();
-    const float add = part ? 0.f : s_half[c];
+    float add = 0.f;
+    for (int p2 = part + 1; p2 < 4; ++p2) add += s_part[p2][c];
 #pragma unroll
-    for (int e = 0; e < 32; ++e) dGs[(32 * part + e) * LDG + c] = x[e] + add;
+    for (int e = 0; e < 16; ++e) dGs[(16 * part + e) * LDG + c] = x[e] + add;
   }
   __syncthreads();
   if constexpr (!GRPD) {
-    for (int i = tid; i < C * 32; i += NTH) {
+    for (int i = tid; i < C * 32; i += NTG) {
       const int r = i >> 5, c4 = i & 31;
       if (r < L)
         *reinterpret_cast<float4*>(dg + ((rb + r) * H + h) * D + 4 * c4) =
@@ -1119,7 +1259,7 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     }
   } else {
     const int ng = D >> gsh, gs = 1 << gsh;
-    for (int i = tid; i < C * ng; i += NTH) {
+    for (int i = tid; i < C * ng; i += NTG) {
       const int r = i / ng, m = i % ng;
       if (r < L) {
         float acc = 0.f;
@@ -1131,7 +1271,7 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   if (tid < L) dbeta[(rb + tid) * H + h] = s_dbeta[tid];
 }
 
-constexpr int kChainNB = 16;
+constexpr int kChainNB = 32;
 
 bool set_attrs() {
   return once_per_device(kOnceBwdTc, []() {
@@ -1202,24 +1342,40 @@ cudaError_t launch_chunk_bwd_tc(const void* q, const void* k, const void* v, con
   if (e == cudaSuccess) {
     using CF = Chain<kChainNB>;
     KDA_TIMED(KDA_KERNEL_BWD_CHAIN, stream,
-              (kda_bwd_chain_kernel<kChainNB><<<dim3(2 * CF::NJB, H, B), NTH, CF::SMEM, stream>>>(
-                  rec, h0, cu_seqlens, static_cast<const bf16*>(dout), dhT, dh0, base + sc.simg,
-                  base + sc.dlimg, base + sc.dsimg, base + sc.ddimg, T, H, sc.nslots)));
+              e = launch_after(kda_bwd_chain_kernel<kChainNB>, dim3(2 * CF::NJB, H, B), dim3(NTC),
+                               CF::SMEM, stream, rec, h0, cu_seqlens,
+                               static_cast<const bf16*>(dout), dhT, dh0, base + sc.simg,
+                               base + sc.dlimg, base + sc.dsimg, base + sc.ddimg, T, H,
+                               sc.nslots));
     note_launches(1);
-    e = cudaGetLastError();
   }
   if (e == cudaSuccess && sc.nslots > 0) {
     auto grad = gsh != 0 ? kda_bwd_grad_kernel<true> : kda_bwd_grad_kernel<false>;
     KDA_TIMED(KDA_KERNEL_BWD_GRAD, stream,
-              grad<<<dim3((unsigned)sc.nslots, H), NTH, GRAD_SMEM, stream>>>(
-                  static_cast<const bf16*>(q), static_cast<const bf16*>(k),
-                  static_cast<const bf16*>(v), g, beta, static_cast<const bf16*>(dout),
-                  cu_seqlens, rec, base + sc.simg, base + sc.dlimg, base + sc.dsimg,
-                  base + sc.ddimg, dq, dk, dv, dg, dbeta, B, T, H, gsh, sc.nslots));
+              e = launch_after(grad, dim3((unsigned)sc.nslots, H), dim3(NTG), GRAD_SMEM, stream,
+                               static_cast<const bf16*>(q), static_cast<const bf16*>(k),
+                               static_cast<const bf16*>(v), g, beta,
+                               static_cast<const bf16*>(dout), cu_seqlens,
+                               static_cast<const uint8_t*>(rec), static_cast<const uint8_t*>(base + sc.simg),
+                               static_cast<const uint8_t*>(base + sc.dlimg),
+                               static_cast<const uint8_t*>(base + sc.dsimg),
+                               static_cast<const uint8_t*>(base + sc.ddimg), dq, dk, dv, dg,
+                               dbeta, B, T, H, gsh, sc.nslots));
     note_launches(1);
-    e = cudaGetLastError();
   }
   if (pooled) cudaFreeAsync(scratch, stream);
+  return e;
+}
+
+// Reads (and with reset clears) g_bwd_tc_timeout; host side of kda_device_status.
+cudaError_t take_bwd_tc_timeout(int* flag, bool reset) {
+  int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_bwd_tc_timeout, sizeof(int));
+  if (e == cudaSuccess && reset && v != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_bwd_tc_timeout, &zero, sizeof(int));
+  }
+  *flag = v;
   return e;
 }
 

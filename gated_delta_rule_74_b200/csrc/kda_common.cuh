@@ -142,6 +142,7 @@ cudaError_t launch_chunk_bwd_tc(const void* q, const void* k, const void* v, con
 cudaError_t take_split_timeout(int* flag, bool reset);
 cudaError_t take_tc_timeout(int* flag, bool reset);
 cudaError_t take_bwd_timeout(int* flag, bool reset);
+cudaError_t take_bwd_tc_timeout(int* flag, bool reset);
 cudaError_t take_combine_timeout(int* flag, bool reset);
 cudaError_t take_selftest_timeout(int* flag, bool reset);
 cudaError_t take_decode_chunk_timeout(int* flag, bool reset);
