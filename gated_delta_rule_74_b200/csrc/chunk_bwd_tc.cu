@@ -610,12 +610,16 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   cp_async_wait_all();
   __syncthreads();
   // unsafe (block, channel) pairs; dGamma_last's state term e^Gamma_last sum_j S dS
-  bool any_uns = false;
+  bool any_uns = false, far = false;
   {
     const int c = tid & 127, a = tid >> 7;
     const bool u = G[16 * a * LDG + c] - G[(16 * a + 15) * LDG + c] > kUnsafeDecay;
     s_uns[a][c] = u ? 1 : 0;
     any_uns = u;
+    // the mid-chunk reference (row 32) serves all pairs when neither half decays by more
+    // than kUnsafeDecay on this channel
+    if (a == 0)
+      far = G[c] - G[32 * LDG + c] > kUnsafeDecay || G[32 * LDG + c] - G[63 * LDG + c] > kUnsafeDecay;
     const int c8 = tid & 15, jg = tid >> 4;           // 32 groups of 4 rows j
     float acc[8];
 #pragma unroll
@@ -642,6 +646,7 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     }
   }
   const bool fix = __syncthreads_or(any_uns) != 0;
+  const bool mid = __syncthreads_or(far) == 0;
 
   const int tb = w & 3, cq = w >> 2, r0 = 16 * tb, c0 = 32 * cq;
   float dQ[4][4], dK[4][4], dG[4][4];
@@ -1016,7 +1021,37 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       *reinterpret_cast<uint4*>(sm + G_RQ + o) = make_uint4(oq[0], oq[1], oq[2], oq[3]);
     }
   };
-  if (fix) {
+  if (mid) {
+    // one reference point for the whole chunk, P = Gamma at row 32 (every factor within
+    // e^{+-kUnsafeDecay}): R = k e^{P - G}, R'k = k e^{G - P}, R'q = q e^{G - P}, 64 rows each
+    for (int i = tid; i < C * 16; i += NTG) {
+      const int x = i >> 4, c8 = i & 15;
+      const float* gx = G + x * LDG + 8 * c8;
+      const float* gp = G + 32 * LDG + 8 * c8;
+      const float4 x0 = *reinterpret_cast<const float4*>(gx), x1 = *reinterpret_cast<const float4*>(gx + 4);
+      const float4 p0 = *reinterpret_cast<const float4*>(gp), p1 = *reinterpret_cast<const float4*>(gp + 4);
+      const uint4 kw = *reinterpret_cast<const uint4*>(sm + G_K + io(x, 8 * c8, 64));
+      const uint4 qw = *reinterpret_cast<const uint4*>(sm + G_Q + io(x, 8 * c8, 64));
+      const float dv8[8] = {p0.x - x0.x, p0.y - x0.y, p0.z - x0.z, p0.w - x0.w,
+                            p1.x - x1.x, p1.y - x1.y, p1.z - x1.z, p1.w - x1.w};
+      const uint32_t kk[4] = {kw.x, kw.y, kw.z, kw.w}, qq[4] = {qw.x, qw.y, qw.z, qw.w};
+      uint32_t orr[4], ork[4], orq[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float up0 = __expf(dv8[2 * e]), up1 = __expf(dv8[2 * e + 1]);
+        const float dn0 = __expf(-dv8[2 * e]), dn1 = __expf(-dv8[2 * e + 1]);
+        const float k0 = __uint_as_float(kk[e] << 16), k1 = __uint_as_float(kk[e] & 0xffff0000u);
+        const float q0 = __uint_as_float(qq[e] << 16), q1 = __uint_as_float(qq[e] & 0xffff0000u);
+        orr[e] = pack_bf16(k0 * up0, k1 * up1);
+        ork[e] = pack_bf16(k0 * dn0, k1 * dn1);
+        orq[e] = pack_bf16(q0 * dn0, q1 * dn1);
+      }
+      const uint32_t o = io(x, 8 * c8, 64);
+      *reinterpret_cast<uint4*>(sm + G_RR + o) = make_uint4(orr[0], orr[1], orr[2], orr[3]);
+      *reinterpret_cast<uint4*>(sm + G_RK + o) = make_uint4(ork[0], ork[1], ork[2], ork[3]);
+      *reinterpret_cast<uint4*>(sm + G_RQ + o) = make_uint4(orq[0], orq[1], orq[2], orq[3]);
+    }
+  } else if (fix) {
     build_r(true);
   } else {
     // No unsafe channel: each row's within-block factor is formed once and scaled by
@@ -1091,7 +1126,8 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       uint32_t aa[4], aq[4], b[4];
       a_mk(sb + G_DA, 64, r0, 16 * ks, lane, aa);
       a_mk(sb + G_AQK, 64, r0, 16 * ks, lane, aq);
-      b_kn(sb + G_RR + r_row(tb), 16 * (tb + 1), c0 + 16 * np, 16 * ks, lane, b);
+      b_kn(sb + G_RR + (mid ? 0u : r_row(tb)), mid ? 64 : 16 * (tb + 1), c0 + 16 * np, 16 * ks,
+           lane, b);
       mma(ya[0], aa, b[0], b[1]);
       mma(ya[1], aa, b[2], b[3]);
       mma(yq[0], aq, b[0], b[1]);
@@ -1100,7 +1136,7 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
 #pragma unroll
     for (int sub = 0; sub < 2; ++sub) {
       const int nt = 2 * np + sub;
-      const float2 gref = gam2(r0, nt);
+      const float2 gref = gam2(mid ? 32 : r0, nt);
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         const float2 gp = gam2(r0 + g8 + 8 * hf, nt);
@@ -1127,8 +1163,10 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       uint32_t aa[4], aq[4], bk[4], bq[4];
       a_km(sb + G_DA, 64, r0, 16 * rho, lane, aa);
       a_km(sb + G_AQK, 64, r0, 16 * rho, lane, aq);
-      b_kn(sb + G_RK + r_col(tb), 64 - 16 * tb, c0 + 16 * np, 16 * (rho - tb), lane, bk);
-      b_kn(sb + G_RQ + r_col(tb), 64 - 16 * tb, c0 + 16 * np, 16 * (rho - tb), lane, bq);
+      const uint32_t co = mid ? 0u : r_col(tb);
+      const int crows = mid ? 64 : 64 - 16 * tb, ck0 = mid ? 16 * rho : 16 * (rho - tb);
+      b_kn(sb + G_RK + co, crows, c0 + 16 * np, ck0, lane, bk);
+      b_kn(sb + G_RQ + co, crows, c0 + 16 * np, ck0, lane, bq);
       mma(z[0], aa, bk[0], bk[1]);
       mma(z[1], aa, bk[2], bk[3]);
       mma(z[0], aq, bq[0], bq[1]);
@@ -1137,7 +1175,7 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
 #pragma unroll
     for (int sub = 0; sub < 2; ++sub) {
       const int nt = 2 * np + sub;
-      const float2 gref = gam2(r0 + 15, nt);
+      const float2 gref = gam2(mid ? 32 : r0 + 15, nt);
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         const float2 gp = gam2(r0 + g8 + 8 * hf, nt), kv = img2(G_K, hf, nt);
