@@ -181,8 +181,8 @@ __device__ __forceinline__ float2 bf2_at(const uint8_t* p) {
 }
 
 // ============================================================================
-// Chains.  CTA (x, h, s): x < NJB walks sequence s of head h forward for the
-// value columns [NB x, NB x + NB); x >= NJB walks it backward for block x - NJB.
+// Chains: per (column block, head, sequence) one CTA of 8 warps walks the chunks forward
+// (S at every chunk start, Delta) or backward (dS after every chunk, dDelta, dh0).
 // Warp w keeps rows 16w .. 16w + 15 of the state (or of its gradient) for the
 // block's columns as m16n8 accumulators: lane (g, qd) holds rows 16w + g (+8),
 // columns 8 nt + 2 qd (+1).
@@ -190,7 +190,6 @@ __device__ __forceinline__ float2 bf2_at(const uint8_t* p) {
 template <int NB>
 struct Chain {
   static constexpr int NJ = NB / 8;        // n8 tiles of the column block
-  static constexpr int NJB = D / NB;       // column blocks per head
   static constexpr int STG = 3;            // record stages in flight
   // forward stage: W^T (16 KB), Kend^T (16 KB), U^T rows of the block, exp(Gamma_last)
   static constexpr uint32_t F_W = 0, F_K = 16384, F_U = 32768, F_DEC = F_U + NB * 128,
@@ -208,251 +207,275 @@ struct Chain {
   static_assert(F_STAGE % 128 == 0 && R_STAGE % 128 == 0, "tiles stay 128-byte aligned");
 };
 
-template <int NB>
-__global__ void __launch_bounds__(NTC, 1)
-kda_bwd_chain_kernel(const uint8_t* __restrict__ rec, const float* __restrict__ h0,
-                     const int32_t* __restrict__ cu_seqlens, const bf16* __restrict__ dout,
-                     const float* __restrict__ dhT, float* __restrict__ dh0,
-                     uint8_t* __restrict__ simg, uint8_t* __restrict__ dlimg,
-                     uint8_t* __restrict__ dsimg, uint8_t* __restrict__ ddimg, int T, int H,
-                     long long nslots) {
-  using CF = Chain<NB>;
-  constexpr int STG = CF::STG;
-  static_assert(NB == 32, "8 warps: 8 row blocks of the state, all 4 n8 tiles");
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = align1024(smem_raw);
-  __shared__ uint64_t full[STG];           // record stage landed (bulk copies)
-  const uint32_t sb = smem_u32(sm);
-  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31, g = lane >> 2, qd = lane & 3;
-  const bool fwd = (int)blockIdx.x < CF::NJB;
-  const int jb = fwd ? (int)blockIdx.x : (int)blockIdx.x - CF::NJB;
-  const int j0 = jb * NB, h = blockIdx.y, s = blockIdx.z;
+// Shared setup of one chain CTA: the sequence's chunk range and its slots.
+struct ChainCtx {
+  const uint8_t* rec;
+  const bf16* dout;
+  uint8_t* sm;
+  uint32_t sb;
+  uint64_t* full;
+  size_t base, st_off;
   long long row0, t_beg, t_end;
-  seq_range(cu_seqlens, s, T, row0, t_beg, t_end);
-  const int nch = (int)chunk_count(t_end - t_beg);
-  const size_t base = (size_t)h * (size_t)nslots + (size_t)seq_chunk_base(cu_seqlens, s, T);
-  const size_t st_off = ((size_t)s * H + h) * D * D;
-  if (tid == 0) {
-#pragma unroll
-    for (int i = 0; i < STG; ++i) mbar_init(&full[i], 1);
-    fence_mbar_init();
-  }
-  grid_dep_launch();                       // the gradient kernel may start preloading its inputs
+  int nch, j0, h, H, tid, w, lane, g, qd;
+};
 
-  // the state (or its gradient): warp w holds rows cr = 16 w .. cr + 15 and the block's
-  // four n8 tiles of columns
-  const int cr = 16 * w;
-  float X[4][4];
-  {
-    const float* init = fwd ? h0 : dhT;
+// The state (or its gradient) of one CTA: warp w holds rows cr = 16 w .. cr + 15 and the
+// block's NB / 8 n8 tiles of columns.  Returns the first chain step's state loaded from init.
+template <int NB>
+__device__ __forceinline__ void chain_load(const ChainCtx& x, const float* init,
+                                           float (&X)[NB / 8][4]) {
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
+  for (int nt = 0; nt < NB / 8; ++nt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int c = cr + g + ((e >> 1) << 3), j = j0 + 8 * nt + 2 * qd + (e & 1);
-        X[nt][e] = init ? init[st_off + (size_t)c * D + j] : 0.f;
-      }
-  }
-  __syncthreads();                         // the barriers are initialised
-  grid_dep_wait();                         // the records are complete
-  const int tb = w & 3, jh = w >> 2;       // Delta / dDelta tiles: token block, n8 tiles 2 jh, 2 jh + 1
+    for (int e = 0; e < 4; ++e) {
+      const int c = 16 * x.w + x.g + ((e >> 1) << 3), j = x.j0 + 8 * nt + 2 * x.qd + (e & 1);
+      X[nt][e] = init ? init[x.st_off + (size_t)c * D + j] : 0.f;
+    }
+}
 
-  // The S (or dS) tile as bf16 [j][c]; each warp then copies its own 16 channels of the
-  // tile's NB rows j out to rows j0.. of the chunk's image (no barrier needed).
-  auto put_state = [&](uint32_t tile_off, uint8_t* img) {
-    st_nm(sb + tile_off, NB, cr, 0, lane, X[0], X[1], 1.f);
-    st_nm(sb + tile_off, NB, cr, 16, lane, X[2], X[3], 1.f);
-    __syncwarp();
+// The state tile as bf16 [j][c]; each warp then copies its own 16 channels of the tile's
+// NB rows j out to rows j0.. of the chunk's image (no barrier needed).
+template <int NB>
+__device__ __forceinline__ void chain_put(const ChainCtx& x, const float (&X)[NB / 8][4],
+                                          uint32_t tile_off, uint8_t* img) {
+  const int cr = 16 * x.w;
 #pragma unroll
-    for (int i = lane; i < 2 * NB; i += 32) {
-      const int rr = i >> 1, ck = (cr >> 3) + (i & 1);          // row j, 16-byte chunk
-      const uint32_t sw = (uint32_t)(((ck & 7) ^ (rr & 7)) << 4);
-      *reinterpret_cast<uint4*>(img + (ck >> 3) * 16384 + (j0 + rr) * 128 + sw) =
-          *reinterpret_cast<const uint4*>(sm + tile_off + (ck >> 3) * NB * 128 + rr * 128 + sw);
-    }
-  };
-  // a bounded wait for a stage failed: raise the flag and let the copies in flight land
-  auto give_up = [&](int n_first, int n_last, bool ascending) {
-    if (tid == 0) {
-      atomicExch(&g_bwd_tc_timeout, 1);
-      for (int m = n_first; ascending ? m <= n_last : m >= n_last; m += ascending ? 1 : -1) {
-        const uint32_t use = ascending ? (uint32_t)(m / STG) : (uint32_t)((nch - 1 - m) / STG);
-        mbar_wait(&full[m % STG], use & 1u, kWaitLimit);
-      }
-    }
-    cp_async_wait_all();
-  };
-  // state update: one K step (16 tokens) of A B into X, or into Y (a second accumulator)
-  auto update = [&](uint32_t a_img, uint32_t b_img, float (&Y)[4][4], int ks, bool into_y) {
-    uint32_t a[4], b[4], b2[4];
-    a_mk(a_img, 128, cr, 16 * ks, lane, a);                       // [c][t] image
-    b_kn(b_img, 64, 0, 16 * ks, lane, b);                         // [t][j] tile
-    b_kn(b_img, 64, 16, 16 * ks, lane, b2);
-    float (&u0)[4] = into_y ? Y[0] : X[0];
-    float (&u1)[4] = into_y ? Y[1] : X[1];
-    float (&u2)[4] = into_y ? Y[2] : X[2];
-    float (&u3)[4] = into_y ? Y[3] : X[3];
+  for (int p = 0; p < NB / 16; ++p)
+    st_nm(x.sb + tile_off, NB, cr, 16 * p, x.lane, X[2 * p], X[2 * p + 1], 1.f);
+  __syncwarp();
+#pragma unroll
+  for (int i = x.lane; i < 2 * NB; i += 32) {
+    const int rr = i >> 1, ck = (cr >> 3) + (i & 1);          // row j, 16-byte chunk
+    const uint32_t sw = (uint32_t)(((ck & 7) ^ (rr & 7)) << 4);
+    *reinterpret_cast<uint4*>(img + (ck >> 3) * 16384 + (x.j0 + rr) * 128 + sw) =
+        *reinterpret_cast<const uint4*>(x.sm + tile_off + (ck >> 3) * NB * 128 + rr * 128 + sw);
+  }
+}
+
+// One K step (16 tokens) of A B added into the state X (set 0) or a partial sum Y:
+// A a [c][t] image (the warp's 16 rows), B a [t][j] tile of the block's NB columns.
+template <int NB>
+__device__ __forceinline__ void chain_update(const ChainCtx& x, uint32_t a_img, uint32_t b_img,
+                                             float (&X)[NB / 8][4], float (&Y)[NB / 8][4],
+                                             int ks, bool into_y) {
+  uint32_t a[4];
+  a_mk(a_img, 128, 16 * x.w, 16 * ks, x.lane, a);
+#pragma unroll
+  for (int p = 0; p < NB / 16; ++p) {
+    uint32_t b[4];
+    b_kn(b_img, 64, 16 * p, 16 * ks, x.lane, b);
+    float (&u0)[4] = into_y ? Y[2 * p] : X[2 * p];
+    float (&u1)[4] = into_y ? Y[2 * p + 1] : X[2 * p + 1];
     mma(u0, a, b[0], b[1]);
     mma(u1, a, b[2], b[3]);
-    mma(u2, a, b2[0], b2[1]);
-    mma(u3, a, b2[2], b2[3]);
-  };
+  }
+}
 
-  if (fwd) {
-    auto issue = [&](int n) {
-      if (tid == NTC - 32 && n < nch) {
-        const uint8_t* rc = rec + (base + n) * rec::BYTES_BWD;
-        uint8_t* st = sm + (n % STG) * CF::F_STAGE;
-        uint64_t* bar = &full[n % STG];
-        fence_async_smem();
-        mbar_arrive_expect_tx(bar, CF::F_BYTES);
-        bulk_g2s(st + CF::F_W, rc + rec::QW + 16384, 16384, bar);
-        bulk_g2s(st + CF::F_K, rc + rec::KA, 16384, bar);
-        bulk_g2s(st + CF::F_U, rc + rec::U + j0 * 128, NB * 128, bar);
-        bulk_g2s(st + CF::F_DEC, rc + rec::DECAY, 512, bar);
-      }
-    };
-    const uint32_t uS = sb + CF::F_S, uDL = sb + CF::F_DL;
+// A bounded wait for a stage failed: raise the flag and let the copies in flight land.
+template <int STG>
+__device__ void chain_give_up(const ChainCtx& x, int n_first, int n_last, bool ascending) {
+  if (x.tid == 0) {
+    atomicExch(&g_bwd_tc_timeout, 1);
+    for (int m = n_first; ascending ? m <= n_last : m >= n_last; m += ascending ? 1 : -1) {
+      const uint32_t use = ascending ? (uint32_t)(m / STG) : (uint32_t)((x.nch - 1 - m) / STG);
+      mbar_wait(&x.full[m % STG], use & 1u, kWaitLimit);
+    }
+  }
+  cp_async_wait_all();
+}
+
+// Forward chain: S at every chunk start and Delta of every chunk.
+template <int NB>
+__device__ __forceinline__ void chain_forward(const ChainCtx& x, const float* h0, uint8_t* simg,
+                                              uint8_t* dlimg) {
+  using CF = Chain<NB>;
+  constexpr int NJ = NB / 8, NH = NB / 16, STG = CF::STG;
+  const int tb = x.w & 3, jh = x.w >> 2, g = x.g, qd = x.qd, lane = x.lane;
+  float X[NJ][4];
+  chain_load<NB>(x, h0, X);
+  auto issue = [&](int n) {
+    if (x.tid == NTC - 32 && n < x.nch) {
+      const uint8_t* rc = x.rec + (x.base + n) * rec::BYTES_BWD;
+      uint8_t* st = x.sm + (n % STG) * CF::F_STAGE;
+      uint64_t* bar = &x.full[n % STG];
+      fence_async_smem();
+      mbar_arrive_expect_tx(bar, CF::F_BYTES);
+      bulk_g2s(st + CF::F_W, rc + rec::QW + 16384, 16384, bar);
+      bulk_g2s(st + CF::F_K, rc + rec::KA, 16384, bar);
+      bulk_g2s(st + CF::F_U, rc + rec::U + x.j0 * 128, NB * 128, bar);
+      bulk_g2s(st + CF::F_DEC, rc + rec::DECAY, 512, bar);
+    }
+  };
+  const uint32_t uS = x.sb + CF::F_S, uDL = x.sb + CF::F_DL;
 #pragma unroll 1
-    for (int n = 0; n < STG - 1; ++n) issue(n);
+  for (int n = 0; n < STG - 1; ++n) issue(n);
 #pragma unroll 1
-    for (int n = 0; n < nch; ++n) {
-      const uint32_t so = (uint32_t)(n % STG) * CF::F_STAGE;
-      put_state(CF::F_S, simg + (base + n) * kImgS);   // S at the start of chunk n
-      const bool ok = mbar_wait(&full[n % STG], (uint32_t)(n / STG) & 1u, kWaitLimit);
-      if (__syncthreads_or(!ok)) {
-        give_up(n, min(n + STG - 2, nch - 1), true);
-        return;
-      }
-      // Delta = U - W S: token block tb, n8 tiles 2 jh, 2 jh + 1 (two accumulators each)
-      float acc[2][2][4] = {};
+  for (int n = 0; n < x.nch; ++n) {
+    const uint32_t so = (uint32_t)(n % STG) * CF::F_STAGE;
+    chain_put<NB>(x, X, CF::F_S, simg + (x.base + n) * kImgS);   // S at the start of chunk n
+    const bool ok = mbar_wait(&x.full[n % STG], (uint32_t)(n / STG) & 1u, kWaitLimit);
+    if (__syncthreads_or(!ok)) {
+      chain_give_up<STG>(x, n, min(n + STG - 2, x.nch - 1), true);
+      return;
+    }
+    // Delta = U - W S: token block tb, n8 tiles jh * NH .. (two accumulators each)
+    float acc[NH][2][4] = {};
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        uint32_t a[4], b[4];
-        a_km(sb + so + CF::F_W, 128, 16 * tb, 16 * ks, lane, a);      // W [t][c] from W^T
-        b_nk(uS, NB, 16 * jh, 16 * ks, lane, b);                      // S [c][j] from [j][c]
+    for (int ks = 0; ks < 8; ++ks) {
+      uint32_t a[4];
+      a_km(x.sb + so + CF::F_W, 128, 16 * tb, 16 * ks, lane, a);       // W [t][c] from W^T
+      if constexpr (NH == 2) {
+        uint32_t b[4];
+        b_nk(uS, NB, 16 * jh, 16 * ks, lane, b);                       // S [c][j] from [j][c]
         mma(acc[0][ks & 1], a, b[0], b[1]);
         mma(acc[1][ks & 1], a, b[2], b[3]);
+      } else {
+        uint32_t b[2];
+        b_nk1(uS, NB, 8 * jh, 16 * ks, lane, b);
+        mma(acc[0][ks & 1], a, b[0], b[1]);
       }
-      uint8_t* gD = dlimg + (base + n) * kImgD;
-#pragma unroll
-      for (int p = 0; p < 2; ++p) {
-        const int n0 = 16 * jh + 8 * p, jl = n0 + 2 * qd;
-        float dl[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int t = 16 * tb + g + ((e >> 1) << 3);
-          dl[e] = bf_at(sm + so + CF::F_U + io(jl + (e & 1), t, NB)) - acc[p][0][e] - acc[p][1][e];
-        }
-        st_mn1(uDL, 64, 16 * tb, n0, lane, dl, 1.f);
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf)
-          *reinterpret_cast<uint32_t*>(gD + io(16 * tb + g + 8 * hf, j0 + jl, 64)) =
-              pack_bf16(dl[2 * hf], dl[2 * hf + 1]);
-      }
-      __syncthreads();
-      // S <- Diag(exp(Gamma_last)) S + Kend^T Delta
-      const float* dec = reinterpret_cast<const float*>(sm + so + CF::F_DEC);
-      const float d0 = dec[cr + g], d1 = dec[cr + g + 8];
-      float Y[4][4] = {};
-#pragma unroll
-      for (int nt = 0; nt < 4; ++nt) {
-        X[nt][0] *= d0; X[nt][1] *= d0; X[nt][2] *= d1; X[nt][3] *= d1;
-      }
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks) update(sb + so + CF::F_K, uDL, Y, ks, ks & 1);
-#pragma unroll
-      for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) X[nt][e] += Y[nt][e];
-      issue(n + STG - 1);               // into chunk n - 1's stage, read before this step's barrier
     }
-    return;
+    uint8_t* gD = dlimg + (x.base + n) * kImgD;
+#pragma unroll
+    for (int p = 0; p < NH; ++p) {
+      const int n0 = 8 * (jh * NH + p), jl = n0 + 2 * qd;
+      float dl[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int t = 16 * tb + g + ((e >> 1) << 3);
+        dl[e] = bf_at(x.sm + so + CF::F_U + io(jl + (e & 1), t, NB)) - acc[p][0][e] - acc[p][1][e];
+      }
+      st_mn1(uDL, 64, 16 * tb, n0, lane, dl, 1.f);
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf)
+        *reinterpret_cast<uint32_t*>(gD + io(16 * tb + g + 8 * hf, x.j0 + jl, 64)) =
+            pack_bf16(dl[2 * hf], dl[2 * hf + 1]);
+    }
+    __syncthreads();
+    // S <- Diag(exp(Gamma_last)) S + Kend^T Delta
+    const float* dec = reinterpret_cast<const float*>(x.sm + so + CF::F_DEC);
+    const float d0 = dec[16 * x.w + g], d1 = dec[16 * x.w + g + 8];
+    float Y[NJ][4] = {};
+#pragma unroll
+    for (int nt = 0; nt < NJ; ++nt) {
+      X[nt][0] *= d0; X[nt][1] *= d0; X[nt][2] *= d1; X[nt][3] *= d1;
+    }
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) chain_update<NB>(x, x.sb + so + CF::F_K, uDL, X, Y, ks, ks & 1);
+#pragma unroll
+    for (int nt = 0; nt < NJ; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) X[nt][e] += Y[nt][e];
+    issue(n + STG - 1);                 // into chunk n - 1's stage, read before this step's barrier
   }
+}
 
-  // ---- reverse chain
+// Reverse chain: dS after every chunk, dDelta of every chunk, and dh0.
+template <int NB>
+__device__ __forceinline__ void chain_reverse(const ChainCtx& x, const float* dhT, float* dh0,
+                                              uint8_t* dsimg, uint8_t* ddimg) {
+  using CF = Chain<NB>;
+  constexpr int NJ = NB / 8, NH = NB / 16, STG = CF::STG;
+  const int tb = x.w & 3, jh = x.w >> 2, g = x.g, qd = x.qd, lane = x.lane;
+  float X[NJ][4];
+  chain_load<NB>(x, dhT, X);
   auto issue = [&](int n) {
     if (n >= 0) {
-      const uint8_t* rc = rec + (base + n) * rec::BYTES_BWD;
-      uint8_t* st = sm + (n % STG) * CF::R_STAGE;
-      if (tid == NTC - 32) {
-        uint64_t* bar = &full[n % STG];
+      const uint8_t* rc = x.rec + (x.base + n) * rec::BYTES_BWD;
+      uint8_t* st = x.sm + (n % STG) * CF::R_STAGE;
+      if (x.tid == NTC - 32) {
+        uint64_t* bar = &x.full[n % STG];
         fence_async_smem();
         mbar_arrive_expect_tx(bar, CF::R_BYTES);
         bulk_g2s(st + CF::R_QW, rc + rec::QW, 32768, bar);
         bulk_g2s(st + CF::R_KA, rc + rec::KA, 24576, bar);
         bulk_g2s(st + CF::R_DEC, rc + rec::DECAY, 512, bar);
       }
-      const long long t0 = t_beg + (long long)n * C;
-      const int L = (int)min((long long)C, t_end - t0);
-      for (int i = tid; i < 64 * CF::NJ; i += NTC) {
-        const int t = i / CF::NJ, ck = i % CF::NJ;
-        const bf16* src = dout + ((row0 + t0 + min(t, L - 1)) * H + h) * D + j0 + 8 * ck;
+      const long long t0 = x.t_beg + (long long)n * C;
+      const int L = (int)min((long long)C, x.t_end - t0);
+      for (int i = x.tid; i < 64 * NJ; i += NTC) {
+        const int t = i / NJ, ck = i % NJ;
+        const bf16* src = x.dout + ((x.row0 + t0 + min(t, L - 1)) * x.H + x.h) * D + x.j0 + 8 * ck;
         cp_async16(st + CF::R_DO + io(t, 8 * ck, 64), src, t < L ? 16u : 0u);
       }
     }
     cp_async_commit();
   };
-  const uint32_t uY = sb + CF::R_Y, uDD = sb + CF::R_DD;
+  const uint32_t uY = x.sb + CF::R_Y, uDD = x.sb + CF::R_DD;
 #pragma unroll 1
-  for (int i = 0; i < STG - 1; ++i) issue(nch - 1 - i);
+  for (int i = 0; i < STG - 1; ++i) issue(x.nch - 1 - i);
 #pragma unroll 1
-  for (int n = nch - 1; n >= 0; --n) {
+  for (int n = x.nch - 1; n >= 0; --n) {
     const uint32_t so = (uint32_t)(n % STG) * CF::R_STAGE;
-    put_state(CF::R_Y, dsimg + (base + n) * kImgS);      // dS after chunk n
+    chain_put<NB>(x, X, CF::R_Y, dsimg + (x.base + n) * kImgS);   // dS after chunk n
     cp_async_wait_group<STG - 2>();
-    const bool ok = mbar_wait(&full[n % STG], (uint32_t)((nch - 1 - n) / STG) & 1u, kWaitLimit);
+    const bool ok =
+        mbar_wait(&x.full[n % STG], (uint32_t)((x.nch - 1 - n) / STG) & 1u, kWaitLimit);
     if (__syncthreads_or(!ok)) {
-      give_up(n, max(n - (STG - 2), 0), false);
+      chain_give_up<STG>(x, n, max(n - (STG - 2), 0), false);
       return;
     }
-    // dDelta = Kend dS + Aqk^T dO: token block tb, n8 tiles 2 jh, 2 jh + 1
-    float acc[2][2][4] = {};
+    // dDelta = Kend dS + Aqk^T dO: token block tb, n8 tiles jh * NH ..
+    float acc[NH][2][4] = {};
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
-      uint32_t a[4], b[4];
-      a_km(sb + so + CF::R_KA, 128, 16 * tb, 16 * ks, lane, a);          // Kend [t][c] from Kend^T
-      b_nk(uY, NB, 16 * jh, 16 * ks, lane, b);                           // dS [c][j] from [j][c]
-      mma(acc[0][ks & 1], a, b[0], b[1]);
-      mma(acc[1][ks & 1], a, b[2], b[3]);
+      uint32_t a[4];
+      a_km(x.sb + so + CF::R_KA, 128, 16 * tb, 16 * ks, lane, a);          // Kend [t][c] from Kend^T
+      if constexpr (NH == 2) {
+        uint32_t b[4];
+        b_nk(uY, NB, 16 * jh, 16 * ks, lane, b);                           // dS [c][j] from [j][c]
+        mma(acc[0][ks & 1], a, b[0], b[1]);
+        mma(acc[1][ks & 1], a, b[2], b[3]);
+      } else {
+        uint32_t b[2];
+        b_nk1(uY, NB, 8 * jh, 16 * ks, lane, b);
+        mma(acc[0][ks & 1], a, b[0], b[1]);
+      }
     }
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) {
-      uint32_t a[4], b[4];
-      a_km(sb + so + CF::R_KA + 16384, 64, 16 * tb, 16 * ks, lane, a);   // Aqk^T [t][r] from Aqk
-      b_kn(sb + so + CF::R_DO, 64, 16 * jh, 16 * ks, lane, b);           // dO [r][j]
-      mma(acc[0][ks & 1], a, b[0], b[1]);
-      mma(acc[1][ks & 1], a, b[2], b[3]);
+      uint32_t a[4];
+      a_km(x.sb + so + CF::R_KA + 16384, 64, 16 * tb, 16 * ks, lane, a);   // Aqk^T [t][r] from Aqk
+      if constexpr (NH == 2) {
+        uint32_t b[4];
+        b_kn(x.sb + so + CF::R_DO, 64, 16 * jh, 16 * ks, lane, b);         // dO [r][j]
+        mma(acc[0][ks & 1], a, b[0], b[1]);
+        mma(acc[1][ks & 1], a, b[2], b[3]);
+      } else {
+        uint32_t b[2];
+        b_kn1(x.sb + so + CF::R_DO, 64, 8 * jh, 16 * ks, lane, b);
+        mma(acc[0][ks & 1], a, b[0], b[1]);
+      }
     }
-    uint8_t* gD = ddimg + (base + n) * kImgD;
+    uint8_t* gD = ddimg + (x.base + n) * kImgD;
 #pragma unroll
-    for (int p = 0; p < 2; ++p) {
-      const int n0 = 16 * jh + 8 * p, jl = n0 + 2 * qd;
+    for (int p = 0; p < NH; ++p) {
+      const int n0 = 8 * (jh * NH + p), jl = n0 + 2 * qd;
       float dd[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) dd[e] = acc[p][0][e] + acc[p][1][e];
       st_mn1(uDD, 64, 16 * tb, n0, lane, dd, -1.f);
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf)
-        *reinterpret_cast<uint32_t*>(gD + io(16 * tb + g + 8 * hf, j0 + jl, 64)) =
+        *reinterpret_cast<uint32_t*>(gD + io(16 * tb + g + 8 * hf, x.j0 + jl, 64)) =
             pack_bf16(dd[2 * hf], dd[2 * hf + 1]);
     }
     __syncthreads();
     // dS <- Diag(exp(Gamma_last)) dS + Qbar^T dO - W^T dDelta
-    const float* dec = reinterpret_cast<const float*>(sm + so + CF::R_DEC);
-    const float d0 = dec[cr + g], d1 = dec[cr + g + 8];
-    float Y[4][4] = {};
+    const float* dec = reinterpret_cast<const float*>(x.sm + so + CF::R_DEC);
+    const float d0 = dec[16 * x.w + g], d1 = dec[16 * x.w + g + 8];
+    float Y[NJ][4] = {};
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
+    for (int nt = 0; nt < NJ; ++nt) {
       X[nt][0] *= d0; X[nt][1] *= d0; X[nt][2] *= d1; X[nt][3] *= d1;
     }
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) {
-      update(sb + so + CF::R_QW, sb + so + CF::R_DO, Y, ks, ks & 1);         // Qbar^T dO
-      update(sb + so + CF::R_QW + 16384, uDD, Y, ks, !(ks & 1));             // W^T (-dDelta)
+      chain_update<NB>(x, x.sb + so + CF::R_QW, x.sb + so + CF::R_DO, X, Y, ks, ks & 1);  // Qbar^T dO
+      chain_update<NB>(x, x.sb + so + CF::R_QW + 16384, uDD, X, Y, ks, !(ks & 1));     // W^T (-dDelta)
     }
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
+    for (int nt = 0; nt < NJ; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) X[nt][e] += Y[nt][e];
     issue(n - (STG - 1));               // into chunk n + 1's stage, read before this step's barrier
@@ -460,13 +483,62 @@ kda_bwd_chain_kernel(const uint8_t* __restrict__ rec, const float* __restrict__ 
   cp_async_wait_all();
   if (dh0) {
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
+    for (int nt = 0; nt < NJ; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int c = cr + g + ((e >> 1) << 3), j = j0 + 8 * nt + 2 * qd + (e & 1);
-        dh0[st_off + (size_t)c * D + j] = X[nt][e];
+        const int c = 16 * x.w + g + ((e >> 1) << 3), j = x.j0 + 8 * nt + 2 * qd + (e & 1);
+        dh0[x.st_off + (size_t)c * D + j] = X[nt][e];
       }
   }
+}
+
+// Chain kernel: CTA (xb, h, s) with xb < D / NBF walks sequence s of head h forward for the
+// value columns [NBF xb, NBF xb + NBF); the others walk it backward, NBR columns each (the
+// reverse step reads more operands, so it takes narrower blocks; both directions fit one wave
+// at the headline shape).
+template <int NBF, int NBR>
+__global__ void __launch_bounds__(NTC, 1)
+kda_bwd_chain_kernel(const uint8_t* __restrict__ rec, const float* __restrict__ h0,
+                     const int32_t* __restrict__ cu_seqlens, const bf16* __restrict__ dout,
+                     const float* __restrict__ dhT, float* __restrict__ dh0,
+                     uint8_t* __restrict__ simg, uint8_t* __restrict__ dlimg,
+                     uint8_t* __restrict__ dsimg, uint8_t* __restrict__ ddimg, int T, int H,
+                     long long nslots) {
+  constexpr int STG = Chain<NBF>::STG;
+  static_assert(Chain<NBR>::STG == STG, "one stage count");
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t full[STG];           // record stage landed (bulk copies)
+  ChainCtx x;
+  x.sm = align1024(smem_raw);
+  x.sb = smem_u32(x.sm);
+  x.full = full;
+  x.rec = rec;
+  x.dout = dout;
+  x.tid = threadIdx.x;
+  x.w = x.tid >> 5;
+  x.lane = x.tid & 31;
+  x.g = x.lane >> 2;
+  x.qd = x.lane & 3;
+  constexpr int NF = D / NBF;
+  const bool fwd = (int)blockIdx.x < NF;
+  x.j0 = fwd ? (int)blockIdx.x * NBF : ((int)blockIdx.x - NF) * NBR;
+  x.h = blockIdx.y;
+  x.H = H;
+  const int s = blockIdx.z;
+  seq_range(cu_seqlens, s, T, x.row0, x.t_beg, x.t_end);
+  x.nch = (int)chunk_count(x.t_end - x.t_beg);
+  x.base = (size_t)x.h * (size_t)nslots + (size_t)seq_chunk_base(cu_seqlens, s, T);
+  x.st_off = ((size_t)s * H + x.h) * D * D;
+  if (x.tid == 0) {
+#pragma unroll
+    for (int i = 0; i < STG; ++i) mbar_init(&full[i], 1);
+    fence_mbar_init();
+  }
+  grid_dep_launch();                       // the gradient kernel may start preloading its inputs
+  __syncthreads();                         // the barriers are initialised
+  grid_dep_wait();                         // the records are complete
+  if (fwd) chain_forward<NBF>(x, h0, simg, dlimg);
+  else chain_reverse<NBR>(x, dhT, dh0, dsimg, ddimg);
 }
 
 // ============================================================================
@@ -1309,13 +1381,15 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   if (tid < L) dbeta[(rb + tid) * H + h] = s_dbeta[tid];
 }
 
-constexpr int kChainNB = 32;
+constexpr int kChainF = 32, kChainR = 16;      // value columns per forward / reverse chain
+constexpr uint32_t kChainSmem = Chain<kChainF>::SMEM > Chain<kChainR>::SMEM ? Chain<kChainF>::SMEM
+                                                                          : Chain<kChainR>::SMEM;
 
 bool set_attrs() {
   return once_per_device(kOnceBwdTc, []() {
-    return cudaFuncSetAttribute(kda_bwd_chain_kernel<kChainNB>,
+    return cudaFuncSetAttribute(kda_bwd_chain_kernel<kChainF, kChainR>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                Chain<kChainNB>::SMEM) == cudaSuccess &&
+                                kChainSmem) == cudaSuccess &&
            cudaFuncSetAttribute(kda_bwd_grad_kernel<false>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, GRAD_SMEM) == cudaSuccess &&
            cudaFuncSetAttribute(kda_bwd_grad_kernel<true>,
@@ -1378,10 +1452,10 @@ cudaError_t launch_chunk_bwd_tc(const void* q, const void* k, const void* v, con
   cudaError_t e = launch_chunk_prep_bwd(q, k, v, g, beta, cu_seqlens, rec, B, T, H, gsh,
                                         sc.nslots, stream);
   if (e == cudaSuccess) {
-    using CF = Chain<kChainNB>;
     KDA_TIMED(KDA_KERNEL_BWD_CHAIN, stream,
-              e = launch_after(kda_bwd_chain_kernel<kChainNB>, dim3(2 * CF::NJB, H, B), dim3(NTC),
-                               CF::SMEM, stream, rec, h0, cu_seqlens,
+              e = launch_after(kda_bwd_chain_kernel<kChainF, kChainR>,
+                               dim3(D / kChainF + D / kChainR, H, B), dim3(NTC), kChainSmem,
+                               stream, rec, h0, cu_seqlens,
                                static_cast<const bf16*>(dout), dhT, dh0, base + sc.simg,
                                base + sc.dlimg, base + sc.dsimg, base + sc.ddimg, T, H,
                                sc.nslots));
