@@ -843,14 +843,20 @@ KERNEL_NAMES = {"prep": "kda_chunk_prep_kernel", "state": "kda_state_pass_kernel
                 "simt": "kda_chunk_simt_kernel"}
 
 
+# the sources the split prefill's kernels (prep kernel, state pass) are compiled from
+TRAFFIC_SOURCES = ("chunk_split.cu", "chunk_record.cuh", "decay_pairs.cuh", "kda_common.cuh",
+                   "segments.cuh", "sm100.cuh", "tma.cuh")
+
+
 def _source_hash() -> str:
-    """Hash of the kernel sources with comments and whitespace removed: DRAM traffic
-    depends on the code, so a comment edit keeps a capture valid."""
+    """Hash of the split prefill's kernel sources with comments and whitespace removed:
+    DRAM traffic depends on that code, so a comment edit (or a change to another kernel)
+    keeps a capture valid."""
     import hashlib
     import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_delta_rule_74_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in TRAFFIC_SOURCES:
         with open(os.path.join(csrc, name), encoding="utf-8") as f:
             text = f.read()
         text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)        # block comments
