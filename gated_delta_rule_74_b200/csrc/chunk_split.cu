@@ -609,51 +609,92 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     prep_unsafe_direct(sm, rc, a, c0, (ux ? 1 : 0) | (uy ? 2 : 0), CONV, BWD, ur);
   }
 
-#pragma unroll
-  for (int ch = 0; ch < 2; ++ch) {
+  // the operand images of this thread's channel pair and 16-row block
+  auto put_rows = [&](int ch, int g8, const float (&lk)[8], const float (&lq)[8],
+                      const float (&kr)[8], float eP, float eE, const float (&f)[4]) {
     const int c = c0 + ch;
-    const float first = ch ? fo.y : fo.x;
     const bool uns = ch ? uy : ux;
-    const float eP = __expf((ch ? off.y : off.x) + first);   // Kbar, Qbar: e^{G_r} = e^{G_r - P_a} e^{P_a}
-    const float eE = __expf((ch ? rel.y : rel.x) - first);   // Kend: e^{G_last - G_i} = e^{P_a - G_i} e^{G_last - P_a}
+    if (c0 < dk) {
+      // the Gram operands (its K loop covers channels < dk only)
+      sts16(sm, Q_L + chunk_mnmajor_sw128(g8, c, D), pack8(lk, 1.f));
+      sts16(sm, Q_L + chunk_mnmajor_sw128(8 + g8, c, D), pack8(lq, 1.f));
+      if (!uns) {
+#pragma unroll
+        for (int a2 = 0; a2 < 4; ++a2)
+          if (a2 >= a) sts16(sm, q_r(a2) + chunk_mnmajor_sw32(g8, c, D), pack8(kr, f[a2]));
+      }
+    }
+    sts16(sm, Q_KB + chunk_kmajor_sw128(c, g8, D), pack8(lk, eP));
+    // record: Qbar^T (MN-major, N = tokens, K = channels) and Kend^T (K-major)
+    *reinterpret_cast<uint4*>(rc + REC_QW + chunk_mnmajor_sw128(g8, c, D)) = pack8(lq, eP);
+    if (!uns)
+      *reinterpret_cast<uint4*>(rc + REC_KA + chunk_kmajor_sw128(c, g8, D)) =
+          BWD ? pack8(kr, eE) : pack8_f16(kr, eE);
+  };
+  if constexpr (GRPD) {
+    // one decay per group of at least two channels: the pair's exponentials are shared
+    const float first = fo.x;
+    const float eP = __expf(off.x + first);   // Kbar, Qbar: e^{G_r} = e^{G_r - P_a} e^{P_a}
+    const float eE = __expf(rel.x - first);   // Kend: e^{G_last - G_i} = e^{P_a - G_i} e^{G_last - P_a}
     float f[4];
 #pragma unroll
-    for (int a2 = 0; a2 < 4; ++a2)
-      f[a2] = a2 > a ? __expf((ch ? d[a2].y : d[a2].x) - first) : 1.f;   // e^{P_{a2} - P_a}
+    for (int a2 = 0; a2 < 4; ++a2) f[a2] = a2 > a ? __expf(d[a2].x - first) : 1.f;
 #pragma unroll
     for (int gg = 0; gg < 2; ++gg) {
       const int g8 = 2 * a + gg;               // group of 8 rows
-      float lk[8], lq[8], kr[8];
-      if (c0 < dk) {
+      float ell[8], rho[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float x = gq[8 * gg + e].x - first;                  // G_r - P_a
+        ell[e] = __expf(x);
+        rho[e] = __expf(fminf(-x, 80.f));
+      }
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
+        float lk[8], lq[8], kr[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const int idx = 8 * gg + e;
-          const float x = (ch ? gq[idx].y : gq[idx].x) - first;   // G_r - P_a
-          const float ell = __expf(x);
-          const float rho = __expf(fminf(-x, 80.f));
-          const float kv = kval(idx, ch), qv = qval(idx, ch);
-          lk[e] = kv * ell;
-          lq[e] = qv * ell;
-          kr[e] = kv * rho;                    // k_i e^{P_a - G_i}
+          const float kv = c0 < dk ? kval(8 * gg + e, ch) : 0.f;
+          const float qv = c0 < dk ? qval(8 * gg + e, ch) : 0.f;
+          lk[e] = kv * ell[e];
+          lq[e] = qv * ell[e];
+          kr[e] = kv * rho[e];                 // k_i e^{P_a - G_i}
         }
-        // the Gram operands (its K loop covers channels < dk only)
-        sts16(sm, Q_L + chunk_mnmajor_sw128(g8, c, D), pack8(lk, 1.f));
-        sts16(sm, Q_L + chunk_mnmajor_sw128(8 + g8, c, D), pack8(lq, 1.f));
-        if (!uns) {
-#pragma unroll
-          for (int a2 = 0; a2 < 4; ++a2)
-            if (a2 >= a) sts16(sm, q_r(a2) + chunk_mnmajor_sw32(g8, c, D), pack8(kr, f[a2]));
-        }
-      } else {                         // padded channels (dk = 64; whole warps): zeros
-#pragma unroll
-        for (int e = 0; e < 8; ++e) lk[e] = lq[e] = kr[e] = 0.f;
+        put_rows(ch, g8, lk, lq, kr, eP, eE, f);
       }
-      sts16(sm, Q_KB + chunk_kmajor_sw128(c, g8, D), pack8(lk, eP));
-      // record: Qbar^T (MN-major, N = tokens, K = channels) and Kend^T (K-major)
-      *reinterpret_cast<uint4*>(rc + REC_QW + chunk_mnmajor_sw128(g8, c, D)) = pack8(lq, eP);
-      if (!uns)
-        *reinterpret_cast<uint4*>(rc + REC_KA + chunk_kmajor_sw128(c, g8, D)) =
-            BWD ? pack8(kr, eE) : pack8_f16(kr, eE);
+    }
+  } else {
+#pragma unroll
+    for (int ch = 0; ch < 2; ++ch) {
+      const float first = ch ? fo.y : fo.x;
+      const float eP = __expf((ch ? off.y : off.x) + first);
+      const float eE = __expf((ch ? rel.y : rel.x) - first);
+      float f[4];
+#pragma unroll
+      for (int a2 = 0; a2 < 4; ++a2)
+        f[a2] = a2 > a ? __expf((ch ? d[a2].y : d[a2].x) - first) : 1.f;   // e^{P_{a2} - P_a}
+#pragma unroll
+      for (int gg = 0; gg < 2; ++gg) {
+        const int g8 = 2 * a + gg;             // group of 8 rows
+        float lk[8], lq[8], kr[8];
+        if (c0 < dk) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int idx = 8 * gg + e;
+            const float x = (ch ? gq[idx].y : gq[idx].x) - first;   // G_r - P_a
+            const float ell = __expf(x);
+            const float rho = __expf(fminf(-x, 80.f));
+            const float kv = kval(idx, ch), qv = qval(idx, ch);
+            lk[e] = kv * ell;
+            lq[e] = qv * ell;
+            kr[e] = kv * rho;                  // k_i e^{P_a - G_i}
+          }
+        } else {                       // padded channels (dk = 64; whole warps): zeros
+#pragma unroll
+          for (int e = 0; e < 8; ++e) lk[e] = lq[e] = kr[e] = 0.f;
+        }
+        put_rows(ch, g8, lk, lq, kr, eP, eE, f);
+      }
     }
   }
   if (a == 3)                                  // exp(G_last), G_last = off + rel
