@@ -1319,55 +1319,74 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       }
   }
 
-  // ---- phase 5: outputs (dq, dk and dGamma through shared memory, [64][LDG] fp32 each)
-  __syncthreads();                      // R images / corrections no longer read
-  float* dGs = reinterpret_cast<float*>(sm + G_S0);
-  float* dQs = dGs + 64 * LDG;
-  float* dKs = dQs + 64 * LDG;
+  // ---- phase 5: outputs.  dq and dk straight from the accumulators (each lane's pairs of
+  // channels: eight rows of 32 contiguous bytes per store); dg = the reverse cumulative sum
+  // of dGamma over the chunk's rows plus dGamma_last's state term: within the warp's 16 rows
+  // by shuffles, across the four row blocks through the block totals.
+  __syncthreads();                      // s_dgl and s_dbeta are complete; s_part is free
 #pragma unroll
   for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
-      const int o = (r0 + g8 + 8 * hf) * LDG + c0 + 8 * nt + 2 * qd;
-      *reinterpret_cast<float2*>(dGs + o) = make_float2(dG[nt][2 * hf], dG[nt][2 * hf + 1]);
-      *reinterpret_cast<float2*>(dQs + o) = make_float2(dQ[nt][2 * hf], dQ[nt][2 * hf + 1]);
-      *reinterpret_cast<float2*>(dKs + o) = make_float2(dK[nt][2 * hf], dK[nt][2 * hf + 1]);
+      const int r = r0 + g8 + 8 * hf;
+      if (r < L) {
+        const long long o = ((rb + r) * H + h) * D + c0 + 8 * nt + 2 * qd;
+        *reinterpret_cast<float2*>(dq + o) = make_float2(dQ[nt][2 * hf], dQ[nt][2 * hf + 1]);
+        *reinterpret_cast<float2*>(dk + o) = make_float2(dK[nt][2 * hf], dK[nt][2 * hf + 1]);
+      }
+    }
+  // suffix sums over the rows g8 (+8) of each half (lanes 4 apart are adjacent rows)
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+#pragma unroll
+      for (int s = 4; s < 32; s <<= 1) {
+        const float y = __shfl_down_sync(0xffffffffu, dG[nt][e], s);
+        if (lane + s < 32) dG[nt][e] += y;
+      }
+    }
+  // the lower half (rows 8..15) adds to every row of the upper one; lanes 0..3 then hold
+  // the block's totals
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+    for (int e1 = 0; e1 < 2; ++e1) {
+      const float lower = __shfl_sync(0xffffffffu, dG[nt][2 + e1], qd);
+      dG[nt][e1] += lower;
+      if (g8 == 0) s_part[tb][c0 + 8 * nt + 2 * qd + e1] = dG[nt][e1];
     }
   __syncthreads();
-  for (int i = tid; i < C * 32; i += NTG) {
-    const int r = i >> 5, c4 = i & 31;
-    if (r < L) {
-      const long long o = ((rb + r) * H + h) * D + 4 * c4;
-      *reinterpret_cast<float4*>(dq + o) = *reinterpret_cast<const float4*>(dQs + r * LDG + 4 * c4);
-      *reinterpret_cast<float4*>(dk + o) = *reinterpret_cast<const float4*>(dKs + r * LDG + 4 * c4);
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+    for (int e1 = 0; e1 < 2; ++e1) {
+      const int c = c0 + 8 * nt + 2 * qd + e1;
+      float add = s_dgl[c];
+      for (int b2 = tb + 1; b2 < 4; ++b2) add += s_part[b2][c];
+      dG[nt][e1] += add;
+      dG[nt][2 + e1] += add;
     }
-  }
-  if (tid < D) dGs[63 * LDG + tid] += s_dgl[tid];
-  __syncthreads();
-  // dg = reverse cumulative sum of dGamma: four threads per channel, 16 rows each
-  {
-    const int c = tid & 127, part = tid >> 7;
-    float x[16];
-#pragma unroll
-    for (int e = 0; e < 16; ++e) x[e] = dGs[(16 * part + e) * LDG + c];
-#pragma unroll
-    for (int e = 14; e >= 0; --e) x[e] += x[e + 1];
-    s_part[part][c] = x[0];
-    __syncthreads();
-    float add = 0.f;
-    for (int p2 = part + 1; p2 < 4; ++p2) add += s_part[p2][c];
-#pragma unroll
-    for (int e = 0; e < 16; ++e) dGs[(16 * part + e) * LDG + c] = x[e] + add;
-  }
-  __syncthreads();
   if constexpr (!GRPD) {
-    for (int i = tid; i < C * 32; i += NTG) {
-      const int r = i >> 5, c4 = i & 31;
-      if (r < L)
-        *reinterpret_cast<float4*>(dg + ((rb + r) * H + h) * D + 4 * c4) =
-            *reinterpret_cast<const float4*>(dGs + r * LDG + 4 * c4);
-    }
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const int r = r0 + g8 + 8 * hf;
+        if (r < L)
+          *reinterpret_cast<float2*>(dg + ((rb + r) * H + h) * D + c0 + 8 * nt + 2 * qd) =
+              make_float2(dG[nt][2 * hf], dG[nt][2 * hf + 1]);
+      }
   } else {
+    // one decay per group of 1 << gsh channels: the group's sum, through shared memory
+    float* dGs = reinterpret_cast<float*>(sm + G_S0);
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf)
+        *reinterpret_cast<float2*>(dGs + (r0 + g8 + 8 * hf) * LDG + c0 + 8 * nt + 2 * qd) =
+            make_float2(dG[nt][2 * hf], dG[nt][2 * hf + 1]);
+    __syncthreads();
     const int ng = D >> gsh, gs = 1 << gsh;
     for (int i = tid; i < C * ng; i += NTG) {
       const int r = i / ng, m = i % ng;
