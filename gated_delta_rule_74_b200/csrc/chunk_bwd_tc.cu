@@ -592,6 +592,7 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   const uint32_t sb = smem_u32(sm);
   __shared__ float s_beta[C], s_dbeta[C], s_dgl[D], s_part[4][D];
   __shared__ __align__(16) uint8_t s_uns[4][D];
+  __shared__ uint64_t s_img_bar;               // the chains' four images landed
 
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31, g8 = lane >> 2, qd = lane & 3;
   const long long slot = blockIdx.x;
@@ -624,6 +625,10 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   float* G = reinterpret_cast<float*>(sm + G_G);
 
   // ---- phase 0: loads (the inputs first; the chains' images once the chains are done)
+  if (tid == 0) {
+    mbar_init(&s_img_bar, 1);
+    fence_mbar_init();
+  }
   for (int i = tid; i < 1024; i += NTG) {
     const int t = i >> 4, c8 = i & 15;
     const long long src = ((rb + min(t, L - 1)) * H + h) * D + 8 * c8;
@@ -641,15 +646,13 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   }
   cp_async_commit();
   grid_dep_wait();
-  for (int i = tid; i < 2048; i += NTG) {
-    cp_async16(sm + G_S0 + 16 * i, simg + ix * kImgS + 16 * i, 16u);
-    cp_async16(sm + G_DS + 16 * i, dsimg + ix * kImgS + 16 * i, 16u);
+  if (tid == 0) {                       // the images: four bulk copies on one barrier
+    mbar_arrive_expect_tx(&s_img_bar, 2 * kImgS + 2 * kImgD);
+    bulk_g2s(sm + G_S0, simg + ix * kImgS, kImgS, &s_img_bar);
+    bulk_g2s(sm + G_DS, dsimg + ix * kImgS, kImgS, &s_img_bar);
+    bulk_g2s(sm + G_DL, dlimg + ix * kImgD, kImgD, &s_img_bar);
+    bulk_g2s(sm + G_DD, ddimg + ix * kImgD, kImgD, &s_img_bar);
   }
-  for (int i = tid; i < 1024; i += NTG) {
-    cp_async16(sm + G_DL + 16 * i, dlimg + ix * kImgD + 16 * i, 16u);
-    cp_async16(sm + G_DD + 16 * i, ddimg + ix * kImgD + 16 * i, 16u);
-  }
-  cp_async_commit();
   if (tid < C) {
     s_beta[tid] = tid < L ? beta[(rb + tid) * H + h] : 0.f;
     s_dbeta[tid] = 0.f;
@@ -662,7 +665,7 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       G[t * LDG + c] = t < L ? g[((rb + t) * H + h) * ng + (c >> gsh)] : 0.f;
     }
   }
-  cp_async_wait_group<1>();             // the inputs (the images may still be in flight)
+  cp_async_wait_all();                  // the inputs (the images may still be in flight)
   __syncthreads();
   // Gamma = cumsum g per channel: four threads per channel, 16 rows each
   {
@@ -679,8 +682,17 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
 #pragma unroll
     for (int e = 0; e < 16; ++e) G[(16 * part + e) * LDG + c] = x[e] + add;
   }
-  cp_async_wait_all();
-  __syncthreads();
+  {
+    bool ok = true;
+    if (w == 0) ok = mbar_wait(&s_img_bar, 0, kWaitLimit);
+    if (__syncthreads_or(!ok)) {        // the images never arrived: flag, let them land, leave
+      if (tid == 0) {
+        atomicExch(&g_bwd_tc_timeout, 1);
+        mbar_wait(&s_img_bar, 0, kWaitLimit);
+      }
+      return;
+    }
+  }
   // unsafe (block, channel) pairs; dGamma_last's state term e^Gamma_last sum_j S dS
   bool any_uns = false, far = false;
   {

@@ -4,7 +4,6 @@
 #include <stdint.h>
 
 #include <initializer_list>
-#include <mutex>
 
 #include "kda_common.cuh"
 
@@ -15,25 +14,16 @@ namespace {
 // is written earlier in the same call, so nothing needs clearing between calls.
 static __device__ __align__(256) float g_noalloc_scratch[KDA_NOALLOC_SCRATCH_BYTES / sizeof(float)];
 
-std::mutex g_mu;
-float* g_addr[64] = {};
-
 // Device address of the array on the current device.  In host code the array's
-// name only stands in for it, so the address is looked up once per device,
-// with that device current, and cached.
+// name only stands in for it, so the address is looked up on every call (the lookup
+// allocates nothing); a cached address would go stale if the context were rebuilt.
 float* scratch_address() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
-      (void)cudaGetLastError();
-      return nullptr;
-    }
-    g_addr[dev] = static_cast<float*>(p);
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
   }
-  return g_addr[dev];
+  return static_cast<float*>(p);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
