@@ -590,7 +590,7 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   const uint32_t sb = smem_u32(sm);
-  __shared__ float s_beta[C], s_dbeta[C], s_dgl[D], s_part[4][D];
+  __shared__ float s_beta[C], s_dbeta[C], s_dgl[D], s_part[4][D], s_daqk[C];
   __shared__ __align__(16) uint8_t s_uns[4][D];
   __shared__ uint64_t s_img_bar;               // the chains' four images landed
 
@@ -841,6 +841,14 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
           const int r = r0 + g8 + ((e >> 1) << 3);
           const int i = 16 * cq + 8 * sub + 2 * qd + (e & 1);
           if (i > r) aa[sub][e] = 0.f;
+          // the diagonal (i = r, decay factor e^0): kept apart in fp32 and left out of the
+          // image, so that the decay-weighted products below never form its dGamma terms,
+          // which cancel exactly (row side + q k dAqk, column side - q k dAqk); its dq and
+          // dk terms are added in phase 5
+          if (i == r) {
+            s_daqk[r] = aa[sub][e];
+            aa[sub][e] = 0.f;
+          }
         }
     }
     st_mn(sb + G_AQK, 64, r0, 16 * cq, lane, aa[0], aa[1], 1.f);
@@ -1341,6 +1349,14 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
       const int r = r0 + g8 + 8 * hf;
+      {                                 // A_qk's diagonal: dq_r += dAqk_rr k_r, dk_r += dAqk_rr q_r
+        const float dd = s_daqk[r];
+        const float2 kv = img2(G_K, hf, nt), qv = img2(G_Q, hf, nt);
+        dQ[nt][2 * hf] = fmaf(dd, kv.x, dQ[nt][2 * hf]);
+        dQ[nt][2 * hf + 1] = fmaf(dd, kv.y, dQ[nt][2 * hf + 1]);
+        dK[nt][2 * hf] = fmaf(dd, qv.x, dK[nt][2 * hf]);
+        dK[nt][2 * hf + 1] = fmaf(dd, qv.y, dK[nt][2 * hf + 1]);
+      }
       if (r < L) {
         const long long o = ((rb + r) * H + h) * D + c0 + 8 * nt + 2 * qd;
         *reinterpret_cast<float2*>(dq + o) = make_float2(dQ[nt][2 * hf], dQ[nt][2 * hf + 1]);

@@ -168,6 +168,22 @@ def test_long_sequence_sampled_heads():
     _assert_close(r, ref, heads=heads)
 
 
+def test_long_many_heads_sampled():
+    """B=1, T=32768, H=96 (the long-prefill shape): 512 chunks x 96 heads, so the chunk
+    records and state images span more than 4 GB of scratch (byte offsets past 2^32); the
+    last head, whose records sit at the end, against the oracle."""
+    spec = ki.PrefillSpec("bwdc", B=1, T=32768, H=96, dk=128, dv=128, dtype="bf16",
+                          decay="alog", seed=32768, h0=False)
+    x = ki.make_prefill(spec)
+    gen = torch.Generator().manual_seed(32769)
+    dout = torch.randn(x["v"].shape, generator=gen).to(torch.bfloat16)
+    r = _bwd(to_dev(x), dout, None, h0=False)
+    heads = (95, 96)
+    ref = oracle.backward(x["q"], x["k"], x["v"], x["g"], x["beta"], dout, None, None,
+                          heads=heads)
+    _assert_close(r, ref, heads=heads)
+
+
 def test_agrees_with_recurrent_sweep():
     spec = ki.PrefillSpec("bwdc", B=2, T=300, H=4, dk=128, dv=128, dtype="bf16",
                           decay="logsigmoid", seed=77, h0=True)

@@ -74,3 +74,50 @@ def test_decode_chunk_graph_replay_matches_eager():
     g.replay()
     torch.cuda.synchronize()
     assert torch.equal(out, out_e) and torch.equal(S, S_e)
+
+
+@pytest.mark.parametrize("packed", [False, True])
+def test_backward_graph_replay_matches_eager(packed):
+    """The chunked backward (its prep, chain and gradient launches under programmatic
+    stream serialization, scratch from the stream-ordered pool) captured into a graph:
+    dq, dk, dv and dh0 replay bit for bit, dg and dbeta (shared-memory atomics) to fp32
+    rounding, and a replay after the cotangent changes in place follows it."""
+    if packed:
+        spec = ki.PrefillSpec("varlen", B=0, T=0, H=2, dk=128, dv=128, dtype="bf16",
+                              decay="alog", seed=51, h0=True, varlen=True)
+        x = ki.make_prefill(spec, doc_lens=[300, 65, 1, 200])
+    else:
+        x = ki.make_prefill(ki.PrefillSpec("graph", B=2, T=700, H=2, dk=128, dv=128,
+                                           dtype="bf16", decay="logsigmoid", seed=52, h0=True))
+    d = to_dev(x)
+    nseq = d["h0"].shape[0]
+    gen = torch.Generator().manual_seed(53)
+    dout = torch.randn(d["v"].shape, generator=gen).to(torch.bfloat16).cuda()
+    dhT = (0.1 * torch.randn((nseq, 2, 128, 128), generator=gen)).cuda()
+
+    def call(grads=None):
+        return kda.kda_chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], dout, h0=d["h0"],
+                                 dhT=dhT, cu_seqlens=d["cu_seqlens"], grads=grads)
+
+    eager = call()
+    torch.cuda.synchronize()
+    grads = {n: torch.empty_like(t) for n, t in eager.items() if t is not None}
+    g = _capture(lambda: call(grads))
+
+    def check(ref):
+        for n in ("dq", "dk", "dv", "dh0"):
+            assert torch.equal(grads[n], ref[n]), n
+        for n in ("dg", "dbeta"):
+            torch.testing.assert_close(grads[n], ref[n], rtol=1e-5, atol=1e-6)
+
+    for _ in range(2):
+        for t in grads.values():
+            t.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        check(eager)
+    dout.copy_(torch.randn(dout.shape, generator=gen).to(torch.bfloat16).cuda())
+    eager2 = call()
+    g.replay()
+    torch.cuda.synchronize()
+    check(eager2)
