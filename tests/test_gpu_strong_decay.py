@@ -248,3 +248,17 @@ def test_backward_every_channel_strong(case):
             assert torch.isfinite(got).all(), name
             tol = 1e-4 if recurrent else (2e-2 if name == "dbeta" else TOL["bf16"])
             assert rel_err(got, ref[name]) <= tol, (recurrent, name, rel_err(got, ref[name]))
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_prefill_every_channel_strong(dtype):
+    """The forward in the same regime (every channel decaying by 5.5-6.5 per token, long
+    enough for the segment split): the output and final state within the bound."""
+    x = ki.make_prefill(_spec(dtype=dtype, B=1, T=1500, H=2, seed=17))
+    gen = torch.Generator().manual_seed(98)
+    x = dict(x)
+    x["g"] = -(5.5 + torch.rand(x["g"].shape, generator=gen))
+    d = to_dev(x)
+    out, hT = kda.kda_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], h0=d["h0"])
+    torch.cuda.synchronize()
+    _check(x, out, hT)
