@@ -17,7 +17,7 @@
 // reverse cumulative sum of dGamma inside the chunk.
 //
 // Three launches after the prep kernel's backward form (per (chunk, head): the
-// record images in bf16, plus T and A in fp32; chunk_split.cu):
+// record images in bf16, T as a bf16 image too, and A in fp32; chunk_split.cu):
 //   chains    the state and its gradient move across a sequence's chunks column
 //             block by column block (every column of S, and of dS, evolves on its
 //             own): per (column block, head, sequence) one CTA walks the chunks
@@ -373,7 +373,7 @@ __device__ __forceinline__ void chain_forward(const ChainCtx& x, const float* h0
 // Reverse chain: dS after every chunk, dDelta of every chunk, and dh0.
 template <int NB>
 __device__ __forceinline__ void chain_reverse(const ChainCtx& x, const float* dhT, float* dh0,
-                                              uint8_t* dsimg, uint8_t* ddimg) {
+                                              uint8_t* dsimg, uint8_t* ddimg, uint8_t* ddlo) {
   using CF = Chain<NB>;
   constexpr int NJ = NB / 8, NH = NB / 16, STG = CF::STG;
   const int tb = x.w & 3, jh = x.w >> 2, g = x.g, qd = x.qd, lane = x.lane;
@@ -448,6 +448,7 @@ __device__ __forceinline__ void chain_reverse(const ChainCtx& x, const float* dh
       }
     }
     uint8_t* gD = ddimg + (x.base + n) * kImgD;
+    uint8_t* gDl = ddlo + (x.base + n) * kImgD;
 #pragma unroll
     for (int p = 0; p < NH; ++p) {
       const int n0 = 8 * (jh * NH + p), jl = n0 + 2 * qd;
@@ -456,9 +457,16 @@ __device__ __forceinline__ void chain_reverse(const ChainCtx& x, const float* dh
       for (int e = 0; e < 4; ++e) dd[e] = acc[p][0][e] + acc[p][1][e];
       st_mn1(uDD, 64, 16 * tb, n0, lane, dd, -1.f);
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf)
-        *reinterpret_cast<uint32_t*>(gD + io(16 * tb + g + 8 * hf, x.j0 + jl, 64)) =
-            pack_bf16(dd[2 * hf], dd[2 * hf + 1]);
+      for (int hf = 0; hf < 2; ++hf) {
+        // dDelta as a bf16 pair: hi, and lo = dDelta - hi (the gradient kernel's
+        // T^T dDelta for dv and dbeta takes both)
+        const uint32_t o = io(16 * tb + g + 8 * hf, x.j0 + jl, 64);
+        const uint32_t hi = pack_bf16(dd[2 * hf], dd[2 * hf + 1]);
+        *reinterpret_cast<uint32_t*>(gD + o) = hi;
+        *reinterpret_cast<uint32_t*>(gDl + o) =
+            pack_bf16(dd[2 * hf] - __uint_as_float(hi << 16),
+                      dd[2 * hf + 1] - __uint_as_float(hi & 0xffff0000u));
+      }
     }
     __syncthreads();
     // dS <- Diag(exp(Gamma_last)) dS + Qbar^T dO - W^T dDelta
@@ -502,8 +510,8 @@ kda_bwd_chain_kernel(const uint8_t* __restrict__ rec, const float* __restrict__ 
                      const int32_t* __restrict__ cu_seqlens, const bf16* __restrict__ dout,
                      const float* __restrict__ dhT, float* __restrict__ dh0,
                      uint8_t* __restrict__ simg, uint8_t* __restrict__ dlimg,
-                     uint8_t* __restrict__ dsimg, uint8_t* __restrict__ ddimg, int T, int H,
-                     long long nslots) {
+                     uint8_t* __restrict__ dsimg, uint8_t* __restrict__ ddimg,
+                     uint8_t* __restrict__ ddlo, int T, int H, long long nslots) {
   constexpr int STG = Chain<NBF>::STG;
   static_assert(Chain<NBR>::STG == STG, "one stage count");
   extern __shared__ uint8_t smem_raw[];
@@ -538,7 +546,7 @@ kda_bwd_chain_kernel(const uint8_t* __restrict__ rec, const float* __restrict__ 
   __syncthreads();                         // the barriers are initialised
   grid_dep_wait();                         // the records are complete
   if (fwd) chain_forward<NBF>(x, h0, simg, dlimg);
-  else chain_reverse<NBR>(x, dhT, dh0, dsimg, ddimg);
+  else chain_reverse<NBR>(x, dhT, dh0, dsimg, ddimg, ddlo);
 }
 
 // ============================================================================
@@ -553,7 +561,7 @@ constexpr int LDG = 136;                       // Gamma / dGamma row stride (flo
 constexpr uint32_t G_Q = 0;                    // q image [t][c]
 constexpr uint32_t G_K = 16384;                // k image [t][c]
 constexpr uint32_t G_G = 32768;                // Gamma fp32 [64][LDG]
-constexpr uint32_t G_S0 = 67584;               // S image [j][c]  | T, A fp32 [64][64] | R images
+constexpr uint32_t G_S0 = 67584;               // S image [j][c]  | dDelta lo image, A fp32 [64][64] | R images
 constexpr uint32_t G_DS = 100352;              // dS image [j][c] | Kb, Vb images | X fp32 [64][68]
 constexpr uint32_t G_DO = 133120;              // dO image [t][j] | V image | dT^T fp32 [64][68]
 constexpr uint32_t G_DL = 149504;              // Delta image     | T image (bf16)
@@ -584,6 +592,7 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
                     const int32_t* __restrict__ cu_seqlens, const uint8_t* __restrict__ rec,
                     const uint8_t* __restrict__ simg, const uint8_t* __restrict__ dlimg,
                     const uint8_t* __restrict__ dsimg, const uint8_t* __restrict__ ddimg,
+                    const uint8_t* __restrict__ ddlo,
                     float* __restrict__ dq, float* __restrict__ dk, float* __restrict__ dv,
                     float* __restrict__ dg, float* __restrict__ dbeta, int B, int T, int H,
                     int gsh, long long nslots) {
@@ -780,8 +789,11 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     }
     st_mn(sb + G_DW, 64, r0, c0 + 16 * np, lane, aw[0], aw[1], -1.f);   // dW = -dDelta S^T
   }
-  __syncthreads();                      // S image no longer read: T and A go there
-  for (int i = tid; i < 2048; i += NTG) cp_async16(sm + G_S0 + 16 * i, rc + rec::TMAT + 16 * i, 16u);
+  __syncthreads();                      // S image no longer read: dDelta's lo image and A go there
+  for (int i = tid; i < 1024; i += NTG) {
+    cp_async16(sm + G_S0 + 16 * i, ddlo + ix * kImgD + 16 * i, 16u);
+    cp_async16(sm + G_S0 + 16384 + 16 * i, rc + rec::AMAT + 16 * i, 16u);
+  }
   cp_async_commit();
 #pragma unroll
   for (int np = 0; np < 2; ++np) {
@@ -859,6 +871,8 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
     cp_async16(sm + G_DO + io(t, 8 * c8, 64), v + ((rb + min(t, L - 1)) * H + h) * D + 8 * c8,
                t < L ? 16u : 0u);
   }
+  // the T image (bf16 [r][i], as the record holds it) to G_DL
+  for (int i = tid; i < 512; i += NTG) cp_async16(sm + G_DL + 16 * i, rc + rec::TMAT + 16 * i, 16u);
   cp_async_commit();
   // Kb = diag(beta) Kbar = beta k e^Gamma (image [i][c] at G_DS)
   for (int i = tid; i < 1024; i += NTG) {
@@ -881,29 +895,19 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
   }
   cp_async_wait_all();
   __syncthreads();
-  const float* Tm = reinterpret_cast<const float*>(sm + G_S0);           // T [r][i]
   const float* Am = reinterpret_cast<const float*>(sm + G_S0 + 16384);   // A [r][i]
-  // T image (bf16 [r][i] at G_DL) and Vb = diag(beta) V (image [i][j] at G_DS + 16384)
-  for (int i = tid; i < 1536; i += NTG) {
-    if (i < 512) {
-      const int r = i >> 3, c8 = i & 7;
-      const float4 a4 = *reinterpret_cast<const float4*>(Tm + r * 64 + 8 * c8);
-      const float4 b4 = *reinterpret_cast<const float4*>(Tm + r * 64 + 8 * c8 + 4);
-      *reinterpret_cast<uint4*>(sm + G_DL + io(r, 8 * c8, 64)) =
-          make_uint4(pack_bf16(a4.x, a4.y), pack_bf16(a4.z, a4.w), pack_bf16(b4.x, b4.y),
-                     pack_bf16(b4.z, b4.w));
-    } else {
-      const int t = (i - 512) >> 4, c8 = (i - 512) & 15;
-      const float bt = s_beta[t];
-      const uint4 vw = *reinterpret_cast<const uint4*>(sm + G_DO + io(t, 8 * c8, 64));
-      const uint32_t vv[4] = {vw.x, vw.y, vw.z, vw.w};
-      uint32_t o[4];
+  // Vb = diag(beta) V (image [i][j] at G_DS + 16384)
+  for (int i = tid; i < 1024; i += NTG) {
+    const int t = i >> 4, c8 = i & 15;
+    const float bt = s_beta[t];
+    const uint4 vw = *reinterpret_cast<const uint4*>(sm + G_DO + io(t, 8 * c8, 64));
+    const uint32_t vv[4] = {vw.x, vw.y, vw.z, vw.w};
+    uint32_t o[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        o[e] = pack_bf16(bt * __uint_as_float(vv[e] << 16), bt * __uint_as_float(vv[e] & 0xffff0000u));
-      *reinterpret_cast<uint4*>(sm + G_DS + 16384 + io(t, 8 * c8, 64)) =
-          make_uint4(o[0], o[1], o[2], o[3]);
-    }
+    for (int e = 0; e < 4; ++e)
+      o[e] = pack_bf16(bt * __uint_as_float(vv[e] << 16), bt * __uint_as_float(vv[e] & 0xffff0000u));
+    *reinterpret_cast<uint4*>(sm + G_DS + 16384 + io(t, 8 * c8, 64)) =
+        make_uint4(o[0], o[1], o[2], o[3]);
   }
   __syncthreads();
 
@@ -918,8 +922,11 @@ kda_bwd_grad_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
         if (ks < tb) continue;                 // T[r][i] = 0 for r < i
         uint32_t a[4], bv[4], bk[4];
         a_km(sb + G_DL, 64, r0, 16 * ks, lane, a);                  // T^T [i][r] from T [r][i]
-        b_kn(sb + G_DD, 64, c0 + 16 * np, 16 * ks, lane, bv);      // dDelta [r][j]
+        b_kn(sb + G_DD, 64, c0 + 16 * np, 16 * ks, lane, bv);      // dDelta [r][j] (hi)
         b_kn(sb + G_DW, 64, c0 + 16 * np, 16 * ks, lane, bk);      // dW [r][c]
+        mma(av[0], a, bv[0], bv[1]);
+        mma(av[1], a, bv[2], bv[3]);
+        b_kn(sb + G_S0, 64, c0 + 16 * np, 16 * ks, lane, bv);      // dDelta (lo)
         mma(av[0], a, bv[0], bv[1]);
         mma(av[1], a, bv[2], bv[3]);
         mma(ak[0], a, bk[0], bk[1]);
@@ -1446,7 +1453,7 @@ bool set_attrs() {
 
 struct BwdTcScratch {
   long long nslots;
-  size_t rec, simg, dlimg, dsimg, ddimg, total;
+  size_t rec, simg, dlimg, dsimg, ddimg, ddlo, total;
 };
 BwdTcScratch bwd_tc_scratch(int B, int T, int H, bool varlen) {
   BwdTcScratch r{};
@@ -1457,7 +1464,8 @@ BwdTcScratch bwd_tc_scratch(int B, int T, int H, bool varlen) {
   r.dlimg = r.simg + per * kImgS;
   r.dsimg = r.dlimg + per * kImgD;
   r.ddimg = r.dsimg + per * kImgS;
-  r.total = r.ddimg + per * kImgD;
+  r.ddlo = r.ddimg + per * kImgD;
+  r.total = r.ddlo + per * kImgD;
   return r;
 }
 
@@ -1504,8 +1512,8 @@ cudaError_t launch_chunk_bwd_tc(const void* q, const void* k, const void* v, con
                                dim3(D / kChainF + D / kChainR, H, B), dim3(NTC), kChainSmem,
                                stream, rec, h0, cu_seqlens,
                                static_cast<const bf16*>(dout), dhT, dh0, base + sc.simg,
-                               base + sc.dlimg, base + sc.dsimg, base + sc.ddimg, T, H,
-                               sc.nslots));
+                               base + sc.dlimg, base + sc.dsimg, base + sc.ddimg,
+                               base + sc.ddlo, T, H, sc.nslots));
     note_launches(1);
   }
   if (e == cudaSuccess && sc.nslots > 0) {
@@ -1518,7 +1526,8 @@ cudaError_t launch_chunk_bwd_tc(const void* q, const void* k, const void* v, con
                                static_cast<const uint8_t*>(rec), static_cast<const uint8_t*>(base + sc.simg),
                                static_cast<const uint8_t*>(base + sc.dlimg),
                                static_cast<const uint8_t*>(base + sc.dsimg),
-                               static_cast<const uint8_t*>(base + sc.ddimg), dq, dk, dv, dg,
+                               static_cast<const uint8_t*>(base + sc.ddimg),
+                               static_cast<const uint8_t*>(base + sc.ddlo), dq, dk, dv, dg,
                                dbeta, B, T, H, gsh, sc.nslots));
     note_launches(1);
   }

@@ -29,11 +29,11 @@ constexpr uint32_t U = 57344;
 // exp(Gamma_last) per key channel, fp32 [128]
 constexpr uint32_t DECAY = 73728;
 constexpr uint32_t BYTES = 74240;           // prefill record
-// backward record only: T = (I + diag(beta) A)^-1 and A (unscaled, strictly lower),
-// fp32 [64][64] row-major each
+// backward record only: T = (I + diag(beta) A)^-1 as a bf16 image [64 r][64 i] (8 KB, the
+// layout above), then A (unscaled, strictly lower) in fp32 [64][64] row-major
 constexpr uint32_t TMAT = 74240;
-constexpr uint32_t AMAT = TMAT + 16384;
-constexpr uint32_t BYTES_BWD = AMAT + 16384;  // 107,008
+constexpr uint32_t AMAT = TMAT + 8192;
+constexpr uint32_t BYTES_BWD = AMAT + 16384;  // 98,816
 
 }  // namespace rec
 }  // namespace kda

@@ -86,8 +86,8 @@ constexpr uint32_t REC_U = rec::U;      // U^T [dv][64 tokens] f16: 128-byte row
 constexpr uint32_t REC_DECAY = rec::DECAY;   // exp(G_last) per key channel, fp32 [dk]
 constexpr uint32_t REC_BYTES = rec::BYTES;
 // The backward's records (BWD instantiation): the same images, but Kend^T, Aqk and
-// U^T in bf16 (gradients can be far below f16's normal range), followed by T and A
-// in fp32.
+// U^T in bf16 (gradients can be far below f16's normal range), followed by T as a bf16
+// image and A in fp32.
 
 // TMA maps of the prep kernel's tiles: q, k, g [rows, H, dk] and v [rows, H, dv]
 // (3-D: channel, head, token row), boxes of 64 token rows of one head.
@@ -300,7 +300,7 @@ __device__ __noinline__ void prep_unsafe_pairs(const float* __restrict__ g, long
 // Prep kernel: one CTA per (chunk slot, head).  CONV: q and k are the raw
 // projections; each is convolved causally per channel (width convW <= 4, history
 // reset at the document start), L2-normalised per token, and q scaled by dk^-1/2.
-// BWD: the backward's record (bf16 images, plus T and A in fp32).
+// BWD: the backward's record (bf16 images, T as a bf16 image too, and A in fp32).
 // ============================================================================
 template <bool CONV, bool GRPD, bool BWD = false>
 __global__ void __launch_bounds__(NT, 2)
@@ -943,15 +943,19 @@ kda_chunk_prep_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k,
       put(48 + i, col, x);
     }
     __syncthreads();
-    if constexpr (BWD) {                       // T for the backward, fp32 [64][64]
+    if constexpr (BWD) {                       // T for the backward, as a bf16 image [r][i]
       // (the blocks above the diagonal were never written: zeros)
-      float4* tr = reinterpret_cast<float4*>(rc + rec::TMAT);
 #pragma unroll
-      for (int it = 0; it < 4; ++it) {
-        const int idx = tid + it * NT, row = idx >> 4, c4 = idx & 15;
-        const float4 x = *reinterpret_cast<const float4*>(T32 + row * LDA + 4 * c4);
-        tr[idx] = make_float4(4 * c4 + 0 <= row ? x.x : 0.f, 4 * c4 + 1 <= row ? x.y : 0.f,
-                              4 * c4 + 2 <= row ? x.z : 0.f, 4 * c4 + 3 <= row ? x.w : 0.f);
+      for (int it = 0; it < 2; ++it) {
+        const int idx = tid + it * NT, row = idx >> 3, c8 = idx & 7;
+        const float4 x0 = *reinterpret_cast<const float4*>(T32 + row * LDA + 8 * c8);
+        const float4 x1 = *reinterpret_cast<const float4*>(T32 + row * LDA + 8 * c8 + 4);
+        const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+        float w[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w[e] = 8 * c8 + e <= row ? xs[e] : 0.f;
+        *reinterpret_cast<uint4*>(rc + rec::TMAT + off_kmajor_sw128((uint32_t)row, (uint32_t)(8 * c8), 64u)) =
+            pack8(w, 1.f);
       }
     }
     // T diag(beta) as bf16: B operand of W^T / U^T, K-major SW128, N = 64 (r'), K = 64 (r)

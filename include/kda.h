@@ -299,7 +299,7 @@ KDA_API int kda_chunk_fwd_fused(const void* q_raw, const void* k_raw, const void
  * gradient are carried across chunks in fp32.  dq, dk, dv and dh0 are
  * reproducible bit for bit; dg and dbeta add a few per-chunk sums with
  * shared-memory atomics, so repeated calls may differ in their last bits.  Scratch:
- * 205,312 B per (chunk slot, head) (ceil(T/64) * B slots, ceil(T/64) + B when
+ * 213,504 B per (chunk slot, head) (ceil(T/64) * B slots, ceil(T/64) + B when
  * packed).
  * Otherwise (KDA_F32, or a 64-wide head): the recurrent reverse sweep of
  * kda_chunk_bwd_recurrent below.
@@ -373,7 +373,7 @@ KDA_API int kda_chunk_bwd_grouped(const void* q, const void* k, const void* v,
  * 4 * 64 KB when the split keeps half-way states (kda_prefill_plan gives the split;
  * segment slots = B * ceil(ceil(T/64) / G), or that count + B when packed).  KDA_F32
  * forward calls need none.  The backward's is, in its chunked form (KDA_BF16,
- * dk = dv = 128), 205,312 B per (chunk slot, head); otherwise 4 * dk * dv B per
+ * dk = dv = 128), 213,504 B per (chunk slot, head); otherwise 4 * dk * dv B per
  * (chunk slot + sequence, head) plus 64 * 4 * dk * dv B per (sequence, head).
  * Returns KDA_OK, KDA_ERR_INVALID_ARG (unknown op, bad sizes, NULL bytes),
  * KDA_ERR_UNSUPPORTED (head sizes) or KDA_ERR_CUDA (sms = 0 and no device).

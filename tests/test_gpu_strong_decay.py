@@ -219,10 +219,10 @@ def test_backward_grouped(kind, G):
 def test_backward_every_channel_strong(case):
     """Every key channel decaying by 5.5-6.5 per token (alpha <= 0.004 on every channel and
     token): the true dg shrinks to ~5e-4 of the unit-scale inputs.  The chunked form keeps
-    dq, dk, dv, dg and dh0 within the bf16 bound (A_qk's diagonal, whose dGamma terms
-    cancel exactly, is kept out of the decay-weighted products); dbeta measures ~1.05e-2
-    here, at the bound's edge, and is held to 2e-2.  The fp32 recurrent sweep stays within
-    1e-4 throughout."""
+    every gradient within the bf16 bound: A_qk's diagonal, whose dGamma terms cancel
+    exactly, is kept out of the decay-weighted products, and dDelta reaches T^T dDelta (dv,
+    and dbeta, which is almost all of sum_j dVb v here) as a hi/lo pair of bf16 images.
+    The fp32 recurrent sweep stays within 1e-4 throughout."""
     x = ki.make_prefill(_spec(B=1, T=200, H=2, seed=16))
     if case == "per_channel":
         gen = torch.Generator().manual_seed(99)
@@ -246,7 +246,7 @@ def test_backward_every_channel_strong(case):
         for name in ("dq", "dk", "dv", "dg", "dbeta", "dh0"):
             got = grads[name]
             assert torch.isfinite(got).all(), name
-            tol = 1e-4 if recurrent else (2e-2 if name == "dbeta" else TOL["bf16"])
+            tol = 1e-4 if recurrent else TOL["bf16"]
             assert rel_err(got, ref[name]) <= tol, (recurrent, name, rel_err(got, ref[name]))
 
 

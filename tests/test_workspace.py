@@ -2,9 +2,10 @@
 forward -- 74,240 B of chunk record per (head, chunk slot), ceil(T/64) * B slots
 (ceil(T/64) + B packed), plus 2 (4 with half points) x 64 KB per (segment slot,
 head) when the prefill splits sequences (kda_prefill_plan); none for fp32 inputs.
-backward -- in the chunked form (bf16, dk = dv = 128) 205,312 B per (chunk slot,
-head): the 107,008-byte record (the forward's 74,240 B plus T and A in fp32) and
-the bf16 images of S, dS (32 KB each), Delta and dDelta (16 KB each); otherwise (the
+backward -- in the chunked form (bf16, dk = dv = 128) 213,504 B per (chunk slot,
+head): the 98,816-byte record (the forward's 74,240 B, T as an 8 KB bf16 image, A in
+fp32) and the bf16 images of S, dS (32 KB each), Delta, and dDelta as a hi/lo pair
+(16 KB each); otherwise (the
 recurrent sweep) 4 dk dv B per (chunk slot + sequence, head) plus 64 x 4 dk dv B
 per (sequence, head)."""
 import math
@@ -44,8 +45,9 @@ def test_backward_size_matches_the_header(B, T, H, packed, dk, dv):
     nch = math.ceil(T / 64)
     slots = nch + B if packed else nch * B
     recurrent = ((slots + B) * H + B * H * 64) * dk * dv * 4
-    chunked = slots * H * (74240 + 2 * 64 * 64 * 4 + 2 * 128 * 128 * 2 + 2 * 64 * 128 * 2)
-    assert chunked == slots * H * 205312
+    chunked = slots * H * (74240 + 64 * 64 * 2 + 64 * 64 * 4 + 2 * 128 * 128 * 2
+                           + 3 * 64 * 128 * 2)
+    assert chunked == slots * H * 213504
     for dtype in (kda.KDA_BF16, kda.KDA_F32):
         got = kda.kda_workspace_size(kda.KDA_OP_CHUNK_BWD, B, T, H, dk, dv, packed=packed,
                                      dtype=dtype, sms=148)
