@@ -47,7 +47,7 @@ extern "C" {
 typedef enum {
   KDA_OK = 0,
   KDA_ERR_INVALID_ARG = -1,   /* null required pointer, bad size, misalignment */
-  KDA_ERR_UNSUPPORTED = -2,   /* valid request this build does not implement   */
+  KDA_ERR_UNSUPPORTED = -2,   /* valid request the library does not implement  */
   KDA_ERR_CUDA = -3,          /* a CUDA runtime call or kernel launch failed    */
   KDA_ERR_TIMEOUT = -4        /* a bounded device-side wait expired (see kda_device_status) */
 } kda_status_t;
