@@ -13,6 +13,12 @@ inside one block, so neither overflows however long the chunk's total decay.
 The Gamma terms follow from the row terms: sum_i dA_ri k_rc k_ic E_ric equals
 k_rc times the pair term of dk_r, and likewise for the other three.
 
+``aqk_diagonal_apart``: the same pair terms with Aqk's diagonal (i = r, decay factor
+exp(0) = 1) taken out of the decay-weighted sums and added to dq and dk alone.  Its
+two Gamma terms, q_rc k_rc dAqk_rr on the row side and its negative on the column
+side, cancel exactly, so dgam is unchanged; the gradient kernel computes it this way
+so that bf16 rounding of the two cancelling terms never reaches dg.
+
 ``reverse_state_segments``: chunked_backward's chunk-start state gradients without the
 forward states.  Substituting dDelta into dS0 gives dS_n = Y_n dS_{n+1} + c_n
 with Y_n = Diag(exp(Gamma_last)) - W^T Kend and c_n = (Qbar - Aqk W)^T dO_n,
@@ -27,7 +33,7 @@ import numpy as np
 
 from oracle.reference import _chunk_terms
 
-__all__ = ["pair_grads_blocked", "reverse_state_segments"]
+__all__ = ["pair_grads_blocked", "reverse_state_segments", "aqk_diagonal_apart"]
 
 
 def reverse_state_segments(q, k, v, g, beta, dout, dhT=None, C: int = 64, G: int = 4):
@@ -98,4 +104,21 @@ def pair_grads_blocked(dA, dAqk, q, k, gam, block: int = 16):
             dk[b0:b1] += col_k
             dgam[a0:a1] += k[a0:a1] * row_k + q[a0:a1] * row_q
             dgam[b0:b1] -= k[b0:b1] * col_k
+    return dq, dk, dgam
+
+
+def aqk_diagonal_apart(dA, dAqk, q, k, gam):
+    """(dq, dk, dgam) of the pairwise-decay sums, Aqk's diagonal apart (module docstring):
+    dA strictly lower, dAqk lower with its diagonal [L, L]; q, k, gam [L, dk]."""
+    d = np.diag(dAqk).copy()
+    off = np.tril(dAqk, -1)
+    L = len(gam)
+    lower = np.tril(np.ones((L, L), dtype=bool))[:, :, None]           # pairs i <= r
+    E = np.exp(np.where(lower, gam[:, None, :] - gam[None, :, :], -np.inf))
+    PA, PQ = dA[:, :, None] * E, off[:, :, None] * E
+    dq = np.einsum("ric,ic->rc", PQ, k) + d[:, None] * k
+    dk = (np.einsum("ric,ic->rc", PA, k) + np.einsum("ric,rc->ic", PA, k)
+          + np.einsum("ric,rc->ic", PQ, q) + d[:, None] * q)
+    tA, tQ = PA * k[:, None, :] * k[None, :, :], PQ * q[:, None, :] * k[None, :, :]
+    dgam = tA.sum(1) - tA.sum(0) + tQ.sum(1) - tQ.sum(0)
     return dq, dk, dgam

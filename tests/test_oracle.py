@@ -371,6 +371,27 @@ def test_pair_grads_blocked_equal_pairwise_terms(L, g_scale):
         assert np.abs(x - w).max() <= 1e-12 * max(np.abs(w).max(), 1e-30), name
 
 
+@pytest.mark.parametrize("L,g_scale", [(64, 0.3), (64, 6.0), (23, 1.0)])
+def test_aqk_diagonal_apart_equals_pairwise_terms(L, g_scale):
+    """Aqk's diagonal (decay factor 1) contributes nothing to dGamma: its row-side and
+    column-side terms cancel exactly, so taking it out of the decay-weighted sums and
+    adding its dq, dk terms alone gives the plain pairwise terms, strong decay included."""
+    rng = np.random.default_rng(L + int(10 * g_scale))
+    q, k, _, g, _ = _rand_inputs(rng, L, 1, 8, 4, g_scale=g_scale)
+    q, k, gam = q[0, :, 0], k[0, :, 0], np.cumsum(g[0, :, 0], axis=0)
+    dA = np.tril(rng.standard_normal((L, L)), -1)
+    dAqk = np.tril(rng.standard_normal((L, L)))
+    want = _pair_terms_einsum(dA, dAqk, q, k, gam)
+    got = kf.aqk_diagonal_apart(dA, dAqk, q, k, gam)
+    for w, x, name in zip(want, got, ("dq", "dk", "dgam")):
+        assert np.abs(x - w).max() <= 1e-12 * max(np.abs(w).max(), 1e-30), name
+    # and the diagonal's own Gamma terms are the cancelling pair: with everything else
+    # zero, the plain terms give dgam = 0 exactly up to rounding
+    only = np.diag(np.diag(dAqk))
+    _, _, dg0 = _pair_terms_einsum(np.zeros_like(dA), only, q, k, gam)
+    assert np.abs(dg0).max() <= 1e-12 * np.abs(q * k).max() * np.abs(np.diag(dAqk)).max()
+
+
 @pytest.mark.parametrize("T,C,G", [(150, 32, 2), (130, 64, 1), (400, 16, 7), (64, 64, 3)])
 def test_reverse_state_segments_equal_chunk_start_gradients(oracle_lib, T, C, G):
     """The reverse state recurrence needs no forward state and splits into segments:
